@@ -1,0 +1,35 @@
+"""CPU oracle for the QLoRA NF4 + double-quant + LoRA linear hot path.
+
+TEST INFRASTRUCTURE, NOT PRODUCT CODE. Only the test suite, the smoke check of
+``__graft_entry__`` and the CPU-baseline / reference legs of ``bench.py`` may
+import or run anything in this package. The library's CUDA path shares no code
+with it, and it imports nothing from the library.
+
+The oracle is deliberately plain and slow: numpy/Python on the host, fp64 for
+every real-valued reduction and GEMM, and exact (integer or rational) arithmetic
+wherever a rounding decides a stored bit pattern. Each function cites the web
+page passage it follows:
+
+* "Guanaco" (chipfoundryservices.com/topic/guanaco), sections "Core
+  Architecture & Training" and "Technical Innovations".
+* "QLoRA: Efficient Finetuning of Quantized LLMs" (ai-papercheck.pages.dev
+  errata list), findings quoting the paper's p.4 Section 2 and p.5 Section 3.
+* "QLoRA vs ChatGPT" (unfragile.ai compare page), capability blurbs 1 (NF4 with
+  block-wise absmax), 2 (LoRA on a frozen 4-bit base), 3 (double quantization)
+  and 5 (training pipeline: block-wise on-the-fly dequantization, gradients for
+  the LoRA parameters only).
+
+Where the pages are silent the oracle takes one stated reading; every reading is
+listed in the repository's design notes.
+"""
+from .fp import bf16_bits_to_f32, f32_to_bf16_bits_rn, fma_f32
+from .nf4 import (BLOCK, DQ_BLOCK, nf4_codebook, quantize_nf4, double_quantize, quantize_nf4_dq,
+                  dequantize_nf4_dq, unpack_codes, storage_bytes, QuantizedNF4)
+from .linear import lora_scale, linear_fwd, linear_bwd
+
+__all__ = [
+    "bf16_bits_to_f32", "f32_to_bf16_bits_rn", "fma_f32",
+    "BLOCK", "DQ_BLOCK", "nf4_codebook", "quantize_nf4", "double_quantize", "quantize_nf4_dq",
+    "dequantize_nf4_dq", "unpack_codes", "storage_bytes", "QuantizedNF4",
+    "lora_scale", "linear_fwd", "linear_bwd",
+]
