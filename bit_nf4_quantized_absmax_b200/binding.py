@@ -1,0 +1,203 @@
+"""Thin ctypes binding of the C ABI in include/qlora.h.
+
+Argument marshalling only: torch tensors supply device memory and the current
+stream; every step of the computation runs in the library's CUDA kernels. The
+functions keep the C names. Loading fails loudly when the shared library has
+not been built; there is no fallback path.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libqlora_b200.so")
+
+QLORA_OK = 0
+STATUS_NAMES = {0: "QLORA_OK", 1: "QLORA_ERR_INVALID_ARG", 2: "QLORA_ERR_UNSUPPORTED", 3: "QLORA_ERR_ALIGNMENT",
+                4: "QLORA_ERR_CUDA", 5: "QLORA_ERR_WORKSPACE", 6: "QLORA_ERR_DEVICE"}
+
+EXPORTED = ("qlora_status_string", "qlora_nf4_codebook", "qlora_nf4_storage_bytes", "qlora_quantize_nf4_dq",
+            "qlora_dequantize_nf4_dq", "qlora_linear_fwd", "qlora_linear_bwd", "qlora_device_error")
+
+
+class QloraError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what} failed: {STATUS_NAMES.get(status, status)}")
+        self.status = status
+
+
+class _Weight(ctypes.Structure):
+    _fields_ = [("packed", ctypes.c_void_p), ("absmax_q", ctypes.c_void_p), ("dq_scale", ctypes.c_void_p),
+                ("mean", ctypes.c_void_p), ("rows", ctypes.c_int64), ("cols", ctypes.c_int64),
+                ("blocksize", ctypes.c_int32), ("dq_blocksize", ctypes.c_int32)]
+
+
+_lib = None
+
+
+def load_library(path: str | None = None) -> ctypes.CDLL:
+    """Load libqlora_b200.so (once). Raises if it is missing."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    p = path or LIB_PATH
+    if not os.path.exists(p):
+        raise RuntimeError(f"{p} is missing: build it with `python -m bit_nf4_quantized_absmax_b200.build`")
+    lib = ctypes.CDLL(p)
+    vp, i64, i32, f32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_float, ctypes.c_size_t
+    wp = ctypes.POINTER(_Weight)
+    szp = ctypes.POINTER(ctypes.c_size_t)
+    lib.qlora_status_string.restype = ctypes.c_char_p
+    lib.qlora_status_string.argtypes = [ctypes.c_int]
+    lib.qlora_nf4_codebook.argtypes = [ctypes.POINTER(ctypes.c_float)]
+    lib.qlora_nf4_storage_bytes.argtypes = [i64, i64, ctypes.POINTER(sz)]
+    lib.qlora_quantize_nf4_dq.argtypes = [vp, wp, vp, szp, vp]
+    lib.qlora_dequantize_nf4_dq.argtypes = [wp, vp, vp]
+    lib.qlora_linear_fwd.argtypes = [wp, vp, i64, vp, vp, i32, f32, vp, vp, vp, szp, vp]
+    lib.qlora_linear_bwd.argtypes = [wp, vp, i64, vp, vp, i32, f32, vp, vp, vp, vp, vp, vp, szp, vp]
+    lib.qlora_device_error.argtypes = [ctypes.POINTER(ctypes.c_int32), vp]
+    for name in EXPORTED:
+        getattr(lib, name).restype = ctypes.c_int if name != "qlora_status_string" else ctypes.c_char_p
+    _lib = lib
+    return lib
+
+
+def _check(status: int, what: str):
+    if status != QLORA_OK:
+        raise QloraError(status, what)
+
+
+def _ptr(t: torch.Tensor | None):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+@dataclass
+class NF4Weight:
+    """Device storage of one quantized frozen weight [rows, cols]."""
+    packed: torch.Tensor     # uint8 [rows*cols/2]
+    absmax_q: torch.Tensor   # int8 [nblk]
+    dq_scale: torch.Tensor   # float32 [ngrp]
+    mean: torch.Tensor       # float32 [1]
+    rows: int
+    cols: int
+
+    def as_c(self) -> _Weight:
+        return _Weight(self.packed.data_ptr(), self.absmax_q.data_ptr(), self.dq_scale.data_ptr(),
+                       self.mean.data_ptr(), self.rows, self.cols, 64, 256)
+
+    @staticmethod
+    def empty(rows: int, cols: int, device="cuda") -> "NF4Weight":
+        sizes = qlora_nf4_storage_bytes(rows, cols)
+        return NF4Weight(torch.empty(sizes[0], dtype=torch.uint8, device=device),
+                         torch.empty(sizes[1], dtype=torch.int8, device=device),
+                         torch.empty(sizes[2] // 4, dtype=torch.float32, device=device),
+                         torch.empty(1, dtype=torch.float32, device=device), rows, cols)
+
+
+def qlora_status_string(status: int) -> str:
+    return load_library().qlora_status_string(status).decode()
+
+
+def qlora_nf4_codebook() -> torch.Tensor:
+    out = (ctypes.c_float * 16)()
+    _check(load_library().qlora_nf4_codebook(out), "qlora_nf4_codebook")
+    return torch.tensor(list(out), dtype=torch.float32)
+
+
+def qlora_nf4_storage_bytes(rows: int, cols: int) -> tuple:
+    out = (ctypes.c_size_t * 4)()
+    _check(load_library().qlora_nf4_storage_bytes(rows, cols, out), "qlora_nf4_storage_bytes")
+    return tuple(int(x) for x in out)
+
+
+def _workspace(query, workspace: torch.Tensor | None, device) -> tuple:
+    """Run the size query; return (workspace tensor, ctypes size)."""
+    need = ctypes.c_size_t(0)
+    _check(query(None, ctypes.byref(need)), "workspace query")
+    if workspace is None or workspace.numel() < need.value:
+        workspace = torch.empty(max(need.value, 256), dtype=torch.uint8, device=device)
+    return workspace, ctypes.c_size_t(workspace.numel())
+
+
+def qlora_quantize_nf4_dq(W: torch.Tensor, out: NF4Weight | None = None, workspace: torch.Tensor | None = None,
+                          stream=None) -> NF4Weight:
+    assert W.dtype == torch.bfloat16 and W.dim() == 2 and W.is_contiguous()
+    lib = load_library()
+    q = out or NF4Weight.empty(W.shape[0], W.shape[1], W.device)
+    qc = q.as_c()
+    st = _stream(stream)
+    ws, nbytes = _workspace(lambda p, n: lib.qlora_quantize_nf4_dq(_ptr(W), ctypes.byref(qc), p, n, st), workspace,
+                            W.device)
+    _check(lib.qlora_quantize_nf4_dq(_ptr(W), ctypes.byref(qc), _ptr(ws), ctypes.byref(nbytes), st),
+           "qlora_quantize_nf4_dq")
+    return q
+
+
+def qlora_dequantize_nf4_dq(q: NF4Weight, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    lib = load_library()
+    if out is None:
+        out = torch.empty(q.rows, q.cols, dtype=torch.bfloat16, device=q.packed.device)
+    qc = q.as_c()
+    _check(lib.qlora_dequantize_nf4_dq(ctypes.byref(qc), _ptr(out), _stream(stream)), "qlora_dequantize_nf4_dq")
+    return out
+
+
+def qlora_linear_fwd(q: NF4Weight, X: torch.Tensor, A: torch.Tensor, B: torch.Tensor, alpha: float,
+                     Y: torch.Tensor | None = None, T_save: torch.Tensor | bool | None = None,
+                     workspace: torch.Tensor | None = None, stream=None):
+    """Returns (Y, T) with T = X A^T in fp32 when T_save is True or a tensor, else (Y, None)."""
+    lib = load_library()
+    M, r = X.shape[0], A.shape[0]
+    dev = X.device
+    if Y is None:
+        Y = torch.empty(M, q.rows, dtype=torch.bfloat16, device=dev)
+    if T_save is True:
+        T_save = torch.empty(M, r, dtype=torch.float32, device=dev)
+    elif T_save is False:
+        T_save = None
+    qc = q.as_c()
+    st = _stream(stream)
+    args = lambda p, n: lib.qlora_linear_fwd(ctypes.byref(qc), _ptr(X), M, _ptr(A), _ptr(B), r, float(alpha),
+                                             _ptr(Y), _ptr(T_save), p, n, st)
+    ws, nbytes = _workspace(args, workspace, dev)
+    _check(args(_ptr(ws), ctypes.byref(nbytes)), "qlora_linear_fwd")
+    return Y, T_save
+
+
+def qlora_linear_bwd(q: NF4Weight, X: torch.Tensor, A: torch.Tensor, B: torch.Tensor, alpha: float,
+                     dY: torch.Tensor, T_saved: torch.Tensor | None = None, need_dX: bool = True,
+                     dX: torch.Tensor | None = None, dA: torch.Tensor | None = None, dB: torch.Tensor | None = None,
+                     workspace: torch.Tensor | None = None, stream=None):
+    """Returns (dX or None, dA, dB)."""
+    lib = load_library()
+    M, r = X.shape[0], A.shape[0]
+    dev = X.device
+    if need_dX and dX is None:
+        dX = torch.empty(M, q.cols, dtype=torch.bfloat16, device=dev)
+    if dA is None:
+        dA = torch.empty(r, q.cols, dtype=torch.bfloat16, device=dev)
+    if dB is None:
+        dB = torch.empty(q.rows, r, dtype=torch.bfloat16, device=dev)
+    qc = q.as_c()
+    st = _stream(stream)
+    args = lambda p, n: lib.qlora_linear_bwd(ctypes.byref(qc), _ptr(X), M, _ptr(A), _ptr(B), r, float(alpha),
+                                             _ptr(dY), _ptr(T_saved), _ptr(dX if need_dX else None), _ptr(dA),
+                                             _ptr(dB), p, n, st)
+    ws, nbytes = _workspace(args, workspace, dev)
+    _check(args(_ptr(ws), ctypes.byref(nbytes)), "qlora_linear_bwd")
+    return (dX if need_dX else None), dA, dB
+
+
+def qlora_device_error(stream=None) -> int:
+    code = ctypes.c_int32(0)
+    _check(load_library().qlora_device_error(ctypes.byref(code), _stream(stream)), "qlora_device_error")
+    return int(code.value)

@@ -1,0 +1,54 @@
+// Block-wise dequantization of NF4 + double-quant storage to bf16
+// ("QLoRA vs ChatGPT", capability 5: weights are dequantized block by block).
+//
+// One thread decodes 32 weights (half a 64-weight block): it forms the block
+// constant m' = fmaf(q_b, dq_scale_g, mean), builds the block's 16-entry bf16
+// table and decodes its 16 packed bytes with byte permutes.
+#include "common.cuh"
+#include "kernels.h"
+#include "nf4_lut.cuh"
+
+namespace qlora {
+namespace {
+
+__global__ void __launch_bounds__(256)
+k_dequant(const uint4* __restrict__ packed, const int8_t* __restrict__ absmax_q,
+          const float* __restrict__ dq_scale, const float* __restrict__ mean, uint4* __restrict__ out,
+          int64_t n_units, const __grid_constant__ Nf4Codebook cb) {
+  const float mu = *mean;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t u = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; u < n_units; u += stride) {
+    const int64_t b = u >> 1;
+    const uint4 nib = __ldcs(packed + u);
+    const float mp = __fmaf_rn(static_cast<float>(absmax_q[b]), dq_scale[b >> 8], mu);
+    const Nf4Lut t = make_nf4_lut(cb, mp);
+    uint32_t o[16];
+    nf4_lookup8(t, nib.x, o + 0);
+    nf4_lookup8(t, nib.y, o + 4);
+    nf4_lookup8(t, nib.z, o + 8);
+    nf4_lookup8(t, nib.w, o + 12);
+    uint4* dst = out + u * 4;
+    __stcs(dst + 0, make_uint4(o[0], o[1], o[2], o[3]));
+    __stcs(dst + 1, make_uint4(o[4], o[5], o[6], o[7]));
+    __stcs(dst + 2, make_uint4(o[8], o[9], o[10], o[11]));
+    __stcs(dst + 3, make_uint4(o[12], o[13], o[14], o[15]));
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_dequantize(const uint8_t* packed, const int8_t* absmax_q, const float* dq_scale,
+                              const float* mean, void* out, int64_t numel, const float codebook[16],
+                              int num_sms, cudaStream_t stream) {
+  Nf4Codebook cb;
+  for (int i = 0; i < 16; ++i) cb.c[i] = codebook[i];
+  const int64_t n_units = numel / 32;
+  int64_t want = (n_units + 255) / 256;
+  int64_t cap = static_cast<int64_t>(num_sms) * 8;
+  const int grid = static_cast<int>(want < cap ? (want > 0 ? want : 1) : cap);
+  k_dequant<<<grid, 256, 0, stream>>>(reinterpret_cast<const uint4*>(packed), absmax_q, dq_scale, mean,
+                                      reinterpret_cast<uint4*>(out), n_units, cb);
+  return cudaGetLastError();
+}
+
+}  // namespace qlora

@@ -1,0 +1,194 @@
+/*
+ * qlora.h -- C ABI of the B200 (sm_100a) QLoRA NF4 library.
+ *
+ * The library implements the data-parallel hot path of QLoRA:
+ *   1. the NF4 ("NormalFloat4") codebook,
+ *   2. block-wise absmax quantization of a frozen bf16 weight to 4-bit codes,
+ *   3. double quantization of the fp32 absmax constants to int8 codes,
+ *   4. block-wise dequantization back to bf16,
+ *   5. the QLoRA linear layer  Y = X W'^T + s (X A^T) B^T  (W' = dequant(W)),
+ *      forward and backward (dX, dA, dB; W stays frozen, no dW).
+ *
+ * Sources (web pages describing the method; no code is printed on them):
+ *   [G]  "Guanaco" (chipfoundryservices.com/topic/guanaco), sections
+ *        "Core Architecture & Training" and "Technical Innovations".
+ *   [E]  "QLoRA: Efficient Finetuning of Quantized LLMs" (ai-papercheck
+ *        errata page), findings quoting the paper's p.4 Section 2 and
+ *        p.5 Section 3.
+ *   [C]  "QLoRA vs ChatGPT" (unfragile.ai compare page), capability blurbs
+ *        1 (NF4, block-wise absmax), 2 (LoRA on a frozen 4-bit base),
+ *        3 (double quantization) and 5 (on-the-fly block-wise dequantization,
+ *        gradients only for the LoRA parameters).
+ *
+ * Conventions for every call below:
+ *   - bf16 tensors are passed as void*, row-major and contiguous, with base
+ *     addresses aligned to 16 bytes (else QLORA_ERR_ALIGNMENT).
+ *   - Device pointers are owned by the caller. The library never allocates,
+ *     frees or synchronizes: every kernel is launched asynchronously on the
+ *     given stream. Argument, shape and alignment errors are returned before
+ *     anything is launched; a launch failure returns QLORA_ERR_CUDA.
+ *   - Outputs are overwritten (no accumulation into them).
+ *   - Workspace: calls that need scratch device memory take (workspace,
+ *     workspace_bytes). With workspace == NULL the call stores the required
+ *     size in *workspace_bytes and returns QLORA_OK without launching. With a
+ *     non-NULL workspace, *workspace_bytes must hold at least that size
+ *     (else QLORA_ERR_WORKSPACE). The workspace base must be 256-byte aligned.
+ *     Workspace contents need no initialisation and are not preserved.
+ *   - The library keeps no state between calls and may be used from several
+ *     host threads at once (on distinct workspaces).
+ *   - Inputs must be finite; non-finite weights give unspecified codes.
+ *   - s = (float)alpha / (float)r, one fp32 division.
+ */
+#ifndef QLORA_B200_H
+#define QLORA_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* The stream type is the CUDA runtime's cudaStream_t (NULL = legacy default). */
+typedef struct CUstream_st* qlora_stream_t;
+
+typedef enum {
+  QLORA_OK = 0,
+  QLORA_ERR_INVALID_ARG = 1,   /* null pointer, negative or inconsistent size  */
+  QLORA_ERR_UNSUPPORTED = 2,   /* block sizes other than 64/256, cols % 64 != 0,
+                                  r outside [8, 256] or r % 8 != 0             */
+  QLORA_ERR_ALIGNMENT = 3,     /* a pointer is not aligned as required          */
+  QLORA_ERR_CUDA = 4,          /* a launch or CUDA runtime call failed          */
+  QLORA_ERR_WORKSPACE = 5,     /* the workspace given is smaller than required  */
+  QLORA_ERR_DEVICE = 6         /* no sm_100 device is current                   */
+} qlora_status;
+
+/* NF4 + double-quant storage of one frozen weight W [rows, cols] (rows = N =
+ * out_features, cols = K = in_features, as in a PyTorch Linear).
+ *
+ *   packed    : rows*cols/2 bytes. Byte i holds code[2i] in its low nibble and
+ *               code[2i+1] in its high nibble (elements in row-major order).
+ *   absmax_q  : nblk = rows*cols/64 int8 codes in [-127, 127], one per block of
+ *               64 consecutive weights (a block never crosses a row).
+ *   dq_scale  : ngrp = ceil(nblk/256) fp32 scales, one per 256 consecutive
+ *               absmax codes (the last group may be shorter).
+ *   mean      : one fp32, the mean of all first-level absmax constants.
+ *   blocksize, dq_blocksize: must be 64 and 256.
+ *
+ * A block's decoded constant is m' = fmaf((float)absmax_q[b], dq_scale[b/256],
+ * mean) and its weights decode to bf16_rn(codebook[code] * m')  ([C] 1, 3, 5).
+ * All pointers are device memory owned by the caller; packed must be 16-byte
+ * aligned, the others 4-byte aligned.
+ */
+typedef struct {
+  uint8_t* packed;
+  int8_t*  absmax_q;
+  float*   dq_scale;
+  float*   mean;
+  int64_t  rows;
+  int64_t  cols;
+  int32_t  blocksize;
+  int32_t  dq_blocksize;
+} qlora_nf4_weight;
+
+/* Human-readable name of a status code (static string). */
+const char* qlora_status_string(qlora_status s);
+
+/* qlora_nf4_codebook -- the 16 NF4 values, ascending, as fp32 (host call,
+ * synchronous, no device needed).
+ *
+ * The values are normal quantiles at equally spaced probabilities: 8 positive
+ * values Phi^-1(1/2 + (d - 1/2) j/8), j = 1..8, 7 negative values
+ * -Phi^-1(1/2 + (d - 1/2) j/7), j = 1..7, and an exact 0, all divided by
+ * Phi^-1(d) with d = 1 - (1/30 + 1/32)/2, then rounded to fp32. Index 0 is -1,
+ * index 7 is 0, index 15 is +1. ([G] "Technical Innovations": a 4-bit type for
+ * normally distributed weights; [E] p.5 Section 3: a discrete zero point and
+ * all 2^k values used. The pages print neither the construction nor d; this
+ * is the library's stated reading.)
+ * Errors: QLORA_ERR_INVALID_ARG if out16 is NULL. */
+qlora_status qlora_nf4_codebook(float out16[16]);
+
+/* qlora_nf4_storage_bytes -- sizes of the four arrays of qlora_nf4_weight for
+ * a [rows, cols] weight (host call). out[0..3] = bytes of packed, absmax_q,
+ * dq_scale, mean. Errors: QLORA_ERR_INVALID_ARG (NULL out, negative sizes),
+ * QLORA_ERR_UNSUPPORTED (cols % 64 != 0). */
+qlora_status qlora_nf4_storage_bytes(int64_t rows, int64_t cols, size_t out[4]);
+
+/* qlora_quantize_nf4_dq -- quantize a frozen bf16 weight W [rows, cols] into
+ * q's arrays ([C] 1: block-wise absmax quantization; [C] 3 and [G] "Core
+ * Architecture & Training": the absmax constants are quantized again to 8 bit
+ * with their own scales).
+ *
+ *   Level 1, per block b of 64 weights: m_b = max |w| (exact); if m_b == 0 all
+ *   codes are 7, else v = fp32(w / m_b) (IEEE division) and the code is the
+ *   index of the nearest codebook value, ties to the lower index.
+ *   Level 2: mu = fp32(fp64(S) / nblk) with S the exact sum of all m_b;
+ *   c_b = fp32(m_b - mu); per group of 256: s_g = max |c_b|,
+ *   dq_scale_g = fp32(s_g / 127), absmax_q_b = clamp(rint_even(fp32(c_b /
+ *   dq_scale_g)), -127, 127); a group with s_g == 0 stores scale 0, codes 0.
+ *
+ * W_bf16: device, [rows, cols] bf16, 16-byte aligned. q: host struct whose
+ * pointers and sizes describe caller-owned device arrays (q->rows, q->cols
+ * must equal the weight's shape). rows == 0 returns QLORA_OK and writes
+ * nothing. The result does not depend on launch configuration (the mean uses
+ * an exact integer accumulation).
+ * Errors: INVALID_ARG, UNSUPPORTED, ALIGNMENT, WORKSPACE, CUDA, DEVICE. */
+qlora_status qlora_quantize_nf4_dq(const void* W_bf16, const qlora_nf4_weight* q,
+                                   void* workspace, size_t* workspace_bytes,
+                                   qlora_stream_t stream);
+
+/* qlora_dequantize_nf4_dq -- decode q to a bf16 matrix out_bf16 [rows, cols]
+ * (device, 16-byte aligned): w' = bf16_rn(fp32(codebook[code] * m'_b)) with
+ * m'_b = fmaf(absmax_q_b, dq_scale_g, mean) ([C] 5: block-wise dequantization).
+ * Bit-identical to the dequantization used inside qlora_linear_fwd/bwd.
+ * Errors: INVALID_ARG, UNSUPPORTED, ALIGNMENT, CUDA, DEVICE. */
+qlora_status qlora_dequantize_nf4_dq(const qlora_nf4_weight* q, void* out_bf16,
+                                     qlora_stream_t stream);
+
+/* qlora_linear_fwd -- Y = X W'^T + s (X A^T) B^T  ([C] 2 and 5).
+ *
+ *   q      : the frozen weight, W' = dequant(q) is [N, K] = [q->rows, q->cols].
+ *   X      : device bf16 [M, K].        A : device bf16 [r, K].
+ *   B      : device bf16 [N, r].        Y : device bf16 [M, N] (output).
+ *   T_save : device fp32 [M, r] or NULL; when given, receives T = X A^T
+ *            (fp32 accumulation) for reuse by qlora_linear_bwd.
+ *   M >= 0 (M == 0: nothing is launched); 8 <= r <= 256, r % 8 == 0.
+ * M <= 16 runs the decode kernels (weight-bandwidth bound, codes decoded in
+ * registers); larger M runs the tcgen05 tensor-core kernels.
+ * Accuracy: relative Frobenius error against an fp64 evaluation with the same
+ * bf16 inputs and the same W' is about 1e-3 (the bf16 rounding of Y).
+ * Errors: INVALID_ARG, UNSUPPORTED, ALIGNMENT, WORKSPACE, CUDA, DEVICE. */
+qlora_status qlora_linear_fwd(const qlora_nf4_weight* q, const void* X, int64_t M,
+                              const void* A, const void* B, int32_t r, float alpha,
+                              void* Y, float* T_save,
+                              void* workspace, size_t* workspace_bytes,
+                              qlora_stream_t stream);
+
+/* qlora_linear_bwd -- gradients of qlora_linear_fwd with W frozen ([C] 5:
+ * gradients only for the LoRA parameters; [E] p.4 Section 2: the input
+ * gradients are produced too):
+ *   dX = dY W' + s (dY B) A          [M, K] bf16 (skipped when dX == NULL)
+ *   dA = s (dY B)^T X                [r, K] bf16
+ *   dB = s dY^T (X A^T)              [N, r] bf16
+ * dY: device bf16 [M, N]. T_saved: device fp32 [M, r] from qlora_linear_fwd,
+ * or NULL to recompute X A^T. M == 0 writes zeros to dA and dB.
+ * Errors: INVALID_ARG, UNSUPPORTED, ALIGNMENT, WORKSPACE, CUDA, DEVICE. */
+qlora_status qlora_linear_bwd(const qlora_nf4_weight* q, const void* X, int64_t M,
+                              const void* A, const void* B, int32_t r, float alpha,
+                              const void* dY, const float* T_saved,
+                              void* dX, void* dA, void* dB,
+                              void* workspace, size_t* workspace_bytes,
+                              qlora_stream_t stream);
+
+/* qlora_device_error -- read and clear the library's device-side error word on
+ * the current device (synchronizes the stream). Kernels whose waits on
+ * asynchronous copies exceed a time bound set this word and return early
+ * instead of hanging; 0 means no such event. *code receives the word.
+ * Errors: INVALID_ARG (NULL code), CUDA. */
+qlora_status qlora_device_error(int32_t* code, qlora_stream_t stream);
+
+#ifdef __cplusplus
+}  /* extern "C" */
+#endif
+
+#endif  /* QLORA_B200_H */

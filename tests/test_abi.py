@@ -1,0 +1,101 @@
+"""CPU-only checks of the C ABI: the library loads, exports every symbol the
+header declares, and its host-side calls and argument checks behave as
+documented. No kernel is launched here."""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle
+from bit_nf4_quantized_absmax_b200 import binding as b
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "qlora.h")
+
+
+def _declared_symbols():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(qlora_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_symbol():
+    lib = b.load_library()
+    declared = _declared_symbols()
+    assert len(declared) >= 8
+    for name in declared:
+        assert hasattr(lib, name), name
+    assert set(declared) == set(b.EXPORTED)
+
+
+def test_status_strings():
+    assert b.qlora_status_string(0) == "QLORA_OK"
+    assert b.qlora_status_string(5) == "QLORA_ERR_WORKSPACE"
+    assert b.qlora_status_string(99) == "QLORA_ERR_UNKNOWN"
+
+
+def test_codebook_equals_oracle_bits():
+    """The library builds the codebook by Newton's method on erfc, the oracle by
+    bisection: the fp32 bits agree."""
+    lib_cb = b.qlora_nf4_codebook().numpy()
+    assert np.array_equal(lib_cb.view(np.uint32), oracle.nf4_codebook().view(np.uint32))
+
+
+def test_storage_bytes():
+    assert b.qlora_nf4_storage_bytes(4096, 4096) == (8388608, 262144, 4096, 4)
+    assert b.qlora_nf4_storage_bytes(3, 64 * 5) == (480, 15, 4, 4)
+    sb = oracle.storage_bytes(11008, 4096)
+    got = b.qlora_nf4_storage_bytes(11008, 4096)
+    assert got == (sb["packed"], sb["absmax_q"], sb["dq_scale"], sb["mean"])
+    with pytest.raises(b.QloraError) as e:
+        b.qlora_nf4_storage_bytes(4, 100)
+    assert e.value.status == 2
+
+
+def _weight(rows=4, cols=128, **kw):
+    fake = ctypes.c_void_p(1 << 20)  # aligned non-null dummies; nothing is launched
+    w = b._Weight(fake.value, fake.value, fake.value, fake.value, rows, cols, 64, 256)
+    for k, v in kw.items():
+        setattr(w, k, v)
+    return w
+
+
+def test_argument_errors_return_before_launch():
+    lib = b.load_library()
+    n = ctypes.c_size_t(0)
+    W = ctypes.c_void_p(1 << 20)
+    # workspace size query launches nothing
+    w = _weight()
+    assert lib.qlora_quantize_nf4_dq(W, ctypes.byref(w), None, ctypes.byref(n), None) == 0
+    assert n.value >= 4 * (4 * 128 // 64)
+    # unsupported block sizes / columns
+    assert lib.qlora_quantize_nf4_dq(W, ctypes.byref(_weight(blocksize=32)), None, ctypes.byref(n), None) == 2
+    assert lib.qlora_quantize_nf4_dq(W, ctypes.byref(_weight(dq_blocksize=128)), None, ctypes.byref(n), None) == 2
+    assert lib.qlora_quantize_nf4_dq(W, ctypes.byref(_weight(cols=100)), None, ctypes.byref(n), None) == 2
+    # null pointers / negative sizes
+    assert lib.qlora_quantize_nf4_dq(W, None, None, ctypes.byref(n), None) == 1
+    assert lib.qlora_quantize_nf4_dq(W, ctypes.byref(_weight(rows=-1)), None, ctypes.byref(n), None) == 1
+    assert lib.qlora_quantize_nf4_dq(W, ctypes.byref(_weight(packed=None)), None, ctypes.byref(n), None) == 1
+    assert lib.qlora_quantize_nf4_dq(W, ctypes.byref(w), None, None, None) == 1
+    # misaligned input or storage
+    assert lib.qlora_quantize_nf4_dq(ctypes.c_void_p((1 << 20) + 2), ctypes.byref(w), None, ctypes.byref(n),
+                                     None) == 3
+    assert lib.qlora_quantize_nf4_dq(W, ctypes.byref(_weight(packed=(1 << 20) + 8)), None, ctypes.byref(n),
+                                     None) == 3
+    # workspace too small / misaligned
+    small = ctypes.c_size_t(16)
+    assert lib.qlora_quantize_nf4_dq(W, ctypes.byref(w), ctypes.c_void_p(1 << 20), ctypes.byref(small), None) == 5
+    big = ctypes.c_size_t(1 << 30)
+    assert lib.qlora_quantize_nf4_dq(W, ctypes.byref(w), ctypes.c_void_p((1 << 20) + 16), ctypes.byref(big),
+                                     None) == 3
+    # dequant: null output, misaligned output
+    assert lib.qlora_dequantize_nf4_dq(ctypes.byref(w), None, None) == 1
+    assert lib.qlora_dequantize_nf4_dq(ctypes.byref(w), ctypes.c_void_p((1 << 20) + 2), None) == 3
+    # empty weight: nothing to do
+    assert lib.qlora_dequantize_nf4_dq(ctypes.byref(_weight(rows=0)), None, None) == 0
+    code = ctypes.c_int32(0)
+    assert lib.qlora_device_error(None, None) == 1
