@@ -1,0 +1,501 @@
+"""Benchmark of the QLoRA NF4 hot path on B200.
+
+One step = one pass of the whole hot path over the Llama-7B linear shapes
+(4096x4096, 11008x4096, 4096x11008), r = 64, alpha = 16, seeded synthetic data:
+  quantize + double-quantize W, dequantize W, decode forward at M = 1, 4, 16,
+  training forward at M = 4096 and training backward (dX, dA, dB) at M = 4096.
+The headline value is training TFLOP/s: the useful flops of the M = 4096
+forward + backward (2MNK + 2Mr(K+N) and 2MNK + 4Mr(K+N)) divided by the time
+of the whole step. Per-part times, decode weight GB/s and the roofline of the
+dominant kernel are reported beside it.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+N > 1 runs under torch.distributed.run, one rank per GPU; every rank runs the
+same step on its own data (weak scaling, no data-path collective) and the
+time is the maximum over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from bit_nf4_quantized_absmax_b200 import binding as qb  # noqa: E402
+from bit_nf4_quantized_absmax_b200 import synthetic as syn  # noqa: E402
+
+METRIC = "fused NF4+LoRA linear TFLOP/s (M=4096) and weight GB/s (M=1..16) vs roofline"
+R, ALPHA, M_TRAIN, M_DECODE = 64, 16.0, 4096, (1, 4, 16)
+SHAPES = syn.LLAMA7B_SHAPES
+
+# kernels each C-ABI call launches on these shapes (see the launchers in csrc/)
+LAUNCHES = {"quantize": 3, "dequantize": 1, "decode_fwd": 2, "train_fwd": 3, "train_bwd": 8}
+
+
+def train_flops(N, K, M=M_TRAIN, r=R):
+    fwd = 2 * M * N * K + 2 * M * r * (K + N)
+    bwd = 2 * M * N * K + 4 * M * r * (K + N)
+    return fwd, bwd
+
+
+def decode_bytes(N, K, M, r=R):
+    return 0.515869 * N * K + 2 * r * (K + N) + 2 * M * (K + N)
+
+
+def quant_bytes(N, K):
+    return 2.516 * N * K  # read bf16 W, write codes + int8 constants + scales
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"qlora_clocks_{os.getpid()}.csv")
+        self.t_begin = self.t_end = None
+
+    def start(self):
+        """Start sampling (before the warm-up, so samples exist when timing starts)."""
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu=timestamp,{self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"], stdout=open(self.path, "w"),
+                stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def mark_begin(self):
+        self.t_begin = time.time()
+
+    def mark_end(self):
+        self.t_end = time.time()
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.3)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        import datetime as _dt
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 10:
+                continue
+            try:
+                ts = _dt.datetime.strptime(f[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+            except ValueError:
+                continue
+            if self.t_begin is not None and not (self.t_begin - 0.25 <= ts <= self.t_end + 0.25):
+                continue
+            f = f[1:]
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# ----------------------------------------------------------------------------
+# our arm
+
+class Workload:
+    """Device-resident inputs, outputs and workspaces of one step."""
+
+    def __init__(self, dev, seed):
+        self.dev = dev
+        self.lin = []
+        for li, (N, K) in enumerate(SHAPES):
+            inp = syn.make_linear(N, K, M_TRAIN, r=R, alpha=ALPHA, seed=seed, workload="llama7b_train", layer=li)
+            d = {k: getattr(inp, k).to(dev).contiguous() for k in ("W", "A", "B", "X", "dY")}
+            d["N"], d["K"] = N, K
+            d["Xdec"] = {M: d["X"][:M].contiguous() for M in M_DECODE}
+            d["q"] = qb.NF4Weight.empty(N, K, dev)
+            d["Wd"] = torch.empty(N, K, dtype=torch.bfloat16, device=dev)
+            d["Ydec"] = {M: torch.empty(M, N, dtype=torch.bfloat16, device=dev) for M in M_DECODE}
+            d["Y"] = torch.empty(M_TRAIN, N, dtype=torch.bfloat16, device=dev)
+            d["T"] = torch.empty(M_TRAIN, R, dtype=torch.float32, device=dev)
+            d["dX"] = torch.empty(M_TRAIN, K, dtype=torch.bfloat16, device=dev)
+            d["dA"] = torch.empty(R, K, dtype=torch.bfloat16, device=dev)
+            d["dB"] = torch.empty(N, R, dtype=torch.bfloat16, device=dev)
+            self.lin.append(d)
+        self.ws = torch.empty(self._ws_bytes(), dtype=torch.uint8, device=dev)
+
+    def _ws_bytes(self):
+        import ctypes
+        lib = qb.load_library()
+        need = 0
+        for d in self.lin:
+            for fn in (self._q_call, self._fwd_call, self._bwd_call):
+                n = ctypes.c_size_t(0)
+                fn(lib, d, None, n, None, M_TRAIN)
+                need = max(need, n.value)
+            n = ctypes.c_size_t(0)
+            self._fwd_call(lib, d, None, n, None, 16)
+            need = max(need, n.value)
+        return need
+
+    # raw C-ABI calls (workspace == None: size query)
+    @staticmethod
+    def _q_call(lib, d, ws, n, st, M):
+        import ctypes
+        qc = d["q"].as_c()
+        return lib.qlora_quantize_nf4_dq(qb._ptr(d["W"]), ctypes.byref(qc), ws, ctypes.byref(n), st)
+
+    @staticmethod
+    def _fwd_call(lib, d, ws, n, st, M):
+        import ctypes
+        qc = d["q"].as_c()
+        X = d["X"] if M == M_TRAIN else d["Xdec"][M]
+        Y = d["Y"] if M == M_TRAIN else d["Ydec"][M]
+        T = d["T"] if M == M_TRAIN else None
+        return lib.qlora_linear_fwd(ctypes.byref(qc), qb._ptr(X), M, qb._ptr(d["A"]), qb._ptr(d["B"]), R, ALPHA,
+                                    qb._ptr(Y), qb._ptr(T), ws, ctypes.byref(n), st)
+
+    @staticmethod
+    def _bwd_call(lib, d, ws, n, st, M):
+        import ctypes
+        qc = d["q"].as_c()
+        return lib.qlora_linear_bwd(ctypes.byref(qc), qb._ptr(d["X"]), M, qb._ptr(d["A"]), qb._ptr(d["B"]), R,
+                                    ALPHA, qb._ptr(d["dY"]), qb._ptr(d["T"]), qb._ptr(d["dX"]), qb._ptr(d["dA"]),
+                                    qb._ptr(d["dB"]), ws, ctypes.byref(n), st)
+
+    def step(self, ev=None):
+        """One pass of the hot path. ev: optional dict part -> list of (start, end) events."""
+        import ctypes
+        lib = qb.load_library()
+        st = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+        ws = ctypes.c_void_p(self.ws.data_ptr())
+        n = ctypes.c_size_t(self.ws.numel())
+
+        def rec(part, fn):
+            if ev is not None:
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record()
+                rc = fn()
+                b.record()
+                ev.setdefault(part, []).append((a, b))
+            else:
+                rc = fn()
+            if rc != 0:
+                raise qb.QloraError(rc, part)
+
+        for li, d in enumerate(self.lin):
+            rec(f"quantize/{li}", lambda: self._q_call(lib, d, ws, n, st, 0))
+            qc = d["q"].as_c()
+            rec(f"dequantize/{li}", lambda: lib.qlora_dequantize_nf4_dq(ctypes.byref(qc), qb._ptr(d["Wd"]), st))
+            for M in M_DECODE:
+                rec(f"decode{M}/{li}", lambda: self._fwd_call(lib, d, ws, n, st, M))
+            rec(f"train_fwd/{li}", lambda: self._fwd_call(lib, d, ws, n, st, M_TRAIN))
+            rec(f"train_bwd/{li}", lambda: self._bwd_call(lib, d, ws, n, st, M_TRAIN))
+
+    def launches_per_step(self):
+        per = LAUNCHES["quantize"] + LAUNCHES["dequantize"] + len(M_DECODE) * LAUNCHES["decode_fwd"] + \
+            LAUNCHES["train_fwd"] + LAUNCHES["train_bwd"]
+        return per * len(self.lin)
+
+
+def e2e_step(work: Workload, host):
+    """The same step through the public API with host buffers: pinned H2D copies
+    of the step's inputs, the step, and a D2H read of its results."""
+    h2d = 0
+    for d, h in zip(work.lin, host):
+        for k in ("W", "A", "B", "X", "dY"):
+            d[k].copy_(h[k], non_blocking=True)
+            h2d += h[k].numel() * h[k].element_size()
+        for M in M_DECODE:
+            d["Xdec"][M].copy_(d["X"][:M], non_blocking=True)
+    work.step()
+    d2h = 0
+    for d, h in zip(work.lin, host):
+        for k in ("dA", "dB"):
+            h["out_" + k].copy_(d[k], non_blocking=True)
+            d2h += d[k].numel() * d[k].element_size()
+        for M in M_DECODE:
+            h[f"out_Y{M}"].copy_(d["Ydec"][M], non_blocking=True)
+            d2h += d["Ydec"][M].numel() * 2
+    return h2d, d2h
+
+
+def run_ours(args, rank, world, dev):
+    peaks = load_peaks()
+    work = Workload(dev, seed=rank)
+    fl_train = sum(sum(train_flops(N, K)) for N, K in SHAPES)
+
+    clocks = ClockSampler(gpu_index_for_smi(dev))
+    clocks.start()
+    t_w = time.time()
+    for i in range(args.warmup):
+        work.step()
+        if i == 0:
+            torch.cuda.synchronize()
+    while time.time() - t_w < 1.0:  # let the sampler produce its first lines
+        work.step()
+        torch.cuda.synchronize()
+    torch.cuda.synchronize()
+
+    # per-part times from events inside the timed region (same stream)
+    ev = {}
+    barrier(world)
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    clocks.mark_begin()
+    t0.record()
+    for _ in range(args.steps):
+        work.step(ev)
+    t1.record()
+    torch.cuda.synchronize()
+    clocks.mark_end()
+    barrier(world)
+    clk = clocks.stop()
+    ms_total = t0.elapsed_time(t1)
+    ms_step = max_over_ranks(ms_total / args.steps, world, dev)
+    err = qb.qlora_device_error()
+
+    parts = {}
+    for part, lst in ev.items():
+        kind, li = part.split("/")
+        N, K = SHAPES[int(li)]
+        us = 1e3 * statistics.mean(a.elapsed_time(b) for a, b in lst)
+        e = {"us": round(us, 2)}
+        if kind in ("quantize", "dequantize"):
+            e["GB_s"] = round(quant_bytes(N, K) / us / 1e3, 1)
+        elif kind.startswith("decode"):
+            M = int(kind[len("decode"):])
+            e["GB_s"] = round(decode_bytes(N, K, M) / us / 1e3, 1)
+            e["weight_GB_s"] = round(0.515869 * N * K / us / 1e3, 1)
+        else:
+            f = train_flops(N, K)[0 if kind == "train_fwd" else 1]
+            e["TFLOP_s"] = round(f / us / 1e6, 1)
+        parts[f"{kind}/{N}x{K}"] = e
+
+    # dominant kernel: the forward at M = 4096 (one dequant, one LoRA-down and the
+    # tcgen05 GEMM with the LoRA slab); its flops over its measured duration.
+    fwd_us = [1e3 * statistics.mean(a.elapsed_time(b) for a, b in ev[f"train_fwd/{li}"]) for li in range(3)]
+    fwd_fl = [train_flops(N, K)[0] for N, K in SHAPES]
+    achieved = sum(fwd_fl) / sum(fwd_us) / 1e6
+    roof = {"kernel": "qlora_linear_fwd M=4096 (dequant + LoRA-down + tcgen05 GEMM), 7B shapes",
+            "bound": "tensor", "achieved": round(achieved, 1), "peak": peaks["bf16_tflops_sustained"],
+            "peak_kind": f"bf16 dense sustained ({peaks['source']})", "unit": "TFLOP/s",
+            "frac": round(achieved / peaks["bf16_tflops_sustained"], 4),
+            "frac_of_burst": round(achieved / peaks["bf16_tflops"], 4), "traffic": None}
+    dec = [parts[f"decode{M}/{N}x{K}"]["weight_GB_s"] for M in M_DECODE for N, K in SHAPES]
+
+    # end to end through the C ABI with host buffers
+    host = []
+    for d in work.lin:
+        h = {k: torch.empty_like(d[k], device="cpu").pin_memory() for k in ("W", "A", "B", "X", "dY")}
+        for k in h:
+            h[k].copy_(d[k])
+        h["out_dA"] = torch.empty_like(d["dA"], device="cpu").pin_memory()
+        h["out_dB"] = torch.empty_like(d["dB"], device="cpu").pin_memory()
+        for M in M_DECODE:
+            h[f"out_Y{M}"] = torch.empty_like(d["Ydec"][M], device="cpu").pin_memory()
+        host.append(h)
+    e2e_steps = max(1, min(args.steps, 5))
+    e2e_step(work, host)
+    torch.cuda.synchronize()
+    barrier(world)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(e2e_steps):
+        h2d, d2h = e2e_step(work, host)
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world, dev)
+
+    value = world * fl_train / (ms_step * 1e-3) / 1e12
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded, per-rank seed)",
+        "config": {"workload": "Llama-7B linear shapes 4096x4096, 11008x4096, 4096x11008; r=64 alpha=16; "
+                               "quantize+DQ, dequant, decode M=1/4/16, train fwd+bwd M=4096",
+                   "global_batch_tokens": M_TRAIN * world, "parallelism": f"dp{world} (independent replicas)",
+                   "l2": "inputs larger than L2 (each step touches ~1.2 GB)"},
+        "decode_weight_GB_s": {"min": min(dec), "max": max(dec)},
+        "parts": parts,
+        "roofline": roof,
+        "e2e": {"value": round(world * fl_train / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+                "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": work.launches_per_step() * args.steps,
+        "clocks": clk,
+        "device_error": err,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline_sample(seconds_budget=args.cpu_seconds)
+    return line
+
+
+# ----------------------------------------------------------------------------
+# oracle (CPU) arm
+
+def _threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [p.get("num_threads", 1) for p in threadpool_info() if p.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:  # noqa: BLE001
+        return os.cpu_count() or 1
+
+
+def oracle_step_sample(N=4096, K=4096, M=256, seed=0):
+    """One pass of the hot path on one linear, computed by the CPU oracle:
+    quantize + DQ, dequant, decode M = 1/4/16 and forward + backward at M tokens."""
+    import numpy as np
+    import oracle
+    inp = syn.make_linear(N, K, M, r=R, alpha=ALPHA, seed=seed, workload="llama7b_train", layer=0)
+    f64 = lambda t: t.float().numpy().astype(np.float64)  # noqa: E731
+    Wf = inp.W.float().numpy()
+    X, A, B, dY = f64(inp.X), f64(inp.A), f64(inp.B), f64(inp.dY)
+    t = time.perf_counter()
+    qw = oracle.quantize_nf4_dq(Wf)
+    Wd = oracle.bf16_bits_to_f32(oracle.dequantize_nf4_dq(qw)).astype(np.float64)
+    s = oracle.lora_scale(ALPHA, R)
+    for Md in M_DECODE:
+        oracle.linear_fwd(Wd, X[:Md], A, B, s)
+    oracle.linear_fwd(Wd, X, A, B, s)
+    oracle.linear_bwd(Wd, X, A, B, dY, s)
+    dt = time.perf_counter() - t
+    return sum(train_flops(N, K, M)), dt
+
+
+def cpu_baseline_sample(seconds_budget=20.0):
+    fl, dt = oracle_step_sample()
+    reps = 1
+    while dt * (reps + 1) / reps < seconds_budget and reps < 8 and dt < seconds_budget / 2:
+        f2, d2 = oracle_step_sample(seed=reps)
+        fl += f2
+        dt += d2
+        reps += 1
+    return {"value": round(fl / dt / 1e12, 6), "unit": "TFLOP/s", "cores": _threads(), "kind": "oracle",
+            "sample": f"{reps} x one pass of the hot path on the 4096x4096 linear (quantize+DQ, dequant, "
+                      f"decode M=1/4/16, fwd+bwd at M=256 in fp64); value = fwd+bwd flops / total oracle time",
+            "seconds": round(dt, 2)}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    for _ in range(args.warmup):
+        oracle_step_sample(M=64)
+    fl = 0.0
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        f, _ = oracle_step_sample(seed=i)
+        fl += f
+    dt = time.perf_counter() - t0
+    v = fl / dt / 1e12
+    return {"impl": "reference", "metric": METRIC, "value": round(v, 6), "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * dt / args.steps, 2),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "one pass of the hot path on the 4096x4096 Llama-7B linear per step "
+                                   "(bounded sample of the GPU arm's workload), train M=256, r=64 alpha=16"},
+            "cpu_baseline": {"value": round(v, 6), "unit": "TFLOP/s", "cores": _threads(), "kind": "oracle",
+                             "sample": "per step: quantize+DQ, dequant, decode M=1/4/16, fwd+bwd M=256 on 4096x4096"},
+            "e2e": {"value": round(v, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+# ----------------------------------------------------------------------------
+# distributed plumbing
+
+def gpu_index_for_smi(dev):
+    """Physical index of `dev` for nvidia-smi (honours CUDA_VISIBLE_DEVICES)."""
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        ids = [v.strip() for v in vis.split(",") if v.strip()]
+        if dev.index < len(ids) and ids[dev.index].isdigit():
+            return int(ids[dev.index])
+    return dev.index
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(x, world, dev):
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--cpu-seconds", type=float, default=20.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        print(f"warning: WORLD_SIZE={world} but --gpus={args.gpus}", file=sys.stderr)
+    if args.impl == "reference":
+        if world > 1:
+            torch.distributed.init_process_group("gloo", timeout=__import__("datetime").timedelta(seconds=600))
+        line = run_reference(args, rank, world)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        if world > 1:
+            torch.distributed.destroy_process_group()
+        return
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (the library has no CPU path)")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                             device_id=dev)
+    qb.load_library()
+    line = run_ours(args, rank, world, dev)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -18,6 +18,7 @@ namespace {
 using namespace qlora;
 
 constexpr size_t kAlign = 256;
+constexpr int kRefSms = 148;  // B200
 inline size_t align_up(size_t x, size_t a = kAlign) { return (x + a - 1) / a * a; }
 inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
@@ -68,7 +69,47 @@ qlora_status workspace_check(void* ws, size_t* ws_bytes, size_t need, bool* laun
   return QLORA_OK;
 }
 
+qlora_status check_linear(const void* X, int64_t M, const void* A, const void* B, int32_t r, const void* out) {
+  if (M < 0) return QLORA_ERR_INVALID_ARG;
+  if (r < 8 || r > 256 || r % 8) return QLORA_ERR_UNSUPPORTED;
+  if (!A || !B || (M > 0 && (!X || !out))) return QLORA_ERR_INVALID_ARG;
+  if ((X && !aligned(X, 16)) || !aligned(A, 16) || !aligned(B, 16) || (out && !aligned(out, 16)))
+    return QLORA_ERR_ALIGNMENT;
+  if (M > (int64_t(1) << 31)) return QLORA_ERR_UNSUPPORTED;
+  return QLORA_OK;
+}
+
+float lora_scale(float alpha, int32_t r) { return alpha / static_cast<float>(r); }
+
+int32_t* device_error_word() {
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, qlora::g_device_error) != cudaSuccess) return nullptr;
+  return static_cast<int32_t*>(p);
+}
+
+// Split count for the token reductions of dA / dB: enough units to cover the SMs.
+int grad_splits(int64_t R, int rpad, int64_t M, int num_sms) {
+  const int64_t tiles = ((R + 127) / 128) * (rpad / 64);
+  const int64_t nkb = 2 * ((M + 63) / 64);
+  int64_t sp = (num_sms + tiles - 1) / tiles;
+  if (sp > nkb) sp = nkb;
+  if (sp < 1) sp = 1;
+  return static_cast<int>(sp);
+}
+
+// Workspace layout: consecutive 256-byte aligned regions.
+struct Layout {
+  size_t off = 0;
+  size_t add(size_t bytes) {
+    const size_t o = off;
+    off += align_up(bytes);
+    return o;
+  }
+  size_t total() const { return off > 0 ? off : kAlign; }
+};
+
 }  // namespace
+
 
 extern "C" {
 
@@ -142,18 +183,109 @@ qlora_status qlora_dequantize_nf4_dq(const qlora_nf4_weight* q, void* out_bf16, 
 qlora_status qlora_linear_fwd(const qlora_nf4_weight* q, const void* X, int64_t M, const void* A,
                               const void* B, int32_t r, float alpha, void* Y, float* T_save, void* workspace,
                               size_t* workspace_bytes, qlora_stream_t stream) {
-  (void)q; (void)X; (void)M; (void)A; (void)B; (void)r; (void)alpha; (void)Y; (void)T_save;
-  (void)workspace; (void)workspace_bytes; (void)stream;
-  return QLORA_ERR_UNSUPPORTED;
+  qlora_status st = check_weight(q, true);
+  if (st != QLORA_OK) return st;
+  if ((st = check_linear(X, M, A, B, r, Y)) != QLORA_OK) return st;
+  if (T_save && !aligned(T_save, 4)) return QLORA_ERR_ALIGNMENT;
+  const int64_t N = q->rows, K = q->cols;
+  const int rpad = (r + 63) / 64 * 64;
+  const float s = lora_scale(alpha, r);
+  DeviceInfo di{kRefSms};  // split choices use the reference SM count so the size query needs no device
+  const bool decode = M <= 16;
+  // workspace layout
+  Layout L;
+  size_t off_T = 0, off_part = 0, off_cnt = 0, off_wd = 0, off_sT = 0;
+  int ksplit = 1;
+  if (decode) {
+    ksplit = decode_ksplit(N, K, di.num_sms);
+    off_T = L.add(T_save ? 0 : static_cast<size_t>(M) * r * sizeof(float));
+    off_part = L.add(decode_partial_elems(M, N, ksplit) * sizeof(float));
+    off_cnt = L.add(decode_counter_words(N) * sizeof(unsigned int));
+  } else {
+    off_wd = L.add(static_cast<size_t>(N) * K * 2);
+    off_sT = L.add(static_cast<size_t>(M) * rpad * 2);
+  }
+  bool launch = false;
+  st = workspace_check(workspace, workspace_bytes, L.total(), &launch);
+  if (st != QLORA_OK || !launch || M == 0) return st;
+  if ((st = device_info(&di)) != QLORA_OK) return st;
+  char* ws = static_cast<char*>(workspace);
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  int32_t* err = device_error_word();
+  const float* cb = quant_tables().codebook;
+  if (decode) {
+    float* T = T_save ? T_save : reinterpret_cast<float*>(ws + off_T);
+    Nf4View w{q->packed, q->absmax_q, q->dq_scale, q->mean, N, K};
+    return cuda_status(launch_decode_fwd(w, X, M, A, B, r, s, Y, T, reinterpret_cast<float*>(ws + off_part),
+                                         reinterpret_cast<unsigned int*>(ws + off_cnt), ksplit, cb, cs));
+  }
+  void* Wd = ws + off_wd;
+  void* sT = ws + off_sT;
+  cudaError_t e = launch_dequantize(q->packed, q->absmax_q, q->dq_scale, q->mean, Wd, N * K, cb, di.num_sms, cs);
+  if (e == cudaSuccess)
+    e = launch_gemm_lora_t(X, A, M, K, r, rpad, s, T_save, sT, nullptr, nullptr, di.num_sms, err, cs);
+  if (e == cudaSuccess) e = launch_gemm_fwd(X, Wd, sT, B, M, N, K, r, rpad, Y, di.num_sms, err, cs);
+  return cuda_status(e);
 }
 
 qlora_status qlora_linear_bwd(const qlora_nf4_weight* q, const void* X, int64_t M, const void* A,
                               const void* B, int32_t r, float alpha, const void* dY, const float* T_saved,
                               void* dX, void* dA, void* dB, void* workspace, size_t* workspace_bytes,
                               qlora_stream_t stream) {
-  (void)q; (void)X; (void)M; (void)A; (void)B; (void)r; (void)alpha; (void)dY; (void)T_saved;
-  (void)dX; (void)dA; (void)dB; (void)workspace; (void)workspace_bytes; (void)stream;
-  return QLORA_ERR_UNSUPPORTED;
+  qlora_status st = check_weight(q, true);
+  if (st != QLORA_OK) return st;
+  if ((st = check_linear(X, M, A, B, r, dA)) != QLORA_OK) return st;
+  if (!dA || !dB || (M > 0 && !dY)) return QLORA_ERR_INVALID_ARG;
+  if (!aligned(dB, 16) || (dY && !aligned(dY, 16)) || (dX && !aligned(dX, 16))) return QLORA_ERR_ALIGNMENT;
+  if (T_saved && !aligned(T_saved, 4)) return QLORA_ERR_ALIGNMENT;
+  const int64_t N = q->rows, K = q->cols;
+  if (N % 8) return QLORA_ERR_UNSUPPORTED;  // dY rows must be 16-byte multiples for the TMA tiles
+  const int rpad = (r + 63) / 64 * 64;
+  const float s = lora_scale(alpha, r);
+  DeviceInfo di{kRefSms};
+  const int splits_a = grad_splits(K, rpad, M, di.num_sms);
+  const int splits_b = grad_splits(N, rpad, M, di.num_sms);
+  Layout L;
+  const size_t mp = static_cast<size_t>(M) * rpad * 2;
+  const size_t off_wd = L.add(dX ? static_cast<size_t>(N) * K * 2 : 0);
+  const size_t off_thi = L.add(mp), off_tlo = L.add(mp);
+  const size_t off_su = L.add(mp), off_uhi = L.add(mp), off_ulo = L.add(mp);
+  const size_t pa = static_cast<size_t>(splits_a) * K * rpad, pb = static_cast<size_t>(splits_b) * N * rpad;
+  const size_t off_p = L.add((pa > pb ? pa : pb) * sizeof(float));
+  bool launch = false;
+  st = workspace_check(workspace, workspace_bytes, L.total(), &launch);
+  if (st != QLORA_OK || !launch) return st;
+  if ((st = device_info(&di)) != QLORA_OK) return st;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  if (M == 0) {
+    cudaError_t e = launch_zero_bf16(dA, static_cast<int64_t>(r) * K, di.num_sms, cs);
+    if (e == cudaSuccess) e = launch_zero_bf16(dB, N * r, di.num_sms, cs);
+    return cuda_status(e);
+  }
+  char* ws = static_cast<char*>(workspace);
+  int32_t* err = device_error_word();
+  const float* cb = quant_tables().codebook;
+  void *Thi = ws + off_thi, *Tlo = ws + off_tlo, *sU = ws + off_su, *Uhi = ws + off_uhi, *Ulo = ws + off_ulo;
+  float* P = reinterpret_cast<float*>(ws + off_p);
+  cudaError_t e = cudaSuccess;
+  // T = X A^T as a two-term bf16 split (from the saved fp32 T or recomputed)
+  if (T_saved) e = launch_split_hilo(T_saved, M, r, rpad, Thi, Tlo, di.num_sms, cs);
+  else e = launch_gemm_lora_t(X, A, M, K, r, rpad, s, nullptr, nullptr, Thi, Tlo, di.num_sms, err, cs);
+  // U = dY B: s U for the dX slab, U as hi + lo for dA
+  if (e == cudaSuccess) e = launch_gemm_lora_u(dY, B, M, N, r, rpad, s, sU, Uhi, Ulo, di.num_sms, err, cs);
+  if (dX) {
+    void* Wd = ws + off_wd;
+    if (e == cudaSuccess)
+      e = launch_dequantize(q->packed, q->absmax_q, q->dq_scale, q->mean, Wd, N * K, cb, di.num_sms, cs);
+    if (e == cudaSuccess) e = launch_gemm_dx(dY, Wd, sU, A, M, N, K, r, rpad, dX, di.num_sms, err, cs);
+  }
+  // dA^T [K, r] = X^T U, reduced over tokens, then dA = s * (.)^T
+  if (e == cudaSuccess) e = launch_gemm_lora_grad(X, K, Uhi, Ulo, M, rpad, P, splits_a, di.num_sms, err, cs);
+  if (e == cudaSuccess) e = launch_grad_reduce(P, splits_a, K, rpad, r, s, true, dA, di.num_sms, cs);
+  // dB [N, r] = dY^T T
+  if (e == cudaSuccess) e = launch_gemm_lora_grad(dY, N, Thi, Tlo, M, rpad, P, splits_b, di.num_sms, err, cs);
+  if (e == cudaSuccess) e = launch_grad_reduce(P, splits_b, N, rpad, r, s, false, dB, di.num_sms, cs);
+  return cuda_status(e);
 }
 
 qlora_status qlora_device_error(int32_t* code, qlora_stream_t stream) {

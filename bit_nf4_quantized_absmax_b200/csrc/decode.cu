@@ -1,0 +1,274 @@
+// Decode-shaped QLoRA forward (M <= 16 tokens), bound by the bandwidth of the
+// packed 4-bit weights ("QLoRA vs ChatGPT", capability 5: the frozen weight is
+// dequantized on the fly, block by block).
+//
+// Y[M, N] = X W'^T + s T B^T with T = X A^T computed first (k_lora_t_small).
+//
+// k_decode computes D = W' X^T with the weight as the MMA's A operand
+// (mma.sync m16n8k16, bf16 in, fp32 accumulate) so that the 16 weight rows fill
+// the MMA's M dimension and the tokens its N dimension. The reduction index is
+// permuted: over a 256-wide "superblock" lane (g, t) supplies k-slots
+// {2t, 2t+1, 2t+8, 2t+9} of every one of the 16 MMAs from the 64 consecutive
+// weights of block 4*sb + t of rows g and g+8, and the matching token values.
+// Each lane therefore decodes whole 64-weight blocks: one 16-entry bf16 table
+// per block (bit-identical to the standalone dequant) and byte-permute lookups.
+// The K range of a row tile may be split across CTAs; the last CTA of a row
+// tile (ticket counter, no waiting) sums the partials in a fixed order and
+// applies the LoRA term.
+#include "common.cuh"
+#include "kernels.h"
+#include "nf4_lut.cuh"
+
+namespace qlora {
+namespace {
+
+constexpr int kDecodeWarps = 4;
+
+__device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+struct RowBlock {
+  uint4 n0, n1;   // 64 codes
+  float mp;       // decoded block constant
+};
+
+__device__ __forceinline__ RowBlock load_row_block(const uint8_t* __restrict__ packed, const int8_t* __restrict__ q,
+                                                   const float* __restrict__ dqs, float mu, int64_t n,
+                                                   int64_t nkb_row, int64_t kb, bool valid) {
+  RowBlock rb;
+  if (valid) {
+    const int64_t blk = n * nkb_row + kb;
+    const uint4* p = reinterpret_cast<const uint4*>(packed + blk * 32);
+    rb.n0 = __ldcs(p);
+    rb.n1 = __ldcs(p + 1);
+    rb.mp = __fmaf_rn(static_cast<float>(q[blk]), dqs[blk >> 8], mu);
+  } else {
+    rb.n0 = make_uint4(0x77777777u, 0x77777777u, 0x77777777u, 0x77777777u);
+    rb.n1 = rb.n0;
+    rb.mp = 0.0f;
+  }
+  return rb;
+}
+
+__device__ __forceinline__ uint32_t nib_word(const RowBlock& rb, int w) {
+  switch (w) {
+    case 0: return rb.n0.x;
+    case 1: return rb.n0.y;
+    case 2: return rb.n0.z;
+    case 3: return rb.n0.w;
+    case 4: return rb.n1.x;
+    case 5: return rb.n1.y;
+    case 6: return rb.n1.z;
+    default: return rb.n1.w;
+  }
+}
+
+template <int MT>
+__global__ void __launch_bounds__(kDecodeWarps * 32)
+k_decode(const uint8_t* __restrict__ packed, const int8_t* __restrict__ q, const float* __restrict__ dqs,
+         const float* __restrict__ mean, const __nv_bfloat16* __restrict__ X, int M, int64_t N, int64_t K,
+         const float* __restrict__ T, const __nv_bfloat16* __restrict__ Bl, int r, float s,
+         __nv_bfloat16* __restrict__ Y, float* __restrict__ partial, unsigned int* __restrict__ counters,
+         int ksplit, const __grid_constant__ Nf4Codebook cb) {
+  __shared__ float red[kDecodeWarps][16][16];
+  __shared__ int s_last;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, t = lane & 3;
+  const int64_t n0 = static_cast<int64_t>(blockIdx.x) * 16;
+  const int split = blockIdx.y;
+  const int64_t nkb_row = K / 64;
+  const int64_t nsb = (nkb_row + 3) / 4;
+  const int64_t per = (nsb + ksplit - 1) / ksplit;
+  const int64_t sb_begin = split * per;
+  const int64_t sb_end = min(nsb, sb_begin + per);
+  const float mu = *mean;
+  const int64_t na = n0 + g, nb = n0 + g + 8;
+
+  float acc[MT][4];
+#pragma unroll
+  for (int j = 0; j < MT; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.0f;
+
+  for (int64_t sb = sb_begin + warp; sb < sb_end; sb += kDecodeWarps) {
+    const int64_t kb = sb * 4 + t;
+    const bool kv = kb < nkb_row;
+    const RowBlock ra = load_row_block(packed, q, dqs, mu, na, nkb_row, kb, kv && na < N);
+    const RowBlock rbk = load_row_block(packed, q, dqs, mu, nb, nkb_row, kb, kv && nb < N);
+    // token values for this lane's 64 k positions: tokens g (tile 0) and g + 8 (tile 1)
+    uint4 xv[MT][8];
+#pragma unroll
+    for (int j = 0; j < MT; ++j) {
+      const int tok = g + 8 * j;
+      const bool ok = kv && tok < M;
+      const uint4* xp = reinterpret_cast<const uint4*>(X + static_cast<int64_t>(tok) * K + kb * 64);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) xv[j][i] = ok ? __ldg(xp + i) : make_uint4(0, 0, 0, 0);
+    }
+    const Nf4Lut la = make_nf4_lut(cb, ra.mp);
+    const Nf4Lut lb = make_nf4_lut(cb, rbk.mp);
+#pragma unroll
+    for (int st = 0; st < 16; ++st) {
+      const uint32_t wa = nib_word(ra, st >> 1) >> (16 * (st & 1));
+      const uint32_t wb = nib_word(rbk, st >> 1) >> (16 * (st & 1));
+      uint32_t a0, a1, a2, a3;
+      nf4_lookup4(la, wa, a0, a2);   // row g: k-slots (2t, 2t+1) and (2t+8, 2t+9)
+      nf4_lookup4(lb, wb, a1, a3);   // row g + 8
+#pragma unroll
+      for (int j = 0; j < MT; ++j) {
+        const uint4 x4 = xv[j][st >> 1];
+        const uint32_t b0 = (st & 1) ? x4.z : x4.x;
+        const uint32_t b1 = (st & 1) ? x4.w : x4.y;
+        mma16816(acc[j], a0, a1, a2, a3, b0, b1);
+      }
+    }
+  }
+
+  // acc[j]: (row g, token 8j + 2t), (g, 8j + 2t + 1), (g + 8, 8j + 2t), (g + 8, 8j + 2t + 1)
+#pragma unroll
+  for (int j = 0; j < MT; ++j) {
+    red[warp][g][8 * j + 2 * t] = acc[j][0];
+    red[warp][g][8 * j + 2 * t + 1] = acc[j][1];
+    red[warp][g + 8][8 * j + 2 * t] = acc[j][2];
+    red[warp][g + 8][8 * j + 2 * t + 1] = acc[j][3];
+  }
+  __syncthreads();
+
+  const int ntok = 8 * MT;
+  if (ksplit == 1) {
+    for (int e = threadIdx.x; e < 16 * ntok; e += blockDim.x) {
+      const int row = e / ntok, tok = e % ntok;
+      const int64_t n = n0 + row;
+      if (tok >= M || n >= N) continue;
+      float y = 0.0f;
+#pragma unroll
+      for (int w = 0; w < kDecodeWarps; ++w) y += red[w][row][tok];
+      float l = 0.0f;
+      for (int jj = 0; jj < r; ++jj)
+        l = fmaf(T[static_cast<int64_t>(tok) * r + jj], __bfloat162float(Bl[n * r + jj]), l);
+      Y[static_cast<int64_t>(tok) * N + n] = __float2bfloat16_rn(fmaf(s, l, y));
+    }
+    return;
+  }
+
+  // split K: publish this CTA's partial, the last CTA of the row tile finishes
+  for (int e = threadIdx.x; e < 16 * ntok; e += blockDim.x) {
+    const int row = e / ntok, tok = e % ntok;
+    const int64_t n = n0 + row;
+    if (tok >= M || n >= N) continue;
+    float y = 0.0f;
+#pragma unroll
+    for (int w = 0; w < kDecodeWarps; ++w) y += red[w][row][tok];
+    partial[(static_cast<int64_t>(split) * M + tok) * N + n] = y;
+  }
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const unsigned int prev = atomicAdd(&counters[blockIdx.x], 1u);
+    s_last = (prev == static_cast<unsigned int>(ksplit - 1)) ? 1 : 0;
+  }
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  for (int e = threadIdx.x; e < 16 * ntok; e += blockDim.x) {
+    const int row = e / ntok, tok = e % ntok;
+    const int64_t n = n0 + row;
+    if (tok >= M || n >= N) continue;
+    float y = 0.0f;
+    for (int sp = 0; sp < ksplit; ++sp) y += __ldcg(&partial[(static_cast<int64_t>(sp) * M + tok) * N + n]);
+    float l = 0.0f;
+    for (int jj = 0; jj < r; ++jj)
+      l = fmaf(T[static_cast<int64_t>(tok) * r + jj], __bfloat162float(Bl[n * r + jj]), l);
+    Y[static_cast<int64_t>(tok) * N + n] = __float2bfloat16_rn(fmaf(s, l, y));
+  }
+  if (threadIdx.x == 0) counters[blockIdx.x] = 0u;
+}
+
+// T[m, j] = sum_k X[m, k] A[j, k] for M <= 16 (fp32 on CUDA cores), one CTA per
+// adapter row j. Block 0 also clears the decode kernel's ticket counters.
+__global__ void __launch_bounds__(256)
+k_lora_t_small(const __nv_bfloat16* __restrict__ X, const __nv_bfloat16* __restrict__ A, int M, int64_t K, int r,
+               float* __restrict__ T, unsigned int* __restrict__ counters, int n_counters) {
+  __shared__ float red[8][16];
+  const int j = blockIdx.x;
+  if (j == 0)
+    for (int i = threadIdx.x; i < n_counters; i += blockDim.x) counters[i] = 0u;
+  float acc[16];
+#pragma unroll
+  for (int m = 0; m < 16; ++m) acc[m] = 0.0f;
+  const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(A + static_cast<int64_t>(j) * K);
+  for (int64_t k2 = threadIdx.x; k2 < K / 2; k2 += blockDim.x) {
+    const float2 av = __bfloat1622float2(a2[k2]);
+#pragma unroll
+    for (int m = 0; m < 16; ++m) {
+      if (m < M) {
+        const float2 xv =
+            __bfloat1622float2(reinterpret_cast<const __nv_bfloat162*>(X + static_cast<int64_t>(m) * K)[k2]);
+        acc[m] = fmaf(av.x, xv.x, fmaf(av.y, xv.y, acc[m]));
+      }
+    }
+  }
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+#pragma unroll
+  for (int m = 0; m < 16; ++m) {
+    float v = acc[m];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    if (lane == 0) red[warp][m] = v;
+  }
+  __syncthreads();
+  if (threadIdx.x < M) {
+    float v = 0.0f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) v += red[w][threadIdx.x];
+    T[static_cast<int64_t>(threadIdx.x) * r + j] = v;
+  }
+}
+
+}  // namespace
+
+int decode_ksplit(int64_t N, int64_t K, int num_sms) {
+  const int64_t row_tiles = (N + 15) / 16;
+  const int64_t nsb = (K / 64 + 3) / 4;
+  int64_t want = (4 * static_cast<int64_t>(num_sms) + row_tiles - 1) / row_tiles;
+  int64_t cap = nsb / 2 > 0 ? nsb / 2 : 1;
+  if (want > cap) want = cap;
+  if (want < 1) want = 1;
+  return static_cast<int>(want);
+}
+
+size_t decode_partial_elems(int64_t M, int64_t N, int ksplit) {
+  return ksplit > 1 ? static_cast<size_t>(ksplit) * M * N : 0;
+}
+
+size_t decode_counter_words(int64_t N) { return static_cast<size_t>((N + 15) / 16); }
+
+cudaError_t launch_decode_fwd(const Nf4View& w, const void* X, int64_t M, const void* A, const void* B, int r,
+                              float s, void* Y, float* T, float* partial, unsigned int* counters, int ksplit,
+                              const float codebook[16], cudaStream_t stream) {
+  Nf4Codebook cb;
+  for (int i = 0; i < 16; ++i) cb.c[i] = codebook[i];
+  const int64_t row_tiles = (w.N + 15) / 16;
+  k_lora_t_small<<<r, 256, 0, stream>>>(reinterpret_cast<const __nv_bfloat16*>(X),
+                                        reinterpret_cast<const __nv_bfloat16*>(A), static_cast<int>(M), w.K, r, T,
+                                        counters, static_cast<int>(row_tiles));
+  dim3 grid(static_cast<unsigned>(row_tiles), static_cast<unsigned>(ksplit));
+  if (M <= 8) {
+    k_decode<1><<<grid, kDecodeWarps * 32, 0, stream>>>(
+        w.packed, w.absmax_q, w.dq_scale, w.mean, reinterpret_cast<const __nv_bfloat16*>(X), static_cast<int>(M), w.N,
+        w.K, T, reinterpret_cast<const __nv_bfloat16*>(B), r, s, reinterpret_cast<__nv_bfloat16*>(Y), partial,
+        counters, ksplit, cb);
+  } else {
+    k_decode<2><<<grid, kDecodeWarps * 32, 0, stream>>>(
+        w.packed, w.absmax_q, w.dq_scale, w.mean, reinterpret_cast<const __nv_bfloat16*>(X), static_cast<int>(M), w.N,
+        w.K, T, reinterpret_cast<const __nv_bfloat16*>(B), r, s, reinterpret_cast<__nv_bfloat16*>(Y), partial,
+        counters, ksplit, cb);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace qlora

@@ -1,0 +1,519 @@
+// Persistent tcgen05 GEMM for sm_100a: TMA loads into 128-byte-swizzled shared
+// memory, one thread issues tcgen05.mma (bf16 x bf16 -> fp32) into a
+// double-buffered TMEM accumulator, four epilogue warps drain TMEM with
+// tcgen05.ld while the next tile's mainloop runs.
+//
+//   C[M, Nc] = A1[M, K1] op(B1) + A2[M, K2] op(B2)
+//
+// The second pair ("slab") carries the rank-r LoRA term: for the forward pass
+// [X | s T] [W' | B]^T, for dX [dY | s U] [W' ; A] ("QLoRA vs ChatGPT",
+// capability 2: the adapter sits beside the frozen weight; capability 5: it is
+// the only part that receives gradients). A and B may each be K-major (the
+// reduction index contiguous) or MN-major (the output index contiguous); the
+// TMA boxes and UMMA shared-memory descriptors follow the operand's layout.
+//
+// Warp roles (192 threads): warp 0 issues TMA, warp 1 allocates TMEM and issues
+// MMAs, warps 2..5 run the epilogue (warp w reads TMEM lanes 32*(w%4)..+31).
+// Every mbarrier wait is bounded; a timeout records an error word and makes the
+// CTA leave its loops.
+#include <cuda.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace qlora {
+namespace {
+
+constexpr int BM = 128;
+constexpr int BK = 64;
+constexpr int kThreads = 192;
+
+enum OutMode : int { OUT_BF16 = 0, OUT_LORA = 1, OUT_PARTIAL = 2 };
+
+struct EpiParams {
+  void* C; int64_t ldc;                    // OUT_BF16: bf16 [M, ldc]
+  float* f32; int64_t ld_f32;              // OUT_LORA: optional fp32 copy [M, ld_f32] (cols < Nc)
+  void* s_bf16; void* hi; void* lo;        // OUT_LORA: bf16 [M, ld_pad]: s*C, C, C - bf16(C)
+  int64_t ld_pad; float s;
+  float* P;                                // OUT_PARTIAL: fp32 [splits][M][Nc]
+};
+
+struct TileSched {
+  int tiles_m, tiles_n, splits;
+  int nkb;        // total k-blocks (main + slab)
+  int nk1;        // k-blocks of the main pair
+  int kb_per_split;
+};
+
+template <int BN>
+struct Cfg {
+  static constexpr int A_BYTES = BM * BK * 2;
+  static constexpr int B_BYTES = BN * BK * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int STAGES = (200 * 1024) / STAGE_BYTES > 8 ? 8 : (200 * 1024) / STAGE_BYTES;
+  static constexpr int TMEM_COLS = (2 * BN) < 32 ? 32 : 2 * BN;
+  static constexpr int SMEM = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+};
+
+__device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16;
+  d |= static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32;
+  d |= static_cast<uint64_t>(1) << 46;  // descriptor version for sm_100
+  d |= static_cast<uint64_t>(2) << 61;  // 128-byte swizzle
+  return d;
+}
+
+constexpr uint32_t instr_desc(int M, int N, bool a_mn, bool b_mn) {
+  return (1u << 4)                       // D format fp32
+         | (1u << 7) | (1u << 10)        // A, B bf16
+         | ((a_mn ? 1u : 0u) << 15) | ((b_mn ? 1u : 0u) << 16)
+         | (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(idesc), "r"(acc));
+}
+
+__device__ __forceinline__ void mma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Bounded wait that also gives up when another role has already aborted.
+__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                              int32_t* err, int32_t code) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity)) {
+    if (*abort_flag) return false;
+    if (clock64() - t0 > kWaitBoundCycles) {
+      report_error(err, code);
+      *abort_flag = 1;
+      return false;
+    }
+  }
+  return true;
+}
+
+__device__ __forceinline__ void decode_unit(const TileSched& ts, int unit, int& tm, int& tn, int& kb0, int& kb1) {
+  tm = unit % ts.tiles_m;
+  const int rest = unit / ts.tiles_m;
+  tn = rest % ts.tiles_n;
+  const int split = rest / ts.tiles_n;
+  kb0 = split * ts.kb_per_split;
+  kb1 = min(ts.nkb, kb0 + ts.kb_per_split);
+}
+
+template <int BN, bool A_MN, bool B_MN, int OUT>
+__global__ void __launch_bounds__(kThreads, 1)
+k_tc_gemm(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmB1,
+          const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2, TileSched ts,
+          int M, int Nc, EpiParams ep, int32_t* err) {
+  using C = Cfg<BN>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
+  uint64_t* empty = full + C::STAGES;
+  uint64_t* accf = empty + C::STAGES;
+  uint64_t* acce = accf + 2;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(acce + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int n_units = ts.tiles_m * ts.tiles_n * ts.splits;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&accf[a], 1);
+      mbar_init(&acce[a], 128);
+    }
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmA1);
+    prefetch_tmap(&tmB1);
+    prefetch_tmap(&tmA2);
+    prefetch_tmap(&tmB2);
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_holder)),
+                 "r"(C::TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  if (warp == 0) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t outstanding = 0;      // stages loaded but not yet seen freed
+      uint32_t out_parity = 0;       // parity each outstanding stage's load completes with
+      bool ok = true;
+      for (int unit = blockIdx.x; unit < n_units && ok; unit += gridDim.x) {
+        int tm, tn, kb0, kb1;
+        decode_unit(ts, unit, tm, tn, kb0, kb1);
+        const int m0 = tm * BM, n0 = tn * BN;
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!wait_or_abort(&empty[stage], phase ^ 1u, abort_flag, err, DEV_TIMEOUT_SMEM_EMPTY)) {
+            ok = false;
+            break;
+          }
+          outstanding &= ~(1u << stage);
+          uint8_t* sa = smem + stage * C::STAGE_BYTES;
+          uint8_t* sb = sa + C::A_BYTES;
+          mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES);
+          const bool slab = kb >= ts.nk1;
+          const CUtensorMap* ta = slab ? &tmA2 : &tmA1;
+          const CUtensorMap* tb = slab ? &tmB2 : &tmB1;
+          const int k0 = (slab ? kb - ts.nk1 : kb) * BK;
+          if (A_MN) {
+            tma_load_2d(sa, ta, &full[stage], m0, k0);
+            tma_load_2d(sa + 8192, ta, &full[stage], m0 + 64, k0);
+          } else {
+            tma_load_2d(sa, ta, &full[stage], k0, m0);
+          }
+          if (B_MN) {
+#pragma unroll
+            for (int j = 0; j < BN / 64; ++j) tma_load_2d(sb + j * 8192, tb, &full[stage], n0 + 64 * j, k0);
+          } else {
+            tma_load_2d(sb, tb, &full[stage], k0, n0);
+          }
+          outstanding |= (1u << stage);
+          out_parity = (out_parity & ~(1u << stage)) | (phase << stage);
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok) {
+        // Let the copies already issued land before the CTA exits.
+        for (int s = 0; s < C::STAGES; ++s)
+          if (outstanding & (1u << s)) mbar_wait_bounded(&full[s], (out_parity >> s) & 1u, err, DEV_TIMEOUT_TMA_FULL);
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      constexpr uint32_t idesc = instr_desc(BM, BN, A_MN, B_MN);
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int unit = blockIdx.x; unit < n_units && ok; unit += gridDim.x) {
+        int tm, tn, kb0, kb1;
+        decode_unit(ts, unit, tm, tn, kb0, kb1);
+        if (!wait_or_abort(&acce[acc], acc_phase ^ 1u, abort_flag, err, DEV_TIMEOUT_TMEM_EMPTY)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!wait_or_abort(&full[stage], phase, abort_flag, err, DEV_TIMEOUT_TMA_FULL)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(smem + stage * C::STAGE_BYTES);
+          const uint32_t sb = sa + C::A_BYTES;
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k) {
+            const uint64_t da = A_MN ? smem_desc(sa + k * 2048, 8192, 1024) : smem_desc(sa + k * 32, 16, 1024);
+            const uint64_t db = B_MN ? smem_desc(sb + k * 2048, 8192, 1024) : smem_desc(sb + k * 32, 16, 1024);
+            mma_bf16(d_tmem, da, db, idesc, (kb > kb0 || k > 0) ? 1u : 0u);
+          }
+          mma_commit(&empty[stage]);  // frees the stage once these MMAs have read it
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        mma_commit(&accf[acc]);       // accumulator ready for the epilogue
+        if (++acc == 2) {
+          acc = 0;
+          acc_phase ^= 1u;
+        }
+      }
+    }
+  } else {
+    // ---------------- epilogue (warps 2..5) ----------------
+    const int quarter = warp & 3;
+    const int row_in_tile = quarter * 32 + lane;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int unit = blockIdx.x; unit < n_units; unit += gridDim.x) {
+      int tm, tn, kb0, kb1;
+      decode_unit(ts, unit, tm, tn, kb0, kb1);
+      const int split = unit / (ts.tiles_m * ts.tiles_n);
+      if (!wait_or_abort(&accf[acc], acc_phase, abort_flag, err, DEV_TIMEOUT_ACCUM)) break;
+      tc_fence_after();
+      const int row = tm * BM + row_in_tile;
+      const bool row_ok = row < M;
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        float v[32];
+        tmem_ld32(tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(acc * BN + c * 32),
+                  v);
+        const int col0 = tn * BN + c * 32;
+        if (!row_ok) continue;
+        if (OUT == OUT_BF16) {
+          __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(ep.C) + static_cast<int64_t>(row) * ep.ldc + col0;
+          if (col0 + 32 <= Nc && (ep.ldc % 8) == 0) {
+            uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              d4[q] = make_uint4(pack_bf16x2(v[8 * q + 0], v[8 * q + 1]), pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
+                                 pack_bf16x2(v[8 * q + 4], v[8 * q + 5]), pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (col0 + j < Nc) dst[j] = __float2bfloat16_rn(v[j]);
+          }
+        } else if (OUT == OUT_LORA) {
+          const int64_t po = static_cast<int64_t>(row) * ep.ld_pad + col0;
+          uint4* sd = ep.s_bf16 ? reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(ep.s_bf16) + po) : nullptr;
+          uint4* hd = ep.hi ? reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(ep.hi) + po) : nullptr;
+          uint4* ld = ep.lo ? reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(ep.lo) + po) : nullptr;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            uint32_t s4[4], h4[4], l4[4];
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+              const float a = v[8 * q + 2 * h], b = v[8 * q + 2 * h + 1];
+              s4[h] = pack_bf16x2(ep.s * a, ep.s * b);
+              h4[h] = pack_bf16x2(a, b);
+              const float ah = bf16lo_to_f32(h4[h]), bh = bf16hi_to_f32(h4[h]);
+              l4[h] = pack_bf16x2(a - ah, b - bh);
+            }
+            if (sd) sd[q] = make_uint4(s4[0], s4[1], s4[2], s4[3]);
+            if (hd) hd[q] = make_uint4(h4[0], h4[1], h4[2], h4[3]);
+            if (ld) ld[q] = make_uint4(l4[0], l4[1], l4[2], l4[3]);
+          }
+          if (ep.f32) {
+            float* fd = ep.f32 + static_cast<int64_t>(row) * ep.ld_f32;
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (col0 + j < Nc) fd[col0 + j] = v[j];
+          }
+        } else {  // OUT_PARTIAL
+          float* pd = ep.P + (static_cast<int64_t>(split) * M + row) * Nc + col0;
+          if (col0 + 32 <= Nc && (Nc % 4) == 0) {
+            float4* p4 = reinterpret_cast<float4*>(pd);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) p4[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (col0 + j < Nc) pd[j] = v[j];
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&acce[acc]);
+      if (++acc == 2) {
+        acc = 0;
+        acc_phase ^= 1u;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(C::TMEM_COLS)
+                 : "memory");
+  }
+}
+
+// ---------------------------------------------------------------------------
+// host side
+
+typedef CUresult (*PFN_encodeTiled)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                    const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                    CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+PFN_encodeTiled get_encoder() {
+  static PFN_encodeTiled fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return static_cast<PFN_encodeTiled>(nullptr);
+    return reinterpret_cast<PFN_encodeTiled>(p);
+  }();
+  return fn;
+}
+
+// 2-D bf16 tensor [outer, inner] with row stride ld (elements); box {64, box_outer}.
+bool make_map(CUtensorMap* m, const void* base, int64_t inner, int64_t outer, int64_t ld, int box_outer) {
+  PFN_encodeTiled enc = get_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(outer)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * 2};
+  cuuint32_t box[2] = {64u, static_cast<cuuint32_t>(box_outer)};
+  cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// Operand description for the host launcher.
+struct Operand {
+  const void* p;
+  int64_t rows_mn;   // extent along the GEMM's M (for A) or N (for B)
+  int64_t k;         // extent along the reduction
+  int64_t ld;        // row stride in elements of the stored matrix
+  bool mn_major;     // stored [k, mn] (mn contiguous) instead of [mn, k]
+};
+
+bool map_operand(CUtensorMap* m, const Operand& o, int tile_mn) {
+  if (o.mn_major) return make_map(m, o.p, o.rows_mn, o.k, o.ld, 64);
+  return make_map(m, o.p, o.k, o.rows_mn, o.ld, tile_mn);
+}
+
+template <int BN, bool A_MN, bool B_MN, int OUT>
+cudaError_t run(const Operand& a1, const Operand& b1, const Operand* a2, const Operand* b2, int M, int Nc,
+                int splits, const EpiParams& ep, int num_sms, int32_t* err, cudaStream_t stream) {
+  using C = Cfg<BN>;
+  CUtensorMap ta1, tb1, ta2, tb2;
+  if (!map_operand(&ta1, a1, BM) || !map_operand(&tb1, b1, BN)) return cudaErrorInvalidValue;
+  if (a2 && b2) {
+    if (!map_operand(&ta2, *a2, BM) || !map_operand(&tb2, *b2, BN)) return cudaErrorInvalidValue;
+  } else {
+    ta2 = ta1;
+    tb2 = tb1;
+  }
+  TileSched ts;
+  ts.tiles_m = static_cast<int>((M + BM - 1) / BM);
+  ts.tiles_n = static_cast<int>((Nc + BN - 1) / BN);
+  ts.nk1 = static_cast<int>((a1.k + BK - 1) / BK);
+  const int nk2 = (a2 && b2) ? static_cast<int>((a2->k + BK - 1) / BK) : 0;
+  ts.nkb = ts.nk1 + nk2;
+  if (splits < 1) splits = 1;
+  if (splits > ts.nkb) splits = ts.nkb;
+  ts.kb_per_split = (ts.nkb + splits - 1) / splits;
+  ts.splits = (ts.nkb + ts.kb_per_split - 1) / ts.kb_per_split;
+  const int units = ts.tiles_m * ts.tiles_n * ts.splits;
+  const int grid = units < num_sms ? units : num_sms;
+  auto kern = k_tc_gemm<BN, A_MN, B_MN, OUT>;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  kern<<<grid, kThreads, C::SMEM, stream>>>(ta1, tb1, ta2, tb2, ts, M, Nc, ep, err);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+// Forward main GEMM: Y[M,N] = X[M,K] W'[N,K]^T + sT[M,rpad] Bl[N,r]^T
+cudaError_t launch_gemm_fwd(const void* X, const void* Wd, const void* sT, const void* Bl, int64_t M, int64_t N,
+                            int64_t K, int r, int rpad, void* Y, int num_sms, int32_t* err, cudaStream_t stream) {
+  Operand a1{X, M, K, K, false}, b1{Wd, N, K, K, false};
+  Operand a2{sT, M, rpad, rpad, false}, b2{Bl, N, r, r, false};
+  EpiParams ep{};
+  ep.C = Y;
+  ep.ldc = N;
+  return run<256, false, false, OUT_BF16>(a1, b1, &a2, &b2, static_cast<int>(M), static_cast<int>(N), 1, ep,
+                                          num_sms, err, stream);
+}
+
+// Backward dX: dX[M,K] = dY[M,N] W'[N,K] + sU[M,rpad] A[r,K]
+cudaError_t launch_gemm_dx(const void* dY, const void* Wd, const void* sU, const void* Al, int64_t M, int64_t N,
+                           int64_t K, int r, int rpad, void* dX, int num_sms, int32_t* err, cudaStream_t stream) {
+  Operand a1{dY, M, N, N, false}, b1{Wd, K, N, K, true};
+  Operand a2{sU, M, rpad, rpad, false}, b2{Al, K, r, K, true};
+  EpiParams ep{};
+  ep.C = dX;
+  ep.ldc = K;
+  return run<256, false, true, OUT_BF16>(a1, b1, &a2, &b2, static_cast<int>(M), static_cast<int>(K), 1, ep,
+                                         num_sms, err, stream);
+}
+
+// LoRA down projection: T[M, r] = X[M,K] A[r,K]^T; writes T (fp32, optional),
+// sT = bf16(s T), T_hi = bf16(T), T_lo = bf16(T - T_hi), all [M, rpad].
+cudaError_t launch_gemm_lora_t(const void* X, const void* Al, int64_t M, int64_t K, int r, int rpad, float s,
+                               float* T, void* sT, void* T_hi, void* T_lo, int num_sms, int32_t* err,
+                               cudaStream_t stream) {
+  Operand a1{X, M, K, K, false}, b1{Al, r, K, K, false};
+  EpiParams ep{};
+  ep.f32 = T;
+  ep.ld_f32 = r;
+  ep.s_bf16 = sT;
+  ep.hi = T_hi;
+  ep.lo = T_lo;
+  ep.ld_pad = rpad;
+  ep.s = s;
+  return run<64, false, false, OUT_LORA>(a1, b1, nullptr, nullptr, static_cast<int>(M), r, 1, ep, num_sms, err,
+                                         stream);
+}
+
+// LoRA up-gradient: U[M, r] = dY[M,N] B[N,r]; writes sU = bf16(s U), U_hi, U_lo [M, rpad].
+cudaError_t launch_gemm_lora_u(const void* dY, const void* Bl, int64_t M, int64_t N, int r, int rpad, float s,
+                               void* sU, void* U_hi, void* U_lo, int num_sms, int32_t* err, cudaStream_t stream) {
+  Operand a1{dY, M, N, N, false}, b1{Bl, r, N, r, true};
+  EpiParams ep{};
+  ep.s_bf16 = sU;
+  ep.hi = U_hi;
+  ep.lo = U_lo;
+  ep.ld_pad = rpad;
+  ep.s = s;
+  return run<64, false, true, OUT_LORA>(a1, b1, nullptr, nullptr, static_cast<int>(M), r, 1, ep, num_sms, err,
+                                        stream);
+}
+
+// Split reduction over tokens: P[split][R][rpad] = sum_m Q[m, R]^T (hi + lo)[m, rpad]
+// with Q bf16 [M, R] (X for dA^T, dY for dB) and hi/lo bf16 [M, rpad].
+cudaError_t launch_gemm_lora_grad(const void* Q, int64_t R, const void* hi, const void* lo, int64_t M, int rpad,
+                                  float* P, int splits, int num_sms, int32_t* err, cudaStream_t stream) {
+  Operand a1{Q, R, M, R, true}, b1{hi, rpad, M, rpad, true};
+  Operand a2{Q, R, M, R, true}, b2{lo, rpad, M, rpad, true};
+  EpiParams ep{};
+  ep.P = P;
+  return run<64, true, true, OUT_PARTIAL>(a1, b1, &a2, &b2, static_cast<int>(R), rpad, splits, ep, num_sms, err,
+                                          stream);
+}
+
+}  // namespace qlora

@@ -1,7 +1,8 @@
-// Host-side launchers of the library's kernels (one per .cu file group).
-// All take device pointers, enqueue on `stream` and return cudaGetLastError().
+// Host-side launchers of the library's kernels. All take device pointers,
+// enqueue on `stream` and return the launch status (cudaGetLastError()).
 #pragma once
 
+#include <cstddef>
 #include <cstdint>
 #include <cuda_runtime.h>
 
@@ -9,6 +10,7 @@ namespace qlora {
 
 constexpr int kQuantBinWords = 257;  // 256 exponent bins + 1 CTA ticket (u64 each)
 
+// ---- quantize.cu / dequant.cu ----
 cudaError_t launch_quantize(const void* W, int64_t numel, uint8_t* packed, int8_t* absmax_q, float* dq_scale,
                             float* mean, float* absmax_scratch, unsigned long long* bins, int num_sms,
                             cudaStream_t stream);
@@ -17,7 +19,7 @@ cudaError_t launch_dequantize(const uint8_t* packed, const int8_t* absmax_q, con
                               const float* mean, void* out, int64_t numel, const float codebook[16],
                               int num_sms, cudaStream_t stream);
 
-// Weight view used by the fused GEMM kernels.
+// Weight view used by the fused decode kernel.
 struct Nf4View {
   const uint8_t* packed;
   const int8_t* absmax_q;
@@ -27,38 +29,34 @@ struct Nf4View {
   int64_t K;  // cols
 };
 
-// ---- LoRA skinny contractions (lora.cu) ----
-// T[M,r] = X[M,K] A[r,K]^T (fp32); optionally sT[M,rpad] = bf16(s*T) with zero padding.
-cudaError_t launch_lora_down(const void* X, const void* A, int64_t M, int64_t K, int r, float s, float* T,
-                             void* sT_bf16, int rpad, int num_sms, cudaStream_t stream);
-// U[M,r] = dY[M,N] B[N,r] (fp32) and sU[M,rpad] = bf16(s*U) (zero padded).
-cudaError_t launch_lora_up_t(const void* dY, const void* B, int64_t M, int64_t N, int r, float s, float* U,
-                             void* sU_bf16, int rpad, int num_sms, cudaStream_t stream);
-// G[R,C] = s * P[M,R]^T Q[M,C], P fp32 (split hi/lo bf16 on the fly), Q bf16, reduced over M.
-// Used for dA (P = U, Q = X) and dB (P = dY as bf16... see lora.cu).
-cudaError_t launch_lora_grad_a(const float* U, const void* X, int64_t M, int64_t K, int r, float s, void* dA,
-                               float* partial, int64_t partial_elems, int num_sms, cudaStream_t stream);
-cudaError_t launch_lora_grad_b(const void* dY, const float* T, int64_t M, int64_t N, int r, float s, void* dB,
-                               float* partial, int64_t partial_elems, int num_sms, cudaStream_t stream);
-size_t lora_grad_partial_elems(int64_t M, int64_t cols, int r, int num_sms);
-cudaError_t launch_zero_bf16(void* p, int64_t n, cudaStream_t stream);
-
-// ---- decode (M <= 16) fused dequant GEMM (decode.cu) ----
-cudaError_t launch_decode_fwd(const Nf4View& w, const void* X, int64_t M, const float* T, const void* B, int r,
-                              float s, void* Y, float* partial, int ksplit, const float codebook[16],
-                              int num_sms, cudaStream_t stream);
+// ---- decode.cu: M <= 16 forward ----
 int decode_ksplit(int64_t N, int64_t K, int num_sms);
 size_t decode_partial_elems(int64_t M, int64_t N, int ksplit);
+size_t decode_counter_words(int64_t N);
+// T [M, r] fp32 receives X A^T; partial [ksplit, M, N] fp32 and counters
+// [decode_counter_words(N)] are scratch.
+cudaError_t launch_decode_fwd(const Nf4View& w, const void* X, int64_t M, const void* A, const void* B, int r,
+                              float s, void* Y, float* T, float* partial, unsigned int* counters, int ksplit,
+                              const float codebook[16], cudaStream_t stream);
 
-// ---- tcgen05 GEMM (gemm_tc.cu) ----
-// C[M, Nc] = A1[M, K1] * op(B1) + A2[M, K2] * op(B2), bf16 in, fp32 accumulate, bf16 out.
-// B1/B2 are K-major ([Nc, K]) when b_mn_major == 0, or MN-major ([K, Nc]) when 1.
-struct TcGemmArgs {
-  const void* A1; const void* B1; int64_t K1;
-  const void* A2; const void* B2; int64_t K2; int64_t lda2; int64_t ldb2;  // slab (may be K2 == 0)
-  void* C; int64_t M; int64_t Nc;
-  int b_mn_major;
-};
-cudaError_t launch_tc_gemm(const TcGemmArgs& a, int num_sms, cudaStream_t stream);
+// ---- gemm_tc.cu: tcgen05 GEMMs ----
+cudaError_t launch_gemm_fwd(const void* X, const void* Wd, const void* sT, const void* Bl, int64_t M, int64_t N,
+                            int64_t K, int r, int rpad, void* Y, int num_sms, int32_t* err, cudaStream_t stream);
+cudaError_t launch_gemm_dx(const void* dY, const void* Wd, const void* sU, const void* Al, int64_t M, int64_t N,
+                           int64_t K, int r, int rpad, void* dX, int num_sms, int32_t* err, cudaStream_t stream);
+cudaError_t launch_gemm_lora_t(const void* X, const void* Al, int64_t M, int64_t K, int r, int rpad, float s,
+                               float* T, void* sT, void* T_hi, void* T_lo, int num_sms, int32_t* err,
+                               cudaStream_t stream);
+cudaError_t launch_gemm_lora_u(const void* dY, const void* Bl, int64_t M, int64_t N, int r, int rpad, float s,
+                               void* sU, void* U_hi, void* U_lo, int num_sms, int32_t* err, cudaStream_t stream);
+cudaError_t launch_gemm_lora_grad(const void* Q, int64_t R, const void* hi, const void* lo, int64_t M, int rpad,
+                                  float* P, int splits, int num_sms, int32_t* err, cudaStream_t stream);
+
+// ---- lora_misc.cu ----
+cudaError_t launch_split_hilo(const float* T, int64_t M, int r, int rpad, void* hi, void* lo, int num_sms,
+                              cudaStream_t stream);
+cudaError_t launch_grad_reduce(const float* P, int splits, int64_t R, int rpad, int r, float s, bool transpose,
+                               void* out, int num_sms, cudaStream_t stream);
+cudaError_t launch_zero_bf16(void* p, int64_t n, int num_sms, cudaStream_t stream);
 
 }  // namespace qlora

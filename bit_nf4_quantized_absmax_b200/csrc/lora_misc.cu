@@ -1,0 +1,84 @@
+// Small element-wise kernels around the LoRA gradient contractions
+// ("QLoRA vs ChatGPT", capability 5: gradients only for the LoRA parameters).
+//
+//   k_split_hilo  T fp32 [M, r] -> T_hi = bf16(T), T_lo = bf16(T - T_hi),
+//                 both [M, rpad] with zero padding, so that a bf16 tensor-core
+//                 contraction with (T_hi + T_lo) keeps ~16 significant bits.
+//   k_grad_reduce out = bf16(s * sum_p P[p]) over the split partials, in a
+//                 fixed order, optionally transposed ([R, rpad] -> [r, R]).
+//   k_zero_bf16   zero fill (gradients of an empty batch).
+#include "common.cuh"
+#include "kernels.h"
+
+namespace qlora {
+namespace {
+
+__global__ void k_split_hilo(const float* __restrict__ T, int64_t M, int r, int rpad, __nv_bfloat16* __restrict__ hi,
+                             __nv_bfloat16* __restrict__ lo) {
+  const int64_t n = M * rpad;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t m = i / rpad;
+    const int j = static_cast<int>(i % rpad);
+    const float v = j < r ? T[m * r + j] : 0.0f;
+    const __nv_bfloat16 h = __float2bfloat16_rn(v);
+    hi[i] = h;
+    lo[i] = __float2bfloat16_rn(v - __bfloat162float(h));
+  }
+}
+
+__global__ void k_grad_reduce(const float* __restrict__ P, int splits, int64_t R, int rpad, int r, float s,
+                              int transpose, __nv_bfloat16* __restrict__ out) {
+  const int64_t n = R * r;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    int64_t row, j;
+    if (transpose) {  // out [r, R]: consecutive threads walk R
+      j = i / R;
+      row = i % R;
+    } else {          // out [R, r]
+      row = i / r;
+      j = i % r;
+    }
+    float acc = 0.0f;
+    for (int p = 0; p < splits; ++p) acc += P[(static_cast<int64_t>(p) * R + row) * rpad + j];
+    out[i] = __float2bfloat16_rn(s * acc);
+  }
+}
+
+__global__ void k_zero_bf16(__nv_bfloat16* __restrict__ p, int64_t n) {
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x)
+    p[i] = __float2bfloat16_rn(0.0f);
+}
+
+int grid_for(int64_t n, int num_sms) {
+  int64_t g = (n + 255) / 256;
+  const int64_t cap = static_cast<int64_t>(num_sms) * 8;
+  if (g > cap) g = cap;
+  return static_cast<int>(g < 1 ? 1 : g);
+}
+
+}  // namespace
+
+cudaError_t launch_split_hilo(const float* T, int64_t M, int r, int rpad, void* hi, void* lo, int num_sms,
+                              cudaStream_t stream) {
+  k_split_hilo<<<grid_for(M * rpad, num_sms), 256, 0, stream>>>(T, M, r, rpad, static_cast<__nv_bfloat16*>(hi),
+                                                                  static_cast<__nv_bfloat16*>(lo));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_grad_reduce(const float* P, int splits, int64_t R, int rpad, int r, float s, bool transpose,
+                               void* out, int num_sms, cudaStream_t stream) {
+  k_grad_reduce<<<grid_for(R * r, num_sms), 256, 0, stream>>>(P, splits, R, rpad, r, s, transpose ? 1 : 0,
+                                                               static_cast<__nv_bfloat16*>(out));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_zero_bf16(void* p, int64_t n, int num_sms, cudaStream_t stream) {
+  if (n <= 0) return cudaSuccess;
+  k_zero_bf16<<<grid_for(n, num_sms), 256, 0, stream>>>(static_cast<__nv_bfloat16*>(p), n);
+  return cudaGetLastError();
+}
+
+}  // namespace qlora
