@@ -21,7 +21,8 @@ STATUS_NAMES = {0: "QLORA_OK", 1: "QLORA_ERR_INVALID_ARG", 2: "QLORA_ERR_UNSUPPO
                 4: "QLORA_ERR_CUDA", 5: "QLORA_ERR_WORKSPACE", 6: "QLORA_ERR_DEVICE"}
 
 EXPORTED = ("qlora_status_string", "qlora_nf4_codebook", "qlora_nf4_storage_bytes", "qlora_quantize_nf4_dq",
-            "qlora_dequantize_nf4_dq", "qlora_linear_fwd", "qlora_linear_bwd", "qlora_device_error")
+            "qlora_quantize_nf4_dq_noalloc", "qlora_dequantize_nf4_dq", "qlora_linear_fwd", "qlora_linear_bwd",
+            "qlora_device_error")
 
 
 class QloraError(RuntimeError):
@@ -56,6 +57,7 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
     lib.qlora_nf4_codebook.argtypes = [ctypes.POINTER(ctypes.c_float)]
     lib.qlora_nf4_storage_bytes.argtypes = [i64, i64, ctypes.POINTER(sz)]
     lib.qlora_quantize_nf4_dq.argtypes = [vp, wp, vp, szp, vp]
+    lib.qlora_quantize_nf4_dq_noalloc.argtypes = [vp, wp, vp]
     lib.qlora_dequantize_nf4_dq.argtypes = [wp, vp, vp]
     lib.qlora_linear_fwd.argtypes = [wp, vp, i64, vp, vp, i32, f32, vp, vp, vp, szp, vp]
     lib.qlora_linear_bwd.argtypes = [wp, vp, i64, vp, vp, i32, f32, vp, vp, vp, vp, vp, vp, szp, vp]
@@ -140,6 +142,16 @@ def qlora_quantize_nf4_dq(W: torch.Tensor, out: NF4Weight | None = None, workspa
     _check(lib.qlora_quantize_nf4_dq(_ptr(W), ctypes.byref(qc), _ptr(ws), ctypes.byref(nbytes), st),
            "qlora_quantize_nf4_dq")
     return q
+
+
+def qlora_quantize_nf4_dq_noalloc(W: torch.Tensor, out: NF4Weight, stream=None) -> NF4Weight:
+    """Quantize into `out` without any device allocation by the library (its
+    scratch is a fixed array inside the library; see include/qlora.h)."""
+    assert W.dtype == torch.bfloat16 and W.dim() == 2 and W.is_contiguous()
+    qc = out.as_c()
+    _check(load_library().qlora_quantize_nf4_dq_noalloc(_ptr(W), ctypes.byref(qc), _stream(stream)),
+           "qlora_quantize_nf4_dq_noalloc")
+    return out
 
 
 def qlora_dequantize_nf4_dq(q: NF4Weight, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:

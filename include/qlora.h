@@ -77,8 +77,8 @@ typedef enum {
  *
  * A block's decoded constant is m' = fmaf((float)absmax_q[b], dq_scale[b/256],
  * mean) and its weights decode to bf16_rn(codebook[code] * m')  ([C] 1, 3, 5).
- * All pointers are device memory owned by the caller; packed must be 16-byte
- * aligned, the others 4-byte aligned.
+ * All pointers are device memory owned by the caller; packed and absmax_q must
+ * be 16-byte aligned, dq_scale and mean 4-byte aligned.
  */
 typedef struct {
   uint8_t* packed;
@@ -136,6 +136,25 @@ qlora_status qlora_nf4_storage_bytes(int64_t rows, int64_t cols, size_t out[4]);
 qlora_status qlora_quantize_nf4_dq(const void* W_bf16, const qlora_nf4_weight* q,
                                    void* workspace, size_t* workspace_bytes,
                                    qlora_stream_t stream);
+
+/* qlora_quantize_nf4_dq_noalloc -- the same quantization as qlora_quantize_nf4_dq
+ * (identical outputs), for callers that cannot allocate device memory or supply
+ * a workspace: serving runtimes whose device memory is fully planned at start-up
+ * and forbid allocation afterwards, or hosts where cudaMalloc's implicit device
+ * synchronization is not acceptable. The paper has no counterpart; this is a
+ * convenience of this library.
+ *
+ * The call allocates nothing. Its scratch (about 16 MiB) is a fixed array in the
+ * library's device memory that every GPU loading the library keeps until the
+ * process exits; the weight may have at most 2^22 blocks of 64 (268,435,456
+ * weights), larger weights return QLORA_ERR_UNSUPPORTED before any launch. The
+ * first call on a device looks up that array's device address (one
+ * cudaGetSymbolAddress with the device current); make that first call before
+ * any stream capture. All calls share the array, so calls that overlap on the
+ * GPU race: order them on one stream. Other arguments, alignment rules and
+ * errors are those of qlora_quantize_nf4_dq. */
+qlora_status qlora_quantize_nf4_dq_noalloc(const void* W_bf16, const qlora_nf4_weight* q,
+                                           qlora_stream_t stream);
 
 /* qlora_dequantize_nf4_dq -- decode q to a bf16 matrix out_bf16 [rows, cols]
  * (device, 16-byte aligned): w' = bf16_rn(fp32(codebook[code] * m'_b)) with
