@@ -39,7 +39,7 @@ R, ALPHA, M_TRAIN, M_DECODE = 64, 16.0, 4096, (1, 4, 16)
 SHAPES = syn.LLAMA7B_SHAPES
 
 # kernels each C-ABI call launches on these shapes (see the launchers in csrc/)
-LAUNCHES = {"quantize": 3, "dequantize": 1, "decode_fwd": 2, "train_fwd": 3, "train_bwd": 8}
+LAUNCHES = {"quantize": 3, "dequantize": 1, "decode_fwd": 2, "train_fwd": 4, "train_bwd": 9}
 
 
 def train_flops(N, K, M=M_TRAIN, r=R):
@@ -432,6 +432,26 @@ def run_reference(args, rank, world):
 
 
 # ----------------------------------------------------------------------------
+# small profiling case (for ncu captures): one call of each entry point on the
+# 11008x4096 linear, training M = 4096 and decode M = 1
+
+def profile_case():
+    dev = torch.device("cuda", 0)
+    N, K = 11008, 4096
+    inp = syn.make_linear(N, K, M_TRAIN, r=R, alpha=ALPHA, seed=0, workload="llama7b_train", layer=1)
+    W, A, B, X, dY = (t.to(dev) for t in (inp.W, inp.A, inp.B, inp.X, inp.dY))
+    q = qb.qlora_quantize_nf4_dq(W)                                   # quantize + DQ
+    qb.qlora_dequantize_nf4_dq(q)                                     # dequant
+    qb.qlora_linear_fwd(q, X[:1].contiguous(), A, B, ALPHA)           # decode M = 1
+    qb.qlora_linear_fwd(q, X[:16].contiguous(), A, B, ALPHA)          # decode M = 16
+    _, T = qb.qlora_linear_fwd(q, X, A, B, ALPHA, T_save=True)        # training forward
+    qb.qlora_linear_bwd(q, X, A, B, ALPHA, dY, T_saved=T)             # training backward
+    torch.cuda.synchronize()
+    assert qb.qlora_device_error() == 0
+    print("profile case ok")
+
+
+# ----------------------------------------------------------------------------
 # distributed plumbing
 
 def gpu_index_for_smi(dev):
@@ -464,7 +484,13 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile-case", action="store_true",
+                    help="run one call of each entry point on 11008x4096 (for ncu) and exit")
     args = ap.parse_args()
+    if args.profile_case:
+        qb.load_library()
+        profile_case()
+        return
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     world = int(os.environ.get("WORLD_SIZE", "1"))

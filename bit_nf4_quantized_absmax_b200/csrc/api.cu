@@ -90,7 +90,19 @@ int32_t* device_error_word() {
 // Split count for the token reductions of dA / dB: enough units to cover the SMs.
 int grad_splits(int64_t R, int rpad, int64_t M, int num_sms) {
   const int64_t tiles = ((R + 127) / 128) * (rpad / 64);
+  if (tiles <= 0) return 1;
   const int64_t nkb = 2 * ((M + 63) / 64);
+  int64_t sp = (num_sms + tiles - 1) / tiles;
+  if (sp > nkb) sp = nkb;
+  if (sp < 1) sp = 1;
+  return static_cast<int>(sp);
+}
+
+// Split count for the K (or N) reduction of the rank-r products X A^T and dY B.
+int red_splits(int64_t M, int rpad, int64_t Kred, int num_sms) {
+  const int64_t tiles = ((M + 127) / 128) * (rpad / 64);
+  if (tiles <= 0) return 1;
+  const int64_t nkb = (Kred + 63) / 64;
   int64_t sp = (num_sms + tiles - 1) / tiles;
   if (sp > nkb) sp = nkb;
   if (sp < 1) sp = 1;
@@ -204,6 +216,7 @@ qlora_status qlora_linear_fwd(const qlora_nf4_weight* q, const void* X, int64_t 
   } else {
     off_wd = L.add(static_cast<size_t>(N) * K * 2);
     off_sT = L.add(static_cast<size_t>(M) * rpad * 2);
+    off_part = L.add(static_cast<size_t>(red_splits(M, rpad, K, di.num_sms)) * M * rpad * sizeof(float));
   }
   bool launch = false;
   st = workspace_check(workspace, workspace_bytes, L.total(), &launch);
@@ -221,9 +234,12 @@ qlora_status qlora_linear_fwd(const qlora_nf4_weight* q, const void* X, int64_t 
   }
   void* Wd = ws + off_wd;
   void* sT = ws + off_sT;
+  float* P = reinterpret_cast<float*>(ws + off_part);
+  const int splits_t = red_splits(M, rpad, K, kRefSms);
   cudaError_t e = launch_dequantize(q->packed, q->absmax_q, q->dq_scale, q->mean, Wd, N * K, cb, di.num_sms, cs);
+  if (e == cudaSuccess) e = launch_gemm_lora_t(X, A, M, K, r, rpad, P, splits_t, di.num_sms, err, cs);
   if (e == cudaSuccess)
-    e = launch_gemm_lora_t(X, A, M, K, r, rpad, s, T_save, sT, nullptr, nullptr, di.num_sms, err, cs);
+    e = launch_lora_finish(P, splits_t, M, r, rpad, s, T_save, sT, nullptr, nullptr, di.num_sms, cs);
   if (e == cudaSuccess) e = launch_gemm_fwd(X, Wd, sT, B, M, N, K, r, rpad, Y, di.num_sms, err, cs);
   return cuda_status(e);
 }
@@ -250,8 +266,16 @@ qlora_status qlora_linear_bwd(const qlora_nf4_weight* q, const void* X, int64_t 
   const size_t off_wd = L.add(dX ? static_cast<size_t>(N) * K * 2 : 0);
   const size_t off_thi = L.add(mp), off_tlo = L.add(mp);
   const size_t off_su = L.add(mp), off_uhi = L.add(mp), off_ulo = L.add(mp);
-  const size_t pa = static_cast<size_t>(splits_a) * K * rpad, pb = static_cast<size_t>(splits_b) * N * rpad;
-  const size_t off_p = L.add((pa > pb ? pa : pb) * sizeof(float));
+  const int splits_t = red_splits(M, rpad, K, di.num_sms);
+  const int splits_u = red_splits(M, rpad, N, di.num_sms);
+  size_t pmax = static_cast<size_t>(splits_a) * K * rpad;
+  const size_t pb = static_cast<size_t>(splits_b) * N * rpad;
+  const size_t pt = static_cast<size_t>(T_saved ? 0 : splits_t) * M * rpad;
+  const size_t pu = static_cast<size_t>(splits_u) * M * rpad;
+  if (pb > pmax) pmax = pb;
+  if (pt > pmax) pmax = pt;
+  if (pu > pmax) pmax = pu;
+  const size_t off_p = L.add(pmax * sizeof(float));
   bool launch = false;
   st = workspace_check(workspace, workspace_bytes, L.total(), &launch);
   if (st != QLORA_OK || !launch) return st;
@@ -269,10 +293,16 @@ qlora_status qlora_linear_bwd(const qlora_nf4_weight* q, const void* X, int64_t 
   float* P = reinterpret_cast<float*>(ws + off_p);
   cudaError_t e = cudaSuccess;
   // T = X A^T as a two-term bf16 split (from the saved fp32 T or recomputed)
-  if (T_saved) e = launch_split_hilo(T_saved, M, r, rpad, Thi, Tlo, di.num_sms, cs);
-  else e = launch_gemm_lora_t(X, A, M, K, r, rpad, s, nullptr, nullptr, Thi, Tlo, di.num_sms, err, cs);
+  if (T_saved) {
+    e = launch_split_hilo(T_saved, M, r, rpad, Thi, Tlo, di.num_sms, cs);
+  } else {
+    e = launch_gemm_lora_t(X, A, M, K, r, rpad, P, splits_t, di.num_sms, err, cs);
+    if (e == cudaSuccess)
+      e = launch_lora_finish(P, splits_t, M, r, rpad, s, nullptr, nullptr, Thi, Tlo, di.num_sms, cs);
+  }
   // U = dY B: s U for the dX slab, U as hi + lo for dA
-  if (e == cudaSuccess) e = launch_gemm_lora_u(dY, B, M, N, r, rpad, s, sU, Uhi, Ulo, di.num_sms, err, cs);
+  if (e == cudaSuccess) e = launch_gemm_lora_u(dY, B, M, N, r, rpad, P, splits_u, di.num_sms, err, cs);
+  if (e == cudaSuccess) e = launch_lora_finish(P, splits_u, M, r, rpad, s, nullptr, sU, Uhi, Ulo, di.num_sms, cs);
   if (dX) {
     void* Wd = ws + off_wd;
     if (e == cudaSuccess)

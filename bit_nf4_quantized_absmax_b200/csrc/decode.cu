@@ -22,7 +22,7 @@
 namespace qlora {
 namespace {
 
-constexpr int kDecodeWarps = 4;
+constexpr int kDecodeWarps = 8;
 
 __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                          uint32_t b0, uint32_t b1) {
@@ -35,7 +35,8 @@ __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1
 
 struct RowBlock {
   uint4 n0, n1;   // 64 codes
-  float mp;       // decoded block constant
+  int qv;         // int8 block constant code
+  float sc;       // its group scale (the decoded constant is formed when the block is used)
 };
 
 __device__ __forceinline__ RowBlock load_row_block(const uint8_t* __restrict__ packed, const int8_t* __restrict__ q,
@@ -47,11 +48,13 @@ __device__ __forceinline__ RowBlock load_row_block(const uint8_t* __restrict__ p
     const uint4* p = reinterpret_cast<const uint4*>(packed + blk * 32);
     rb.n0 = __ldcs(p);
     rb.n1 = __ldcs(p + 1);
-    rb.mp = __fmaf_rn(static_cast<float>(q[blk]), dqs[blk >> 8], mu);
+    rb.qv = static_cast<int>(__ldg(q + blk));
+    rb.sc = __ldg(dqs + (blk >> 8));
   } else {
     rb.n0 = make_uint4(0x77777777u, 0x77777777u, 0x77777777u, 0x77777777u);
     rb.n1 = rb.n0;
-    rb.mp = 0.0f;
+    rb.qv = 0;
+    rb.sc = 0.0f;
   }
   return rb;
 }
@@ -70,7 +73,7 @@ __device__ __forceinline__ uint32_t nib_word(const RowBlock& rb, int w) {
 }
 
 template <int MT>
-__global__ void __launch_bounds__(kDecodeWarps * 32)
+__global__ void __launch_bounds__(kDecodeWarps * 32, 2)
 k_decode(const uint8_t* __restrict__ packed, const int8_t* __restrict__ q, const float* __restrict__ dqs,
          const float* __restrict__ mean, const __nv_bfloat16* __restrict__ X, int M, int64_t N, int64_t K,
          const float* __restrict__ T, const __nv_bfloat16* __restrict__ Bl, int r, float s,
@@ -90,29 +93,54 @@ k_decode(const uint8_t* __restrict__ packed, const int8_t* __restrict__ q, const
   const float mu = *mean;
   const int64_t na = n0 + g, nb = n0 + g + 8;
 
-  float acc[MT][4];
+  // two independent accumulator chains (even and odd MMA steps)
+  float acc[2][MT][4];
 #pragma unroll
-  for (int j = 0; j < MT; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.0f;
+  for (int c = 0; c < 2; ++c)
+#pragma unroll
+    for (int j = 0; j < MT; ++j) acc[c][j][0] = acc[c][j][1] = acc[c][j][2] = acc[c][j][3] = 0.0f;
 
-  for (int64_t sb = sb_begin + warp; sb < sb_end; sb += kDecodeWarps) {
+  int64_t sb = sb_begin + warp;
+  RowBlock na_next, nb_next;  // codes and block constants of the warp's next superblock
+  if (sb < sb_end) {
     const int64_t kb = sb * 4 + t;
     const bool kv = kb < nkb_row;
-    const RowBlock ra = load_row_block(packed, q, dqs, mu, na, nkb_row, kb, kv && na < N);
-    const RowBlock rbk = load_row_block(packed, q, dqs, mu, nb, nkb_row, kb, kv && nb < N);
-    // token values for this lane's 64 k positions: tokens g (tile 0) and g + 8 (tile 1)
-    uint4 xv[MT][8];
+    na_next = load_row_block(packed, q, dqs, mu, na, nkb_row, kb, kv && na < N);
+    nb_next = load_row_block(packed, q, dqs, mu, nb, nkb_row, kb, kv && nb < N);
+  }
+  for (; sb < sb_end; sb += kDecodeWarps) {
+    const int64_t kb = sb * 4 + t;
+    const bool kv = kb < nkb_row;
+    const RowBlock ra = na_next, rbk = nb_next;
+    // token values for this lane's 64 k positions: tokens g (tile 0) and g + 8 (tile 1),
+    // fetched 16 at a time (L1-resident; X is small)
+    const uint4* xp[MT];
+    bool xok[MT];
 #pragma unroll
     for (int j = 0; j < MT; ++j) {
       const int tok = g + 8 * j;
-      const bool ok = kv && tok < M;
-      const uint4* xp = reinterpret_cast<const uint4*>(X + static_cast<int64_t>(tok) * K + kb * 64);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) xv[j][i] = ok ? __ldg(xp + i) : make_uint4(0, 0, 0, 0);
+      xok[j] = kv && tok < M;
+      xp[j] = reinterpret_cast<const uint4*>(X + static_cast<int64_t>(tok) * K + kb * 64);
     }
-    const Nf4Lut la = make_nf4_lut(cb, ra.mp);
-    const Nf4Lut lb = make_nf4_lut(cb, rbk.mp);
+    const int64_t sbn = sb + kDecodeWarps;  // prefetch while this superblock is decoded
+    if (sbn < sb_end) {
+      const int64_t kbn = sbn * 4 + t;
+      const bool kvn = kbn < nkb_row;
+      na_next = load_row_block(packed, q, dqs, mu, na, nkb_row, kbn, kvn && na < N);
+      nb_next = load_row_block(packed, q, dqs, mu, nb, nkb_row, kbn, kvn && nb < N);
+    }
+    const Nf4Lut la = make_nf4_lut(cb, __fmaf_rn(static_cast<float>(ra.qv), ra.sc, mu));
+    const Nf4Lut lb = make_nf4_lut(cb, __fmaf_rn(static_cast<float>(rbk.qv), rbk.sc, mu));
+    uint4 xv[MT][2];
 #pragma unroll
     for (int st = 0; st < 16; ++st) {
+      if ((st & 3) == 0) {
+#pragma unroll
+        for (int j = 0; j < MT; ++j) {
+          xv[j][0] = xok[j] ? __ldg(xp[j] + (st >> 1)) : make_uint4(0, 0, 0, 0);
+          xv[j][1] = xok[j] ? __ldg(xp[j] + (st >> 1) + 1) : make_uint4(0, 0, 0, 0);
+        }
+      }
       const uint32_t wa = nib_word(ra, st >> 1) >> (16 * (st & 1));
       const uint32_t wb = nib_word(rbk, st >> 1) >> (16 * (st & 1));
       uint32_t a0, a1, a2, a3;
@@ -120,10 +148,10 @@ k_decode(const uint8_t* __restrict__ packed, const int8_t* __restrict__ q, const
       nf4_lookup4(lb, wb, a1, a3);   // row g + 8
 #pragma unroll
       for (int j = 0; j < MT; ++j) {
-        const uint4 x4 = xv[j][st >> 1];
+        const uint4 x4 = xv[j][(st >> 1) & 1];
         const uint32_t b0 = (st & 1) ? x4.z : x4.x;
         const uint32_t b1 = (st & 1) ? x4.w : x4.y;
-        mma16816(acc[j], a0, a1, a2, a3, b0, b1);
+        mma16816(acc[st & 1][j], a0, a1, a2, a3, b0, b1);
       }
     }
   }
@@ -131,10 +159,10 @@ k_decode(const uint8_t* __restrict__ packed, const int8_t* __restrict__ q, const
   // acc[j]: (row g, token 8j + 2t), (g, 8j + 2t + 1), (g + 8, 8j + 2t), (g + 8, 8j + 2t + 1)
 #pragma unroll
   for (int j = 0; j < MT; ++j) {
-    red[warp][g][8 * j + 2 * t] = acc[j][0];
-    red[warp][g][8 * j + 2 * t + 1] = acc[j][1];
-    red[warp][g + 8][8 * j + 2 * t] = acc[j][2];
-    red[warp][g + 8][8 * j + 2 * t + 1] = acc[j][3];
+    red[warp][g][8 * j + 2 * t] = acc[0][j][0] + acc[1][j][0];
+    red[warp][g][8 * j + 2 * t + 1] = acc[0][j][1] + acc[1][j][1];
+    red[warp][g + 8][8 * j + 2 * t] = acc[0][j][2] + acc[1][j][2];
+    red[warp][g + 8][8 * j + 2 * t + 1] = acc[0][j][3] + acc[1][j][3];
   }
   __syncthreads();
 
@@ -189,32 +217,44 @@ k_decode(const uint8_t* __restrict__ packed, const int8_t* __restrict__ q, const
 }
 
 // T[m, j] = sum_k X[m, k] A[j, k] for M <= 16 (fp32 on CUDA cores), one CTA per
-// adapter row j. Block 0 also clears the decode kernel's ticket counters.
+// adapter row j, 16-byte loads (8 k per thread and step). Block 0 also clears
+// the decode kernel's ticket counters.
+template <int MT>
 __global__ void __launch_bounds__(256)
 k_lora_t_small(const __nv_bfloat16* __restrict__ X, const __nv_bfloat16* __restrict__ A, int M, int64_t K, int r,
                float* __restrict__ T, unsigned int* __restrict__ counters, int n_counters) {
-  __shared__ float red[8][16];
+  __shared__ float red[8][8 * MT];
   const int j = blockIdx.x;
   if (j == 0)
     for (int i = threadIdx.x; i < n_counters; i += blockDim.x) counters[i] = 0u;
-  float acc[16];
+  float acc[8 * MT];
 #pragma unroll
-  for (int m = 0; m < 16; ++m) acc[m] = 0.0f;
-  const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(A + static_cast<int64_t>(j) * K);
-  for (int64_t k2 = threadIdx.x; k2 < K / 2; k2 += blockDim.x) {
-    const float2 av = __bfloat1622float2(a2[k2]);
+  for (int m = 0; m < 8 * MT; ++m) acc[m] = 0.0f;
+  const uint4* a4 = reinterpret_cast<const uint4*>(A + static_cast<int64_t>(j) * K);
+  for (int64_t k8 = threadIdx.x; k8 < K / 8; k8 += blockDim.x) {
+    const uint4 av = __ldg(a4 + k8);
+    const float a[8] = {bf16lo_to_f32(av.x), bf16hi_to_f32(av.x), bf16lo_to_f32(av.y), bf16hi_to_f32(av.y),
+                        bf16lo_to_f32(av.z), bf16hi_to_f32(av.z), bf16lo_to_f32(av.w), bf16hi_to_f32(av.w)};
 #pragma unroll
-    for (int m = 0; m < 16; ++m) {
+    for (int m = 0; m < 8 * MT; ++m) {
       if (m < M) {
-        const float2 xv =
-            __bfloat1622float2(reinterpret_cast<const __nv_bfloat162*>(X + static_cast<int64_t>(m) * K)[k2]);
-        acc[m] = fmaf(av.x, xv.x, fmaf(av.y, xv.y, acc[m]));
+        const uint4 xv = __ldg(reinterpret_cast<const uint4*>(X + static_cast<int64_t>(m) * K) + k8);
+        float s = acc[m];
+        s = fmaf(a[0], bf16lo_to_f32(xv.x), s);
+        s = fmaf(a[1], bf16hi_to_f32(xv.x), s);
+        s = fmaf(a[2], bf16lo_to_f32(xv.y), s);
+        s = fmaf(a[3], bf16hi_to_f32(xv.y), s);
+        s = fmaf(a[4], bf16lo_to_f32(xv.z), s);
+        s = fmaf(a[5], bf16hi_to_f32(xv.z), s);
+        s = fmaf(a[6], bf16lo_to_f32(xv.w), s);
+        s = fmaf(a[7], bf16hi_to_f32(xv.w), s);
+        acc[m] = s;
       }
     }
   }
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 #pragma unroll
-  for (int m = 0; m < 16; ++m) {
+  for (int m = 0; m < 8 * MT; ++m) {
     float v = acc[m];
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
@@ -234,8 +274,8 @@ k_lora_t_small(const __nv_bfloat16* __restrict__ X, const __nv_bfloat16* __restr
 int decode_ksplit(int64_t N, int64_t K, int num_sms) {
   const int64_t row_tiles = (N + 15) / 16;
   const int64_t nsb = (K / 64 + 3) / 4;
-  int64_t want = (4 * static_cast<int64_t>(num_sms) + row_tiles - 1) / row_tiles;
-  int64_t cap = nsb / 2 > 0 ? nsb / 2 : 1;
+  int64_t want = (3 * static_cast<int64_t>(num_sms) + row_tiles - 1) / row_tiles;
+  int64_t cap = nsb / kDecodeWarps > 0 ? nsb / kDecodeWarps : 1;  // at least one superblock per warp
   if (want > cap) want = cap;
   if (want < 1) want = 1;
   return static_cast<int>(want);
@@ -253,9 +293,14 @@ cudaError_t launch_decode_fwd(const Nf4View& w, const void* X, int64_t M, const 
   Nf4Codebook cb;
   for (int i = 0; i < 16; ++i) cb.c[i] = codebook[i];
   const int64_t row_tiles = (w.N + 15) / 16;
-  k_lora_t_small<<<r, 256, 0, stream>>>(reinterpret_cast<const __nv_bfloat16*>(X),
-                                        reinterpret_cast<const __nv_bfloat16*>(A), static_cast<int>(M), w.K, r, T,
-                                        counters, static_cast<int>(row_tiles));
+  if (M <= 8)
+    k_lora_t_small<1><<<r, 256, 0, stream>>>(reinterpret_cast<const __nv_bfloat16*>(X),
+                                             reinterpret_cast<const __nv_bfloat16*>(A), static_cast<int>(M), w.K, r,
+                                             T, counters, static_cast<int>(row_tiles));
+  else
+    k_lora_t_small<2><<<r, 256, 0, stream>>>(reinterpret_cast<const __nv_bfloat16*>(X),
+                                             reinterpret_cast<const __nv_bfloat16*>(A), static_cast<int>(M), w.K, r,
+                                             T, counters, static_cast<int>(row_tiles));
   dim3 grid(static_cast<unsigned>(row_tiles), static_cast<unsigned>(ksplit));
   if (M <= 8) {
     k_decode<1><<<grid, kDecodeWarps * 32, 0, stream>>>(

@@ -11,27 +11,51 @@
 namespace qlora {
 namespace {
 
+constexpr int kDeqUnroll = 4;
+
+__device__ __forceinline__ void dequant_unit(const uint4 nib, int64_t u, float mp, uint4* __restrict__ out,
+                                             const Nf4Codebook& cb) {
+  const Nf4Lut t = make_nf4_lut(cb, mp);
+  uint32_t o[16];
+  nf4_lookup8(t, nib.x, o + 0);
+  nf4_lookup8(t, nib.y, o + 4);
+  nf4_lookup8(t, nib.z, o + 8);
+  nf4_lookup8(t, nib.w, o + 12);
+  uint4* dst = out + u * 4;
+  __stcs(dst + 0, make_uint4(o[0], o[1], o[2], o[3]));
+  __stcs(dst + 1, make_uint4(o[4], o[5], o[6], o[7]));
+  __stcs(dst + 2, make_uint4(o[8], o[9], o[10], o[11]));
+  __stcs(dst + 3, make_uint4(o[12], o[13], o[14], o[15]));
+}
+
+// Grid-stride over 32-weight units; each thread keeps kDeqUnroll 16-byte
+// loads in flight before decoding them.
 __global__ void __launch_bounds__(256)
 k_dequant(const uint4* __restrict__ packed, const int8_t* __restrict__ absmax_q,
           const float* __restrict__ dq_scale, const float* __restrict__ mean, uint4* __restrict__ out,
           int64_t n_units, const __grid_constant__ Nf4Codebook cb) {
   const float mu = *mean;
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  for (int64_t u = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; u < n_units; u += stride) {
-    const int64_t b = u >> 1;
-    const uint4 nib = __ldcs(packed + u);
-    const float mp = __fmaf_rn(static_cast<float>(absmax_q[b]), dq_scale[b >> 8], mu);
-    const Nf4Lut t = make_nf4_lut(cb, mp);
-    uint32_t o[16];
-    nf4_lookup8(t, nib.x, o + 0);
-    nf4_lookup8(t, nib.y, o + 4);
-    nf4_lookup8(t, nib.z, o + 8);
-    nf4_lookup8(t, nib.w, o + 12);
-    uint4* dst = out + u * 4;
-    __stcs(dst + 0, make_uint4(o[0], o[1], o[2], o[3]));
-    __stcs(dst + 1, make_uint4(o[4], o[5], o[6], o[7]));
-    __stcs(dst + 2, make_uint4(o[8], o[9], o[10], o[11]));
-    __stcs(dst + 3, make_uint4(o[12], o[13], o[14], o[15]));
+  for (int64_t u0 = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; u0 < n_units;
+       u0 += stride * kDeqUnroll) {
+    // issue every load of the iteration (codes and block constants) before any use
+    uint4 nib[kDeqUnroll];
+    int qv[kDeqUnroll];
+    float sc[kDeqUnroll];
+#pragma unroll
+    for (int i = 0; i < kDeqUnroll; ++i) {
+      const int64_t u = u0 + i * stride;
+      const bool ok = u < n_units;
+      nib[i] = ok ? __ldcs(packed + u) : make_uint4(0, 0, 0, 0);
+      qv[i] = ok ? static_cast<int>(__ldg(absmax_q + (u >> 1))) : 0;
+      sc[i] = ok ? __ldg(dq_scale + (u >> 9)) : 0.0f;
+    }
+#pragma unroll
+    for (int i = 0; i < kDeqUnroll; ++i) {
+      const int64_t u = u0 + i * stride;
+      if (u < n_units)
+        dequant_unit(nib[i], u, __fmaf_rn(static_cast<float>(qv[i]), sc[i], mu), out, cb);
+    }
   }
 }
 
@@ -43,7 +67,7 @@ cudaError_t launch_dequantize(const uint8_t* packed, const int8_t* absmax_q, con
   Nf4Codebook cb;
   for (int i = 0; i < 16; ++i) cb.c[i] = codebook[i];
   const int64_t n_units = numel / 32;
-  int64_t want = (n_units + 255) / 256;
+  int64_t want = (n_units + 256 * kDeqUnroll - 1) / (256 * kDeqUnroll);
   int64_t cap = static_cast<int64_t>(num_sms) * 8;
   const int grid = static_cast<int>(want < cap ? (want > 0 ? want : 1) : cap);
   k_dequant<<<grid, 256, 0, stream>>>(reinterpret_cast<const uint4*>(packed), absmax_q, dq_scale, mean,

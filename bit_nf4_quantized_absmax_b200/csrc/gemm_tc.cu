@@ -18,6 +18,8 @@
 // CTA leave its loops.
 #include <cuda.h>
 
+#include <cstdlib>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -365,6 +367,267 @@ k_tc_gemm(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUte
 }
 
 // ---------------------------------------------------------------------------
+// 2-CTA variant for the large GEMMs: a cluster of two CTAs computes a 256x256
+// tile with tcgen05.mma.cta_group::2 (M = 256 split 128/128 across the pair's
+// tensor memories, B split 128/128 across their shared memories), so each SM
+// streams 32 KB of operands per 64-deep k-block instead of 48 KB.
+//   - Both CTAs load their halves with TMA; the loads complete on the even
+//     (leader) CTA's full barrier, which the leader's producer arms with the
+//     bytes of both halves.
+//   - The leader's MMA thread issues the MMAs and commits with multicast to the
+//     empty and accumulator-full barriers of both CTAs.
+//   - Each CTA drains its own accumulator rows; both epilogues arrive on the
+//     leader's accumulator-empty barrier (the odd CTA remotely).
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+__device__ __forceinline__ uint32_t map_to_cta(uint32_t saddr, uint32_t rank) {
+  uint32_t d;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(d) : "r"(saddr), "r"(rank));
+  return d;
+}
+
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tma_load_2d_pair(void* smem_dst, const void* tmap, uint32_t bar_cluster_addr,
+                                                 int32_t x, int32_t y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, "
+      "%4}], [%2];" ::"r"(smem_u32(smem_dst)),
+      "l"(tmap), "r"(bar_cluster_addr), "r"(x), "r"(y)
+      : "memory");
+}
+
+__device__ __forceinline__ void mma_bf16_pair(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(idesc), "r"(acc));
+}
+
+__device__ __forceinline__ void mma_commit_pair(uint64_t* bar) {
+  const uint16_t mask = 0x3;
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+          smem_u32(bar)),
+      "h"(mask)
+      : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster_addr) : "memory");
+}
+
+template <bool B_MN>
+struct Cfg2 {
+  static constexpr int A_BYTES = 128 * BK * 2;   // this CTA's half of A
+  static constexpr int B_BYTES = 128 * BK * 2;   // this CTA's half of B
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int STAGES = 6;
+  static constexpr int TMEM_COLS = 512;          // two 256-column accumulators
+  static constexpr int SMEM = STAGES * STAGE_BYTES + 1024 + 256;
+};
+
+template <bool B_MN>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+k_tc_gemm2(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmB1,
+           const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2, TileSched ts, int M,
+           int Nc, EpiParams ep, int32_t* err) {
+  using C = Cfg2<B_MN>;
+  constexpr int BN2 = 256;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
+  uint64_t* empty = full + C::STAGES;
+  uint64_t* accf = empty + C::STAGES;
+  uint64_t* acce = accf + 2;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(acce + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const int pair = blockIdx.x >> 1;
+  const int npairs = gridDim.x >> 1;
+  const int n_units = ts.tiles_m * ts.tiles_n * ts.splits;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&accf[a], 1);
+      mbar_init(&acce[a], 256);
+    }
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmA1);
+    prefetch_tmap(&tmB1);
+    prefetch_tmap(&tmA2);
+    prefetch_tmap(&tmB2);
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_holder)),
+                 "r"(C::TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();  // the peer's barriers are initialised before any remote use
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  if (warp == 0) {
+    // ---------------- TMA producer (both CTAs) ----------------
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int unit = pair; unit < n_units && ok; unit += npairs) {
+        int tm, tn, kb0, kb1;
+        decode_unit(ts, unit, tm, tn, kb0, kb1);
+        const int m0 = tm * 256 + static_cast<int>(rank) * 128;
+        const int n0 = tn * BN2 + static_cast<int>(rank) * 128;
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!wait_or_abort(&empty[stage], phase ^ 1u, abort_flag, err, DEV_TIMEOUT_SMEM_EMPTY)) {
+            ok = false;
+            break;
+          }
+          uint8_t* sa = smem + stage * C::STAGE_BYTES;
+          uint8_t* sb = sa + C::A_BYTES;
+          if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * C::STAGE_BYTES);
+          const uint32_t fbar = map_to_cta(smem_u32(&full[stage]), 0);
+          const bool slab = kb >= ts.nk1;
+          const CUtensorMap* ta = slab ? &tmA2 : &tmA1;
+          const CUtensorMap* tb = slab ? &tmB2 : &tmB1;
+          const int k0 = (slab ? kb - ts.nk1 : kb) * BK;
+          tma_load_2d_pair(sa, ta, fbar, k0, m0);
+          if (B_MN) {
+            tma_load_2d_pair(sb, tb, fbar, n0, k0);
+            tma_load_2d_pair(sb + 8192, tb, fbar, n0 + 64, k0);
+          } else {
+            tma_load_2d_pair(sb, tb, fbar, k0, n0);
+          }
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer (leader CTA only) ----------------
+    if (lane == 0 && rank == 0) {
+      constexpr uint32_t idesc = instr_desc(256, BN2, false, B_MN);
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int unit = pair; unit < n_units && ok; unit += npairs) {
+        int tm, tn, kb0, kb1;
+        decode_unit(ts, unit, tm, tn, kb0, kb1);
+        if (!wait_or_abort(&acce[acc], acc_phase ^ 1u, abort_flag, err, DEV_TIMEOUT_TMEM_EMPTY)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN2);
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!wait_or_abort(&full[stage], phase, abort_flag, err, DEV_TIMEOUT_TMA_FULL)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(smem + stage * C::STAGE_BYTES);
+          const uint32_t sb = sa + C::A_BYTES;
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k) {
+            const uint64_t da = smem_desc(sa + k * 32, 16, 1024);
+            const uint64_t db = B_MN ? smem_desc(sb + k * 2048, 8192, 1024) : smem_desc(sb + k * 32, 16, 1024);
+            mma_bf16_pair(d_tmem, da, db, idesc, (kb > kb0 || k > 0) ? 1u : 0u);
+          }
+          mma_commit_pair(&empty[stage]);
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        mma_commit_pair(&accf[acc]);
+        if (++acc == 2) {
+          acc = 0;
+          acc_phase ^= 1u;
+        }
+      }
+    }
+  } else {
+    // ---------------- epilogue (warps 2..5, both CTAs) ----------------
+    const int quarter = warp & 3;
+    const int row_in_tile = quarter * 32 + lane;
+    const uint32_t acce_leader0 = map_to_cta(smem_u32(&acce[0]), 0);
+    const uint32_t acce_leader1 = map_to_cta(smem_u32(&acce[1]), 0);
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int unit = pair; unit < n_units; unit += npairs) {
+      int tm, tn, kb0, kb1;
+      decode_unit(ts, unit, tm, tn, kb0, kb1);
+      if (!wait_or_abort(&accf[acc], acc_phase, abort_flag, err, DEV_TIMEOUT_ACCUM)) break;
+      tc_fence_after();
+      const int row = tm * 256 + static_cast<int>(rank) * 128 + row_in_tile;
+      const bool row_ok = row < M;
+#pragma unroll 1
+      for (int c = 0; c < BN2 / 32; ++c) {
+        float v[32];
+        tmem_ld32(tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
+                      static_cast<uint32_t>(acc * BN2 + c * 32),
+                  v);
+        const int col0 = tn * BN2 + c * 32;
+        if (!row_ok) continue;
+        __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(ep.C) + static_cast<int64_t>(row) * ep.ldc + col0;
+        if (col0 + 32 <= Nc && (ep.ldc % 8) == 0) {
+          uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            d4[q] = make_uint4(pack_bf16x2(v[8 * q + 0], v[8 * q + 1]), pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
+                               pack_bf16x2(v[8 * q + 4], v[8 * q + 5]), pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
+        } else {
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if (col0 + j < Nc) dst[j] = __float2bfloat16_rn(v[j]);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive_cluster(acc ? acce_leader1 : acce_leader0);
+      if (++acc == 2) {
+        acc = 0;
+        acc_phase ^= 1u;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();  // no CTA leaves while its peer may still signal it
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(C::TMEM_COLS)
+                 : "memory");
+  }
+}
+
+// ---------------------------------------------------------------------------
 // host side
 
 typedef CUresult (*PFN_encodeTiled)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -446,7 +709,47 @@ cudaError_t run(const Operand& a1, const Operand& b1, const Operand* a2, const O
   return cudaGetLastError();
 }
 
+template <bool B_MN>
+cudaError_t run_pair(const Operand& a1, const Operand& b1, const Operand& a2, const Operand& b2, int M, int Nc,
+                     const EpiParams& ep, int num_sms, int32_t* err, cudaStream_t stream) {
+  using C = Cfg2<B_MN>;
+  CUtensorMap ta1, tb1, ta2, tb2;
+  // each CTA loads 128 rows of A and 128 of B's output dimension per box
+  if (!map_operand(&ta1, a1, 128) || !map_operand(&tb1, b1, 128)) return cudaErrorInvalidValue;
+  if (!map_operand(&ta2, a2, 128) || !map_operand(&tb2, b2, 128)) return cudaErrorInvalidValue;
+  TileSched ts;
+  ts.tiles_m = static_cast<int>((M + 255) / 256);
+  ts.tiles_n = static_cast<int>((Nc + 255) / 256);
+  ts.nk1 = static_cast<int>((a1.k + BK - 1) / BK);
+  ts.nkb = ts.nk1 + static_cast<int>((a2.k + BK - 1) / BK);
+  ts.splits = 1;
+  ts.kb_per_split = ts.nkb;
+  const int units = ts.tiles_m * ts.tiles_n;
+  int pairs = num_sms / 2;
+  if (pairs > units) pairs = units;
+  if (pairs < 1) pairs = 1;
+  auto kern = k_tc_gemm2<B_MN>;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  kern<<<2 * pairs, kThreads, C::SMEM, stream>>>(ta1, tb1, ta2, tb2, ts, M, Nc, ep, err);
+  return cudaGetLastError();
+}
+
 }  // namespace
+
+// The 2-CTA kernel serves the large GEMMs (M >= 256 tokens) when QLORA_TC_PAIR=1
+// is set in the environment; otherwise the 1-CTA kernel runs.
+bool use_pair_kernel(int64_t M) {
+  static const bool enabled = [] {
+    const char* e = std::getenv("QLORA_TC_PAIR");
+    return e && e[0] == '1';
+  }();
+  return enabled && M >= 256;
+}
 
 // Forward main GEMM: Y[M,N] = X[M,K] W'[N,K]^T + sT[M,rpad] Bl[N,r]^T
 cudaError_t launch_gemm_fwd(const void* X, const void* Wd, const void* sT, const void* Bl, int64_t M, int64_t N,
@@ -456,6 +759,8 @@ cudaError_t launch_gemm_fwd(const void* X, const void* Wd, const void* sT, const
   EpiParams ep{};
   ep.C = Y;
   ep.ldc = N;
+  if (use_pair_kernel(M))
+    return run_pair<false>(a1, b1, a2, b2, static_cast<int>(M), static_cast<int>(N), ep, num_sms, err, stream);
   return run<256, false, false, OUT_BF16>(a1, b1, &a2, &b2, static_cast<int>(M), static_cast<int>(N), 1, ep,
                                           num_sms, err, stream);
 }
@@ -468,40 +773,32 @@ cudaError_t launch_gemm_dx(const void* dY, const void* Wd, const void* sU, const
   EpiParams ep{};
   ep.C = dX;
   ep.ldc = K;
+  if (use_pair_kernel(M))
+    return run_pair<true>(a1, b1, a2, b2, static_cast<int>(M), static_cast<int>(K), ep, num_sms, err, stream);
   return run<256, false, true, OUT_BF16>(a1, b1, &a2, &b2, static_cast<int>(M), static_cast<int>(K), 1, ep,
                                          num_sms, err, stream);
 }
 
-// LoRA down projection: T[M, r] = X[M,K] A[r,K]^T; writes T (fp32, optional),
-// sT = bf16(s T), T_hi = bf16(T), T_lo = bf16(T - T_hi), all [M, rpad].
-cudaError_t launch_gemm_lora_t(const void* X, const void* Al, int64_t M, int64_t K, int r, int rpad, float s,
-                               float* T, void* sT, void* T_hi, void* T_lo, int num_sms, int32_t* err,
-                               cudaStream_t stream) {
+// LoRA down projection, split over K: P[split][M][rpad] = partial sums of
+// X[M,K] A[r,K]^T (columns >= r are zero); launch_lora_finish turns them into
+// T (fp32, optional), sT = bf16(s T), T_hi = bf16(T), T_lo = bf16(T - T_hi).
+cudaError_t launch_gemm_lora_t(const void* X, const void* Al, int64_t M, int64_t K, int r, int rpad, float* P,
+                               int splits, int num_sms, int32_t* err, cudaStream_t stream) {
   Operand a1{X, M, K, K, false}, b1{Al, r, K, K, false};
   EpiParams ep{};
-  ep.f32 = T;
-  ep.ld_f32 = r;
-  ep.s_bf16 = sT;
-  ep.hi = T_hi;
-  ep.lo = T_lo;
-  ep.ld_pad = rpad;
-  ep.s = s;
-  return run<64, false, false, OUT_LORA>(a1, b1, nullptr, nullptr, static_cast<int>(M), r, 1, ep, num_sms, err,
-                                         stream);
+  ep.P = P;
+  return run<64, false, false, OUT_PARTIAL>(a1, b1, nullptr, nullptr, static_cast<int>(M), rpad, splits, ep,
+                                            num_sms, err, stream);
 }
 
-// LoRA up-gradient: U[M, r] = dY[M,N] B[N,r]; writes sU = bf16(s U), U_hi, U_lo [M, rpad].
-cudaError_t launch_gemm_lora_u(const void* dY, const void* Bl, int64_t M, int64_t N, int r, int rpad, float s,
-                               void* sU, void* U_hi, void* U_lo, int num_sms, int32_t* err, cudaStream_t stream) {
+// LoRA up-gradient, split over N: P[split][M][rpad] = partial sums of dY[M,N] B[N,r].
+cudaError_t launch_gemm_lora_u(const void* dY, const void* Bl, int64_t M, int64_t N, int r, int rpad, float* P,
+                               int splits, int num_sms, int32_t* err, cudaStream_t stream) {
   Operand a1{dY, M, N, N, false}, b1{Bl, r, N, r, true};
   EpiParams ep{};
-  ep.s_bf16 = sU;
-  ep.hi = U_hi;
-  ep.lo = U_lo;
-  ep.ld_pad = rpad;
-  ep.s = s;
-  return run<64, false, true, OUT_LORA>(a1, b1, nullptr, nullptr, static_cast<int>(M), r, 1, ep, num_sms, err,
-                                        stream);
+  ep.P = P;
+  return run<64, false, true, OUT_PARTIAL>(a1, b1, nullptr, nullptr, static_cast<int>(M), rpad, splits, ep,
+                                           num_sms, err, stream);
 }
 
 // Split reduction over tokens: P[split][R][rpad] = sum_m Q[m, R]^T (hi + lo)[m, rpad]

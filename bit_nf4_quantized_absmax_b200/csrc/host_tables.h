@@ -8,8 +8,10 @@
 namespace qlora {
 
 // Bin mapping used by the quantize kernel: x = fmaf(v, kBinScale, 3.0f) lies
-// in [2, 4) for v in [-1, 1]; the top 8 mantissa bits of x index the bin.
+// in [2, 4) for v in [-1, 1]; the top kBinBits mantissa bits of x index the bin.
 constexpr float kBinScale = 0.9990234375f;  // 1 - 2^-10, exact in fp32
+constexpr int kBinBits = 5;
+constexpr int kBins = 1 << kBinBits;
 
 struct BinEntry {
   float threshold;  // T_j
@@ -19,7 +21,7 @@ struct BinEntry {
 struct QuantTables {
   float codebook[16];     // ascending NF4 values, fp32
   float thresholds[15];   // T_i = smallest fp32 above the midpoint of codes i, i+1
-  BinEntry bins[256];
+  BinEntry bins[kBins];
 };
 
 // Computed once on first use (thread-safe static initialisation).

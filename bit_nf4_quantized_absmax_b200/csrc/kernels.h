@@ -44,17 +44,20 @@ cudaError_t launch_gemm_fwd(const void* X, const void* Wd, const void* sT, const
                             int64_t K, int r, int rpad, void* Y, int num_sms, int32_t* err, cudaStream_t stream);
 cudaError_t launch_gemm_dx(const void* dY, const void* Wd, const void* sU, const void* Al, int64_t M, int64_t N,
                            int64_t K, int r, int rpad, void* dX, int num_sms, int32_t* err, cudaStream_t stream);
-cudaError_t launch_gemm_lora_t(const void* X, const void* Al, int64_t M, int64_t K, int r, int rpad, float s,
-                               float* T, void* sT, void* T_hi, void* T_lo, int num_sms, int32_t* err,
-                               cudaStream_t stream);
-cudaError_t launch_gemm_lora_u(const void* dY, const void* Bl, int64_t M, int64_t N, int r, int rpad, float s,
-                               void* sU, void* U_hi, void* U_lo, int num_sms, int32_t* err, cudaStream_t stream);
+// Split-reduction partials P[splits][M][rpad] of X A^T (lora_t) and dY B (lora_u);
+// launch_lora_finish sums them and writes the fp32 / scaled / hi+lo operands.
+cudaError_t launch_gemm_lora_t(const void* X, const void* Al, int64_t M, int64_t K, int r, int rpad, float* P,
+                               int splits, int num_sms, int32_t* err, cudaStream_t stream);
+cudaError_t launch_gemm_lora_u(const void* dY, const void* Bl, int64_t M, int64_t N, int r, int rpad, float* P,
+                               int splits, int num_sms, int32_t* err, cudaStream_t stream);
 cudaError_t launch_gemm_lora_grad(const void* Q, int64_t R, const void* hi, const void* lo, int64_t M, int rpad,
                                   float* P, int splits, int num_sms, int32_t* err, cudaStream_t stream);
 
 // ---- lora_misc.cu ----
 cudaError_t launch_split_hilo(const float* T, int64_t M, int r, int rpad, void* hi, void* lo, int num_sms,
                               cudaStream_t stream);
+cudaError_t launch_lora_finish(const float* P, int splits, int64_t M, int r, int rpad, float s, float* f32,
+                               void* s_bf16, void* hi, void* lo, int num_sms, cudaStream_t stream);
 cudaError_t launch_grad_reduce(const float* P, int splits, int64_t R, int rpad, int r, float s, bool transpose,
                                void* out, int num_sms, cudaStream_t stream);
 cudaError_t launch_zero_bf16(void* p, int64_t n, int num_sms, cudaStream_t stream);

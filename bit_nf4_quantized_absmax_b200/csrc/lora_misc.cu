@@ -27,6 +27,37 @@ __global__ void k_split_hilo(const float* __restrict__ T, int64_t M, int r, int 
   }
 }
 
+// Sum the split partials P[p][m][j] (fixed order) and emit the LoRA operands:
+// f32[m][j] (j < r, optional), s_bf16 = bf16(s v), hi = bf16(v), lo = bf16(v - hi)
+// for j < rpad (zero columns stay zero). Two adjacent columns per thread.
+__global__ void k_lora_finish(const float* __restrict__ P, int splits, int64_t M, int r, int rpad, float s,
+                              float* __restrict__ f32, __nv_bfloat16* __restrict__ s_bf16,
+                              __nv_bfloat16* __restrict__ hi, __nv_bfloat16* __restrict__ lo) {
+  const int64_t n2 = M * rpad / 2;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n2;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t e = 2 * i;
+    const int64_t m = e / rpad;
+    const int j = static_cast<int>(e % rpad);
+    float2 v = make_float2(0.0f, 0.0f);
+    for (int p = 0; p < splits; ++p) {
+      const float2 pv = reinterpret_cast<const float2*>(P + (static_cast<int64_t>(p) * M) * rpad)[i];
+      v.x += pv.x;
+      v.y += pv.y;
+    }
+    if (f32) {
+      if (j < r) f32[m * r + j] = v.x;
+      if (j + 1 < r) f32[m * r + j + 1] = v.y;
+    }
+    if (s_bf16) reinterpret_cast<uint32_t*>(s_bf16)[i] = pack_bf16x2(s * v.x, s * v.y);
+    if (hi) {
+      const uint32_t h = pack_bf16x2(v.x, v.y);
+      reinterpret_cast<uint32_t*>(hi)[i] = h;
+      reinterpret_cast<uint32_t*>(lo)[i] = pack_bf16x2(v.x - bf16lo_to_f32(h), v.y - bf16hi_to_f32(h));
+    }
+  }
+}
+
 __global__ void k_grad_reduce(const float* __restrict__ P, int splits, int64_t R, int rpad, int r, float s,
                               int transpose, __nv_bfloat16* __restrict__ out) {
   const int64_t n = R * r;
@@ -65,6 +96,14 @@ cudaError_t launch_split_hilo(const float* T, int64_t M, int r, int rpad, void* 
                               cudaStream_t stream) {
   k_split_hilo<<<grid_for(M * rpad, num_sms), 256, 0, stream>>>(T, M, r, rpad, static_cast<__nv_bfloat16*>(hi),
                                                                   static_cast<__nv_bfloat16*>(lo));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_lora_finish(const float* P, int splits, int64_t M, int r, int rpad, float s, float* f32,
+                               void* s_bf16, void* hi, void* lo, int num_sms, cudaStream_t stream) {
+  k_lora_finish<<<grid_for(M * rpad / 2, num_sms), 256, 0, stream>>>(
+      P, splits, M, r, rpad, s, f32, static_cast<__nv_bfloat16*>(s_bf16), static_cast<__nv_bfloat16*>(hi),
+      static_cast<__nv_bfloat16*>(lo));
   return cudaGetLastError();
 }
 

@@ -6,7 +6,7 @@
 //   k_quant_zero   clears the 256 exponent bins and the CTA ticket.
 //   k_quant_pass1  streams W once: per 64-weight block the absmax (8-lane
 //                  shuffle reduction over 16-byte loads), the exact quotient
-//                  v = w / m, the nearest code (one bin lookup + one compare),
+//                  v = w / m, the nearest code (one lookup in a 32-bin table + one compare),
 //                  4-bit packing; it also accumulates the exact sum of the
 //                  absmax constants as integer significand sums per exponent.
 //                  The last CTA to finish turns that sum into the mean.
@@ -19,7 +19,7 @@
 namespace qlora {
 
 struct QuantBinTable {
-  BinEntry bins[256];
+  BinEntry bins[kBins];
 };
 
 namespace {
@@ -34,58 +34,73 @@ __global__ void k_quant_zero(unsigned long long* bins) {
 
 // Exact fp64 value of sum_E hist[E] * 2^(E - 134) (E = biased exponent, the
 // significand sums are integers): the sum is formed in a 320-bit fixed-point
-// integer with unit 2^-133, then rounded once to fp64 (nearest, ties to even).
+// integer with unit 2^-133 (five 64-bit limbs kept in registers), then rounded
+// once to fp64 (nearest, ties to even).
 __device__ double exact_sum_to_double(const unsigned long long* hist) {
-  unsigned long long limb[5] = {0, 0, 0, 0, 0};
+  unsigned long long L[5] = {0, 0, 0, 0, 0};
   for (int E = 1; E < 256; ++E) {
-    unsigned long long x = hist[E];
+    const unsigned long long x = hist[E];
     if (!x) continue;
     const int pos = E - 1;  // bit position of x's lsb
     const int li = pos >> 6, off = pos & 63;
-    unsigned long long lo = x << off;
-    unsigned long long hi = off ? (x >> (64 - off)) : 0ull;
-    // add (hi:lo) at limb li with carry propagation
-    unsigned long long old = limb[li];
-    limb[li] = old + lo;
-    unsigned long long carry = (limb[li] < old) ? 1ull : 0ull;
-    for (int k = li + 1; k < 5; ++k) {
-      unsigned long long add = (k == li + 1 ? hi : 0ull);
-      unsigned long long o = limb[k];
-      unsigned long long s1 = o + add;
-      unsigned long long c1 = (s1 < o) ? 1ull : 0ull;
-      unsigned long long s2 = s1 + carry;
-      unsigned long long c2 = (s2 < s1) ? 1ull : 0ull;
-      limb[k] = s2;
+    const unsigned long long lo = x << off;
+    const unsigned long long hi = off ? (x >> (64 - off)) : 0ull;
+    unsigned long long carry = 0ull;
+#pragma unroll
+    for (int k = 0; k < 5; ++k) {
+      const unsigned long long add = (k == li) ? lo : ((k == li + 1) ? hi : 0ull);
+      const unsigned long long s1 = L[k] + add;
+      const unsigned long long c1 = s1 < L[k] ? 1ull : 0ull;
+      const unsigned long long s2 = s1 + carry;
+      const unsigned long long c2 = s2 < s1 ? 1ull : 0ull;
+      L[k] = s2;
       carry = c1 + c2;
-      if (!carry && k > li + 1) break;
     }
   }
+  // highest set bit
   int top = -1;
-  for (int k = 4; k >= 0; --k) {
-    if (limb[k]) { top = k * 64 + 63 - __clzll((long long)limb[k]); break; }
-  }
+#pragma unroll
+  for (int k = 0; k < 5; ++k)
+    if (L[k]) top = k * 64 + 63 - __clzll(static_cast<long long>(L[k]));
   if (top < 0) return 0.0;
-  auto bit = [&](int p) -> unsigned long long { return (limb[p >> 6] >> (p & 63)) & 1ull; };
-  if (top < 53) {
-    return ldexp(static_cast<double>(limb[0]), -133);
+  if (top < 53) return ldexp(static_cast<double>(L[0]), -133);
+  // 53-bit significand = bits [top-52, top]; guard = bit top-53; sticky = below
+  const int sh = top - 52;  // >= 1
+  const int w = sh >> 6, b = sh & 63;
+  unsigned long long lo_w = 0ull, hi_w = 0ull;
+#pragma unroll
+  for (int k = 0; k < 5; ++k) {
+    if (k == w) lo_w = L[k];
+    if (k == w + 1) hi_w = L[k];
   }
-  // 53-bit significand from bits [top-52, top]
-  unsigned long long mant = 0;
-  for (int p = top; p >= top - 52; --p) mant = (mant << 1) | bit(p);
-  const int g = top - 53;
-  const unsigned long long guard = bit(g);
+  unsigned long long mant = b ? ((lo_w >> b) | (hi_w << (64 - b))) : lo_w;
+  mant &= (1ull << 53) - 1ull;
+  const int g = sh - 1;
+  const int gw = g >> 6, gb = g & 63;
+  unsigned long long gword = 0ull;
   bool sticky = false;
-  for (int p = g - 1; p >= 0 && !sticky; --p) sticky = bit(p) != 0;
-  if (guard && (sticky || (mant & 1ull))) mant += 1;
-  int exp2 = top - 52 - 133;
-  if (mant == (1ull << 53)) { mant >>= 1; exp2 += 1; }
+#pragma unroll
+  for (int k = 0; k < 5; ++k) {
+    if (k == gw) {
+      gword = L[k];
+      sticky = sticky || ((L[k] & ((1ull << gb) - 1ull)) != 0ull);
+    }
+    if (k < gw) sticky = sticky || (L[k] != 0ull);
+  }
+  const unsigned long long guard = (gword >> gb) & 1ull;
+  if (guard && (sticky || (mant & 1ull))) mant += 1ull;
+  int exp2 = sh - 133;
+  if (mant == (1ull << 53)) {
+    mant >>= 1;
+    exp2 += 1;
+  }
   return ldexp(static_cast<double>(mant), exp2);
 }
 
 __device__ __forceinline__ void quant_item(const uint4 d, bool valid, int lane, int64_t item,
                                            uint32_t* __restrict__ packed, float* __restrict__ absmax,
                                            const uint2* __restrict__ s_bins,
-                                           unsigned long long* __restrict__ s_hist) {
+                                           unsigned int* __restrict__ s_hist) {
   float w[8];
   w[0] = bf16lo_to_f32(d.x); w[1] = bf16hi_to_f32(d.x);
   w[2] = bf16lo_to_f32(d.y); w[3] = bf16hi_to_f32(d.y);
@@ -107,7 +122,7 @@ __device__ __forceinline__ void quant_item(const uint4 d, bool valid, int lane, 
       const uint32_t mant7 = (u >> 16) & 0x7Fu;
       const uint32_t sig = e ? (mant7 | 0x80u) : mant7;
       const uint32_t E = e ? e : 1u;
-      atomicAdd(&s_hist[E], static_cast<unsigned long long>(sig));
+      atomicAdd(&s_hist[E], sig);
     }
   }
   uint32_t word;
@@ -117,22 +132,25 @@ __device__ __forceinline__ void quant_item(const uint4 d, bool valid, int lane, 
     // Keep 1/m normal: scale w and m by a power of two (exact for bf16 values;
     // only weights whose quotient is below 2^-126 can lose bits, and those map
     // to the zero code either way).
-    float sc = 1.0f;
-    if (m < 5.421010862e-20f) sc = 1.8446744e19f;        // m < 2^-64: times 2^64
-    else if (m > 1.8446744e19f) sc = 5.421010862e-20f;   // m > 2^64: times 2^-64
-    const float ms = m * sc;
+    float ms = m;
+    if (m < 5.421010862e-20f || m > 1.8446744e19f) {     // outside [2^-64, 2^64]: rare
+      const float sc = m < 5.421010862e-20f ? 1.8446744e19f : 5.421010862e-20f;
+      ms = m * sc;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) w[i] *= sc;
+    }
     const float r = __frcp_rn(ms);
     word = 0u;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      const float wi = w[i] * sc;
+      const float wi = w[i];
       // v = RN(w / m): q0 = RN(w * RN(1/m)) is within one ulp, the remainder
       // w - q0 m is exact, and one correction step rounds correctly (Markstein).
       const float q0 = __fmul_rn(wi, r);
       const float res = __fmaf_rn(-q0, ms, wi);
       const float v = __fmaf_rn(res, r, q0);
       const float x = __fmaf_rn(v, kBinScale, 3.0f);
-      const uint2 e = s_bins[(__float_as_uint(x) >> 15) & 0xFFu];
+      const uint2 e = s_bins[(__float_as_uint(x) >> (23 - kBinBits)) & (kBins - 1)];
       const uint32_t code = e.y + (v >= __uint_as_float(e.x) ? 1u : 0u);
       word |= code << (4 * i);
     }
@@ -144,13 +162,14 @@ __global__ void __launch_bounds__(kPass1Threads)
 k_quant_pass1(const uint4* __restrict__ W, int64_t n_items, uint32_t* __restrict__ packed,
               float* __restrict__ absmax, unsigned long long* __restrict__ gbins, float* __restrict__ mean_out,
               int64_t nblk, const __grid_constant__ QuantBinTable tab) {
-  __shared__ uint2 s_bins[256];
-  __shared__ unsigned long long s_hist[256];
+  __shared__ uint2 s_bins[kBins];
+  __shared__ unsigned int s_hist[256];          // per-CTA significand sums (native 32-bit atomics)
+  __shared__ unsigned long long s_tot[256];
   __shared__ int s_last;
   const int tid = threadIdx.x;
   const int lane = tid & 31;
-  s_bins[tid] = make_uint2(__float_as_uint(tab.bins[tid].threshold), tab.bins[tid].j);
-  s_hist[tid] = 0ull;
+  if (tid < kBins) s_bins[tid] = make_uint2(__float_as_uint(tab.bins[tid].threshold), tab.bins[tid].j);
+  s_hist[tid] = 0u;
   __syncthreads();
 
   const int64_t stride = static_cast<int64_t>(gridDim.x) * kPass1Threads;
@@ -169,7 +188,7 @@ k_quant_pass1(const uint4* __restrict__ W, int64_t n_items, uint32_t* __restrict
     }
   }
   __syncthreads();
-  if (s_hist[tid]) atomicAdd(&gbins[tid], s_hist[tid]);
+  if (s_hist[tid]) atomicAdd(&gbins[tid], static_cast<unsigned long long>(s_hist[tid]));
   __threadfence();
   __syncthreads();
   if (tid == 0) {
@@ -179,10 +198,10 @@ k_quant_pass1(const uint4* __restrict__ W, int64_t n_items, uint32_t* __restrict
   __syncthreads();
   if (s_last) {
     __threadfence();
-    s_hist[tid] = atomicAdd(&gbins[tid], 0ull);  // coherent read of the final bins
+    s_tot[tid] = atomicAdd(&gbins[tid], 0ull);  // coherent read of the final bins
     __syncthreads();
     if (tid == 0) {
-      const double S = exact_sum_to_double(s_hist);
+      const double S = exact_sum_to_double(s_tot);
       const double mu = __ddiv_rn(S, static_cast<double>(nblk));
       *mean_out = __double2float_rn(mu);
     }
@@ -250,7 +269,7 @@ cudaError_t launch_quantize(const void* W, int64_t numel, uint8_t* packed, int8_
                             cudaStream_t stream) {
   const QuantTables& tabs = quant_tables();
   QuantBinTable tab;
-  for (int i = 0; i < 256; ++i) tab.bins[i] = tabs.bins[i];
+  for (int i = 0; i < kBins; ++i) tab.bins[i] = tabs.bins[i];
   const int64_t n_items = numel / 8;
   const int64_t nblk = numel / 64;
   const int64_t ngrp = (nblk + 255) / 256;
@@ -258,7 +277,11 @@ cudaError_t launch_quantize(const void* W, int64_t numel, uint8_t* packed, int8_
   k_quant_zero<<<1, 320, 0, stream>>>(bins);
   int64_t want = (n_items + kPass1Threads * kPass1Unroll - 1) / (kPass1Threads * kPass1Unroll);
   int64_t cap = static_cast<int64_t>(num_sms) * 8;
-  const int grid = static_cast<int>(want < cap ? (want > 0 ? want : 1) : cap);
+  int64_t g = want < cap ? (want > 0 ? want : 1) : cap;
+  // A CTA sums at most 2^24 significands of 8 bits, so its 32-bit bins cannot overflow.
+  const int64_t min_grid = (nblk + (int64_t(1) << 24) - 1) >> 24;
+  if (g < min_grid) g = min_grid;
+  const int grid = static_cast<int>(g);
   k_quant_pass1<<<grid, kPass1Threads, 0, stream>>>(reinterpret_cast<const uint4*>(W), n_items,
                                                     reinterpret_cast<uint32_t*>(packed), absmax_scratch, bins,
                                                     mean, nblk, tab);
