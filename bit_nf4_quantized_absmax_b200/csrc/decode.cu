@@ -39,6 +39,7 @@ struct RowBlock {
   float sc;       // its group scale (the decoded constant is formed when the block is used)
 };
 
+template <bool V8>
 __device__ __forceinline__ RowBlock load_row_block(const uint8_t* __restrict__ packed, const int8_t* __restrict__ q,
                                                    const float* __restrict__ dqs, float mu, int64_t n,
                                                    int64_t nkb_row, int64_t kb, bool valid) {
@@ -46,8 +47,15 @@ __device__ __forceinline__ RowBlock load_row_block(const uint8_t* __restrict__ p
   if (valid) {
     const int64_t blk = n * nkb_row + kb;
     const uint4* p = reinterpret_cast<const uint4*>(packed + blk * 32);
-    rb.n0 = __ldcs(p);
-    rb.n1 = __ldcs(p + 1);
+    if (V8) {
+      uint32_t r[8];
+      ld_global_cs_v8(p, r);
+      rb.n0 = make_uint4(r[0], r[1], r[2], r[3]);
+      rb.n1 = make_uint4(r[4], r[5], r[6], r[7]);
+    } else {
+      rb.n0 = __ldcs(p);
+      rb.n1 = __ldcs(p + 1);
+    }
     rb.qv = static_cast<int>(__ldg(q + blk));
     rb.sc = __ldg(dqs + (blk >> 8));
   } else {
@@ -72,7 +80,7 @@ __device__ __forceinline__ uint32_t nib_word(const RowBlock& rb, int w) {
   }
 }
 
-template <int MT>
+template <int MT, bool V8>
 __global__ void __launch_bounds__(kDecodeWarps * 32, 2)
 k_decode(const uint8_t* __restrict__ packed, const int8_t* __restrict__ q, const float* __restrict__ dqs,
          const float* __restrict__ mean, const __nv_bfloat16* __restrict__ X, int M, int64_t N, int64_t K,
@@ -105,8 +113,8 @@ k_decode(const uint8_t* __restrict__ packed, const int8_t* __restrict__ q, const
   if (sb < sb_end) {
     const int64_t kb = sb * 4 + t;
     const bool kv = kb < nkb_row;
-    na_next = load_row_block(packed, q, dqs, mu, na, nkb_row, kb, kv && na < N);
-    nb_next = load_row_block(packed, q, dqs, mu, nb, nkb_row, kb, kv && nb < N);
+    na_next = load_row_block<V8>(packed, q, dqs, mu, na, nkb_row, kb, kv && na < N);
+    nb_next = load_row_block<V8>(packed, q, dqs, mu, nb, nkb_row, kb, kv && nb < N);
   }
   for (; sb < sb_end; sb += kDecodeWarps) {
     const int64_t kb = sb * 4 + t;
@@ -126,8 +134,8 @@ k_decode(const uint8_t* __restrict__ packed, const int8_t* __restrict__ q, const
     if (sbn < sb_end) {
       const int64_t kbn = sbn * 4 + t;
       const bool kvn = kbn < nkb_row;
-      na_next = load_row_block(packed, q, dqs, mu, na, nkb_row, kbn, kvn && na < N);
-      nb_next = load_row_block(packed, q, dqs, mu, nb, nkb_row, kbn, kvn && nb < N);
+      na_next = load_row_block<V8>(packed, q, dqs, mu, na, nkb_row, kbn, kvn && na < N);
+      nb_next = load_row_block<V8>(packed, q, dqs, mu, nb, nkb_row, kbn, kvn && nb < N);
     }
     const Nf4Lut la = make_nf4_lut(cb, __fmaf_rn(static_cast<float>(ra.qv), ra.sc, mu));
     const Nf4Lut lb = make_nf4_lut(cb, __fmaf_rn(static_cast<float>(rbk.qv), rbk.sc, mu));
@@ -137,8 +145,17 @@ k_decode(const uint8_t* __restrict__ packed, const int8_t* __restrict__ q, const
       if ((st & 3) == 0) {
 #pragma unroll
         for (int j = 0; j < MT; ++j) {
-          xv[j][0] = xok[j] ? __ldg(xp[j] + (st >> 1)) : make_uint4(0, 0, 0, 0);
-          xv[j][1] = xok[j] ? __ldg(xp[j] + (st >> 1) + 1) : make_uint4(0, 0, 0, 0);
+          if (!xok[j]) {
+            xv[j][0] = xv[j][1] = make_uint4(0, 0, 0, 0);
+          } else if (V8) {
+            uint32_t r[8];
+            ld_global_nc_v8(xp[j] + (st >> 1), r);
+            xv[j][0] = make_uint4(r[0], r[1], r[2], r[3]);
+            xv[j][1] = make_uint4(r[4], r[5], r[6], r[7]);
+          } else {
+            xv[j][0] = __ldg(xp[j] + (st >> 1));
+            xv[j][1] = __ldg(xp[j] + (st >> 1) + 1);
+          }
         }
       }
       const uint32_t wa = nib_word(ra, st >> 1) >> (16 * (st & 1));
@@ -302,16 +319,19 @@ cudaError_t launch_decode_fwd(const Nf4View& w, const void* X, int64_t M, const 
                                              reinterpret_cast<const __nv_bfloat16*>(A), static_cast<int>(M), w.K, r,
                                              T, counters, static_cast<int>(row_tiles));
   dim3 grid(static_cast<unsigned>(row_tiles), static_cast<unsigned>(ksplit));
+  const bool v8 = ((reinterpret_cast<uintptr_t>(X) | reinterpret_cast<uintptr_t>(w.packed)) & 31u) == 0;
+  auto launch = [&](auto kern) {
+    kern<<<grid, kDecodeWarps * 32, 0, stream>>>(w.packed, w.absmax_q, w.dq_scale, w.mean,
+                                                  reinterpret_cast<const __nv_bfloat16*>(X), static_cast<int>(M), w.N,
+                                                  w.K, T, reinterpret_cast<const __nv_bfloat16*>(B), r, s,
+                                                  reinterpret_cast<__nv_bfloat16*>(Y), partial, counters, ksplit, cb);
+  };
   if (M <= 8) {
-    k_decode<1><<<grid, kDecodeWarps * 32, 0, stream>>>(
-        w.packed, w.absmax_q, w.dq_scale, w.mean, reinterpret_cast<const __nv_bfloat16*>(X), static_cast<int>(M), w.N,
-        w.K, T, reinterpret_cast<const __nv_bfloat16*>(B), r, s, reinterpret_cast<__nv_bfloat16*>(Y), partial,
-        counters, ksplit, cb);
+    if (v8) launch(k_decode<1, true>);
+    else launch(k_decode<1, false>);
   } else {
-    k_decode<2><<<grid, kDecodeWarps * 32, 0, stream>>>(
-        w.packed, w.absmax_q, w.dq_scale, w.mean, reinterpret_cast<const __nv_bfloat16*>(X), static_cast<int>(M), w.N,
-        w.K, T, reinterpret_cast<const __nv_bfloat16*>(B), r, s, reinterpret_cast<__nv_bfloat16*>(Y), partial,
-        counters, ksplit, cb);
+    if (v8) launch(k_decode<2, true>);
+    else launch(k_decode<2, false>);
   }
   return cudaGetLastError();
 }

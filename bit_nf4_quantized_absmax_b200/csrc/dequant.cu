@@ -13,23 +13,30 @@ namespace {
 
 constexpr int kDeqUnroll = 4;
 
+template <bool V8>
 __device__ __forceinline__ void dequant_unit(const uint4 nib, int64_t u, float mp, uint4* __restrict__ out,
                                              const Nf4Codebook& cb) {
   const Nf4Lut t = make_nf4_lut(cb, mp);
-  uint32_t o[16];
-  nf4_lookup8(t, nib.x, o + 0);
-  nf4_lookup8(t, nib.y, o + 4);
-  nf4_lookup8(t, nib.z, o + 8);
-  nf4_lookup8(t, nib.w, o + 12);
+  uint32_t o[2][8];
+  nf4_lookup8(t, nib.x, o[0] + 0);
+  nf4_lookup8(t, nib.y, o[0] + 4);
+  nf4_lookup8(t, nib.z, o[1] + 0);
+  nf4_lookup8(t, nib.w, o[1] + 4);
   uint4* dst = out + u * 4;
-  __stcs(dst + 0, make_uint4(o[0], o[1], o[2], o[3]));
-  __stcs(dst + 1, make_uint4(o[4], o[5], o[6], o[7]));
-  __stcs(dst + 2, make_uint4(o[8], o[9], o[10], o[11]));
-  __stcs(dst + 3, make_uint4(o[12], o[13], o[14], o[15]));
+  if (V8) {  // two full 32-byte sectors per thread
+    st_global_cs_v8(dst, o[0]);
+    st_global_cs_v8(dst + 2, o[1]);
+  } else {
+    __stcs(dst + 0, make_uint4(o[0][0], o[0][1], o[0][2], o[0][3]));
+    __stcs(dst + 1, make_uint4(o[0][4], o[0][5], o[0][6], o[0][7]));
+    __stcs(dst + 2, make_uint4(o[1][0], o[1][1], o[1][2], o[1][3]));
+    __stcs(dst + 3, make_uint4(o[1][4], o[1][5], o[1][6], o[1][7]));
+  }
 }
 
 // Grid-stride over 32-weight units; each thread keeps kDeqUnroll 16-byte
 // loads in flight before decoding them.
+template <bool V8>
 __global__ void __launch_bounds__(256)
 k_dequant(const uint4* __restrict__ packed, const int8_t* __restrict__ absmax_q,
           const float* __restrict__ dq_scale, const float* __restrict__ mean, uint4* __restrict__ out,
@@ -54,7 +61,7 @@ k_dequant(const uint4* __restrict__ packed, const int8_t* __restrict__ absmax_q,
     for (int i = 0; i < kDeqUnroll; ++i) {
       const int64_t u = u0 + i * stride;
       if (u < n_units)
-        dequant_unit(nib[i], u, __fmaf_rn(static_cast<float>(qv[i]), sc[i], mu), out, cb);
+        dequant_unit<V8>(nib[i], u, __fmaf_rn(static_cast<float>(qv[i]), sc[i], mu), out, cb);
     }
   }
 }
@@ -70,8 +77,12 @@ cudaError_t launch_dequantize(const uint8_t* packed, const int8_t* absmax_q, con
   int64_t want = (n_units + 256 * kDeqUnroll - 1) / (256 * kDeqUnroll);
   int64_t cap = static_cast<int64_t>(num_sms) * 8;
   const int grid = static_cast<int>(want < cap ? (want > 0 ? want : 1) : cap);
-  k_dequant<<<grid, 256, 0, stream>>>(reinterpret_cast<const uint4*>(packed), absmax_q, dq_scale, mean,
-                                      reinterpret_cast<uint4*>(out), n_units, cb);
+  if ((reinterpret_cast<uintptr_t>(out) & 31u) == 0)
+    k_dequant<true><<<grid, 256, 0, stream>>>(reinterpret_cast<const uint4*>(packed), absmax_q, dq_scale, mean,
+                                              reinterpret_cast<uint4*>(out), n_units, cb);
+  else
+    k_dequant<false><<<grid, 256, 0, stream>>>(reinterpret_cast<const uint4*>(packed), absmax_q, dq_scale, mean,
+                                               reinterpret_cast<uint4*>(out), n_units, cb);
   return cudaGetLastError();
 }
 

@@ -741,12 +741,12 @@ cudaError_t run_pair(const Operand& a1, const Operand& b1, const Operand& a2, co
 
 }  // namespace
 
-// The 2-CTA kernel serves the large GEMMs (M >= 256 tokens) when QLORA_TC_PAIR=1
-// is set in the environment; otherwise the 1-CTA kernel runs.
+// The 2-CTA kernel serves the large GEMMs (M >= 256 tokens); QLORA_TC_PAIR=0 in
+// the environment selects the 1-CTA kernel instead (for comparisons).
 bool use_pair_kernel(int64_t M) {
   static const bool enabled = [] {
     const char* e = std::getenv("QLORA_TC_PAIR");
-    return e && e[0] == '1';
+    return !(e && e[0] == '0');
   }();
   return enabled && M >= 256;
 }
