@@ -91,11 +91,9 @@ int32_t* device_error_word() {
 int grad_splits(int64_t R, int rpad, int64_t M, int num_sms) {
   const int64_t tiles = ((R + 127) / 128) * (rpad / 64);
   if (tiles <= 0) return 1;
-  const int64_t nkb = 2 * ((M + 63) / 64);
-  int64_t sp = (num_sms + tiles - 1) / tiles;
-  if (sp > nkb) sp = nkb;
-  if (sp < 1) sp = 1;
-  return static_cast<int>(sp);
+  const int64_t nkb = 2 * ((M + 63) / 64);  // hi and lo halves
+  const int64_t sp = (2 * num_sms) / tiles;  // at most one round of the two resident CTAs per SM
+  return split_count(nkb, static_cast<int>(sp < 1 ? 1 : sp));
 }
 
 // Split count for the K (or N) reduction of the rank-r products X A^T and dY B.
@@ -103,10 +101,8 @@ int red_splits(int64_t M, int rpad, int64_t Kred, int num_sms) {
   const int64_t tiles = ((M + 127) / 128) * (rpad / 64);
   if (tiles <= 0) return 1;
   const int64_t nkb = (Kred + 63) / 64;
-  int64_t sp = (num_sms + tiles - 1) / tiles;
-  if (sp > nkb) sp = nkb;
-  if (sp < 1) sp = 1;
-  return static_cast<int>(sp);
+  const int64_t sp = (2 * num_sms) / tiles;  // at most one round of the two resident CTAs per SM
+  return split_count(nkb, static_cast<int>(sp < 1 ? 1 : sp));
 }
 
 // Workspace layout: consecutive 256-byte aligned regions.

@@ -97,13 +97,38 @@ __device__ __forceinline__ void prefetch_tmap(const void* tmap) {
 }
 
 // ---------------------------------------------------------------------------
-// Programmatic dependent launch
+// Programmatic dependent launch. Every kernel of the library is launched with
+// programmatic stream serialization, does its prologue (no global memory), then
+// pdl_enter(): it waits for the preceding grid to complete (and its writes to be
+// visible) and only then lets the next grid launch. Waiting before triggering
+// keeps the ordering transitive across the whole stream.
 
 __device__ __forceinline__ void grid_dependency_wait() {
   asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 __device__ __forceinline__ void grid_dependency_launch_dependents() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_enter() {
+  grid_dependency_wait();
+  grid_dependency_launch_dependents();
+}
+
+// Host side: launch a kernel with programmatic stream serialization allowed.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                              Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
 }
 
 // ---------------------------------------------------------------------------
@@ -128,6 +153,35 @@ __device__ __forceinline__ void ld_global_cs_v8(const void* p, uint32_t (&r)[8])
 }
 
 __device__ __forceinline__ bool aligned32(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 31u) == 0; }
+
+// ---------------------------------------------------------------------------
+// Packed fp32x2 arithmetic (sm_100): two independent IEEE operations, each
+// rounded to nearest even, in one instruction.
+
+struct f32x2 {
+  float x, y;
+};
+
+__device__ __forceinline__ f32x2 mul_f32x2(f32x2 a, f32x2 b) {
+  unsigned long long A, B, D;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(A) : "f"(a.x), "f"(a.y));
+  asm("mov.b64 %0, {%1, %2};" : "=l"(B) : "f"(b.x), "f"(b.y));
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(D) : "l"(A), "l"(B));
+  f32x2 d;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(d.x), "=f"(d.y) : "l"(D));
+  return d;
+}
+
+__device__ __forceinline__ f32x2 fma_f32x2(f32x2 a, f32x2 b, f32x2 c) {
+  unsigned long long A, B, C, D;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(A) : "f"(a.x), "f"(a.y));
+  asm("mov.b64 %0, {%1, %2};" : "=l"(B) : "f"(b.x), "f"(b.y));
+  asm("mov.b64 %0, {%1, %2};" : "=l"(C) : "f"(c.x), "f"(c.y));
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(D) : "l"(A), "l"(B), "l"(C));
+  f32x2 d;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(d.x), "=f"(d.y) : "l"(D));
+  return d;
+}
 
 // ---------------------------------------------------------------------------
 // bf16 helpers

@@ -41,6 +41,7 @@ __global__ void __launch_bounds__(256)
 k_dequant(const uint4* __restrict__ packed, const int8_t* __restrict__ absmax_q,
           const float* __restrict__ dq_scale, const float* __restrict__ mean, uint4* __restrict__ out,
           int64_t n_units, const __grid_constant__ Nf4Codebook cb) {
+  pdl_enter();
   const float mu = *mean;
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
   for (int64_t u0 = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; u0 < n_units;
@@ -77,13 +78,10 @@ cudaError_t launch_dequantize(const uint8_t* packed, const int8_t* absmax_q, con
   int64_t want = (n_units + 256 * kDeqUnroll - 1) / (256 * kDeqUnroll);
   int64_t cap = static_cast<int64_t>(num_sms) * 8;
   const int grid = static_cast<int>(want < cap ? (want > 0 ? want : 1) : cap);
-  if ((reinterpret_cast<uintptr_t>(out) & 31u) == 0)
-    k_dequant<true><<<grid, 256, 0, stream>>>(reinterpret_cast<const uint4*>(packed), absmax_q, dq_scale, mean,
-                                              reinterpret_cast<uint4*>(out), n_units, cb);
-  else
-    k_dequant<false><<<grid, 256, 0, stream>>>(reinterpret_cast<const uint4*>(packed), absmax_q, dq_scale, mean,
-                                               reinterpret_cast<uint4*>(out), n_units, cb);
-  return cudaGetLastError();
+  const bool v8 = (reinterpret_cast<uintptr_t>(out) & 31u) == 0;
+  return launch_pdl(v8 ? k_dequant<true> : k_dequant<false>, dim3(grid), dim3(256), 0, stream,
+                    reinterpret_cast<const uint4*>(packed), absmax_q, dq_scale, mean, reinterpret_cast<uint4*>(out),
+                    n_units, cb);
 }
 
 }  // namespace qlora

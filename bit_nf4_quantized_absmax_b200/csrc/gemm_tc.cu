@@ -52,7 +52,8 @@ struct Cfg {
   static constexpr int A_BYTES = BM * BK * 2;
   static constexpr int B_BYTES = BN * BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr int STAGES = (200 * 1024) / STAGE_BYTES > 8 ? 8 : (200 * 1024) / STAGE_BYTES;
+  // BN = 64 (the rank-r contractions) keeps 4 stages so that two CTAs fit on an SM.
+  static constexpr int STAGES = BN == 64 ? 4 : ((200 * 1024) / STAGE_BYTES > 8 ? 8 : (200 * 1024) / STAGE_BYTES);
   static constexpr int TMEM_COLS = (2 * BN) < 32 ? 32 : 2 * BN;
   static constexpr int SMEM = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
 };
@@ -130,7 +131,7 @@ __device__ __forceinline__ void decode_unit(const TileSched& ts, int unit, int& 
 }
 
 template <int BN, bool A_MN, bool B_MN, int OUT>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads)
 k_tc_gemm(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmB1,
           const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2, TileSched ts,
           int M, int Nc, EpiParams ep, int32_t* err) {
@@ -176,6 +177,7 @@ k_tc_gemm(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUte
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
+  pdl_enter();  // inputs written by the preceding kernel are visible from here on
 
   if (warp == 0) {
     // ---------------- TMA producer ----------------
@@ -486,6 +488,7 @@ k_tc_gemm2(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUt
   cluster_sync_all();  // the peer's barriers are initialised before any remote use
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
+  pdl_enter();  // inputs written by the preceding kernel are visible from here on
 
   if (warp == 0) {
     // ---------------- TMA producer (both CTAs) ----------------
@@ -692,12 +695,14 @@ cudaError_t run(const Operand& a1, const Operand& b1, const Operand* a2, const O
   ts.nk1 = static_cast<int>((a1.k + BK - 1) / BK);
   const int nk2 = (a2 && b2) ? static_cast<int>((a2->k + BK - 1) / BK) : 0;
   ts.nkb = ts.nk1 + nk2;
-  if (splits < 1) splits = 1;
-  if (splits > ts.nkb) splits = ts.nkb;
+  // callers pass a count from split_count(), so every piece is non-empty and the
+  // number of partial slices written equals `splits`
+  if (splits != split_count(ts.nkb, splits)) return cudaErrorInvalidValue;
   ts.kb_per_split = (ts.nkb + splits - 1) / splits;
-  ts.splits = (ts.nkb + ts.kb_per_split - 1) / ts.kb_per_split;
+  ts.splits = splits;
   const int units = ts.tiles_m * ts.tiles_n * ts.splits;
-  const int grid = units < num_sms ? units : num_sms;
+  const int slots = (BN == 64 ? 2 : 1) * num_sms;  // resident CTAs
+  const int grid = units < slots ? units : slots;
   auto kern = k_tc_gemm<BN, A_MN, B_MN, OUT>;
   static bool attr_set = false;
   if (!attr_set) {
@@ -705,8 +710,7 @@ cudaError_t run(const Operand& a1, const Operand& b1, const Operand* a2, const O
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  kern<<<grid, kThreads, C::SMEM, stream>>>(ta1, tb1, ta2, tb2, ts, M, Nc, ep, err);
-  return cudaGetLastError();
+  return launch_pdl(kern, dim3(grid), dim3(kThreads), C::SMEM, stream, ta1, tb1, ta2, tb2, ts, M, Nc, ep, err);
 }
 
 template <bool B_MN>
@@ -735,8 +739,7 @@ cudaError_t run_pair(const Operand& a1, const Operand& b1, const Operand& a2, co
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  kern<<<2 * pairs, kThreads, C::SMEM, stream>>>(ta1, tb1, ta2, tb2, ts, M, Nc, ep, err);
-  return cudaGetLastError();
+  return launch_pdl(kern, dim3(2 * pairs), dim3(kThreads), C::SMEM, stream, ta1, tb1, ta2, tb2, ts, M, Nc, ep, err);
 }
 
 }  // namespace

@@ -10,6 +10,17 @@ namespace qlora {
 
 constexpr int kQuantBinWords = 257;  // 256 exponent bins + 1 CTA ticket (u64 each)
 
+// Number of non-empty pieces when `nkb` k-blocks are cut into pieces of
+// ceil(nkb / want) blocks. The split-reduction GEMMs and the kernels that sum
+// their partials must both use this count.
+inline int split_count(int64_t nkb, int want) {
+  if (nkb <= 0) return 1;
+  if (want < 1) want = 1;
+  if (want > nkb) want = static_cast<int>(nkb);
+  const int64_t per = (nkb + want - 1) / want;
+  return static_cast<int>((nkb + per - 1) / per);
+}
+
 // ---- quantize.cu / dequant.cu ----
 cudaError_t launch_quantize(const void* W, int64_t numel, uint8_t* packed, int8_t* absmax_q, float* dq_scale,
                             float* mean, float* absmax_scratch, unsigned long long* bins, int num_sms,

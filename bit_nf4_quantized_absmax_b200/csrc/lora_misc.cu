@@ -15,6 +15,7 @@ namespace {
 
 __global__ void k_split_hilo(const float* __restrict__ T, int64_t M, int r, int rpad, __nv_bfloat16* __restrict__ hi,
                              __nv_bfloat16* __restrict__ lo) {
+  pdl_enter();
   const int64_t n = M * rpad;
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
@@ -33,6 +34,7 @@ __global__ void k_split_hilo(const float* __restrict__ T, int64_t M, int r, int 
 __global__ void k_lora_finish(const float* __restrict__ P, int splits, int64_t M, int r, int rpad, float s,
                               float* __restrict__ f32, __nv_bfloat16* __restrict__ s_bf16,
                               __nv_bfloat16* __restrict__ hi, __nv_bfloat16* __restrict__ lo) {
+  pdl_enter();
   const int64_t n2 = M * rpad / 2;
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n2;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
@@ -58,26 +60,53 @@ __global__ void k_lora_finish(const float* __restrict__ P, int splits, int64_t M
   }
 }
 
-__global__ void k_grad_reduce(const float* __restrict__ P, int splits, int64_t R, int rpad, int r, float s,
-                              int transpose, __nv_bfloat16* __restrict__ out) {
-  const int64_t n = R * r;
-  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    int64_t row, j;
-    if (transpose) {  // out [r, R]: consecutive threads walk R
-      j = i / R;
-      row = i % R;
-    } else {          // out [R, r]
-      row = i / r;
-      j = i % r;
+// out = bf16(s * sum_p P[p]) for a [R, rpad] partial stack (rows R, the first r
+// columns kept). A CTA owns a 32-row x 64-column tile: coalesced float2 reads of
+// every split (fixed order), then either direct row-major writes ([R, r]) or a
+// transpose through shared memory so that the [r, R] writes are coalesced too.
+__global__ void __launch_bounds__(256)
+k_grad_reduce(const float* __restrict__ P, int splits, int64_t R, int rpad, int r, float s, int transpose,
+              __nv_bfloat16* __restrict__ out) {
+  pdl_enter();
+  __shared__ float tile[64][33];
+  const int64_t row0 = static_cast<int64_t>(blockIdx.x) * 32;
+  const int col0 = blockIdx.y * 64;
+  const int tx = threadIdx.x & 31;   // column pair within the tile
+  const int ty = threadIdx.x >> 5;   // 8 row lanes
+  for (int rr = ty; rr < 32; rr += 8) {
+    const int64_t row = row0 + rr;
+    float2 v = make_float2(0.0f, 0.0f);
+    if (row < R) {
+      for (int p = 0; p < splits; ++p) {
+        const float2 pv =
+            reinterpret_cast<const float2*>(P + (static_cast<int64_t>(p) * R + row) * rpad + col0)[tx];
+        v.x += pv.x;
+        v.y += pv.y;
+      }
     }
-    float acc = 0.0f;
-    for (int p = 0; p < splits; ++p) acc += P[(static_cast<int64_t>(p) * R + row) * rpad + j];
-    out[i] = __float2bfloat16_rn(s * acc);
+    const int c = 2 * tx;
+    if (!transpose) {
+      if (row < R) {
+        if (col0 + c < r) out[row * r + col0 + c] = __float2bfloat16_rn(s * v.x);
+        if (col0 + c + 1 < r) out[row * r + col0 + c + 1] = __float2bfloat16_rn(s * v.y);
+      }
+    } else {
+      tile[c][rr] = v.x;
+      tile[c + 1][rr] = v.y;
+    }
+  }
+  if (!transpose) return;
+  __syncthreads();
+  // out[j][row]: 32 consecutive rows per column j, one warp per column
+  for (int cc = ty; cc < 64; cc += 8) {
+    const int j = col0 + cc;
+    const int64_t row = row0 + tx;
+    if (j < r && row < R) out[static_cast<int64_t>(j) * R + row] = __float2bfloat16_rn(s * tile[cc][tx]);
   }
 }
 
 __global__ void k_zero_bf16(__nv_bfloat16* __restrict__ p, int64_t n) {
+  pdl_enter();
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x)
     p[i] = __float2bfloat16_rn(0.0f);
@@ -94,30 +123,28 @@ int grid_for(int64_t n, int num_sms) {
 
 cudaError_t launch_split_hilo(const float* T, int64_t M, int r, int rpad, void* hi, void* lo, int num_sms,
                               cudaStream_t stream) {
-  k_split_hilo<<<grid_for(M * rpad, num_sms), 256, 0, stream>>>(T, M, r, rpad, static_cast<__nv_bfloat16*>(hi),
-                                                                  static_cast<__nv_bfloat16*>(lo));
-  return cudaGetLastError();
+  return launch_pdl(k_split_hilo, dim3(grid_for(M * rpad, num_sms)), dim3(256), 0, stream, T, M, r, rpad,
+                    static_cast<__nv_bfloat16*>(hi), static_cast<__nv_bfloat16*>(lo));
 }
 
 cudaError_t launch_lora_finish(const float* P, int splits, int64_t M, int r, int rpad, float s, float* f32,
                                void* s_bf16, void* hi, void* lo, int num_sms, cudaStream_t stream) {
-  k_lora_finish<<<grid_for(M * rpad / 2, num_sms), 256, 0, stream>>>(
-      P, splits, M, r, rpad, s, f32, static_cast<__nv_bfloat16*>(s_bf16), static_cast<__nv_bfloat16*>(hi),
-      static_cast<__nv_bfloat16*>(lo));
-  return cudaGetLastError();
+  return launch_pdl(k_lora_finish, dim3(grid_for(M * rpad / 2, num_sms)), dim3(256), 0, stream, P, splits, M, r,
+                    rpad, s, f32, static_cast<__nv_bfloat16*>(s_bf16), static_cast<__nv_bfloat16*>(hi),
+                    static_cast<__nv_bfloat16*>(lo));
 }
 
 cudaError_t launch_grad_reduce(const float* P, int splits, int64_t R, int rpad, int r, float s, bool transpose,
                                void* out, int num_sms, cudaStream_t stream) {
-  k_grad_reduce<<<grid_for(R * r, num_sms), 256, 0, stream>>>(P, splits, R, rpad, r, s, transpose ? 1 : 0,
-                                                               static_cast<__nv_bfloat16*>(out));
-  return cudaGetLastError();
+  const dim3 grid(static_cast<unsigned>((R + 31) / 32), static_cast<unsigned>(rpad / 64));
+  return launch_pdl(k_grad_reduce, grid, dim3(256), 0, stream, P, splits, R, rpad, r, s, transpose ? 1 : 0,
+                    static_cast<__nv_bfloat16*>(out));
 }
 
 cudaError_t launch_zero_bf16(void* p, int64_t n, int num_sms, cudaStream_t stream) {
   if (n <= 0) return cudaSuccess;
-  k_zero_bf16<<<grid_for(n, num_sms), 256, 0, stream>>>(static_cast<__nv_bfloat16*>(p), n);
-  return cudaGetLastError();
+  return launch_pdl(k_zero_bf16, dim3(grid_for(n, num_sms)), dim3(256), 0, stream, static_cast<__nv_bfloat16*>(p),
+                    n);
 }
 
 }  // namespace qlora

@@ -28,6 +28,7 @@ constexpr int kPass1Threads = 256;
 constexpr int kPass1Unroll = 4;
 
 __global__ void k_quant_zero(unsigned long long* bins) {
+  pdl_enter();
   const int i = threadIdx.x;
   if (i < kQuantBinWords) bins[i] = 0ull;
 }
@@ -140,19 +141,23 @@ __device__ __forceinline__ void quant_item(const uint4 d, bool valid, int lane, 
       for (int i = 0; i < 8; ++i) w[i] *= sc;
     }
     const float r = __frcp_rn(ms);
+    const f32x2 r2{r, r}, nms2{-ms, -ms}, S2{kBinScale, kBinScale}, three2{3.0f, 3.0f};
     word = 0u;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const float wi = w[i];
-      // v = RN(w / m): q0 = RN(w * RN(1/m)) is within one ulp, the remainder
-      // w - q0 m is exact, and one correction step rounds correctly (Markstein).
-      const float q0 = __fmul_rn(wi, r);
-      const float res = __fmaf_rn(-q0, ms, wi);
-      const float v = __fmaf_rn(res, r, q0);
-      const float x = __fmaf_rn(v, kBinScale, 3.0f);
-      const uint2 e = s_bins[(__float_as_uint(x) >> (23 - kBinBits)) & (kBins - 1)];
-      const uint32_t code = e.y + (v >= __uint_as_float(e.x) ? 1u : 0u);
-      word |= code << (4 * i);
+    for (int i = 0; i < 8; i += 2) {
+      // v = RN(w / m), two elements per packed instruction: q0 = RN(w * RN(1/m))
+      // is within one ulp, the remainder w - q0 m is exact, and one correction
+      // step rounds correctly (Markstein).
+      const f32x2 wi{w[i], w[i + 1]};
+      const f32x2 q0 = mul_f32x2(wi, r2);
+      const f32x2 res = fma_f32x2(q0, nms2, wi);
+      const f32x2 v = fma_f32x2(res, r2, q0);
+      const f32x2 x = fma_f32x2(v, S2, three2);
+      const uint2 e0 = s_bins[(__float_as_uint(x.x) >> (23 - kBinBits)) & (kBins - 1)];
+      const uint2 e1 = s_bins[(__float_as_uint(x.y) >> (23 - kBinBits)) & (kBins - 1)];
+      const uint32_t c0 = e0.y + (v.x >= __uint_as_float(e0.x) ? 1u : 0u);
+      const uint32_t c1 = e1.y + (v.y >= __uint_as_float(e1.x) ? 1u : 0u);
+      word |= (c0 | (c1 << 4)) << (4 * i);
     }
   }
   packed[item] = word;
@@ -171,6 +176,7 @@ k_quant_pass1(const uint4* __restrict__ W, int64_t n_items, uint32_t* __restrict
   if (tid < kBins) s_bins[tid] = make_uint2(__float_as_uint(tab.bins[tid].threshold), tab.bins[tid].j);
   s_hist[tid] = 0u;
   __syncthreads();
+  pdl_enter();
 
   const int64_t stride = static_cast<int64_t>(gridDim.x) * kPass1Threads;
   for (int64_t base = static_cast<int64_t>(blockIdx.x) * kPass1Threads + tid; base - tid < n_items;
@@ -211,6 +217,7 @@ k_quant_pass1(const uint4* __restrict__ W, int64_t n_items, uint32_t* __restrict
 __global__ void __launch_bounds__(256)
 k_dq_quantize(const float* __restrict__ absmax, int64_t nblk, const float* __restrict__ mean,
               int8_t* __restrict__ q, float* __restrict__ dq_scale, int64_t ngrp) {
+  pdl_enter();
   const int lane = threadIdx.x & 31;
   const int64_t g = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
   if (g >= ngrp) return;  // whole warp leaves together
@@ -274,7 +281,8 @@ cudaError_t launch_quantize(const void* W, int64_t numel, uint8_t* packed, int8_
   const int64_t nblk = numel / 64;
   const int64_t ngrp = (nblk + 255) / 256;
 
-  k_quant_zero<<<1, 320, 0, stream>>>(bins);
+  cudaError_t e = launch_pdl(k_quant_zero, dim3(1), dim3(320), 0, stream, bins);
+  if (e != cudaSuccess) return e;
   int64_t want = (n_items + kPass1Threads * kPass1Unroll - 1) / (kPass1Threads * kPass1Unroll);
   int64_t cap = static_cast<int64_t>(num_sms) * 8;
   int64_t g = want < cap ? (want > 0 ? want : 1) : cap;
@@ -282,12 +290,12 @@ cudaError_t launch_quantize(const void* W, int64_t numel, uint8_t* packed, int8_
   const int64_t min_grid = (nblk + (int64_t(1) << 24) - 1) >> 24;
   if (g < min_grid) g = min_grid;
   const int grid = static_cast<int>(g);
-  k_quant_pass1<<<grid, kPass1Threads, 0, stream>>>(reinterpret_cast<const uint4*>(W), n_items,
-                                                    reinterpret_cast<uint32_t*>(packed), absmax_scratch, bins,
-                                                    mean, nblk, tab);
+  e = launch_pdl(k_quant_pass1, dim3(grid), dim3(kPass1Threads), 0, stream, reinterpret_cast<const uint4*>(W),
+                 n_items, reinterpret_cast<uint32_t*>(packed), absmax_scratch, bins, mean, nblk, tab);
+  if (e != cudaSuccess) return e;
   const int dq_grid = static_cast<int>((ngrp + 7) / 8);
-  k_dq_quantize<<<dq_grid, 256, 0, stream>>>(absmax_scratch, nblk, mean, absmax_q, dq_scale, ngrp);
-  return cudaGetLastError();
+  return launch_pdl(k_dq_quantize, dim3(dq_grid), dim3(256), 0, stream, static_cast<const float*>(absmax_scratch),
+                    nblk, static_cast<const float*>(mean), absmax_q, dq_scale, ngrp);
 }
 
 }  // namespace qlora
