@@ -38,6 +38,23 @@ METRIC = "fused NF4+LoRA linear TFLOP/s (M=4096) and weight GB/s (M=1..16) vs ro
 R, ALPHA, M_TRAIN, M_DECODE = 64, 16.0, 4096, (1, 4, 16)
 SHAPES = syn.LLAMA7B_SHAPES
 
+# DRAM traffic of the roofline call (qlora_linear_fwd, M=4096, 11008x4096: dequant,
+# LoRA-down GEMM, finish, 2-CTA GEMM) summed from one ncu capture of
+# `bench.py --profile-case` (dram__bytes_read.sum + dram__bytes_write.sum per
+# launch, see profiles/). Valid only for the kernel sources it was taken on.
+ROOFLINE_SHAPE = (11008, 4096)
+TRAFFIC_RECORD = {"fingerprint": "ff0eae1bb5b3545b", "bytes": 315.7e6}  # profiles/k_tc_gemm2_*, lora_*, k_dequant_*
+TRAFFIC_SOURCES = ("common.cuh", "nf4_lut.cuh", "dequant.cu", "gemm_tc.cu", "lora_misc.cu", "api.cu")
+
+
+def source_fingerprint():
+    import hashlib
+    h = hashlib.sha1()
+    for f in TRAFFIC_SOURCES:
+        h.update(open(os.path.join(ROOT, "bit_nf4_quantized_absmax_b200", "csrc", f), "rb").read())
+    return h.hexdigest()[:16]
+
+
 # kernels each C-ABI call launches on these shapes (see the launchers in csrc/)
 LAUNCHES = {"quantize": 3, "dequantize": 1, "decode_fwd": 2, "train_fwd": 4, "train_bwd": 9}
 
@@ -303,16 +320,19 @@ def run_ours(args, rank, world, dev):
             e["TFLOP_s"] = round(f / us / 1e6, 1)
         parts[f"{kind}/{N}x{K}"] = e
 
-    # dominant kernel: the forward at M = 4096 (one dequant, one LoRA-down and the
-    # tcgen05 GEMM with the LoRA slab); its flops over its measured duration.
-    fwd_us = [1e3 * statistics.mean(a.elapsed_time(b) for a, b in ev[f"train_fwd/{li}"]) for li in range(3)]
-    fwd_fl = [train_flops(N, K)[0] for N, K in SHAPES]
-    achieved = sum(fwd_fl) / sum(fwd_us) / 1e6
-    roof = {"kernel": "qlora_linear_fwd M=4096 (dequant + LoRA-down + tcgen05 GEMM), 7B shapes",
+    # dominant call: the training forward (M = 4096) on the 11008x4096 linear, i.e.
+    # one dequant, the LoRA-down GEMM + finish and the 2-CTA tcgen05 GEMM with the
+    # LoRA slab; algorithmic flops over its measured duration (events on the stream).
+    li = SHAPES.index(ROOFLINE_SHAPE)
+    fwd_us = 1e3 * statistics.mean(a.elapsed_time(b) for a, b in ev[f"train_fwd/{li}"])
+    achieved = train_flops(*ROOFLINE_SHAPE)[0] / fwd_us / 1e6
+    traffic = TRAFFIC_RECORD["bytes"] if TRAFFIC_RECORD["fingerprint"] == source_fingerprint() else None
+    roof = {"kernel": "qlora_linear_fwd M=4096 on 11008x4096 (dequant, LoRA-down, 2-CTA tcgen05 GEMM)",
             "bound": "tensor", "achieved": round(achieved, 1), "peak": peaks["bf16_tflops_sustained"],
             "peak_kind": f"bf16 dense sustained ({peaks['source']})", "unit": "TFLOP/s",
             "frac": round(achieved / peaks["bf16_tflops_sustained"], 4),
-            "frac_of_burst": round(achieved / peaks["bf16_tflops"], 4), "traffic": None}
+            "frac_of_burst": round(achieved / peaks["bf16_tflops"], 4), "traffic": traffic,
+            "us_per_launch": round(fwd_us, 2)}
     dec = [parts[f"decode{M}/{N}x{K}"]["weight_GB_s"] for M in M_DECODE for N, K in SHAPES]
 
     # end to end through the C ABI with host buffers
