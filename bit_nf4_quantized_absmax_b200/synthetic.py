@@ -106,6 +106,47 @@ def make_linear(N: int, K: int, M: int, r: int = 64, alpha: float = 16.0, *, see
     return LinearInputs(W, A, B, X, dY, r, alpha)
 
 
+def _gen_cuda(seed: int, workload: str, tensor_id: int, device) -> torch.Generator:
+    g = torch.Generator(device=device)
+    g.manual_seed(tensor_seed(seed, workload, tensor_id))
+    return g
+
+
+def normal_bf16_device(shape, std: float, seed: int, workload: str, tensor_id: int, device="cuda",
+                       out: torch.Tensor | None = None) -> torch.Tensor:
+    """N(0, std) drawn on the device by torch's seeded (Philox) CUDA generator,
+    rounded to bf16. Used where the workload is too large to draw on the host
+    (the whole-model sweep); the values are reproducible for a given seed."""
+    g = _gen_cuda(seed, workload, tensor_id, device)
+    t = torch.randn(*shape, generator=g, dtype=torch.float32, device=device)
+    t.mul_(std)
+    if out is None:
+        return t.to(torch.bfloat16)
+    out.copy_(t)
+    return out
+
+
+def student_t_bf16_device(shape, nu: int, std: float, seed: int, workload: str, tensor_id: int,
+                          device="cuda") -> torch.Tensor:
+    """Student-t(nu) on the device (same definition as student_t_bf16), bf16."""
+    assert nu > 2 and int(nu) == nu
+    g = _gen_cuda(seed, workload, tensor_id, device)
+    z = torch.randn(*shape, generator=g, dtype=torch.float32, device=device)
+    v = torch.zeros(*shape, dtype=torch.float32, device=device)
+    for _ in range(int(nu)):
+        e = torch.randn(*shape, generator=g, dtype=torch.float32, device=device)
+        v.addcmul_(e, e)
+    t = z / torch.sqrt(v / nu)
+    t.mul_(std / math.sqrt(nu / (nu - 2.0)))
+    return t.to(torch.bfloat16)
+
+
+# Per-layer linear shapes (out x in) of Llama-65B: q, k, v, o, gate, up, down.
+LLAMA65B_LAYER = ((8192, 8192), (8192, 8192), (8192, 8192), (8192, 8192), (22016, 8192), (22016, 8192),
+                  (8192, 22016))
+LLAMA65B_LAYERS = 80
+
+
 def single_linear(seed: int = 0) -> LinearInputs:
     """The 1024x1024 single-linear workload (r=16, alpha=16, dY ~ N(0,1))."""
     return make_linear(1024, 1024, 16, r=16, alpha=16.0, seed=seed, workload="single", dy_std=1.0)
