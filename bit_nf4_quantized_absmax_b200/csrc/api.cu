@@ -203,12 +203,12 @@ qlora_status qlora_linear_fwd(const qlora_nf4_weight* q, const void* X, int64_t 
   // workspace layout
   Layout L;
   size_t off_T = 0, off_part = 0, off_cnt = 0, off_wd = 0, off_sT = 0;
-  int ksplit = 1;
+  DecodePlan dplan{};
   if (decode) {
-    ksplit = decode_ksplit(N, K, di.num_sms);
+    dplan = decode_plan(M, N, K, kRefSms);
     off_T = L.add(T_save ? 0 : static_cast<size_t>(M) * r * sizeof(float));
-    off_part = L.add(decode_partial_elems(M, N, ksplit) * sizeof(float));
-    off_cnt = L.add(decode_counter_words(N) * sizeof(unsigned int));
+    off_part = L.add(decode_partial_elems(dplan) * sizeof(float));
+    off_cnt = L.add(decode_counter_words(dplan) * sizeof(unsigned int));
   } else {
     off_wd = L.add(static_cast<size_t>(N) * K * 2);
     off_sT = L.add(static_cast<size_t>(M) * rpad * 2);
@@ -226,7 +226,7 @@ qlora_status qlora_linear_fwd(const qlora_nf4_weight* q, const void* X, int64_t 
     float* T = T_save ? T_save : reinterpret_cast<float*>(ws + off_T);
     Nf4View w{q->packed, q->absmax_q, q->dq_scale, q->mean, N, K};
     return cuda_status(launch_decode_fwd(w, X, M, A, B, r, s, Y, T, reinterpret_cast<float*>(ws + off_part),
-                                         reinterpret_cast<unsigned int*>(ws + off_cnt), ksplit, cb, cs));
+                                         reinterpret_cast<unsigned int*>(ws + off_cnt), dplan, cb, cs));
   }
   void* Wd = ws + off_wd;
   void* sT = ws + off_sT;

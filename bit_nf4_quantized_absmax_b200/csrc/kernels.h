@@ -41,14 +41,25 @@ struct Nf4View {
 };
 
 // ---- decode.cu: M <= 16 forward ----
-int decode_ksplit(int64_t N, int64_t K, int num_sms);
-size_t decode_partial_elems(int64_t M, int64_t N, int ksplit);
-size_t decode_counter_words(int64_t N);
-// T [M, r] fp32 receives X A^T; partial [ksplit, M, N] fp32 and counters
-// [decode_counter_words(N)] are scratch.
+// Work split of the decode kernel: (16-row tile, 256-wide K superblock) items
+// cut into equal per-warp ranges; fixed by (M, N, K) and a reference SM count.
+struct DecodePlan {
+  int mt;             // token tiles of 8 (1: M <= 8, 2: M <= 16)
+  int64_t row_tiles;  // ceil(N / 16)
+  int64_t nsb;        // ceil(K / 256)
+  int64_t n_items;    // row_tiles * nsb
+  int grid;           // CTAs of 8 warps (the last one may be partly idle)
+  int64_t n_warps;    // working warps: min(n_items, 8 * CTA capacity)
+  int max_seg;        // most warps sharing one row tile
+};
+DecodePlan decode_plan(int64_t M, int64_t N, int64_t K, int ref_sms);
+size_t decode_partial_elems(const DecodePlan& p);
+size_t decode_counter_words(const DecodePlan& p);
+// T [M, r] fp32 receives X A^T; partial [decode_partial_elems] fp32 and
+// counters [decode_counter_words] are scratch.
 cudaError_t launch_decode_fwd(const Nf4View& w, const void* X, int64_t M, const void* A, const void* B, int r,
-                              float s, void* Y, float* T, float* partial, unsigned int* counters, int ksplit,
-                              const float codebook[16], cudaStream_t stream);
+                              float s, void* Y, float* T, float* partial, unsigned int* counters,
+                              const DecodePlan& p, const float codebook[16], cudaStream_t stream);
 
 // ---- gemm_tc.cu: tcgen05 GEMMs ----
 cudaError_t launch_gemm_fwd(const void* X, const void* Wd, const void* sT, const void* Bl, int64_t M, int64_t N,
