@@ -226,7 +226,7 @@ qlora_status qlora_linear_fwd(const qlora_nf4_weight* q, const void* X, int64_t 
     float* T = T_save ? T_save : reinterpret_cast<float*>(ws + off_T);
     Nf4View w{q->packed, q->absmax_q, q->dq_scale, q->mean, N, K};
     return cuda_status(launch_decode_fwd(w, X, M, A, B, r, s, Y, T, reinterpret_cast<float*>(ws + off_part),
-                                         reinterpret_cast<unsigned int*>(ws + off_cnt), dplan, cb, cs));
+                                         reinterpret_cast<unsigned int*>(ws + off_cnt), dplan, cb, err, cs));
   }
   void* Wd = ws + off_wd;
   void* sT = ws + off_sT;

@@ -21,15 +21,17 @@
 // in slot order, adds the LoRA term s (T B^T) with a bf16 hi/lo split of T on
 // the tensor cores, and writes Y. The result depends only on the shapes, not on
 // timing.
+#include <cuda.h>
+
 #include "common.cuh"
 #include "kernels.h"
 #include "nf4_lut.cuh"
+#include "tensor_map.h"
 
 namespace qlora {
 namespace {
 
 constexpr int kDecodeWarps = 8;
-constexpr int kDecodeCtasPerSm = 2;
 
 __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                          uint32_t b0, uint32_t b1) {
@@ -45,51 +47,6 @@ __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1
 __device__ __forceinline__ uint32_t hi16(uint32_t x) { return __umulhi(x, 0x10000u); }
 __device__ __forceinline__ uint32_t shr1(uint32_t x) { return __umulhi(x, 0x80000000u); }
 
-// One lane's 64 codes of a row block and the block's double-quant code and scale.
-struct RowBlock {
-  uint32_t w[8];
-  int qv;
-  float sc;
-};
-
-template <bool V8>
-__device__ __forceinline__ void load_row_block(RowBlock& rb, const uint8_t* __restrict__ packed,
-                                               const int8_t* __restrict__ q, const float* __restrict__ dqs,
-                                               int64_t blk, bool valid) {
-  if (valid) {
-    const uint4* p = reinterpret_cast<const uint4*>(packed + blk * 32);
-    if (V8) {
-      ld_global_cs_v8(p, rb.w);
-    } else {
-      const uint4 a = __ldcs(p), b = __ldcs(p + 1);
-      rb.w[0] = a.x; rb.w[1] = a.y; rb.w[2] = a.z; rb.w[3] = a.w;
-      rb.w[4] = b.x; rb.w[5] = b.y; rb.w[6] = b.z; rb.w[7] = b.w;
-    }
-    rb.qv = static_cast<int>(__ldg(q + blk));
-    rb.sc = __ldg(dqs + (blk >> 8));
-  } else {  // outside the matrix: zero codes (weight 0)
-#pragma unroll
-    for (int i = 0; i < 8; ++i) rb.w[i] = 0x77777777u;
-    rb.qv = 0;
-    rb.sc = 0.0f;
-  }
-}
-
-// 16 tokens' values (k = 16 j .. 16 j + 15 of one block) for one token row.
-template <bool V8>
-__device__ __forceinline__ void load_x16(uint32_t (&x)[8], const __nv_bfloat16* __restrict__ p, bool valid) {
-  if (!valid) {
-#pragma unroll
-    for (int i = 0; i < 8; ++i) x[i] = 0u;
-  } else if (V8) {
-    ld_global_nc_v8(p, x);
-  } else {
-    const uint4 a = __ldg(reinterpret_cast<const uint4*>(p)), b = __ldg(reinterpret_cast<const uint4*>(p) + 1);
-    x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
-    x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
-  }
-}
-
 // Byte-permute lookup of four codes with precomputed selectors: `s` holds the
 // low three bits of each code (nibbles 0..3), `sel` picks the table half by
 // bit 3. Returns the bf16 pairs for codes (0, 1) and (2, 3).
@@ -101,186 +58,296 @@ __device__ __forceinline__ void lookup4_sel(const Nf4Lut& L, uint32_t s, uint32_
   o23 = prmt(lo, hi, 0x7362);
 }
 
-// Owner warp of item i when n_items items are cut into n_warps ranges
-// [w * n_items / n_warps, (w + 1) * n_items / n_warps).
-__host__ __device__ __forceinline__ int64_t item_owner(int64_t i, int64_t n_items, int64_t n_warps) {
-  return ((i + 1) * n_warps - 1) / n_items;
+// Owner unit of item i when n_items items are cut into n_units ranges
+// [u * n_items / n_units, (u + 1) * n_items / n_units).
+__host__ __device__ __forceinline__ int64_t item_owner(int64_t i, int64_t n_items, int64_t n_units) {
+  return ((i + 1) * n_units - 1) / n_items;
 }
 
-template <int MT, bool V8>
-__global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeCtasPerSm)
-k_decode(const uint8_t* __restrict__ packed, const int8_t* __restrict__ q, const float* __restrict__ dqs,
-         const float* __restrict__ mean, const __nv_bfloat16* __restrict__ X, int M, int64_t N, int64_t K,
-         const float* __restrict__ T, const __nv_bfloat16* __restrict__ Bl, int r, float s,
-         __nv_bfloat16* __restrict__ Y, float* __restrict__ partial, unsigned int* __restrict__ counters,
-         int64_t n_items, int64_t n_warps, int max_seg, const __grid_constant__ Nf4Codebook cb) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+// Ticket of a split tile: release this warp's partial sums, acquire the others'.
+__device__ __forceinline__ unsigned int atom_add_acq_rel_gpu(unsigned int* p, unsigned int v) {
+  unsigned int old;
+  asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+
+// End of a work unit's piece of 16-row tile `tile` (item row `item_row` of the
+// unit ranges): store the warp's fp32 partial sums in the tile's slot; the warp that brings the tile's last piece (ticket counter, no
+// waiting) sums the slots in slot order, adds s (T B^T) computed on the tensor
+// cores with T split into bf16 hi + lo, and writes Y.
+template <int MT>
+__device__ __forceinline__ void publish_segment(const float (&acc)[2][MT][4], int64_t item_row, int64_t tile,
+                                                int64_t unit, int lane, int64_t nsb, int64_t n_items,
+                                                int64_t n_units, int max_seg,
+                                                float* __restrict__ partial, unsigned int* __restrict__ counters,
+                                                const float* __restrict__ T, const __nv_bfloat16* __restrict__ Bl,
+                                                int r, float s, __nv_bfloat16* __restrict__ Y, int M, int64_t N) {
   const int g = lane >> 2, t = lane & 3;
-  const int64_t gw = static_cast<int64_t>(blockIdx.x) * kDecodeWarps + warp;
-  if (gw >= n_warps) return;
-  const int64_t i_begin = gw * n_items / n_warps;
-  const int64_t i_end = (gw + 1) * n_items / n_warps;
-  if (i_begin >= i_end) return;
+  const int64_t w_first = item_owner(item_row * nsb, n_items, n_units);
+  const int64_t w_last = item_owner((item_row + 1) * nsb - 1, n_items, n_units);
+  const int nseg = static_cast<int>(w_last - w_first + 1);
+  const int slot = static_cast<int>(unit - w_first);
+  float* tile_part = partial + static_cast<int64_t>(tile) * max_seg * (32 * 4 * MT);
+#pragma unroll
+  for (int m = 0; m < MT; ++m) {
+    const float4 v = make_float4(acc[0][m][0] + acc[1][m][0], acc[0][m][1] + acc[1][m][1],
+                                 acc[0][m][2] + acc[1][m][2], acc[0][m][3] + acc[1][m][3]);
+    __stcg(reinterpret_cast<float4*>(tile_part + (slot * 32 + lane) * 4 * MT) + m, v);
+  }
+  __syncwarp();  // the lanes' partial stores are ordered before lane 0's release below
+  if (nseg > 1) {
+    unsigned int ticket = 0;
+    if (lane == 0) ticket = atom_add_acq_rel_gpu(&counters[tile], 1u);
+    ticket = __shfl_sync(0xffffffffu, ticket, 0);
+    if (ticket != static_cast<unsigned int>(nseg - 1)) return;  // another warp completes the tile
+    __syncwarp();  // lane 0's acquire is ordered before every lane's reads of the slots
+  }
 
-  const int64_t nkb_row = K / 64;
-  const int64_t nsb = (nkb_row + 3) / 4;
-  const float mu = *mean;
-  bool entered = false;  // waited for the LoRA-down kernel (T, zeroed counters)
-
-  // item -> (rows, block) of this lane
-  auto row_blocks = [&](int64_t item, RowBlock& ra, RowBlock& rb) {
-    const int64_t tile = item / nsb;
-    const int64_t kb = (item - tile * nsb) * 4 + t;
-    const int64_t na = tile * 16 + g, nb = na + 8;
-    const bool kv = kb < nkb_row;
-    load_row_block<V8>(ra, packed, q, dqs, na * nkb_row + kb, kv && na < N);
-    load_row_block<V8>(rb, packed, q, dqs, nb * nkb_row + kb, kv && nb < N);
-  };
-  // token values of group j (k = 16 j .. 16 j + 15 of the lane's block) of an item
-  auto x_group = [&](int64_t item, int j, uint32_t (&x)[MT][8]) {
-    const int64_t kb = (item % nsb) * 4 + t;
-    const bool kv = kb < nkb_row;
+  float y[MT][4];
+#pragma unroll
+  for (int m = 0; m < MT; ++m) y[m][0] = y[m][1] = y[m][2] = y[m][3] = 0.0f;
+  for (int sl = 0; sl < nseg; ++sl) {
+#pragma unroll
+    for (int m = 0; m < MT; ++m) {
+      const float4 v = __ldcg(reinterpret_cast<const float4*>(tile_part + (sl * 32 + lane) * 4 * MT) + m);
+      y[m][0] += v.x; y[m][1] += v.y; y[m][2] += v.z; y[m][3] += v.w;
+    }
+  }
+  // LoRA up: rows of B are the A operand, T^T (split into bf16 hi + lo) the B operand.
+  const int64_t na = tile * 16 + g, nb = na + 8;
+  float l[MT][4];
+#pragma unroll
+  for (int m = 0; m < MT; ++m) l[m][0] = l[m][1] = l[m][2] = l[m][3] = 0.0f;
+  for (int j0 = 0; j0 < r; j0 += 16) {
+    const uint32_t b_a0 = na < N ? *reinterpret_cast<const uint32_t*>(Bl + na * r + j0 + 2 * t) : 0u;
+    const uint32_t b_a2 = na < N ? *reinterpret_cast<const uint32_t*>(Bl + na * r + j0 + 2 * t + 8) : 0u;
+    const uint32_t b_a1 = nb < N ? *reinterpret_cast<const uint32_t*>(Bl + nb * r + j0 + 2 * t) : 0u;
+    const uint32_t b_a3 = nb < N ? *reinterpret_cast<const uint32_t*>(Bl + nb * r + j0 + 2 * t + 8) : 0u;
 #pragma unroll
     for (int m = 0; m < MT; ++m) {
       const int tok = g + 8 * m;
-      load_x16<V8>(x[m], X + static_cast<int64_t>(tok) * K + kb * 64 + 16 * j, kv && tok < M);
+      float tv[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+      if (tok < M) {
+        const float* tp = T + static_cast<int64_t>(tok) * r + j0 + 2 * t;
+        tv[0] = __ldcg(tp);
+        tv[1] = __ldcg(tp + 1);
+        tv[2] = __ldcg(tp + 8);
+        tv[3] = __ldcg(tp + 9);
+      }
+      uint32_t hi[2], lo[2];
+#pragma unroll
+      for (int p = 0; p < 2; ++p) {
+        const uint32_t h = pack_bf16x2(tv[2 * p], tv[2 * p + 1]);
+        hi[p] = h;
+        lo[p] = pack_bf16x2(tv[2 * p] - bf16lo_to_f32(h), tv[2 * p + 1] - bf16hi_to_f32(h));
+      }
+      mma16816(l[m], b_a0, b_a1, b_a2, b_a3, hi[0], hi[1]);
+      mma16816(l[m], b_a0, b_a1, b_a2, b_a3, lo[0], lo[1]);
     }
+  }
+#pragma unroll
+  for (int m = 0; m < MT; ++m) {
+    const int tok0 = 8 * m + 2 * t, tok1 = tok0 + 1;
+    if (na < N) {
+      if (tok0 < M) Y[static_cast<int64_t>(tok0) * N + na] = __float2bfloat16_rn(fmaf(s, l[m][0], y[m][0]));
+      if (tok1 < M) Y[static_cast<int64_t>(tok1) * N + na] = __float2bfloat16_rn(fmaf(s, l[m][1], y[m][1]));
+    }
+    if (nb < N) {
+      if (tok0 < M) Y[static_cast<int64_t>(tok0) * N + nb] = __float2bfloat16_rn(fmaf(s, l[m][2], y[m][2]));
+      if (tok1 < M) Y[static_cast<int64_t>(tok1) * N + nb] = __float2bfloat16_rn(fmaf(s, l[m][3], y[m][3]));
+    }
+  }
+}
+
+// CTA items are (128-row group, 256-wide K superblock) pairs in group-major
+// order; each CTA takes one contiguous, equally sized range of items. Warp w of
+// the 8 consumer warps decodes rows 16 w .. 16 w + 15 of the group. A ninth warp
+// feeds a kStages-deep ring by TMA: per stage one box of the packed weights
+// (128 rows x 128 bytes) and four boxes of the token values (64 k x 8 MT rows,
+// one per 64-weight block of the superblock), all with the 128-byte swizzle so
+// that the lanes' 16-byte reads are free of bank conflicts.
+constexpr int kStages = 4;
+constexpr int kRowsPerItem = kDecodeWarps * 16;
+constexpr int kWBytes = kRowsPerItem * 128;
+
+__host__ __device__ constexpr int decode_x_bytes(int mt) { return 4 * 8 * mt * 128; }
+__host__ __device__ constexpr int decode_stage_bytes(int mt) { return kWBytes + decode_x_bytes(mt); }
+__host__ __device__ constexpr int decode_smem_bytes(int mt) { return kStages * decode_stage_bytes(mt) + 1024; }
+constexpr int kDecodeCtasPerSm = 2;
+
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+  return v;
+}
+
+template <int MT>
+__global__ void __launch_bounds__((kDecodeWarps + 1) * 32, kDecodeCtasPerSm)
+k_decode(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
+         const int8_t* __restrict__ q, const float* __restrict__ dqs, const float* __restrict__ mean, int M,
+         int64_t N, int64_t K, const float* __restrict__ T, const __nv_bfloat16* __restrict__ Bl, int r, float s,
+         __nv_bfloat16* __restrict__ Y, float* __restrict__ partial, unsigned int* __restrict__ counters,
+         int64_t n_items, int64_t n_ctas, int max_seg, int32_t* __restrict__ err,
+         const __grid_constant__ Nf4Codebook cb) {
+  constexpr int kStage = decode_stage_bytes(MT);
+  extern __shared__ uint8_t dsm_raw[];
+  __shared__ __align__(8) uint64_t full[kStages];
+  __shared__ __align__(8) uint64_t empty[kStages];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t cta = blockIdx.x;
+  const int64_t i_begin = cta * n_items / n_ctas;
+  const int64_t i_end = (cta + 1) * n_items / n_ctas;
+  const int n_my = static_cast<int>(i_end - i_begin);
+  const int nkb_row = static_cast<int>(K / 64);
+  const int nsb = (nkb_row + 3) / 4;
+  const int64_t rg0 = i_begin / nsb;  // (row group, superblock) of the first item
+  const int sb0 = static_cast<int>(i_begin - rg0 * nsb);
+  uint8_t* dsm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~uintptr_t(1023));
+
+  if (threadIdx.x == 0) {
+#pragma unroll
+    for (int st = 0; st < kStages; ++st) {
+      mbar_init(&full[st], 1);
+      mbar_init(&empty[st], kDecodeWarps);
+    }
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (n_my <= 0) return;
+
+  if (warp == kDecodeWarps) {  // ---- producer warp: TMA ring ----
+    if (lane == 0) {
+      prefetch_tmap(&tm_w);
+      prefetch_tmap(&tm_x);
+      int64_t rg = rg0;
+      int sb = sb0, st = 0;
+      uint32_t ph = 0;
+      for (int n = 0; n < n_my; ++n) {
+        if (n >= kStages && !mbar_wait_bounded(&empty[st], ph ^ 1u, err, DEV_TIMEOUT_SMEM_EMPTY)) break;
+        uint8_t* dst = dsm + st * kStage;
+        mbar_arrive_expect_tx(&full[st], kStage);
+        tma_load_2d(dst, &tm_w, &full[st], sb * 128, static_cast<int32_t>(rg * kRowsPerItem));
+#pragma unroll
+        for (int b = 0; b < 4; ++b)
+          tma_load_2d(dst + kWBytes + b * (8 * MT * 128), &tm_x, &full[st], sb * 256 + 64 * b, 0);
+        if (++st == kStages) {
+          st = 0;
+          ph ^= 1u;
+        }
+        if (++sb == nsb) {
+          sb = 0;
+          ++rg;
+        }
+      }
+    }
+    grid_dependency_launch_dependents();
+    return;
+  }
+  // ---- consumer warps ----
+  const int g = lane >> 2, t = lane & 3;
+  const uint32_t smem0 = smem_u32(dsm);
+  // the lane's weight chunks (2t + c) of rows 16 w + g and 16 w + g + 8, and the
+  // token rows g + 8 m of its block's token box, under the 128-byte swizzle
+  const uint32_t offW0 = (warp * 16 + g) * 128 + (((2 * t) ^ g) << 4);
+  const uint32_t offW1 = (warp * 16 + g) * 128 + (((2 * t + 1) ^ g) << 4);
+  const uint32_t offX = kWBytes + t * (8 * MT * 128) + g * 128;
+
+  const float mu = *mean;
+  // block constants of rows 16 w + g and + 8 (m' = 0 outside the matrix)
+  auto consts = [&](int64_t rg, int sb, int& qa, float& sa, int& qb, float& sbv, bool& va, bool& vb) {
+    const int kb = sb * 4 + t;
+    const int64_t na = rg * kRowsPerItem + warp * 16 + g, nb = na + 8;
+    va = kb < nkb_row && na < N;
+    vb = kb < nkb_row && nb < N;
+    const int64_t ba = na * nkb_row + kb, bb = nb * nkb_row + kb;
+    qa = va ? static_cast<int>(__ldg(q + ba)) : 0;
+    sa = va ? __ldg(dqs + (ba >> 8)) : 0.0f;
+    qb = vb ? static_cast<int>(__ldg(q + bb)) : 0;
+    sbv = vb ? __ldg(dqs + (bb >> 8)) : 0.0f;
   };
 
-  RowBlock nA, nB;
-  uint32_t xn[MT][8];
-  row_blocks(i_begin, nA, nB);
-  x_group(i_begin, 0, xn);
+  int nqa, nqb;
+  float nsa, nsc;
+  bool nva, nvb;
+  consts(rg0, sb0, nqa, nsa, nqb, nsc, nva, nvb);
 
-  int64_t i = i_begin;
-  while (i < i_end) {
-    const int64_t tile = i / nsb;
-    const int64_t seg_end = min(i_end, (tile + 1) * nsb);
+  bool entered = false;  // waited for the LoRA-down kernel (T, zeroed counters)
+  bool ok = true;
+  int n = 0, stage = 0;
+  uint32_t phase = 0;
+  int64_t rg = rg0;
+  int sb = sb0;
+  while (n < n_my) {
+    const int seg_items = min(n_my - n, nsb - sb);  // items of this row group in the CTA's range
     float acc[2][MT][4];
 #pragma unroll
     for (int c = 0; c < 2; ++c)
 #pragma unroll
       for (int m = 0; m < MT; ++m) acc[c][m][0] = acc[c][m][1] = acc[c][m][2] = acc[c][m][3] = 0.0f;
 
-    for (; i < seg_end; ++i) {
-      const RowBlock cA = nA, cB = nB;
-      const bool more = i + 1 < i_end;
-      if (more) row_blocks(i + 1, nA, nB);  // next item's codes stream in while this one is decoded
-      const Nf4Lut la = make_nf4_lut(cb, __fmaf_rn(static_cast<float>(cA.qv), cA.sc, mu));
-      const Nf4Lut lb = make_nf4_lut(cb, __fmaf_rn(static_cast<float>(cB.qv), cB.sc, mu));
+    for (int e = 0; e < seg_items; ++e, ++n, ++sb) {
+      const float mA = nva ? __fmaf_rn(static_cast<float>(nqa), nsa, mu) : 0.0f;
+      const float mB = nvb ? __fmaf_rn(static_cast<float>(nqb), nsc, mu) : 0.0f;
+      if (n + 1 < n_my) {  // next item's constants
+        const bool wrap = sb + 1 == nsb;
+        consts(wrap ? rg + 1 : rg, wrap ? 0 : sb + 1, nqa, nsa, nqb, nsc, nva, nvb);
+      }
+      const Nf4Lut la = make_nf4_lut(cb, mA);
+      const Nf4Lut lb = make_nf4_lut(cb, mB);
+      const bool got = mbar_wait_bounded(&full[stage], phase, err, DEV_TIMEOUT_TMA_FULL);
+      if (!__all_sync(0xffffffffu, got)) {
+        ok = false;
+        break;
+      }
+      const uint32_t st = smem0 + static_cast<uint32_t>(stage) * kStage;
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        uint32_t xc[MT][8];
+      for (int c = 0; c < 2; ++c) {  // weight chunk c: words 4c .. 4c + 3 of the lane's block
+        const uint4 ca = lds128(st + (c ? offW1 : offW0));
+        const uint4 cbk = lds128(st + 8 * 128 + (c ? offW1 : offW0));
 #pragma unroll
-        for (int m = 0; m < MT; ++m)
+        for (int jj = 0; jj < 2; ++jj) {
+          const int j = 2 * c + jj;  // group: k = 16 j .. 16 j + 15 of the block
 #pragma unroll
-          for (int e = 0; e < 8; ++e) xc[m][e] = xn[m][e];
-        if (j < 3)
-          x_group(i, j + 1, xn);
-        else if (more)
-          x_group(i + 1, 0, xn);
+          for (int h = 0; h < 2; ++h) {  // word 2j + h holds k = 16 j + 8 h .. + 7
+            uint4 xv[MT];  // token values of k = 16 j + 8 h .. + 7: 16-byte chunk 2j + h of the box row
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {  // word 2j + h holds k = 16 j + 8 h .. + 7
-          const uint32_t wa = cA.w[2 * j + h], wb = cB.w[2 * j + h];
-          const uint32_t sa = wa & 0x77777777u, sb = wb & 0x77777777u;
-          const uint32_t ta = (shr1(wa) & 0x44444444u) | 0x32103210u;
-          const uint32_t tb = (shr1(wb) & 0x44444444u) | 0x32103210u;
+            for (int m = 0; m < MT; ++m)
+              xv[m] = lds128(st + offX + m * (8 * 128) + (((2 * j + h) ^ g) << 4));
+            const uint32_t wa = jj ? (h ? ca.w : ca.z) : (h ? ca.y : ca.x);
+            const uint32_t wb = jj ? (h ? cbk.w : cbk.z) : (h ? cbk.y : cbk.x);
+            const uint32_t sa = wa & 0x77777777u, sbw = wb & 0x77777777u;
+            const uint32_t ta = (shr1(wa) & 0x44444444u) | 0x32103210u;
+            const uint32_t tb = (shr1(wb) & 0x44444444u) | 0x32103210u;
 #pragma unroll
-          for (int half = 0; half < 2; ++half) {  // step st = 2 h + half: k = 16 j + 4 st .. + 3
-            const int st = 2 * h + half;
-            uint32_t a0, a1, a2, a3;
-            lookup4_sel(la, half ? hi16(sa) : sa, half ? hi16(ta) : ta, a0, a2);  // row g
-            lookup4_sel(lb, half ? hi16(sb) : sb, half ? hi16(tb) : tb, a1, a3);  // row g + 8
+            for (int half = 0; half < 2; ++half) {  // step 2 h + half: k = 16 j + 8 h + 4 half .. + 3
+              uint32_t a0, a1, a2, a3;
+              lookup4_sel(la, half ? hi16(sa) : sa, half ? hi16(ta) : ta, a0, a2);    // row g
+              lookup4_sel(lb, half ? hi16(sbw) : sbw, half ? hi16(tb) : tb, a1, a3);  // row g + 8
 #pragma unroll
-            for (int m = 0; m < MT; ++m) mma16816(acc[st & 1][m], a0, a1, a2, a3, xc[m][2 * st], xc[m][2 * st + 1]);
+              for (int m = 0; m < MT; ++m)
+                mma16816(acc[half][m], a0, a1, a2, a3, half ? xv[m].z : xv[m].x, half ? xv[m].w : xv[m].y);
+            }
           }
         }
       }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[stage]);  // this warp is done with the stage
+      if (++stage == kStages) {
+        stage = 0;
+        phase ^= 1u;
+      }
     }
-
-    // ---- segment done: publish the partial sums of this tile piece ----
+    if (!ok) break;
     if (!entered) {  // T and the zeroed counters come from the preceding LoRA-down kernel
       pdl_enter();
       entered = true;
     }
-    const int64_t w_first = item_owner(tile * nsb, n_items, n_warps);
-    const int64_t w_last = item_owner((tile + 1) * nsb - 1, n_items, n_warps);
-    const int nseg = static_cast<int>(w_last - w_first + 1);
-    const int slot = static_cast<int>(gw - w_first);
-    float* tile_part = partial + static_cast<int64_t>(tile) * max_seg * (32 * 4 * MT);
-#pragma unroll
-    for (int m = 0; m < MT; ++m) {
-      const float4 v = make_float4(acc[0][m][0] + acc[1][m][0], acc[0][m][1] + acc[1][m][1],
-                                   acc[0][m][2] + acc[1][m][2], acc[0][m][3] + acc[1][m][3]);
-      __stcg(reinterpret_cast<float4*>(tile_part + (slot * 32 + lane) * 4 * MT) + m, v);
-    }
-    __threadfence();
-    __syncwarp();
-    unsigned int ticket = 0;
-    if (nseg > 1) {
-      if (lane == 0) ticket = atomicAdd(&counters[tile], 1u);
-      ticket = __shfl_sync(0xffffffffu, ticket, 0);
-      if (ticket != static_cast<unsigned int>(nseg - 1)) continue;  // another warp completes the tile
-      __threadfence();
-    }
-
-    // ---- complete the tile: sum the slots in order, add s (T B^T), store Y ----
-    float y[MT][4];
-#pragma unroll
-    for (int m = 0; m < MT; ++m) y[m][0] = y[m][1] = y[m][2] = y[m][3] = 0.0f;
-    for (int sl = 0; sl < nseg; ++sl) {
-#pragma unroll
-      for (int m = 0; m < MT; ++m) {
-        const float4 v = __ldcg(reinterpret_cast<const float4*>(tile_part + (sl * 32 + lane) * 4 * MT) + m);
-        y[m][0] += v.x; y[m][1] += v.y; y[m][2] += v.z; y[m][3] += v.w;
-      }
-    }
-    // LoRA up: rows of B are the A operand, T^T (split into bf16 hi + lo) the B operand.
-    const int64_t na = tile * 16 + g, nb = na + 8;
-    float l[MT][4];
-#pragma unroll
-    for (int m = 0; m < MT; ++m) l[m][0] = l[m][1] = l[m][2] = l[m][3] = 0.0f;
-    for (int j0 = 0; j0 < r; j0 += 16) {
-      const uint32_t b_a0 = na < N ? *reinterpret_cast<const uint32_t*>(Bl + na * r + j0 + 2 * t) : 0u;
-      const uint32_t b_a2 = na < N ? *reinterpret_cast<const uint32_t*>(Bl + na * r + j0 + 2 * t + 8) : 0u;
-      const uint32_t b_a1 = nb < N ? *reinterpret_cast<const uint32_t*>(Bl + nb * r + j0 + 2 * t) : 0u;
-      const uint32_t b_a3 = nb < N ? *reinterpret_cast<const uint32_t*>(Bl + nb * r + j0 + 2 * t + 8) : 0u;
-#pragma unroll
-      for (int m = 0; m < MT; ++m) {
-        const int tok = g + 8 * m;
-        float tv[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-        if (tok < M) {
-          const float* tp = T + static_cast<int64_t>(tok) * r + j0 + 2 * t;
-          tv[0] = __ldcg(tp);
-          tv[1] = __ldcg(tp + 1);
-          tv[2] = __ldcg(tp + 8);
-          tv[3] = __ldcg(tp + 9);
-        }
-        uint32_t hi[2], lo[2];
-#pragma unroll
-        for (int p = 0; p < 2; ++p) {
-          const uint32_t h = pack_bf16x2(tv[2 * p], tv[2 * p + 1]);
-          hi[p] = h;
-          lo[p] = pack_bf16x2(tv[2 * p] - bf16lo_to_f32(h), tv[2 * p + 1] - bf16hi_to_f32(h));
-        }
-        mma16816(l[m], b_a0, b_a1, b_a2, b_a3, hi[0], hi[1]);
-        mma16816(l[m], b_a0, b_a1, b_a2, b_a3, lo[0], lo[1]);
-      }
-    }
-#pragma unroll
-    for (int m = 0; m < MT; ++m) {
-      const int tok0 = 8 * m + 2 * t, tok1 = tok0 + 1;
-      if (na < N) {
-        if (tok0 < M) Y[static_cast<int64_t>(tok0) * N + na] = __float2bfloat16_rn(fmaf(s, l[m][0], y[m][0]));
-        if (tok1 < M) Y[static_cast<int64_t>(tok1) * N + na] = __float2bfloat16_rn(fmaf(s, l[m][1], y[m][1]));
-      }
-      if (nb < N) {
-        if (tok0 < M) Y[static_cast<int64_t>(tok0) * N + nb] = __float2bfloat16_rn(fmaf(s, l[m][2], y[m][2]));
-        if (tok1 < M) Y[static_cast<int64_t>(tok1) * N + nb] = __float2bfloat16_rn(fmaf(s, l[m][3], y[m][3]));
-      }
-    }
-    if (nseg > 1 && lane == 0) counters[tile] = 0u;  // ready for the next call
+    publish_segment<MT>(acc, rg, rg * kDecodeWarps + warp, cta, lane, nsb, n_items, n_ctas, max_seg, partial,
+                        counters, T, Bl, r, s, Y, M, N);
+    ++rg;
+    sb = 0;
   }
+  if (!entered) grid_dependency_launch_dependents();
 }
 
 // T[m, j] = sum_k X[m, k] A[j, k] for M <= 16 (fp32 on CUDA cores), one CTA per
@@ -342,19 +409,20 @@ k_lora_t_small(const __nv_bfloat16* __restrict__ X, const __nv_bfloat16* __restr
 DecodePlan decode_plan(int64_t M, int64_t N, int64_t K, int ref_sms) {
   DecodePlan p;
   p.mt = M <= 8 ? 1 : 2;
-  p.row_tiles = (N + 15) / 16;
+  p.n_groups = (N + kRowsPerItem - 1) / kRowsPerItem;
+  p.row_tiles = p.n_groups * kDecodeWarps;
   p.nsb = (K / 64 + 3) / 4;
-  p.n_items = p.row_tiles * p.nsb;
-  // At most one warp per item, so every warp's range is non-empty and the
-  // owners of consecutive items are consecutive warps (slot = warp - first owner).
-  const int64_t cap = static_cast<int64_t>(ref_sms) * kDecodeCtasPerSm * kDecodeWarps;
-  p.n_warps = p.n_items < cap ? p.n_items : cap;
-  if (p.n_warps < 1) p.n_warps = 1;
-  p.grid = static_cast<int>((p.n_warps + kDecodeWarps - 1) / kDecodeWarps);
+  p.n_items = p.n_groups * p.nsb;
+  // At most one CTA per item, so every CTA's range is non-empty and the owners
+  // of consecutive items are consecutive CTAs (slot = CTA - first owner).
+  const int64_t cap = static_cast<int64_t>(ref_sms) * kDecodeCtasPerSm;
+  int64_t grid = p.n_items < cap ? p.n_items : cap;
+  if (grid < 1) grid = 1;
+  p.grid = static_cast<int>(grid);
   p.max_seg = 1;
-  for (int64_t tile = 0; tile < p.row_tiles; ++tile) {
-    const int64_t a = item_owner(tile * p.nsb, p.n_items, p.n_warps);
-    const int64_t b = item_owner((tile + 1) * p.nsb - 1, p.n_items, p.n_warps);
+  for (int64_t rg = 0; rg < p.n_groups; ++rg) {
+    const int64_t a = item_owner(rg * p.nsb, p.n_items, grid);
+    const int64_t b = item_owner((rg + 1) * p.nsb - 1, p.n_items, grid);
     if (b - a + 1 > p.max_seg) p.max_seg = static_cast<int>(b - a + 1);
   }
   return p;
@@ -366,27 +434,57 @@ size_t decode_partial_elems(const DecodePlan& p) {
 
 size_t decode_counter_words(const DecodePlan& p) { return static_cast<size_t>(p.row_tiles); }
 
+namespace {
+
+bool encode_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t inner, uint64_t outer,
+               uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer) {
+  PFN_encodeTiled enc = get_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1u, 1u};
+  return enc(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
 cudaError_t launch_decode_fwd(const Nf4View& w, const void* X, int64_t M, const void* A, const void* B, int r,
                               float s, void* Y, float* T, float* partial, unsigned int* counters,
-                              const DecodePlan& p, const float codebook[16], cudaStream_t stream) {
+                              const DecodePlan& p, const float codebook[16], int32_t* err, cudaStream_t stream) {
+  if (w.N >= (int64_t(1) << 31) || w.K >= (int64_t(1) << 31)) return cudaErrorInvalidValue;  // TMA coordinates
   Nf4Codebook cb;
   for (int i = 0; i < 16; ++i) cb.c[i] = codebook[i];
-  const __nv_bfloat16* Xb = reinterpret_cast<const __nv_bfloat16*>(X);
-  cudaError_t e = launch_pdl(p.mt == 1 ? k_lora_t_small<1> : k_lora_t_small<2>, dim3(r), dim3(256), 0, stream, Xb,
-                             reinterpret_cast<const __nv_bfloat16*>(A), static_cast<int>(M), w.K, r, T, counters,
-                             p.row_tiles);
+  // packed weights as a [N, K/2] byte matrix, box = 128 rows x 128 bytes;
+  // token values [M, K] bf16, box = 64 k x 8 MT rows (rows >= M read as zero)
+  CUtensorMap tw, tx;
+  if (!encode_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, w.packed, static_cast<uint64_t>(w.K / 2),
+                 static_cast<uint64_t>(w.N), static_cast<uint64_t>(w.K / 2), 128u, kRowsPerItem) ||
+      !encode_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, static_cast<uint64_t>(w.K), static_cast<uint64_t>(M),
+                 static_cast<uint64_t>(w.K) * 2, 64u, 8u * p.mt))
+    return cudaErrorInvalidValue;
+  cudaError_t e = launch_pdl(p.mt == 1 ? k_lora_t_small<1> : k_lora_t_small<2>, dim3(r), dim3(256), 0, stream,
+                             reinterpret_cast<const __nv_bfloat16*>(X), reinterpret_cast<const __nv_bfloat16*>(A),
+                             static_cast<int>(M), w.K, r, T, counters, p.row_tiles);
   if (e != cudaSuccess) return e;
   // Programmatic dependent launch: the main loop overlaps the LoRA-down kernel;
-  // each warp waits for it (griddepcontrol.wait) before its first ticket.
-  const bool v8 = ((reinterpret_cast<uintptr_t>(X) | reinterpret_cast<uintptr_t>(w.packed)) & 31u) == 0;
+  // each consumer warp waits for it (griddepcontrol.wait) before its first ticket.
   const __nv_bfloat16* Bb = reinterpret_cast<const __nv_bfloat16*>(B);
   __nv_bfloat16* Yb = reinterpret_cast<__nv_bfloat16*>(Y);
   const int Mi = static_cast<int>(M);
-  auto kern = p.mt == 1 ? (v8 ? k_decode<1, true> : k_decode<1, false>)
-                        : (v8 ? k_decode<2, true> : k_decode<2, false>);
-  e = launch_pdl(kern, dim3(p.grid), dim3(kDecodeWarps * 32), 0, stream, w.packed, w.absmax_q, w.dq_scale, w.mean,
-                 Xb, Mi, w.N, w.K, static_cast<const float*>(T), Bb, r, s, Yb, partial, counters, p.n_items,
-                 p.n_warps, p.max_seg, cb);
+  auto kern = p.mt == 1 ? k_decode<1> : k_decode<2>;
+  const int smem = decode_smem_bytes(p.mt);
+  static bool smem_set[2] = {false, false};
+  if (!smem_set[p.mt - 1]) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    smem_set[p.mt - 1] = true;
+  }
+  e = launch_pdl(kern, dim3(p.grid), dim3((kDecodeWarps + 1) * 32), smem, stream, tw, tx, w.absmax_q, w.dq_scale,
+                 w.mean, Mi, w.N, w.K, static_cast<const float*>(T), Bb, r, s, Yb, partial, counters, p.n_items,
+                 static_cast<int64_t>(p.grid), p.max_seg, err, cb);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

@@ -22,6 +22,7 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "tensor_map.h"
 
 namespace qlora {
 namespace {
@@ -632,22 +633,6 @@ k_tc_gemm2(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUt
 
 // ---------------------------------------------------------------------------
 // host side
-
-typedef CUresult (*PFN_encodeTiled)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                    const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                    CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-PFN_encodeTiled get_encoder() {
-  static PFN_encodeTiled fn = [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
-        q != cudaDriverEntryPointSuccess)
-      return static_cast<PFN_encodeTiled>(nullptr);
-    return reinterpret_cast<PFN_encodeTiled>(p);
-  }();
-  return fn;
-}
 
 // 2-D bf16 tensor [outer, inner] with row stride ld (elements); box {64, box_outer}.
 bool make_map(CUtensorMap* m, const void* base, int64_t inner, int64_t outer, int64_t ld, int box_outer) {

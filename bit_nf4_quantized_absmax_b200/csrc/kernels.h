@@ -41,16 +41,17 @@ struct Nf4View {
 };
 
 // ---- decode.cu: M <= 16 forward ----
-// Work split of the decode kernel: (16-row tile, 256-wide K superblock) items
-// cut into equal per-warp ranges; fixed by (M, N, K) and a reference SM count.
+// Work split of the decode kernel: (128-row group, 256-wide K superblock)
+// items cut into equal per-CTA ranges; fixed by (M, N, K) and a reference SM
+// count.
 struct DecodePlan {
   int mt;             // token tiles of 8 (1: M <= 8, 2: M <= 16)
-  int64_t row_tiles;  // ceil(N / 16)
+  int64_t n_groups;   // ceil(N / 128)
+  int64_t row_tiles;  // 16-row tiles: 8 * n_groups
   int64_t nsb;        // ceil(K / 256)
-  int64_t n_items;    // row_tiles * nsb
-  int grid;           // CTAs of 8 warps (the last one may be partly idle)
-  int64_t n_warps;    // working warps: min(n_items, 8 * CTA capacity)
-  int max_seg;        // most warps sharing one row tile
+  int64_t n_items;    // n_groups * nsb
+  int grid;           // CTAs = work ranges: min(n_items, CTA capacity)
+  int max_seg;        // most CTAs sharing one row group
 };
 DecodePlan decode_plan(int64_t M, int64_t N, int64_t K, int ref_sms);
 size_t decode_partial_elems(const DecodePlan& p);
@@ -59,7 +60,7 @@ size_t decode_counter_words(const DecodePlan& p);
 // counters [decode_counter_words] are scratch.
 cudaError_t launch_decode_fwd(const Nf4View& w, const void* X, int64_t M, const void* A, const void* B, int r,
                               float s, void* Y, float* T, float* partial, unsigned int* counters,
-                              const DecodePlan& p, const float codebook[16], cudaStream_t stream);
+                              const DecodePlan& p, const float codebook[16], int32_t* err, cudaStream_t stream);
 
 // ---- gemm_tc.cu: tcgen05 GEMMs ----
 cudaError_t launch_gemm_fwd(const void* X, const void* Wd, const void* sT, const void* Bl, int64_t M, int64_t N,
