@@ -210,8 +210,9 @@ class Workload:
                                     ALPHA, qb._ptr(d["dY"]), qb._ptr(d["T"]), qb._ptr(d["dX"]), qb._ptr(d["dA"]),
                                     qb._ptr(d["dB"]), ws, ctypes.byref(n), st)
 
-    def step(self, ev=None):
-        """One pass of the hot path. ev: optional dict part -> list of (start, end) events."""
+    def step(self, ev=None, only=None):
+        """One pass of the hot path. ev: optional dict part -> list of (start, end)
+        events, recorded for the parts named in `only` (all parts if None)."""
         import ctypes
         lib = qb.load_library()
         st = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
@@ -219,7 +220,7 @@ class Workload:
         n = ctypes.c_size_t(self.ws.numel())
 
         def rec(part, fn):
-            if ev is not None:
+            if ev is not None and (only is None or part in only):
                 a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
                 a.record()
                 rc = fn()
@@ -267,13 +268,75 @@ def e2e_step(work: Workload, host):
     return h2d, d2h
 
 
+def breakdown(work, dev, reps=24):
+    """Mean time per call (us) of every part of the step, L2-cold inputs."""
+    import ctypes
+    lib = qb.load_library()
+    st = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    ws = ctypes.c_void_p(work.ws.data_ptr())
+    n = ctypes.c_size_t(work.ws.numel())
+    l2 = getattr(torch.cuda.get_device_properties(dev), "L2_cache_size", 128 << 20)
+    out = {}
+
+    def timed(part, calls):
+        for c in calls[:3]:
+            c()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for i in range(reps):
+            rc = calls[i % len(calls)]()
+            if rc != 0:
+                raise qb.QloraError(rc, part)
+        b.record()
+        torch.cuda.synchronize()
+        out[part] = 1e3 * a.elapsed_time(b) / reps
+
+    for li, d in enumerate(work.lin):
+        N, K = d["N"], d["K"]
+        nw = max(2, math.ceil(2 * l2 / (2 * N * K)))
+        nq = max(2, math.ceil(2 * l2 / (0.515869 * N * K)))
+        Ws = [d["W"]] + [d["W"].clone() for _ in range(nw - 1)]
+        Wds = [d["Wd"]] + [torch.empty_like(d["Wd"]) for _ in range(nw - 1)]
+        qs = [d["q"]]
+        for _ in range(nq - 1):
+            qn = qb.NF4Weight.empty(N, K, dev)
+            for name in ("packed", "absmax_q", "dq_scale", "mean"):
+                getattr(qn, name).copy_(getattr(d["q"], name))
+            qs.append(qn)
+        qcs = [q.as_c() for q in qs]
+
+        def q_call(i, li=li):
+            return lib.qlora_quantize_nf4_dq(qb._ptr(Ws[i % nw]), ctypes.byref(qcs[i % nq]), ws, ctypes.byref(n), st)
+
+        timed(f"quantize/{li}", [lambda i=i: q_call(i) for i in range(max(nw, nq))])
+        timed(f"dequantize/{li}", [lambda i=i: lib.qlora_dequantize_nf4_dq(ctypes.byref(qcs[i % nq]),
+                                                                            qb._ptr(Wds[i % nw]), st)
+                                   for i in range(max(nw, nq))])
+        for M in M_DECODE:
+            X, Y = d["Xdec"][M], d["Ydec"][M]
+            timed(f"decode{M}/{li}", [lambda qc=qc, X=X, Y=Y, M=M: lib.qlora_linear_fwd(
+                ctypes.byref(qc), qb._ptr(X), M, qb._ptr(d["A"]), qb._ptr(d["B"]), R, ALPHA, qb._ptr(Y), None, ws,
+                ctypes.byref(n), st) for qc in qcs])
+        timed(f"train_fwd/{li}", [lambda d=d: work._fwd_call(lib, d, ws, n, st, M_TRAIN)])
+        timed(f"train_bwd/{li}", [lambda d=d: work._bwd_call(lib, d, ws, n, st, M_TRAIN)])
+        del Ws, Wds, qs, qcs
+        torch.cuda.empty_cache()
+    return out
+
+
 def run_ours(args, rank, world, dev):
+    def say(msg):  # progress on stderr (stdout carries only the JSON line)
+        if args.verbose or rank == 0:
+            print(f"[bench rank {rank}] {msg}", file=sys.stderr, flush=True)
+
     peaks = load_peaks()
+    say("allocating the workload")
     work = Workload(dev, seed=rank)
     fl_train = sum(sum(train_flops(N, K)) for N, K in SHAPES)
 
     clocks = ClockSampler(gpu_index_for_smi(dev))
     clocks.start()
+    say("warm-up")
     t_w = time.time()
     for i in range(args.warmup):
         work.step()
@@ -284,7 +347,11 @@ def run_ours(args, rank, world, dev):
         torch.cuda.synchronize()
     torch.cuda.synchronize()
 
-    # per-part times from events inside the timed region (same stream)
+    # timed region: K whole steps; events on the launching stream bracket the
+    # region and (for the roofline) the dominant call of every step
+    say("timed region")
+    li_roof = SHAPES.index(ROOFLINE_SHAPE)
+    roof_part = f"train_fwd/{li_roof}"
     ev = {}
     barrier(world)
     torch.cuda.synchronize()
@@ -293,7 +360,7 @@ def run_ours(args, rank, world, dev):
     clocks.mark_begin()
     t0.record()
     for _ in range(args.steps):
-        work.step(ev)
+        work.step(ev, only={roof_part})
     t1.record()
     torch.cuda.synchronize()
     clocks.mark_end()
@@ -303,11 +370,15 @@ def run_ours(args, rank, world, dev):
     ms_step = max_over_ranks(ms_total / args.steps, world, dev)
     err = qb.qlora_device_error()
 
+    # per-part breakdown (outside the timed region): each call run back to back,
+    # cycling through enough copies of its inputs and outputs to exceed twice the
+    # L2, so that every call reads its weights from HBM
+    say("per-part breakdown")
+    part_us = breakdown(work, dev)
     parts = {}
-    for part, lst in ev.items():
+    for part, us in part_us.items():
         kind, li = part.split("/")
         N, K = SHAPES[int(li)]
-        us = 1e3 * statistics.mean(a.elapsed_time(b) for a, b in lst)
         e = {"us": round(us, 2)}
         if kind in ("quantize", "dequantize"):
             e["GB_s"] = round(quant_bytes(N, K) / us / 1e3, 1)
@@ -323,8 +394,7 @@ def run_ours(args, rank, world, dev):
     # dominant call: the training forward (M = 4096) on the 11008x4096 linear, i.e.
     # one dequant, the LoRA-down GEMM + finish and the 2-CTA tcgen05 GEMM with the
     # LoRA slab; algorithmic flops over its measured duration (events on the stream).
-    li = SHAPES.index(ROOFLINE_SHAPE)
-    fwd_us = 1e3 * statistics.mean(a.elapsed_time(b) for a, b in ev[f"train_fwd/{li}"])
+    fwd_us = 1e3 * statistics.mean(a.elapsed_time(b) for a, b in ev[roof_part])
     achieved = train_flops(*ROOFLINE_SHAPE)[0] / fwd_us / 1e6
     traffic = TRAFFIC_RECORD["bytes"] if TRAFFIC_RECORD["fingerprint"] == source_fingerprint() else None
     roof = {"kernel": "qlora_linear_fwd M=4096 on 11008x4096 (dequant, LoRA-down, 2-CTA tcgen05 GEMM)",
@@ -335,6 +405,7 @@ def run_ours(args, rank, world, dev):
             "us_per_launch": round(fwd_us, 2)}
     dec = [parts[f"decode{M}/{N}x{K}"]["weight_GB_s"] for M in M_DECODE for N, K in SHAPES]
 
+    say("end to end with host buffers")
     # end to end through the C ABI with host buffers
     host = []
     for d in work.lin:
@@ -367,8 +438,10 @@ def run_ours(args, rank, world, dev):
         "config": {"workload": "Llama-7B linear shapes 4096x4096, 11008x4096, 4096x11008; r=64 alpha=16; "
                                "quantize+DQ, dequant, decode M=1/4/16, train fwd+bwd M=4096",
                    "global_batch_tokens": M_TRAIN * world, "parallelism": f"dp{world} (independent replicas)",
-                   "l2": "inputs larger than L2 (each step touches ~1.2 GB)"},
+                   "l2": "inputs larger than L2 (each step touches ~1.2 GB)",
+                   "parts": "each call back to back over rotating input copies > 2x L2, outside the timed region"},
         "decode_weight_GB_s": {"min": min(dec), "max": max(dec)},
+        "hbm_frac": {k: round(v["GB_s"] / peaks["hbm_gbs"], 4) for k, v in parts.items() if "GB_s" in v},
         "parts": parts,
         "roofline": roof,
         "e2e": {"value": round(world * fl_train / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
@@ -504,6 +577,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--verbose", action="store_true", help="print progress to stderr")
     ap.add_argument("--profile-case", action="store_true",
                     help="run one call of each entry point on 11008x4096 (for ncu) and exit")
     args = ap.parse_args()

@@ -58,16 +58,14 @@ void build(QuantTables& t) {
     t.thresholds[i] = f;
   }
 
-  // Bin table. Bin b holds x = RN(v * S + 3) in [2 + 2b/kBins, 2 + 2(b+1)/kBins);
-  // rounding moves x by at most 2^-23, so bin b can only see
-  // v in [(2 + 2b/kBins - 2^-23 - 3) / S, (2 + 2(b+1)/kBins + 2^-23 - 3) / S];
-  // widen by another 2^-20 for margin. Each widened bin must contain at most one
+  // Bin table. Bin b holds u = 128 + r in [8b, 8b + 7], r = round(v * 127) (ties
+  // to even), so it can only see v with v * 127 in [8b - 128.5, 8b - 120.5];
+  // widen by 2^-20 for margin. Each widened bin must contain at most one
   // threshold (bins are ~0.063 wide, thresholds >= 0.08 apart); checked below.
-  const double S = static_cast<double>(kBinScale);
-  const double w = 2.0 / kBins;
+  const double P = static_cast<double>(kBinMul);
   for (int b = 0; b < kBins; ++b) {
-    double lo = (2.0 + b * w - std::ldexp(1.0, -23) - 3.0) / S - std::ldexp(1.0, -20);
-    double hi = (2.0 + (b + 1) * w + std::ldexp(1.0, -23) - 3.0) / S + std::ldexp(1.0, -20);
+    double lo = (8.0 * b - 128.5) / P - std::ldexp(1.0, -20);
+    double hi = (8.0 * b - 120.5) / P + std::ldexp(1.0, -20);
     int inside = -1, count = 0, below = 0;
     for (int i = 0; i < 15; ++i) {
       double T = t.thresholds[i];

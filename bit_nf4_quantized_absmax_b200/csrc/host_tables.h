@@ -7,11 +7,14 @@
 
 namespace qlora {
 
-// Bin mapping used by the quantize kernel: x = fmaf(v, kBinScale, 3.0f) lies
-// in [2, 4) for v in [-1, 1]; the top kBinBits mantissa bits of x index the bin.
-constexpr float kBinScale = 0.9990234375f;  // 1 - 2^-10, exact in fp32
-constexpr int kBinBits = 5;
-constexpr int kBins = 1 << kBinBits;
+// Bin mapping used by the quantize kernel: x = fmaf(v, kBinMul, kBinAdd) is
+// 1.5 * 2^23 + 128 + r with r = v * 127 rounded to the nearest integer (one
+// rounding; |r| <= 127 for v in [-1, 1]), so the low byte of x's bit pattern is
+// u = 128 + r in [1, 255], and bin = u >> 3 (the byte offset of the bin's
+// 8-byte table entry is u & 0xF8).
+constexpr float kBinMul = 127.0f;
+constexpr float kBinAdd = 12583040.0f;  // 1.5 * 2^23 + 128, exact in fp32
+constexpr int kBins = 32;
 
 struct BinEntry {
   float threshold;  // T_j

@@ -141,23 +141,23 @@ __device__ __forceinline__ void quant_item(const uint4 d, bool valid, int lane, 
       for (int i = 0; i < 8; ++i) w[i] *= sc;
     }
     const float r = __frcp_rn(ms);
-    const f32x2 r2{r, r}, nms2{-ms, -ms}, S2{kBinScale, kBinScale}, three2{3.0f, 3.0f};
+    const unsigned char* bins = reinterpret_cast<const unsigned char*>(s_bins);
     word = 0u;
 #pragma unroll
-    for (int i = 0; i < 8; i += 2) {
-      // v = RN(w / m), two elements per packed instruction: q0 = RN(w * RN(1/m))
-      // is within one ulp, the remainder w - q0 m is exact, and one correction
-      // step rounds correctly (Markstein).
-      const f32x2 wi{w[i], w[i + 1]};
-      const f32x2 q0 = mul_f32x2(wi, r2);
-      const f32x2 res = fma_f32x2(q0, nms2, wi);
-      const f32x2 v = fma_f32x2(res, r2, q0);
-      const f32x2 x = fma_f32x2(v, S2, three2);
-      const uint2 e0 = s_bins[(__float_as_uint(x.x) >> (23 - kBinBits)) & (kBins - 1)];
-      const uint2 e1 = s_bins[(__float_as_uint(x.y) >> (23 - kBinBits)) & (kBins - 1)];
-      const uint32_t c0 = e0.y + (v.x >= __uint_as_float(e0.x) ? 1u : 0u);
-      const uint32_t c1 = e1.y + (v.y >= __uint_as_float(e1.x) ? 1u : 0u);
-      word |= (c0 | (c1 << 4)) << (4 * i);
+    for (int i = 0; i < 8; ++i) {
+      // v = RN(w / m): q0 = RN(w * RN(1/m)) is within one ulp, the remainder
+      // w - q0 m is exact, and one correction step rounds correctly (Markstein).
+      const float q0 = __fmul_rn(w[i], r);
+      const float res = __fmaf_rn(q0, -ms, w[i]);
+      const float v = __fmaf_rn(res, r, q0);
+      // bin: low byte of RN(v * 127 + 1.5 * 2^23 + 128); entry = (T_j, j + 1)
+      const float x = __fmaf_rn(v, kBinMul, kBinAdd);
+      const uint2 e = *reinterpret_cast<const uint2*>(bins + (__float_as_uint(x) & 0xF8u));
+      // code = j + (v >= T_j) = (j + 1) - [v < T_j]; RN(v - T_j) has the sign of
+      // v - T_j and is +0 when they are equal
+      const float d = __fsub_rn(v, __uint_as_float(e.x));
+      const uint32_t c = e.y - __umulhi(__float_as_uint(d), 2u);
+      word += c * (1u << (4 * i));
     }
   }
   packed[item] = word;
@@ -173,7 +173,7 @@ k_quant_pass1(const uint4* __restrict__ W, int64_t n_items, uint32_t* __restrict
   __shared__ int s_last;
   const int tid = threadIdx.x;
   const int lane = tid & 31;
-  if (tid < kBins) s_bins[tid] = make_uint2(__float_as_uint(tab.bins[tid].threshold), tab.bins[tid].j);
+  if (tid < kBins) s_bins[tid] = make_uint2(__float_as_uint(tab.bins[tid].threshold), tab.bins[tid].j + 1u);
   s_hist[tid] = 0u;
   __syncthreads();
   pdl_enter();
