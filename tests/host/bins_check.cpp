@@ -1,0 +1,59 @@
+// Exhaustive host check of the quantize kernel's binning rule: for every fp32 v
+// in [-1, 1], the code the kernel forms from its 32-bin table,
+//   x = fmaf(v, kBinMul, kBinAdd), entry = bins[(bits(x) & 0xF8) >> 3],
+//   code = (entry.j + 1) - [RN(v - entry.threshold) < 0],
+// must equal the number of decision thresholds T_i with v >= T_i (the nearest
+// code, ties to the lower index). Exit status 0 iff no value disagrees.
+#include <cmath>
+#include <cstdint>
+#include <cstdio>
+#include <cstring>
+#include <thread>
+#include <vector>
+
+#include "host_tables.h"
+
+using namespace qlora;
+
+static uint64_t check_range(uint32_t lo, uint32_t hi, int sign) {
+  const QuantTables& t = quant_tables();
+  uint64_t bad = 0;
+  for (uint32_t bits = lo; bits < hi; ++bits) {
+    const uint32_t b = bits | (sign ? 0x80000000u : 0u);
+    float v;
+    std::memcpy(&v, &b, 4);
+    int ref = 0;
+    for (int i = 0; i < 15; ++i) ref += (v >= t.thresholds[i]) ? 1 : 0;
+    const float x = std::fmaf(v, kBinMul, kBinAdd);
+    uint32_t xb;
+    std::memcpy(&xb, &x, 4);
+    const BinEntry& e = t.bins[(xb & 0xF8u) >> 3];
+    const float d = v - e.threshold;
+    uint32_t db;
+    std::memcpy(&db, &d, 4);
+    const int code = static_cast<int>(e.j + 1) - static_cast<int>(db >> 31);
+    if (code != ref) {
+      if (bad < 3) std::printf("mismatch: v=%a expected %d got %d\n", v, ref, code);
+      ++bad;
+    }
+  }
+  return bad;
+}
+
+int main() {
+  const uint32_t end = 0x3F800001u;  // every bit pattern of [+0, 1]
+  const unsigned nt = std::thread::hardware_concurrency() ? std::thread::hardware_concurrency() : 4;
+  std::vector<std::thread> th;
+  std::vector<uint64_t> bad(2 * nt, 0);
+  for (int sign = 0; sign < 2; ++sign)
+    for (unsigned k = 0; k < nt; ++k) {
+      const uint32_t lo = static_cast<uint32_t>(uint64_t(end) * k / nt);
+      const uint32_t hi = static_cast<uint32_t>(uint64_t(end) * (k + 1) / nt);
+      th.emplace_back([&, lo, hi, sign, k] { bad[sign * nt + k] = check_range(lo, hi, sign); });
+    }
+  for (auto& x : th) x.join();
+  uint64_t total = 0;
+  for (uint64_t b : bad) total += b;
+  std::printf("checked %llu values, %llu mismatches\n", 2ull * end, static_cast<unsigned long long>(total));
+  return total == 0 ? 0 : 1;
+}
