@@ -160,7 +160,7 @@ qlora_status qlora_quantize_nf4_dq(const void* W_bf16, const qlora_nf4_weight* q
   if (W_bf16 && !aligned(W_bf16, 16)) return QLORA_ERR_ALIGNMENT;
   const int64_t numel = q->rows * q->cols;
   const int64_t nblk = numel / 64;
-  const size_t off_absmax = align_up(kQuantBinWords * sizeof(unsigned long long));
+  const size_t off_absmax = align_up(kQuantScratchBytes);
   const size_t need = off_absmax + align_up(static_cast<size_t>(nblk) * sizeof(float));
   bool launch = false;
   st = workspace_check(workspace, workspace_bytes, need, &launch);
@@ -170,7 +170,7 @@ qlora_status qlora_quantize_nf4_dq(const void* W_bf16, const qlora_nf4_weight* q
   char* ws = static_cast<char*>(workspace);
   return cuda_status(launch_quantize(W_bf16, numel, q->packed, q->absmax_q, q->dq_scale, q->mean,
                                      reinterpret_cast<float*>(ws + off_absmax),
-                                     reinterpret_cast<unsigned long long*>(ws), di.num_sms,
+                                     ws, di.num_sms,
                                      reinterpret_cast<cudaStream_t>(stream)));
 }
 

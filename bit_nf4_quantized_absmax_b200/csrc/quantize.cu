@@ -3,14 +3,15 @@
 // "Core Architecture & Training").
 //
 // Three launches:
-//   k_quant_zero   clears the 256 exponent bins and the CTA ticket.
-//   k_quant_pass1  streams W once: per 64-weight block the absmax (8-lane
-//                  shuffle reduction over 16-byte loads), the exact quotient
-//                  v = w / m, the nearest code (one lookup in a 32-bin table + one compare),
-//                  4-bit packing; it also accumulates the exact sum of the
-//                  absmax constants as integer significand sums per exponent.
+//   k_quant_pass1  streams W once, four lanes per 64-weight block (one 32-byte
+//                  load each, 1 KB contiguous per warp instruction): the absmax (packed 16-bit max of the magnitude bits), the exact
+//                  quotient v = w / m, the nearest code (one lookup in a 32-bin
+//                  table + one compare), 4-bit packing; it also accumulates the
+//                  exact sum of the absmax constants as integer significand sums
+//                  per exponent.
 //                  The last CTA to finish turns that sum into the mean.
-//   k_dq_quantize  one warp per 256 constants: centre on the mean, group
+//   k_dq_quantize  forms the mean from the exact bin totals (every CTA, warp 0),
+//                  then one warp per 256 constants: centre on the mean, group
 //                  absmax, int8 codes with round-to-nearest-even.
 #include "common.cuh"
 #include "host_tables.h"
@@ -25,39 +26,31 @@ struct QuantBinTable {
 namespace {
 
 constexpr int kPass1Threads = 256;
-constexpr int kPass1Unroll = 4;
 
-__global__ void k_quant_zero(unsigned long long* bins) {
-  pdl_enter();
-  const int i = threadIdx.x;
-  if (i < kQuantBinWords) bins[i] = 0ull;
+// Exact sums of the absmax constants: each constant m = sig * 2^(E - 134)
+// (E the biased exponent, sig its 8-bit significand) is counted as the integer
+// sig in exponent bin E. The total sum_E bins[E] * 2^(E - 134) is formed in a
+// 320-bit fixed-point integer with unit 2^-133 (five 64-bit limbs kept in
+// registers), then rounded once to fp64 (nearest, ties to even).
+__device__ __forceinline__ void acc_bin(unsigned long long (&L)[5], unsigned long long x, int E) {
+  const int pos = E - 1;  // bit position of x's lsb
+  const int li = pos >> 6, off = pos & 63;
+  const unsigned long long lo = x << off;
+  const unsigned long long hi = off ? (x >> (64 - off)) : 0ull;
+  unsigned long long carry = 0ull;
+#pragma unroll
+  for (int k = 0; k < 5; ++k) {
+    const unsigned long long add = (k == li) ? lo : ((k == li + 1) ? hi : 0ull);
+    const unsigned long long s1 = L[k] + add;
+    const unsigned long long c1 = s1 < L[k] ? 1ull : 0ull;
+    const unsigned long long s2 = s1 + carry;
+    const unsigned long long c2 = s2 < s1 ? 1ull : 0ull;
+    L[k] = s2;
+    carry = c1 + c2;
+  }
 }
 
-// Exact fp64 value of sum_E hist[E] * 2^(E - 134) (E = biased exponent, the
-// significand sums are integers): the sum is formed in a 320-bit fixed-point
-// integer with unit 2^-133 (five 64-bit limbs kept in registers), then rounded
-// once to fp64 (nearest, ties to even).
-__device__ double exact_sum_to_double(const unsigned long long* hist) {
-  unsigned long long L[5] = {0, 0, 0, 0, 0};
-  for (int E = 1; E < 256; ++E) {
-    const unsigned long long x = hist[E];
-    if (!x) continue;
-    const int pos = E - 1;  // bit position of x's lsb
-    const int li = pos >> 6, off = pos & 63;
-    const unsigned long long lo = x << off;
-    const unsigned long long hi = off ? (x >> (64 - off)) : 0ull;
-    unsigned long long carry = 0ull;
-#pragma unroll
-    for (int k = 0; k < 5; ++k) {
-      const unsigned long long add = (k == li) ? lo : ((k == li + 1) ? hi : 0ull);
-      const unsigned long long s1 = L[k] + add;
-      const unsigned long long c1 = s1 < L[k] ? 1ull : 0ull;
-      const unsigned long long s2 = s1 + carry;
-      const unsigned long long c2 = s2 < s1 ? 1ull : 0ull;
-      L[k] = s2;
-      carry = c1 + c2;
-    }
-  }
+__device__ double limbs_to_double(const unsigned long long (&L)[5]) {
   // highest set bit
   int top = -1;
 #pragma unroll
@@ -98,130 +91,193 @@ __device__ double exact_sum_to_double(const unsigned long long* hist) {
   return ldexp(static_cast<double>(mant), exp2);
 }
 
-__device__ __forceinline__ void quant_item(const uint4 d, bool valid, int lane, int64_t item,
-                                           uint32_t* __restrict__ packed, float* __restrict__ absmax,
-                                           const uint2* __restrict__ s_bins,
-                                           unsigned int* __restrict__ s_hist) {
-  float w[8];
-  w[0] = bf16lo_to_f32(d.x); w[1] = bf16hi_to_f32(d.x);
-  w[2] = bf16lo_to_f32(d.y); w[3] = bf16hi_to_f32(d.y);
-  w[4] = bf16lo_to_f32(d.z); w[5] = bf16hi_to_f32(d.z);
-  w[6] = bf16lo_to_f32(d.w); w[7] = bf16hi_to_f32(d.w);
-  float a = fabsf(w[0]);
+__device__ __forceinline__ uint32_t max_u16x2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("max.u16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
+// Codes of 16 weights of a block given m (possibly scaled by a power of two
+// together with the weights) and r = RN(1/m); out[k] packs weights 8k..8k+7.
+template <bool SCALED>
+__device__ __forceinline__ void encode16(const uint32_t (&d)[8], float ms, float r, float wsc,
+                                         const unsigned char* bins, uint32_t (&out)[2]) {
 #pragma unroll
-  for (int i = 1; i < 8; ++i) a = fmaxf(a, fabsf(w[i]));
-  a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 1));
-  a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 2));
-  a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 4));
-  if (!valid) return;
-  const float m = a;  // block absmax (exact)
-  if ((lane & 7) == 0) {
-    absmax[item >> 3] = m;
-    if (m > 0.0f) {
-      const uint32_t u = __float_as_uint(m);
-      const uint32_t e = u >> 23;
-      const uint32_t mant7 = (u >> 16) & 0x7Fu;
-      const uint32_t sig = e ? (mant7 | 0x80u) : mant7;
-      const uint32_t E = e ? e : 1u;
-      atomicAdd(&s_hist[E], sig);
-    }
-  }
-  uint32_t word;
-  if (m == 0.0f) {
-    word = 0x77777777u;  // an all-zero block: every code is the exact zero
-  } else {
-    // Keep 1/m normal: scale w and m by a power of two (exact for bf16 values;
-    // only weights whose quotient is below 2^-126 can lose bits, and those map
-    // to the zero code either way).
-    float ms = m;
-    if (m < 5.421010862e-20f || m > 1.8446744e19f) {     // outside [2^-64, 2^64]: rare
-      const float sc = m < 5.421010862e-20f ? 1.8446744e19f : 5.421010862e-20f;
-      ms = m * sc;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) w[i] *= sc;
-    }
-    const float r = __frcp_rn(ms);
-    const unsigned char* bins = reinterpret_cast<const unsigned char*>(s_bins);
-    word = 0u;
+  for (int k = 0; k < 2; ++k) {
+    uint32_t word = 0u;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
+      const uint32_t bits = d[4 * k + (i >> 1)];
+      float w = __uint_as_float((i & 1) ? (bits & 0xFFFF0000u) : (bits << 16));
+      if (SCALED) w = __fmul_rn(w, wsc);
       // v = RN(w / m): q0 = RN(w * RN(1/m)) is within one ulp, the remainder
       // w - q0 m is exact, and one correction step rounds correctly (Markstein).
-      const float q0 = __fmul_rn(w[i], r);
-      const float res = __fmaf_rn(q0, -ms, w[i]);
+      const float q0 = __fmul_rn(w, r);
+      const float res = __fmaf_rn(q0, -ms, w);
       const float v = __fmaf_rn(res, r, q0);
       // bin: low byte of RN(v * 127 + 1.5 * 2^23 + 128); entry = (T_j, j + 1)
       const float x = __fmaf_rn(v, kBinMul, kBinAdd);
       const uint2 e = *reinterpret_cast<const uint2*>(bins + (__float_as_uint(x) & 0xF8u));
       // code = j + (v >= T_j) = (j + 1) - [v < T_j]; RN(v - T_j) has the sign of
       // v - T_j and is +0 when they are equal
-      const float d = __fsub_rn(v, __uint_as_float(e.x));
-      const uint32_t c = e.y - __umulhi(__float_as_uint(d), 2u);
+      const float dv = __fsub_rn(v, __uint_as_float(e.x));
+      const uint32_t c = e.y - __umulhi(__float_as_uint(dv), 2u);
       word += c * (1u << (4 * i));
     }
+    out[k] = word;
   }
-  packed[item] = word;
+}
+
+// Four lanes per 64-weight block (16 weights each, one 32-byte load): a warp
+// reads 1 KB of contiguous weights per load instruction. Every lane of a warp
+// runs the same iterations so that the histogram update can be combined across
+// the warp (lanes whose blocks share an exponent add their significands first,
+// then one of them updates the shared bin).
+template <bool V8>
+__device__ __forceinline__ void pass1_loop(const uint4* __restrict__ W, int64_t nblk, uint32_t* __restrict__ packed,
+                                           float* __restrict__ absmax, const unsigned char* bins,
+                                           unsigned int* __restrict__ s_hist) {
+  const int lane = threadIdx.x & 31;
+  const int qtr = lane & 3;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * (kPass1Threads / 4);
+  int64_t blk = (static_cast<int64_t>(blockIdx.x) * kPass1Threads + threadIdx.x) >> 2;
+  for (; blk - (lane >> 2) < nblk; blk += stride) {
+    const bool valid = blk < nblk;
+    uint32_t d[8];
+    if (valid) {
+      const uint4* src = W + blk * 8 + qtr * 2;
+      if (V8) {
+        ld_global_cs_v8(src, d);
+      } else {
+        const uint4 a = __ldcs(src), b = __ldcs(src + 1);
+        d[0] = a.x; d[1] = a.y; d[2] = a.z; d[3] = a.w; d[4] = b.x; d[5] = b.y; d[6] = b.z; d[7] = b.w;
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) d[i] = 0u;
+    }
+    // absmax on the bit patterns: for finite bf16, |w| orders as the unsigned 15-bit magnitude field
+    uint32_t mx = d[0] & 0x7FFF7FFFu;
+#pragma unroll
+    for (int i = 1; i < 8; ++i) mx = max_u16x2(mx, d[i] & 0x7FFF7FFFu);
+    mx = max(mx & 0xFFFFu, mx >> 16);
+    mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+    mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+    const float m = __uint_as_float(mx << 16);  // block absmax (exact)
+    uint32_t hE = 0u, hsig = 0u;  // the block's share of the exact sum: significand hsig at exponent bin hE
+    if (valid) {
+      if (qtr == 0) {
+        absmax[blk] = m;
+        const uint32_t u = __float_as_uint(m);
+        const uint32_t e = u >> 23;
+        const uint32_t mant7 = (u >> 16) & 0x7Fu;
+        hE = e ? e : 1u;
+        hsig = e ? (mant7 | 0x80u) : mant7;
+      }
+      uint32_t out[2];
+      if (m == 0.0f) {
+        out[0] = out[1] = 0x77777777u;  // an all-zero block: every code is the exact zero
+      } else {
+        // Keep 1/m normal: scale w and m by a power of two (exact for bf16 values;
+        // only weights whose quotient is below 2^-126 can lose bits, and those map
+        // to the zero code either way).
+        const bool rare = m < 5.421010862e-20f || m > 1.8446744e19f;  // outside [2^-64, 2^64]
+        if (!rare) {
+          encode16<false>(d, m, __frcp_rn(m), 1.0f, bins, out);
+        } else {
+          const float wsc = m < 5.421010862e-20f ? 1.8446744e19f : 5.421010862e-20f;
+          const float ms = m * wsc;
+          encode16<true>(d, ms, __frcp_rn(ms), wsc, bins, out);
+        }
+      }
+      *reinterpret_cast<uint2*>(packed + blk * 8 + qtr * 2) = make_uint2(out[0], out[1]);
+    }
+    const unsigned int same = __match_any_sync(0xffffffffu, hE);
+    const unsigned int tot = __reduce_add_sync(same, hsig);
+    if (lane == __ffs(same) - 1 && tot) atomicAdd(&s_hist[hE], tot);
+  }
 }
 
 __global__ void __launch_bounds__(kPass1Threads)
-k_quant_pass1(const uint4* __restrict__ W, int64_t n_items, uint32_t* __restrict__ packed,
-              float* __restrict__ absmax, unsigned long long* __restrict__ gbins, float* __restrict__ mean_out,
-              int64_t nblk, const __grid_constant__ QuantBinTable tab) {
+k_quant_pass1(const uint4* __restrict__ W, bool v8, uint32_t* __restrict__ packed,
+              float* __restrict__ absmax, unsigned int* __restrict__ hist_part, int64_t nblk,
+              const __grid_constant__ QuantBinTable tab) {
   __shared__ uint2 s_bins[kBins];
   __shared__ unsigned int s_hist[256];          // per-CTA significand sums (native 32-bit atomics)
-  __shared__ unsigned long long s_tot[256];
-  __shared__ int s_last;
   const int tid = threadIdx.x;
-  const int lane = tid & 31;
   if (tid < kBins) s_bins[tid] = make_uint2(__float_as_uint(tab.bins[tid].threshold), tab.bins[tid].j + 1u);
   s_hist[tid] = 0u;
   __syncthreads();
   pdl_enter();
 
-  const int64_t stride = static_cast<int64_t>(gridDim.x) * kPass1Threads;
-  for (int64_t base = static_cast<int64_t>(blockIdx.x) * kPass1Threads + tid; base - tid < n_items;
-       base += stride * kPass1Unroll) {
-    uint4 d[kPass1Unroll];
+  const unsigned char* bins = reinterpret_cast<const unsigned char*>(s_bins);
+  if (v8)
+    pass1_loop<true>(W, nblk, packed, absmax, bins, s_hist);
+  else
+    pass1_loop<false>(W, nblk, packed, absmax, bins, s_hist);
+  __syncthreads();
+  hist_part[static_cast<int64_t>(tid) * kQuantMaxGrid + blockIdx.x] = s_hist[tid];  // bin-major
+}
+
+// totals[e] = sum over the pass-1 CTAs of their bin e (one CTA per bin).
+__global__ void __launch_bounds__(128)
+k_quant_bins(const unsigned int* __restrict__ hist_part, int grid, unsigned long long* __restrict__ totals) {
+  __shared__ unsigned long long red[4];
+  pdl_enter();
+  const unsigned int* row = hist_part + static_cast<int64_t>(blockIdx.x) * kQuantMaxGrid;
+  unsigned long long v = 0ull;
+  for (int i = threadIdx.x; i < grid; i += blockDim.x) v += row[i];
 #pragma unroll
-    for (int u = 0; u < kPass1Unroll; ++u) {
-      const int64_t it = base + u * stride;
-      d[u] = (it < n_items) ? __ldcs(W + it) : make_uint4(0, 0, 0, 0);
-    }
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+  __syncthreads();
+  if (threadIdx.x == 0) totals[blockIdx.x] = red[0] + red[1] + red[2] + red[3];
+}
+
+// mu = fp32(RN_fp64(S) / nblk) from the exact bin totals (warp 0 of the CTA);
+// CTA 0 also stores it.
+__device__ float mean_from_bins(const unsigned long long* __restrict__ totals, int64_t nblk, float* mean_out) {
+  __shared__ unsigned long long s_tot[256];
+  __shared__ unsigned int s_mask[8];
+  __shared__ float s_mu;
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x;
 #pragma unroll
-    for (int u = 0; u < kPass1Unroll; ++u) {
-      const int64_t it = base + u * stride;
-      quant_item(d[u], it < n_items, lane, it, packed, absmax, s_bins, s_hist);
+    for (int k = 0; k < 8; ++k) {
+      const unsigned long long x = totals[32 * k + lane];
+      s_tot[32 * k + lane] = x;
+      const unsigned int m = __ballot_sync(0xffffffffu, x != 0ull);
+      if (lane == 0) s_mask[k] = m;
+    }
+    __syncwarp();
+    if (lane == 0) {
+      unsigned long long L[5] = {0, 0, 0, 0, 0};
+      for (int k = 0; k < 8; ++k) {
+        unsigned int m = s_mask[k];
+        while (m) {
+          const int b = __ffs(m) - 1;
+          m &= m - 1u;
+          acc_bin(L, s_tot[32 * k + b], 32 * k + b);
+        }
+      }
+      const double S = limbs_to_double(L);
+      const float mu = __double2float_rn(__ddiv_rn(S, static_cast<double>(nblk)));
+      s_mu = mu;
+      if (blockIdx.x == 0) *mean_out = mu;
     }
   }
   __syncthreads();
-  if (s_hist[tid]) atomicAdd(&gbins[tid], static_cast<unsigned long long>(s_hist[tid]));
-  __threadfence();
-  __syncthreads();
-  if (tid == 0) {
-    const unsigned long long t = atomicAdd(&gbins[256], 1ull);
-    s_last = (t == gridDim.x - 1) ? 1 : 0;
-  }
-  __syncthreads();
-  if (s_last) {
-    __threadfence();
-    s_tot[tid] = atomicAdd(&gbins[tid], 0ull);  // coherent read of the final bins
-    __syncthreads();
-    if (tid == 0) {
-      const double S = exact_sum_to_double(s_tot);
-      const double mu = __ddiv_rn(S, static_cast<double>(nblk));
-      *mean_out = __double2float_rn(mu);
-    }
-  }
+  return s_mu;
 }
 
 __global__ void __launch_bounds__(256)
-k_dq_quantize(const float* __restrict__ absmax, int64_t nblk, const float* __restrict__ mean,
-              int8_t* __restrict__ q, float* __restrict__ dq_scale, int64_t ngrp) {
+k_dq_quantize(const float* __restrict__ absmax, int64_t nblk, const unsigned long long* __restrict__ totals,
+              float* __restrict__ mean_out, int8_t* __restrict__ q, float* __restrict__ dq_scale, int64_t ngrp) {
   pdl_enter();
+  const float mu = mean_from_bins(totals, nblk, mean_out);
   const int lane = threadIdx.x & 31;
   const int64_t g = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
   if (g >= ngrp) return;  // whole warp leaves together
-  const float mu = *mean;
   const int64_t i0 = g * 256 + lane * 8;
   float c[8];
   bool ok[8];
@@ -272,30 +328,46 @@ k_dq_quantize(const float* __restrict__ absmax, int64_t nblk, const float* __res
 }  // namespace
 
 cudaError_t launch_quantize(const void* W, int64_t numel, uint8_t* packed, int8_t* absmax_q, float* dq_scale,
-                            float* mean, float* absmax_scratch, unsigned long long* bins, int num_sms,
+                            float* mean, float* absmax_scratch, void* hist_scratch, int num_sms,
                             cudaStream_t stream) {
   const QuantTables& tabs = quant_tables();
   QuantBinTable tab;
   for (int i = 0; i < kBins; ++i) tab.bins[i] = tabs.bins[i];
-  const int64_t n_items = numel / 8;
   const int64_t nblk = numel / 64;
   const int64_t ngrp = (nblk + 255) / 256;
+  unsigned int* hist_part = static_cast<unsigned int*>(hist_scratch);
+  unsigned long long* totals =
+      reinterpret_cast<unsigned long long*>(static_cast<char*>(hist_scratch) + kQuantHistBytes);
 
-  cudaError_t e = launch_pdl(k_quant_zero, dim3(1), dim3(320), 0, stream, bins);
-  if (e != cudaSuccess) return e;
-  int64_t want = (n_items + kPass1Threads * kPass1Unroll - 1) / (kPass1Threads * kPass1Unroll);
-  int64_t cap = static_cast<int64_t>(num_sms) * 8;
+  // four lanes per 64-weight block; a persistent grid of exactly the CTAs that
+  // are resident at once, so no SM idles through a partial last wave
+  static int per_sm = 0;
+  if (per_sm == 0) {
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k_quant_pass1, kPass1Threads, 0) != cudaSuccess || n < 1)
+      n = 4;
+    per_sm = n;
+  }
+  int64_t want = (nblk * 4 + kPass1Threads - 1) / kPass1Threads;
+  int64_t cap = static_cast<int64_t>(num_sms) * per_sm;
+  if (cap > kQuantMaxGrid) cap = kQuantMaxGrid;
   int64_t g = want < cap ? (want > 0 ? want : 1) : cap;
   // A CTA sums at most 2^24 significands of 8 bits, so its 32-bit bins cannot overflow.
   const int64_t min_grid = (nblk + (int64_t(1) << 24) - 1) >> 24;
   if (g < min_grid) g = min_grid;
+  if (g > kQuantMaxGrid) return cudaErrorInvalidValue;  // more than 2^35 blocks
   const int grid = static_cast<int>(g);
-  e = launch_pdl(k_quant_pass1, dim3(grid), dim3(kPass1Threads), 0, stream, reinterpret_cast<const uint4*>(W),
-                 n_items, reinterpret_cast<uint32_t*>(packed), absmax_scratch, bins, mean, nblk, tab);
+  const bool v8 = ((reinterpret_cast<uintptr_t>(W) | reinterpret_cast<uintptr_t>(packed)) & 31u) == 0;
+  cudaError_t e = launch_pdl(k_quant_pass1, dim3(grid), dim3(kPass1Threads), 0, stream,
+                             reinterpret_cast<const uint4*>(W), v8, reinterpret_cast<uint32_t*>(packed),
+                             absmax_scratch, hist_part, nblk, tab);
+  if (e != cudaSuccess) return e;
+  e = launch_pdl(k_quant_bins, dim3(256), dim3(128), 0, stream, static_cast<const unsigned int*>(hist_part), grid,
+                 totals);
   if (e != cudaSuccess) return e;
   const int dq_grid = static_cast<int>((ngrp + 7) / 8);
   return launch_pdl(k_dq_quantize, dim3(dq_grid), dim3(256), 0, stream, static_cast<const float*>(absmax_scratch),
-                    nblk, static_cast<const float*>(mean), absmax_q, dq_scale, ngrp);
+                    nblk, static_cast<const unsigned long long*>(totals), mean, absmax_q, dq_scale, ngrp);
 }
 
 }  // namespace qlora

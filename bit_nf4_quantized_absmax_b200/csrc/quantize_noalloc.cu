@@ -4,13 +4,13 @@
 // forbid allocation afterwards, and hosts where cudaMalloc's implicit device
 // synchronization would stall other work.
 //
-// The scratch the quantize kernels need (256 exponent bins + a CTA ticket, and
-// one fp32 absmax per 64-weight block) lives in a file-scope device array of a
+// The scratch the quantize kernels need (per-CTA exponent-bin sums and their
+// totals, and one fp32 absmax per 64-weight block) lives in a file-scope device array of a
 // fixed size. Every GPU that loads this code holds that array until the process
 // exits. All calls share it, so calls that overlap on the GPU (different
 // streams, or different host threads on one device) race and must be ordered by
-// the caller. The bins and ticket are cleared by the first kernel of every call;
-// the absmax region is fully written before it is read.
+// the caller. Every region is fully written by a kernel of the call before
+// another kernel of the call reads it.
 #include <mutex>
 
 #include "qlora.h"
@@ -21,9 +21,9 @@
 namespace {
 
 // At most 2^22 blocks of 64 weights (268,435,456 weights, e.g. any single
-// Llama-65B linear weight): 4 KiB of bins + 16 MiB of absmax per device.
+// Llama-65B linear weight): 2 MiB of bin sums + 16 MiB of absmax per device.
 constexpr int64_t kNoAllocMaxBlocks = int64_t(1) << 22;
-constexpr size_t kBinsBytes = 4096;
+constexpr size_t kBinsBytes = (qlora::kQuantScratchBytes + 255) / 256 * 256;
 constexpr size_t kScratchBytes = kBinsBytes + static_cast<size_t>(kNoAllocMaxBlocks) * sizeof(float);
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
@@ -86,7 +86,7 @@ extern "C" qlora_status qlora_quantize_nf4_dq_noalloc(const void* W_bf16, const 
   char* base = static_cast<char*>(scratch);
   cudaError_t e = qlora::launch_quantize(W_bf16, numel, q->packed, q->absmax_q, q->dq_scale, q->mean,
                                          reinterpret_cast<float*>(base + kBinsBytes),
-                                         reinterpret_cast<unsigned long long*>(base), sms,
+                                         base, sms,
                                          reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
 }
