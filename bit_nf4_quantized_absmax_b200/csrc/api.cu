@@ -91,7 +91,7 @@ int32_t* device_error_word() {
 int grad_splits(int64_t R, int rpad, int64_t M, int num_sms) {
   const int64_t tiles = ((R + 127) / 128) * (rpad / 64);
   if (tiles <= 0) return 1;
-  const int64_t nkb = 2 * ((M + 63) / 64);  // hi and lo halves
+  const int64_t nkb = (M + 63) / 64;  // each k-block multiplies by the hi and lo halves together
   const int64_t sp = (2 * num_sms) / tiles;  // at most one round of the two resident CTAs per SM
   return split_count(nkb, static_cast<int>(sp < 1 ? 1 : sp));
 }

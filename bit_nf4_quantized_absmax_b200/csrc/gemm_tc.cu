@@ -48,13 +48,17 @@ struct TileSched {
   int kb_per_split;
 };
 
-template <int BN>
+// DUAL: every k-block multiplies one A tile by two B tiles (B1 then B2) into
+// the same accumulator, e.g. X^T by the hi and lo halves of a split operand, so
+// that A is read once.
+template <int BN, bool DUAL = false>
 struct Cfg {
   static constexpr int A_BYTES = BM * BK * 2;
   static constexpr int B_BYTES = BN * BK * 2;
-  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  // BN = 64 (the rank-r contractions) keeps 4 stages so that two CTAs fit on an SM.
-  static constexpr int STAGES = BN == 64 ? 4 : ((200 * 1024) / STAGE_BYTES > 8 ? 8 : (200 * 1024) / STAGE_BYTES);
+  static constexpr int STAGE_BYTES = A_BYTES + (DUAL ? 2 : 1) * B_BYTES;
+  // BN = 64 (the rank-r contractions) keeps 4 stages (3 when dual) so that two CTAs fit on an SM.
+  static constexpr int STAGES =
+      BN == 64 ? (DUAL ? 3 : 4) : ((200 * 1024) / STAGE_BYTES > 8 ? 8 : (200 * 1024) / STAGE_BYTES);
   static constexpr int TMEM_COLS = (2 * BN) < 32 ? 32 : 2 * BN;
   static constexpr int SMEM = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
 };
@@ -131,12 +135,12 @@ __device__ __forceinline__ void decode_unit(const TileSched& ts, int unit, int& 
   kb1 = min(ts.nkb, kb0 + ts.kb_per_split);
 }
 
-template <int BN, bool A_MN, bool B_MN, int OUT>
+template <int BN, bool A_MN, bool B_MN, int OUT, bool DUAL = false>
 __global__ void __launch_bounds__(kThreads)
 k_tc_gemm(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmB1,
           const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2, TileSched ts,
           int M, int Nc, EpiParams ep, int32_t* err) {
-  using C = Cfg<BN>;
+  using C = Cfg<BN, DUAL>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
@@ -217,6 +221,15 @@ k_tc_gemm(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUte
           } else {
             tma_load_2d(sb, tb, &full[stage], k0, n0);
           }
+          if (DUAL) {  // the second B tile, same coordinates
+            if (B_MN) {
+#pragma unroll
+              for (int j = 0; j < BN / 64; ++j)
+                tma_load_2d(sb + C::B_BYTES + j * 8192, &tmB2, &full[stage], n0 + 64 * j, k0);
+            } else {
+              tma_load_2d(sb + C::B_BYTES, &tmB2, &full[stage], k0, n0);
+            }
+          }
           outstanding |= (1u << stage);
           out_parity = (out_parity & ~(1u << stage)) | (phase << stage);
           if (++stage == C::STAGES) {
@@ -262,6 +275,12 @@ k_tc_gemm(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUte
             const uint64_t da = A_MN ? smem_desc(sa + k * 2048, 8192, 1024) : smem_desc(sa + k * 32, 16, 1024);
             const uint64_t db = B_MN ? smem_desc(sb + k * 2048, 8192, 1024) : smem_desc(sb + k * 32, 16, 1024);
             mma_bf16(d_tmem, da, db, idesc, (kb > kb0 || k > 0) ? 1u : 0u);
+            if (DUAL) {
+              const uint32_t sb2 = sb + C::B_BYTES;
+              const uint64_t db2 =
+                  B_MN ? smem_desc(sb2 + k * 2048, 8192, 1024) : smem_desc(sb2 + k * 32, 16, 1024);
+              mma_bf16(d_tmem, da, db2, idesc, 1u);
+            }
           }
           mma_commit(&empty[stage]);  // frees the stage once these MMAs have read it
           if (++stage == C::STAGES) {
@@ -662,10 +681,10 @@ bool map_operand(CUtensorMap* m, const Operand& o, int tile_mn) {
   return make_map(m, o.p, o.k, o.rows_mn, o.ld, tile_mn);
 }
 
-template <int BN, bool A_MN, bool B_MN, int OUT>
+template <int BN, bool A_MN, bool B_MN, int OUT, bool DUAL = false>
 cudaError_t run(const Operand& a1, const Operand& b1, const Operand* a2, const Operand* b2, int M, int Nc,
                 int splits, const EpiParams& ep, int num_sms, int32_t* err, cudaStream_t stream) {
-  using C = Cfg<BN>;
+  using C = Cfg<BN, DUAL>;
   CUtensorMap ta1, tb1, ta2, tb2;
   if (!map_operand(&ta1, a1, BM) || !map_operand(&tb1, b1, BN)) return cudaErrorInvalidValue;
   if (a2 && b2) {
@@ -678,7 +697,8 @@ cudaError_t run(const Operand& a1, const Operand& b1, const Operand* a2, const O
   ts.tiles_m = static_cast<int>((M + BM - 1) / BM);
   ts.tiles_n = static_cast<int>((Nc + BN - 1) / BN);
   ts.nk1 = static_cast<int>((a1.k + BK - 1) / BK);
-  const int nk2 = (a2 && b2) ? static_cast<int>((a2->k + BK - 1) / BK) : 0;
+  // DUAL: b2 is the second B operand of every k-block, not a slab of its own
+  const int nk2 = (a2 && b2 && !DUAL) ? static_cast<int>((a2->k + BK - 1) / BK) : 0;
   ts.nkb = ts.nk1 + nk2;
   // callers pass a count from split_count(), so every piece is non-empty and the
   // number of partial slices written equals `splits`
@@ -688,7 +708,7 @@ cudaError_t run(const Operand& a1, const Operand& b1, const Operand* a2, const O
   const int units = ts.tiles_m * ts.tiles_n * ts.splits;
   const int slots = (BN == 64 ? 2 : 1) * num_sms;  // resident CTAs
   const int grid = units < slots ? units : slots;
-  auto kern = k_tc_gemm<BN, A_MN, B_MN, OUT>;
+  auto kern = k_tc_gemm<BN, A_MN, B_MN, OUT, DUAL>;
   static bool attr_set = false;
   if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
@@ -793,12 +813,14 @@ cudaError_t launch_gemm_lora_u(const void* dY, const void* Bl, int64_t M, int64_
 // with Q bf16 [M, R] (X for dA^T, dY for dB) and hi/lo bf16 [M, rpad].
 cudaError_t launch_gemm_lora_grad(const void* Q, int64_t R, const void* hi, const void* lo, int64_t M, int rpad,
                                   float* P, int splits, int num_sms, int32_t* err, cudaStream_t stream) {
+  // Q^T [R, M] times hi and lo [M, rpad]: each k-block of Q is read once and
+  // multiplied by both halves
   Operand a1{Q, R, M, R, true}, b1{hi, rpad, M, rpad, true};
-  Operand a2{Q, R, M, R, true}, b2{lo, rpad, M, rpad, true};
+  Operand b2{lo, rpad, M, rpad, true};
   EpiParams ep{};
   ep.P = P;
-  return run<64, true, true, OUT_PARTIAL>(a1, b1, &a2, &b2, static_cast<int>(R), rpad, splits, ep, num_sms, err,
-                                          stream);
+  return run<64, true, true, OUT_PARTIAL, true>(a1, b1, &a1, &b2, static_cast<int>(R), rpad, splits, ep, num_sms,
+                                                err, stream);
 }
 
 }  // namespace qlora
