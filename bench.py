@@ -324,6 +324,34 @@ def breakdown(work, dev, reps=24):
     return out
 
 
+def merge_measure(work, dev, reps=10):
+    """Adapter merge (SURVEY next item, outside the step): one r = 64 adapter
+    merged into the 11008x4096 base, W' + s B A in fp64, back to back."""
+    import ctypes
+    lib = qb.load_library()
+    st = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    d = work.lin[SHAPES.index(ROOFLINE_SHAPE)]
+    N, K = d["N"], d["K"]
+    out = d["Wd"]
+    arr = (qb._Adapter * 1)(qb._Adapter(qb._ptr(d["A"]), qb._ptr(d["B"]), R, ALPHA, 1.0))
+    qc = d["q"].as_c()
+    call = lambda: lib.qlora_merge_lora(ctypes.byref(qc), arr, 1, qb._ptr(out), st)  # noqa: E731
+    for _ in range(2):
+        call()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(reps):
+        if call() != 0:
+            raise qb.QloraError(1, "qlora_merge_lora")
+    b.record()
+    torch.cuda.synchronize()
+    us = 1e3 * a.elapsed_time(b) / reps
+    flops = 2.0 * R * N * K
+    return {"shape": f"{N}x{K}", "r": R, "us": round(us, 1), "fp64_TFLOP_s": round(flops / us / 1e6, 2),
+            "peak_fp64_TFLOP_s": 40.0, "peak_kind": "nominal B200 fp64 (no measured figure)",
+            "frac": round(flops / us / 1e6 / 40.0, 4)}
+
+
 def run_ours(args, rank, world, dev):
     def say(msg):  # progress on stderr (stdout carries only the JSON line)
         if args.verbose or rank == 0:
@@ -405,6 +433,8 @@ def run_ours(args, rank, world, dev):
             "us_per_launch": round(fwd_us, 2)}
     dec = [parts[f"decode{M}/{N}x{K}"]["weight_GB_s"] for M in M_DECODE for N, K in SHAPES]
 
+    say("adapter merge")
+    merge = merge_measure(work, dev)
     say("end to end with host buffers")
     # end to end through the C ABI with host buffers
     host = []
@@ -444,6 +474,7 @@ def run_ours(args, rank, world, dev):
         "hbm_frac": {k: round(v["GB_s"] / peaks["hbm_gbs"], 4) for k, v in parts.items() if "GB_s" in v},
         "parts": parts,
         "roofline": roof,
+        "merge": merge,
         "e2e": {"value": round(world * fl_train / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
                 "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": work.launches_per_step() * args.steps,

@@ -22,7 +22,7 @@ STATUS_NAMES = {0: "QLORA_OK", 1: "QLORA_ERR_INVALID_ARG", 2: "QLORA_ERR_UNSUPPO
 
 EXPORTED = ("qlora_status_string", "qlora_nf4_codebook", "qlora_nf4_storage_bytes", "qlora_quantize_nf4_dq",
             "qlora_quantize_nf4_dq_noalloc", "qlora_dequantize_nf4_dq", "qlora_linear_fwd", "qlora_linear_bwd",
-            "qlora_device_error")
+            "qlora_merge_lora", "qlora_device_error")
 
 
 class QloraError(RuntimeError):
@@ -38,6 +38,11 @@ class _Weight(ctypes.Structure):
 
 
 _lib = None
+
+
+class _Adapter(ctypes.Structure):
+    _fields_ = [("A", ctypes.c_void_p), ("B", ctypes.c_void_p), ("r", ctypes.c_int32), ("alpha", ctypes.c_float),
+                ("weight", ctypes.c_float)]
 
 
 def load_library(path: str | None = None) -> ctypes.CDLL:
@@ -61,6 +66,7 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
     lib.qlora_dequantize_nf4_dq.argtypes = [wp, vp, vp]
     lib.qlora_linear_fwd.argtypes = [wp, vp, i64, vp, vp, i32, f32, vp, vp, vp, szp, vp]
     lib.qlora_linear_bwd.argtypes = [wp, vp, i64, vp, vp, i32, f32, vp, vp, vp, vp, vp, vp, szp, vp]
+    lib.qlora_merge_lora.argtypes = [wp, ctypes.POINTER(_Adapter), i32, vp, vp]
     lib.qlora_device_error.argtypes = [ctypes.POINTER(ctypes.c_int32), vp]
     for name in EXPORTED:
         getattr(lib, name).restype = ctypes.c_int if name != "qlora_status_string" else ctypes.c_char_p
@@ -207,6 +213,21 @@ def qlora_linear_bwd(q: NF4Weight, X: torch.Tensor, A: torch.Tensor, B: torch.Te
     ws, nbytes = _workspace(args, workspace, dev)
     _check(args(_ptr(ws), ctypes.byref(nbytes)), "qlora_linear_bwd")
     return (dX if need_dX else None), dA, dB
+
+
+def qlora_merge_lora(q: NF4Weight, adapters, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Merged bf16 weight [rows, cols] from the NF4 base and a sequence of
+    adapters (A [r, cols], B [rows, r], alpha, weight); see include/qlora.h."""
+    lib = load_library()
+    if out is None:
+        out = torch.empty(q.rows, q.cols, dtype=torch.bfloat16, device=q.packed.device)
+    arr = (_Adapter * max(1, len(adapters)))()
+    for i, (A, B, alpha, weight) in enumerate(adapters):
+        arr[i] = _Adapter(_ptr(A), _ptr(B), A.shape[0], float(alpha), float(weight))
+    qc = q.as_c()
+    _check(lib.qlora_merge_lora(ctypes.byref(qc), arr, len(adapters), _ptr(out), _stream(stream)),
+           "qlora_merge_lora")
+    return out
 
 
 def qlora_device_error(stream=None) -> int:

@@ -314,6 +314,35 @@ qlora_status qlora_linear_bwd(const qlora_nf4_weight* q, const void* X, int64_t 
   return cuda_status(e);
 }
 
+qlora_status qlora_merge_lora(const qlora_nf4_weight* q, const qlora_lora_adapter* adapters,
+                              int32_t n_adapters, void* W_out, qlora_stream_t stream) {
+  qlora_status st = check_weight(q, false);
+  if (st != QLORA_OK) return st;
+  if (n_adapters < 0 || (n_adapters > 0 && !adapters)) return QLORA_ERR_INVALID_ARG;
+  if (n_adapters > kMaxMergeAdapters) return QLORA_ERR_UNSUPPORTED;
+  MergeAdapter ma[kMaxMergeAdapters];
+  for (int a = 0; a < n_adapters; ++a) {
+    const qlora_lora_adapter& ad = adapters[a];
+    if (ad.r < 8 || ad.r > 256 || ad.r % 8) return QLORA_ERR_UNSUPPORTED;
+    if (!ad.A || !ad.B) return QLORA_ERR_INVALID_ARG;
+    if (!aligned(ad.A, 16) || !aligned(ad.B, 16)) return QLORA_ERR_ALIGNMENT;
+    ma[a].A = ad.A;
+    ma[a].B = ad.B;
+    ma[a].r = ad.r;
+    ma[a].c = ad.weight * lora_scale(ad.alpha, ad.r);  // fp32(w * s)
+  }
+  const int64_t numel = q->rows * q->cols;
+  if (numel == 0) return QLORA_OK;
+  if (!W_out) return QLORA_ERR_INVALID_ARG;
+  if (!aligned(W_out, 16)) return QLORA_ERR_ALIGNMENT;
+  if ((q->rows + 63) / 64 > 65535) return QLORA_ERR_UNSUPPORTED;
+  DeviceInfo di;
+  if ((st = device_info(&di)) != QLORA_OK) return st;
+  Nf4View w{q->packed, q->absmax_q, q->dq_scale, q->mean, q->rows, q->cols};
+  return cuda_status(launch_merge(w, ma, n_adapters, W_out, quant_tables().codebook, di.num_sms,
+                                  reinterpret_cast<cudaStream_t>(stream)));
+}
+
 qlora_status qlora_device_error(int32_t* code, qlora_stream_t stream) {
   if (!code) return QLORA_ERR_INVALID_ARG;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);

@@ -66,6 +66,18 @@ cudaError_t launch_decode_fwd(const Nf4View& w, const void* X, int64_t M, const 
                               float s, void* Y, float* T, float* partial, unsigned int* counters,
                               const DecodePlan& p, const float codebook[16], int32_t* err, cudaStream_t stream);
 
+// ---- merge.cu: weighted LoRA adapters merged into the dequantized base ----
+constexpr int kMaxMergeAdapters = 8;
+struct MergeAdapter {
+  const void* A;  // bf16 [r, K]
+  const void* B;  // bf16 [N, r]
+  int r;
+  float c;        // fp32(weight * s)
+};
+// out (bf16 [N, K]) = bf16_rn(W' + sum_a c_a B_a A_a), sums in fp64 (order in merge.cu).
+cudaError_t launch_merge(const Nf4View& w, const MergeAdapter* adapters, int n_adapters, void* out,
+                         const float codebook[16], int num_sms, cudaStream_t stream);
+
 // ---- gemm_tc.cu: tcgen05 GEMMs ----
 cudaError_t launch_gemm_fwd(const void* X, const void* Wd, const void* sT, const void* Bl, int64_t M, int64_t N,
                             int64_t K, int r, int rpad, void* Y, int num_sms, int32_t* err, cudaStream_t stream);

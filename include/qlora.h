@@ -7,7 +7,8 @@
  *   3. double quantization of the fp32 absmax constants to int8 codes,
  *   4. block-wise dequantization back to bf16,
  *   5. the QLoRA linear layer  Y = X W'^T + s (X A^T) B^T  (W' = dequant(W)),
- *      forward and backward (dX, dA, dB; W stays frozen, no dW).
+ *      forward and backward (dX, dA, dB; W stays frozen, no dW),
+ *   6. merging weighted LoRA adapters into the base weight.
  *
  * Sources (web pages describing the method; no code is printed on them):
  *   [G]  "Guanaco" (chipfoundryservices.com/topic/guanaco), sections
@@ -17,8 +18,9 @@
  *        p.5 Section 3.
  *   [C]  "QLoRA vs ChatGPT" (unfragile.ai compare page), capability blurbs
  *        1 (NF4, block-wise absmax), 2 (LoRA on a frozen 4-bit base),
- *        3 (double quantization) and 5 (on-the-fly block-wise dequantization,
- *        gradients only for the LoRA parameters).
+ *        3 (double quantization), 5 (on-the-fly block-wise dequantization,
+ *        gradients only for the LoRA parameters) and 6 (adapter composition
+ *        and merging).
  *
  * Conventions for every call below:
  *   - bf16 tensors are passed as void*, row-major and contiguous, with base
@@ -198,6 +200,34 @@ qlora_status qlora_linear_bwd(const qlora_nf4_weight* q, const void* X, int64_t 
                               void* dX, void* dA, void* dB,
                               void* workspace, size_t* workspace_bytes,
                               qlora_stream_t stream);
+
+/* One LoRA adapter of a merge: A [r, cols] and B [rows, r] (device bf16,
+ * 16-byte aligned, row-major), 8 <= r <= 256 with r % 8 == 0, scale
+ * s = (float)alpha / (float)r, composition weight w. */
+typedef struct {
+  const void* A;
+  const void* B;
+  int32_t r;
+  float alpha;
+  float weight;
+} qlora_lora_adapter;
+
+/* qlora_merge_lora -- merge weighted adapters into the frozen base ([C] 6:
+ * adapters trained on one quantized base are composed with weights and merged
+ * into the base weights to give a standalone checkpoint):
+ *   W_out = bf16_rn( W' + sum_a c_a (B_a A_a) ),  c_a = fp32(w_a * s_a),
+ * evaluated in fp64 in a fixed order (for each element: start from W', then for
+ * a = 0, 1, ...: P = sum over j = 0 .. r_a - 1 of B_a[n, j] A_a[j, k] added in
+ * that order, y = y + c_a * P), rounded once to bf16 (nearest, ties to even).
+ *   q         : the base weight, W' = dequant(q), [rows, cols].
+ *   adapters  : host array of n_adapters entries (read before returning);
+ *               0 <= n_adapters <= 8 (0 writes W' itself).
+ *   W_out     : device bf16 [rows, cols] (16-byte aligned), overwritten.
+ * The merged weight can be re-quantized with qlora_quantize_nf4_dq.
+ * Errors: INVALID_ARG, UNSUPPORTED (r out of range, more than 8 adapters),
+ * ALIGNMENT, CUDA, DEVICE. */
+qlora_status qlora_merge_lora(const qlora_nf4_weight* q, const qlora_lora_adapter* adapters,
+                              int32_t n_adapters, void* W_out, qlora_stream_t stream);
 
 /* qlora_device_error -- read and clear the library's device-side error word on
  * the current device (synchronizes the stream). Kernels whose waits on

@@ -99,3 +99,23 @@ def test_argument_errors_return_before_launch():
     assert lib.qlora_dequantize_nf4_dq(ctypes.byref(_weight(rows=0)), None, None) == 0
     code = ctypes.c_int32(0)
     assert lib.qlora_device_error(None, None) == 1
+
+
+def test_merge_argument_errors_return_before_launch():
+    lib = b.load_library()
+    w = _weight()
+    fake = 1 << 20
+    out = ctypes.c_void_p(fake)
+    ok = b._Adapter(fake, fake, 16, 16.0, 1.0)
+    arr = (b._Adapter * 9)(*([ok] * 9))
+    assert lib.qlora_merge_lora(None, arr, 1, out, None) == 1                       # no weight
+    assert lib.qlora_merge_lora(ctypes.byref(w), None, 1, out, None) == 1           # no adapter array
+    assert lib.qlora_merge_lora(ctypes.byref(w), arr, -1, out, None) == 1           # negative count
+    assert lib.qlora_merge_lora(ctypes.byref(w), arr, 9, out, None) == 2            # more than 8 adapters
+    for bad, code in ((b._Adapter(fake, fake, 12, 16.0, 1.0), 2), (b._Adapter(fake, fake, 512, 16.0, 1.0), 2),
+                      (b._Adapter(None, fake, 16, 16.0, 1.0), 1), (b._Adapter(fake + 8, fake, 16, 16.0, 1.0), 3)):
+        one = (b._Adapter * 1)(bad)
+        assert lib.qlora_merge_lora(ctypes.byref(w), one, 1, out, None) == code
+    assert lib.qlora_merge_lora(ctypes.byref(w), arr, 1, None, None) == 1            # no output
+    assert lib.qlora_merge_lora(ctypes.byref(w), arr, 1, ctypes.c_void_p(fake + 2), None) == 3  # misaligned output
+    assert lib.qlora_merge_lora(ctypes.byref(_weight(rows=0)), arr, 1, None, None) == 0  # empty weight
