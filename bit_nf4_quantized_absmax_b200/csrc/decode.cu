@@ -42,10 +42,10 @@ __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// x >> 16 and x >> 1 as high halves of products, so they can issue on the
-// multiply-add pipe instead of the integer ALU that the lookups saturate.
-__device__ __forceinline__ uint32_t hi16(uint32_t x) { return __umulhi(x, 0x10000u); }
-__device__ __forceinline__ uint32_t shr1(uint32_t x) { return __umulhi(x, 0x80000000u); }
+// (Writing these shifts as high halves of products, to move them off the
+// integer ALU, measured 4% slower than plain shifts.)
+__device__ __forceinline__ uint32_t hi16(uint32_t x) { return x >> 16; }
+__device__ __forceinline__ uint32_t shr1(uint32_t x) { return x >> 1; }
 
 // Byte-permute lookup of four codes with precomputed selectors: `s` holds the
 // low three bits of each code (nibbles 0..3), `sel` picks the table half by
