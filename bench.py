@@ -419,6 +419,9 @@ def run_ours(args, rank, world, dev):
     if not args.no_graph:
         say("timed region (CUDA graph replay)")
         graph = capture_step_graph(work, say)
+        # every rank takes the same collective steps: replay only if all captured
+        if world > 1 and max_over_ranks(0.0 if graph is not None else 1.0, world, dev) > 0.0:
+            graph = None
         if graph is not None:
             for _ in range(3):
                 graph.replay()
