@@ -58,6 +58,15 @@ __device__ __forceinline__ void lookup4_sel(const Nf4Lut& L, uint32_t s, uint32_
   o23 = prmt(lo, hi, 0x7362);
 }
 
+// Orders this thread's generic-proxy reads of shared memory before later
+// async-proxy writes (TMA) to it. The consumer warps read the TMA-filled stages
+// with ordinary loads, so each executes it before releasing a stage for the
+// next copy; without it, a copy into a released stage was seen to overwrite
+// token values that a warp had not read yet.
+__device__ __forceinline__ void fence_proxy_async_shared() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // Owner unit of item i when n_items items are cut into n_units ranges
 // [u * n_items / n_units, (u + 1) * n_items / n_units).
 __host__ __device__ __forceinline__ int64_t item_owner(int64_t i, int64_t n_items, int64_t n_units) {
@@ -113,16 +122,19 @@ __device__ __forceinline__ void publish_segment(const float (&acc)[2][MT][4], in
       y[m][0] += v.x; y[m][1] += v.y; y[m][2] += v.z; y[m][3] += v.w;
     }
   }
-  // LoRA up: rows of B are the A operand, T^T (split into bf16 hi + lo) the B operand.
+  // LoRA up: rows of B are the A operand, T^T (split into bf16 hi + lo) the B
+  // operand. A step covers ranks j0 .. j0 + 15; since r % 8 == 0 its upper half
+  // is either wholly inside [0, r) or wholly outside (and then zero).
   const int64_t na = tile * 16 + g, nb = na + 8;
   float l[MT][4];
 #pragma unroll
   for (int m = 0; m < MT; ++m) l[m][0] = l[m][1] = l[m][2] = l[m][3] = 0.0f;
   for (int j0 = 0; j0 < r; j0 += 16) {
+    const bool hi_in = j0 + 8 < r;
     const uint32_t b_a0 = na < N ? *reinterpret_cast<const uint32_t*>(Bl + na * r + j0 + 2 * t) : 0u;
-    const uint32_t b_a2 = na < N ? *reinterpret_cast<const uint32_t*>(Bl + na * r + j0 + 2 * t + 8) : 0u;
+    const uint32_t b_a2 = na < N && hi_in ? *reinterpret_cast<const uint32_t*>(Bl + na * r + j0 + 2 * t + 8) : 0u;
     const uint32_t b_a1 = nb < N ? *reinterpret_cast<const uint32_t*>(Bl + nb * r + j0 + 2 * t) : 0u;
-    const uint32_t b_a3 = nb < N ? *reinterpret_cast<const uint32_t*>(Bl + nb * r + j0 + 2 * t + 8) : 0u;
+    const uint32_t b_a3 = nb < N && hi_in ? *reinterpret_cast<const uint32_t*>(Bl + nb * r + j0 + 2 * t + 8) : 0u;
 #pragma unroll
     for (int m = 0; m < MT; ++m) {
       const int tok = g + 8 * m;
@@ -131,8 +143,10 @@ __device__ __forceinline__ void publish_segment(const float (&acc)[2][MT][4], in
         const float* tp = T + static_cast<int64_t>(tok) * r + j0 + 2 * t;
         tv[0] = __ldcg(tp);
         tv[1] = __ldcg(tp + 1);
-        tv[2] = __ldcg(tp + 8);
-        tv[3] = __ldcg(tp + 9);
+        if (hi_in) {
+          tv[2] = __ldcg(tp + 8);
+          tv[3] = __ldcg(tp + 9);
+        }
       }
       uint32_t hi[2], lo[2];
 #pragma unroll
@@ -330,6 +344,7 @@ k_decode(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUten
           }
         }
       }
+      fence_proxy_async_shared();  // this warp's reads of the stage precede the next TMA into it
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[stage]);  // this warp is done with the stage
       if (++stage == kStages) {

@@ -105,6 +105,31 @@ def test_decode_ragged(N, K):
     assert b.qlora_device_error() == 0
 
 
+@pytest.mark.parametrize("r", [8, 24, 72])
+def test_decode_ranks_not_multiple_of_16(r):
+    """Decode forward with r % 16 == 8: the LoRA-up runs in 16-rank steps, and the
+    upper half of the last step lies outside the adapter. With W = 0 the output is
+    the LoRA term alone (a zero weight dequantizes to exact zeros), so a wrong
+    rank anywhere in it shows."""
+    dev = require_gpu()
+    for M in (1, 9, 16):
+        inp = syn.make_linear(136, 320, M, r=r, alpha=16.0, seed=6, workload="test", dy_std=1.0)
+        Xn, An, Bn = (bf16_to_f32_np(t).astype(np.float64) for t in (inp.X, inp.A, inp.B))
+        s = oracle.lora_scale(inp.alpha, inp.r)
+        for zero_w in (True, False):
+            W = torch.zeros_like(inp.W) if zero_w else inp.W
+            X, A, B = (t.to(dev).contiguous() for t in (inp.X, inp.A, inp.B))
+            q = b.qlora_quantize_nf4_dq(W.to(dev))
+            Y, T = b.qlora_linear_fwd(q, X, A, B, inp.alpha, T_save=True)
+            torch.cuda.synchronize()
+            Wd = np.zeros((136, 320)) if zero_w else _oracle_wd(inp.W)
+            Yr, Tr = oracle.linear_fwd(Wd, Xn, An, Bn, s)
+            ok, err = gemm_close(bf16_to_f32_np(Y), Yr)
+            assert ok, (M, zero_w, err)
+            assert rel_fro(T.cpu().numpy().astype(np.float64), Tr) < 1e-5
+    assert b.qlora_device_error() == 0
+
+
 def test_recomputed_T_matches_saved_T_path():
     inp = syn.make_linear(512, 768, 300, r=32, alpha=16.0, seed=4, workload="test", dy_std=0.5)
     _check_full(inp, use_saved_T=False)
@@ -142,7 +167,8 @@ def test_llama7b_decode_full_size(shape):
         Wd = _oracle_wd_cached(("llama7b", shape), inp.W)
         Xn, An, Bn = (bf16_to_f32_np(t).astype(np.float64) for t in (inp.X, inp.A, inp.B))
         Yr, _ = oracle.linear_fwd(Wd, Xn, An, Bn, oracle.lora_scale(inp.alpha, inp.r))
-        assert gemm_close(bf16_to_f32_np(Y), Yr)[0]
+        ok, err = gemm_close(bf16_to_f32_np(Y), Yr)
+        assert ok, (M, err)
 
 
 @pytest.mark.parametrize("shape", syn.LLAMA7B_SHAPES)
