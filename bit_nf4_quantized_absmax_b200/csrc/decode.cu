@@ -491,12 +491,8 @@ cudaError_t launch_decode_fwd(const Nf4View& w, const void* X, int64_t M, const 
   const int Mi = static_cast<int>(M);
   auto kern = p.mt == 1 ? k_decode<1> : k_decode<2>;
   const int smem = decode_smem_bytes(p.mt);
-  static bool smem_set[2] = {false, false};
-  if (!smem_set[p.mt - 1]) {
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    smem_set[p.mt - 1] = true;
-  }
+  e = p.mt == 1 ? ensure_smem_limit<k_decode<1>>(smem) : ensure_smem_limit<k_decode<2>>(smem);
+  if (e != cudaSuccess) return e;
   e = launch_pdl(kern, dim3(p.grid), dim3((kDecodeWarps + 1) * 32), smem, stream, tw, tx, w.absmax_q, w.dq_scale,
                  w.mean, Mi, w.N, w.K, static_cast<const float*>(T), Bb, r, s, Yb, partial, counters, p.n_items,
                  static_cast<int64_t>(p.grid), p.max_seg, err, cb);

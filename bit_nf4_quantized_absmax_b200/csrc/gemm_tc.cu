@@ -709,12 +709,8 @@ cudaError_t run(const Operand& a1, const Operand& b1, const Operand* a2, const O
   const int slots = (BN == 64 ? 2 : 1) * num_sms;  // resident CTAs
   const int grid = units < slots ? units : slots;
   auto kern = k_tc_gemm<BN, A_MN, B_MN, OUT, DUAL>;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  const cudaError_t e = ensure_smem_limit<k_tc_gemm<BN, A_MN, B_MN, OUT, DUAL>>(C::SMEM);
+  if (e != cudaSuccess) return e;
   return launch_pdl(kern, dim3(grid), dim3(kThreads), C::SMEM, stream, ta1, tb1, ta2, tb2, ts, M, Nc, ep, err);
 }
 
@@ -738,12 +734,8 @@ cudaError_t run_pair(const Operand& a1, const Operand& b1, const Operand& a2, co
   if (pairs > units) pairs = units;
   if (pairs < 1) pairs = 1;
   auto kern = k_tc_gemm2<B_MN>;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  const cudaError_t e = ensure_smem_limit<k_tc_gemm2<B_MN>>(C::SMEM);
+  if (e != cudaSuccess) return e;
   return launch_pdl(kern, dim3(2 * pairs), dim3(kThreads), C::SMEM, stream, ta1, tb1, ta2, tb2, ts, M, Nc, ep, err);
 }
 

@@ -2,11 +2,28 @@
 // enqueue on `stream` and return the launch status (cudaGetLastError()).
 #pragma once
 
+#include <atomic>
 #include <cstddef>
 #include <cstdint>
 #include <cuda_runtime.h>
 
 namespace qlora {
+
+// Raises a kernel's dynamic shared memory limit once per device, safely from
+// several host threads: one flag bit per device ordinal (for ordinals above 63
+// the attribute is set on every call).
+template <auto Kern>
+cudaError_t ensure_smem_limit(int bytes) {
+  static std::atomic<unsigned long long> done{0};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const unsigned long long bit = dev < 64 ? (1ull << dev) : 0ull;
+  if (bit && (done.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+  e = cudaFuncSetAttribute(Kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) done.fetch_or(bit, std::memory_order_release);
+  return e;
+}
 
 // Quantize scratch besides the fp32 absmax: per-CTA exponent-bin sums of the
 // first pass (u32 [256][kQuantMaxGrid], bin-major) and the 256 bin totals (u64).

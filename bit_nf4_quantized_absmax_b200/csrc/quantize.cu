@@ -341,12 +341,13 @@ cudaError_t launch_quantize(const void* W, int64_t numel, uint8_t* packed, int8_
 
   // four lanes per 64-weight block; a persistent grid of exactly the CTAs that
   // are resident at once, so no SM idles through a partial last wave
-  static int per_sm = 0;
+  static std::atomic<int> per_sm_cache{0};  // the same on every B200; racing writers store equal values
+  int per_sm = per_sm_cache.load(std::memory_order_relaxed);
   if (per_sm == 0) {
-    int n = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k_quant_pass1, kPass1Threads, 0) != cudaSuccess || n < 1)
-      n = 4;
-    per_sm = n;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_quant_pass1, kPass1Threads, 0) != cudaSuccess ||
+        per_sm < 1)
+      per_sm = 4;
+    per_sm_cache.store(per_sm, std::memory_order_relaxed);
   }
   int64_t want = (nblk * 4 + kPass1Threads - 1) / kPass1Threads;
   int64_t cap = static_cast<int64_t>(num_sms) * per_sm;
