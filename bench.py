@@ -65,12 +65,17 @@ def train_flops(N, K, M=M_TRAIN, r=R):
     return fwd, bwd
 
 
-def decode_bytes(N, K, M, r=R):
-    return 0.515869 * N * K + 2 * r * (K + N) + 2 * M * (K + N)
+def decode_bytes(N, K, M, r=R, single=False):
+    return weight_bytes(N, K, single) + 2 * r * (K + N) + 2 * M * (K + N)
 
 
-def quant_bytes(N, K):
-    return 2.516 * N * K  # read bf16 W, write codes + int8 constants + scales
+def quant_bytes(N, K, single=False):
+    # read bf16 W, write codes + int8 constants + scales (single-level: + fp32 constants)
+    return (2.5625 if single else 2.516) * N * K
+
+
+def weight_bytes(N, K, single=False):
+    return (0.5625 if single else 0.515869) * N * K
 
 
 def load_peaks():
@@ -319,6 +324,20 @@ def breakdown(work, dev, reps=24):
                 ctypes.byref(n), st) for qc in qcs])
         timed(f"train_fwd/{li}", [lambda d=d: work._fwd_call(lib, d, ws, n, st, M_TRAIN)])
         timed(f"train_bwd/{li}", [lambda d=d: work._bwd_call(lib, d, ws, n, st, M_TRAIN)])
+        if li == 1:  # single-level storage (fp32 block constants), outside the step: one shape
+            ns = max(2, math.ceil(2 * l2 / (0.5625 * N * K)))
+            ss = [qb.qlora_quantize_nf4(d["W"]) for _ in range(ns)]
+            scs = [q.as_c() for q in ss]
+            timed(f"quantize_single/{li}", [lambda i=i: lib.qlora_quantize_nf4(
+                qb._ptr(Ws[i % nw]), ctypes.byref(scs[i % ns]), st) for i in range(max(nw, ns))])
+            timed(f"dequantize_single/{li}", [lambda i=i: lib.qlora_dequantize_nf4(
+                ctypes.byref(scs[i % ns]), qb._ptr(Wds[i % nw]), st) for i in range(max(nw, ns))])
+            for M in M_DECODE:
+                X, Y = d["Xdec"][M], d["Ydec"][M]
+                timed(f"decode{M}_single/{li}", [lambda qc=qc, X=X, Y=Y, M=M: lib.qlora_linear_fwd(
+                    ctypes.byref(qc), qb._ptr(X), M, qb._ptr(d["A"]), qb._ptr(d["B"]), R, ALPHA, qb._ptr(Y), None,
+                    ws, ctypes.byref(n), st) for qc in scs])
+            del ss, scs
         del Ws, Wds, qs, qcs
         torch.cuda.empty_cache()
     return out
@@ -344,7 +363,7 @@ def capture_step_graph(work, say):
 
 
 def merge_measure(work, dev, reps=10):
-    """Adapter merge (SURVEY next item, outside the step): one r = 64 adapter
+    """Adapter merge (outside the step): one r = 64 adapter
     merged into the 11008x4096 base, W' + s B A in fp64, back to back."""
     import ctypes
     lib = qb.load_library()
@@ -453,12 +472,14 @@ def run_ours(args, rank, world, dev):
         kind, li = part.split("/")
         N, K = SHAPES[int(li)]
         e = {"us": round(us, 2)}
-        if kind in ("quantize", "dequantize"):
-            e["GB_s"] = round(quant_bytes(N, K) / us / 1e3, 1)
-        elif kind.startswith("decode"):
-            M = int(kind[len("decode"):])
-            e["GB_s"] = round(decode_bytes(N, K, M) / us / 1e3, 1)
-            e["weight_GB_s"] = round(0.515869 * N * K / us / 1e3, 1)
+        single = kind.endswith("_single")
+        base = kind[: -len("_single")] if single else kind
+        if base in ("quantize", "dequantize"):
+            e["GB_s"] = round(quant_bytes(N, K, single) / us / 1e3, 1)
+        elif base.startswith("decode"):
+            M = int(base[len("decode"):])
+            e["GB_s"] = round(decode_bytes(N, K, M, single=single) / us / 1e3, 1)
+            e["weight_GB_s"] = round(weight_bytes(N, K, single) / us / 1e3, 1)
         else:
             f = train_flops(N, K)[0 if kind == "train_fwd" else 1]
             e["TFLOP_s"] = round(f / us / 1e6, 1)

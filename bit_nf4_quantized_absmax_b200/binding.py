@@ -20,9 +20,10 @@ QLORA_OK = 0
 STATUS_NAMES = {0: "QLORA_OK", 1: "QLORA_ERR_INVALID_ARG", 2: "QLORA_ERR_UNSUPPORTED", 3: "QLORA_ERR_ALIGNMENT",
                 4: "QLORA_ERR_CUDA", 5: "QLORA_ERR_WORKSPACE", 6: "QLORA_ERR_DEVICE"}
 
-EXPORTED = ("qlora_status_string", "qlora_nf4_codebook", "qlora_nf4_storage_bytes", "qlora_quantize_nf4_dq",
-            "qlora_quantize_nf4_dq_noalloc", "qlora_dequantize_nf4_dq", "qlora_linear_fwd", "qlora_linear_bwd",
-            "qlora_merge_lora", "qlora_device_error")
+EXPORTED = ("qlora_status_string", "qlora_nf4_codebook", "qlora_nf4_storage_bytes", "qlora_nf4_single_storage_bytes",
+            "qlora_quantize_nf4", "qlora_quantize_nf4_dq", "qlora_quantize_nf4_dq_noalloc", "qlora_dequantize_nf4",
+            "qlora_dequantize_nf4_dq", "qlora_linear_fwd", "qlora_linear_bwd", "qlora_merge_lora",
+            "qlora_device_error")
 
 
 class QloraError(RuntimeError):
@@ -34,7 +35,7 @@ class QloraError(RuntimeError):
 class _Weight(ctypes.Structure):
     _fields_ = [("packed", ctypes.c_void_p), ("absmax_q", ctypes.c_void_p), ("dq_scale", ctypes.c_void_p),
                 ("mean", ctypes.c_void_p), ("rows", ctypes.c_int64), ("cols", ctypes.c_int64),
-                ("blocksize", ctypes.c_int32), ("dq_blocksize", ctypes.c_int32)]
+                ("blocksize", ctypes.c_int32), ("dq_blocksize", ctypes.c_int32), ("absmax", ctypes.c_void_p)]
 
 
 _lib = None
@@ -61,6 +62,9 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
     lib.qlora_status_string.argtypes = [ctypes.c_int]
     lib.qlora_nf4_codebook.argtypes = [ctypes.POINTER(ctypes.c_float)]
     lib.qlora_nf4_storage_bytes.argtypes = [i64, i64, ctypes.POINTER(sz)]
+    lib.qlora_nf4_single_storage_bytes.argtypes = [i64, i64, ctypes.POINTER(sz)]
+    lib.qlora_quantize_nf4.argtypes = [vp, wp, vp]
+    lib.qlora_dequantize_nf4.argtypes = [wp, vp, vp]
     lib.qlora_quantize_nf4_dq.argtypes = [vp, wp, vp, szp, vp]
     lib.qlora_quantize_nf4_dq_noalloc.argtypes = [vp, wp, vp]
     lib.qlora_dequantize_nf4_dq.argtypes = [wp, vp, vp]
@@ -111,6 +115,26 @@ class NF4Weight:
                          torch.empty(1, dtype=torch.float32, device=device), rows, cols)
 
 
+@dataclass
+class SingleNF4Weight:
+    """Single-level storage of one quantized weight [rows, cols]: codes and the
+    fp32 block constants (no double quantization)."""
+    packed: torch.Tensor     # uint8 [rows*cols/2]
+    absmax: torch.Tensor     # float32 [nblk]
+    rows: int
+    cols: int
+
+    def as_c(self) -> _Weight:
+        return _Weight(self.packed.data_ptr(), None, None, None, self.rows, self.cols, 64, 0,
+                       self.absmax.data_ptr())
+
+    @staticmethod
+    def empty(rows: int, cols: int, device="cuda") -> "SingleNF4Weight":
+        sizes = qlora_nf4_single_storage_bytes(rows, cols)
+        return SingleNF4Weight(torch.empty(sizes[0], dtype=torch.uint8, device=device),
+                               torch.empty(sizes[1] // 4, dtype=torch.float32, device=device), rows, cols)
+
+
 def qlora_status_string(status: int) -> str:
     return load_library().qlora_status_string(status).decode()
 
@@ -124,6 +148,12 @@ def qlora_nf4_codebook() -> torch.Tensor:
 def qlora_nf4_storage_bytes(rows: int, cols: int) -> tuple:
     out = (ctypes.c_size_t * 4)()
     _check(load_library().qlora_nf4_storage_bytes(rows, cols, out), "qlora_nf4_storage_bytes")
+    return tuple(int(x) for x in out)
+
+
+def qlora_nf4_single_storage_bytes(rows: int, cols: int) -> tuple:
+    out = (ctypes.c_size_t * 2)()
+    _check(load_library().qlora_nf4_single_storage_bytes(rows, cols, out), "qlora_nf4_single_storage_bytes")
     return tuple(int(x) for x in out)
 
 
@@ -150,6 +180,15 @@ def qlora_quantize_nf4_dq(W: torch.Tensor, out: NF4Weight | None = None, workspa
     return q
 
 
+def qlora_quantize_nf4(W: torch.Tensor, out: SingleNF4Weight | None = None, stream=None) -> SingleNF4Weight:
+    """Single-level quantization (codes and fp32 block constants)."""
+    assert W.dtype == torch.bfloat16 and W.dim() == 2 and W.is_contiguous()
+    q = out or SingleNF4Weight.empty(W.shape[0], W.shape[1], W.device)
+    qc = q.as_c()
+    _check(load_library().qlora_quantize_nf4(_ptr(W), ctypes.byref(qc), _stream(stream)), "qlora_quantize_nf4")
+    return q
+
+
 def qlora_quantize_nf4_dq_noalloc(W: torch.Tensor, out: NF4Weight, stream=None) -> NF4Weight:
     """Quantize into `out` without any device allocation by the library (its
     scratch is a fixed array inside the library; see include/qlora.h)."""
@@ -160,7 +199,19 @@ def qlora_quantize_nf4_dq_noalloc(W: torch.Tensor, out: NF4Weight, stream=None) 
     return out
 
 
-def qlora_dequantize_nf4_dq(q: NF4Weight, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+def qlora_dequantize_nf4(q: NF4Weight | SingleNF4Weight, out: torch.Tensor | None = None,
+                         stream=None) -> torch.Tensor:
+    """Dequantize either storage kind to bf16."""
+    lib = load_library()
+    if out is None:
+        out = torch.empty(q.rows, q.cols, dtype=torch.bfloat16, device=q.packed.device)
+    qc = q.as_c()
+    _check(lib.qlora_dequantize_nf4(ctypes.byref(qc), _ptr(out), _stream(stream)), "qlora_dequantize_nf4")
+    return out
+
+
+def qlora_dequantize_nf4_dq(q: NF4Weight | SingleNF4Weight, out: torch.Tensor | None = None,
+                            stream=None) -> torch.Tensor:
     lib = load_library()
     if out is None:
         out = torch.empty(q.rows, q.cols, dtype=torch.bfloat16, device=q.packed.device)
@@ -169,7 +220,7 @@ def qlora_dequantize_nf4_dq(q: NF4Weight, out: torch.Tensor | None = None, strea
     return out
 
 
-def qlora_linear_fwd(q: NF4Weight, X: torch.Tensor, A: torch.Tensor, B: torch.Tensor, alpha: float,
+def qlora_linear_fwd(q: NF4Weight | SingleNF4Weight, X: torch.Tensor, A: torch.Tensor, B: torch.Tensor, alpha: float,
                      Y: torch.Tensor | None = None, T_save: torch.Tensor | bool | None = None,
                      workspace: torch.Tensor | None = None, stream=None):
     """Returns (Y, T) with T = X A^T in fp32 when T_save is True or a tensor, else (Y, None)."""
@@ -191,7 +242,7 @@ def qlora_linear_fwd(q: NF4Weight, X: torch.Tensor, A: torch.Tensor, B: torch.Te
     return Y, T_save
 
 
-def qlora_linear_bwd(q: NF4Weight, X: torch.Tensor, A: torch.Tensor, B: torch.Tensor, alpha: float,
+def qlora_linear_bwd(q: NF4Weight | SingleNF4Weight, X: torch.Tensor, A: torch.Tensor, B: torch.Tensor, alpha: float,
                      dY: torch.Tensor, T_saved: torch.Tensor | None = None, need_dX: bool = True,
                      dX: torch.Tensor | None = None, dA: torch.Tensor | None = None, dB: torch.Tensor | None = None,
                      workspace: torch.Tensor | None = None, stream=None):
@@ -215,7 +266,8 @@ def qlora_linear_bwd(q: NF4Weight, X: torch.Tensor, A: torch.Tensor, B: torch.Te
     return (dX if need_dX else None), dA, dB
 
 
-def qlora_merge_lora(q: NF4Weight, adapters, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+def qlora_merge_lora(q: NF4Weight | SingleNF4Weight, adapters, out: torch.Tensor | None = None,
+                     stream=None) -> torch.Tensor:
     """Merged bf16 weight [rows, cols] from the NF4 base and a sequence of
     adapters (A [r, cols], B [rows, r], alpha, weight); see include/qlora.h."""
     lib = load_library()

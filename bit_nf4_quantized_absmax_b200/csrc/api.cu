@@ -37,19 +37,36 @@ qlora_status device_info(DeviceInfo* info) {
   return QLORA_OK;
 }
 
-qlora_status check_weight(const qlora_nf4_weight* q, bool need_rows) {
+// Storage kinds: dq_blocksize == 256 is double-quantized (absmax_q, dq_scale,
+// mean), dq_blocksize == 0 is single-level (absmax). kind: 0 either, 1 only
+// double-quantized, 2 only single-level.
+qlora_status check_weight(const qlora_nf4_weight* q, bool need_rows, int kind = 0) {
   if (!q) return QLORA_ERR_INVALID_ARG;
   if (q->rows < 0 || q->cols <= 0) return QLORA_ERR_INVALID_ARG;
-  if (q->blocksize != 64 || q->dq_blocksize != 256) return QLORA_ERR_UNSUPPORTED;
+  const bool single = q->dq_blocksize == 0;
+  if (q->blocksize != 64 || (q->dq_blocksize != 256 && !single)) return QLORA_ERR_UNSUPPORTED;
+  if ((kind == 1 && single) || (kind == 2 && !single)) return QLORA_ERR_UNSUPPORTED;
   if (q->cols % 64) return QLORA_ERR_UNSUPPORTED;
   if (q->rows > (int64_t(1) << 31) || q->cols > (int64_t(1) << 31)) return QLORA_ERR_UNSUPPORTED;
   if (need_rows && q->rows == 0) return QLORA_ERR_INVALID_ARG;
   if (q->rows > 0) {
-    if (!q->packed || !q->absmax_q || !q->dq_scale || !q->mean) return QLORA_ERR_INVALID_ARG;
-    if (!aligned(q->packed, 16) || !aligned(q->absmax_q, 16) || !aligned(q->dq_scale, 4) || !aligned(q->mean, 4))
-      return QLORA_ERR_ALIGNMENT;
+    if (single) {
+      if (!q->packed || !q->absmax) return QLORA_ERR_INVALID_ARG;
+      if (!aligned(q->packed, 16) || !aligned(q->absmax, 4)) return QLORA_ERR_ALIGNMENT;
+    } else {
+      if (!q->packed || !q->absmax_q || !q->dq_scale || !q->mean) return QLORA_ERR_INVALID_ARG;
+      if (!aligned(q->packed, 16) || !aligned(q->absmax_q, 16) || !aligned(q->dq_scale, 4) ||
+          !aligned(q->mean, 4))
+        return QLORA_ERR_ALIGNMENT;
+    }
   }
   return QLORA_OK;
+}
+
+// The kernels' view of a checked weight (absmax non-null marks single-level storage).
+Nf4View view(const qlora_nf4_weight* q) {
+  if (q->dq_blocksize == 0) return Nf4View{q->packed, nullptr, nullptr, nullptr, q->rows, q->cols, q->absmax};
+  return Nf4View{q->packed, q->absmax_q, q->dq_scale, q->mean, q->rows, q->cols, nullptr};
 }
 
 qlora_status cuda_status(cudaError_t e) { return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA; }
@@ -152,9 +169,31 @@ qlora_status qlora_nf4_storage_bytes(int64_t rows, int64_t cols, size_t out[4]) 
   return QLORA_OK;
 }
 
+qlora_status qlora_nf4_single_storage_bytes(int64_t rows, int64_t cols, size_t out[2]) {
+  if (!out || rows < 0 || cols < 0) return QLORA_ERR_INVALID_ARG;
+  if (cols % 64) return QLORA_ERR_UNSUPPORTED;
+  const int64_t numel = rows * cols;
+  out[0] = static_cast<size_t>(numel / 2);
+  out[1] = static_cast<size_t>(numel / 64) * sizeof(float);
+  return QLORA_OK;
+}
+
+qlora_status qlora_quantize_nf4(const void* W_bf16, const qlora_nf4_weight* q, qlora_stream_t stream) {
+  qlora_status st = check_weight(q, false, 2);
+  if (st != QLORA_OK) return st;
+  if (!W_bf16 && q->rows > 0) return QLORA_ERR_INVALID_ARG;
+  if (W_bf16 && !aligned(W_bf16, 16)) return QLORA_ERR_ALIGNMENT;
+  const int64_t numel = q->rows * q->cols;
+  if (numel == 0) return QLORA_OK;
+  DeviceInfo di;
+  if ((st = device_info(&di)) != QLORA_OK) return st;
+  return cuda_status(launch_quantize_single(W_bf16, numel, q->packed, q->absmax, di.num_sms,
+                                            reinterpret_cast<cudaStream_t>(stream)));
+}
+
 qlora_status qlora_quantize_nf4_dq(const void* W_bf16, const qlora_nf4_weight* q, void* workspace,
                                    size_t* workspace_bytes, qlora_stream_t stream) {
-  qlora_status st = check_weight(q, false);
+  qlora_status st = check_weight(q, false, 1);
   if (st != QLORA_OK) return st;
   if (!W_bf16 && q->rows > 0) return QLORA_ERR_INVALID_ARG;
   if (W_bf16 && !aligned(W_bf16, 16)) return QLORA_ERR_ALIGNMENT;
@@ -174,7 +213,7 @@ qlora_status qlora_quantize_nf4_dq(const void* W_bf16, const qlora_nf4_weight* q
                                      reinterpret_cast<cudaStream_t>(stream)));
 }
 
-qlora_status qlora_dequantize_nf4_dq(const qlora_nf4_weight* q, void* out_bf16, qlora_stream_t stream) {
+qlora_status qlora_dequantize_nf4(const qlora_nf4_weight* q, void* out_bf16, qlora_stream_t stream) {
   qlora_status st = check_weight(q, false);
   if (st != QLORA_OK) return st;
   const int64_t numel = q->rows * q->cols;
@@ -183,9 +222,12 @@ qlora_status qlora_dequantize_nf4_dq(const qlora_nf4_weight* q, void* out_bf16, 
   if (!aligned(out_bf16, 16)) return QLORA_ERR_ALIGNMENT;
   DeviceInfo di;
   if ((st = device_info(&di)) != QLORA_OK) return st;
-  return cuda_status(launch_dequantize(q->packed, q->absmax_q, q->dq_scale, q->mean, out_bf16, numel,
-                                       quant_tables().codebook, di.num_sms,
+  return cuda_status(launch_dequantize(view(q), out_bf16, quant_tables().codebook, di.num_sms,
                                        reinterpret_cast<cudaStream_t>(stream)));
+}
+
+qlora_status qlora_dequantize_nf4_dq(const qlora_nf4_weight* q, void* out_bf16, qlora_stream_t stream) {
+  return qlora_dequantize_nf4(q, out_bf16, stream);
 }
 
 qlora_status qlora_linear_fwd(const qlora_nf4_weight* q, const void* X, int64_t M, const void* A,
@@ -224,15 +266,14 @@ qlora_status qlora_linear_fwd(const qlora_nf4_weight* q, const void* X, int64_t 
   const float* cb = quant_tables().codebook;
   if (decode) {
     float* T = T_save ? T_save : reinterpret_cast<float*>(ws + off_T);
-    Nf4View w{q->packed, q->absmax_q, q->dq_scale, q->mean, N, K};
-    return cuda_status(launch_decode_fwd(w, X, M, A, B, r, s, Y, T, reinterpret_cast<float*>(ws + off_part),
+    return cuda_status(launch_decode_fwd(view(q), X, M, A, B, r, s, Y, T, reinterpret_cast<float*>(ws + off_part),
                                          reinterpret_cast<unsigned int*>(ws + off_cnt), dplan, cb, err, cs));
   }
   void* Wd = ws + off_wd;
   void* sT = ws + off_sT;
   float* P = reinterpret_cast<float*>(ws + off_part);
   const int splits_t = red_splits(M, rpad, K, kRefSms);
-  cudaError_t e = launch_dequantize(q->packed, q->absmax_q, q->dq_scale, q->mean, Wd, N * K, cb, di.num_sms, cs);
+  cudaError_t e = launch_dequantize(view(q), Wd, cb, di.num_sms, cs);
   if (e == cudaSuccess) e = launch_gemm_lora_t(X, A, M, K, r, rpad, P, splits_t, di.num_sms, err, cs);
   if (e == cudaSuccess)
     e = launch_lora_finish(P, splits_t, M, r, rpad, s, T_save, sT, nullptr, nullptr, di.num_sms, cs);
@@ -302,7 +343,7 @@ qlora_status qlora_linear_bwd(const qlora_nf4_weight* q, const void* X, int64_t 
   if (dX) {
     void* Wd = ws + off_wd;
     if (e == cudaSuccess)
-      e = launch_dequantize(q->packed, q->absmax_q, q->dq_scale, q->mean, Wd, N * K, cb, di.num_sms, cs);
+      e = launch_dequantize(view(q), Wd, cb, di.num_sms, cs);
     if (e == cudaSuccess) e = launch_gemm_dx(dY, Wd, sU, A, M, N, K, r, rpad, dX, di.num_sms, err, cs);
   }
   // dA^T [K, r] = X^T U, reduced over tokens, then dA = s * (.)^T
@@ -338,8 +379,7 @@ qlora_status qlora_merge_lora(const qlora_nf4_weight* q, const qlora_lora_adapte
   if ((q->rows + 63) / 64 > 65535) return QLORA_ERR_UNSUPPORTED;
   DeviceInfo di;
   if ((st = device_info(&di)) != QLORA_OK) return st;
-  Nf4View w{q->packed, q->absmax_q, q->dq_scale, q->mean, q->rows, q->cols};
-  return cuda_status(launch_merge(w, ma, n_adapters, W_out, quant_tables().codebook, di.num_sms,
+  return cuda_status(launch_merge(view(q), ma, n_adapters, W_out, quant_tables().codebook, di.num_sms,
                                   reinterpret_cast<cudaStream_t>(stream)));
 }
 

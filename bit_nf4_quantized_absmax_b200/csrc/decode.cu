@@ -195,10 +195,13 @@ __device__ __forceinline__ uint4 lds128(uint32_t addr) {
   return v;
 }
 
-template <int MT>
+// SINGLE: single-level storage, the block constant is absmax[b] itself (q, dqs
+// and mean unused); otherwise m'_b = fmaf(q[b], dqs[b / 256], mean).
+template <int MT, bool SINGLE>
 __global__ void __launch_bounds__((kDecodeWarps + 1) * 32, kDecodeCtasPerSm)
 k_decode(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
-         const int8_t* __restrict__ q, const float* __restrict__ dqs, const float* __restrict__ mean, int M,
+         const int8_t* __restrict__ q, const float* __restrict__ dqs, const float* __restrict__ mean,
+         const float* __restrict__ absmax, int M,
          int64_t N, int64_t K, const float* __restrict__ T, const __nv_bfloat16* __restrict__ Bl, int r, float s,
          __nv_bfloat16* __restrict__ Y, float* __restrict__ partial, unsigned int* __restrict__ counters,
          int64_t n_items, int64_t n_ctas, int max_seg, int32_t* __restrict__ err,
@@ -266,7 +269,7 @@ k_decode(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUten
   const uint32_t offW1 = (warp * 16 + g) * 128 + (((2 * t + 1) ^ g) << 4);
   const uint32_t offX = kWBytes + t * (8 * MT * 128) + g * 128;
 
-  const float mu = *mean;
+  const float mu = SINGLE ? 0.0f : *mean;
   // block constants of rows 16 w + g and + 8 (m' = 0 outside the matrix)
   auto consts = [&](int64_t rg, int sb, int& qa, float& sa, int& qb, float& sbv, bool& va, bool& vb) {
     const int kb = sb * 4 + t;
@@ -274,10 +277,16 @@ k_decode(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUten
     va = kb < nkb_row && na < N;
     vb = kb < nkb_row && nb < N;
     const int64_t ba = na * nkb_row + kb, bb = nb * nkb_row + kb;
-    qa = va ? static_cast<int>(__ldg(q + ba)) : 0;
-    sa = va ? __ldg(dqs + (ba >> 8)) : 0.0f;
-    qb = vb ? static_cast<int>(__ldg(q + bb)) : 0;
-    sbv = vb ? __ldg(dqs + (bb >> 8)) : 0.0f;
+    if (SINGLE) {
+      qa = qb = 0;
+      sa = va ? __ldg(absmax + ba) : 0.0f;
+      sbv = vb ? __ldg(absmax + bb) : 0.0f;
+    } else {
+      qa = va ? static_cast<int>(__ldg(q + ba)) : 0;
+      sa = va ? __ldg(dqs + (ba >> 8)) : 0.0f;
+      qb = vb ? static_cast<int>(__ldg(q + bb)) : 0;
+      sbv = vb ? __ldg(dqs + (bb >> 8)) : 0.0f;
+    }
   };
 
   int nqa, nqb;
@@ -300,8 +309,8 @@ k_decode(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUten
       for (int m = 0; m < MT; ++m) acc[c][m][0] = acc[c][m][1] = acc[c][m][2] = acc[c][m][3] = 0.0f;
 
     for (int e = 0; e < seg_items; ++e, ++n, ++sb) {
-      const float mA = nva ? __fmaf_rn(static_cast<float>(nqa), nsa, mu) : 0.0f;
-      const float mB = nvb ? __fmaf_rn(static_cast<float>(nqb), nsc, mu) : 0.0f;
+      const float mA = nva ? (SINGLE ? nsa : __fmaf_rn(static_cast<float>(nqa), nsa, mu)) : 0.0f;
+      const float mB = nvb ? (SINGLE ? nsc : __fmaf_rn(static_cast<float>(nqb), nsc, mu)) : 0.0f;
       if (n + 1 < n_my) {  // next item's constants
         const bool wrap = sb + 1 == nsb;
         consts(wrap ? rg + 1 : rg, wrap ? 0 : sb + 1, nqa, nsa, nqb, nsc, nva, nvb);
@@ -489,13 +498,16 @@ cudaError_t launch_decode_fwd(const Nf4View& w, const void* X, int64_t M, const 
   const __nv_bfloat16* Bb = reinterpret_cast<const __nv_bfloat16*>(B);
   __nv_bfloat16* Yb = reinterpret_cast<__nv_bfloat16*>(Y);
   const int Mi = static_cast<int>(M);
-  auto kern = p.mt == 1 ? k_decode<1> : k_decode<2>;
+  const bool single = w.absmax != nullptr;
+  auto kern = p.mt == 1 ? (single ? k_decode<1, true> : k_decode<1, false>)
+                        : (single ? k_decode<2, true> : k_decode<2, false>);
   const int smem = decode_smem_bytes(p.mt);
-  e = p.mt == 1 ? ensure_smem_limit<k_decode<1>>(smem) : ensure_smem_limit<k_decode<2>>(smem);
+  e = p.mt == 1 ? (single ? ensure_smem_limit<k_decode<1, true>>(smem) : ensure_smem_limit<k_decode<1, false>>(smem))
+                : (single ? ensure_smem_limit<k_decode<2, true>>(smem) : ensure_smem_limit<k_decode<2, false>>(smem));
   if (e != cudaSuccess) return e;
   e = launch_pdl(kern, dim3(p.grid), dim3((kDecodeWarps + 1) * 32), smem, stream, tw, tx, w.absmax_q, w.dq_scale,
-                 w.mean, Mi, w.N, w.K, static_cast<const float*>(T), Bb, r, s, Yb, partial, counters, p.n_items,
-                 static_cast<int64_t>(p.grid), p.max_seg, err, cb);
+                 w.mean, w.absmax, Mi, w.N, w.K, static_cast<const float*>(T), Bb, r, s, Yb, partial, counters,
+                 p.n_items, static_cast<int64_t>(p.grid), p.max_seg, err, cb);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

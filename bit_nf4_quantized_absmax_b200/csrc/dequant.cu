@@ -1,8 +1,9 @@
-// Block-wise dequantization of NF4 + double-quant storage to bf16
-// ("QLoRA vs ChatGPT", capability 5: weights are dequantized block by block).
+// Block-wise dequantization of NF4 storage to bf16 ("QLoRA vs ChatGPT",
+// capability 5: weights are dequantized block by block).
 //
 // One thread decodes 32 weights (half a 64-weight block): it forms the block
-// constant m' = fmaf(q_b, dq_scale_g, mean), builds the block's 16-entry bf16
+// constant (m' = fmaf(q_b, dq_scale_g, mean) for double-quantized storage, the
+// stored fp32 m_b for single-level storage), builds the block's 16-entry bf16
 // table and decodes its 16 packed bytes with byte permutes.
 #include "common.cuh"
 #include "kernels.h"
@@ -36,13 +37,13 @@ __device__ __forceinline__ void dequant_unit(const uint4 nib, int64_t u, float m
 
 // Grid-stride over 32-weight units; each thread keeps kDeqUnroll 16-byte
 // loads in flight before decoding them.
-template <bool V8>
+template <bool V8, bool SINGLE>
 __global__ void __launch_bounds__(256)
 k_dequant(const uint4* __restrict__ packed, const int8_t* __restrict__ absmax_q,
-          const float* __restrict__ dq_scale, const float* __restrict__ mean, uint4* __restrict__ out,
-          int64_t n_units, const __grid_constant__ Nf4Codebook cb) {
+          const float* __restrict__ dq_scale, const float* __restrict__ mean, const float* __restrict__ absmax,
+          uint4* __restrict__ out, int64_t n_units, const __grid_constant__ Nf4Codebook cb) {
   pdl_enter();
-  const float mu = *mean;
+  const float mu = SINGLE ? 0.0f : *mean;
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
   for (int64_t u0 = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; u0 < n_units;
        u0 += stride * kDeqUnroll) {
@@ -55,33 +56,39 @@ k_dequant(const uint4* __restrict__ packed, const int8_t* __restrict__ absmax_q,
       const int64_t u = u0 + i * stride;
       const bool ok = u < n_units;
       nib[i] = ok ? __ldcs(packed + u) : make_uint4(0, 0, 0, 0);
-      qv[i] = ok ? static_cast<int>(__ldg(absmax_q + (u >> 1))) : 0;
-      sc[i] = ok ? __ldg(dq_scale + (u >> 9)) : 0.0f;
+      if (SINGLE) {
+        qv[i] = 0;
+        sc[i] = ok ? __ldg(absmax + (u >> 1)) : 0.0f;
+      } else {
+        qv[i] = ok ? static_cast<int>(__ldg(absmax_q + (u >> 1))) : 0;
+        sc[i] = ok ? __ldg(dq_scale + (u >> 9)) : 0.0f;
+      }
     }
 #pragma unroll
     for (int i = 0; i < kDeqUnroll; ++i) {
       const int64_t u = u0 + i * stride;
       if (u < n_units)
-        dequant_unit<V8>(nib[i], u, __fmaf_rn(static_cast<float>(qv[i]), sc[i], mu), out, cb);
+        dequant_unit<V8>(nib[i], u, SINGLE ? sc[i] : __fmaf_rn(static_cast<float>(qv[i]), sc[i], mu), out, cb);
     }
   }
 }
 
 }  // namespace
 
-cudaError_t launch_dequantize(const uint8_t* packed, const int8_t* absmax_q, const float* dq_scale,
-                              const float* mean, void* out, int64_t numel, const float codebook[16],
-                              int num_sms, cudaStream_t stream) {
+cudaError_t launch_dequantize(const Nf4View& w, void* out, const float codebook[16], int num_sms,
+                              cudaStream_t stream) {
   Nf4Codebook cb;
   for (int i = 0; i < 16; ++i) cb.c[i] = codebook[i];
-  const int64_t n_units = numel / 32;
+  const int64_t n_units = w.N * w.K / 32;
   int64_t want = (n_units + 256 * kDeqUnroll - 1) / (256 * kDeqUnroll);
   int64_t cap = static_cast<int64_t>(num_sms) * 8;
   const int grid = static_cast<int>(want < cap ? (want > 0 ? want : 1) : cap);
   const bool v8 = (reinterpret_cast<uintptr_t>(out) & 31u) == 0;
-  return launch_pdl(v8 ? k_dequant<true> : k_dequant<false>, dim3(grid), dim3(256), 0, stream,
-                    reinterpret_cast<const uint4*>(packed), absmax_q, dq_scale, mean, reinterpret_cast<uint4*>(out),
-                    n_units, cb);
+  const bool single = w.absmax != nullptr;
+  auto kern = single ? (v8 ? k_dequant<true, true> : k_dequant<false, true>)
+                     : (v8 ? k_dequant<true, false> : k_dequant<false, false>);
+  return launch_pdl(kern, dim3(grid), dim3(256), 0, stream, reinterpret_cast<const uint4*>(w.packed), w.absmax_q,
+                    w.dq_scale, w.mean, w.absmax, reinterpret_cast<uint4*>(out), n_units, cb);
 }
 
 }  // namespace qlora

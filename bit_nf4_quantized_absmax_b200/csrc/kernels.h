@@ -47,11 +47,13 @@ cudaError_t launch_quantize(const void* W, int64_t numel, uint8_t* packed, int8_
                             float* mean, float* absmax_scratch, void* hist_scratch, int num_sms,
                             cudaStream_t stream);
 
-cudaError_t launch_dequantize(const uint8_t* packed, const int8_t* absmax_q, const float* dq_scale,
-                              const float* mean, void* out, int64_t numel, const float codebook[16],
-                              int num_sms, cudaStream_t stream);
+// Single-level storage: the codes and the fp32 block constants m_b only (pass 1).
+cudaError_t launch_quantize_single(const void* W, int64_t numel, uint8_t* packed, float* absmax, int num_sms,
+                                   cudaStream_t stream);
 
-// Weight view used by the fused decode kernel.
+// A stored weight. Double-quantized: absmax_q, dq_scale and mean give the block
+// constant m'_b = fmaf(absmax_q[b], dq_scale[b / 256], mean) and absmax is null.
+// Single-level: absmax[b] is the constant itself and the other three are null.
 struct Nf4View {
   const uint8_t* packed;
   const int8_t* absmax_q;
@@ -59,7 +61,11 @@ struct Nf4View {
   const float* mean;
   int64_t N;  // rows
   int64_t K;  // cols
+  const float* absmax;
 };
+
+cudaError_t launch_dequantize(const Nf4View& w, void* out, const float codebook[16], int num_sms,
+                              cudaStream_t stream);
 
 // ---- decode.cu: M <= 16 forward ----
 // Work split of the decode kernel: (128-row group, 256-wide K superblock)

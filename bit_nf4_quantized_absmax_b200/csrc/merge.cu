@@ -111,8 +111,7 @@ k_merge(__nv_bfloat16* __restrict__ W, int64_t N, int64_t K, const __grid_consta
 cudaError_t launch_merge(const Nf4View& w, const MergeAdapter* adapters, int n_adapters, void* out,
                          const float codebook[16], int num_sms, cudaStream_t stream) {
   if (n_adapters < 0 || n_adapters > kMaxMergeAdapters) return cudaErrorInvalidValue;
-  cudaError_t e = launch_dequantize(w.packed, w.absmax_q, w.dq_scale, w.mean, out, w.N * w.K, codebook, num_sms,
-                                    stream);
+  cudaError_t e = launch_dequantize(w, out, codebook, num_sms, stream);
   if (e != cudaSuccess || n_adapters == 0) return e;
   MergeArgs ma{};
   ma.n = n_adapters;

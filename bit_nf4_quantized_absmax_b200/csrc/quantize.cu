@@ -132,8 +132,9 @@ __device__ __forceinline__ void encode16(const uint32_t (&d)[8], float ms, float
 // reads 1 KB of contiguous weights per load instruction. Every lane of a warp
 // runs the same iterations so that the histogram update can be combined across
 // the warp (lanes whose blocks share an exponent add their significands first,
-// then one of them updates the shared bin).
-template <bool V8>
+// then one of them updates the shared bin). Without HIST (single-level
+// storage, no mean needed) the histogram work is left out.
+template <bool V8, bool HIST>
 __device__ __forceinline__ void pass1_loop(const uint4* __restrict__ W, int64_t nblk, uint32_t* __restrict__ packed,
                                            float* __restrict__ absmax, const unsigned char* bins,
                                            unsigned int* __restrict__ s_hist) {
@@ -192,12 +193,15 @@ __device__ __forceinline__ void pass1_loop(const uint4* __restrict__ W, int64_t 
       }
       *reinterpret_cast<uint2*>(packed + blk * 8 + qtr * 2) = make_uint2(out[0], out[1]);
     }
-    const unsigned int same = __match_any_sync(0xffffffffu, hE);
-    const unsigned int tot = __reduce_add_sync(same, hsig);
-    if (lane == __ffs(same) - 1 && tot) atomicAdd(&s_hist[hE], tot);
+    if (HIST) {
+      const unsigned int same = __match_any_sync(0xffffffffu, hE);
+      const unsigned int tot = __reduce_add_sync(same, hsig);
+      if (lane == __ffs(same) - 1 && tot) atomicAdd(&s_hist[hE], tot);
+    }
   }
 }
 
+template <bool HIST>
 __global__ void __launch_bounds__(kPass1Threads)
 k_quant_pass1(const uint4* __restrict__ W, bool v8, uint32_t* __restrict__ packed,
               float* __restrict__ absmax, unsigned int* __restrict__ hist_part, int64_t nblk,
@@ -206,17 +210,19 @@ k_quant_pass1(const uint4* __restrict__ W, bool v8, uint32_t* __restrict__ packe
   __shared__ unsigned int s_hist[256];          // per-CTA significand sums (native 32-bit atomics)
   const int tid = threadIdx.x;
   if (tid < kBins) s_bins[tid] = make_uint2(__float_as_uint(tab.bins[tid].threshold), tab.bins[tid].j + 1u);
-  s_hist[tid] = 0u;
+  if (HIST) s_hist[tid] = 0u;
   __syncthreads();
   pdl_enter();
 
   const unsigned char* bins = reinterpret_cast<const unsigned char*>(s_bins);
   if (v8)
-    pass1_loop<true>(W, nblk, packed, absmax, bins, s_hist);
+    pass1_loop<true, HIST>(W, nblk, packed, absmax, bins, s_hist);
   else
-    pass1_loop<false>(W, nblk, packed, absmax, bins, s_hist);
-  __syncthreads();
-  hist_part[static_cast<int64_t>(tid) * kQuantMaxGrid + blockIdx.x] = s_hist[tid];  // bin-major
+    pass1_loop<false, HIST>(W, nblk, packed, absmax, bins, s_hist);
+  if (HIST) {
+    __syncthreads();
+    hist_part[static_cast<int64_t>(tid) * kQuantMaxGrid + blockIdx.x] = s_hist[tid];  // bin-major
+  }
 }
 
 // totals[e] = sum over the pass-1 CTAs of their bin e (one CTA per bin).
@@ -325,6 +331,29 @@ k_dq_quantize(const float* __restrict__ absmax, int64_t nblk, const unsigned lon
   if (lane == 0) dq_scale[g] = sc;
 }
 
+// Persistent grid of pass 1: exactly the CTAs that are resident at once (four
+// lanes per 64-weight block), so no SM idles through a partial last wave.
+template <bool HIST>
+int pass1_grid(int64_t nblk, int num_sms) {
+  static std::atomic<int> per_sm_cache{0};  // the same on every B200; racing writers store equal values
+  int per_sm = per_sm_cache.load(std::memory_order_relaxed);
+  if (per_sm == 0) {
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_quant_pass1<HIST>, kPass1Threads, 0) !=
+            cudaSuccess ||
+        per_sm < 1)
+      per_sm = 4;
+    per_sm_cache.store(per_sm, std::memory_order_relaxed);
+  }
+  int64_t want = (nblk * 4 + kPass1Threads - 1) / kPass1Threads;
+  int64_t cap = static_cast<int64_t>(num_sms) * per_sm;
+  if (cap > kQuantMaxGrid) cap = kQuantMaxGrid;
+  int64_t g = want < cap ? (want > 0 ? want : 1) : cap;
+  // A CTA sums at most 2^24 significands of 8 bits, so its 32-bit bins cannot overflow.
+  const int64_t min_grid = (nblk + (int64_t(1) << 24) - 1) >> 24;
+  if (g < min_grid) g = min_grid;
+  return g > kQuantMaxGrid ? -1 : static_cast<int>(g);  // -1: more than 2^35 blocks
+}
+
 }  // namespace
 
 cudaError_t launch_quantize(const void* W, int64_t numel, uint8_t* packed, int8_t* absmax_q, float* dq_scale,
@@ -338,28 +367,10 @@ cudaError_t launch_quantize(const void* W, int64_t numel, uint8_t* packed, int8_
   unsigned int* hist_part = static_cast<unsigned int*>(hist_scratch);
   unsigned long long* totals =
       reinterpret_cast<unsigned long long*>(static_cast<char*>(hist_scratch) + kQuantHistBytes);
-
-  // four lanes per 64-weight block; a persistent grid of exactly the CTAs that
-  // are resident at once, so no SM idles through a partial last wave
-  static std::atomic<int> per_sm_cache{0};  // the same on every B200; racing writers store equal values
-  int per_sm = per_sm_cache.load(std::memory_order_relaxed);
-  if (per_sm == 0) {
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_quant_pass1, kPass1Threads, 0) != cudaSuccess ||
-        per_sm < 1)
-      per_sm = 4;
-    per_sm_cache.store(per_sm, std::memory_order_relaxed);
-  }
-  int64_t want = (nblk * 4 + kPass1Threads - 1) / kPass1Threads;
-  int64_t cap = static_cast<int64_t>(num_sms) * per_sm;
-  if (cap > kQuantMaxGrid) cap = kQuantMaxGrid;
-  int64_t g = want < cap ? (want > 0 ? want : 1) : cap;
-  // A CTA sums at most 2^24 significands of 8 bits, so its 32-bit bins cannot overflow.
-  const int64_t min_grid = (nblk + (int64_t(1) << 24) - 1) >> 24;
-  if (g < min_grid) g = min_grid;
-  if (g > kQuantMaxGrid) return cudaErrorInvalidValue;  // more than 2^35 blocks
-  const int grid = static_cast<int>(g);
+  const int grid = pass1_grid<true>(nblk, num_sms);
+  if (grid < 0) return cudaErrorInvalidValue;
   const bool v8 = ((reinterpret_cast<uintptr_t>(W) | reinterpret_cast<uintptr_t>(packed)) & 31u) == 0;
-  cudaError_t e = launch_pdl(k_quant_pass1, dim3(grid), dim3(kPass1Threads), 0, stream,
+  cudaError_t e = launch_pdl(k_quant_pass1<true>, dim3(grid), dim3(kPass1Threads), 0, stream,
                              reinterpret_cast<const uint4*>(W), v8, reinterpret_cast<uint32_t*>(packed),
                              absmax_scratch, hist_part, nblk, tab);
   if (e != cudaSuccess) return e;
@@ -369,6 +380,20 @@ cudaError_t launch_quantize(const void* W, int64_t numel, uint8_t* packed, int8_
   const int dq_grid = static_cast<int>((ngrp + 7) / 8);
   return launch_pdl(k_dq_quantize, dim3(dq_grid), dim3(256), 0, stream, static_cast<const float*>(absmax_scratch),
                     nblk, static_cast<const unsigned long long*>(totals), mean, absmax_q, dq_scale, ngrp);
+}
+
+cudaError_t launch_quantize_single(const void* W, int64_t numel, uint8_t* packed, float* absmax, int num_sms,
+                                   cudaStream_t stream) {
+  const QuantTables& tabs = quant_tables();
+  QuantBinTable tab;
+  for (int i = 0; i < kBins; ++i) tab.bins[i] = tabs.bins[i];
+  const int64_t nblk = numel / 64;
+  const int grid = pass1_grid<false>(nblk, num_sms);
+  if (grid < 0) return cudaErrorInvalidValue;
+  const bool v8 = ((reinterpret_cast<uintptr_t>(W) | reinterpret_cast<uintptr_t>(packed)) & 31u) == 0;
+  return launch_pdl(k_quant_pass1<false>, dim3(grid), dim3(kPass1Threads), 0, stream,
+                    reinterpret_cast<const uint4*>(W), v8, reinterpret_cast<uint32_t*>(packed), absmax,
+                    static_cast<unsigned int*>(nullptr), nblk, tab);
 }
 
 }  // namespace qlora

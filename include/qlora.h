@@ -4,7 +4,9 @@
  * The library implements the data-parallel hot path of QLoRA:
  *   1. the NF4 ("NormalFloat4") codebook,
  *   2. block-wise absmax quantization of a frozen bf16 weight to 4-bit codes,
- *   3. double quantization of the fp32 absmax constants to int8 codes,
+ *   3. double quantization of the fp32 absmax constants to int8 codes (or,
+ *      as the variant the paper compares it with, single-level storage that
+ *      keeps the fp32 constants),
  *   4. block-wise dequantization back to bf16,
  *   5. the QLoRA linear layer  Y = X W'^T + s (X A^T) B^T  (W' = dequant(W)),
  *      forward and backward (dX, dA, dB; W stays frozen, no dW),
@@ -57,7 +59,9 @@ typedef struct CUstream_st* qlora_stream_t;
 typedef enum {
   QLORA_OK = 0,
   QLORA_ERR_INVALID_ARG = 1,   /* null pointer, negative or inconsistent size  */
-  QLORA_ERR_UNSUPPORTED = 2,   /* block sizes other than 64/256, cols % 64 != 0,
+  QLORA_ERR_UNSUPPORTED = 2,   /* block size other than 64, dq_blocksize other
+                                  than 256 (or 0 where single-level is allowed),
+                                  cols % 64 != 0,
                                   r outside [8, 256] or r % 8 != 0             */
   QLORA_ERR_ALIGNMENT = 3,     /* a pointer is not aligned as required          */
   QLORA_ERR_CUDA = 4,          /* a launch or CUDA runtime call failed          */
@@ -65,22 +69,33 @@ typedef enum {
   QLORA_ERR_DEVICE = 6         /* no sm_100 device is current                   */
 } qlora_status;
 
-/* NF4 + double-quant storage of one frozen weight W [rows, cols] (rows = N =
- * out_features, cols = K = in_features, as in a PyTorch Linear).
+/* NF4 storage of one frozen weight W [rows, cols] (rows = N = out_features,
+ * cols = K = in_features, as in a PyTorch Linear), in one of two kinds.
  *
  *   packed    : rows*cols/2 bytes. Byte i holds code[2i] in its low nibble and
  *               code[2i+1] in its high nibble (elements in row-major order).
+ *
+ * Double-quantized (dq_blocksize == 256, the QLoRA format; [C] 3):
  *   absmax_q  : nblk = rows*cols/64 int8 codes in [-127, 127], one per block of
  *               64 consecutive weights (a block never crosses a row).
  *   dq_scale  : ngrp = ceil(nblk/256) fp32 scales, one per 256 consecutive
  *               absmax codes (the last group may be shorter).
  *   mean      : one fp32, the mean of all first-level absmax constants.
- *   blocksize, dq_blocksize: must be 64 and 256.
+ *   absmax    : unused (NULL).
+ *   A block's decoded constant is m' = fmaf((float)absmax_q[b], dq_scale[b/256],
+ *   mean).
  *
- * A block's decoded constant is m' = fmaf((float)absmax_q[b], dq_scale[b/256],
- * mean) and its weights decode to bf16_rn(codebook[code] * m')  ([C] 1, 3, 5).
- * All pointers are device memory owned by the caller; packed and absmax_q must
- * be 16-byte aligned, dq_scale and mean 4-byte aligned.
+ * Single-level (dq_blocksize == 0; "NFloat4" without DQ in the paper's p.8
+ * Table 4, quoted on [E]; [C] 3 contrasts it with double quantization):
+ *   absmax    : nblk fp32 constants m_b, the block's absmax itself (0.5625
+ *               bytes per weight in all, against 0.515869 double-quantized).
+ *   absmax_q, dq_scale, mean: unused (NULL).
+ *   The block's constant is m' = absmax[b].
+ *
+ * Either way a block's weights decode to bf16_rn(codebook[code] * m')
+ * ([C] 1, 5), and blocksize must be 64. All pointers are device memory owned
+ * by the caller; packed and absmax_q must be 16-byte aligned, dq_scale, mean
+ * and absmax 4-byte aligned.
  */
 typedef struct {
   uint8_t* packed;
@@ -91,6 +106,7 @@ typedef struct {
   int64_t  cols;
   int32_t  blocksize;
   int32_t  dq_blocksize;
+  float*   absmax;
 } qlora_nf4_weight;
 
 /* Human-readable name of a status code (static string). */
@@ -116,6 +132,19 @@ qlora_status qlora_nf4_codebook(float out16[16]);
  * QLORA_ERR_UNSUPPORTED (cols % 64 != 0). */
 qlora_status qlora_nf4_storage_bytes(int64_t rows, int64_t cols, size_t out[4]);
 
+/* qlora_nf4_single_storage_bytes -- sizes of the arrays of a single-level
+ * qlora_nf4_weight (host call): out[0] = bytes of packed, out[1] = bytes of
+ * absmax. Errors: as qlora_nf4_storage_bytes. */
+qlora_status qlora_nf4_single_storage_bytes(int64_t rows, int64_t cols, size_t out[2]);
+
+/* qlora_quantize_nf4 -- single-level quantization: the level-1 step of
+ * qlora_quantize_nf4_dq alone. Per block b of 64 weights: m_b = max |w|, stored
+ * in q->absmax[b]; the codes are those qlora_quantize_nf4_dq writes (bit for
+ * bit: level 1 does not depend on level 2). q->dq_blocksize must be 0 (else
+ * QLORA_ERR_UNSUPPORTED). No workspace. rows == 0 writes nothing.
+ * Errors: INVALID_ARG, UNSUPPORTED, ALIGNMENT, CUDA, DEVICE. */
+qlora_status qlora_quantize_nf4(const void* W_bf16, const qlora_nf4_weight* q, qlora_stream_t stream);
+
 /* qlora_quantize_nf4_dq -- quantize a frozen bf16 weight W [rows, cols] into
  * q's arrays ([C] 1: block-wise absmax quantization; [C] 3 and [G] "Core
  * Architecture & Training": the absmax constants are quantized again to 8 bit
@@ -131,8 +160,8 @@ qlora_status qlora_nf4_storage_bytes(int64_t rows, int64_t cols, size_t out[4]);
  *
  * W_bf16: device, [rows, cols] bf16, 16-byte aligned. q: host struct whose
  * pointers and sizes describe caller-owned device arrays (q->rows, q->cols
- * must equal the weight's shape). rows == 0 returns QLORA_OK and writes
- * nothing. The result does not depend on launch configuration (the mean uses
+ * must equal the weight's shape; q->dq_blocksize must be 256). rows == 0
+ * returns QLORA_OK and writes nothing. The result does not depend on launch configuration (the mean uses
  * an exact integer accumulation).
  * Errors: INVALID_ARG, UNSUPPORTED, ALIGNMENT, WORKSPACE, CUDA, DEVICE. */
 qlora_status qlora_quantize_nf4_dq(const void* W_bf16, const qlora_nf4_weight* q,
@@ -158,17 +187,23 @@ qlora_status qlora_quantize_nf4_dq(const void* W_bf16, const qlora_nf4_weight* q
 qlora_status qlora_quantize_nf4_dq_noalloc(const void* W_bf16, const qlora_nf4_weight* q,
                                            qlora_stream_t stream);
 
-/* qlora_dequantize_nf4_dq -- decode q to a bf16 matrix out_bf16 [rows, cols]
- * (device, 16-byte aligned): w' = bf16_rn(fp32(codebook[code] * m'_b)) with
- * m'_b = fmaf(absmax_q_b, dq_scale_g, mean) ([C] 5: block-wise dequantization).
- * Bit-identical to the dequantization used inside qlora_linear_fwd/bwd.
+/* qlora_dequantize_nf4 -- decode q (either storage kind) to a bf16 matrix
+ * out_bf16 [rows, cols] (device, 16-byte aligned): w' = bf16_rn(fp32(
+ * codebook[code] * m'_b)) with the block constant m'_b of the storage kind
+ * ([C] 5: block-wise dequantization). Bit-identical to the dequantization used
+ * inside qlora_linear_fwd/bwd and qlora_merge_lora.
  * Errors: INVALID_ARG, UNSUPPORTED, ALIGNMENT, CUDA, DEVICE. */
+qlora_status qlora_dequantize_nf4(const qlora_nf4_weight* q, void* out_bf16, qlora_stream_t stream);
+
+/* qlora_dequantize_nf4_dq -- the same call as qlora_dequantize_nf4 (kept under
+ * the name of the double-quantized format; it accepts both kinds). */
 qlora_status qlora_dequantize_nf4_dq(const qlora_nf4_weight* q, void* out_bf16,
                                      qlora_stream_t stream);
 
 /* qlora_linear_fwd -- Y = X W'^T + s (X A^T) B^T  ([C] 2 and 5).
  *
- *   q      : the frozen weight, W' = dequant(q) is [N, K] = [q->rows, q->cols].
+ *   q      : the frozen weight (either storage kind), W' = dequant(q) is
+ *            [N, K] = [q->rows, q->cols].
  *   X      : device bf16 [M, K].        A : device bf16 [r, K].
  *   B      : device bf16 [N, r].        Y : device bf16 [M, N] (output).
  *   T_save : device fp32 [M, r] or NULL; when given, receives T = X A^T
@@ -219,7 +254,7 @@ typedef struct {
  * evaluated in fp64 in a fixed order (for each element: start from W', then for
  * a = 0, 1, ...: P = sum over j = 0 .. r_a - 1 of B_a[n, j] A_a[j, k] added in
  * that order, y = y + c_a * P), rounded once to bf16 (nearest, ties to even).
- *   q         : the base weight, W' = dequant(q), [rows, cols].
+ *   q         : the base weight (either storage kind), W' = dequant(q), [rows, cols].
  *   adapters  : host array of n_adapters entries (read before returning);
  *               0 <= n_adapters <= 8 (0 writes W' itself).
  *   W_out     : device bf16 [rows, cols] (16-byte aligned), overwritten.

@@ -15,7 +15,9 @@ page passage it follows:
 * "QLoRA: Efficient Finetuning of Quantized LLMs" (ai-papercheck.pages.dev
   errata list), findings quoting the paper's p.4 Section 2 and p.5 Section 3.
 * "QLoRA vs ChatGPT" (unfragile.ai compare page), capability blurbs 1 (NF4 with
-  block-wise absmax), 2 (LoRA on a frozen 4-bit base), 3 (double quantization),
+  block-wise absmax), 2 (LoRA on a frozen 4-bit base), 3 (double quantization,
+  contrasted with single-level constants; the errata page's p.8 Table 4
+  findings compare NFloat4 with and without DQ),
   5 (training pipeline: block-wise on-the-fly dequantization, gradients for
   the LoRA parameters only) and 6 (composing adapters and merging them into the
   base weights).
@@ -25,14 +27,16 @@ listed in the repository's design notes.
 """
 from .fp import bf16_bits_to_f32, f32_to_bf16_bits_rn, fma_f32
 from .nf4 import (BLOCK, DQ_BLOCK, nf4_codebook, quantize_nf4, double_quantize, quantize_nf4_dq,
-                  dequantize_nf4_dq, unpack_codes, storage_bytes, QuantizedNF4)
+                  dequantize_nf4_dq, unpack_codes, storage_bytes, QuantizedNF4, QuantizedNF4Single,
+                  quantize_nf4_single, dequantize_nf4_single)
 from .linear import lora_scale, linear_fwd, linear_bwd
 from .merge import f64_to_bf16_bits_rn, merge_lora, merge_scale
 
 __all__ = [
     "bf16_bits_to_f32", "f32_to_bf16_bits_rn", "fma_f32",
     "BLOCK", "DQ_BLOCK", "nf4_codebook", "quantize_nf4", "double_quantize", "quantize_nf4_dq",
-    "dequantize_nf4_dq", "unpack_codes", "storage_bytes", "QuantizedNF4",
+    "dequantize_nf4_dq", "unpack_codes", "storage_bytes", "QuantizedNF4", "QuantizedNF4Single",
+    "quantize_nf4_single", "dequantize_nf4_single",
     "lora_scale", "linear_fwd", "linear_bwd",
     "f64_to_bf16_bits_rn", "merge_lora", "merge_scale",
 ]

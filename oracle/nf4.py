@@ -18,6 +18,11 @@ Passages followed:
   8 bit and stored with their own scales, a nested hierarchy).
 * Dequantization: "QLoRA vs ChatGPT", capability 5 (weights are dequantized
   on the fly, block by block, in the forward pass).
+* Single-level storage (no double quantization): the QLoRA errata page,
+  findings on the paper's p.8 Table 4, which compares NFloat4 with and without
+  DQ; "QLoRA vs ChatGPT", capability 3, which contrasts the nested scheme with
+  keeping the constants as full-precision metadata. The first-level constants
+  m_b are stored as fp32 and used directly as the block scale.
 """
 from __future__ import annotations
 
@@ -218,6 +223,31 @@ def dequantize_nf4_dq(qw: QuantizedNF4, codebook: np.ndarray | None = None) -> n
     codes = unpack_codes(qw.packed).reshape(-1, BLOCK)
     mprime = dequant_constants(qw.absmax_q, qw.dq_scale, qw.mean)
     prod = (cb[codes] * mprime[:, None]).astype(np.float32)
+    return f32_to_bf16_bits_rn(prod).reshape(qw.rows, qw.cols)
+
+
+@dataclass
+class QuantizedNF4Single:
+    """Single-level NF4 storage of one [rows, cols] weight: codes and fp32 m_b."""
+    packed: np.ndarray     # uint8 [rows*cols/2]
+    absmax: np.ndarray     # fp32 [nblk]
+    rows: int
+    cols: int
+
+
+def quantize_nf4_single(W: np.ndarray, codebook: np.ndarray | None = None) -> QuantizedNF4Single:
+    """Level-1 quantization alone: the codes of quantize_nf4 and its exact m_b."""
+    cb = nf4_codebook() if codebook is None else codebook
+    codes, absmax = quantize_nf4(W, cb)
+    return QuantizedNF4Single(pack_codes(codes), absmax, W.shape[0], W.shape[1])
+
+
+def dequantize_nf4_single(qw: QuantizedNF4Single, codebook: np.ndarray | None = None) -> np.ndarray:
+    """w' = bf16_rn(fp32(c[code] * m_b)) with the stored m_b; bf16 bit patterns [rows, cols]."""
+    cb = (nf4_codebook() if codebook is None else codebook).astype(np.float32)
+    codes = unpack_codes(qw.packed).reshape(-1, BLOCK)
+    m = np.asarray(qw.absmax, dtype=np.float32)
+    prod = (cb[codes] * m[:, None]).astype(np.float32)
     return f32_to_bf16_bits_rn(prod).reshape(qw.rows, qw.cols)
 
 

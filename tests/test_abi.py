@@ -119,3 +119,59 @@ def test_merge_argument_errors_return_before_launch():
     assert lib.qlora_merge_lora(ctypes.byref(w), arr, 1, None, None) == 1            # no output
     assert lib.qlora_merge_lora(ctypes.byref(w), arr, 1, ctypes.c_void_p(fake + 2), None) == 3  # misaligned output
     assert lib.qlora_merge_lora(ctypes.byref(_weight(rows=0)), arr, 1, None, None) == 0  # empty weight
+
+
+def _single(rows=4, cols=128, **kw):
+    fake = 1 << 20  # aligned non-null dummies; nothing is launched
+    w = b._Weight(fake, None, None, None, rows, cols, 64, 0, fake)
+    for k, v in kw.items():
+        setattr(w, k, v)
+    return w
+
+
+def test_single_level_storage_bytes():
+    assert b.qlora_nf4_single_storage_bytes(4096, 4096) == (8388608, 1048576)
+    sb = oracle.storage_bytes(11008, 4096, double_quant=False)
+    assert b.qlora_nf4_single_storage_bytes(11008, 4096) == (sb["packed"], sb["absmax"])
+    assert sb["bits_per_param"] == 4.5  # 4-bit codes plus one fp32 constant per 64 weights
+    with pytest.raises(b.QloraError) as e:
+        b.qlora_nf4_single_storage_bytes(4, 100)
+    assert e.value.status == 2
+
+
+def test_single_level_argument_errors_return_before_launch():
+    lib = b.load_library()
+    W = ctypes.c_void_p(1 << 20)
+    n = ctypes.c_size_t(0)
+    fake = 1 << 20
+    # each quantizer accepts only its own storage kind
+    assert lib.qlora_quantize_nf4(W, ctypes.byref(_weight()), None) == 2
+    assert lib.qlora_quantize_nf4_dq(W, ctypes.byref(_single()), None, ctypes.byref(n), None) == 2
+    assert lib.qlora_quantize_nf4_dq_noalloc(W, ctypes.byref(_single()), None) == 2
+    # null or misaligned single-level storage, input or output
+    assert lib.qlora_quantize_nf4(W, ctypes.byref(_single(absmax=None)), None) == 1
+    assert lib.qlora_quantize_nf4(W, ctypes.byref(_single(packed=None)), None) == 1
+    assert lib.qlora_quantize_nf4(W, ctypes.byref(_single(absmax=fake + 2)), None) == 3
+    assert lib.qlora_quantize_nf4(W, ctypes.byref(_single(packed=fake + 8)), None) == 3
+    assert lib.qlora_quantize_nf4(None, ctypes.byref(_single()), None) == 1
+    assert lib.qlora_quantize_nf4(ctypes.c_void_p(fake + 2), ctypes.byref(_single()), None) == 3
+    assert lib.qlora_quantize_nf4(W, None, None) == 1
+    assert lib.qlora_quantize_nf4(W, ctypes.byref(_single(cols=100)), None) == 2
+    assert lib.qlora_quantize_nf4(W, ctypes.byref(_single(blocksize=32)), None) == 2
+    assert lib.qlora_quantize_nf4(W, ctypes.byref(_single(rows=0)), None) == 0  # nothing to do
+    # the dequantizers take either kind; other dq_blocksize values are unsupported
+    for fn in (lib.qlora_dequantize_nf4, lib.qlora_dequantize_nf4_dq):
+        assert fn(ctypes.byref(_single(absmax=None)), ctypes.c_void_p(fake), None) == 1
+        assert fn(ctypes.byref(_single()), None, None) == 1
+        assert fn(ctypes.byref(_single()), ctypes.c_void_p(fake + 2), None) == 3
+        assert fn(ctypes.byref(_single(dq_blocksize=128)), ctypes.c_void_p(fake), None) == 2
+        assert fn(ctypes.byref(_single(rows=0)), None, None) == 0
+    # the linear layer and the merge check the single-level storage the same way
+    assert lib.qlora_linear_fwd(ctypes.byref(_single(absmax=None)), W, 1, W, W, 16, 16.0, W, None, None,
+                                ctypes.byref(n), None) == 1
+    assert lib.qlora_linear_fwd(ctypes.byref(_single()), W, 1, W, W, 12, 16.0, W, None, None,
+                                ctypes.byref(n), None) == 2
+    assert lib.qlora_linear_fwd(ctypes.byref(_single()), W, 1, W, W, 16, 16.0, W, None, None,
+                                ctypes.byref(n), None) == 0 and n.value > 0  # size query
+    ok = (b._Adapter * 1)(b._Adapter(fake, fake, 16, 16.0, 1.0))
+    assert lib.qlora_merge_lora(ctypes.byref(_single(absmax=fake + 1)), ok, 1, ctypes.c_void_p(fake), None) == 3
