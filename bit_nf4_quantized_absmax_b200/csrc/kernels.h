@@ -25,11 +25,9 @@ cudaError_t ensure_smem_limit(int bytes) {
   return e;
 }
 
-// Quantize scratch besides the fp32 absmax: per-CTA exponent-bin sums of the
-// first pass (u32 [256][kQuantMaxGrid], bin-major) and the 256 bin totals (u64).
-constexpr int kQuantMaxGrid = 2048;
-constexpr size_t kQuantHistBytes = static_cast<size_t>(256) * kQuantMaxGrid * sizeof(unsigned int);
-constexpr size_t kQuantScratchBytes = kQuantHistBytes + 256 * sizeof(unsigned long long);
+// Quantize scratch besides the fp32 absmax: the 256 exponent-bin totals (u64)
+// of the exact sum of the constants.
+constexpr size_t kQuantScratchBytes = 256 * sizeof(unsigned long long);
 
 // Number of non-empty pieces when `nkb` k-blocks are cut into pieces of
 // ceil(nkb / want) blocks. The split-reduction GEMMs and the kernels that sum
@@ -44,7 +42,7 @@ inline int split_count(int64_t nkb, int want) {
 
 // ---- quantize.cu / dequant.cu ----
 cudaError_t launch_quantize(const void* W, int64_t numel, uint8_t* packed, int8_t* absmax_q, float* dq_scale,
-                            float* mean, float* absmax_scratch, void* hist_scratch, int num_sms,
+                            float* mean, float* absmax_scratch, void* totals_scratch, int num_sms,
                             cudaStream_t stream);
 
 // Single-level storage: the codes and the fp32 block constants m_b only (pass 1).

@@ -2,16 +2,16 @@
 // the absmax constants ("QLoRA vs ChatGPT", capabilities 1 and 3; "Guanaco",
 // "Core Architecture & Training").
 //
-// Three launches:
+// Three launches (the first alone gives single-level storage):
 //   k_quant_pass1  streams W once, four lanes per 64-weight block (one 32-byte
-//                  load each, 1 KB contiguous per warp instruction): the absmax (packed 16-bit max of the magnitude bits), the exact
-//                  quotient v = w / m, the nearest code (one lookup in a 32-bin
-//                  table + one compare), 4-bit packing; it also accumulates the
-//                  exact sum of the absmax constants as integer significand sums
-//                  per exponent.
-//                  The last CTA to finish turns that sum into the mean.
-//   k_dq_quantize  forms the mean from the exact bin totals (every CTA, warp 0),
-//                  then one warp per 256 constants: centre on the mean, group
+//                  load each, 1 KB contiguous per warp instruction): the absmax
+//                  (packed 16-bit max of the magnitude bits), stored as fp32,
+//                  the exact quotient v = w / m, the nearest code (one lookup in
+//                  a 32-bin table + one compare), 4-bit packing.
+//   k_quant_sums   the exact sum of the absmax constants, as integer sums of
+//                  their 8-bit significands per exponent (order-independent).
+//   k_dq_quantize  forms the mean from those totals (every CTA, warp 0), then
+//                  one warp per 256 constants: centre on the mean, group
 //                  absmax, int8 codes with round-to-nearest-even.
 #include "common.cuh"
 #include "host_tables.h"
@@ -129,15 +129,12 @@ __device__ __forceinline__ void encode16(const uint32_t (&d)[8], float ms, float
 }
 
 // Four lanes per 64-weight block (16 weights each, one 32-byte load): a warp
-// reads 1 KB of contiguous weights per load instruction. Every lane of a warp
-// runs the same iterations so that the histogram update can be combined across
-// the warp (lanes whose blocks share an exponent add their significands first,
-// then one of them updates the shared bin). Without HIST (single-level
-// storage, no mean needed) the histogram work is left out.
-template <bool V8, bool HIST>
+// reads 1 KB of contiguous weights per load instruction, and every lane of a
+// warp runs the same iterations (the block's four lanes share its absmax
+// through two shuffles).
+template <bool V8>
 __device__ __forceinline__ void pass1_loop(const uint4* __restrict__ W, int64_t nblk, uint32_t* __restrict__ packed,
-                                           float* __restrict__ absmax, const unsigned char* bins,
-                                           unsigned int* __restrict__ s_hist) {
+                                           float* __restrict__ absmax, const unsigned char* bins) {
   const int lane = threadIdx.x & 31;
   const int qtr = lane & 3;
   const int64_t stride = static_cast<int64_t>(gridDim.x) * (kPass1Threads / 4);
@@ -165,16 +162,8 @@ __device__ __forceinline__ void pass1_loop(const uint4* __restrict__ W, int64_t 
     mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
     mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
     const float m = __uint_as_float(mx << 16);  // block absmax (exact)
-    uint32_t hE = 0u, hsig = 0u;  // the block's share of the exact sum: significand hsig at exponent bin hE
     if (valid) {
-      if (qtr == 0) {
-        absmax[blk] = m;
-        const uint32_t u = __float_as_uint(m);
-        const uint32_t e = u >> 23;
-        const uint32_t mant7 = (u >> 16) & 0x7Fu;
-        hE = e ? e : 1u;
-        hsig = e ? (mant7 | 0x80u) : mant7;
-      }
+      if (qtr == 0) absmax[blk] = m;
       uint32_t out[2];
       if (m == 0.0f) {
         out[0] = out[1] = 0x77777777u;  // an all-zero block: every code is the exact zero
@@ -193,51 +182,61 @@ __device__ __forceinline__ void pass1_loop(const uint4* __restrict__ W, int64_t 
       }
       *reinterpret_cast<uint2*>(packed + blk * 8 + qtr * 2) = make_uint2(out[0], out[1]);
     }
-    if (HIST) {
-      const unsigned int same = __match_any_sync(0xffffffffu, hE);
-      const unsigned int tot = __reduce_add_sync(same, hsig);
-      if (lane == __ffs(same) - 1 && tot) atomicAdd(&s_hist[hE], tot);
-    }
   }
 }
 
-template <bool HIST>
+// zero_totals (double-quantized storage only): the 256 bin totals that
+// k_quant_sums adds into, cleared here by CTA 0 before that kernel starts.
 __global__ void __launch_bounds__(kPass1Threads)
 k_quant_pass1(const uint4* __restrict__ W, bool v8, uint32_t* __restrict__ packed,
-              float* __restrict__ absmax, unsigned int* __restrict__ hist_part, int64_t nblk,
+              float* __restrict__ absmax, unsigned long long* __restrict__ zero_totals, int64_t nblk,
               const __grid_constant__ QuantBinTable tab) {
   __shared__ uint2 s_bins[kBins];
-  __shared__ unsigned int s_hist[256];          // per-CTA significand sums (native 32-bit atomics)
   const int tid = threadIdx.x;
   if (tid < kBins) s_bins[tid] = make_uint2(__float_as_uint(tab.bins[tid].threshold), tab.bins[tid].j + 1u);
-  if (HIST) s_hist[tid] = 0u;
   __syncthreads();
   pdl_enter();
+  if (zero_totals && blockIdx.x == 0) zero_totals[tid] = 0ull;  // kPass1Threads == 256 bins
 
   const unsigned char* bins = reinterpret_cast<const unsigned char*>(s_bins);
   if (v8)
-    pass1_loop<true, HIST>(W, nblk, packed, absmax, bins, s_hist);
+    pass1_loop<true>(W, nblk, packed, absmax, bins);
   else
-    pass1_loop<false, HIST>(W, nblk, packed, absmax, bins, s_hist);
-  if (HIST) {
-    __syncthreads();
-    hist_part[static_cast<int64_t>(tid) * kQuantMaxGrid + blockIdx.x] = s_hist[tid];  // bin-major
-  }
+    pass1_loop<false>(W, nblk, packed, absmax, bins);
 }
 
-// totals[e] = sum over the pass-1 CTAs of their bin e (one CTA per bin).
-__global__ void __launch_bounds__(128)
-k_quant_bins(const unsigned int* __restrict__ hist_part, int grid, unsigned long long* __restrict__ totals) {
-  __shared__ unsigned long long red[4];
-  pdl_enter();
-  const unsigned int* row = hist_part + static_cast<int64_t>(blockIdx.x) * kQuantMaxGrid;
-  unsigned long long v = 0ull;
-  for (int i = threadIdx.x; i < grid; i += blockDim.x) v += row[i];
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+// totals[e] += the 8-bit significands of the constants with exponent bin e (a
+// constant m = sig * 2^(E - 134), E = max(exponent field, 1)). Each CTA takes a
+// contiguous chunk of at most 2^24 constants, so its 32-bit shared bins cannot
+// overflow; lanes that share a bin add first (match + reduce), then one shared
+// atomic; then one 64-bit global atomic per nonzero bin. Integer additions in
+// any order give the same totals.
+__global__ void __launch_bounds__(256)
+k_quant_sums(const float* __restrict__ absmax, int64_t nblk, int64_t per_cta,
+             unsigned long long* __restrict__ totals) {
+  __shared__ unsigned int s_hist[256];
+  s_hist[threadIdx.x] = 0u;
   __syncthreads();
-  if (threadIdx.x == 0) totals[blockIdx.x] = red[0] + red[1] + red[2] + red[3];
+  pdl_enter();
+  const int lane = threadIdx.x & 31;
+  const int64_t b0 = static_cast<int64_t>(blockIdx.x) * per_cta;
+  const int64_t b1 = b0 + per_cta < nblk ? b0 + per_cta : nblk;
+  for (int64_t i = b0 + threadIdx.x; i - lane < b1; i += blockDim.x) {  // warp-uniform trip count
+    uint32_t hE = 1u, hsig = 0u;
+    if (i < b1) {
+      const uint32_t u = __float_as_uint(__ldg(absmax + i));
+      const uint32_t e = u >> 23;
+      const uint32_t mant7 = (u >> 16) & 0x7Fu;
+      hE = e ? e : 1u;
+      hsig = e ? (mant7 | 0x80u) : mant7;
+    }
+    const unsigned int same = __match_any_sync(0xffffffffu, hE);
+    const unsigned int tot = __reduce_add_sync(same, hsig);
+    if (lane == __ffs(same) - 1 && tot) atomicAdd(&s_hist[hE], tot);
+  }
+  __syncthreads();
+  const unsigned int v = s_hist[threadIdx.x];
+  if (v) atomicAdd(&totals[threadIdx.x], static_cast<unsigned long long>(v));
 }
 
 // mu = fp32(RN_fp64(S) / nblk) from the exact bin totals (warp 0 of the CTA);
@@ -333,49 +332,52 @@ k_dq_quantize(const float* __restrict__ absmax, int64_t nblk, const unsigned lon
 
 // Persistent grid of pass 1: exactly the CTAs that are resident at once (four
 // lanes per 64-weight block), so no SM idles through a partial last wave.
-template <bool HIST>
 int pass1_grid(int64_t nblk, int num_sms) {
   static std::atomic<int> per_sm_cache{0};  // the same on every B200; racing writers store equal values
   int per_sm = per_sm_cache.load(std::memory_order_relaxed);
   if (per_sm == 0) {
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_quant_pass1<HIST>, kPass1Threads, 0) !=
-            cudaSuccess ||
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_quant_pass1, kPass1Threads, 0) != cudaSuccess ||
         per_sm < 1)
       per_sm = 4;
     per_sm_cache.store(per_sm, std::memory_order_relaxed);
   }
-  int64_t want = (nblk * 4 + kPass1Threads - 1) / kPass1Threads;
-  int64_t cap = static_cast<int64_t>(num_sms) * per_sm;
-  if (cap > kQuantMaxGrid) cap = kQuantMaxGrid;
-  int64_t g = want < cap ? (want > 0 ? want : 1) : cap;
-  // A CTA sums at most 2^24 significands of 8 bits, so its 32-bit bins cannot overflow.
-  const int64_t min_grid = (nblk + (int64_t(1) << 24) - 1) >> 24;
-  if (g < min_grid) g = min_grid;
-  return g > kQuantMaxGrid ? -1 : static_cast<int>(g);  // -1: more than 2^35 blocks
+  const int64_t want = (nblk * 4 + kPass1Threads - 1) / kPass1Threads;
+  const int64_t cap = static_cast<int64_t>(num_sms) * per_sm;
+  const int64_t g = want < cap ? (want > 0 ? want : 1) : cap;
+  return static_cast<int>(g);
+}
+
+cudaError_t launch_pass1(const void* W, int64_t nblk, uint8_t* packed, float* absmax, unsigned long long* zero_totals,
+                         int num_sms, cudaStream_t stream) {
+  const QuantTables& tabs = quant_tables();
+  QuantBinTable tab;
+  for (int i = 0; i < kBins; ++i) tab.bins[i] = tabs.bins[i];
+  const bool v8 = ((reinterpret_cast<uintptr_t>(W) | reinterpret_cast<uintptr_t>(packed)) & 31u) == 0;
+  return launch_pdl(k_quant_pass1, dim3(pass1_grid(nblk, num_sms)), dim3(kPass1Threads), 0, stream,
+                    reinterpret_cast<const uint4*>(W), v8, reinterpret_cast<uint32_t*>(packed), absmax, zero_totals,
+                    nblk, tab);
 }
 
 }  // namespace
 
 cudaError_t launch_quantize(const void* W, int64_t numel, uint8_t* packed, int8_t* absmax_q, float* dq_scale,
-                            float* mean, float* absmax_scratch, void* hist_scratch, int num_sms,
+                            float* mean, float* absmax_scratch, void* totals_scratch, int num_sms,
                             cudaStream_t stream) {
-  const QuantTables& tabs = quant_tables();
-  QuantBinTable tab;
-  for (int i = 0; i < kBins; ++i) tab.bins[i] = tabs.bins[i];
   const int64_t nblk = numel / 64;
   const int64_t ngrp = (nblk + 255) / 256;
-  unsigned int* hist_part = static_cast<unsigned int*>(hist_scratch);
-  unsigned long long* totals =
-      reinterpret_cast<unsigned long long*>(static_cast<char*>(hist_scratch) + kQuantHistBytes);
-  const int grid = pass1_grid<true>(nblk, num_sms);
-  if (grid < 0) return cudaErrorInvalidValue;
-  const bool v8 = ((reinterpret_cast<uintptr_t>(W) | reinterpret_cast<uintptr_t>(packed)) & 31u) == 0;
-  cudaError_t e = launch_pdl(k_quant_pass1<true>, dim3(grid), dim3(kPass1Threads), 0, stream,
-                             reinterpret_cast<const uint4*>(W), v8, reinterpret_cast<uint32_t*>(packed),
-                             absmax_scratch, hist_part, nblk, tab);
+  unsigned long long* totals = static_cast<unsigned long long*>(totals_scratch);
+  cudaError_t e = launch_pass1(W, nblk, packed, absmax_scratch, totals, num_sms, stream);
   if (e != cudaSuccess) return e;
-  e = launch_pdl(k_quant_bins, dim3(256), dim3(128), 0, stream, static_cast<const unsigned int*>(hist_part), grid,
-                 totals);
+  // chunks of at least 2048 constants, at most two CTAs per SM, and at most 2^24 constants each
+  int64_t g = (nblk + 2047) / 2048;
+  if (g > 2 * num_sms) g = 2 * num_sms;
+  const int64_t min_g = (nblk + (int64_t(1) << 24) - 1) >> 24;
+  if (g < min_g) g = min_g;
+  if (g < 1) g = 1;
+  if (g > 0x7fffffff) return cudaErrorInvalidValue;
+  const int64_t per_cta = (nblk + g - 1) / g;
+  e = launch_pdl(k_quant_sums, dim3(static_cast<unsigned>(g)), dim3(256), 0, stream,
+                 static_cast<const float*>(absmax_scratch), nblk, per_cta, totals);
   if (e != cudaSuccess) return e;
   const int dq_grid = static_cast<int>((ngrp + 7) / 8);
   return launch_pdl(k_dq_quantize, dim3(dq_grid), dim3(256), 0, stream, static_cast<const float*>(absmax_scratch),
@@ -384,16 +386,7 @@ cudaError_t launch_quantize(const void* W, int64_t numel, uint8_t* packed, int8_
 
 cudaError_t launch_quantize_single(const void* W, int64_t numel, uint8_t* packed, float* absmax, int num_sms,
                                    cudaStream_t stream) {
-  const QuantTables& tabs = quant_tables();
-  QuantBinTable tab;
-  for (int i = 0; i < kBins; ++i) tab.bins[i] = tabs.bins[i];
-  const int64_t nblk = numel / 64;
-  const int grid = pass1_grid<false>(nblk, num_sms);
-  if (grid < 0) return cudaErrorInvalidValue;
-  const bool v8 = ((reinterpret_cast<uintptr_t>(W) | reinterpret_cast<uintptr_t>(packed)) & 31u) == 0;
-  return launch_pdl(k_quant_pass1<false>, dim3(grid), dim3(kPass1Threads), 0, stream,
-                    reinterpret_cast<const uint4*>(W), v8, reinterpret_cast<uint32_t*>(packed), absmax,
-                    static_cast<unsigned int*>(nullptr), nblk, tab);
+  return launch_pass1(W, numel / 64, packed, absmax, nullptr, num_sms, stream);
 }
 
 }  // namespace qlora

@@ -4,9 +4,9 @@
 // forbid allocation afterwards, and hosts where cudaMalloc's implicit device
 // synchronization would stall other work.
 //
-// The scratch the quantize kernels need (per-CTA exponent-bin sums and their
-// totals, and one fp32 absmax per 64-weight block) lives in a file-scope device array of a
-// fixed size. Every GPU that loads this code holds that array until the process
+// The scratch the quantize kernels need (the exponent-bin totals of the exact
+// sum of the constants, and one fp32 absmax per 64-weight block) lives in a
+// file-scope device array of a fixed size. Every GPU that loads this code holds that array until the process
 // exits. All calls share it, so calls that overlap on the GPU (different
 // streams, or different host threads on one device) race and must be ordered by
 // the caller. Every region is fully written by a kernel of the call before
@@ -21,7 +21,7 @@
 namespace {
 
 // At most 2^22 blocks of 64 weights (268,435,456 weights, e.g. any single
-// Llama-65B linear weight): 2 MiB of bin sums + 16 MiB of absmax per device.
+// Llama-65B linear weight): 2 KiB of bin totals + 16 MiB of absmax per device.
 constexpr int64_t kNoAllocMaxBlocks = int64_t(1) << 22;
 constexpr size_t kBinsBytes = (qlora::kQuantScratchBytes + 255) / 256 * 256;
 constexpr size_t kScratchBytes = kBinsBytes + static_cast<size_t>(kNoAllocMaxBlocks) * sizeof(float);
