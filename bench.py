@@ -390,6 +390,47 @@ def merge_measure(work, dev, reps=10):
             "frac": round(flops / us / 1e6 / 40.0, 4)}
 
 
+def adamw_measure(dev, peaks, n=1 << 26, reps=10):
+    """Paged AdamW step (outside the step) over n flat fp32 parameters with bf16
+    gradients: once with device-resident state, once with the moments in paged
+    (managed) memory prefetched to the GPU. 28 bytes per parameter: p, m, v read
+    and written (24), the bf16 gradient read and the bf16 copy of p written (4)."""
+    import ctypes
+    lib = qb.load_library()
+    st = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    p = torch.randn(n, device=dev) * 0.02
+    g = (torch.randn(n, device=dev) * 1e-2).to(torch.bfloat16)
+    pb = torch.empty(n, dtype=torch.bfloat16, device=dev)
+    m, v = torch.zeros(n, device=dev), torch.zeros(n, device=dev)
+    bm, bv = qb.PagedBuffer(4 * n), qb.PagedBuffer(4 * n)
+    mp, vp = bm.tensor(torch.float32, n), bv.tensor(torch.float32, n)
+    mp.zero_()
+    vp.zero_()
+    bm.prefetch(bm.device)
+    bv.prefetch(bv.device)
+    out = {"n": n, "bytes_per_param": 28}
+    for name, (mm, vv) in (("device", (m, v)), ("paged", (mp, vp))):
+        def call(t):
+            return lib.qlora_adamw_step(qb._ptr(p), qb._ptr(pb), qb._ptr(g), qb._ptr(mm), qb._ptr(vv), n, 1e-4, 0.9,
+                                        0.999, 1e-8, 0.0, t, st)
+        for t in range(1, 3):
+            call(t)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for t in range(3, 3 + reps):
+            if call(t) != 0:
+                raise qb.QloraError(1, "qlora_adamw_step")
+        b.record()
+        torch.cuda.synchronize()
+        us = 1e3 * a.elapsed_time(b) / reps
+        gbs = 28.0 * n / us / 1e3
+        out[name] = {"us": round(us, 1), "GB_s": round(gbs, 1), "hbm_frac": round(gbs / peaks["hbm_gbs"], 4)}
+    del mp, vp
+    bm.free()
+    bv.free()
+    return out
+
+
 def run_ours(args, rank, world, dev):
     def say(msg):  # progress on stderr (stdout carries only the JSON line)
         if args.verbose or rank == 0:
@@ -501,6 +542,8 @@ def run_ours(args, rank, world, dev):
 
     say("adapter merge")
     merge = merge_measure(work, dev)
+    say("paged AdamW")
+    adamw = adamw_measure(dev, peaks)
     say("end to end with host buffers")
     # end to end through the C ABI with host buffers
     host = []
@@ -543,6 +586,7 @@ def run_ours(args, rank, world, dev):
         "parts": parts,
         "roofline": roof,
         "merge": merge,
+        "adamw": adamw,
         "e2e": {"value": round(world * fl_train / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
                 "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": work.launches_per_step() * args.steps,

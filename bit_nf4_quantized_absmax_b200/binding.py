@@ -23,6 +23,7 @@ STATUS_NAMES = {0: "QLORA_OK", 1: "QLORA_ERR_INVALID_ARG", 2: "QLORA_ERR_UNSUPPO
 EXPORTED = ("qlora_status_string", "qlora_nf4_codebook", "qlora_nf4_storage_bytes", "qlora_nf4_single_storage_bytes",
             "qlora_quantize_nf4", "qlora_quantize_nf4_dq", "qlora_quantize_nf4_dq_noalloc", "qlora_dequantize_nf4",
             "qlora_dequantize_nf4_dq", "qlora_linear_fwd", "qlora_linear_bwd", "qlora_merge_lora",
+            "qlora_paged_alloc", "qlora_paged_free", "qlora_paged_prefetch", "qlora_adamw_step",
             "qlora_device_error")
 
 
@@ -72,6 +73,10 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
     lib.qlora_linear_bwd.argtypes = [wp, vp, i64, vp, vp, i32, f32, vp, vp, vp, vp, vp, vp, szp, vp]
     lib.qlora_merge_lora.argtypes = [wp, ctypes.POINTER(_Adapter), i32, vp, vp]
     lib.qlora_device_error.argtypes = [ctypes.POINTER(ctypes.c_int32), vp]
+    lib.qlora_paged_alloc.argtypes = [sz, i32, ctypes.POINTER(vp)]
+    lib.qlora_paged_free.argtypes = [vp]
+    lib.qlora_paged_prefetch.argtypes = [vp, sz, i32, vp]
+    lib.qlora_adamw_step.argtypes = [vp, vp, vp, vp, vp, i64, f32, f32, f32, f32, f32, i64, vp]
     for name in EXPORTED:
         getattr(lib, name).restype = ctypes.c_int if name != "qlora_status_string" else ctypes.c_char_p
     _lib = lib
@@ -286,3 +291,58 @@ def qlora_device_error(stream=None) -> int:
     code = ctypes.c_int32(0)
     _check(load_library().qlora_device_error(ctypes.byref(code), _stream(stream)), "qlora_device_error")
     return int(code.value)
+
+
+class PagedBuffer:
+    """Paged (managed) device memory from qlora_paged_alloc, freed with the object
+    or by free(). tensor(dtype, n) views it as a torch tensor; keep the buffer
+    alive while such views are in use."""
+
+    def __init__(self, nbytes: int, device: int | None = None):
+        dev = torch.cuda.current_device() if device is None else device
+        ptr = ctypes.c_void_p()
+        _check(load_library().qlora_paged_alloc(nbytes, dev, ctypes.byref(ptr)), "qlora_paged_alloc")
+        self.ptr, self.nbytes, self.device = ptr.value, nbytes, dev
+
+    def tensor(self, dtype: torch.dtype, n: int) -> torch.Tensor:
+        itemsize = torch.empty(0, dtype=dtype).element_size()
+        assert n * itemsize <= self.nbytes
+        typestr = {torch.float32: "<f4", torch.bfloat16: "<i2", torch.uint8: "|u1"}[dtype]
+        owner = self
+
+        class _View:
+            __cuda_array_interface__ = {"shape": (n,), "typestr": typestr, "data": (owner.ptr, False),
+                                        "version": 3, "strides": None}
+        t = torch.as_tensor(_View(), device=f"cuda:{self.device}")
+        return t.view(dtype) if dtype == torch.bfloat16 else t
+
+    def prefetch(self, device: int, stream=None):
+        """Move the buffer to GPU `device`, or to host memory with device == -1."""
+        _check(load_library().qlora_paged_prefetch(ctypes.c_void_p(self.ptr), self.nbytes, device, _stream(stream)),
+               "qlora_paged_prefetch")
+
+    def free(self):
+        if self.ptr:
+            _check(load_library().qlora_paged_free(ctypes.c_void_p(self.ptr)), "qlora_paged_free")
+            self.ptr = None
+
+    def __del__(self):
+        try:
+            if self.ptr:
+                torch.cuda.synchronize(self.device)
+                self.free()
+        except Exception:  # noqa: BLE001 -- interpreter shutdown
+            pass
+
+
+def qlora_adamw_step(param: torch.Tensor, grad: torch.Tensor, exp_avg: torch.Tensor, exp_avg_sq: torch.Tensor,
+                     step: int, lr: float = 1e-3, beta1: float = 0.9, beta2: float = 0.999, eps: float = 1e-8,
+                     weight_decay: float = 0.0, param_bf16: torch.Tensor | None = None, stream=None):
+    """One AdamW step over flat fp32 parameters with bf16 gradients (see include/qlora.h)."""
+    assert param.dtype == torch.float32 and exp_avg.dtype == torch.float32 and exp_avg_sq.dtype == torch.float32
+    assert grad.dtype == torch.bfloat16
+    n = param.numel()
+    assert grad.numel() == n and exp_avg.numel() == n and exp_avg_sq.numel() == n
+    _check(load_library().qlora_adamw_step(_ptr(param), _ptr(param_bf16), _ptr(grad), _ptr(exp_avg),
+                                           _ptr(exp_avg_sq), n, float(lr), float(beta1), float(beta2), float(eps),
+                                           float(weight_decay), int(step), _stream(stream)), "qlora_adamw_step")

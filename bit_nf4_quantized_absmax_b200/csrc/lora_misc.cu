@@ -64,6 +64,9 @@ __global__ void k_lora_finish(const float* __restrict__ P, int splits, int64_t M
 // columns kept). A CTA owns a 32-row x 64-column tile: coalesced float2 reads of
 // every split (fixed order), then either direct row-major writes ([R, r]) or a
 // transpose through shared memory so that the [r, R] writes are coalesced too.
+// One CTA per 32 rows x 64 columns; thread (ty, tx) sums the split partials of
+// rows ty and ty + 16, columns 4 tx .. 4 tx + 3 (float4 loads), with the loads
+// of four splits in flight at a time; the sum runs over p = 0, 1, ... in order.
 __global__ void __launch_bounds__(256)
 k_grad_reduce(const float* __restrict__ P, int splits, int64_t R, int rpad, int r, float s, int transpose,
               __nv_bfloat16* __restrict__ out) {
@@ -71,37 +74,54 @@ k_grad_reduce(const float* __restrict__ P, int splits, int64_t R, int rpad, int 
   __shared__ float tile[64][33];
   const int64_t row0 = static_cast<int64_t>(blockIdx.x) * 32;
   const int col0 = blockIdx.y * 64;
-  const int tx = threadIdx.x & 31;   // column pair within the tile
-  const int ty = threadIdx.x >> 5;   // 8 row lanes
-  for (int rr = ty; rr < 32; rr += 8) {
+  const int tx = threadIdx.x & 15;   // column quad within the tile
+  const int ty = threadIdx.x >> 4;   // 16 row lanes
+  const int64_t pstride = R * rpad / 4;  // float4 elements per split
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int rr = ty + 16 * h;
     const int64_t row = row0 + rr;
-    float2 v = make_float2(0.0f, 0.0f);
+    float4 v = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
     if (row < R) {
-      for (int p = 0; p < splits; ++p) {
-        const float2 pv =
-            reinterpret_cast<const float2*>(P + (static_cast<int64_t>(p) * R + row) * rpad + col0)[tx];
-        v.x += pv.x;
-        v.y += pv.y;
+      const float4* src = reinterpret_cast<const float4*>(P + row * rpad + col0) + tx;
+      int p = 0;
+      for (; p + 4 <= splits; p += 4) {
+        float4 q[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) q[i] = __ldcs(src + (p + i) * pstride);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          v.x += q[i].x; v.y += q[i].y; v.z += q[i].z; v.w += q[i].w;
+        }
+      }
+      for (; p < splits; ++p) {
+        const float4 q = __ldcs(src + p * pstride);
+        v.x += q.x; v.y += q.y; v.z += q.z; v.w += q.w;
       }
     }
-    const int c = 2 * tx;
+    const int c = 4 * tx;
     if (!transpose) {
       if (row < R) {
-        if (col0 + c < r) out[row * r + col0 + c] = __float2bfloat16_rn(s * v.x);
-        if (col0 + c + 1 < r) out[row * r + col0 + c + 1] = __float2bfloat16_rn(s * v.y);
+        const float vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          if (col0 + c + i < r) out[row * r + col0 + c + i] = __float2bfloat16_rn(s * vv[i]);
       }
     } else {
       tile[c][rr] = v.x;
       tile[c + 1][rr] = v.y;
+      tile[c + 2][rr] = v.z;
+      tile[c + 3][rr] = v.w;
     }
   }
   if (!transpose) return;
   __syncthreads();
   // out[j][row]: 32 consecutive rows per column j, one warp per column
-  for (int cc = ty; cc < 64; cc += 8) {
+  const int wx = threadIdx.x & 31, wy = threadIdx.x >> 5;
+  for (int cc = wy; cc < 64; cc += 8) {
     const int j = col0 + cc;
-    const int64_t row = row0 + tx;
-    if (j < r && row < R) out[static_cast<int64_t>(j) * R + row] = __float2bfloat16_rn(s * tile[cc][tx]);
+    const int64_t row = row0 + wx;
+    if (j < r && row < R) out[static_cast<int64_t>(j) * R + row] = __float2bfloat16_rn(s * tile[cc][wx]);
   }
 }
 

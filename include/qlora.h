@@ -10,7 +10,9 @@
  *   4. block-wise dequantization back to bf16,
  *   5. the QLoRA linear layer  Y = X W'^T + s (X A^T) B^T  (W' = dequant(W)),
  *      forward and backward (dX, dA, dB; W stays frozen, no dW),
- *   6. merging weighted LoRA adapters into the base weight.
+ *   6. merging weighted LoRA adapters into the base weight,
+ *   7. paged AdamW for the LoRA parameters (optimizer state in managed memory
+ *      that pages between GPU and CPU).
  *
  * Sources (web pages describing the method; no code is printed on them):
  *   [G]  "Guanaco" (chipfoundryservices.com/topic/guanaco), sections
@@ -20,16 +22,17 @@
  *        p.5 Section 3.
  *   [C]  "QLoRA vs ChatGPT" (unfragile.ai compare page), capability blurbs
  *        1 (NF4, block-wise absmax), 2 (LoRA on a frozen 4-bit base),
- *        3 (double quantization), 5 (on-the-fly block-wise dequantization,
- *        gradients only for the LoRA parameters) and 6 (adapter composition
- *        and merging).
+ *        3 (double quantization), 4 (paged optimizers), 5 (on-the-fly
+ *        block-wise dequantization, gradients only for the LoRA parameters)
+ *        and 6 (adapter composition and merging).
  *
  * Conventions for every call below:
  *   - bf16 tensors are passed as void*, row-major and contiguous, with base
  *     addresses aligned to 16 bytes (else QLORA_ERR_ALIGNMENT).
  *   - Device pointers are owned by the caller. The library never allocates,
- *     frees or synchronizes: every kernel is launched asynchronously on the
- *     given stream. Argument, shape and alignment errors are returned before
+ *     frees or synchronizes (except qlora_paged_alloc / qlora_paged_free, whose
+ *     purpose that is): every kernel is launched asynchronously on the given
+ *     stream. Argument, shape and alignment errors are returned before
  *     anything is launched; a launch failure returns QLORA_ERR_CUDA.
  *   - Outputs are overwritten (no accumulation into them).
  *   - Workspace: calls that need scratch device memory take (workspace,
@@ -263,6 +266,52 @@ typedef struct {
  * ALIGNMENT, CUDA, DEVICE. */
 qlora_status qlora_merge_lora(const qlora_nf4_weight* q, const qlora_lora_adapter* adapters,
                               int32_t n_adapters, void* W_out, qlora_stream_t stream);
+
+/* qlora_paged_alloc -- allocate `bytes` of paged memory for optimizer state
+ * ([C] 4: a unified pool that pages between GPU and CPU memory, so the state
+ * need not be pre-allocated in device memory; [G] "Core Architecture &
+ * Training": paged optimizers). The memory is CUDA managed memory whose
+ * preferred location is GPU `device`: its pages live in that GPU's memory while
+ * it has room, move to host memory under memory pressure and move back when a
+ * kernel touches them. Unlike every other call, this one allocates; free with
+ * qlora_paged_free. *out receives the pointer (NULL on error). Contents are
+ * uninitialized.
+ * Errors: INVALID_ARG (NULL out, bytes == 0, no such device), CUDA. */
+qlora_status qlora_paged_alloc(size_t bytes, int32_t device, void** out);
+
+/* qlora_paged_free -- free memory from qlora_paged_alloc (NULL is a no-op). The
+ * caller orders it after every kernel that uses the memory. Errors: CUDA. */
+qlora_status qlora_paged_free(void* p);
+
+/* qlora_paged_prefetch -- move [p, p + bytes) of paged memory asynchronously on
+ * `stream` to GPU `device`, or to host memory with device == -1: to device
+ * before the optimizer step, back to the host after it when device memory is
+ * needed for something else. The data are unchanged.
+ * Errors: INVALID_ARG (NULL p, device < -1 or no such device), CUDA. */
+qlora_status qlora_paged_prefetch(const void* p, size_t bytes, int32_t device, qlora_stream_t stream);
+
+/* qlora_adamw_step -- one AdamW update (decoupled weight decay) of n
+ * parameters held as flat buffers (lay out every LoRA A and B of a model
+ * contiguously to update them with one call). Step t >= 1:
+ *   p <- p * (1 - lr * weight_decay)
+ *   m <- beta1 * m + (1 - beta1) * g
+ *   v <- beta2 * v + (1 - beta2) * g^2
+ *   p <- p - (lr / (1 - beta1^t)) * m / (sqrt(v) / sqrt(1 - beta2^t) + eps)
+ * with the bias corrections computed in double precision on the host and the
+ * rest in fp32 on the device. (The pages name the paged optimizer but print no
+ * formula; this is the usual AdamW with 32-bit state, the library's reading.)
+ *   param      : device fp32 [n] master parameters, updated in place (16-byte aligned).
+ *   param_bf16 : device bf16 [n] or NULL; receives bf16_rn(p) for the next
+ *                forward (8-byte aligned).
+ *   grad_bf16  : device bf16 [n] gradients, e.g. dA and dB of qlora_linear_bwd
+ *                (8-byte aligned).
+ *   exp_avg, exp_avg_sq : fp32 [n] first and second moments (16-byte aligned),
+ *                zero before the first step; device or paged memory.
+ * Errors: INVALID_ARG (n < 0, step < 1, beta outside [0, 1), eps <= 0, lr < 0,
+ * weight_decay < 0, NULL pointers when n > 0), ALIGNMENT, CUDA, DEVICE. */
+qlora_status qlora_adamw_step(float* param, void* param_bf16, const void* grad_bf16, float* exp_avg,
+                              float* exp_avg_sq, int64_t n, float lr, float beta1, float beta2, float eps,
+                              float weight_decay, int64_t step, qlora_stream_t stream);
 
 /* qlora_device_error -- read and clear the library's device-side error word on
  * the current device (synchronizes the stream). Kernels whose waits on

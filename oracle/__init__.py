@@ -18,9 +18,9 @@ page passage it follows:
   block-wise absmax), 2 (LoRA on a frozen 4-bit base), 3 (double quantization,
   contrasted with single-level constants; the errata page's p.8 Table 4
   findings compare NFloat4 with and without DQ),
-  5 (training pipeline: block-wise on-the-fly dequantization, gradients for
-  the LoRA parameters only) and 6 (composing adapters and merging them into the
-  base weights).
+  4 (paged optimizers), 5 (training pipeline: block-wise on-the-fly
+  dequantization, gradients for the LoRA parameters only) and 6 (composing
+  adapters and merging them into the base weights).
 
 Where the pages are silent the oracle takes one stated reading; every reading is
 listed in the repository's design notes.
@@ -31,6 +31,7 @@ from .nf4 import (BLOCK, DQ_BLOCK, nf4_codebook, quantize_nf4, double_quantize, 
                   quantize_nf4_single, dequantize_nf4_single)
 from .linear import lora_scale, linear_fwd, linear_bwd
 from .merge import f64_to_bf16_bits_rn, merge_lora, merge_scale
+from .optim import adamw_step
 
 __all__ = [
     "bf16_bits_to_f32", "f32_to_bf16_bits_rn", "fma_f32",
@@ -38,5 +39,5 @@ __all__ = [
     "dequantize_nf4_dq", "unpack_codes", "storage_bytes", "QuantizedNF4", "QuantizedNF4Single",
     "quantize_nf4_single", "dequantize_nf4_single",
     "lora_scale", "linear_fwd", "linear_bwd",
-    "f64_to_bf16_bits_rn", "merge_lora", "merge_scale",
+    "f64_to_bf16_bits_rn", "merge_lora", "merge_scale", "adamw_step",
 ]

@@ -175,3 +175,29 @@ def test_single_level_argument_errors_return_before_launch():
                                 ctypes.byref(n), None) == 0 and n.value > 0  # size query
     ok = (b._Adapter * 1)(b._Adapter(fake, fake, 16, 16.0, 1.0))
     assert lib.qlora_merge_lora(ctypes.byref(_single(absmax=fake + 1)), ok, 1, ctypes.c_void_p(fake), None) == 3
+
+
+def test_optimizer_argument_errors_return_before_launch():
+    lib = b.load_library()
+    fake = 1 << 20
+    P = ctypes.c_void_p(fake)
+    args = dict(lr=1e-3, b1=0.9, b2=0.999, eps=1e-8, wd=0.0, step=1)
+
+    def call(p=P, pb=None, g=P, m=P, v=P, n=1024, **kw):
+        a = {**args, **kw}
+        return lib.qlora_adamw_step(p, pb, g, m, v, n, a["lr"], a["b1"], a["b2"], a["eps"], a["wd"], a["step"], None)
+
+    assert call(n=0) == 0                         # nothing to do
+    assert call(n=-1) == 1
+    assert call(step=0) == 1
+    assert call(b1=1.0) == 1 and call(b2=-0.1) == 1 and call(eps=0.0) == 1 and call(lr=-1.0) == 1
+    assert call(wd=-0.5) == 1
+    assert call(g=None) == 1 and call(m=None) == 1 and call(p=None) == 1
+    assert call(p=ctypes.c_void_p(fake + 4)) == 3  # fp32 buffers need 16-byte alignment
+    assert call(g=ctypes.c_void_p(fake + 2)) == 3  # bf16 buffers need 8-byte alignment
+    assert call(pb=ctypes.c_void_p(fake + 2)) == 3
+    out = ctypes.c_void_p(123)
+    assert lib.qlora_paged_alloc(0, 0, ctypes.byref(out)) == 1 and out.value in (None, 0, 123)
+    assert lib.qlora_paged_alloc(1024, 0, None) == 1
+    assert lib.qlora_paged_free(None) == 0
+    assert lib.qlora_paged_prefetch(None, 16, 0, None) == 1
