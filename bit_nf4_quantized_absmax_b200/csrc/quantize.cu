@@ -368,9 +368,11 @@ cudaError_t launch_quantize(const void* W, int64_t numel, uint8_t* packed, int8_
   unsigned long long* totals = static_cast<unsigned long long*>(totals_scratch);
   cudaError_t e = launch_pass1(W, nblk, packed, absmax_scratch, totals, num_sms, stream);
   if (e != cudaSuccess) return e;
-  // chunks of at least 2048 constants, at most two CTAs per SM, and at most 2^24 constants each
-  int64_t g = (nblk + 2047) / 2048;
-  if (g > 2 * num_sms) g = 2 * num_sms;
+  // chunks of at least 512 constants and at most 8 CTAs per SM (the loop of a
+  // CTA is latency bound, so many short chunks beat few long ones), at most
+  // 2^24 constants each
+  int64_t g = (nblk + 511) / 512;
+  if (g > 8 * num_sms) g = 8 * num_sms;
   const int64_t min_g = (nblk + (int64_t(1) << 24) - 1) >> 24;
   if (g < min_g) g = min_g;
   if (g < 1) g = 1;
