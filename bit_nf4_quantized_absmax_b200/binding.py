@@ -22,7 +22,8 @@ STATUS_NAMES = {0: "QLORA_OK", 1: "QLORA_ERR_INVALID_ARG", 2: "QLORA_ERR_UNSUPPO
 
 EXPORTED = ("qlora_status_string", "qlora_nf4_codebook", "qlora_nf4_storage_bytes", "qlora_nf4_single_storage_bytes",
             "qlora_quantize_nf4", "qlora_quantize_nf4_dq", "qlora_quantize_nf4_dq_noalloc", "qlora_dequantize_nf4",
-            "qlora_dequantize_nf4_dq", "qlora_linear_fwd", "qlora_linear_bwd", "qlora_merge_lora",
+            "qlora_dequantize_nf4_dq", "qlora_linear_fwd", "qlora_linear_bwd", "qlora_linear_bwd_f32",
+            "qlora_merge_lora",
             "qlora_paged_alloc", "qlora_paged_free", "qlora_paged_prefetch", "qlora_adamw_step",
             "qlora_device_error")
 
@@ -71,6 +72,7 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
     lib.qlora_dequantize_nf4_dq.argtypes = [wp, vp, vp]
     lib.qlora_linear_fwd.argtypes = [wp, vp, i64, vp, vp, i32, f32, vp, vp, vp, szp, vp]
     lib.qlora_linear_bwd.argtypes = [wp, vp, i64, vp, vp, i32, f32, vp, vp, vp, vp, vp, vp, szp, vp]
+    lib.qlora_linear_bwd_f32.argtypes = [wp, vp, i64, vp, vp, i32, f32, vp, vp, vp, vp, vp, vp, szp, vp]
     lib.qlora_merge_lora.argtypes = [wp, ctypes.POINTER(_Adapter), i32, vp, vp]
     lib.qlora_device_error.argtypes = [ctypes.POINTER(ctypes.c_int32), vp]
     lib.qlora_paged_alloc.argtypes = [sz, i32, ctypes.POINTER(vp)]
@@ -250,24 +252,26 @@ def qlora_linear_fwd(q: NF4Weight | SingleNF4Weight, X: torch.Tensor, A: torch.T
 def qlora_linear_bwd(q: NF4Weight | SingleNF4Weight, X: torch.Tensor, A: torch.Tensor, B: torch.Tensor, alpha: float,
                      dY: torch.Tensor, T_saved: torch.Tensor | None = None, need_dX: bool = True,
                      dX: torch.Tensor | None = None, dA: torch.Tensor | None = None, dB: torch.Tensor | None = None,
-                     workspace: torch.Tensor | None = None, stream=None):
-    """Returns (dX or None, dA, dB)."""
+                     workspace: torch.Tensor | None = None, grads_fp32: bool = False, stream=None):
+    """Returns (dX or None, dA, dB); dA and dB are fp32 with grads_fp32 (qlora_linear_bwd_f32), else bf16."""
     lib = load_library()
     M, r = X.shape[0], A.shape[0]
     dev = X.device
+    gdt = torch.float32 if grads_fp32 else torch.bfloat16
     if need_dX and dX is None:
         dX = torch.empty(M, q.cols, dtype=torch.bfloat16, device=dev)
     if dA is None:
-        dA = torch.empty(r, q.cols, dtype=torch.bfloat16, device=dev)
+        dA = torch.empty(r, q.cols, dtype=gdt, device=dev)
     if dB is None:
-        dB = torch.empty(q.rows, r, dtype=torch.bfloat16, device=dev)
+        dB = torch.empty(q.rows, r, dtype=gdt, device=dev)
+    assert dA.dtype == gdt and dB.dtype == gdt
     qc = q.as_c()
     st = _stream(stream)
-    args = lambda p, n: lib.qlora_linear_bwd(ctypes.byref(qc), _ptr(X), M, _ptr(A), _ptr(B), r, float(alpha),
-                                             _ptr(dY), _ptr(T_saved), _ptr(dX if need_dX else None), _ptr(dA),
-                                             _ptr(dB), p, n, st)
+    fn = lib.qlora_linear_bwd_f32 if grads_fp32 else lib.qlora_linear_bwd
+    args = lambda p, n: fn(ctypes.byref(qc), _ptr(X), M, _ptr(A), _ptr(B), r, float(alpha), _ptr(dY), _ptr(T_saved),
+                           _ptr(dX if need_dX else None), _ptr(dA), _ptr(dB), p, n, st)
     ws, nbytes = _workspace(args, workspace, dev)
-    _check(args(_ptr(ws), ctypes.byref(nbytes)), "qlora_linear_bwd")
+    _check(args(_ptr(ws), ctypes.byref(nbytes)), "qlora_linear_bwd_f32" if grads_fp32 else "qlora_linear_bwd")
     return (dX if need_dX else None), dA, dB
 
 

@@ -133,6 +133,85 @@ struct Layout {
   size_t total() const { return off > 0 ? off : kAlign; }
 };
 
+// Backward shared by qlora_linear_bwd (bf16 dA, dB) and qlora_linear_bwd_f32 (fp32 dA, dB).
+qlora_status linear_bwd_impl(const qlora_nf4_weight* q, const void* X, int64_t M, const void* A, const void* B,
+                             int32_t r, float alpha, const void* dY, const float* T_saved, void* dX, void* dA,
+                             void* dB, bool f32, void* workspace, size_t* workspace_bytes, qlora_stream_t stream) {
+  qlora_status st = check_weight(q, true);
+  if (st != QLORA_OK) return st;
+  if ((st = check_linear(X, M, A, B, r, dA)) != QLORA_OK) return st;
+  if (!dA || !dB || (M > 0 && !dY)) return QLORA_ERR_INVALID_ARG;
+  if (!aligned(dB, 16) || (dY && !aligned(dY, 16)) || (dX && !aligned(dX, 16))) return QLORA_ERR_ALIGNMENT;
+  if (T_saved && !aligned(T_saved, 4)) return QLORA_ERR_ALIGNMENT;
+  const int64_t N = q->rows, K = q->cols;
+  if (N % 8) return QLORA_ERR_UNSUPPORTED;  // dY rows must be 16-byte multiples for the TMA tiles
+  const int rpad = (r + 63) / 64 * 64;
+  const float s = lora_scale(alpha, r);
+  DeviceInfo di{kRefSms};
+  const int splits_a = grad_splits(K, rpad, M, di.num_sms);
+  const int splits_b = grad_splits(N, rpad, M, di.num_sms);
+  Layout L;
+  const size_t mp = static_cast<size_t>(M) * rpad * 2;
+  const size_t off_wd = L.add(dX ? static_cast<size_t>(N) * K * 2 : 0);
+  const size_t off_thi = L.add(mp), off_tlo = L.add(mp);
+  const size_t off_su = L.add(mp), off_uhi = L.add(mp), off_ulo = L.add(mp);
+  const int splits_t = red_splits(M, rpad, K, di.num_sms);
+  const int splits_u = red_splits(M, rpad, N, di.num_sms);
+  size_t pmax = static_cast<size_t>(splits_a) * K * rpad;
+  const size_t pb = static_cast<size_t>(splits_b) * N * rpad;
+  const size_t pt = static_cast<size_t>(T_saved ? 0 : splits_t) * M * rpad;
+  const size_t pu = static_cast<size_t>(splits_u) * M * rpad;
+  if (pb > pmax) pmax = pb;
+  if (pt > pmax) pmax = pt;
+  if (pu > pmax) pmax = pu;
+  const size_t off_p = L.add(pmax * sizeof(float));
+  bool launch = false;
+  st = workspace_check(workspace, workspace_bytes, L.total(), &launch);
+  if (st != QLORA_OK || !launch) return st;
+  if ((st = device_info(&di)) != QLORA_OK) return st;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  if (M == 0) {
+    if (f32) {
+      cudaError_t e = cudaMemsetAsync(dA, 0, static_cast<size_t>(r) * K * sizeof(float), cs);
+      if (e == cudaSuccess) e = cudaMemsetAsync(dB, 0, static_cast<size_t>(N) * r * sizeof(float), cs);
+      return cuda_status(e);
+    }
+    cudaError_t e = launch_zero_bf16(dA, static_cast<int64_t>(r) * K, di.num_sms, cs);
+    if (e == cudaSuccess) e = launch_zero_bf16(dB, N * r, di.num_sms, cs);
+    return cuda_status(e);
+  }
+  char* ws = static_cast<char*>(workspace);
+  int32_t* err = device_error_word();
+  const float* cb = quant_tables().codebook;
+  void *Thi = ws + off_thi, *Tlo = ws + off_tlo, *sU = ws + off_su, *Uhi = ws + off_uhi, *Ulo = ws + off_ulo;
+  float* P = reinterpret_cast<float*>(ws + off_p);
+  cudaError_t e = cudaSuccess;
+  // T = X A^T as a two-term bf16 split (from the saved fp32 T or recomputed)
+  if (T_saved) {
+    e = launch_split_hilo(T_saved, M, r, rpad, Thi, Tlo, di.num_sms, cs);
+  } else {
+    e = launch_gemm_lora_t(X, A, M, K, r, rpad, P, splits_t, di.num_sms, err, cs);
+    if (e == cudaSuccess)
+      e = launch_lora_finish(P, splits_t, M, r, rpad, s, nullptr, nullptr, Thi, Tlo, di.num_sms, cs);
+  }
+  // U = dY B: s U for the dX slab, U as hi + lo for dA
+  if (e == cudaSuccess) e = launch_gemm_lora_u(dY, B, M, N, r, rpad, P, splits_u, di.num_sms, err, cs);
+  if (e == cudaSuccess) e = launch_lora_finish(P, splits_u, M, r, rpad, s, nullptr, sU, Uhi, Ulo, di.num_sms, cs);
+  if (dX) {
+    void* Wd = ws + off_wd;
+    if (e == cudaSuccess)
+      e = launch_dequantize(view(q), Wd, cb, di.num_sms, cs);
+    if (e == cudaSuccess) e = launch_gemm_dx(dY, Wd, sU, A, M, N, K, r, rpad, dX, di.num_sms, err, cs);
+  }
+  // dA^T [K, r] = X^T U, reduced over tokens, then dA = s * (.)^T
+  if (e == cudaSuccess) e = launch_gemm_lora_grad(X, K, Uhi, Ulo, M, rpad, P, splits_a, di.num_sms, err, cs);
+  if (e == cudaSuccess) e = launch_grad_reduce(P, splits_a, K, rpad, r, s, true, dA, f32, di.num_sms, cs);
+  // dB [N, r] = dY^T T
+  if (e == cudaSuccess) e = launch_gemm_lora_grad(dY, N, Thi, Tlo, M, rpad, P, splits_b, di.num_sms, err, cs);
+  if (e == cudaSuccess) e = launch_grad_reduce(P, splits_b, N, rpad, r, s, false, dB, f32, di.num_sms, cs);
+  return cuda_status(e);
+}
+
 }  // namespace
 
 
@@ -285,74 +364,16 @@ qlora_status qlora_linear_bwd(const qlora_nf4_weight* q, const void* X, int64_t 
                               const void* B, int32_t r, float alpha, const void* dY, const float* T_saved,
                               void* dX, void* dA, void* dB, void* workspace, size_t* workspace_bytes,
                               qlora_stream_t stream) {
-  qlora_status st = check_weight(q, true);
-  if (st != QLORA_OK) return st;
-  if ((st = check_linear(X, M, A, B, r, dA)) != QLORA_OK) return st;
-  if (!dA || !dB || (M > 0 && !dY)) return QLORA_ERR_INVALID_ARG;
-  if (!aligned(dB, 16) || (dY && !aligned(dY, 16)) || (dX && !aligned(dX, 16))) return QLORA_ERR_ALIGNMENT;
-  if (T_saved && !aligned(T_saved, 4)) return QLORA_ERR_ALIGNMENT;
-  const int64_t N = q->rows, K = q->cols;
-  if (N % 8) return QLORA_ERR_UNSUPPORTED;  // dY rows must be 16-byte multiples for the TMA tiles
-  const int rpad = (r + 63) / 64 * 64;
-  const float s = lora_scale(alpha, r);
-  DeviceInfo di{kRefSms};
-  const int splits_a = grad_splits(K, rpad, M, di.num_sms);
-  const int splits_b = grad_splits(N, rpad, M, di.num_sms);
-  Layout L;
-  const size_t mp = static_cast<size_t>(M) * rpad * 2;
-  const size_t off_wd = L.add(dX ? static_cast<size_t>(N) * K * 2 : 0);
-  const size_t off_thi = L.add(mp), off_tlo = L.add(mp);
-  const size_t off_su = L.add(mp), off_uhi = L.add(mp), off_ulo = L.add(mp);
-  const int splits_t = red_splits(M, rpad, K, di.num_sms);
-  const int splits_u = red_splits(M, rpad, N, di.num_sms);
-  size_t pmax = static_cast<size_t>(splits_a) * K * rpad;
-  const size_t pb = static_cast<size_t>(splits_b) * N * rpad;
-  const size_t pt = static_cast<size_t>(T_saved ? 0 : splits_t) * M * rpad;
-  const size_t pu = static_cast<size_t>(splits_u) * M * rpad;
-  if (pb > pmax) pmax = pb;
-  if (pt > pmax) pmax = pt;
-  if (pu > pmax) pmax = pu;
-  const size_t off_p = L.add(pmax * sizeof(float));
-  bool launch = false;
-  st = workspace_check(workspace, workspace_bytes, L.total(), &launch);
-  if (st != QLORA_OK || !launch) return st;
-  if ((st = device_info(&di)) != QLORA_OK) return st;
-  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
-  if (M == 0) {
-    cudaError_t e = launch_zero_bf16(dA, static_cast<int64_t>(r) * K, di.num_sms, cs);
-    if (e == cudaSuccess) e = launch_zero_bf16(dB, N * r, di.num_sms, cs);
-    return cuda_status(e);
-  }
-  char* ws = static_cast<char*>(workspace);
-  int32_t* err = device_error_word();
-  const float* cb = quant_tables().codebook;
-  void *Thi = ws + off_thi, *Tlo = ws + off_tlo, *sU = ws + off_su, *Uhi = ws + off_uhi, *Ulo = ws + off_ulo;
-  float* P = reinterpret_cast<float*>(ws + off_p);
-  cudaError_t e = cudaSuccess;
-  // T = X A^T as a two-term bf16 split (from the saved fp32 T or recomputed)
-  if (T_saved) {
-    e = launch_split_hilo(T_saved, M, r, rpad, Thi, Tlo, di.num_sms, cs);
-  } else {
-    e = launch_gemm_lora_t(X, A, M, K, r, rpad, P, splits_t, di.num_sms, err, cs);
-    if (e == cudaSuccess)
-      e = launch_lora_finish(P, splits_t, M, r, rpad, s, nullptr, nullptr, Thi, Tlo, di.num_sms, cs);
-  }
-  // U = dY B: s U for the dX slab, U as hi + lo for dA
-  if (e == cudaSuccess) e = launch_gemm_lora_u(dY, B, M, N, r, rpad, P, splits_u, di.num_sms, err, cs);
-  if (e == cudaSuccess) e = launch_lora_finish(P, splits_u, M, r, rpad, s, nullptr, sU, Uhi, Ulo, di.num_sms, cs);
-  if (dX) {
-    void* Wd = ws + off_wd;
-    if (e == cudaSuccess)
-      e = launch_dequantize(view(q), Wd, cb, di.num_sms, cs);
-    if (e == cudaSuccess) e = launch_gemm_dx(dY, Wd, sU, A, M, N, K, r, rpad, dX, di.num_sms, err, cs);
-  }
-  // dA^T [K, r] = X^T U, reduced over tokens, then dA = s * (.)^T
-  if (e == cudaSuccess) e = launch_gemm_lora_grad(X, K, Uhi, Ulo, M, rpad, P, splits_a, di.num_sms, err, cs);
-  if (e == cudaSuccess) e = launch_grad_reduce(P, splits_a, K, rpad, r, s, true, dA, di.num_sms, cs);
-  // dB [N, r] = dY^T T
-  if (e == cudaSuccess) e = launch_gemm_lora_grad(dY, N, Thi, Tlo, M, rpad, P, splits_b, di.num_sms, err, cs);
-  if (e == cudaSuccess) e = launch_grad_reduce(P, splits_b, N, rpad, r, s, false, dB, di.num_sms, cs);
-  return cuda_status(e);
+  return linear_bwd_impl(q, X, M, A, B, r, alpha, dY, T_saved, dX, dA, dB, false, workspace, workspace_bytes,
+                         stream);
+}
+
+qlora_status qlora_linear_bwd_f32(const qlora_nf4_weight* q, const void* X, int64_t M, const void* A,
+                                  const void* B, int32_t r, float alpha, const void* dY, const float* T_saved,
+                                  void* dX, float* dA, float* dB, void* workspace, size_t* workspace_bytes,
+                                  qlora_stream_t stream) {
+  return linear_bwd_impl(q, X, M, A, B, r, alpha, dY, T_saved, dX, dA, dB, true, workspace, workspace_bytes,
+                         stream);
 }
 
 qlora_status qlora_merge_lora(const qlora_nf4_weight* q, const qlora_lora_adapter* adapters,

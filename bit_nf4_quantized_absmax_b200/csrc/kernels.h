@@ -119,7 +119,7 @@ cudaError_t launch_split_hilo(const float* T, int64_t M, int r, int rpad, void* 
 cudaError_t launch_lora_finish(const float* P, int splits, int64_t M, int r, int rpad, float s, float* f32,
                                void* s_bf16, void* hi, void* lo, int num_sms, cudaStream_t stream);
 cudaError_t launch_grad_reduce(const float* P, int splits, int64_t R, int rpad, int r, float s, bool transpose,
-                               void* out, int num_sms, cudaStream_t stream);
+                               void* out, bool out_f32, int num_sms, cudaStream_t stream);
 cudaError_t launch_zero_bf16(void* p, int64_t n, int num_sms, cudaStream_t stream);
 
 }  // namespace qlora

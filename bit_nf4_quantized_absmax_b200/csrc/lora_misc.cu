@@ -4,8 +4,9 @@
 //   k_split_hilo  T fp32 [M, r] -> T_hi = bf16(T), T_lo = bf16(T - T_hi),
 //                 both [M, rpad] with zero padding, so that a bf16 tensor-core
 //                 contraction with (T_hi + T_lo) keeps ~16 significant bits.
-//   k_grad_reduce out = bf16(s * sum_p P[p]) over the split partials, in a
-//                 fixed order, optionally transposed ([R, rpad] -> [r, R]).
+//   k_grad_reduce out = s * sum_p P[p] over the split partials, in a fixed
+//                 order, optionally transposed ([R, rpad] -> [r, R]), written
+//                 as bf16 or (for a later cross-rank sum) as fp32.
 //   k_zero_bf16   zero fill (gradients of an empty batch).
 #include "common.cuh"
 #include "kernels.h"
@@ -67,9 +68,17 @@ __global__ void k_lora_finish(const float* __restrict__ P, int splits, int64_t M
 // One CTA per 32 rows x 64 columns; thread (ty, tx) sums the split partials of
 // rows ty and ty + 16, columns 4 tx .. 4 tx + 3 (float4 loads), with the loads
 // of four splits in flight at a time; the sum runs over p = 0, 1, ... in order.
+template <typename OutT>
+__device__ __forceinline__ OutT to_out(float v);
+template <>
+__device__ __forceinline__ __nv_bfloat16 to_out<__nv_bfloat16>(float v) { return __float2bfloat16_rn(v); }
+template <>
+__device__ __forceinline__ float to_out<float>(float v) { return v; }
+
+template <typename OutT>
 __global__ void __launch_bounds__(256)
 k_grad_reduce(const float* __restrict__ P, int splits, int64_t R, int rpad, int r, float s, int transpose,
-              __nv_bfloat16* __restrict__ out) {
+              OutT* __restrict__ out) {
   pdl_enter();
   __shared__ float tile[64][33];
   const int64_t row0 = static_cast<int64_t>(blockIdx.x) * 32;
@@ -105,7 +114,7 @@ k_grad_reduce(const float* __restrict__ P, int splits, int64_t R, int rpad, int 
         const float vv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
         for (int i = 0; i < 4; ++i)
-          if (col0 + c + i < r) out[row * r + col0 + c + i] = __float2bfloat16_rn(s * vv[i]);
+          if (col0 + c + i < r) out[row * r + col0 + c + i] = to_out<OutT>(s * vv[i]);
       }
     } else {
       tile[c][rr] = v.x;
@@ -121,7 +130,7 @@ k_grad_reduce(const float* __restrict__ P, int splits, int64_t R, int rpad, int 
   for (int cc = wy; cc < 64; cc += 8) {
     const int j = col0 + cc;
     const int64_t row = row0 + wx;
-    if (j < r && row < R) out[static_cast<int64_t>(j) * R + row] = __float2bfloat16_rn(s * tile[cc][wx]);
+    if (j < r && row < R) out[static_cast<int64_t>(j) * R + row] = to_out<OutT>(s * tile[cc][wx]);
   }
 }
 
@@ -155,10 +164,13 @@ cudaError_t launch_lora_finish(const float* P, int splits, int64_t M, int r, int
 }
 
 cudaError_t launch_grad_reduce(const float* P, int splits, int64_t R, int rpad, int r, float s, bool transpose,
-                               void* out, int num_sms, cudaStream_t stream) {
+                               void* out, bool out_f32, int num_sms, cudaStream_t stream) {
   const dim3 grid(static_cast<unsigned>((R + 31) / 32), static_cast<unsigned>(rpad / 64));
-  return launch_pdl(k_grad_reduce, grid, dim3(256), 0, stream, P, splits, R, rpad, r, s, transpose ? 1 : 0,
-                    static_cast<__nv_bfloat16*>(out));
+  if (out_f32)
+    return launch_pdl(k_grad_reduce<float>, grid, dim3(256), 0, stream, P, splits, R, rpad, r, s, transpose ? 1 : 0,
+                      static_cast<float*>(out));
+  return launch_pdl(k_grad_reduce<__nv_bfloat16>, grid, dim3(256), 0, stream, P, splits, R, rpad, r, s,
+                    transpose ? 1 : 0, static_cast<__nv_bfloat16*>(out));
 }
 
 cudaError_t launch_zero_bf16(void* p, int64_t n, int num_sms, cudaStream_t stream) {

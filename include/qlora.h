@@ -239,6 +239,19 @@ qlora_status qlora_linear_bwd(const qlora_nf4_weight* q, const void* X, int64_t 
                               void* workspace, size_t* workspace_bytes,
                               qlora_stream_t stream);
 
+/* qlora_linear_bwd_f32 -- qlora_linear_bwd with dA [r, K] and dB [N, r] written
+ * in fp32 (16-byte aligned) instead of bf16, i.e. before their rounding to bf16.
+ * For data-parallel training: the gradients of the ranks' token shards are
+ * summed in fp32 and rounded once, so the sum keeps the accuracy of a
+ * single-GPU backward. dX (when not NULL) is bf16 as in qlora_linear_bwd.
+ * Errors: as qlora_linear_bwd. */
+qlora_status qlora_linear_bwd_f32(const qlora_nf4_weight* q, const void* X, int64_t M,
+                                  const void* A, const void* B, int32_t r, float alpha,
+                                  const void* dY, const float* T_saved,
+                                  void* dX, float* dA, float* dB,
+                                  void* workspace, size_t* workspace_bytes,
+                                  qlora_stream_t stream);
+
 /* One LoRA adapter of a merge: A [r, cols] and B [rows, r] (device bf16,
  * 16-byte aligned, row-major), 8 <= r <= 256 with r % 8 == 0, scale
  * s = (float)alpha / (float)r, composition weight w. */
