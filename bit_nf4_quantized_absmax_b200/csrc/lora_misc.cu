@@ -65,9 +65,6 @@ __global__ void k_lora_finish(const float* __restrict__ P, int splits, int64_t M
 // columns kept). A CTA owns a 32-row x 64-column tile: coalesced float2 reads of
 // every split (fixed order), then either direct row-major writes ([R, r]) or a
 // transpose through shared memory so that the [r, R] writes are coalesced too.
-// One CTA per 32 rows x 64 columns; thread (ty, tx) sums the split partials of
-// rows ty and ty + 16, columns 4 tx .. 4 tx + 3 (float4 loads), with the loads
-// of four splits in flight at a time; the sum runs over p = 0, 1, ... in order.
 template <typename OutT>
 __device__ __forceinline__ OutT to_out(float v);
 template <>
@@ -75,62 +72,59 @@ __device__ __forceinline__ __nv_bfloat16 to_out<__nv_bfloat16>(float v) { return
 template <>
 __device__ __forceinline__ float to_out<float>(float v) { return v; }
 
+// One CTA per 16 rows x 64 columns; thread (ty, tx) sums the split partials of
+// row ty, columns 4 tx .. 4 tx + 3 (float4 loads), with the loads of four
+// splits in flight at a time; the sum runs over p = 0, 1, ... in order.
 template <typename OutT>
 __global__ void __launch_bounds__(256)
 k_grad_reduce(const float* __restrict__ P, int splits, int64_t R, int rpad, int r, float s, int transpose,
               OutT* __restrict__ out) {
   pdl_enter();
-  __shared__ float tile[64][33];
-  const int64_t row0 = static_cast<int64_t>(blockIdx.x) * 32;
+  __shared__ float tile[64][17];
+  const int64_t row0 = static_cast<int64_t>(blockIdx.x) * 16;
   const int col0 = blockIdx.y * 64;
   const int tx = threadIdx.x & 15;   // column quad within the tile
-  const int ty = threadIdx.x >> 4;   // 16 row lanes
+  const int ty = threadIdx.x >> 4;   // row within the tile
   const int64_t pstride = R * rpad / 4;  // float4 elements per split
+  const int64_t row = row0 + ty;
+  float4 v = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+  if (row < R) {
+    const float4* src = reinterpret_cast<const float4*>(P + row * rpad + col0) + tx;
+    int p = 0;
+    for (; p + 4 <= splits; p += 4) {
+      float4 q[4];
 #pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    const int rr = ty + 16 * h;
-    const int64_t row = row0 + rr;
-    float4 v = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-    if (row < R) {
-      const float4* src = reinterpret_cast<const float4*>(P + row * rpad + col0) + tx;
-      int p = 0;
-      for (; p + 4 <= splits; p += 4) {
-        float4 q[4];
+      for (int i = 0; i < 4; ++i) q[i] = __ldcs(src + (p + i) * pstride);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) q[i] = __ldcs(src + (p + i) * pstride);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          v.x += q[i].x; v.y += q[i].y; v.z += q[i].z; v.w += q[i].w;
-        }
-      }
-      for (; p < splits; ++p) {
-        const float4 q = __ldcs(src + p * pstride);
-        v.x += q.x; v.y += q.y; v.z += q.z; v.w += q.w;
+      for (int i = 0; i < 4; ++i) {
+        v.x += q[i].x; v.y += q[i].y; v.z += q[i].z; v.w += q[i].w;
       }
     }
-    const int c = 4 * tx;
-    if (!transpose) {
-      if (row < R) {
-        const float vv[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-          if (col0 + c + i < r) out[row * r + col0 + c + i] = to_out<OutT>(s * vv[i]);
-      }
-    } else {
-      tile[c][rr] = v.x;
-      tile[c + 1][rr] = v.y;
-      tile[c + 2][rr] = v.z;
-      tile[c + 3][rr] = v.w;
+    for (; p < splits; ++p) {
+      const float4 q = __ldcs(src + p * pstride);
+      v.x += q.x; v.y += q.y; v.z += q.z; v.w += q.w;
     }
   }
-  if (!transpose) return;
+  const int c = 4 * tx;
+  if (!transpose) {
+    if (row < R) {
+      const float vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        if (col0 + c + i < r) out[row * r + col0 + c + i] = to_out<OutT>(s * vv[i]);
+    }
+    return;
+  }
+  tile[c][ty] = v.x;
+  tile[c + 1][ty] = v.y;
+  tile[c + 2][ty] = v.z;
+  tile[c + 3][ty] = v.w;
   __syncthreads();
-  // out[j][row]: 32 consecutive rows per column j, one warp per column
-  const int wx = threadIdx.x & 31, wy = threadIdx.x >> 5;
-  for (int cc = wy; cc < 64; cc += 8) {
-    const int j = col0 + cc;
-    const int64_t row = row0 + wx;
-    if (j < r && row < R) out[static_cast<int64_t>(j) * R + row] = to_out<OutT>(s * tile[cc][wx]);
+  // out[j][row]: 16 consecutive rows per column j
+  for (int idx = threadIdx.x; idx < 64 * 16; idx += blockDim.x) {
+    const int j = col0 + (idx >> 4);
+    const int64_t rr = row0 + (idx & 15);
+    if (j < r && rr < R) out[static_cast<int64_t>(j) * R + rr] = to_out<OutT>(s * tile[idx >> 4][idx & 15]);
   }
 }
 
@@ -165,7 +159,7 @@ cudaError_t launch_lora_finish(const float* P, int splits, int64_t M, int r, int
 
 cudaError_t launch_grad_reduce(const float* P, int splits, int64_t R, int rpad, int r, float s, bool transpose,
                                void* out, bool out_f32, int num_sms, cudaStream_t stream) {
-  const dim3 grid(static_cast<unsigned>((R + 31) / 32), static_cast<unsigned>(rpad / 64));
+  const dim3 grid(static_cast<unsigned>((R + 15) / 16), static_cast<unsigned>(rpad / 64));
   if (out_f32)
     return launch_pdl(k_grad_reduce<float>, grid, dim3(256), 0, stream, P, splits, R, rpad, r, s, transpose ? 1 : 0,
                       static_cast<float*>(out));
