@@ -186,17 +186,18 @@ qlora_status linear_bwd_impl(const qlora_nf4_weight* q, const void* X, int64_t M
   void *Thi = ws + off_thi, *Tlo = ws + off_tlo, *sU = ws + off_su, *Uhi = ws + off_uhi, *Ulo = ws + off_ulo;
   float* P = reinterpret_cast<float*>(ws + off_p);
   cudaError_t e = cudaSuccess;
-  // T = X A^T as a two-term bf16 split (from the saved fp32 T or recomputed)
-  if (T_saved) {
-    e = launch_split_hilo(T_saved, M, r, rpad, Thi, Tlo, di.num_sms, cs);
-  } else {
+  // T = X A^T as a two-term bf16 split: recomputed here, or split from the saved
+  // fp32 T by the launch that finishes U below
+  if (!T_saved) {
     e = launch_gemm_lora_t(X, A, M, K, r, rpad, P, splits_t, di.num_sms, err, cs);
     if (e == cudaSuccess)
       e = launch_lora_finish(P, splits_t, M, r, rpad, s, nullptr, nullptr, Thi, Tlo, di.num_sms, cs);
   }
   // U = dY B: s U for the dX slab, U as hi + lo for dA
   if (e == cudaSuccess) e = launch_gemm_lora_u(dY, B, M, N, r, rpad, P, splits_u, di.num_sms, err, cs);
-  if (e == cudaSuccess) e = launch_lora_finish(P, splits_u, M, r, rpad, s, nullptr, sU, Uhi, Ulo, di.num_sms, cs);
+  if (e == cudaSuccess)
+    e = launch_lora_finish(P, splits_u, M, r, rpad, s, nullptr, sU, Uhi, Ulo, di.num_sms, cs, T_saved,
+                           T_saved ? Thi : nullptr, T_saved ? Tlo : nullptr);
   if (dX) {
     void* Wd = ws + off_wd;
     if (e == cudaSuccess)

@@ -114,10 +114,10 @@ cudaError_t launch_gemm_lora_grad(const void* Q, int64_t R, const void* hi, cons
                                   float* P, int splits, int num_sms, int32_t* err, cudaStream_t stream);
 
 // ---- lora_misc.cu ----
-cudaError_t launch_split_hilo(const float* T, int64_t M, int r, int rpad, void* hi, void* lo, int num_sms,
-                              cudaStream_t stream);
+// Optionally also splits the fp32 [M, r] matrix t_src into bf16 t_hi + t_lo [M, rpad] in the same launch.
 cudaError_t launch_lora_finish(const float* P, int splits, int64_t M, int r, int rpad, float s, float* f32,
-                               void* s_bf16, void* hi, void* lo, int num_sms, cudaStream_t stream);
+                               void* s_bf16, void* hi, void* lo, int num_sms, cudaStream_t stream,
+                               const float* t_src = nullptr, void* t_hi = nullptr, void* t_lo = nullptr);
 cudaError_t launch_grad_reduce(const float* P, int splits, int64_t R, int rpad, int r, float s, bool transpose,
                                void* out, bool out_f32, int num_sms, cudaStream_t stream);
 cudaError_t launch_zero_bf16(void* p, int64_t n, int num_sms, cudaStream_t stream);

@@ -1,9 +1,11 @@
 // Small element-wise kernels around the LoRA gradient contractions
 // ("QLoRA vs ChatGPT", capability 5: gradients only for the LoRA parameters).
 //
-//   k_split_hilo  T fp32 [M, r] -> T_hi = bf16(T), T_lo = bf16(T - T_hi),
-//                 both [M, rpad] with zero padding, so that a bf16 tensor-core
-//                 contraction with (T_hi + T_lo) keeps ~16 significant bits.
+//   k_lora_finish sums the split partials of T = X A^T or U = dY B in a fixed
+//                 order and writes fp32, s * (.) in bf16, and the bf16 split
+//                 hi = bf16(v), lo = bf16(v - hi) ([M, rpad], zero padding) that
+//                 lets a bf16 tensor-core contraction keep ~16 significant bits;
+//                 the same launch can split a saved fp32 T the same way.
 //   k_grad_reduce out = s * sum_p P[p] over the split partials, in a fixed
 //                 order, optionally transposed ([R, rpad] -> [r, R]), written
 //                 as bf16 or (for a later cross-rank sum) as fp32.
@@ -14,27 +16,17 @@
 namespace qlora {
 namespace {
 
-__global__ void k_split_hilo(const float* __restrict__ T, int64_t M, int r, int rpad, __nv_bfloat16* __restrict__ hi,
-                             __nv_bfloat16* __restrict__ lo) {
-  pdl_enter();
-  const int64_t n = M * rpad;
-  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t m = i / rpad;
-    const int j = static_cast<int>(i % rpad);
-    const float v = j < r ? T[m * r + j] : 0.0f;
-    const __nv_bfloat16 h = __float2bfloat16_rn(v);
-    hi[i] = h;
-    lo[i] = __float2bfloat16_rn(v - __bfloat162float(h));
-  }
-}
 
 // Sum the split partials P[p][m][j] (fixed order) and emit the LoRA operands:
 // f32[m][j] (j < r, optional), s_bf16 = bf16(s v), hi = bf16(v), lo = bf16(v - hi)
 // for j < rpad (zero columns stay zero). Two adjacent columns per thread.
+// t_src (optional): a second job in the same launch, splitting the fp32 [M, r]
+// matrix t_src into bf16 hi + lo [M, rpad] (zero columns past r).
 __global__ void k_lora_finish(const float* __restrict__ P, int splits, int64_t M, int r, int rpad, float s,
                               float* __restrict__ f32, __nv_bfloat16* __restrict__ s_bf16,
-                              __nv_bfloat16* __restrict__ hi, __nv_bfloat16* __restrict__ lo) {
+                              __nv_bfloat16* __restrict__ hi, __nv_bfloat16* __restrict__ lo,
+                              const float* __restrict__ t_src, __nv_bfloat16* __restrict__ t_hi,
+                              __nv_bfloat16* __restrict__ t_lo) {
   pdl_enter();
   const int64_t n2 = M * rpad / 2;
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n2;
@@ -57,6 +49,13 @@ __global__ void k_lora_finish(const float* __restrict__ P, int splits, int64_t M
       const uint32_t h = pack_bf16x2(v.x, v.y);
       reinterpret_cast<uint32_t*>(hi)[i] = h;
       reinterpret_cast<uint32_t*>(lo)[i] = pack_bf16x2(v.x - bf16lo_to_f32(h), v.y - bf16hi_to_f32(h));
+    }
+    if (t_src) {
+      const float t0 = j < r ? t_src[m * r + j] : 0.0f;
+      const float t1 = j + 1 < r ? t_src[m * r + j + 1] : 0.0f;
+      const uint32_t h = pack_bf16x2(t0, t1);
+      reinterpret_cast<uint32_t*>(t_hi)[i] = h;
+      reinterpret_cast<uint32_t*>(t_lo)[i] = pack_bf16x2(t0 - bf16lo_to_f32(h), t1 - bf16hi_to_f32(h));
     }
   }
 }
@@ -144,17 +143,14 @@ int grid_for(int64_t n, int num_sms) {
 
 }  // namespace
 
-cudaError_t launch_split_hilo(const float* T, int64_t M, int r, int rpad, void* hi, void* lo, int num_sms,
-                              cudaStream_t stream) {
-  return launch_pdl(k_split_hilo, dim3(grid_for(M * rpad, num_sms)), dim3(256), 0, stream, T, M, r, rpad,
-                    static_cast<__nv_bfloat16*>(hi), static_cast<__nv_bfloat16*>(lo));
-}
 
 cudaError_t launch_lora_finish(const float* P, int splits, int64_t M, int r, int rpad, float s, float* f32,
-                               void* s_bf16, void* hi, void* lo, int num_sms, cudaStream_t stream) {
+                               void* s_bf16, void* hi, void* lo, int num_sms, cudaStream_t stream,
+                               const float* t_src, void* t_hi, void* t_lo) {
   return launch_pdl(k_lora_finish, dim3(grid_for(M * rpad / 2, num_sms)), dim3(256), 0, stream, P, splits, M, r,
                     rpad, s, f32, static_cast<__nv_bfloat16*>(s_bf16), static_cast<__nv_bfloat16*>(hi),
-                    static_cast<__nv_bfloat16*>(lo));
+                    static_cast<__nv_bfloat16*>(lo), t_src, static_cast<__nv_bfloat16*>(t_hi),
+                    static_cast<__nv_bfloat16*>(t_lo));
 }
 
 cudaError_t launch_grad_reduce(const float* P, int splits, int64_t R, int rpad, int r, float s, bool transpose,
