@@ -56,7 +56,7 @@ def source_fingerprint():
 
 
 # kernels each C-ABI call launches on these shapes (see the launchers in csrc/)
-LAUNCHES = {"quantize": 3, "dequantize": 1, "decode_fwd": 2, "train_fwd": 4, "train_bwd": 8}
+LAUNCHES = {"quantize": 3, "dequantize": 1, "decode_fwd": 2, "train_fwd": 3, "train_bwd": 7}
 
 
 def train_flops(N, K, M=M_TRAIN, r=R):

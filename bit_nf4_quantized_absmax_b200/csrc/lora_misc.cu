@@ -12,6 +12,7 @@
 //   k_zero_bf16   zero fill (gradients of an empty batch).
 #include "common.cuh"
 #include "kernels.h"
+#include "lora_finish.cuh"
 
 namespace qlora {
 namespace {
@@ -20,44 +21,10 @@ namespace {
 // Sum the split partials P[p][m][j] (fixed order) and emit the LoRA operands:
 // f32[m][j] (j < r, optional), s_bf16 = bf16(s v), hi = bf16(v), lo = bf16(v - hi)
 // for j < rpad (zero columns stay zero). Two adjacent columns per thread.
-// t_src (optional): a second job in the same launch, splitting the fp32 [M, r]
-// matrix t_src into bf16 hi + lo [M, rpad] (zero columns past r).
-__global__ void k_lora_finish(const float* __restrict__ P, int splits, int64_t M, int r, int rpad, float s,
-                              float* __restrict__ f32, __nv_bfloat16* __restrict__ s_bf16,
-                              __nv_bfloat16* __restrict__ hi, __nv_bfloat16* __restrict__ lo,
-                              const float* __restrict__ t_src, __nv_bfloat16* __restrict__ t_hi,
-                              __nv_bfloat16* __restrict__ t_lo) {
+__global__ void k_lora_finish(const __grid_constant__ LoraFinishJob job) {
   pdl_enter();
-  const int64_t n2 = M * rpad / 2;
-  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n2;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t e = 2 * i;
-    const int64_t m = e / rpad;
-    const int j = static_cast<int>(e % rpad);
-    float2 v = make_float2(0.0f, 0.0f);
-    for (int p = 0; p < splits; ++p) {
-      const float2 pv = reinterpret_cast<const float2*>(P + (static_cast<int64_t>(p) * M) * rpad)[i];
-      v.x += pv.x;
-      v.y += pv.y;
-    }
-    if (f32) {
-      if (j < r) f32[m * r + j] = v.x;
-      if (j + 1 < r) f32[m * r + j + 1] = v.y;
-    }
-    if (s_bf16) reinterpret_cast<uint32_t*>(s_bf16)[i] = pack_bf16x2(s * v.x, s * v.y);
-    if (hi) {
-      const uint32_t h = pack_bf16x2(v.x, v.y);
-      reinterpret_cast<uint32_t*>(hi)[i] = h;
-      reinterpret_cast<uint32_t*>(lo)[i] = pack_bf16x2(v.x - bf16lo_to_f32(h), v.y - bf16hi_to_f32(h));
-    }
-    if (t_src) {
-      const float t0 = j < r ? t_src[m * r + j] : 0.0f;
-      const float t1 = j + 1 < r ? t_src[m * r + j + 1] : 0.0f;
-      const uint32_t h = pack_bf16x2(t0, t1);
-      reinterpret_cast<uint32_t*>(t_hi)[i] = h;
-      reinterpret_cast<uint32_t*>(t_lo)[i] = pack_bf16x2(t0 - bf16lo_to_f32(h), t1 - bf16hi_to_f32(h));
-    }
-  }
+  lora_finish_range(job, static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x,
+                    static_cast<int64_t>(gridDim.x) * blockDim.x);
 }
 
 // out = bf16(s * sum_p P[p]) for a [R, rpad] partial stack (rows R, the first r
@@ -147,10 +114,21 @@ int grid_for(int64_t n, int num_sms) {
 cudaError_t launch_lora_finish(const float* P, int splits, int64_t M, int r, int rpad, float s, float* f32,
                                void* s_bf16, void* hi, void* lo, int num_sms, cudaStream_t stream,
                                const float* t_src, void* t_hi, void* t_lo) {
-  return launch_pdl(k_lora_finish, dim3(grid_for(M * rpad / 2, num_sms)), dim3(256), 0, stream, P, splits, M, r,
-                    rpad, s, f32, static_cast<__nv_bfloat16*>(s_bf16), static_cast<__nv_bfloat16*>(hi),
-                    static_cast<__nv_bfloat16*>(lo), t_src, static_cast<__nv_bfloat16*>(t_hi),
-                    static_cast<__nv_bfloat16*>(t_lo));
+  LoraFinishJob job;
+  job.P = P;
+  job.splits = splits;
+  job.M = M;
+  job.r = r;
+  job.rpad = rpad;
+  job.s = s;
+  job.f32 = f32;
+  job.s_bf16 = s_bf16;
+  job.hi = hi;
+  job.lo = lo;
+  job.t_src = t_src;
+  job.t_hi = t_hi;
+  job.t_lo = t_lo;
+  return launch_pdl(k_lora_finish, dim3(grid_for(M * rpad / 2, num_sms)), dim3(256), 0, stream, job);
 }
 
 cudaError_t launch_grad_reduce(const float* P, int splits, int64_t R, int rpad, int r, float s, bool transpose,
