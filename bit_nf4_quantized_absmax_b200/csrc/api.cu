@@ -186,36 +186,22 @@ qlora_status linear_bwd_impl(const qlora_nf4_weight* q, const void* X, int64_t M
   void *Thi = ws + off_thi, *Tlo = ws + off_tlo, *sU = ws + off_su, *Uhi = ws + off_uhi, *Ulo = ws + off_ulo;
   float* P = reinterpret_cast<float*>(ws + off_p);
   cudaError_t e = cudaSuccess;
-  // T = X A^T as a two-term bf16 split: recomputed here, or split from the saved
-  // fp32 T by the launch that finishes U below
-  if (!T_saved) {
+  // T = X A^T as a two-term bf16 split (from the saved fp32 T or recomputed)
+  if (T_saved) {
+    e = launch_split_hilo(T_saved, M, r, rpad, Thi, Tlo, di.num_sms, cs);
+  } else {
     e = launch_gemm_lora_t(X, A, M, K, r, rpad, P, splits_t, di.num_sms, err, cs);
     if (e == cudaSuccess)
       e = launch_lora_finish(P, splits_t, M, r, rpad, s, nullptr, nullptr, Thi, Tlo, di.num_sms, cs);
   }
-  // U = dY B: s U for the dX slab, U as hi + lo for dA; the launch that finishes
-  // U (the dequant of W' when dX is wanted) also splits a saved T into hi + lo
+  // U = dY B: s U for the dX slab, U as hi + lo for dA
   if (e == cudaSuccess) e = launch_gemm_lora_u(dY, B, M, N, r, rpad, P, splits_u, di.num_sms, err, cs);
-  LoraFinishJob fin;
-  fin.P = P;
-  fin.splits = splits_u;
-  fin.M = M;
-  fin.r = r;
-  fin.rpad = rpad;
-  fin.s = s;
-  fin.s_bf16 = sU;
-  fin.hi = Uhi;
-  fin.lo = Ulo;
-  fin.t_src = T_saved;
-  fin.t_hi = T_saved ? Thi : nullptr;
-  fin.t_lo = T_saved ? Tlo : nullptr;
+  if (e == cudaSuccess) e = launch_lora_finish(P, splits_u, M, r, rpad, s, nullptr, sU, Uhi, Ulo, di.num_sms, cs);
   if (dX) {
     void* Wd = ws + off_wd;
-    if (e == cudaSuccess) e = launch_dequantize(view(q), Wd, cb, di.num_sms, cs, &fin);
+    if (e == cudaSuccess)
+      e = launch_dequantize(view(q), Wd, cb, di.num_sms, cs);
     if (e == cudaSuccess) e = launch_gemm_dx(dY, Wd, sU, A, M, N, K, r, rpad, dX, di.num_sms, err, cs);
-  } else if (e == cudaSuccess) {
-    e = launch_lora_finish(P, splits_u, M, r, rpad, s, nullptr, sU, Uhi, Ulo, di.num_sms, cs, T_saved,
-                           fin.t_hi, fin.t_lo);
   }
   // dA^T [K, r] = X^T U, reduced over tokens, then dA = s * (.)^T
   if (e == cudaSuccess) e = launch_gemm_lora_grad(X, K, Uhi, Ulo, M, rpad, P, splits_a, di.num_sms, err, cs);
@@ -366,19 +352,10 @@ qlora_status qlora_linear_fwd(const qlora_nf4_weight* q, const void* X, int64_t 
   void* sT = ws + off_sT;
   float* P = reinterpret_cast<float*>(ws + off_part);
   const int splits_t = red_splits(M, rpad, K, kRefSms);
-  // T = X A^T split over K, then one launch that dequantizes W' and finishes T
-  // (T_save in fp32, s T in bf16 for the LoRA slab), then the main GEMM
-  cudaError_t e = launch_gemm_lora_t(X, A, M, K, r, rpad, P, splits_t, di.num_sms, err, cs);
-  LoraFinishJob fin;
-  fin.P = P;
-  fin.splits = splits_t;
-  fin.M = M;
-  fin.r = r;
-  fin.rpad = rpad;
-  fin.s = s;
-  fin.f32 = T_save;
-  fin.s_bf16 = sT;
-  if (e == cudaSuccess) e = launch_dequantize(view(q), Wd, cb, di.num_sms, cs, &fin);
+  cudaError_t e = launch_dequantize(view(q), Wd, cb, di.num_sms, cs);
+  if (e == cudaSuccess) e = launch_gemm_lora_t(X, A, M, K, r, rpad, P, splits_t, di.num_sms, err, cs);
+  if (e == cudaSuccess)
+    e = launch_lora_finish(P, splits_t, M, r, rpad, s, T_save, sT, nullptr, nullptr, di.num_sms, cs);
   if (e == cudaSuccess) e = launch_gemm_fwd(X, Wd, sT, B, M, N, K, r, rpad, Y, di.num_sms, err, cs);
   return cuda_status(e);
 }

@@ -4,12 +4,9 @@
 // One thread decodes 32 weights (half a 64-weight block): it forms the block
 // constant (m' = fmaf(q_b, dq_scale_g, mean) for double-quantized storage, the
 // stored fp32 m_b for single-level storage), builds the block's 16-entry bf16
-// table and decodes its 16 packed bytes with byte permutes. The launch can also
-// carry a LoRA finish job (summing the split partials of T or U), which saves
-// the linear layer a launch of its own.
+// table and decodes its 16 packed bytes with byte permutes.
 #include "common.cuh"
 #include "kernels.h"
-#include "lora_finish.cuh"
 #include "nf4_lut.cuh"
 
 namespace qlora {
@@ -44,8 +41,7 @@ template <bool V8, bool SINGLE>
 __global__ void __launch_bounds__(256)
 k_dequant(const uint4* __restrict__ packed, const int8_t* __restrict__ absmax_q,
           const float* __restrict__ dq_scale, const float* __restrict__ mean, const float* __restrict__ absmax,
-          uint4* __restrict__ out, int64_t n_units, const __grid_constant__ Nf4Codebook cb,
-          const __grid_constant__ LoraFinishJob fin) {
+          uint4* __restrict__ out, int64_t n_units, const __grid_constant__ Nf4Codebook cb) {
   pdl_enter();
   const float mu = SINGLE ? 0.0f : *mean;
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
@@ -75,14 +71,12 @@ k_dequant(const uint4* __restrict__ packed, const int8_t* __restrict__ absmax_q,
         dequant_unit<V8>(nib[i], u, SINGLE ? sc[i] : __fmaf_rn(static_cast<float>(qv[i]), sc[i], mu), out, cb);
     }
   }
-  if (fin.P)  // the finish job carried by this launch (its partials come from an earlier kernel)
-    lora_finish_range(fin, static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x, stride);
 }
 
 }  // namespace
 
 cudaError_t launch_dequantize(const Nf4View& w, void* out, const float codebook[16], int num_sms,
-                              cudaStream_t stream, const LoraFinishJob* fin) {
+                              cudaStream_t stream) {
   Nf4Codebook cb;
   for (int i = 0; i < 16; ++i) cb.c[i] = codebook[i];
   const int64_t n_units = w.N * w.K / 32;
@@ -94,8 +88,7 @@ cudaError_t launch_dequantize(const Nf4View& w, void* out, const float codebook[
   auto kern = single ? (v8 ? k_dequant<true, true> : k_dequant<false, true>)
                      : (v8 ? k_dequant<true, false> : k_dequant<false, false>);
   return launch_pdl(kern, dim3(grid), dim3(256), 0, stream, reinterpret_cast<const uint4*>(w.packed), w.absmax_q,
-                    w.dq_scale, w.mean, w.absmax, reinterpret_cast<uint4*>(out), n_units, cb,
-                    fin ? *fin : LoraFinishJob{});
+                    w.dq_scale, w.mean, w.absmax, reinterpret_cast<uint4*>(out), n_units, cb);
 }
 
 }  // namespace qlora

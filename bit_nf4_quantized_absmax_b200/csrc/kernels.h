@@ -62,28 +62,8 @@ struct Nf4View {
   const float* absmax;
 };
 
-// Finishing the split partials P[splits][M][rpad] of T = X A^T or U = dY B:
-// sum in a fixed order, then any of f32 [M, r], s * (.) bf16 [M, rpad] and the
-// bf16 split hi + lo [M, rpad]; optionally also split a saved fp32 t_src [M, r]
-// into t_hi + t_lo. Run by its own launch or inside the dequant launch.
-struct LoraFinishJob {
-  const float* P = nullptr;  // null: no job
-  int splits = 0;
-  int64_t M = 0;
-  int r = 0, rpad = 0;
-  float s = 0.0f;
-  float* f32 = nullptr;
-  void* s_bf16 = nullptr;
-  void* hi = nullptr;
-  void* lo = nullptr;
-  const float* t_src = nullptr;
-  void* t_hi = nullptr;
-  void* t_lo = nullptr;
-};
-
-// fin (optional): a finish job run by the same launch after the dequantization.
 cudaError_t launch_dequantize(const Nf4View& w, void* out, const float codebook[16], int num_sms,
-                              cudaStream_t stream, const LoraFinishJob* fin = nullptr);
+                              cudaStream_t stream);
 
 // ---- decode.cu: M <= 16 forward ----
 // Work split of the decode kernel: (128-row group, 256-wide K superblock)
@@ -134,10 +114,10 @@ cudaError_t launch_gemm_lora_grad(const void* Q, int64_t R, const void* hi, cons
                                   float* P, int splits, int num_sms, int32_t* err, cudaStream_t stream);
 
 // ---- lora_misc.cu ----
-// Optionally also splits the fp32 [M, r] matrix t_src into bf16 t_hi + t_lo [M, rpad] in the same launch.
+cudaError_t launch_split_hilo(const float* T, int64_t M, int r, int rpad, void* hi, void* lo, int num_sms,
+                              cudaStream_t stream);
 cudaError_t launch_lora_finish(const float* P, int splits, int64_t M, int r, int rpad, float s, float* f32,
-                               void* s_bf16, void* hi, void* lo, int num_sms, cudaStream_t stream,
-                               const float* t_src = nullptr, void* t_hi = nullptr, void* t_lo = nullptr);
+                               void* s_bf16, void* hi, void* lo, int num_sms, cudaStream_t stream);
 cudaError_t launch_grad_reduce(const float* P, int splits, int64_t R, int rpad, int r, float s, bool transpose,
                                void* out, bool out_f32, int num_sms, cudaStream_t stream);
 cudaError_t launch_zero_bf16(void* p, int64_t n, int num_sms, cudaStream_t stream);

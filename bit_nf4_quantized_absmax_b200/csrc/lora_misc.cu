@@ -1,36 +1,73 @@
 // Small element-wise kernels around the LoRA gradient contractions
 // ("QLoRA vs ChatGPT", capability 5: gradients only for the LoRA parameters).
 //
-//   k_lora_finish sums the split partials of T = X A^T or U = dY B in a fixed
-//                 order and writes fp32, s * (.) in bf16, and the bf16 split
-//                 hi = bf16(v), lo = bf16(v - hi) ([M, rpad], zero padding) that
-//                 lets a bf16 tensor-core contraction keep ~16 significant bits;
-//                 the same launch can split a saved fp32 T the same way.
+//   k_split_hilo  T fp32 [M, r] -> T_hi = bf16(T), T_lo = bf16(T - T_hi),
+//                 both [M, rpad] with zero padding, so that a bf16 tensor-core
+//                 contraction with (T_hi + T_lo) keeps ~16 significant bits.
 //   k_grad_reduce out = s * sum_p P[p] over the split partials, in a fixed
 //                 order, optionally transposed ([R, rpad] -> [r, R]), written
 //                 as bf16 or (for a later cross-rank sum) as fp32.
 //   k_zero_bf16   zero fill (gradients of an empty batch).
 #include "common.cuh"
 #include "kernels.h"
-#include "lora_finish.cuh"
 
 namespace qlora {
 namespace {
 
+__global__ void k_split_hilo(const float* __restrict__ T, int64_t M, int r, int rpad, __nv_bfloat16* __restrict__ hi,
+                             __nv_bfloat16* __restrict__ lo) {
+  pdl_enter();
+  const int64_t n = M * rpad;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t m = i / rpad;
+    const int j = static_cast<int>(i % rpad);
+    const float v = j < r ? T[m * r + j] : 0.0f;
+    const __nv_bfloat16 h = __float2bfloat16_rn(v);
+    hi[i] = h;
+    lo[i] = __float2bfloat16_rn(v - __bfloat162float(h));
+  }
+}
 
 // Sum the split partials P[p][m][j] (fixed order) and emit the LoRA operands:
 // f32[m][j] (j < r, optional), s_bf16 = bf16(s v), hi = bf16(v), lo = bf16(v - hi)
 // for j < rpad (zero columns stay zero). Two adjacent columns per thread.
-__global__ void k_lora_finish(const __grid_constant__ LoraFinishJob job) {
+__global__ void k_lora_finish(const float* __restrict__ P, int splits, int64_t M, int r, int rpad, float s,
+                              float* __restrict__ f32, __nv_bfloat16* __restrict__ s_bf16,
+                              __nv_bfloat16* __restrict__ hi, __nv_bfloat16* __restrict__ lo) {
   pdl_enter();
-  lora_finish_range(job, static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x,
-                    static_cast<int64_t>(gridDim.x) * blockDim.x);
+  const int64_t n2 = M * rpad / 2;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n2;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t e = 2 * i;
+    const int64_t m = e / rpad;
+    const int j = static_cast<int>(e % rpad);
+    float2 v = make_float2(0.0f, 0.0f);
+    for (int p = 0; p < splits; ++p) {
+      const float2 pv = reinterpret_cast<const float2*>(P + (static_cast<int64_t>(p) * M) * rpad)[i];
+      v.x += pv.x;
+      v.y += pv.y;
+    }
+    if (f32) {
+      if (j < r) f32[m * r + j] = v.x;
+      if (j + 1 < r) f32[m * r + j + 1] = v.y;
+    }
+    if (s_bf16) reinterpret_cast<uint32_t*>(s_bf16)[i] = pack_bf16x2(s * v.x, s * v.y);
+    if (hi) {
+      const uint32_t h = pack_bf16x2(v.x, v.y);
+      reinterpret_cast<uint32_t*>(hi)[i] = h;
+      reinterpret_cast<uint32_t*>(lo)[i] = pack_bf16x2(v.x - bf16lo_to_f32(h), v.y - bf16hi_to_f32(h));
+    }
+  }
 }
 
 // out = bf16(s * sum_p P[p]) for a [R, rpad] partial stack (rows R, the first r
 // columns kept). A CTA owns a 32-row x 64-column tile: coalesced float2 reads of
 // every split (fixed order), then either direct row-major writes ([R, r]) or a
 // transpose through shared memory so that the [r, R] writes are coalesced too.
+// One CTA per 32 rows x 64 columns; thread (ty, tx) sums the split partials of
+// rows ty and ty + 16, columns 4 tx .. 4 tx + 3 (float4 loads), with the loads
+// of four splits in flight at a time; the sum runs over p = 0, 1, ... in order.
 template <typename OutT>
 __device__ __forceinline__ OutT to_out(float v);
 template <>
@@ -38,59 +75,62 @@ __device__ __forceinline__ __nv_bfloat16 to_out<__nv_bfloat16>(float v) { return
 template <>
 __device__ __forceinline__ float to_out<float>(float v) { return v; }
 
-// One CTA per 16 rows x 64 columns; thread (ty, tx) sums the split partials of
-// row ty, columns 4 tx .. 4 tx + 3 (float4 loads), with the loads of four
-// splits in flight at a time; the sum runs over p = 0, 1, ... in order.
 template <typename OutT>
 __global__ void __launch_bounds__(256)
 k_grad_reduce(const float* __restrict__ P, int splits, int64_t R, int rpad, int r, float s, int transpose,
               OutT* __restrict__ out) {
   pdl_enter();
-  __shared__ float tile[64][17];
-  const int64_t row0 = static_cast<int64_t>(blockIdx.x) * 16;
+  __shared__ float tile[64][33];
+  const int64_t row0 = static_cast<int64_t>(blockIdx.x) * 32;
   const int col0 = blockIdx.y * 64;
   const int tx = threadIdx.x & 15;   // column quad within the tile
-  const int ty = threadIdx.x >> 4;   // row within the tile
+  const int ty = threadIdx.x >> 4;   // 16 row lanes
   const int64_t pstride = R * rpad / 4;  // float4 elements per split
-  const int64_t row = row0 + ty;
-  float4 v = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-  if (row < R) {
-    const float4* src = reinterpret_cast<const float4*>(P + row * rpad + col0) + tx;
-    int p = 0;
-    for (; p + 4 <= splits; p += 4) {
-      float4 q[4];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) q[i] = __ldcs(src + (p + i) * pstride);
+  for (int h = 0; h < 2; ++h) {
+    const int rr = ty + 16 * h;
+    const int64_t row = row0 + rr;
+    float4 v = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    if (row < R) {
+      const float4* src = reinterpret_cast<const float4*>(P + row * rpad + col0) + tx;
+      int p = 0;
+      for (; p + 4 <= splits; p += 4) {
+        float4 q[4];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        v.x += q[i].x; v.y += q[i].y; v.z += q[i].z; v.w += q[i].w;
+        for (int i = 0; i < 4; ++i) q[i] = __ldcs(src + (p + i) * pstride);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          v.x += q[i].x; v.y += q[i].y; v.z += q[i].z; v.w += q[i].w;
+        }
+      }
+      for (; p < splits; ++p) {
+        const float4 q = __ldcs(src + p * pstride);
+        v.x += q.x; v.y += q.y; v.z += q.z; v.w += q.w;
       }
     }
-    for (; p < splits; ++p) {
-      const float4 q = __ldcs(src + p * pstride);
-      v.x += q.x; v.y += q.y; v.z += q.z; v.w += q.w;
-    }
-  }
-  const int c = 4 * tx;
-  if (!transpose) {
-    if (row < R) {
-      const float vv[4] = {v.x, v.y, v.z, v.w};
+    const int c = 4 * tx;
+    if (!transpose) {
+      if (row < R) {
+        const float vv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
-        if (col0 + c + i < r) out[row * r + col0 + c + i] = to_out<OutT>(s * vv[i]);
+        for (int i = 0; i < 4; ++i)
+          if (col0 + c + i < r) out[row * r + col0 + c + i] = to_out<OutT>(s * vv[i]);
+      }
+    } else {
+      tile[c][rr] = v.x;
+      tile[c + 1][rr] = v.y;
+      tile[c + 2][rr] = v.z;
+      tile[c + 3][rr] = v.w;
     }
-    return;
   }
-  tile[c][ty] = v.x;
-  tile[c + 1][ty] = v.y;
-  tile[c + 2][ty] = v.z;
-  tile[c + 3][ty] = v.w;
+  if (!transpose) return;
   __syncthreads();
-  // out[j][row]: 16 consecutive rows per column j
-  for (int idx = threadIdx.x; idx < 64 * 16; idx += blockDim.x) {
-    const int j = col0 + (idx >> 4);
-    const int64_t rr = row0 + (idx & 15);
-    if (j < r && rr < R) out[static_cast<int64_t>(j) * R + rr] = to_out<OutT>(s * tile[idx >> 4][idx & 15]);
+  // out[j][row]: 32 consecutive rows per column j, one warp per column
+  const int wx = threadIdx.x & 31, wy = threadIdx.x >> 5;
+  for (int cc = wy; cc < 64; cc += 8) {
+    const int j = col0 + cc;
+    const int64_t row = row0 + wx;
+    if (j < r && row < R) out[static_cast<int64_t>(j) * R + row] = to_out<OutT>(s * tile[cc][wx]);
   }
 }
 
@@ -110,30 +150,22 @@ int grid_for(int64_t n, int num_sms) {
 
 }  // namespace
 
+cudaError_t launch_split_hilo(const float* T, int64_t M, int r, int rpad, void* hi, void* lo, int num_sms,
+                              cudaStream_t stream) {
+  return launch_pdl(k_split_hilo, dim3(grid_for(M * rpad, num_sms)), dim3(256), 0, stream, T, M, r, rpad,
+                    static_cast<__nv_bfloat16*>(hi), static_cast<__nv_bfloat16*>(lo));
+}
 
 cudaError_t launch_lora_finish(const float* P, int splits, int64_t M, int r, int rpad, float s, float* f32,
-                               void* s_bf16, void* hi, void* lo, int num_sms, cudaStream_t stream,
-                               const float* t_src, void* t_hi, void* t_lo) {
-  LoraFinishJob job;
-  job.P = P;
-  job.splits = splits;
-  job.M = M;
-  job.r = r;
-  job.rpad = rpad;
-  job.s = s;
-  job.f32 = f32;
-  job.s_bf16 = s_bf16;
-  job.hi = hi;
-  job.lo = lo;
-  job.t_src = t_src;
-  job.t_hi = t_hi;
-  job.t_lo = t_lo;
-  return launch_pdl(k_lora_finish, dim3(grid_for(M * rpad / 2, num_sms)), dim3(256), 0, stream, job);
+                               void* s_bf16, void* hi, void* lo, int num_sms, cudaStream_t stream) {
+  return launch_pdl(k_lora_finish, dim3(grid_for(M * rpad / 2, num_sms)), dim3(256), 0, stream, P, splits, M, r,
+                    rpad, s, f32, static_cast<__nv_bfloat16*>(s_bf16), static_cast<__nv_bfloat16*>(hi),
+                    static_cast<__nv_bfloat16*>(lo));
 }
 
 cudaError_t launch_grad_reduce(const float* P, int splits, int64_t R, int rpad, int r, float s, bool transpose,
                                void* out, bool out_f32, int num_sms, cudaStream_t stream) {
-  const dim3 grid(static_cast<unsigned>((R + 15) / 16), static_cast<unsigned>(rpad / 64));
+  const dim3 grid(static_cast<unsigned>((R + 31) / 32), static_cast<unsigned>(rpad / 64));
   if (out_f32)
     return launch_pdl(k_grad_reduce<float>, grid, dim3(256), 0, stream, P, splits, R, rpad, r, s, transpose ? 1 : 0,
                       static_cast<float*>(out));
