@@ -21,7 +21,8 @@ STATUS_NAMES = {0: "QLORA_OK", 1: "QLORA_ERR_INVALID_ARG", 2: "QLORA_ERR_UNSUPPO
                 4: "QLORA_ERR_CUDA", 5: "QLORA_ERR_WORKSPACE", 6: "QLORA_ERR_DEVICE"}
 
 EXPORTED = ("qlora_status_string", "qlora_nf4_codebook", "qlora_nf4_storage_bytes", "qlora_nf4_single_storage_bytes",
-            "qlora_quantize_nf4", "qlora_quantize_nf4_dq", "qlora_quantize_nf4_dq_noalloc", "qlora_dequantize_nf4",
+            "qlora_quantize_nf4", "qlora_quantize_nf4_dq", "qlora_quantize_nf4_dq_noalloc",
+            "qlora_quantize_nf4_dq_shard_begin", "qlora_quantize_nf4_dq_shard_end", "qlora_dequantize_nf4",
             "qlora_dequantize_nf4_dq", "qlora_linear_fwd", "qlora_linear_bwd", "qlora_linear_bwd_f32",
             "qlora_merge_lora",
             "qlora_paged_alloc", "qlora_paged_free", "qlora_paged_prefetch", "qlora_adamw_step",
@@ -69,6 +70,8 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
     lib.qlora_dequantize_nf4.argtypes = [wp, vp, vp]
     lib.qlora_quantize_nf4_dq.argtypes = [vp, wp, vp, szp, vp]
     lib.qlora_quantize_nf4_dq_noalloc.argtypes = [vp, wp, vp]
+    lib.qlora_quantize_nf4_dq_shard_begin.argtypes = [vp, wp, i64, i64, vp, vp, szp, vp]
+    lib.qlora_quantize_nf4_dq_shard_end.argtypes = [wp, i64, i64, vp, vp, sz, vp]
     lib.qlora_dequantize_nf4_dq.argtypes = [wp, vp, vp]
     lib.qlora_linear_fwd.argtypes = [wp, vp, i64, vp, vp, i32, f32, vp, vp, vp, szp, vp]
     lib.qlora_linear_bwd.argtypes = [wp, vp, i64, vp, vp, i32, f32, vp, vp, vp, vp, vp, vp, szp, vp]
@@ -204,6 +207,46 @@ def qlora_quantize_nf4_dq_noalloc(W: torch.Tensor, out: NF4Weight, stream=None) 
     _check(load_library().qlora_quantize_nf4_dq_noalloc(_ptr(W), ctypes.byref(qc), _stream(stream)),
            "qlora_quantize_nf4_dq_noalloc")
     return out
+
+
+def qlora_quantize_nf4_dq_shard_begin(W_shard: torch.Tensor, row_offset: int, total_rows: int,
+                                      out: NF4Weight | None = None, bin_totals: torch.Tensor | None = None,
+                                      workspace: torch.Tensor | None = None, stream=None) -> tuple:
+    """Level 1 of rows [row_offset, row_offset + rows) of a weight with total_rows
+    rows that several callers quantize in row shards. Returns (q, bin_totals,
+    workspace): q holds the shard's codes, bin_totals (int64 [256], device) the
+    exact sum of its block constants by exponent bin, to be summed over all
+    shards before qlora_quantize_nf4_dq_shard_end, and the workspace the shard's
+    fp32 constants, to be kept until then."""
+    assert W_shard.dtype == torch.bfloat16 and W_shard.dim() == 2 and W_shard.is_contiguous()
+    lib = load_library()
+    dev = W_shard.device
+    q = out or NF4Weight.empty(W_shard.shape[0], W_shard.shape[1], dev)
+    if bin_totals is None:
+        bin_totals = torch.empty(256, dtype=torch.int64, device=dev)
+    assert bin_totals.dtype == torch.int64 and bin_totals.numel() == 256 and bin_totals.is_contiguous()
+    qc = q.as_c()
+    st = _stream(stream)
+    ws, nbytes = _workspace(lambda p, n: lib.qlora_quantize_nf4_dq_shard_begin(
+        _ptr(W_shard), ctypes.byref(qc), row_offset, total_rows, _ptr(bin_totals), p, n, st), workspace, dev)
+    _check(lib.qlora_quantize_nf4_dq_shard_begin(_ptr(W_shard), ctypes.byref(qc), row_offset, total_rows,
+                                                 _ptr(bin_totals), _ptr(ws), ctypes.byref(nbytes), st),
+           "qlora_quantize_nf4_dq_shard_begin")
+    return q, bin_totals, ws
+
+
+def qlora_quantize_nf4_dq_shard_end(q: NF4Weight, row_offset: int, total_rows: int, bin_totals: torch.Tensor,
+                                    workspace: torch.Tensor, stream=None) -> NF4Weight:
+    """Level 2 of a row shard once bin_totals holds the sum over all shards: the
+    mean of all constants of the weight, then this shard's int8 codes and group
+    scales (bit-identical to the same rows of a whole-weight quantization)."""
+    assert bin_totals.dtype == torch.int64 and bin_totals.numel() == 256 and bin_totals.is_contiguous()
+    qc = q.as_c()
+    _check(load_library().qlora_quantize_nf4_dq_shard_end(ctypes.byref(qc), row_offset, total_rows,
+                                                          _ptr(bin_totals), _ptr(workspace), workspace.numel(),
+                                                          _stream(stream)),
+           "qlora_quantize_nf4_dq_shard_end")
+    return q
 
 
 def qlora_dequantize_nf4(q: NF4Weight | SingleNF4Weight, out: torch.Tensor | None = None,

@@ -45,6 +45,17 @@ cudaError_t launch_quantize(const void* W, int64_t numel, uint8_t* packed, int8_
                             float* mean, float* absmax_scratch, void* totals_scratch, int num_sms,
                             cudaStream_t stream);
 
+// The two halves of launch_quantize, for a weight quantized in row shards:
+// first, the codes, the fp32 constants and the 256 exact bin totals of their
+// sum (zeroed and then added into); second, after the totals of all shards have
+// been summed, the mean over nblk_mean constants and the int8 codes and group
+// scales of this shard's nblk constants.
+cudaError_t launch_quantize_first(const void* W, int64_t nblk, uint8_t* packed, float* absmax_scratch,
+                                  unsigned long long* totals, int num_sms, cudaStream_t stream);
+cudaError_t launch_quantize_second(const float* absmax_scratch, int64_t nblk, const unsigned long long* totals,
+                                   int64_t nblk_mean, int8_t* absmax_q, float* dq_scale, float* mean,
+                                   cudaStream_t stream);
+
 // Single-level storage: the codes and the fp32 block constants m_b only (pass 1).
 cudaError_t launch_quantize_single(const void* W, int64_t numel, uint8_t* packed, float* absmax, int num_sms,
                                    cudaStream_t stream);

@@ -240,7 +240,8 @@ k_quant_sums(const float* __restrict__ absmax, int64_t nblk, int64_t per_cta,
 }
 
 // mu = fp32(RN_fp64(S) / nblk) from the exact bin totals (warp 0 of the CTA);
-// CTA 0 also stores it.
+// CTA 0 also stores it. nblk counts every constant the totals cover (the whole
+// tensor when this call only codes one shard of its constants).
 __device__ float mean_from_bins(const unsigned long long* __restrict__ totals, int64_t nblk, float* mean_out) {
   __shared__ unsigned long long s_tot[256];
   __shared__ unsigned int s_mask[8];
@@ -277,9 +278,10 @@ __device__ float mean_from_bins(const unsigned long long* __restrict__ totals, i
 
 __global__ void __launch_bounds__(256)
 k_dq_quantize(const float* __restrict__ absmax, int64_t nblk, const unsigned long long* __restrict__ totals,
-              float* __restrict__ mean_out, int8_t* __restrict__ q, float* __restrict__ dq_scale, int64_t ngrp) {
+              int64_t nblk_mean, float* __restrict__ mean_out, int8_t* __restrict__ q, float* __restrict__ dq_scale,
+              int64_t ngrp) {
   pdl_enter();
-  const float mu = mean_from_bins(totals, nblk, mean_out);
+  const float mu = mean_from_bins(totals, nblk_mean, mean_out);
   const int lane = threadIdx.x & 31;
   const int64_t g = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
   if (g >= ngrp) return;  // whole warp leaves together
@@ -360,12 +362,8 @@ cudaError_t launch_pass1(const void* W, int64_t nblk, uint8_t* packed, float* ab
 
 }  // namespace
 
-cudaError_t launch_quantize(const void* W, int64_t numel, uint8_t* packed, int8_t* absmax_q, float* dq_scale,
-                            float* mean, float* absmax_scratch, void* totals_scratch, int num_sms,
-                            cudaStream_t stream) {
-  const int64_t nblk = numel / 64;
-  const int64_t ngrp = (nblk + 255) / 256;
-  unsigned long long* totals = static_cast<unsigned long long*>(totals_scratch);
+cudaError_t launch_quantize_first(const void* W, int64_t nblk, uint8_t* packed, float* absmax_scratch,
+                                  unsigned long long* totals, int num_sms, cudaStream_t stream) {
   cudaError_t e = launch_pass1(W, nblk, packed, absmax_scratch, totals, num_sms, stream);
   if (e != cudaSuccess) return e;
   // chunks of at least 512 constants and at most 8 CTAs per SM (the loop of a
@@ -378,12 +376,28 @@ cudaError_t launch_quantize(const void* W, int64_t numel, uint8_t* packed, int8_
   if (g < 1) g = 1;
   if (g > 0x7fffffff) return cudaErrorInvalidValue;
   const int64_t per_cta = (nblk + g - 1) / g;
-  e = launch_pdl(k_quant_sums, dim3(static_cast<unsigned>(g)), dim3(256), 0, stream,
-                 static_cast<const float*>(absmax_scratch), nblk, per_cta, totals);
+  return launch_pdl(k_quant_sums, dim3(static_cast<unsigned>(g)), dim3(256), 0, stream,
+                    static_cast<const float*>(absmax_scratch), nblk, per_cta, totals);
+}
+
+cudaError_t launch_quantize_second(const float* absmax_scratch, int64_t nblk, const unsigned long long* totals,
+                                   int64_t nblk_mean, int8_t* absmax_q, float* dq_scale, float* mean,
+                                   cudaStream_t stream) {
+  const int64_t ngrp = (nblk + 255) / 256;
+  const int64_t dq_grid = (ngrp + 7) / 8;
+  if (dq_grid > 0x7fffffff) return cudaErrorInvalidValue;
+  return launch_pdl(k_dq_quantize, dim3(static_cast<unsigned>(dq_grid)), dim3(256), 0, stream, absmax_scratch,
+                    nblk, totals, nblk_mean, mean, absmax_q, dq_scale, ngrp);
+}
+
+cudaError_t launch_quantize(const void* W, int64_t numel, uint8_t* packed, int8_t* absmax_q, float* dq_scale,
+                            float* mean, float* absmax_scratch, void* totals_scratch, int num_sms,
+                            cudaStream_t stream) {
+  const int64_t nblk = numel / 64;
+  unsigned long long* totals = static_cast<unsigned long long*>(totals_scratch);
+  cudaError_t e = launch_quantize_first(W, nblk, packed, absmax_scratch, totals, num_sms, stream);
   if (e != cudaSuccess) return e;
-  const int dq_grid = static_cast<int>((ngrp + 7) / 8);
-  return launch_pdl(k_dq_quantize, dim3(dq_grid), dim3(256), 0, stream, static_cast<const float*>(absmax_scratch),
-                    nblk, static_cast<const unsigned long long*>(totals), mean, absmax_q, dq_scale, ngrp);
+  return launch_quantize_second(absmax_scratch, nblk, totals, nblk, absmax_q, dq_scale, mean, stream);
 }
 
 cudaError_t launch_quantize_single(const void* W, int64_t numel, uint8_t* packed, float* absmax, int num_sms,

@@ -15,8 +15,17 @@ buffers and issues the collective.
 ("QLoRA vs ChatGPT", capability 5: gradients are computed only for the LoRA
 parameters, which is what makes the exchange small: r (K + N) values per
 linear.)
+
+A weight too large to quantize on one rank can instead be quantized in row
+shards (quantize_nf4_dq_sharded): each rank codes its rows, and the only
+exchange is the exact sum of the block constants for the double-quantization
+mean, as 256 integer bin totals ("Guanaco", "Core Architecture & Training":
+the constants are quantized again, mean-centred). The shards' outputs are
+bit-identical to quantizing the whole weight on one GPU.
 """
 from __future__ import annotations
+
+import math
 
 import torch
 import torch.distributed as dist
@@ -69,3 +78,39 @@ def shard_tokens(M: int, rank: int, world: int) -> slice:
     lo = rank * M // world
     hi = (rank + 1) * M // world
     return slice(lo, hi)
+
+
+def group_aligned_rows(cols: int) -> int:
+    """Smallest row count whose blocks fill whole 256-constant groups
+    (rows * cols a multiple of 256 * 64 weights)."""
+    return 16384 // math.gcd(16384, cols)
+
+
+def shard_rows(total_rows: int, cols: int, rank: int, world: int) -> slice:
+    """Row range of a rank for sharded quantization: boundaries on whole
+    256-constant groups, sizes as even as that allows (the last shard takes the
+    ragged end; a shard may be empty)."""
+    u = group_aligned_rows(cols)
+    units = -(-total_rows // u)
+    lo = min(total_rows, (rank * units // world) * u)
+    hi = min(total_rows, ((rank + 1) * units // world) * u)
+    return slice(lo, hi)
+
+
+def allreduce_bin_totals(bin_totals: torch.Tensor, group=None) -> torch.Tensor:
+    """Sum the int64 exponent-bin totals of the ranks' constants in place
+    (integer addition: exact, in any order)."""
+    assert bin_totals.dtype == torch.int64
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size(group) > 1:
+        dist.all_reduce(bin_totals, op=dist.ReduceOp.SUM, group=group)
+    return bin_totals
+
+
+def quantize_nf4_dq_sharded(W_local: torch.Tensor, row_offset: int, total_rows: int, group=None, **kw):
+    """Double-quantize rows [row_offset, row_offset + W_local.shape[0]) of a
+    weight of total_rows rows whose other rows the other ranks of `group` hold
+    (boundaries from shard_rows). Returns this rank's NF4Weight."""
+    q, totals, ws = binding.qlora_quantize_nf4_dq_shard_begin(W_local, row_offset, total_rows, **kw)
+    allreduce_bin_totals(totals, group)
+    return binding.qlora_quantize_nf4_dq_shard_end(q, row_offset, total_rows, totals, ws,
+                                                   stream=kw.get("stream"))

@@ -190,6 +190,50 @@ qlora_status qlora_quantize_nf4_dq(const void* W_bf16, const qlora_nf4_weight* q
 qlora_status qlora_quantize_nf4_dq_noalloc(const void* W_bf16, const qlora_nf4_weight* q,
                                            qlora_stream_t stream);
 
+/* qlora_quantize_nf4_dq_shard_begin / qlora_quantize_nf4_dq_shard_end --
+ * qlora_quantize_nf4_dq of one weight W [total_rows, cols] whose rows are
+ * split over several callers (e.g. one row shard per GPU of a data-parallel
+ * job), with outputs bit-identical to quantizing W at once ([C] 1 and 3, [G]
+ * "Core Architecture & Training"). Level 1 is local to each 64-weight block;
+ * level 2 couples the shards only through the mean mu of all constants, which
+ * is exchanged as an exact integer sum.
+ *
+ * Each shard covers rows [row_offset, row_offset + q->rows) of W; q describes
+ * that shard's storage (q->rows rows, its own packed codes, absmax_q of
+ * q->rows*cols/64 codes, dq_scale of ceil(q->rows*cols/16384) groups, one mean).
+ * A shard starts on a 256-constant group boundary ((row_offset*cols) % 16384
+ * == 0) and every shard but the last (row_offset + q->rows < total_rows) also
+ * ends on one; else QLORA_ERR_INVALID_ARG. The groups of the shards are then
+ * the groups of W, and their concatenated outputs equal W's. W may hold at
+ * most 2^56 weights (else QLORA_ERR_UNSUPPORTED).
+ *
+ * begin: level 1 of the shard's rows W_bf16 [q->rows, cols] (device): the codes
+ *   into q->packed, the fp32 constants m_b into the workspace, and the exact
+ *   sum of those constants into bin_totals (device, 256 uint64, 8-byte
+ *   aligned, overwritten): each m_b is an 8-bit significand sig times
+ *   2^(E - 134) with E = max(exponent field, 1), and bin_totals[E] is the sum of
+ *   the significands of the bin. The workspace follows the library's
+ *   convention (NULL: size query), except that its contents must be kept
+ *   unchanged until the matching end call.
+ * Between the calls the caller adds bin_totals over all shards, element-wise as
+ *   integers (e.g. an all-reduce SUM of 256 uint64, or of int64: the totals stay
+ *   below 2^58). Any order gives the same exact totals.
+ * end: mu = fp32(fp64(S) / (total_rows*cols/64)) from the summed totals, stored
+ *   in *q->mean (the same value on every shard), then the int8 codes and group
+ *   scales of this shard's constants, as qlora_quantize_nf4_dq computes them.
+ *   workspace / workspace_bytes: the begin call's workspace and its size.
+ * Both calls are asynchronous on `stream`; an empty shard (q->rows == 0) writes
+ * zero totals in begin and nothing in end.
+ * Errors: INVALID_ARG, UNSUPPORTED, ALIGNMENT, WORKSPACE, CUDA, DEVICE. */
+qlora_status qlora_quantize_nf4_dq_shard_begin(const void* W_bf16, const qlora_nf4_weight* q,
+                                               int64_t row_offset, int64_t total_rows,
+                                               uint64_t* bin_totals, void* workspace,
+                                               size_t* workspace_bytes, qlora_stream_t stream);
+qlora_status qlora_quantize_nf4_dq_shard_end(const qlora_nf4_weight* q, int64_t row_offset,
+                                             int64_t total_rows, const uint64_t* bin_totals,
+                                             const void* workspace, size_t workspace_bytes,
+                                             qlora_stream_t stream);
+
 /* qlora_dequantize_nf4 -- decode q (either storage kind) to a bf16 matrix
  * out_bf16 [rows, cols] (device, 16-byte aligned): w' = bf16_rn(fp32(
  * codebook[code] * m'_b)) with the block constant m'_b of the storage kind

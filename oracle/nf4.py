@@ -163,18 +163,21 @@ def dq_mean(absmax: np.ndarray) -> np.float32:
     return np.float32(np.float64(S) / np.float64(n))
 
 
-def double_quantize(absmax: np.ndarray):
+def double_quantize(absmax: np.ndarray, mean=None):
     """Second-level quantization of the fp32 absmax constants to int8.
 
     mu = dq_mean(absmax); c_b = fp32(m_b - mu). Per group of 256 consecutive
     constants (the last group may be shorter): s_g = max |c_b|,
     dq_scale_g = fp32(s_g / 127), q_b = clamp(rint_even(fp32(c_b / dq_scale_g)),
     -127, 127). A group with s_g == 0 gets dq_scale_g = 0 and q_b = 0.
+    `mean`, when given, is the mean of a larger set of constants that `absmax`
+    is a group-aligned part of (a row shard of the weight), used in place of
+    dq_mean(absmax).
     Returns (q int8 [nblk], dq_scale fp32 [ngrp], mu fp32).
     """
     m = np.asarray(absmax, dtype=np.float32)
     n = m.size
-    mu = dq_mean(m)
+    mu = dq_mean(m) if mean is None else np.float32(mean)
     c = (m - mu).astype(np.float32)
     ngrp = (n + DQ_BLOCK - 1) // DQ_BLOCK
     cp = np.zeros(ngrp * DQ_BLOCK, dtype=np.float32)
