@@ -449,6 +449,10 @@ def run_ours(args, rank, world, dev):
         work.step()
         if i == 0:
             torch.cuda.synchronize()
+            # a kernel wait that gave up (device error word) makes every later
+            # number meaningless: stop here, on every rank, instead of timing it
+            if max_over_ranks(float(qb.qlora_device_error()), world, dev):
+                raise RuntimeError(f"device error {qb.qlora_device_error()} after the first warm-up step")
     while time.time() - t_w < 1.0:  # let the sampler produce its first lines
         work.step()
         torch.cuda.synchronize()
