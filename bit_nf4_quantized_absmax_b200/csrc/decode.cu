@@ -257,7 +257,9 @@ k_decode(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUten
         }
       }
     }
-    grid_dependency_launch_dependents();
+    // no launch_dependents here: the consumer warps signal the next grid after
+    // they have waited for the LoRA-down kernel (wait, then trigger, as in
+    // every kernel of the library), so at most two grids are ever in flight
     return;
   }
   // ---- consumer warps ----
