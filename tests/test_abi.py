@@ -32,6 +32,19 @@ def test_library_exports_every_declared_symbol():
     assert set(declared) == set(b.EXPORTED)
 
 
+def test_header_is_plain_c():
+    """The boundary header compiles as C99 and as C++ (no torch or CUDA types)."""
+    import shutil
+    import subprocess
+    for cc, std, lang in (("gcc", "-std=c99", "c"), ("g++", "-std=c++17", "c++")):
+        exe = shutil.which(cc)
+        if exe is None:
+            pytest.skip(f"{cc} not installed")
+        res = subprocess.run([exe, std, "-Wall", "-Wextra", "-Werror", "-fsyntax-only", "-x", lang, HEADER],
+                             capture_output=True, text=True)
+        assert res.returncode == 0, res.stderr
+
+
 def test_status_strings():
     assert b.qlora_status_string(0) == "QLORA_OK"
     assert b.qlora_status_string(5) == "QLORA_ERR_WORKSPACE"
