@@ -385,9 +385,9 @@ def merge_measure(work, dev, reps=10):
     torch.cuda.synchronize()
     us = 1e3 * a.elapsed_time(b) / reps
     flops = 2.0 * R * N * K
+    # no fp64 peak was measured on this machine, so no roofline fraction is given
     return {"shape": f"{N}x{K}", "r": R, "us": round(us, 1), "fp64_TFLOP_s": round(flops / us / 1e6, 2),
-            "peak_fp64_TFLOP_s": 40.0, "peak_kind": "nominal B200 fp64 (no measured figure)",
-            "frac": round(flops / us / 1e6 / 40.0, 4)}
+            "peak": None, "peak_note": "fp64 peak not measured here (nominal B200 fp64 is about 40 TFLOP/s)"}
 
 
 def adamw_measure(dev, peaks, n=1 << 26, reps=10):
@@ -536,11 +536,13 @@ def run_ours(args, rank, world, dev):
     fwd_us = 1e3 * statistics.mean(a.elapsed_time(b) for a, b in ev[roof_part])
     achieved = train_flops(*ROOFLINE_SHAPE)[0] / fwd_us / 1e6
     traffic = TRAFFIC_RECORD["bytes"] if TRAFFIC_RECORD["fingerprint"] == source_fingerprint() else None
+    # the call is timed alone (its own event pair, a few hundred microseconds), so
+    # the burst figure is its peak; the sustained one is reported beside it
     roof = {"kernel": "qlora_linear_fwd M=4096 on 11008x4096 (dequant, LoRA-down, 2-CTA tcgen05 GEMM)",
-            "bound": "tensor", "achieved": round(achieved, 1), "peak": peaks["bf16_tflops_sustained"],
-            "peak_kind": f"bf16 dense sustained ({peaks['source']})", "unit": "TFLOP/s",
-            "frac": round(achieved / peaks["bf16_tflops_sustained"], 4),
-            "frac_of_burst": round(achieved / peaks["bf16_tflops"], 4), "traffic": traffic,
+            "bound": "tensor", "achieved": round(achieved, 1), "peak": peaks["bf16_tflops"],
+            "peak_kind": f"bf16 dense burst ({peaks['source']})", "unit": "TFLOP/s",
+            "frac": round(achieved / peaks["bf16_tflops"], 4),
+            "frac_of_sustained": round(achieved / peaks["bf16_tflops_sustained"], 4), "traffic": traffic,
             "us_per_launch": round(fwd_us, 2)}
     dec = [parts[f"decode{M}/{N}x{K}"]["weight_GB_s"] for M in M_DECODE for N, K in SHAPES]
 

@@ -24,7 +24,7 @@ EXPORTED = ("qlora_status_string", "qlora_nf4_codebook", "qlora_nf4_storage_byte
             "qlora_quantize_nf4", "qlora_quantize_nf4_dq", "qlora_quantize_nf4_dq_noalloc",
             "qlora_quantize_nf4_dq_shard_begin", "qlora_quantize_nf4_dq_shard_end", "qlora_dequantize_nf4",
             "qlora_dequantize_nf4_dq", "qlora_linear_fwd", "qlora_linear_bwd", "qlora_linear_bwd_f32",
-            "qlora_merge_lora",
+            "qlora_linear_bwd_dp", "qlora_round_bf16", "qlora_merge_lora",
             "qlora_paged_alloc", "qlora_paged_free", "qlora_paged_prefetch", "qlora_adamw_step",
             "qlora_device_error")
 
@@ -76,6 +76,8 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
     lib.qlora_linear_fwd.argtypes = [wp, vp, i64, vp, vp, i32, f32, vp, vp, vp, szp, vp]
     lib.qlora_linear_bwd.argtypes = [wp, vp, i64, vp, vp, i32, f32, vp, vp, vp, vp, vp, vp, szp, vp]
     lib.qlora_linear_bwd_f32.argtypes = [wp, vp, i64, vp, vp, i32, f32, vp, vp, vp, vp, vp, vp, szp, vp]
+    lib.qlora_linear_bwd_dp.argtypes = [wp, vp, i64, vp, vp, i32, f32, vp, vp, vp, vp, vp, vp, szp, vp]
+    lib.qlora_round_bf16.argtypes = [vp, vp, i64, vp]
     lib.qlora_merge_lora.argtypes = [wp, ctypes.POINTER(_Adapter), i32, vp, vp]
     lib.qlora_device_error.argtypes = [ctypes.POINTER(ctypes.c_int32), vp]
     lib.qlora_paged_alloc.argtypes = [sz, i32, ctypes.POINTER(vp)]
@@ -316,6 +318,44 @@ def qlora_linear_bwd(q: NF4Weight | SingleNF4Weight, X: torch.Tensor, A: torch.T
     ws, nbytes = _workspace(args, workspace, dev)
     _check(args(_ptr(ws), ctypes.byref(nbytes)), "qlora_linear_bwd_f32" if grads_fp32 else "qlora_linear_bwd")
     return (dX if need_dX else None), dA, dB
+
+
+def qlora_linear_bwd_dp(q: NF4Weight | SingleNF4Weight, X: torch.Tensor, A: torch.Tensor, B: torch.Tensor,
+                        alpha: float, dY: torch.Tensor, grads: torch.Tensor, T_saved: torch.Tensor | None = None,
+                        need_dX: bool = True, dX: torch.Tensor | None = None, grads_ready=None,
+                        workspace: torch.Tensor | None = None, stream=None):
+    """Backward of one token shard with dA and dB in fp32 in one flat buffer
+    `grads` [r*K + N*r] (dA first); `grads_ready` (a torch.cuda.Event or None) is
+    recorded on the stream once `grads` is complete, before the dX kernels.
+    Returns dX or None."""
+    lib = load_library()
+    M, r = X.shape[0], A.shape[0]
+    dev = X.device
+    assert grads.dtype == torch.float32 and grads.is_contiguous() and grads.numel() == r * q.cols + q.rows * r
+    if need_dX and dX is None:
+        dX = torch.empty(M, q.cols, dtype=torch.bfloat16, device=dev)
+    ev = None
+    if grads_ready is not None:
+        grads_ready.record(torch.cuda.current_stream() if stream is None else stream)  # creates the CUDA event
+        ev = ctypes.c_void_p(grads_ready.cuda_event)
+    qc = q.as_c()
+    st = _stream(stream)
+    args = lambda p, n: lib.qlora_linear_bwd_dp(ctypes.byref(qc), _ptr(X), M, _ptr(A), _ptr(B), r, float(alpha),
+                                                _ptr(dY), _ptr(T_saved), _ptr(dX if need_dX else None), _ptr(grads),
+                                                ev, p, n, st)
+    ws, nbytes = _workspace(args, workspace, dev)
+    _check(args(_ptr(ws), ctypes.byref(nbytes)), "qlora_linear_bwd_dp")
+    return dX if need_dX else None
+
+
+def qlora_round_bf16(src: torch.Tensor, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """bf16_rn of an fp32 tensor, in the library's kernel."""
+    assert src.dtype == torch.float32 and src.is_contiguous()
+    if out is None:
+        out = torch.empty(src.shape, dtype=torch.bfloat16, device=src.device)
+    assert out.dtype == torch.bfloat16 and out.is_contiguous() and out.numel() == src.numel()
+    _check(load_library().qlora_round_bf16(_ptr(src), _ptr(out), src.numel(), _stream(stream)), "qlora_round_bf16")
+    return out
 
 
 def qlora_merge_lora(q: NF4Weight | SingleNF4Weight, adapters, out: torch.Tensor | None = None,

@@ -133,10 +133,13 @@ struct Layout {
   size_t total() const { return off > 0 ? off : kAlign; }
 };
 
-// Backward shared by qlora_linear_bwd (bf16 dA, dB) and qlora_linear_bwd_f32 (fp32 dA, dB).
+// Backward shared by qlora_linear_bwd (bf16 dA, dB), qlora_linear_bwd_f32 and
+// qlora_linear_bwd_dp (fp32 dA, dB). The LoRA gradients are finished before the
+// dX GEMM; `grads_ready`, when given, is recorded on the stream right after them.
 qlora_status linear_bwd_impl(const qlora_nf4_weight* q, const void* X, int64_t M, const void* A, const void* B,
                              int32_t r, float alpha, const void* dY, const float* T_saved, void* dX, void* dA,
-                             void* dB, bool f32, void* workspace, size_t* workspace_bytes, qlora_stream_t stream) {
+                             void* dB, bool f32, void* workspace, size_t* workspace_bytes, qlora_stream_t stream,
+                             cudaEvent_t grads_ready = nullptr) {
   qlora_status st = check_weight(q, true);
   if (st != QLORA_OK) return st;
   if ((st = check_linear(X, M, A, B, r, dA)) != QLORA_OK) return st;
@@ -174,6 +177,7 @@ qlora_status linear_bwd_impl(const qlora_nf4_weight* q, const void* X, int64_t M
     if (f32) {
       cudaError_t e = cudaMemsetAsync(dA, 0, static_cast<size_t>(r) * K * sizeof(float), cs);
       if (e == cudaSuccess) e = cudaMemsetAsync(dB, 0, static_cast<size_t>(N) * r * sizeof(float), cs);
+      if (e == cudaSuccess && grads_ready) e = cudaEventRecord(grads_ready, cs);
       return cuda_status(e);
     }
     cudaError_t e = launch_zero_bf16(dA, static_cast<int64_t>(r) * K, di.num_sms, cs);
@@ -197,18 +201,20 @@ qlora_status linear_bwd_impl(const qlora_nf4_weight* q, const void* X, int64_t M
   // U = dY B: s U for the dX slab, U as hi + lo for dA
   if (e == cudaSuccess) e = launch_gemm_lora_u(dY, B, M, N, r, rpad, P, splits_u, di.num_sms, err, cs);
   if (e == cudaSuccess) e = launch_lora_finish(P, splits_u, M, r, rpad, s, nullptr, sU, Uhi, Ulo, di.num_sms, cs);
-  if (dX) {
-    void* Wd = ws + off_wd;
-    if (e == cudaSuccess)
-      e = launch_dequantize(view(q), Wd, cb, di.num_sms, cs);
-    if (e == cudaSuccess) e = launch_gemm_dx(dY, Wd, sU, A, M, N, K, r, rpad, dX, di.num_sms, err, cs);
-  }
   // dA^T [K, r] = X^T U, reduced over tokens, then dA = s * (.)^T
   if (e == cudaSuccess) e = launch_gemm_lora_grad(X, K, Uhi, Ulo, M, rpad, P, splits_a, di.num_sms, err, cs);
   if (e == cudaSuccess) e = launch_grad_reduce(P, splits_a, K, rpad, r, s, true, dA, f32, di.num_sms, cs);
   // dB [N, r] = dY^T T
   if (e == cudaSuccess) e = launch_gemm_lora_grad(dY, N, Thi, Tlo, M, rpad, P, splits_b, di.num_sms, err, cs);
   if (e == cudaSuccess) e = launch_grad_reduce(P, splits_b, N, rpad, r, s, false, dB, f32, di.num_sms, cs);
+  // the LoRA gradients are complete: a cross-rank sum may start while dX runs
+  if (e == cudaSuccess && grads_ready) e = cudaEventRecord(grads_ready, cs);
+  if (dX) {
+    void* Wd = ws + off_wd;
+    if (e == cudaSuccess)
+      e = launch_dequantize(view(q), Wd, cb, di.num_sms, cs);
+    if (e == cudaSuccess) e = launch_gemm_dx(dY, Wd, sU, A, M, N, K, r, rpad, dX, di.num_sms, err, cs);
+  }
   return cuda_status(e);
 }
 
@@ -374,6 +380,29 @@ qlora_status qlora_linear_bwd_f32(const qlora_nf4_weight* q, const void* X, int6
                                   qlora_stream_t stream) {
   return linear_bwd_impl(q, X, M, A, B, r, alpha, dY, T_saved, dX, dA, dB, true, workspace, workspace_bytes,
                          stream);
+}
+
+qlora_status qlora_linear_bwd_dp(const qlora_nf4_weight* q, const void* X, int64_t M, const void* A,
+                                 const void* B, int32_t r, float alpha, const void* dY, const float* T_saved,
+                                 void* dX, float* grads, qlora_event_t grads_ready, void* workspace,
+                                 size_t* workspace_bytes, qlora_stream_t stream) {
+  if (!q || !grads) return QLORA_ERR_INVALID_ARG;
+  if (!aligned(grads, 16)) return QLORA_ERR_ALIGNMENT;
+  // dA [r, K] then dB [N, r]; r % 8 == 0 keeps dB's start 16-byte aligned
+  float* dB = grads + static_cast<int64_t>(r) * q->cols;
+  return linear_bwd_impl(q, X, M, A, B, r, alpha, dY, T_saved, dX, grads, dB, true, workspace, workspace_bytes,
+                         stream, reinterpret_cast<cudaEvent_t>(grads_ready));
+}
+
+qlora_status qlora_round_bf16(const float* src, void* dst_bf16, int64_t n, qlora_stream_t stream) {
+  if (n < 0) return QLORA_ERR_INVALID_ARG;
+  if (n == 0) return QLORA_OK;
+  if (!src || !dst_bf16) return QLORA_ERR_INVALID_ARG;
+  if (!aligned(src, 4) || !aligned(dst_bf16, 2)) return QLORA_ERR_ALIGNMENT;
+  DeviceInfo di;
+  qlora_status st = device_info(&di);
+  if (st != QLORA_OK) return st;
+  return cuda_status(launch_round_bf16(src, dst_bf16, n, di.num_sms, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 qlora_status qlora_merge_lora(const qlora_nf4_weight* q, const qlora_lora_adapter* adapters,

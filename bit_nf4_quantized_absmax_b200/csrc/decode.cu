@@ -373,7 +373,9 @@ k_decode(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUten
     ++rg;
     sb = 0;
   }
-  if (!entered) grid_dependency_launch_dependents();
+  // a warp that published nothing (a bounded wait gave up) still waits for the
+  // LoRA-down kernel before it lets the next grid launch, like every other path
+  if (!entered) pdl_enter();
 }
 
 // T[m, j] = sum_k X[m, k] A[j, k] for M <= 16 (fp32 on CUDA cores), one CTA per

@@ -132,5 +132,7 @@ cudaError_t launch_lora_finish(const float* P, int splits, int64_t M, int r, int
 cudaError_t launch_grad_reduce(const float* P, int splits, int64_t R, int rpad, int r, float s, bool transpose,
                                void* out, bool out_f32, int num_sms, cudaStream_t stream);
 cudaError_t launch_zero_bf16(void* p, int64_t n, int num_sms, cudaStream_t stream);
+// dst (bf16 [n]) = bf16_rn(src (fp32 [n])).
+cudaError_t launch_round_bf16(const float* src, void* dst, int64_t n, int num_sms, cudaStream_t stream);
 
 }  // namespace qlora

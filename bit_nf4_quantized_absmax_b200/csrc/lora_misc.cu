@@ -8,6 +8,8 @@
 //                 order, optionally transposed ([R, rpad] -> [r, R]), written
 //                 as bf16 or (for a later cross-rank sum) as fp32.
 //   k_zero_bf16   zero fill (gradients of an empty batch).
+//   k_round_bf16  fp32 -> bf16 (nearest, ties to even), e.g. the LoRA gradients
+//                 of a data-parallel step once the ranks' fp32 sums are in.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -141,6 +143,24 @@ __global__ void k_zero_bf16(__nv_bfloat16* __restrict__ p, int64_t n) {
     p[i] = __float2bfloat16_rn(0.0f);
 }
 
+// Four elements per thread and step (16-byte loads, 8-byte stores) when both
+// pointers allow it; the tail and unaligned buffers go element by element.
+__global__ void k_round_bf16(const float* __restrict__ src, __nv_bfloat16* __restrict__ dst, int64_t n, int vec) {
+  pdl_enter();
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  const int64_t t0 = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  int64_t done = 0;
+  if (vec) {
+    const int64_t n4 = n / 4;
+    for (int64_t i = t0; i < n4; i += stride) {
+      const float4 v = reinterpret_cast<const float4*>(src)[i];
+      reinterpret_cast<uint2*>(dst)[i] = make_uint2(pack_bf16x2(v.x, v.y), pack_bf16x2(v.z, v.w));
+    }
+    done = 4 * n4;
+  }
+  for (int64_t i = done + t0; i < n; i += stride) dst[i] = __float2bfloat16_rn(src[i]);
+}
+
 int grid_for(int64_t n, int num_sms) {
   int64_t g = (n + 255) / 256;
   const int64_t cap = static_cast<int64_t>(num_sms) * 8;
@@ -171,6 +191,13 @@ cudaError_t launch_grad_reduce(const float* P, int splits, int64_t R, int rpad, 
                       static_cast<float*>(out));
   return launch_pdl(k_grad_reduce<__nv_bfloat16>, grid, dim3(256), 0, stream, P, splits, R, rpad, r, s,
                     transpose ? 1 : 0, static_cast<__nv_bfloat16*>(out));
+}
+
+cudaError_t launch_round_bf16(const float* src, void* dst, int64_t n, int num_sms, cudaStream_t stream) {
+  if (n <= 0) return cudaSuccess;
+  const int vec = ((reinterpret_cast<uintptr_t>(src) & 15u) == 0 && (reinterpret_cast<uintptr_t>(dst) & 7u) == 0) ? 1 : 0;
+  return launch_pdl(k_round_bf16, dim3(grid_for(vec ? (n + 3) / 4 : n, num_sms)), dim3(256), 0, stream, src,
+                    static_cast<__nv_bfloat16*>(dst), n, vec);
 }
 
 cudaError_t launch_zero_bf16(void* p, int64_t n, int num_sms, cudaStream_t stream) {

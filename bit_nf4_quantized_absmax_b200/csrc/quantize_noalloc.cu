@@ -31,27 +31,31 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
 constexpr int kMaxDevices = 64;
 
 struct DeviceScratch {
-  std::once_flag once;
-  void* ptr = nullptr;
-  cudaError_t err = cudaSuccess;
+  std::mutex mu;
+  void* ptr = nullptr;  // set once the lookup has succeeded
 };
 
 DeviceScratch g_scratch[kMaxDevices];
 
 // Device address of the scratch array on the current device. In host code the
 // array's name is only a host-side stand-in, so its device address is looked
-// up once per device, with that device current, on the first call.
+// up with that device current. Only a successful lookup is kept: a call that
+// fails (for instance the first call made inside a stream capture) returns
+// QLORA_ERR_CUDA and the next call on that device tries again.
 qlora_status scratch_on_current_device(void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return QLORA_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return QLORA_ERR_DEVICE;
   DeviceScratch& d = g_scratch[dev];
-  std::call_once(d.once, [&d] {
+  std::lock_guard<std::mutex> lock(d.mu);
+  if (!d.ptr) {
     void* p = nullptr;
-    d.err = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) {
+      (void)cudaGetLastError();  // do not leave the failure for the caller's next error check
+      return QLORA_ERR_CUDA;
+    }
     d.ptr = p;
-  });
-  if (d.err != cudaSuccess || !d.ptr) return QLORA_ERR_CUDA;
+  }
   *out = d.ptr;
   return QLORA_OK;
 }

@@ -58,6 +58,8 @@ extern "C" {
 
 /* The stream type is the CUDA runtime's cudaStream_t (NULL = legacy default). */
 typedef struct CUstream_st* qlora_stream_t;
+/* The event type is the CUDA runtime's cudaEvent_t. */
+typedef struct CUevent_st* qlora_event_t;
 
 typedef enum {
   QLORA_OK = 0,
@@ -184,7 +186,10 @@ qlora_status qlora_quantize_nf4_dq(const void* W_bf16, const qlora_nf4_weight* q
  * weights), larger weights return QLORA_ERR_UNSUPPORTED before any launch. The
  * first call on a device looks up that array's device address (one
  * cudaGetSymbolAddress with the device current); make that first call before
- * any stream capture. All calls share the array, so calls that overlap on the
+ * any stream capture. A failed lookup is not kept: that call returns
+ * QLORA_ERR_CUDA and the next one tries again. The address is kept for the
+ * life of the process, so after cudaDeviceReset on a device this call must not
+ * be used on it again. All calls share the array, so calls that overlap on the
  * GPU race: order them on one stream. Other arguments, alignment rules and
  * errors are those of qlora_quantize_nf4_dq. */
 qlora_status qlora_quantize_nf4_dq_noalloc(const void* W_bf16, const qlora_nf4_weight* q,
@@ -295,6 +300,35 @@ qlora_status qlora_linear_bwd_f32(const qlora_nf4_weight* q, const void* X, int6
                                   void* dX, float* dA, float* dB,
                                   void* workspace, size_t* workspace_bytes,
                                   qlora_stream_t stream);
+
+/* qlora_linear_bwd_dp -- the backward of one rank's token shard in data-parallel
+ * training ([C] 5: gradients are computed only for the LoRA parameters, so the
+ * ranks exchange only r (K + N) values per linear). The same gradients as
+ * qlora_linear_bwd_f32, laid out for the exchange and ordered so that it can
+ * overlap the dX GEMM:
+ *   grads       : device fp32 [r*K + N*r], 16-byte aligned: dA [r, K] row-major
+ *                 followed by dB [N, r] row-major, both before any rounding.
+ *   grads_ready : a cudaEvent_t or NULL. When given, it is recorded on `stream`
+ *                 as soon as `grads` is complete, before the kernels of dX are
+ *                 launched, so that another stream can wait on it and sum
+ *                 `grads` over the ranks (e.g. an NCCL all-reduce) while dX is
+ *                 computed. Round the sums with qlora_round_bf16.
+ * dX (bf16 [M, K], or NULL), the other arguments and the errors are those of
+ * qlora_linear_bwd. */
+qlora_status qlora_linear_bwd_dp(const qlora_nf4_weight* q, const void* X, int64_t M,
+                                 const void* A, const void* B, int32_t r, float alpha,
+                                 const void* dY, const float* T_saved, void* dX, float* grads,
+                                 qlora_event_t grads_ready, void* workspace, size_t* workspace_bytes,
+                                 qlora_stream_t stream);
+
+/* qlora_round_bf16 -- dst[i] = bf16_rn(src[i]) (nearest, ties to even) for
+ * 0 <= i < n: the one rounding that qlora_linear_bwd applies to its fp32
+ * gradients, applied by a data-parallel step to the sums over its ranks
+ * ([C] 5). src: device fp32 [n], 4-byte aligned; dst_bf16: device bf16 [n],
+ * 2-byte aligned (16- and 8-byte alignment take a vector path). n == 0 launches
+ * nothing. Asynchronous on `stream`.
+ * Errors: INVALID_ARG (n < 0, NULL pointers with n > 0), ALIGNMENT, CUDA, DEVICE. */
+qlora_status qlora_round_bf16(const float* src, void* dst_bf16, int64_t n, qlora_stream_t stream);
 
 /* One LoRA adapter of a merge: A [r, cols] and B [rows, r] (device bf16,
  * 16-byte aligned, row-major), 8 <= r <= 256 with r % 8 == 0, scale

@@ -51,13 +51,15 @@ def _worker(rank, world, port, out_dir):
     inp = _case()
     sl = dp.shard_tokens(inp.X.shape[0], rank, world)
     dA_l, dB_l = _oracle_grads(inp, sl)
-    dA32 = torch.from_numpy(dA_l.astype(np.float32))  # fp32, as qlora_linear_bwd_f32 returns them
-    dB32 = torch.from_numpy(dB_l.astype(np.float32))
-    dA = torch.empty(dA32.shape, dtype=torch.bfloat16)
-    dB = torch.empty(dB32.shape, dtype=torch.bfloat16)
-    dp.allreduce_lora_grads(dA32, dB32, out_A=dA, out_B=dB)
+    # fp32, in the flat layout qlora_linear_bwd_dp writes (dA then dB)
+    buf, vA, vB = dp.flat_grads(inp.r, inp.X.shape[1], inp.W.shape[0])
+    vA.copy_(torch.from_numpy(dA_l.astype(np.float32)))
+    vB.copy_(torch.from_numpy(dB_l.astype(np.float32)))
+    dp.allreduce_grads(buf)
     dist.barrier()
     dist.destroy_process_group()
+    # the one rounding to bf16 (the library's qlora_round_bf16 on a GPU); here torch's
+    dA, dB = vA.to(torch.bfloat16), vB.to(torch.bfloat16)
     np.save(os.path.join(out_dir, f"dA{rank}.npy"), dA.float().numpy())
     np.save(os.path.join(out_dir, f"dB{rank}.npy"), dB.float().numpy())
     with open(os.path.join(out_dir, f"rank{rank}.json"), "w") as f:

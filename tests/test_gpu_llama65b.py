@@ -112,7 +112,7 @@ def test_llama65b_whole_model_sweep():
         A_l.append(syn.normal_bf16((r, K), 0.02, 0, "sweep65b", 9000 + 4 * j).to(dev))
         B_l.append(syn.normal_bf16((N, r), 0.02, 0, "sweep65b", 9001 + 4 * j).to(dev))
         X_l.append(syn.normal_bf16((1, K), 1.0, 0, "sweep65b", 9002 + 4 * j).to(dev))
-    outs = {}
+    outs, dq_kept = {}, {}
     dq_out = wbuf
     for i, q in enumerate(stor):
         layer, j = divmod(i, len(shapes))
@@ -121,6 +121,7 @@ def test_llama65b_whole_model_sweep():
         Y, _ = b.qlora_linear_fwd(q, X_l[j], A_l[j], B_l[j], alpha, workspace=ws)
         if (layer, j) in sampled:
             outs[(layer, j)] = Y
+            dq_kept[(layer, j)] = dq_out[:N * K].view(N, K).cpu()
     torch.cuda.synchronize()
     assert b.qlora_device_error() == 0
 
@@ -130,7 +131,10 @@ def test_llama65b_whole_model_sweep():
         ref = oracle.quantize_nf4_dq(bf16_to_f32_np(Wc))
         rows = np.concatenate([[0, N - 1], np.random.default_rng(layer).choice(N, 14, replace=False)])
         _check_constants_and_rows(q, ref, rows, K)
-        Wd = oracle.bf16_bits_to_f32(oracle.dequantize_nf4_dq(ref)).astype(np.float64)
+        wd_bits = oracle.dequantize_nf4_dq(ref)
+        # the sweep's own dequant pass of this linear, bit for bit
+        assert np.array_equal(bf16_bits_np(dq_kept[(layer, j)]), wd_bits)
+        Wd = oracle.bf16_bits_to_f32(wd_bits).astype(np.float64)
         Yr, _ = oracle.linear_fwd(Wd, bf16_to_f32_np(X_l[j]).astype(np.float64),
                                   bf16_to_f32_np(A_l[j]).astype(np.float64),
                                   bf16_to_f32_np(B_l[j]).astype(np.float64), oracle.lora_scale(alpha, r))

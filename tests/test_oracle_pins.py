@@ -294,6 +294,84 @@ def test_dq_rint_ties_to_even_and_bound():
     assert q.min() >= -127 and q.max() <= 127
 
 
+def _dq_codes_exact(c: list, mu: np.float32) -> tuple:
+    """Int8 codes and scale of one group by exact rational arithmetic, written
+    from the definition: c_b = fp32(m_b - mu), s = max |c_b|, scale =
+    fp32(s / 127), q_b = clamp(round-half-even(fp32(c_b / scale)), -127, 127)."""
+    cc = [frac_round_f32(Fraction(float(m)) - Fraction(float(mu))) for m in c]
+    s = max(abs(Fraction(float(x))) for x in cc)
+    scale = frac_round_f32(s / 127)
+    if scale == 0:
+        return [0] * len(cc), scale
+    out = []
+    for x in cc:
+        quo = Fraction(float(frac_round_f32(Fraction(float(x)) / Fraction(float(scale)))))
+        fl = math.floor(quo)
+        d = quo - fl
+        k = fl + 1 if (d > Fraction(1, 2) or (d == Fraction(1, 2) and fl % 2 == 1)) else fl
+        out.append(max(-127, min(127, int(k))))
+    return out, scale
+
+
+def test_dq_quotient_exact_rationals():
+    """The int8 code of each constant is round-half-even of the fp32-rounded
+    quotient c_b / scale ("QLoRA vs ChatGPT", capability 3: the first-level
+    constants are quantized to 8 bit with scales of their own).
+
+    Checked against exact rationals on 10^4 random groups (a sample of their
+    constants by Fraction, all of them through an fp64 quotient rounded once to
+    fp32, which is the correctly rounded fp32 quotient because 53 >= 2*24 + 2),
+    and on constructed constants whose quotient lies within a few fp32 ulps of
+    k + 1/2, where rounding the quotient to fp32 first decides the code: there
+    a reciprocal multiply, or rounding the unrounded quotient, gives other codes."""
+    rng = np.random.default_rng(777)
+    ngrp = 10_000
+    m = np.abs(_rand_bf16((ngrp, 256), std=0.02, seed=3)).astype(np.float32).reshape(-1)
+    m = np.maximum(m, np.float32(1e-4))
+    mu = np.float32(0.0123)
+    q, sc, mu_out = onf4.double_quantize(m, mean=mu)
+    assert mu_out == mu and sc.shape == (ngrp,)
+    # every constant: fp64 quotient of the two fp32 values, one rounding to fp32, rint (ties to even)
+    c = (m - mu).astype(np.float32)
+    grp = np.arange(m.size) // 256
+    ref = np.rint(np.float32(c.astype(np.float64) / sc[grp].astype(np.float64)))
+    assert np.array_equal(q.astype(np.int64), np.clip(ref, -127, 127).astype(np.int64))
+    # a random sample of groups by exact rationals
+    for g in rng.choice(ngrp, 12, replace=False):
+        want, scale = _dq_codes_exact(m[256 * g:256 * (g + 1)].tolist(), mu)
+        assert sc[g] == scale
+        assert q[256 * g:256 * (g + 1)].tolist() == want
+
+    # constructed near-ties: scale fixed by one constant, the others near (k + 1/2) * scale
+    cases_recip, cases_unrounded, checked = 0, 0, 0
+    for trial in range(40):
+        s = np.float32(rng.uniform(0.01, 0.2))
+        scale = frac_round_f32(Fraction(float(s)) / 127)
+        group = [s]
+        for k in rng.integers(-126, 126, size=24):
+            target = np.float32((k + 0.5) * float(scale))
+            x = target
+            for step in range(-3, 4):
+                y = x
+                for _ in range(abs(step)):
+                    y = np.nextafter(y, np.float32(np.inf if step > 0 else -np.inf))
+                if abs(float(y)) <= float(s):
+                    group.append(np.float32(y))
+        group = np.array(group, dtype=np.float32)
+        q, sc, _ = onf4.double_quantize(group, mean=np.float32(0.0))
+        want, scale_x = _dq_codes_exact(group.tolist(), np.float32(0.0))
+        assert sc[0] == scale_x and q.tolist() == want
+        checked += group.size
+        r = np.float32(np.float32(1.0) / sc[0])
+        recip = np.clip(np.rint(np.float32(group * r)), -127, 127).astype(int)
+        unrounded = np.clip(np.rint(group.astype(np.float64) / np.float64(sc[0])), -127, 127).astype(int)
+        cases_recip += int(np.sum(recip != np.array(want)))
+        cases_unrounded += int(np.sum(unrounded != np.array(want)))
+    assert checked > 5000
+    # the construction has teeth: both plausible wrong quotient steps disagree somewhere
+    assert cases_recip > 0 and cases_unrounded > 0
+
+
 def test_dq_groups_of_256_and_ragged_tail():
     """Group boundaries at multiples of 256 constants; the last group shorter."""
     m = np.concatenate([np.full(256, 1.0), np.full(256, 2.0), np.array([3.0, 5.0])]).astype(np.float32)
