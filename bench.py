@@ -11,9 +11,11 @@ dominant kernel are reported beside it.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
-N > 1 runs under torch.distributed.run, one rank per GPU; every rank runs the
-same step on its own data (weak scaling, no data-path collective) and the
-time is the maximum over ranks.
+N > 1 runs under torch.distributed.run, one rank per GPU, as data-parallel
+training (weak scaling): every rank runs the step on its own 4096 training
+tokens per linear and the LoRA gradients of the backward are summed over the
+ranks in fp32 by one NCCL all-reduce per linear, on a side stream that overlaps
+the rank's dX GEMM; the time is the maximum over ranks.
 """
 from __future__ import annotations
 
@@ -155,10 +157,15 @@ class ClockSampler:
 # our arm
 
 class Workload:
-    """Device-resident inputs, outputs and workspaces of one step."""
+    """Device-resident inputs, outputs and workspaces of one step. With dp=True
+    (N > 1 ranks) every rank's backward is the data-parallel one: dA and dB in
+    fp32 in one flat buffer, summed over the ranks by an NCCL all-reduce on a side
+    stream while the rank's dX GEMM runs, then rounded once to bf16."""
 
-    def __init__(self, dev, seed):
+    def __init__(self, dev, seed, dp=False):
         self.dev = dev
+        self.dp = dp
+        self.side = torch.cuda.Stream(device=dev) if dp else None
         self.lin = []
         for li, (N, K) in enumerate(SHAPES):
             inp = syn.make_linear(N, K, M_TRAIN, r=R, alpha=ALPHA, seed=seed, workload="llama7b_train", layer=li)
@@ -173,6 +180,11 @@ class Workload:
             d["dX"] = torch.empty(M_TRAIN, K, dtype=torch.bfloat16, device=dev)
             d["dA"] = torch.empty(R, K, dtype=torch.bfloat16, device=dev)
             d["dB"] = torch.empty(N, R, dtype=torch.bfloat16, device=dev)
+            if dp:  # flat fp32 sums and their bf16 rounding: dA [R, K] then dB [N, R]
+                d["grads"] = torch.empty(R * K + N * R, dtype=torch.float32, device=dev)
+                d["grads_bf16"] = torch.empty(R * K + N * R, dtype=torch.bfloat16, device=dev)
+                d["ev"] = torch.cuda.Event()
+                d["ev"].record()  # creates the CUDA event
             self.lin.append(d)
         self.ws = torch.empty(self._ws_bytes(), dtype=torch.uint8, device=dev)
 
@@ -215,6 +227,28 @@ class Workload:
                                     ALPHA, qb._ptr(d["dY"]), qb._ptr(d["T"]), qb._ptr(d["dX"]), qb._ptr(d["dA"]),
                                     qb._ptr(d["dB"]), ws, ctypes.byref(n), st)
 
+    @staticmethod
+    def _bwd_dp_call(lib, d, ws, n, st, M):
+        import ctypes
+        qc = d["q"].as_c()
+        return lib.qlora_linear_bwd_dp(ctypes.byref(qc), qb._ptr(d["X"]), M, qb._ptr(d["A"]), qb._ptr(d["B"]), R,
+                                       ALPHA, qb._ptr(d["dY"]), qb._ptr(d["T"]), qb._ptr(d["dX"]),
+                                       qb._ptr(d["grads"]), ctypes.c_void_p(d["ev"].cuda_event), ws, ctypes.byref(n),
+                                       st)
+
+    def _exchange(self, lib, d):
+        """Sum the rank's flat fp32 LoRA gradients over all ranks on the side stream
+        (after the backward's event, overlapping its dX GEMM) and round them to bf16."""
+        import ctypes
+        main = torch.cuda.current_stream()
+        self.side.wait_event(d["ev"])
+        with torch.cuda.stream(self.side):
+            torch.distributed.all_reduce(d["grads"])
+            rc = lib.qlora_round_bf16(qb._ptr(d["grads"]), qb._ptr(d["grads_bf16"]), d["grads"].numel(),
+                                      ctypes.c_void_p(self.side.cuda_stream))
+        main.wait_stream(self.side)
+        return rc
+
     def step(self, ev=None, only=None):
         """One pass of the hot path. ev: optional dict part -> list of (start, end)
         events, recorded for the parts named in `only` (all parts if None)."""
@@ -243,11 +277,15 @@ class Workload:
             for M in M_DECODE:
                 rec(f"decode{M}/{li}", lambda: self._fwd_call(lib, d, ws, n, st, M))
             rec(f"train_fwd/{li}", lambda: self._fwd_call(lib, d, ws, n, st, M_TRAIN))
-            rec(f"train_bwd/{li}", lambda: self._bwd_call(lib, d, ws, n, st, M_TRAIN))
+            if self.dp:
+                rec(f"train_bwd/{li}", lambda: self._bwd_dp_call(lib, d, ws, n, st, M_TRAIN))
+                rec(f"exchange/{li}", lambda: self._exchange(lib, d))
+            else:
+                rec(f"train_bwd/{li}", lambda: self._bwd_call(lib, d, ws, n, st, M_TRAIN))
 
     def launches_per_step(self):
         per = LAUNCHES["quantize"] + LAUNCHES["dequantize"] + len(M_DECODE) * LAUNCHES["decode_fwd"] + \
-            LAUNCHES["train_fwd"] + LAUNCHES["train_bwd"]
+            LAUNCHES["train_fwd"] + LAUNCHES["train_bwd"] + (1 if self.dp else 0)  # + the bf16 rounding
         return per * len(self.lin)
 
 
@@ -264,7 +302,7 @@ def e2e_step(work: Workload, host):
     work.step()
     d2h = 0
     for d, h in zip(work.lin, host):
-        for k in ("dA", "dB"):
+        for k in (("grads_bf16",) if work.dp else ("dA", "dB")):  # the LoRA gradients of the step
             h["out_" + k].copy_(d[k], non_blocking=True)
             d2h += d[k].numel() * d[k].element_size()
         for M in M_DECODE:
@@ -431,6 +469,220 @@ def adamw_measure(dev, peaks, n=1 << 26, reps=10):
     return out
 
 
+def _timed_calls(calls, reps):
+    """Mean time per call (us) of `reps` calls cycling through `calls`, back to back."""
+    for c in calls[:3]:
+        c()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for i in range(reps):
+        rc = calls[i % len(calls)]()
+        if rc not in (0, None):
+            raise qb.QloraError(rc, "timed call")
+    b.record()
+    torch.cuda.synchronize()
+    return 1e3 * a.elapsed_time(b) / reps
+
+
+def measure_llama65b(dev, peaks, reps=12):
+    """Llama-65B linear shapes (8192x8192, 22016x8192, 8192x22016) with Student-t(4)
+    weights scaled to std 0.02: quantize + DQ and dequant GB/s, decode (M = 1)
+    weight GB/s, and forward + backward TFLOP/s at M = 2048 tokens. Each call back
+    to back, rotating copies of its inputs beyond twice the L2 where they fit in it."""
+    import ctypes
+    lib = qb.load_library()
+    st = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    l2 = getattr(torch.cuda.get_device_properties(dev), "L2_cache_size", 128 << 20)
+    M = 2048
+    out, fl_tot, us_tot = {}, 0.0, 0.0
+    for li, (N, K) in enumerate(syn.LLAMA65B_SHAPES):
+        base = 16 * li
+        W = syn.student_t_bf16_device((N, K), 4, 0.02, 0, "llama65b", base + 0, device=dev)
+        A = syn.normal_bf16_device((R, K), 0.02, 0, "llama65b", base + 1, device=dev)
+        B = syn.normal_bf16_device((N, R), 0.02, 0, "llama65b", base + 2, device=dev)
+        X = syn.normal_bf16_device((M, K), 1.0, 0, "llama65b", base + 3, device=dev)
+        dY = syn.normal_bf16_device((M, N), 0.01, 0, "llama65b", base + 4, device=dev)
+        q0 = qb.NF4Weight.empty(N, K, dev)
+        nq = max(2, math.ceil(2 * l2 / (0.515869 * N * K)))
+        qs = [q0] + [qb.NF4Weight.empty(N, K, dev) for _ in range(nq - 1)]
+        qcs = [q.as_c() for q in qs]
+        Wd = torch.empty(N, K, dtype=torch.bfloat16, device=dev)
+        Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+        T = torch.empty(M, R, dtype=torch.float32, device=dev)
+        dX = torch.empty(M, K, dtype=torch.bfloat16, device=dev)
+        dA = torch.empty(R, K, dtype=torch.bfloat16, device=dev)
+        dB = torch.empty(N, R, dtype=torch.bfloat16, device=dev)
+        Y1 = torch.empty(1, N, dtype=torch.bfloat16, device=dev)
+        X1 = X[:1].contiguous()
+        need = 0
+        for qc in qcs[:1]:
+            n = ctypes.c_size_t(0)
+            lib.qlora_quantize_nf4_dq(qb._ptr(W), ctypes.byref(qc), None, ctypes.byref(n), st)
+            need = max(need, n.value)
+            lib.qlora_linear_fwd(ctypes.byref(qc), qb._ptr(X), M, qb._ptr(A), qb._ptr(B), R, ALPHA, qb._ptr(Y),
+                                 qb._ptr(T), None, ctypes.byref(n), st)
+            need = max(need, n.value)
+            lib.qlora_linear_bwd(ctypes.byref(qc), qb._ptr(X), M, qb._ptr(A), qb._ptr(B), R, ALPHA, qb._ptr(dY),
+                                 qb._ptr(T), qb._ptr(dX), qb._ptr(dA), qb._ptr(dB), None, ctypes.byref(n), st)
+            need = max(need, n.value)
+            lib.qlora_linear_fwd(ctypes.byref(qc), qb._ptr(X1), 1, qb._ptr(A), qb._ptr(B), R, ALPHA, qb._ptr(Y1),
+                                 None, None, ctypes.byref(n), st)
+            need = max(need, n.value)
+        wsb = torch.empty(need, dtype=torch.uint8, device=dev)
+        ws, n = ctypes.c_void_p(wsb.data_ptr()), ctypes.c_size_t(need)
+        for qc in qcs:  # every copy holds the quantized weight
+            lib.qlora_quantize_nf4_dq(qb._ptr(W), ctypes.byref(qc), ws, ctypes.byref(n), st)
+        us_q = _timed_calls([lambda qc=qc: lib.qlora_quantize_nf4_dq(qb._ptr(W), ctypes.byref(qc), ws,
+                                                                      ctypes.byref(n), st) for qc in qcs], reps)
+        us_d = _timed_calls([lambda qc=qc: lib.qlora_dequantize_nf4_dq(ctypes.byref(qc), qb._ptr(Wd), st)
+                             for qc in qcs], reps)
+        us_dec = _timed_calls([lambda qc=qc: lib.qlora_linear_fwd(
+            ctypes.byref(qc), qb._ptr(X1), 1, qb._ptr(A), qb._ptr(B), R, ALPHA, qb._ptr(Y1), None, ws,
+            ctypes.byref(n), st) for qc in qcs], 3 * reps)
+        qc = qcs[0]
+        us_f = _timed_calls([lambda: lib.qlora_linear_fwd(ctypes.byref(qc), qb._ptr(X), M, qb._ptr(A), qb._ptr(B),
+                                                          R, ALPHA, qb._ptr(Y), qb._ptr(T), ws, ctypes.byref(n),
+                                                          st)], reps)
+        us_b = _timed_calls([lambda: lib.qlora_linear_bwd(ctypes.byref(qc), qb._ptr(X), M, qb._ptr(A), qb._ptr(B),
+                                                          R, ALPHA, qb._ptr(dY), qb._ptr(T), qb._ptr(dX),
+                                                          qb._ptr(dA), qb._ptr(dB), ws, ctypes.byref(n), st)], reps)
+        ff, fb = train_flops(N, K, M)
+        fl_tot += ff + fb
+        us_tot += us_f + us_b
+        key = f"{N}x{K}"
+        gq = quant_bytes(N, K) / us_q / 1e3
+        gd = quant_bytes(N, K) / us_d / 1e3
+        gw = weight_bytes(N, K) / us_dec / 1e3
+        out[f"quantize/{key}"] = {"us": round(us_q, 2), "GB_s": round(gq, 1), "hbm_frac": round(gq / peaks["hbm_gbs"], 4)}
+        out[f"dequantize/{key}"] = {"us": round(us_d, 2), "GB_s": round(gd, 1),
+                                    "hbm_frac": round(gd / peaks["hbm_gbs"], 4)}
+        out[f"decode1/{key}"] = {"us": round(us_dec, 2), "weight_GB_s": round(gw, 1),
+                                 "GB_s": round(decode_bytes(N, K, 1) / us_dec / 1e3, 1),
+                                 "hbm_frac": round(decode_bytes(N, K, 1) / us_dec / 1e3 / peaks["hbm_gbs"], 4)}
+        out[f"train_fwd/{key}"] = {"us": round(us_f, 2), "TFLOP_s": round(ff / us_f / 1e6, 1),
+                                   "tensor_frac": round(ff / us_f / 1e6 / peaks["bf16_tflops"], 4)}
+        out[f"train_bwd/{key}"] = {"us": round(us_b, 2), "TFLOP_s": round(fb / us_b / 1e6, 1),
+                                   "tensor_frac": round(fb / us_b / 1e6 / peaks["bf16_tflops"], 4)}
+        del W, A, B, X, dY, qs, qcs, Wd, Y, T, dX, dA, dB, wsb
+        torch.cuda.empty_cache()
+    err = qb.qlora_device_error()
+    return {"workload": "Llama-65B linear shapes, W ~ Student-t(4) scaled to std 0.02, r=64 alpha=16, "
+                        "train M=2048, decode M=1",
+            "train_fwd_bwd_TFLOP_s": round(fl_tot / us_tot / 1e6, 1),
+            "train_tensor_frac": round(fl_tot / us_tot / 1e6 / peaks["bf16_tflops"], 4),
+            "parts": out, "device_error": err}
+
+
+def measure_sweep65b(dev, peaks):
+    """The 80-layer Llama-65B sweep (560 linears, 64.76e9 weights ~ N(0, 0.02)
+    drawn on the device layer by layer): quantize + DQ of every linear into resident
+    NF4 storage (33.4 GB), then one dequant pass and one M = 1 decode pass over all
+    560 linears. Quantize time is the sum of per-layer event pairs around the seven
+    calls of a layer (the weight generation stays outside them)."""
+    import ctypes
+    lib = qb.load_library()
+    st = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    shapes = syn.LLAMA65B_LAYER
+    nlin = len(shapes)
+    layer_numel = sum(N * K for N, K in shapes)
+    wbuf = torch.empty(layer_numel, dtype=torch.bfloat16, device=dev)
+    offs, o = [], 0
+    for N, K in shapes:
+        offs.append(o)
+        o += N * K
+    need = 0
+    for N, K in shapes:  # workspace size queries (nothing is launched)
+        qq = qb.NF4Weight.empty(N, K, dev)
+        qc = qq.as_c()
+        n = ctypes.c_size_t(0)
+        X1 = torch.empty(1, K, dtype=torch.bfloat16, device=dev)
+        if lib.qlora_quantize_nf4_dq(qb._ptr(X1), ctypes.byref(qc), None, ctypes.byref(n), st) != 0:
+            raise qb.QloraError(1, "sweep workspace query")
+        need = max(need, n.value)
+        if lib.qlora_linear_fwd(ctypes.byref(qc), qb._ptr(X1), 1, qb._ptr(X1), qb._ptr(X1), R, ALPHA, qb._ptr(X1),
+                                None, None, ctypes.byref(n), st) != 0:
+            raise qb.QloraError(1, "sweep workspace query")
+        need = max(need, n.value)
+        del qq, X1
+    wsb = torch.empty(need, dtype=torch.uint8, device=dev)
+    ws, n = ctypes.c_void_p(wsb.data_ptr()), ctypes.c_size_t(need)
+    stor, qcs = [], []
+    us_q = 0.0
+    for layer in range(syn.LLAMA65B_LAYERS):
+        for j, (N, K) in enumerate(shapes):
+            syn.normal_bf16_device((N, K), 0.02, 0, "sweep65b", 16 * (nlin * layer + j), device=dev,
+                                   out=wbuf[offs[j]:offs[j] + N * K].view(N, K))
+        lq = [qb.NF4Weight.empty(N, K, dev) for N, K in shapes]
+        lc = [q.as_c() for q in lq]
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for j in range(nlin):
+            rc = lib.qlora_quantize_nf4_dq(qb._ptr(wbuf[offs[j]:]), ctypes.byref(lc[j]), ws, ctypes.byref(n), st)
+            if rc != 0:
+                raise qb.QloraError(rc, "sweep quantize")
+        b.record()
+        torch.cuda.synchronize()
+        us_q += 1e3 * a.elapsed_time(b)
+        stor.extend(lq)
+        qcs.extend(lc)
+    del wbuf
+    torch.cuda.empty_cache()
+    stored = sum(t.numel() * t.element_size() for q in stor for t in (q.packed, q.absmax_q, q.dq_scale, q.mean))
+    nmax = max(N * K for N, K in shapes)
+    dq_out = torch.empty(nmax, dtype=torch.bfloat16, device=dev)
+    A_l = [syn.normal_bf16_device((R, K), 0.02, 0, "sweep65b", 9000 + 4 * j, device=dev) for j, (N, K) in
+           enumerate(shapes)]
+    B_l = [syn.normal_bf16_device((N, R), 0.02, 0, "sweep65b", 9001 + 4 * j, device=dev) for j, (N, K) in
+           enumerate(shapes)]
+    X_l = [syn.normal_bf16_device((1, K), 1.0, 0, "sweep65b", 9002 + 4 * j, device=dev) for j, (N, K) in
+           enumerate(shapes)]
+    Y_l = [torch.empty(1, N, dtype=torch.bfloat16, device=dev) for N, K in shapes]
+
+    def dequant_all():
+        for i, qc in enumerate(qcs):
+            rc = lib.qlora_dequantize_nf4_dq(ctypes.byref(qc), qb._ptr(dq_out), st)
+            if rc != 0:
+                raise qb.QloraError(rc, "sweep dequant")
+
+    def decode_all():
+        for i, qc in enumerate(qcs):
+            j = i % nlin
+            rc = lib.qlora_linear_fwd(ctypes.byref(qc), qb._ptr(X_l[j]), 1, qb._ptr(A_l[j]), qb._ptr(B_l[j]), R,
+                                      ALPHA, qb._ptr(Y_l[j]), None, ws, ctypes.byref(n), st)
+            if rc != 0:
+                raise qb.QloraError(rc, "sweep decode")
+
+    res = {}
+    for name, fn in (("dequant_all", dequant_all), ("decode1_all", decode_all)):
+        fn()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        fn()
+        b.record()
+        torch.cuda.synchronize()
+        res[name] = 1e3 * a.elapsed_time(b)
+    err = qb.qlora_device_error()
+    nw = syn.LLAMA65B_LAYERS * layer_numel
+    lora_bytes = syn.LLAMA65B_LAYERS * sum(2 * R * (K + N) + 2 * (K + N) for N, K in shapes)
+    gq = 2.516 * nw / us_q / 1e3
+    gd = 2.516 * nw / res["dequant_all"] / 1e3
+    gw = stored / res["decode1_all"] / 1e3
+    gall = (stored + lora_bytes) / res["decode1_all"] / 1e3
+    out = {"workload": "80 layers x 7 Llama-65B linears (560), 64.76e9 weights ~ N(0, 0.02) drawn on the device; "
+                       "r=64 adapters per linear shape; decode M=1",
+           "weights": nw, "nf4_bytes": stored,
+           "quantize_all": {"ms": round(us_q / 1e3, 3), "GB_s": round(gq, 1), "hbm_frac": round(gq / peaks["hbm_gbs"], 4)},
+           "dequant_all": {"ms": round(res["dequant_all"] / 1e3, 3), "GB_s": round(gd, 1),
+                           "hbm_frac": round(gd / peaks["hbm_gbs"], 4)},
+           "decode1_all": {"ms": round(res["decode1_all"] / 1e3, 3), "weight_GB_s": round(gw, 1),
+                           "GB_s": round(gall, 1), "hbm_frac": round(gall / peaks["hbm_gbs"], 4)},
+           "device_error": err}
+    del stor, qcs, dq_out, A_l, B_l, X_l, Y_l, wsb
+    torch.cuda.empty_cache()
+    return out
+
+
 def run_ours(args, rank, world, dev):
     def say(msg):  # progress on stderr (stdout carries only the JSON line)
         if args.verbose or rank == 0:
@@ -438,7 +690,8 @@ def run_ours(args, rank, world, dev):
 
     peaks = load_peaks()
     say("allocating the workload")
-    work = Workload(dev, seed=rank)
+    dp = world > 1
+    work = Workload(dev, seed=rank, dp=dp)
     fl_train = sum(sum(train_flops(N, K)) for N, K in SHAPES)
 
     clocks = ClockSampler(gpu_index_for_smi(dev))
@@ -480,7 +733,7 @@ def run_ours(args, rank, world, dev):
     # the same step captured once into a CUDA graph (the library's launches keep
     # their programmatic-dependent-launch edges) and replayed K times
     ms_graph = None
-    if not args.no_graph:
+    if not args.no_graph and not dp:  # the data-parallel step (NCCL on a side stream) runs as stream launches
         say("timed region (CUDA graph replay)")
         graph = capture_step_graph(work, say)
         # every rank takes the same collective steps: replay only if all captured
@@ -550,6 +803,12 @@ def run_ours(args, rank, world, dev):
     merge = merge_measure(work, dev)
     say("paged AdamW")
     adamw = adamw_measure(dev, peaks)
+    llama65b = sweep = None
+    if not args.no_65b:
+        say("Llama-65B shapes (Student-t weights)")
+        llama65b = measure_llama65b(dev, peaks)
+        say("80-layer Llama-65B sweep")
+        sweep = measure_sweep65b(dev, peaks)
     say("end to end with host buffers")
     # end to end through the C ABI with host buffers
     host = []
@@ -557,8 +816,8 @@ def run_ours(args, rank, world, dev):
         h = {k: torch.empty_like(d[k], device="cpu").pin_memory() for k in ("W", "A", "B", "X", "dY")}
         for k in h:
             h[k].copy_(d[k])
-        h["out_dA"] = torch.empty_like(d["dA"], device="cpu").pin_memory()
-        h["out_dB"] = torch.empty_like(d["dB"], device="cpu").pin_memory()
+        for k in (("grads_bf16",) if work.dp else ("dA", "dB")):
+            h["out_" + k] = torch.empty_like(d[k], device="cpu").pin_memory()
         for M in M_DECODE:
             h[f"out_Y{M}"] = torch.empty_like(d["Ydec"][M], device="cpu").pin_memory()
         host.append(h)
@@ -584,7 +843,9 @@ def run_ours(args, rank, world, dev):
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded, per-rank seed)",
         "config": {"workload": "Llama-7B linear shapes 4096x4096, 11008x4096, 4096x11008; r=64 alpha=16; "
                                "quantize+DQ, dequant, decode M=1/4/16, train fwd+bwd M=4096",
-                   "global_batch_tokens": M_TRAIN * world, "parallelism": f"dp{world} (independent replicas)",
+                   "global_batch_tokens": M_TRAIN * world,
+                   "parallelism": (f"dp{world} (token shards of {M_TRAIN} per rank; fp32 LoRA gradients all-reduced "
+                                   "over NCCL on a side stream, overlapping the dX GEMM)") if dp else "dp1 (one GPU)",
                    "l2": "inputs larger than L2 (each step touches ~1.2 GB)",
                    "parts": "each call back to back over rotating input copies > 2x L2, outside the timed region"},
         "decode_weight_GB_s": {"min": min(dec), "max": max(dec)},
@@ -593,6 +854,8 @@ def run_ours(args, rank, world, dev):
         "roofline": roof,
         "merge": merge,
         "adamw": adamw,
+        "llama65b": llama65b,
+        "sweep65b": sweep,
         "e2e": {"value": round(world * fl_train / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
                 "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": work.launches_per_step() * args.steps,
@@ -728,6 +991,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--verbose", action="store_true", help="print progress to stderr")
     ap.add_argument("--no-graph", action="store_true", help="time stream launches only (no CUDA graph replay)")
+    ap.add_argument("--no-65b", action="store_true", help="skip the Llama-65B shape and 80-layer sweep measurements")
     ap.add_argument("--profile-case", action="store_true",
                     help="run one call of each entry point on 11008x4096 (for ncu) and exit")
     args = ap.parse_args()

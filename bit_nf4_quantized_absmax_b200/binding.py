@@ -24,7 +24,8 @@ EXPORTED = ("qlora_status_string", "qlora_nf4_codebook", "qlora_nf4_storage_byte
             "qlora_quantize_nf4", "qlora_quantize_nf4_dq", "qlora_quantize_nf4_dq_noalloc",
             "qlora_quantize_nf4_dq_shard_begin", "qlora_quantize_nf4_dq_shard_end", "qlora_dequantize_nf4",
             "qlora_dequantize_nf4_dq", "qlora_linear_fwd", "qlora_linear_bwd", "qlora_linear_bwd_f32",
-            "qlora_linear_bwd_dp", "qlora_round_bf16", "qlora_merge_lora",
+            "qlora_linear_bwd_dp", "qlora_round_bf16", "qlora_merge_lora", "qlora_codebook", "qlora_quantize_4bit",
+            "qlora_dequantize_4bit",
             "qlora_paged_alloc", "qlora_paged_free", "qlora_paged_prefetch", "qlora_adamw_step",
             "qlora_device_error")
 
@@ -78,6 +79,9 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
     lib.qlora_linear_bwd_f32.argtypes = [wp, vp, i64, vp, vp, i32, f32, vp, vp, vp, vp, vp, vp, szp, vp]
     lib.qlora_linear_bwd_dp.argtypes = [wp, vp, i64, vp, vp, i32, f32, vp, vp, vp, vp, vp, vp, szp, vp]
     lib.qlora_round_bf16.argtypes = [vp, vp, i64, vp]
+    lib.qlora_codebook.argtypes = [ctypes.c_int, ctypes.POINTER(ctypes.c_float)]
+    lib.qlora_quantize_4bit.argtypes = [vp, wp, ctypes.c_int, vp, szp, vp]
+    lib.qlora_dequantize_4bit.argtypes = [wp, ctypes.c_int, vp, vp]
     lib.qlora_merge_lora.argtypes = [wp, ctypes.POINTER(_Adapter), i32, vp, vp]
     lib.qlora_device_error.argtypes = [ctypes.POINTER(ctypes.c_int32), vp]
     lib.qlora_paged_alloc.argtypes = [sz, i32, ctypes.POINTER(vp)]
@@ -155,6 +159,43 @@ def qlora_nf4_codebook() -> torch.Tensor:
     out = (ctypes.c_float * 16)()
     _check(load_library().qlora_nf4_codebook(out), "qlora_nf4_codebook")
     return torch.tensor(list(out), dtype=torch.float32)
+
+
+DTYPE_NF4, DTYPE_FP4 = 0, 1
+
+
+def qlora_codebook(dtype: int = DTYPE_NF4) -> torch.Tensor:
+    """The 16 values of a 4-bit data type (DTYPE_NF4 or DTYPE_FP4), ascending."""
+    out = (ctypes.c_float * 16)()
+    _check(load_library().qlora_codebook(dtype, out), "qlora_codebook")
+    return torch.tensor(list(out), dtype=torch.float32)
+
+
+def qlora_quantize_4bit(W: torch.Tensor, dtype: int, double_quant: bool = True, out=None,
+                        workspace: torch.Tensor | None = None, stream=None):
+    """Quantize with the codebook of `dtype`; double-quantized (NF4Weight) or
+    single-level (SingleNF4Weight) storage."""
+    assert W.dtype == torch.bfloat16 and W.dim() == 2 and W.is_contiguous()
+    lib = load_library()
+    if out is None:
+        out = (NF4Weight if double_quant else SingleNF4Weight).empty(W.shape[0], W.shape[1], W.device)
+    qc = out.as_c()
+    st = _stream(stream)
+    ws, nbytes = _workspace(lambda p, n: lib.qlora_quantize_4bit(_ptr(W), ctypes.byref(qc), dtype, p, n, st),
+                            workspace, W.device)
+    _check(lib.qlora_quantize_4bit(_ptr(W), ctypes.byref(qc), dtype, _ptr(ws), ctypes.byref(nbytes), st),
+           "qlora_quantize_4bit")
+    return out
+
+
+def qlora_dequantize_4bit(q, dtype: int, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Dequantize either storage kind with the codebook of `dtype` to bf16."""
+    if out is None:
+        out = torch.empty(q.rows, q.cols, dtype=torch.bfloat16, device=q.packed.device)
+    qc = q.as_c()
+    _check(load_library().qlora_dequantize_4bit(ctypes.byref(qc), dtype, _ptr(out), _stream(stream)),
+           "qlora_dequantize_4bit")
+    return out
 
 
 def qlora_nf4_storage_bytes(rows: int, cols: int) -> tuple:

@@ -3,6 +3,7 @@
 // qlora_device_error, which reads the device error word.
 #include "qlora.h"
 
+#include <cstdlib>
 #include <cstring>
 
 #include "common.cuh"
@@ -97,6 +98,16 @@ qlora_status check_linear(const void* X, int64_t M, const void* A, const void* B
 }
 
 float lora_scale(float alpha, int32_t r) { return alpha / static_cast<float>(r); }
+
+// QLORA_DECODE_RES=0 in the environment selects the TMA-ring decode kernel for
+// every shape instead of the X-resident one where it fits (for comparisons).
+bool res_disabled() {
+  static const bool off = [] {
+    const char* e = std::getenv("QLORA_DECODE_RES");
+    return e && e[0] == '0';
+  }();
+  return off;
+}
 
 int32_t* device_error_word() {
   void* p = nullptr;
@@ -218,6 +229,55 @@ qlora_status linear_bwd_impl(const qlora_nf4_weight* q, const void* X, int64_t M
   return cuda_status(e);
 }
 
+int dtype_index(qlora_dtype d) { return d == QLORA_DTYPE_FP4 ? kDtypeFp4 : kDtypeNf4; }
+
+qlora_status quantize_single_impl(const void* W_bf16, const qlora_nf4_weight* q, int dtype, qlora_stream_t stream) {
+  qlora_status st = check_weight(q, false, 2);
+  if (st != QLORA_OK) return st;
+  if (!W_bf16 && q->rows > 0) return QLORA_ERR_INVALID_ARG;
+  if (W_bf16 && !aligned(W_bf16, 16)) return QLORA_ERR_ALIGNMENT;
+  const int64_t numel = q->rows * q->cols;
+  if (numel == 0) return QLORA_OK;
+  DeviceInfo di;
+  if ((st = device_info(&di)) != QLORA_OK) return st;
+  return cuda_status(launch_quantize_single(W_bf16, numel, q->packed, q->absmax, di.num_sms,
+                                            reinterpret_cast<cudaStream_t>(stream), dtype));
+}
+
+qlora_status quantize_dq_impl(const void* W_bf16, const qlora_nf4_weight* q, int dtype, void* workspace,
+                              size_t* workspace_bytes, qlora_stream_t stream) {
+  qlora_status st = check_weight(q, false, 1);
+  if (st != QLORA_OK) return st;
+  if (!W_bf16 && q->rows > 0) return QLORA_ERR_INVALID_ARG;
+  if (W_bf16 && !aligned(W_bf16, 16)) return QLORA_ERR_ALIGNMENT;
+  const int64_t numel = q->rows * q->cols;
+  const int64_t nblk = numel / 64;
+  const size_t off_absmax = align_up(kQuantScratchBytes);
+  const size_t need = off_absmax + align_up(static_cast<size_t>(nblk) * sizeof(float));
+  bool launch = false;
+  st = workspace_check(workspace, workspace_bytes, need, &launch);
+  if (st != QLORA_OK || !launch || numel == 0) return st;
+  DeviceInfo di;
+  if ((st = device_info(&di)) != QLORA_OK) return st;
+  char* ws = static_cast<char*>(workspace);
+  return cuda_status(launch_quantize(W_bf16, numel, q->packed, q->absmax_q, q->dq_scale, q->mean,
+                                     reinterpret_cast<float*>(ws + off_absmax), ws, di.num_sms,
+                                     reinterpret_cast<cudaStream_t>(stream), dtype));
+}
+
+qlora_status dequantize_impl(const qlora_nf4_weight* q, int dtype, void* out_bf16, qlora_stream_t stream) {
+  qlora_status st = check_weight(q, false);
+  if (st != QLORA_OK) return st;
+  const int64_t numel = q->rows * q->cols;
+  if (numel == 0) return QLORA_OK;
+  if (!out_bf16) return QLORA_ERR_INVALID_ARG;
+  if (!aligned(out_bf16, 16)) return QLORA_ERR_ALIGNMENT;
+  DeviceInfo di;
+  if ((st = device_info(&di)) != QLORA_OK) return st;
+  return cuda_status(launch_dequantize(view(q), out_bf16, quant_tables(dtype).codebook, di.num_sms,
+                                       reinterpret_cast<cudaStream_t>(stream)));
+}
+
 }  // namespace
 
 
@@ -264,51 +324,45 @@ qlora_status qlora_nf4_single_storage_bytes(int64_t rows, int64_t cols, size_t o
 }
 
 qlora_status qlora_quantize_nf4(const void* W_bf16, const qlora_nf4_weight* q, qlora_stream_t stream) {
-  qlora_status st = check_weight(q, false, 2);
-  if (st != QLORA_OK) return st;
-  if (!W_bf16 && q->rows > 0) return QLORA_ERR_INVALID_ARG;
-  if (W_bf16 && !aligned(W_bf16, 16)) return QLORA_ERR_ALIGNMENT;
-  const int64_t numel = q->rows * q->cols;
-  if (numel == 0) return QLORA_OK;
-  DeviceInfo di;
-  if ((st = device_info(&di)) != QLORA_OK) return st;
-  return cuda_status(launch_quantize_single(W_bf16, numel, q->packed, q->absmax, di.num_sms,
-                                            reinterpret_cast<cudaStream_t>(stream)));
+  return quantize_single_impl(W_bf16, q, kDtypeNf4, stream);
 }
 
 qlora_status qlora_quantize_nf4_dq(const void* W_bf16, const qlora_nf4_weight* q, void* workspace,
                                    size_t* workspace_bytes, qlora_stream_t stream) {
-  qlora_status st = check_weight(q, false, 1);
-  if (st != QLORA_OK) return st;
-  if (!W_bf16 && q->rows > 0) return QLORA_ERR_INVALID_ARG;
-  if (W_bf16 && !aligned(W_bf16, 16)) return QLORA_ERR_ALIGNMENT;
-  const int64_t numel = q->rows * q->cols;
-  const int64_t nblk = numel / 64;
-  const size_t off_absmax = align_up(kQuantScratchBytes);
-  const size_t need = off_absmax + align_up(static_cast<size_t>(nblk) * sizeof(float));
-  bool launch = false;
-  st = workspace_check(workspace, workspace_bytes, need, &launch);
-  if (st != QLORA_OK || !launch || numel == 0) return st;
-  DeviceInfo di;
-  if ((st = device_info(&di)) != QLORA_OK) return st;
-  char* ws = static_cast<char*>(workspace);
-  return cuda_status(launch_quantize(W_bf16, numel, q->packed, q->absmax_q, q->dq_scale, q->mean,
-                                     reinterpret_cast<float*>(ws + off_absmax),
-                                     ws, di.num_sms,
-                                     reinterpret_cast<cudaStream_t>(stream)));
+  return quantize_dq_impl(W_bf16, q, kDtypeNf4, workspace, workspace_bytes, stream);
 }
 
 qlora_status qlora_dequantize_nf4(const qlora_nf4_weight* q, void* out_bf16, qlora_stream_t stream) {
-  qlora_status st = check_weight(q, false);
-  if (st != QLORA_OK) return st;
-  const int64_t numel = q->rows * q->cols;
-  if (numel == 0) return QLORA_OK;
-  if (!out_bf16) return QLORA_ERR_INVALID_ARG;
-  if (!aligned(out_bf16, 16)) return QLORA_ERR_ALIGNMENT;
-  DeviceInfo di;
-  if ((st = device_info(&di)) != QLORA_OK) return st;
-  return cuda_status(launch_dequantize(view(q), out_bf16, quant_tables().codebook, di.num_sms,
-                                       reinterpret_cast<cudaStream_t>(stream)));
+  return dequantize_impl(q, kDtypeNf4, out_bf16, stream);
+}
+
+qlora_status qlora_codebook(qlora_dtype dtype, float out16[16]) {
+  if (!out16) return QLORA_ERR_INVALID_ARG;
+  if (dtype != QLORA_DTYPE_NF4 && dtype != QLORA_DTYPE_FP4) return QLORA_ERR_UNSUPPORTED;
+  std::memcpy(out16, quant_tables(dtype_index(dtype)).codebook, sizeof(float) * 16);
+  return QLORA_OK;
+}
+
+qlora_status qlora_quantize_4bit(const void* W_bf16, const qlora_nf4_weight* q, qlora_dtype dtype, void* workspace,
+                                 size_t* workspace_bytes, qlora_stream_t stream) {
+  if (dtype != QLORA_DTYPE_NF4 && dtype != QLORA_DTYPE_FP4) return QLORA_ERR_UNSUPPORTED;
+  if (!q) return QLORA_ERR_INVALID_ARG;
+  if (q->dq_blocksize == 0) {  // single level: no workspace
+    if (!workspace_bytes) return QLORA_ERR_INVALID_ARG;
+    if (!workspace) {
+      *workspace_bytes = kAlign;
+      qlora_status st = check_weight(q, false, 2);
+      return st;
+    }
+    return quantize_single_impl(W_bf16, q, dtype_index(dtype), stream);
+  }
+  return quantize_dq_impl(W_bf16, q, dtype_index(dtype), workspace, workspace_bytes, stream);
+}
+
+qlora_status qlora_dequantize_4bit(const qlora_nf4_weight* q, qlora_dtype dtype, void* out_bf16,
+                                   qlora_stream_t stream) {
+  if (dtype != QLORA_DTYPE_NF4 && dtype != QLORA_DTYPE_FP4) return QLORA_ERR_UNSUPPORTED;
+  return dequantize_impl(q, dtype_index(dtype), out_bf16, stream);
 }
 
 qlora_status qlora_dequantize_nf4_dq(const qlora_nf4_weight* q, void* out_bf16, qlora_stream_t stream) {
@@ -331,11 +385,14 @@ qlora_status qlora_linear_fwd(const qlora_nf4_weight* q, const void* X, int64_t 
   Layout L;
   size_t off_T = 0, off_part = 0, off_cnt = 0, off_wd = 0, off_sT = 0;
   DecodePlan dplan{};
+  ResPlan rplan{};
   if (decode) {
     dplan = decode_plan(M, N, K, kRefSms);
+    rplan = M > 0 && !res_disabled() ? res_plan(M, N, K, kRefSms) : ResPlan{};
     off_T = L.add(T_save ? 0 : static_cast<size_t>(M) * r * sizeof(float));
-    off_part = L.add(decode_partial_elems(dplan) * sizeof(float));
-    off_cnt = L.add(decode_counter_words(dplan) * sizeof(unsigned int));
+    off_part = L.add((rplan.ok ? res_partial_elems(rplan) : decode_partial_elems(dplan)) * sizeof(float));
+    off_cnt = L.add((rplan.ok ? static_cast<size_t>(rplan.n_tiles) : decode_counter_words(dplan)) *
+                    sizeof(unsigned int));
   } else {
     off_wd = L.add(static_cast<size_t>(N) * K * 2);
     off_sT = L.add(static_cast<size_t>(M) * rpad * 2);
@@ -352,7 +409,7 @@ qlora_status qlora_linear_fwd(const qlora_nf4_weight* q, const void* X, int64_t 
   if (decode) {
     float* T = T_save ? T_save : reinterpret_cast<float*>(ws + off_T);
     return cuda_status(launch_decode_fwd(view(q), X, M, A, B, r, s, Y, T, reinterpret_cast<float*>(ws + off_part),
-                                         reinterpret_cast<unsigned int*>(ws + off_cnt), dplan, cb, err, cs));
+                                         reinterpret_cast<unsigned int*>(ws + off_cnt), dplan, rplan, cb, err, cs));
   }
   void* Wd = ws + off_wd;
   void* sT = ws + off_sT;

@@ -380,12 +380,14 @@ k_decode(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUten
 
 // T[m, j] = sum_k X[m, k] A[j, k] for M <= 16 (fp32 on CUDA cores), one CTA per
 // adapter row j, 16-byte loads (8 k per thread and step). Block 0 also clears
-// the decode kernel's ticket counters.
+// the decode kernel's ticket counters. Small CTAs (128 threads, at most 64
+// registers each) so that one fits on an SM beside a CTA of either decode kernel.
+constexpr int kLoraDownThreads = 128;
 template <int MT>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(kLoraDownThreads, 8)
 k_lora_t_small(const __nv_bfloat16* __restrict__ X, const __nv_bfloat16* __restrict__ A, int M, int64_t K, int r,
                float* __restrict__ T, unsigned int* __restrict__ counters, int64_t n_counters) {
-  __shared__ float red[8][8 * MT];
+  __shared__ float red[kLoraDownThreads / 32][8 * MT];
   pdl_enter();  // after this, the decode kernel may start its main loop
   const int j = blockIdx.x;
   if (j == 0)
@@ -427,7 +429,7 @@ k_lora_t_small(const __nv_bfloat16* __restrict__ X, const __nv_bfloat16* __restr
   if (threadIdx.x < M) {
     float v = 0.0f;
 #pragma unroll
-    for (int w = 0; w < 8; ++w) v += red[w][threadIdx.x];
+    for (int w = 0; w < kLoraDownThreads / 32; ++w) v += red[w][threadIdx.x];
     T[static_cast<int64_t>(threadIdx.x) * r + j] = v;
   }
 }
@@ -481,7 +483,15 @@ bool encode_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_
 
 cudaError_t launch_decode_fwd(const Nf4View& w, const void* X, int64_t M, const void* A, const void* B, int r,
                               float s, void* Y, float* T, float* partial, unsigned int* counters,
-                              const DecodePlan& p, const float codebook[16], int32_t* err, cudaStream_t stream) {
+                              const DecodePlan& p, const ResPlan& rp, const float codebook[16], int32_t* err,
+                              cudaStream_t stream) {
+  if (rp.ok) {  // token values resident in shared memory (decode_res.cu)
+    cudaError_t e = launch_pdl(rp.mt == 1 ? k_lora_t_small<1> : k_lora_t_small<2>, dim3(r), dim3(kLoraDownThreads), 0, stream,
+                               reinterpret_cast<const __nv_bfloat16*>(X), reinterpret_cast<const __nv_bfloat16*>(A),
+                               static_cast<int>(M), w.K, r, T, counters, rp.n_tiles);
+    if (e != cudaSuccess) return e;
+    return launch_decode_res_main(w, X, M, B, r, s, Y, T, partial, counters, rp, codebook, err, stream);
+  }
   if (w.N >= (int64_t(1) << 31) || w.K >= (int64_t(1) << 31)) return cudaErrorInvalidValue;  // TMA coordinates
   Nf4Codebook cb;
   for (int i = 0; i < 16; ++i) cb.c[i] = codebook[i];
@@ -493,7 +503,7 @@ cudaError_t launch_decode_fwd(const Nf4View& w, const void* X, int64_t M, const 
       !encode_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, static_cast<uint64_t>(w.K), static_cast<uint64_t>(M),
                  static_cast<uint64_t>(w.K) * 2, 64u, 8u * p.mt))
     return cudaErrorInvalidValue;
-  cudaError_t e = launch_pdl(p.mt == 1 ? k_lora_t_small<1> : k_lora_t_small<2>, dim3(r), dim3(256), 0, stream,
+  cudaError_t e = launch_pdl(p.mt == 1 ? k_lora_t_small<1> : k_lora_t_small<2>, dim3(r), dim3(kLoraDownThreads), 0, stream,
                              reinterpret_cast<const __nv_bfloat16*>(X), reinterpret_cast<const __nv_bfloat16*>(A),
                              static_cast<int>(M), w.K, r, T, counters, p.row_tiles);
   if (e != cudaSuccess) return e;

@@ -1,0 +1,552 @@
+// Decode-shaped QLoRA forward (M <= 16 tokens) with the token values resident
+// in shared memory ("QLoRA vs ChatGPT", capability 5: the frozen weight is
+// dequantized on the fly, block by block; capability 2: the LoRA term beside
+// it).
+//
+// Y[M, N] = X W'^T + s T B^T, T = X A^T from the LoRA-down kernel that runs
+// first (k_lora_t_small in decode.cu).
+//
+// Used when X (M x K bf16, padded) fits in shared memory beside the reduction
+// slots: every M = 1 shape, and M <= 16 up to K of about 4096. Otherwise the
+// TMA-ring kernel of decode.cu runs.
+//
+// Work items are (16-row tile, 256-wide K superblock) pairs in tile-major
+// order, and every warp of the grid takes one contiguous, equally sized range
+// of them, so all warps decode the same number of weights. Since only the
+// packed codes stream from memory (X was copied to shared memory once per CTA),
+// item ranges need not be shared by the warps of a CTA, and most tiles lie
+// within the consecutive warps of one CTA: their pieces are summed through
+// shared memory. Only the tiles that straddle two CTAs go through global slots
+// and a ticket counter. The last warp of each CTA walks its range backwards, so
+// that the pieces of both straddling tiles of a CTA are the first work of the
+// warps that hold them.
+//
+// Within an item the weight is the A operand of mma.sync m16n8k16 (16 rows x 16
+// k, bf16 in, fp32 accumulate) and the tokens are its N dimension. Lane (g, t)
+// supplies k-slots {2t, 2t+1, 2t+8, 2t+9} of each MMA from the 64 consecutive
+// weights of block 4 sb + t of rows g and g + 8 and the matching token values
+// (the reduction index is permuted, X alike), so each lane decodes whole
+// 64-weight blocks with one 16-entry bf16 table per block, bit-identical to the
+// standalone dequant. A lane loads its two blocks' codes (2 x 32 bytes) with
+// plain global loads one item ahead, and prefetches the item after that into
+// L2.
+//
+// Every sum runs in an order fixed by the shapes (pieces in warp order within a
+// CTA, then CTAs in order), so repeated calls give identical bits.
+#include "common.cuh"
+#include "kernels.h"
+#include "nf4_lut.cuh"
+
+namespace qlora {
+namespace {
+
+constexpr int kResWarps = 16;                 // consumer warps per CTA (one CTA per SM)
+constexpr int kXBlockBytes = 64 * 2 + 16;     // one 64-k block of one token, padded for bank spread
+// Registers per thread: 16 warps x 96 leaves a quarter of the SM's registers
+// free, so that a CTA of the LoRA-down kernel that precedes this one fits beside
+// a CTA of this one.
+constexpr int kResRegs = 112;
+
+__device__ __forceinline__ void mma16816r(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                          uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ void lookup4(const Nf4Lut& L, uint32_t s, uint32_t sel, uint32_t& o01, uint32_t& o23) {
+  const uint32_t lo = prmt(prmt(L.lo[0], L.lo[1], s), prmt(L.lo[2], L.lo[3], s), sel);
+  const uint32_t hi = prmt(prmt(L.hi[0], L.hi[1], s), prmt(L.hi[2], L.hi[3], s), sel);
+  o01 = prmt(lo, hi, 0x5140);
+  o23 = prmt(lo, hi, 0x7362);
+}
+
+__device__ __forceinline__ uint4 lds128r(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+  return v;
+}
+
+__device__ __forceinline__ uint4 ldg_stream(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+__device__ __forceinline__ void prefetch_l2(const void* p) { asm volatile("prefetch.global.L2 [%0];" ::"l"(p)); }
+
+__device__ __forceinline__ unsigned int atom_add_acq_rel_cta_shared(uint32_t addr, unsigned int v) {
+  unsigned int old;
+  asm volatile("atom.acq_rel.cta.shared::cta.add.u32 %0, [%1], %2;" : "=r"(old) : "r"(addr), "r"(v) : "memory");
+  return old;
+}
+
+__device__ __forceinline__ unsigned int atom_add_acq_rel_gpu_r(unsigned int* p, unsigned int v) {
+  unsigned int old;
+  asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+
+// Owner unit of item i when n_items items are cut into n_units ranges
+// [u * n_items / n_units, (u + 1) * n_items / n_units).
+__host__ __device__ __forceinline__ int64_t owner_of(int64_t i, int64_t n_items, int64_t n_units) {
+  return ((i + 1) * n_units - 1) / n_items;
+}
+__host__ __device__ __forceinline__ int64_t range_begin(int64_t u, int64_t n_items, int64_t n_units) {
+  return u * n_items / n_units;
+}
+
+struct ResParams {
+  const uint8_t* packed;
+  const int8_t* q;
+  const float* dqs;
+  const float* mean;
+  const float* absmax;
+  const __nv_bfloat16* X;
+  const float* T;
+  const __nv_bfloat16* Bl;
+  __nv_bfloat16* Y;
+  float* gpart;            // [n_tiles][max_cta_seg][32 lanes][4 MT] fp32
+  unsigned int* gcnt;      // [n_tiles], zeroed by the LoRA-down kernel
+  int64_t N, K;
+  int64_t n_items, n_units;
+  int M, r;
+  float s;
+  int x_stride;            // bytes per token row of the shared X copy
+  int p_max;               // reduction slots per warp
+  int cta_tiles;           // CTA-local tile counters per CTA
+  int max_cta_seg;         // most CTAs holding pieces of one tile
+  int32_t* err;
+};
+
+// Shared memory: X [M][x_stride] | slots [kResWarps][p_max][32][4 MT] fp32 | counters [cta_tiles] u32
+__host__ __device__ inline size_t res_slot_off(const ResParams& p) {
+  return (static_cast<size_t>(p.M) * p.x_stride + 15) / 16 * 16;
+}
+
+template <int MT>
+__device__ __forceinline__ void lora_up_store(const float (&y)[MT][4], int64_t tile, int lane, const ResParams& p) {
+  const int g = lane >> 2, t = lane & 3;
+  const int64_t na = tile * 16 + g, nb = na + 8;
+  const int r = p.r;
+  float l[MT][4];
+#pragma unroll
+  for (int m = 0; m < MT; ++m) l[m][0] = l[m][1] = l[m][2] = l[m][3] = 0.0f;
+  // LoRA up: rows of B are the A operand, T^T (split into bf16 hi + lo) the B
+  // operand. A step covers ranks j0 .. j0 + 15; since r % 8 == 0 its upper half
+  // is either wholly inside [0, r) or wholly outside (and then zero).
+  for (int j0 = 0; j0 < r; j0 += 16) {
+    const bool hi_in = j0 + 8 < r;
+    const __nv_bfloat16* Ba = p.Bl + na * r + j0 + 2 * t;
+    const __nv_bfloat16* Bb = p.Bl + nb * r + j0 + 2 * t;
+    const uint32_t b_a0 = na < p.N ? *reinterpret_cast<const uint32_t*>(Ba) : 0u;
+    const uint32_t b_a2 = na < p.N && hi_in ? *reinterpret_cast<const uint32_t*>(Ba + 8) : 0u;
+    const uint32_t b_a1 = nb < p.N ? *reinterpret_cast<const uint32_t*>(Bb) : 0u;
+    const uint32_t b_a3 = nb < p.N && hi_in ? *reinterpret_cast<const uint32_t*>(Bb + 8) : 0u;
+#pragma unroll
+    for (int m = 0; m < MT; ++m) {
+      const int tok = g + 8 * m;
+      float tv[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+      if (tok < p.M) {
+        const float* tp = p.T + static_cast<int64_t>(tok) * r + j0 + 2 * t;
+        tv[0] = __ldcg(tp);
+        tv[1] = __ldcg(tp + 1);
+        if (hi_in) {
+          tv[2] = __ldcg(tp + 8);
+          tv[3] = __ldcg(tp + 9);
+        }
+      }
+      uint32_t hi[2], lo[2];
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        const uint32_t h = pack_bf16x2(tv[2 * q], tv[2 * q + 1]);
+        hi[q] = h;
+        lo[q] = pack_bf16x2(tv[2 * q] - bf16lo_to_f32(h), tv[2 * q + 1] - bf16hi_to_f32(h));
+      }
+      mma16816r(l[m], b_a0, b_a1, b_a2, b_a3, hi[0], hi[1]);
+      mma16816r(l[m], b_a0, b_a1, b_a2, b_a3, lo[0], lo[1]);
+    }
+  }
+#pragma unroll
+  for (int m = 0; m < MT; ++m) {
+    const int tok0 = 8 * m + 2 * t, tok1 = tok0 + 1;
+    if (na < p.N) {
+      if (tok0 < p.M) p.Y[static_cast<int64_t>(tok0) * p.N + na] = __float2bfloat16_rn(fmaf(p.s, l[m][0], y[m][0]));
+      if (tok1 < p.M) p.Y[static_cast<int64_t>(tok1) * p.N + na] = __float2bfloat16_rn(fmaf(p.s, l[m][1], y[m][1]));
+    }
+    if (nb < p.N) {
+      if (tok0 < p.M) p.Y[static_cast<int64_t>(tok0) * p.N + nb] = __float2bfloat16_rn(fmaf(p.s, l[m][2], y[m][2]));
+      if (tok1 < p.M) p.Y[static_cast<int64_t>(tok1) * p.N + nb] = __float2bfloat16_rn(fmaf(p.s, l[m][3], y[m][3]));
+    }
+  }
+}
+
+// A warp has finished its piece of tile `tile`. Store the piece in the warp's
+// shared slot; the last of the CTA's warps holding pieces of the tile sums them
+// in warp order. A tile that other CTAs hold pieces of too goes on through a
+// global slot and ticket; the CTA that brings the last piece sums the CTAs'
+// pieces in CTA order. Whoever completes the tile adds the LoRA term and writes Y.
+template <int MT>
+__device__ __forceinline__ void publish(const float (&acc)[2][MT][4], int64_t tile, int lane, int warp,
+                                        float* slots, uint32_t cnt_base, const ResParams& p) {
+  const int64_t nsb = (p.K / 64 + 3) / 4;
+  const int64_t cta = blockIdx.x;
+  const int64_t gw = cta * kResWarps + warp;
+  const int64_t wf = owner_of(tile * nsb, p.n_items, p.n_units);
+  const int64_t wl = owner_of(tile * nsb + nsb - 1, p.n_items, p.n_units);
+  const int64_t lw0 = (wf > cta * kResWarps ? wf : cta * kResWarps);
+  const int64_t lw1 = (wl < cta * kResWarps + kResWarps - 1 ? wl : cta * kResWarps + kResWarps - 1);  // wl < n_units
+  const int n_local = static_cast<int>(lw1 - lw0 + 1);
+  constexpr int kSlot = 32 * 4 * MT;  // floats per warp slot
+  // this warp's slot for the tile: index = tile - first tile of the warp's range
+  const int64_t my_first_tile = range_begin(gw, p.n_items, p.n_units) / nsb;
+  float* my_slot = slots + (static_cast<int64_t>(warp) * p.p_max + (tile - my_first_tile)) * kSlot;
+  float y[MT][4];
+#pragma unroll
+  for (int m = 0; m < MT; ++m) {
+    y[m][0] = acc[0][m][0] + acc[1][m][0];
+    y[m][1] = acc[0][m][1] + acc[1][m][1];
+    y[m][2] = acc[0][m][2] + acc[1][m][2];
+    y[m][3] = acc[0][m][3] + acc[1][m][3];
+  }
+  if (n_local > 1) {
+#pragma unroll
+    for (int m = 0; m < MT; ++m)
+      reinterpret_cast<float4*>(my_slot + lane * 4 * MT)[m] = make_float4(y[m][0], y[m][1], y[m][2], y[m][3]);
+    __syncwarp();  // the lanes' slot stores are ordered before lane 0's release below
+    const int64_t cta_first_tile = range_begin(cta * kResWarps, p.n_items, p.n_units) / nsb;
+    unsigned int old = 0;
+    if (lane == 0)
+      old = atom_add_acq_rel_cta_shared(cnt_base + static_cast<uint32_t>(tile - cta_first_tile) * 4u, 1u);
+    old = __shfl_sync(0xffffffffu, old, 0);
+    if (old != static_cast<unsigned int>(n_local - 1)) return;  // another warp of the CTA finishes the tile
+    __syncwarp();  // lane 0's acquire is ordered before every lane's reads of the slots
+#pragma unroll
+    for (int m = 0; m < MT; ++m) y[m][0] = y[m][1] = y[m][2] = y[m][3] = 0.0f;
+    for (int64_t w = lw0; w <= lw1; ++w) {  // warp order
+      const int64_t wt = range_begin(w, p.n_items, p.n_units) / nsb;
+      const float* sl = slots + (static_cast<int64_t>(w - cta * kResWarps) * p.p_max + (tile - wt)) * kSlot;
+#pragma unroll
+      for (int m = 0; m < MT; ++m) {
+        const float4 v = reinterpret_cast<const float4*>(sl + lane * 4 * MT)[m];
+        y[m][0] += v.x; y[m][1] += v.y; y[m][2] += v.z; y[m][3] += v.w;
+      }
+    }
+  }
+  const int64_t cf = wf / kResWarps, cl = wl / kResWarps;
+  if (cf != cl) {  // pieces in other CTAs too
+    float* tp = p.gpart + static_cast<int64_t>(tile) * p.max_cta_seg * kSlot;
+#pragma unroll
+    for (int m = 0; m < MT; ++m)
+      __stcg(reinterpret_cast<float4*>(tp + (cta - cf) * kSlot + lane * 4 * MT) + m,
+             make_float4(y[m][0], y[m][1], y[m][2], y[m][3]));
+    __syncwarp();
+    unsigned int ticket = 0;
+    if (lane == 0) ticket = atom_add_acq_rel_gpu_r(&p.gcnt[tile], 1u);
+    ticket = __shfl_sync(0xffffffffu, ticket, 0);
+    if (ticket != static_cast<unsigned int>(cl - cf)) return;  // another CTA completes the tile
+    __syncwarp();
+#pragma unroll
+    for (int m = 0; m < MT; ++m) y[m][0] = y[m][1] = y[m][2] = y[m][3] = 0.0f;
+    for (int64_t c = 0; c <= cl - cf; ++c) {  // CTA order
+#pragma unroll
+      for (int m = 0; m < MT; ++m) {
+        const float4 v = __ldcg(reinterpret_cast<const float4*>(tp + c * kSlot + lane * 4 * MT) + m);
+        y[m][0] += v.x; y[m][1] += v.y; y[m][2] += v.z; y[m][3] += v.w;
+      }
+    }
+  }
+  lora_up_store<MT>(y, tile, lane, p);
+}
+
+// SINGLE: single-level storage (the block constant is absmax[b]); V8: the packed
+// codes are 32-byte aligned, so each block is one 256-bit load.
+template <int MT, bool SINGLE>
+__global__ void __maxnreg__(kResRegs)
+k_decode_res(const __grid_constant__ ResParams p, const __grid_constant__ Nf4Codebook cb) {
+  extern __shared__ __align__(16) uint8_t res_sm[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, t = lane & 3;
+  const int64_t K = p.K, N = p.N;
+  const int nkb_row = static_cast<int>(K / 64);
+  const int nsb = (nkb_row + 3) / 4;
+  const int nblk_pad = nsb * 4;
+  const int M = p.M;
+  float* slots = reinterpret_cast<float*>(res_sm + res_slot_off(p));
+  unsigned int* cnt = reinterpret_cast<unsigned int*>(slots + static_cast<size_t>(kResWarps) * p.p_max * 32 * 4 * MT);
+  const uint32_t cnt_base = smem_u32(cnt);
+
+  // ---- prologue: counters, and X copied into shared memory (padded blocks,
+  // zero beyond K). X is an input of the call, complete before the LoRA-down
+  // kernel that precedes this one started.
+  for (int i = threadIdx.x; i < p.cta_tiles; i += blockDim.x) cnt[i] = 0u;
+  {
+    const int chunks = M * nblk_pad * 8;  // 16-byte chunks of X to place
+    for (int c = threadIdx.x; c < chunks; c += blockDim.x) {
+      const int m = c / (nblk_pad * 8);
+      const int rem = c - m * nblk_pad * 8;
+      const int b = rem >> 3, q = rem & 7;
+      uint4 v = make_uint4(0u, 0u, 0u, 0u);
+      if (b < nkb_row) v = __ldg(reinterpret_cast<const uint4*>(p.X + static_cast<int64_t>(m) * K + b * 64) + q);
+      *reinterpret_cast<uint4*>(res_sm + m * p.x_stride + b * kXBlockBytes + q * 16) = v;
+    }
+  }
+  __syncthreads();
+
+  const int64_t gw = static_cast<int64_t>(blockIdx.x) * kResWarps + warp;
+  const int64_t i0 = gw < p.n_units ? range_begin(gw, p.n_items, p.n_units) : 0;
+  const int64_t i1 = gw < p.n_units ? range_begin(gw + 1, p.n_items, p.n_units) : 0;
+  const int n_my = static_cast<int>(i1 - i0);
+  const bool reverse = warp == kResWarps - 1;
+  const float mu = SINGLE ? 0.0f : __ldg(p.mean);
+  const uint32_t xbase = smem_u32(res_sm);
+  // token rows of this lane's B fragments (tokens >= M read the last token:
+  // those output columns are never stored)
+  uint32_t xrow[MT];
+#pragma unroll
+  for (int m = 0; m < MT; ++m) xrow[m] = xbase + static_cast<uint32_t>(min(g + 8 * m, M - 1) * p.x_stride);
+
+  // item e of this warp's walk
+  auto item_at = [&](int e) -> int64_t { return reverse ? i1 - 1 - e : i0 + e; };
+  struct Fetch {
+    uint4 a0, a1, b0, b1;  // codes of rows g and g + 8 (32 bytes each)
+    int qa, qb;
+    float sa, sb;
+    bool va, vb;
+  };
+  auto fetch = [&](int64_t i, Fetch& f) {
+    const int64_t tile = i / nsb;
+    const int kb = static_cast<int>(i - tile * nsb) * 4 + t;
+    const int64_t na = tile * 16 + g, nb = na + 8;
+    f.va = kb < nkb_row && na < N;
+    f.vb = kb < nkb_row && nb < N;
+    const int64_t ba = na * nkb_row + kb, bb = nb * nkb_row + kb;
+    const uint8_t* pa = p.packed + ba * 32;
+    const uint8_t* pb = p.packed + bb * 32;
+    f.a0 = f.va ? ldg_stream(pa) : make_uint4(0u, 0u, 0u, 0u);
+    f.a1 = f.va ? ldg_stream(pa + 16) : make_uint4(0u, 0u, 0u, 0u);
+    f.b0 = f.vb ? ldg_stream(pb) : make_uint4(0u, 0u, 0u, 0u);
+    f.b1 = f.vb ? ldg_stream(pb + 16) : make_uint4(0u, 0u, 0u, 0u);
+    if (SINGLE) {
+      f.qa = f.qb = 0;
+      f.sa = f.va ? __ldg(p.absmax + ba) : 0.0f;
+      f.sb = f.vb ? __ldg(p.absmax + bb) : 0.0f;
+    } else {
+      f.qa = f.va ? static_cast<int>(__ldg(p.q + ba)) : 0;
+      f.sa = f.va ? __ldg(p.dqs + (ba >> 8)) : 0.0f;
+      f.qb = f.vb ? static_cast<int>(__ldg(p.q + bb)) : 0;
+      f.sb = f.vb ? __ldg(p.dqs + (bb >> 8)) : 0.0f;
+    }
+  };
+  // L2 prefetch of an item's codes: lane t == 0 of each row pair touches the
+  // 128-byte line that the row's four lanes read
+  auto prefetch_item = [&](int64_t i) {
+    const int64_t tile = i / nsb;
+    const int64_t sbk = i - tile * nsb;
+    if (t == 0) {
+      const int64_t na = tile * 16 + g, nb = na + 8;
+      if (na < N) prefetch_l2(p.packed + (na * nkb_row + sbk * 4) * 32);
+      if (nb < N) prefetch_l2(p.packed + (nb * nkb_row + sbk * 4) * 32);
+    }
+  };
+
+  bool entered = false;  // waited for the LoRA-down kernel (T, zeroed tickets)
+  if (n_my > 0) {
+    Fetch cur, nxt;
+    fetch(item_at(0), cur);
+    if (n_my > 1) prefetch_item(item_at(1));
+    float acc[2][MT][4];
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+      for (int m = 0; m < MT; ++m) acc[h][m][0] = acc[h][m][1] = acc[h][m][2] = acc[h][m][3] = 0.0f;
+    int64_t tile = item_at(0) / nsb;
+    // L2 prefetch of the tile's LoRA-up rows of B (read by whoever completes it)
+    if (lane < 16 && tile * 16 + lane < N) prefetch_l2(p.Bl + (tile * 16 + lane) * p.r);
+    for (int e = 0; e < n_my; ++e) {
+      const int64_t i = item_at(e);
+      const int sb = static_cast<int>(i - tile * nsb);
+      if (e + 1 < n_my) fetch(item_at(e + 1), nxt);
+      if (e + 2 < n_my) prefetch_item(item_at(e + 2));
+      const float mA = cur.va ? (SINGLE ? cur.sa : __fmaf_rn(static_cast<float>(cur.qa), cur.sa, mu)) : 0.0f;
+      const float mB = cur.vb ? (SINGLE ? cur.sb : __fmaf_rn(static_cast<float>(cur.qb), cur.sb, mu)) : 0.0f;
+      const Nf4Lut la = make_nf4_lut(cb, mA);
+      const Nf4Lut lb = make_nf4_lut(cb, mB);
+      const uint32_t xblk = static_cast<uint32_t>((sb * 4 + t) * kXBlockBytes);
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {  // 16-byte half c of the lane's 32 code bytes: words 4c .. 4c + 3
+        const uint4 ca = c ? cur.a1 : cur.a0;
+        const uint4 cbw = c ? cur.b1 : cur.b0;
+#pragma unroll
+        for (int jj = 0; jj < 2; ++jj) {
+          const int j = 2 * c + jj;  // group: k = 16 j .. 16 j + 15 of the block
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {  // word 2 j + h holds k = 16 j + 8 h .. + 7
+            uint4 xv[MT];
+#pragma unroll
+            for (int m = 0; m < MT; ++m) xv[m] = lds128r(xrow[m] + xblk + (16 * j + 8 * h) * 2);
+            const uint32_t wa = jj ? (h ? ca.w : ca.z) : (h ? ca.y : ca.x);
+            const uint32_t wb = jj ? (h ? cbw.w : cbw.z) : (h ? cbw.y : cbw.x);
+            const uint32_t sa = wa & 0x77777777u, sbw = wb & 0x77777777u;
+            const uint32_t ta = ((wa >> 1) & 0x44444444u) | 0x32103210u;
+            const uint32_t tb = ((wb >> 1) & 0x44444444u) | 0x32103210u;
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {  // k = 16 j + 8 h + 4 half .. + 3
+              uint32_t a0, a1, a2, a3;
+              lookup4(la, half ? (sa >> 16) : sa, half ? (ta >> 16) : ta, a0, a2);     // row g
+              lookup4(lb, half ? (sbw >> 16) : sbw, half ? (tb >> 16) : tb, a1, a3);   // row g + 8
+#pragma unroll
+              for (int m = 0; m < MT; ++m)
+                mma16816r(acc[half][m], a0, a1, a2, a3, half ? xv[m].z : xv[m].x, half ? xv[m].w : xv[m].y);
+            }
+          }
+        }
+      }
+      if (e + 1 < n_my) cur = nxt;
+      const int64_t next_tile = e + 1 < n_my ? item_at(e + 1) / nsb : -1;
+      if (next_tile != tile) {  // end of this warp's piece of `tile`
+        if (!entered) {  // T and the zeroed tickets come from the preceding LoRA-down kernel
+          pdl_enter();
+          entered = true;
+        }
+        publish<MT>(acc, tile, lane, warp, slots, cnt_base, p);
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+          for (int m = 0; m < MT; ++m) acc[h][m][0] = acc[h][m][1] = acc[h][m][2] = acc[h][m][3] = 0.0f;
+        tile = next_tile;
+        if (tile >= 0 && lane < 16 && tile * 16 + lane < N) prefetch_l2(p.Bl + (tile * 16 + lane) * p.r);
+      }
+    }
+  }
+  // every path waits for the preceding grid before the next one may launch
+  if (!entered) pdl_enter();
+}
+
+}  // namespace
+
+// Work split and shared-memory plan of the X-resident kernel; ok == false when X
+// and the slots do not fit (the TMA-ring kernel then serves the call).
+ResPlan res_plan(int64_t M, int64_t N, int64_t K, int num_sms) {
+  ResPlan p{};
+  p.ok = false;
+  if (M < 1 || M > 16 || N < 1 || K < 64) return p;
+  p.mt = M <= 8 ? 1 : 2;
+  const int64_t nkb_row = K / 64;
+  const int64_t nsb = (nkb_row + 3) / 4;
+  p.n_tiles = (N + 15) / 16;
+  p.n_items = p.n_tiles * nsb;
+  p.grid = num_sms;
+  if (p.n_items < static_cast<int64_t>(num_sms) * kResWarps) {
+    // fewer items than warps: fewer CTAs, so that no warp is idle
+    p.grid = static_cast<int>((p.n_items + kResWarps - 1) / kResWarps);
+    if (p.grid < 1) p.grid = 1;
+  }
+  // at most one warp per item, so that every working warp's range is non-empty
+  // and the owners of a tile's items are consecutive working warps (warps
+  // numbered n_units and above, in the last CTA, have no range)
+  p.n_units = static_cast<int64_t>(p.grid) * kResWarps;
+  if (p.n_units > p.n_items) p.n_units = p.n_items;
+  // token row stride: whole padded blocks, then rounded to 64 mod 128 bytes so
+  // the 8 lanes of each shared-memory phase hit 8 distinct 16-byte bank groups
+  int64_t xs = nsb * 4 * kXBlockBytes;
+  xs = (xs + 63) / 128 * 128 + 64;
+  p.x_stride = static_cast<int>(xs);
+  // reduction slots: the most tiles one warp's range touches
+  int64_t pmax = 1, ctiles = 1, maxcs = 1;
+  for (int64_t u = 0; u < p.n_units; ++u) {
+    const int64_t a = range_begin(u, p.n_items, p.n_units), b = range_begin(u + 1, p.n_items, p.n_units);
+    if (b > a) {
+      const int64_t tp = (b - 1) / nsb - a / nsb + 1;
+      if (tp > pmax) pmax = tp;
+    }
+  }
+  for (int64_t c = 0; c < p.grid; ++c) {
+    const int64_t u0 = c * kResWarps, u1 = (c + 1) * kResWarps < p.n_units ? (c + 1) * kResWarps : p.n_units;
+    if (u0 >= u1) continue;
+    const int64_t a = range_begin(u0, p.n_items, p.n_units);
+    const int64_t b = range_begin(u1, p.n_items, p.n_units);
+    if (b > a) {
+      const int64_t tc = (b - 1) / nsb - a / nsb + 1;
+      if (tc > ctiles) ctiles = tc;
+    }
+  }
+  for (int64_t tile = 0; tile < p.n_tiles; ++tile) {
+    const int64_t wf = owner_of(tile * nsb, p.n_items, p.n_units);
+    const int64_t wl = owner_of(tile * nsb + nsb - 1, p.n_items, p.n_units);
+    const int64_t cs = wl / kResWarps - wf / kResWarps + 1;
+    if (cs > maxcs) maxcs = cs;
+  }
+  p.p_max = static_cast<int>(pmax);
+  p.cta_tiles = static_cast<int>(ctiles);
+  p.max_cta_seg = static_cast<int>(maxcs);
+  const size_t xbytes = (static_cast<size_t>(M) * p.x_stride + 15) / 16 * 16;
+  const size_t sbytes = static_cast<size_t>(kResWarps) * p.p_max * 32 * 4 * p.mt * sizeof(float);
+  p.smem = xbytes + sbytes + static_cast<size_t>(p.cta_tiles) * 4;
+  p.ok = p.smem <= 200 * 1024;
+  return p;
+}
+
+size_t res_partial_elems(const ResPlan& p) {
+  return static_cast<size_t>(p.n_tiles) * p.max_cta_seg * 32 * 4 * p.mt;
+}
+
+cudaError_t launch_decode_res_main(const Nf4View& w, const void* X, int64_t M, const void* B, int r, float s,
+                                   void* Y, const float* T, float* partial, unsigned int* counters,
+                                   const ResPlan& rp, const float codebook[16], int32_t* err,
+                                   cudaStream_t stream) {
+  Nf4Codebook cb;
+  for (int i = 0; i < 16; ++i) cb.c[i] = codebook[i];
+  ResParams p;
+  p.packed = w.packed;
+  p.q = w.absmax_q;
+  p.dqs = w.dq_scale;
+  p.mean = w.mean;
+  p.absmax = w.absmax;
+  p.X = static_cast<const __nv_bfloat16*>(X);
+  p.T = T;
+  p.Bl = static_cast<const __nv_bfloat16*>(B);
+  p.Y = static_cast<__nv_bfloat16*>(Y);
+  p.gpart = partial;
+  p.gcnt = counters;
+  p.N = w.N;
+  p.K = w.K;
+  p.n_items = rp.n_items;
+  p.n_units = rp.n_units;
+  p.M = static_cast<int>(M);
+  p.r = r;
+  p.s = s;
+  p.x_stride = rp.x_stride;
+  p.p_max = rp.p_max;
+  p.cta_tiles = rp.cta_tiles;
+  p.max_cta_seg = rp.max_cta_seg;
+  p.err = err;
+  const bool single = w.absmax != nullptr;
+  const int smem = static_cast<int>(rp.smem);
+  cudaError_t e;
+  if (rp.mt == 1) {
+    if (single) {
+      if ((e = ensure_smem_limit<k_decode_res<1, true>>(smem)) != cudaSuccess) return e;
+      e = launch_pdl(k_decode_res<1, true>, dim3(rp.grid), dim3(kResWarps * 32), smem, stream, p, cb);
+    } else {
+      if ((e = ensure_smem_limit<k_decode_res<1, false>>(smem)) != cudaSuccess) return e;
+      e = launch_pdl(k_decode_res<1, false>, dim3(rp.grid), dim3(kResWarps * 32), smem, stream, p, cb);
+    }
+  } else {
+    if (single) {
+      if ((e = ensure_smem_limit<k_decode_res<2, true>>(smem)) != cudaSuccess) return e;
+      e = launch_pdl(k_decode_res<2, true>, dim3(rp.grid), dim3(kResWarps * 32), smem, stream, p, cb);
+    } else {
+      if ((e = ensure_smem_limit<k_decode_res<2, false>>(smem)) != cudaSuccess) return e;
+      e = launch_pdl(k_decode_res<2, false>, dim3(rp.grid), dim3(kResWarps * 32), smem, stream, p, cb);
+    }
+  }
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+}  // namespace qlora

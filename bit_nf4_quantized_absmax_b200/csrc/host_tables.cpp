@@ -1,4 +1,4 @@
-// NF4 codebook and quantization tables, computed on the host.
+// NF4 (and FP4) codebooks and quantization tables, computed on the host.
 //
 // Codebook: normal quantiles at equally spaced probabilities ("Guanaco",
 // "Technical Innovations": a 4-bit type for normally distributed weights;
@@ -35,10 +35,9 @@ double normal_quantile_upper(double p) {
   return x;
 }
 
-void build(QuantTables& t) {
+void nf4_values(double (&vals)[16]) {
   const double d = 1.0 - 0.5 * (1.0 / 30.0 + 1.0 / 32.0);
   const double top = normal_quantile_upper(d);
-  double vals[16];
   int n = 0;
   for (int j = 7; j >= 1; --j) vals[n++] = -normal_quantile_upper(0.5 + (d - 0.5) * j / 7.0) / top;
   vals[n++] = 0.0;
@@ -46,11 +45,35 @@ void build(QuantTables& t) {
   // the end points are exactly -1 and +1 (p = d on both sides)
   vals[0] = -1.0;
   vals[15] = 1.0;
+}
+
+// FP4 ("Float4" of the QLoRA errata page's findings on the paper's p.8 Table 4,
+// which compares it with NFloat4; the pages give no format). Reading: the 4-bit
+// float with 1 sign, 2 exponent and 1 mantissa bit, magnitudes
+// {0, 0.5, 1, 1.5, 2, 3, 4, 6}, divided by 6 so that the range is [-1, 1]. Its
+// two zero encodings are one value, kept once: 15 distinct values in ascending
+// order at indices 0..14, and index 15 repeats +1, so that no value ever maps
+// to it (the nearest code takes the lower index on a tie).
+void fp4_values(double (&vals)[16]) {
+  static const double mag[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
+  int n = 0;
+  for (int k = 7; k >= 1; --k) vals[n++] = -mag[k] / 6.0;
+  for (int k = 0; k < 8; ++k) vals[n++] = mag[k] / 6.0;
+  vals[15] = 1.0;
+}
+
+void build(QuantTables& t, int dtype) {
+  double vals[16];
+  if (dtype == kDtypeFp4)
+    fp4_values(vals);
+  else
+    nf4_values(vals);
   for (int i = 0; i < 16; ++i) t.codebook[i] = static_cast<float>(vals[i]);
 
   // Decision thresholds: nearest code with ties to the lower index means
   // code(v) = #{i : v > mid_i}, mid_i = (c_i + c_{i+1}) / 2 (exact in double).
   // For fp32 v that is #{i : v >= T_i} with T_i the smallest float above mid_i.
+  // (A repeated last value, as in FP4, puts its threshold above 1: never reached.)
   for (int i = 0; i < 15; ++i) {
     double mid = 0.5 * (static_cast<double>(t.codebook[i]) + static_cast<double>(t.codebook[i + 1]));
     float f = static_cast<float>(mid);
@@ -91,14 +114,20 @@ void build(QuantTables& t) {
 
 }  // namespace
 
-const QuantTables& quant_tables() {
-  static const QuantTables tables = [] {
+const QuantTables& quant_tables(int dtype) {
+  static const QuantTables nf4 = [] {
     QuantTables t;
     std::memset(&t, 0, sizeof(t));
-    build(t);
+    build(t, kDtypeNf4);
     return t;
   }();
-  return tables;
+  static const QuantTables fp4 = [] {
+    QuantTables t;
+    std::memset(&t, 0, sizeof(t));
+    build(t, kDtypeFp4);
+    return t;
+  }();
+  return dtype == kDtypeFp4 ? fp4 : nf4;
 }
 
 }  // namespace qlora

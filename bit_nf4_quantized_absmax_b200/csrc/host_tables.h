@@ -27,7 +27,11 @@ struct QuantTables {
   BinEntry bins[kBins];
 };
 
+// 4-bit data types: the NF4 codebook (default) and the FP4 comparison variant.
+constexpr int kDtypeNf4 = 0;
+constexpr int kDtypeFp4 = 1;
+
 // Computed once on first use (thread-safe static initialisation).
-const QuantTables& quant_tables();
+const QuantTables& quant_tables(int dtype = kDtypeNf4);
 
 }  // namespace qlora

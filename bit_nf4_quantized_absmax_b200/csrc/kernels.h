@@ -41,9 +41,10 @@ inline int split_count(int64_t nkb, int want) {
 }
 
 // ---- quantize.cu / dequant.cu ----
+// dtype: the 4-bit codebook (kDtypeNf4, or kDtypeFp4 of host_tables.h).
 cudaError_t launch_quantize(const void* W, int64_t numel, uint8_t* packed, int8_t* absmax_q, float* dq_scale,
                             float* mean, float* absmax_scratch, void* totals_scratch, int num_sms,
-                            cudaStream_t stream);
+                            cudaStream_t stream, int dtype = 0);
 
 // The two halves of launch_quantize, for a weight quantized in row shards:
 // first, the codes, the fp32 constants and the 256 exact bin totals of their
@@ -51,14 +52,14 @@ cudaError_t launch_quantize(const void* W, int64_t numel, uint8_t* packed, int8_
 // been summed, the mean over nblk_mean constants and the int8 codes and group
 // scales of this shard's nblk constants.
 cudaError_t launch_quantize_first(const void* W, int64_t nblk, uint8_t* packed, float* absmax_scratch,
-                                  unsigned long long* totals, int num_sms, cudaStream_t stream);
+                                  unsigned long long* totals, int num_sms, cudaStream_t stream, int dtype = 0);
 cudaError_t launch_quantize_second(const float* absmax_scratch, int64_t nblk, const unsigned long long* totals,
                                    int64_t nblk_mean, int8_t* absmax_q, float* dq_scale, float* mean,
                                    cudaStream_t stream);
 
 // Single-level storage: the codes and the fp32 block constants m_b only (pass 1).
 cudaError_t launch_quantize_single(const void* W, int64_t numel, uint8_t* packed, float* absmax, int num_sms,
-                                   cudaStream_t stream);
+                                   cudaStream_t stream, int dtype = 0);
 
 // A stored weight. Double-quantized: absmax_q, dq_scale and mean give the block
 // constant m'_b = fmaf(absmax_q[b], dq_scale[b / 256], mean) and absmax is null.
@@ -92,11 +93,34 @@ struct DecodePlan {
 DecodePlan decode_plan(int64_t M, int64_t N, int64_t K, int ref_sms);
 size_t decode_partial_elems(const DecodePlan& p);
 size_t decode_counter_words(const DecodePlan& p);
+// Plan of the X-resident decode kernel (decode_res.cu): token values held in
+// shared memory, warp-level item ranges. ok is false when it does not fit.
+struct ResPlan {
+  bool ok;
+  int mt;
+  int64_t n_tiles;     // 16-row tiles
+  int64_t n_items;     // n_tiles * ceil(K / 256)
+  int64_t n_units;     // warps of the grid
+  int grid;            // CTAs (one per SM)
+  int x_stride;        // bytes per token row of the shared X copy
+  int p_max;           // reduction slots per warp
+  int cta_tiles;       // tile counters per CTA
+  int max_cta_seg;     // most CTAs holding pieces of one tile
+  size_t smem;         // dynamic shared memory per CTA
+};
+ResPlan res_plan(int64_t M, int64_t N, int64_t K, int num_sms);
+size_t res_partial_elems(const ResPlan& p);
+cudaError_t launch_decode_res_main(const Nf4View& w, const void* X, int64_t M, const void* B, int r, float s,
+                                   void* Y, const float* T, float* partial, unsigned int* counters,
+                                   const ResPlan& rp, const float codebook[16], int32_t* err, cudaStream_t stream);
+
 // T [M, r] fp32 receives X A^T; partial [decode_partial_elems] fp32 and
-// counters [decode_counter_words] are scratch.
+// counters [decode_counter_words] are scratch. With rp.ok the X-resident kernel
+// runs (partial then holds res_partial_elems(rp) floats, counters rp.n_tiles words).
 cudaError_t launch_decode_fwd(const Nf4View& w, const void* X, int64_t M, const void* A, const void* B, int r,
                               float s, void* Y, float* T, float* partial, unsigned int* counters,
-                              const DecodePlan& p, const float codebook[16], int32_t* err, cudaStream_t stream);
+                              const DecodePlan& p, const ResPlan& rp, const float codebook[16], int32_t* err,
+                              cudaStream_t stream);
 
 // ---- merge.cu: weighted LoRA adapters merged into the dequantized base ----
 constexpr int kMaxMergeAdapters = 8;

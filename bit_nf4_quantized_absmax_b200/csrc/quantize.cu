@@ -350,8 +350,8 @@ int pass1_grid(int64_t nblk, int num_sms) {
 }
 
 cudaError_t launch_pass1(const void* W, int64_t nblk, uint8_t* packed, float* absmax, unsigned long long* zero_totals,
-                         int num_sms, cudaStream_t stream) {
-  const QuantTables& tabs = quant_tables();
+                         int num_sms, cudaStream_t stream, int dtype) {
+  const QuantTables& tabs = quant_tables(dtype);
   QuantBinTable tab;
   for (int i = 0; i < kBins; ++i) tab.bins[i] = tabs.bins[i];
   const bool v8 = ((reinterpret_cast<uintptr_t>(W) | reinterpret_cast<uintptr_t>(packed)) & 31u) == 0;
@@ -363,8 +363,8 @@ cudaError_t launch_pass1(const void* W, int64_t nblk, uint8_t* packed, float* ab
 }  // namespace
 
 cudaError_t launch_quantize_first(const void* W, int64_t nblk, uint8_t* packed, float* absmax_scratch,
-                                  unsigned long long* totals, int num_sms, cudaStream_t stream) {
-  cudaError_t e = launch_pass1(W, nblk, packed, absmax_scratch, totals, num_sms, stream);
+                                  unsigned long long* totals, int num_sms, cudaStream_t stream, int dtype) {
+  cudaError_t e = launch_pass1(W, nblk, packed, absmax_scratch, totals, num_sms, stream, dtype);
   if (e != cudaSuccess) return e;
   // chunks of at least 512 constants and at most 8 CTAs per SM (the loop of a
   // CTA is latency bound, so many short chunks beat few long ones), at most
@@ -392,17 +392,17 @@ cudaError_t launch_quantize_second(const float* absmax_scratch, int64_t nblk, co
 
 cudaError_t launch_quantize(const void* W, int64_t numel, uint8_t* packed, int8_t* absmax_q, float* dq_scale,
                             float* mean, float* absmax_scratch, void* totals_scratch, int num_sms,
-                            cudaStream_t stream) {
+                            cudaStream_t stream, int dtype) {
   const int64_t nblk = numel / 64;
   unsigned long long* totals = static_cast<unsigned long long*>(totals_scratch);
-  cudaError_t e = launch_quantize_first(W, nblk, packed, absmax_scratch, totals, num_sms, stream);
+  cudaError_t e = launch_quantize_first(W, nblk, packed, absmax_scratch, totals, num_sms, stream, dtype);
   if (e != cudaSuccess) return e;
   return launch_quantize_second(absmax_scratch, nblk, totals, nblk, absmax_q, dq_scale, mean, stream);
 }
 
 cudaError_t launch_quantize_single(const void* W, int64_t numel, uint8_t* packed, float* absmax, int num_sms,
-                                   cudaStream_t stream) {
-  return launch_pass1(W, numel / 64, packed, absmax, nullptr, num_sms, stream);
+                                   cudaStream_t stream, int dtype) {
+  return launch_pass1(W, numel / 64, packed, absmax, nullptr, num_sms, stream, dtype);
 }
 
 }  // namespace qlora

@@ -131,6 +131,24 @@ const char* qlora_status_string(qlora_status s);
  * Errors: QLORA_ERR_INVALID_ARG if out16 is NULL. */
 qlora_status qlora_nf4_codebook(float out16[16]);
 
+/* 4-bit data types. NF4 is the QLoRA type ([G] "Technical Innovations", [C] 1);
+ * FP4 is the 4-bit float the paper compares it with (the errata page [E],
+ * findings on the paper's p.8 Table 4: NFloat4 against Float4; the pages print
+ * no FP4 format). Reading taken for FP4: 1 sign, 2 exponent and 1 mantissa
+ * bit, magnitudes {0, 0.5, 1, 1.5, 2, 3, 4, 6} divided by 6 (range [-1, 1]),
+ * ascending; its two encodings of zero are one value, kept once, so indices
+ * 0..14 hold the 15 distinct values and index 15 repeats +1 (the nearest code
+ * takes the lower index on a tie, so no weight is ever coded 15). */
+typedef enum {
+  QLORA_DTYPE_NF4 = 0,
+  QLORA_DTYPE_FP4 = 1
+} qlora_dtype;
+
+/* qlora_codebook -- the 16 values of a 4-bit data type, ascending, fp32 (host
+ * call). QLORA_DTYPE_NF4 gives qlora_nf4_codebook's values.
+ * Errors: INVALID_ARG (NULL out16), UNSUPPORTED (unknown dtype). */
+qlora_status qlora_codebook(qlora_dtype dtype, float out16[16]);
+
 /* qlora_nf4_storage_bytes -- sizes of the four arrays of qlora_nf4_weight for
  * a [rows, cols] weight (host call). out[0..3] = bytes of packed, absmax_q,
  * dq_scale, mean. Errors: QLORA_ERR_INVALID_ARG (NULL out, negative sizes),
@@ -238,6 +256,23 @@ qlora_status qlora_quantize_nf4_dq_shard_end(const qlora_nf4_weight* q, int64_t 
                                              int64_t total_rows, const uint64_t* bin_totals,
                                              const void* workspace, size_t workspace_bytes,
                                              qlora_stream_t stream);
+
+/* qlora_quantize_4bit -- block-wise absmax quantization with the codebook of
+ * `dtype`: the computation of qlora_quantize_nf4_dq (q->dq_blocksize == 256,
+ * double-quantized constants) or of qlora_quantize_nf4 (q->dq_blocksize == 0,
+ * fp32 constants), with codebook[code] taken from qlora_codebook(dtype). The
+ * nearest code ties to the lower index, as for NF4. Workspace as in
+ * qlora_quantize_nf4_dq; single-level storage uses none of it (a size query
+ * returns 256, and any non-NULL workspace is accepted and left untouched).
+ * Errors: those of the two calls, and UNSUPPORTED for an unknown dtype. */
+qlora_status qlora_quantize_4bit(const void* W_bf16, const qlora_nf4_weight* q, qlora_dtype dtype,
+                                 void* workspace, size_t* workspace_bytes, qlora_stream_t stream);
+
+/* qlora_dequantize_4bit -- qlora_dequantize_nf4 with the codebook of `dtype`:
+ * w' = bf16_rn(fp32(codebook[code] * m'_b)) for either storage kind.
+ * Errors: those of qlora_dequantize_nf4, and UNSUPPORTED for an unknown dtype. */
+qlora_status qlora_dequantize_4bit(const qlora_nf4_weight* q, qlora_dtype dtype, void* out_bf16,
+                                   qlora_stream_t stream);
 
 /* qlora_dequantize_nf4 -- decode q (either storage kind) to a bf16 matrix
  * out_bf16 [rows, cols] (device, 16-byte aligned): w' = bf16_rn(fp32(

@@ -26,7 +26,7 @@ Where the pages are silent the oracle takes one stated reading; every reading is
 listed in the repository's design notes.
 """
 from .fp import bf16_bits_to_f32, f32_to_bf16_bits_rn, fma_f32
-from .nf4 import (BLOCK, DQ_BLOCK, nf4_codebook, quantize_nf4, dq_mean, double_quantize, quantize_nf4_dq,
+from .nf4 import (BLOCK, DQ_BLOCK, nf4_codebook, fp4_codebook, quantize_nf4, dq_mean, double_quantize, quantize_nf4_dq,
                   dequantize_nf4_dq, pack_codes, unpack_codes, storage_bytes, QuantizedNF4, QuantizedNF4Single,
                   quantize_nf4_single, dequantize_nf4_single)
 from .linear import lora_scale, linear_fwd, linear_bwd
@@ -35,7 +35,7 @@ from .optim import adamw_step
 
 __all__ = [
     "bf16_bits_to_f32", "f32_to_bf16_bits_rn", "fma_f32",
-    "BLOCK", "DQ_BLOCK", "nf4_codebook", "quantize_nf4", "dq_mean", "double_quantize", "quantize_nf4_dq",
+    "BLOCK", "DQ_BLOCK", "nf4_codebook", "fp4_codebook", "quantize_nf4", "dq_mean", "double_quantize", "quantize_nf4_dq",
     "dequantize_nf4_dq", "pack_codes", "unpack_codes", "storage_bytes", "QuantizedNF4", "QuantizedNF4Single",
     "quantize_nf4_single", "dequantize_nf4_single",
     "lora_scale", "linear_fwd", "linear_bwd",

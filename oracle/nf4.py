@@ -92,6 +92,44 @@ def nf4_codebook() -> np.ndarray:
     return nf4_codebook_f64().astype(np.float32)
 
 
+def fp4_codebook() -> np.ndarray:
+    """The FP4 comparison codebook as fp32[16], ascending.
+
+    Reading (the QLoRA errata page's findings on the paper's p.8 Table 4 compare
+    NFloat4 with Float4; the pages give no format): the 4-bit float with one sign
+    bit, two exponent bits e and one mantissa bit f, exponent bias 1, with
+    subnormals at e = 0: value = f / 2 for e = 0, (1 + f / 2) * 2^(e - 1)
+    otherwise. Divided by its largest magnitude so the range is [-1, 1], like
+    NF4. Its +0 and -0 are one value, kept once: the 15 distinct values fill
+    indices 0..14 and index 15 repeats the largest value, which the nearest code
+    (ties to the lower index) never selects.
+    """
+    mags = set()
+    for e in range(4):
+        for f in range(2):
+            mags.add(Fraction(f, 2) if e == 0 else (1 + Fraction(f, 2)) * Fraction(2) ** (e - 1))
+    top = max(mags)
+    vals = sorted({s * m / top for m in mags for s in (1, -1)})
+    assert len(vals) == 15
+    vals.append(vals[-1])
+    out = np.empty(16, dtype=np.float32)
+    for i, v in enumerate(vals):
+        out[i] = _fraction_to_f32(v)
+    return out
+
+
+def _fraction_to_f32(x: Fraction) -> np.float32:
+    """Round an exact rational to the nearest fp32 (ties to even): the two fp32
+    neighbours of the fp64 value bracket it, and the nearer one wins."""
+    f = np.float32(float(x))
+    best = f
+    for g in (np.nextafter(f, np.float32(-np.inf)), np.nextafter(f, np.float32(np.inf))):
+        dg, db = abs(Fraction(float(g)) - x), abs(Fraction(float(best)) - x)
+        if dg < db or (dg == db and int(np.array(g).view(np.uint32)) % 2 == 0):
+            best = g
+    return np.float32(best)
+
+
 def nearest_code(v: np.ndarray, codebook: np.ndarray) -> np.ndarray:
     """argmin_i |v - c_i| for fp32 v in [-1, 1]; ties go to the lower index.
 

@@ -1,5 +1,6 @@
-// Exhaustive host check of the quantize kernel's binning rule: for every fp32 v
-// in [-1, 1], the code the kernel forms from its 32-bin table,
+// Exhaustive host check of the quantize kernel's binning rule, for the NF4 and
+// the FP4 tables: for every fp32 v in [-1, 1], the code the kernel forms from
+// its 32-bin table,
 //   x = fmaf(v, kBinMul, kBinAdd), entry = bins[(bits(x) & 0xF8) >> 3],
 //   code = (entry.j + 1) - [RN(v - entry.threshold) < 0],
 // must equal the number of decision thresholds T_i with v >= T_i (the nearest
@@ -15,8 +16,8 @@
 
 using namespace qlora;
 
-static uint64_t check_range(uint32_t lo, uint32_t hi, int sign) {
-  const QuantTables& t = quant_tables();
+static uint64_t check_range(uint32_t lo, uint32_t hi, int sign, int dtype) {
+  const QuantTables& t = quant_tables(dtype);
   uint64_t bad = 0;
   for (uint32_t bits = lo; bits < hi; ++bits) {
     const uint32_t b = bits | (sign ? 0x80000000u : 0u);
@@ -43,17 +44,23 @@ static uint64_t check_range(uint32_t lo, uint32_t hi, int sign) {
 int main() {
   const uint32_t end = 0x3F800001u;  // every bit pattern of [+0, 1]
   const unsigned nt = std::thread::hardware_concurrency() ? std::thread::hardware_concurrency() : 4;
-  std::vector<std::thread> th;
-  std::vector<uint64_t> bad(2 * nt, 0);
-  for (int sign = 0; sign < 2; ++sign)
-    for (unsigned k = 0; k < nt; ++k) {
-      const uint32_t lo = static_cast<uint32_t>(uint64_t(end) * k / nt);
-      const uint32_t hi = static_cast<uint32_t>(uint64_t(end) * (k + 1) / nt);
-      th.emplace_back([&, lo, hi, sign, k] { bad[sign * nt + k] = check_range(lo, hi, sign); });
-    }
-  for (auto& x : th) x.join();
   uint64_t total = 0;
-  for (uint64_t b : bad) total += b;
-  std::printf("checked %llu values, %llu mismatches\n", 2ull * end, static_cast<unsigned long long>(total));
+  for (int dtype : {kDtypeNf4, kDtypeFp4}) {
+    std::vector<std::thread> th;
+    std::vector<uint64_t> bad(2 * nt, 0);
+    for (int sign = 0; sign < 2; ++sign)
+      for (unsigned k = 0; k < nt; ++k) {
+        const uint32_t lo = static_cast<uint32_t>(uint64_t(end) * k / nt);
+        const uint32_t hi = static_cast<uint32_t>(uint64_t(end) * (k + 1) / nt);
+        th.emplace_back([&, lo, hi, sign, k] { bad[sign * nt + k] = check_range(lo, hi, sign, dtype); });
+      }
+    for (auto& x : th) x.join();
+    uint64_t sub = 0;
+    for (uint64_t b : bad) sub += b;
+    std::printf("dtype %d: checked %llu values, %llu mismatches\n", dtype, 2ull * end,
+                static_cast<unsigned long long>(sub));
+    total += sub;
+  }
+  std::printf("%llu mismatches\n", static_cast<unsigned long long>(total));
   return total == 0 ? 0 : 1;
 }

@@ -1,6 +1,6 @@
-"""Host logic: the quantize kernel's bin table and nearest-code rule, checked
-exhaustively over every fp32 v in [-1, 1] by a small C++ program built against
-the library's host tables (no GPU)."""
+"""Host logic: the quantize kernel's bin tables (NF4 and FP4) and nearest-code
+rule, checked exhaustively over every fp32 v in [-1, 1] by a small C++ program
+built against the library's host tables (no GPU)."""
 from __future__ import annotations
 
 import os
@@ -24,4 +24,6 @@ def test_bin_rule_matches_threshold_count_for_every_fp32(tmp_path):
                     "-o", exe], check=True)
     p = subprocess.run([exe], capture_output=True, text=True, timeout=560)
     assert p.returncode == 0, p.stdout + p.stderr
-    assert "0 mismatches" in p.stdout
+    lines = p.stdout.strip().splitlines()
+    assert lines[-1] == "0 mismatches", p.stdout
+    assert sum(1 for l in lines if l.endswith(", 0 mismatches")) == 2, p.stdout  # NF4 and FP4 tables
