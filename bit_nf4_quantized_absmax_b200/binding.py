@@ -25,7 +25,7 @@ EXPORTED = ("qlora_status_string", "qlora_nf4_codebook", "qlora_nf4_storage_byte
             "qlora_quantize_nf4_dq_shard_begin", "qlora_quantize_nf4_dq_shard_end", "qlora_dequantize_nf4",
             "qlora_dequantize_nf4_dq", "qlora_linear_fwd", "qlora_linear_bwd", "qlora_linear_bwd_f32",
             "qlora_linear_bwd_dp", "qlora_round_bf16", "qlora_merge_lora", "qlora_codebook", "qlora_quantize_4bit",
-            "qlora_dequantize_4bit",
+            "qlora_dequantize_4bit", "qlora_linear_fwd_multi", "qlora_pack_adapters",
             "qlora_paged_alloc", "qlora_paged_free", "qlora_paged_prefetch", "qlora_adamw_step",
             "qlora_device_error")
 
@@ -82,6 +82,8 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
     lib.qlora_codebook.argtypes = [ctypes.c_int, ctypes.POINTER(ctypes.c_float)]
     lib.qlora_quantize_4bit.argtypes = [vp, wp, ctypes.c_int, vp, szp, vp]
     lib.qlora_dequantize_4bit.argtypes = [wp, ctypes.c_int, vp, vp]
+    lib.qlora_linear_fwd_multi.argtypes = [wp, vp, i64, vp, vp, i32, vp, vp, vp, szp, vp]
+    lib.qlora_pack_adapters.argtypes = [ctypes.POINTER(_Adapter), i32, i64, i64, vp, vp, vp, vp]
     lib.qlora_merge_lora.argtypes = [wp, ctypes.POINTER(_Adapter), i32, vp, vp]
     lib.qlora_device_error.argtypes = [ctypes.POINTER(ctypes.c_int32), vp]
     lib.qlora_paged_alloc.argtypes = [sz, i32, ctypes.POINTER(vp)]
@@ -397,6 +399,38 @@ def qlora_round_bf16(src: torch.Tensor, out: torch.Tensor | None = None, stream=
     assert out.dtype == torch.bfloat16 and out.is_contiguous() and out.numel() == src.numel()
     _check(load_library().qlora_round_bf16(_ptr(src), _ptr(out), src.numel(), _stream(stream)), "qlora_round_bf16")
     return out
+
+
+def qlora_pack_adapters(adapters, rows: int, cols: int, device=None, stream=None) -> tuple:
+    """Concatenate adapters [(A [r, cols], B [rows, r], alpha, weight), ...] along
+    the rank for qlora_linear_fwd_multi. Returns (A_cat, B_cat, col_scale)."""
+    dev = device or adapters[0][0].device
+    rt = sum(A.shape[0] for A, _, _, _ in adapters)
+    A_cat = torch.empty(rt, cols, dtype=torch.bfloat16, device=dev)
+    B_cat = torch.empty(rows, rt, dtype=torch.bfloat16, device=dev)
+    col_scale = torch.empty(rt, dtype=torch.float32, device=dev)
+    arr = (_Adapter * len(adapters))()
+    for i, (A, B, alpha, weight) in enumerate(adapters):
+        arr[i] = _Adapter(_ptr(A), _ptr(B), A.shape[0], float(alpha), float(weight))
+    _check(load_library().qlora_pack_adapters(arr, len(adapters), rows, cols, _ptr(A_cat), _ptr(B_cat),
+                                              _ptr(col_scale), _stream(stream)), "qlora_pack_adapters")
+    return A_cat, B_cat, col_scale
+
+
+def qlora_linear_fwd_multi(q, X: torch.Tensor, A_cat: torch.Tensor, B_cat: torch.Tensor, col_scale: torch.Tensor,
+                           Y: torch.Tensor | None = None, workspace: torch.Tensor | None = None, stream=None):
+    """Y = X W'^T + sum_a c_a (X A_a^T) B_a^T from the packed adapters."""
+    lib = load_library()
+    M, rt = X.shape[0], A_cat.shape[0]
+    if Y is None:
+        Y = torch.empty(M, q.rows, dtype=torch.bfloat16, device=X.device)
+    qc = q.as_c()
+    st = _stream(stream)
+    args = lambda p, n: lib.qlora_linear_fwd_multi(ctypes.byref(qc), _ptr(X), M, _ptr(A_cat), _ptr(B_cat), rt,
+                                                   _ptr(col_scale), _ptr(Y), p, n, st)
+    ws, nbytes = _workspace(args, workspace, X.device)
+    _check(args(_ptr(ws), ctypes.byref(nbytes)), "qlora_linear_fwd_multi")
+    return Y
 
 
 def qlora_merge_lora(q: NF4Weight | SingleNF4Weight, adapters, out: torch.Tensor | None = None,

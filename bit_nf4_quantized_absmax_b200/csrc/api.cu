@@ -99,14 +99,15 @@ qlora_status check_linear(const void* X, int64_t M, const void* A, const void* B
 
 float lora_scale(float alpha, int32_t r) { return alpha / static_cast<float>(r); }
 
-// QLORA_DECODE_RES=0 in the environment selects the TMA-ring decode kernel for
-// every shape instead of the X-resident one where it fits (for comparisons).
-bool res_disabled() {
-  static const bool off = [] {
-    const char* e = std::getenv("QLORA_DECODE_RES");
-    return e && e[0] == '0';
-  }();
-  return off;
+// Decode kernel choice, read on every call: QLORA_DECODE_RES=0 in the
+// environment selects the TMA-ring kernel for every shape, =1 the X-resident
+// kernel wherever it fits (for comparisons and tests); unset, the measured
+// crossover decides.
+int res_mode() {
+  const char* e = std::getenv("QLORA_DECODE_RES");
+  if (e && e[0] == '0') return 0;
+  if (e && e[0] == '1') return 1;
+  return 2;
 }
 
 int32_t* device_error_word() {
@@ -278,6 +279,64 @@ qlora_status dequantize_impl(const qlora_nf4_weight* q, int dtype, void* out_bf1
                                        reinterpret_cast<cudaStream_t>(stream)));
 }
 
+// Forward shared by qlora_linear_fwd (one adapter, scale s = alpha / r) and
+// qlora_linear_fwd_multi (col_scale: one scale per rank column, s = 1).
+qlora_status linear_fwd_impl(const qlora_nf4_weight* q, const void* X, int64_t M, const void* A, const void* B,
+                             int32_t r, float alpha, void* Y, float* T_save, void* workspace,
+                             size_t* workspace_bytes, qlora_stream_t stream, const float* col_scale) {
+  qlora_status st = check_weight(q, true);
+  if (st != QLORA_OK) return st;
+  if ((st = check_linear(X, M, A, B, r, Y)) != QLORA_OK) return st;
+  if (T_save && !aligned(T_save, 4)) return QLORA_ERR_ALIGNMENT;
+  const int64_t N = q->rows, K = q->cols;
+  const int rpad = (r + 63) / 64 * 64;
+  const float s = col_scale ? 1.0f : lora_scale(alpha, r);
+  DeviceInfo di{kRefSms};  // split choices use the reference SM count so the size query needs no device
+  const bool decode = M <= 16;
+  // workspace layout
+  Layout L;
+  size_t off_T = 0, off_part = 0, off_cnt = 0, off_wd = 0, off_sT = 0;
+  DecodePlan dplan{};
+  ResPlan rplan{};
+  if (decode) {
+    dplan = decode_plan(M, N, K, kRefSms);
+    const int mode = res_mode();
+    rplan = M > 0 && mode != 0 ? res_plan(M, N, K, kRefSms, mode == 1) : ResPlan{};
+    off_T = L.add(T_save ? 0 : static_cast<size_t>(M) * r * sizeof(float));
+    off_part = L.add((rplan.ok ? res_partial_elems(rplan) : decode_partial_elems(dplan)) * sizeof(float));
+    off_cnt = L.add((rplan.ok ? static_cast<size_t>(rplan.n_tiles) : decode_counter_words(dplan)) *
+                    sizeof(unsigned int));
+  } else {
+    off_wd = L.add(static_cast<size_t>(N) * K * 2);
+    off_sT = L.add(static_cast<size_t>(M) * rpad * 2);
+    off_part = L.add(static_cast<size_t>(red_splits(M, rpad, K, di.num_sms)) * M * rpad * sizeof(float));
+  }
+  bool launch = false;
+  st = workspace_check(workspace, workspace_bytes, L.total(), &launch);
+  if (st != QLORA_OK || !launch || M == 0) return st;
+  if ((st = device_info(&di)) != QLORA_OK) return st;
+  char* ws = static_cast<char*>(workspace);
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  int32_t* err = device_error_word();
+  const float* cb = quant_tables().codebook;
+  if (decode) {
+    float* T = T_save ? T_save : reinterpret_cast<float*>(ws + off_T);
+    return cuda_status(launch_decode_fwd(view(q), X, M, A, B, r, s, Y, T, reinterpret_cast<float*>(ws + off_part),
+                                         reinterpret_cast<unsigned int*>(ws + off_cnt), dplan, rplan, cb, err, cs,
+                                         col_scale));
+  }
+  void* Wd = ws + off_wd;
+  void* sT = ws + off_sT;
+  float* P = reinterpret_cast<float*>(ws + off_part);
+  const int splits_t = red_splits(M, rpad, K, kRefSms);
+  cudaError_t e = launch_dequantize(view(q), Wd, cb, di.num_sms, cs);
+  if (e == cudaSuccess) e = launch_gemm_lora_t(X, A, M, K, r, rpad, P, splits_t, di.num_sms, err, cs);
+  if (e == cudaSuccess)
+    e = launch_lora_finish(P, splits_t, M, r, rpad, s, T_save, sT, nullptr, nullptr, di.num_sms, cs, col_scale);
+  if (e == cudaSuccess) e = launch_gemm_fwd(X, Wd, sT, B, M, N, K, r, rpad, Y, di.num_sms, err, cs);
+  return cuda_status(e);
+}
+
 }  // namespace
 
 
@@ -372,55 +431,43 @@ qlora_status qlora_dequantize_nf4_dq(const qlora_nf4_weight* q, void* out_bf16, 
 qlora_status qlora_linear_fwd(const qlora_nf4_weight* q, const void* X, int64_t M, const void* A,
                               const void* B, int32_t r, float alpha, void* Y, float* T_save, void* workspace,
                               size_t* workspace_bytes, qlora_stream_t stream) {
-  qlora_status st = check_weight(q, true);
+  return linear_fwd_impl(q, X, M, A, B, r, alpha, Y, T_save, workspace, workspace_bytes, stream, nullptr);
+}
+
+qlora_status qlora_linear_fwd_multi(const qlora_nf4_weight* q, const void* X, int64_t M, const void* A_cat,
+                                    const void* B_cat, int32_t r_total, const float* col_scale, void* Y,
+                                    void* workspace, size_t* workspace_bytes, qlora_stream_t stream) {
+  if (!col_scale) return QLORA_ERR_INVALID_ARG;
+  if (!aligned(col_scale, 4)) return QLORA_ERR_ALIGNMENT;
+  return linear_fwd_impl(q, X, M, A_cat, B_cat, r_total, 1.0f, Y, nullptr, workspace, workspace_bytes, stream,
+                         col_scale);
+}
+
+qlora_status qlora_pack_adapters(const qlora_lora_adapter* adapters, int32_t n_adapters, int64_t rows, int64_t cols,
+                                 void* A_cat, void* B_cat, float* col_scale, qlora_stream_t stream) {
+  if (n_adapters < 1 || !adapters || rows <= 0 || cols <= 0) return QLORA_ERR_INVALID_ARG;
+  if (n_adapters > kMaxMergeAdapters) return QLORA_ERR_UNSUPPORTED;
+  if (!A_cat || !B_cat || !col_scale) return QLORA_ERR_INVALID_ARG;
+  if (!aligned(A_cat, 16) || !aligned(B_cat, 16) || !aligned(col_scale, 4)) return QLORA_ERR_ALIGNMENT;
+  MergeAdapter ma[kMaxMergeAdapters];
+  int rt = 0;
+  for (int a = 0; a < n_adapters; ++a) {
+    const qlora_lora_adapter& ad = adapters[a];
+    if (ad.r < 8 || ad.r > 256 || ad.r % 8) return QLORA_ERR_UNSUPPORTED;
+    if (!ad.A || !ad.B) return QLORA_ERR_INVALID_ARG;
+    if (!aligned(ad.A, 16) || !aligned(ad.B, 16)) return QLORA_ERR_ALIGNMENT;
+    ma[a].A = ad.A;
+    ma[a].B = ad.B;
+    ma[a].r = ad.r;
+    ma[a].c = ad.weight * lora_scale(ad.alpha, ad.r);  // fp32(w * s), as in qlora_merge_lora
+    rt += ad.r;
+  }
+  if (rt > 256) return QLORA_ERR_UNSUPPORTED;
+  DeviceInfo di;
+  qlora_status st = device_info(&di);
   if (st != QLORA_OK) return st;
-  if ((st = check_linear(X, M, A, B, r, Y)) != QLORA_OK) return st;
-  if (T_save && !aligned(T_save, 4)) return QLORA_ERR_ALIGNMENT;
-  const int64_t N = q->rows, K = q->cols;
-  const int rpad = (r + 63) / 64 * 64;
-  const float s = lora_scale(alpha, r);
-  DeviceInfo di{kRefSms};  // split choices use the reference SM count so the size query needs no device
-  const bool decode = M <= 16;
-  // workspace layout
-  Layout L;
-  size_t off_T = 0, off_part = 0, off_cnt = 0, off_wd = 0, off_sT = 0;
-  DecodePlan dplan{};
-  ResPlan rplan{};
-  if (decode) {
-    dplan = decode_plan(M, N, K, kRefSms);
-    rplan = M > 0 && !res_disabled() ? res_plan(M, N, K, kRefSms) : ResPlan{};
-    off_T = L.add(T_save ? 0 : static_cast<size_t>(M) * r * sizeof(float));
-    off_part = L.add((rplan.ok ? res_partial_elems(rplan) : decode_partial_elems(dplan)) * sizeof(float));
-    off_cnt = L.add((rplan.ok ? static_cast<size_t>(rplan.n_tiles) : decode_counter_words(dplan)) *
-                    sizeof(unsigned int));
-  } else {
-    off_wd = L.add(static_cast<size_t>(N) * K * 2);
-    off_sT = L.add(static_cast<size_t>(M) * rpad * 2);
-    off_part = L.add(static_cast<size_t>(red_splits(M, rpad, K, di.num_sms)) * M * rpad * sizeof(float));
-  }
-  bool launch = false;
-  st = workspace_check(workspace, workspace_bytes, L.total(), &launch);
-  if (st != QLORA_OK || !launch || M == 0) return st;
-  if ((st = device_info(&di)) != QLORA_OK) return st;
-  char* ws = static_cast<char*>(workspace);
-  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
-  int32_t* err = device_error_word();
-  const float* cb = quant_tables().codebook;
-  if (decode) {
-    float* T = T_save ? T_save : reinterpret_cast<float*>(ws + off_T);
-    return cuda_status(launch_decode_fwd(view(q), X, M, A, B, r, s, Y, T, reinterpret_cast<float*>(ws + off_part),
-                                         reinterpret_cast<unsigned int*>(ws + off_cnt), dplan, rplan, cb, err, cs));
-  }
-  void* Wd = ws + off_wd;
-  void* sT = ws + off_sT;
-  float* P = reinterpret_cast<float*>(ws + off_part);
-  const int splits_t = red_splits(M, rpad, K, kRefSms);
-  cudaError_t e = launch_dequantize(view(q), Wd, cb, di.num_sms, cs);
-  if (e == cudaSuccess) e = launch_gemm_lora_t(X, A, M, K, r, rpad, P, splits_t, di.num_sms, err, cs);
-  if (e == cudaSuccess)
-    e = launch_lora_finish(P, splits_t, M, r, rpad, s, T_save, sT, nullptr, nullptr, di.num_sms, cs);
-  if (e == cudaSuccess) e = launch_gemm_fwd(X, Wd, sT, B, M, N, K, r, rpad, Y, di.num_sms, err, cs);
-  return cuda_status(e);
+  return cuda_status(launch_pack_adapters(ma, n_adapters, rows, cols, A_cat, B_cat, col_scale, di.num_sms,
+                                          reinterpret_cast<cudaStream_t>(stream)));
 }
 
 qlora_status qlora_linear_bwd(const qlora_nf4_weight* q, const void* X, int64_t M, const void* A,

@@ -386,7 +386,8 @@ constexpr int kLoraDownThreads = 128;
 template <int MT>
 __global__ void __launch_bounds__(kLoraDownThreads, 8)
 k_lora_t_small(const __nv_bfloat16* __restrict__ X, const __nv_bfloat16* __restrict__ A, int M, int64_t K, int r,
-               float* __restrict__ T, unsigned int* __restrict__ counters, int64_t n_counters) {
+               float* __restrict__ T, unsigned int* __restrict__ counters, int64_t n_counters,
+               const float* __restrict__ col_scale) {
   __shared__ float red[kLoraDownThreads / 32][8 * MT];
   pdl_enter();  // after this, the decode kernel may start its main loop
   const int j = blockIdx.x;
@@ -430,6 +431,8 @@ k_lora_t_small(const __nv_bfloat16* __restrict__ X, const __nv_bfloat16* __restr
     float v = 0.0f;
 #pragma unroll
     for (int w = 0; w < kLoraDownThreads / 32; ++w) v += red[w][threadIdx.x];
+    // several adapters at once: each rank column carries its adapter's scale
+    if (col_scale) v = __fmul_rn(col_scale[j], v);
     T[static_cast<int64_t>(threadIdx.x) * r + j] = v;
   }
 }
@@ -484,11 +487,11 @@ bool encode_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_
 cudaError_t launch_decode_fwd(const Nf4View& w, const void* X, int64_t M, const void* A, const void* B, int r,
                               float s, void* Y, float* T, float* partial, unsigned int* counters,
                               const DecodePlan& p, const ResPlan& rp, const float codebook[16], int32_t* err,
-                              cudaStream_t stream) {
+                              cudaStream_t stream, const float* col_scale) {
   if (rp.ok) {  // token values resident in shared memory (decode_res.cu)
     cudaError_t e = launch_pdl(rp.mt == 1 ? k_lora_t_small<1> : k_lora_t_small<2>, dim3(r), dim3(kLoraDownThreads), 0, stream,
                                reinterpret_cast<const __nv_bfloat16*>(X), reinterpret_cast<const __nv_bfloat16*>(A),
-                               static_cast<int>(M), w.K, r, T, counters, rp.n_tiles);
+                               static_cast<int>(M), w.K, r, T, counters, rp.n_tiles, col_scale);
     if (e != cudaSuccess) return e;
     return launch_decode_res_main(w, X, M, B, r, s, Y, T, partial, counters, rp, codebook, err, stream);
   }
@@ -505,7 +508,7 @@ cudaError_t launch_decode_fwd(const Nf4View& w, const void* X, int64_t M, const 
     return cudaErrorInvalidValue;
   cudaError_t e = launch_pdl(p.mt == 1 ? k_lora_t_small<1> : k_lora_t_small<2>, dim3(r), dim3(kLoraDownThreads), 0, stream,
                              reinterpret_cast<const __nv_bfloat16*>(X), reinterpret_cast<const __nv_bfloat16*>(A),
-                             static_cast<int>(M), w.K, r, T, counters, p.row_tiles);
+                             static_cast<int>(M), w.K, r, T, counters, p.row_tiles, col_scale);
   if (e != cudaSuccess) return e;
   // Programmatic dependent launch: the main loop overlaps the LoRA-down kernel;
   // each consumer warp waits for it (griddepcontrol.wait) before its first ticket.

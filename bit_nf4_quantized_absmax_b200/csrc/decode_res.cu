@@ -6,9 +6,9 @@
 // Y[M, N] = X W'^T + s T B^T, T = X A^T from the LoRA-down kernel that runs
 // first (k_lora_t_small in decode.cu).
 //
-// Used when X (M x K bf16, padded) fits in shared memory beside the reduction
-// slots: every M = 1 shape, and M <= 16 up to K of about 4096. Otherwise the
-// TMA-ring kernel of decode.cu runs.
+// Used where it measured faster than the TMA-ring kernel of decode.cu (one
+// token on weights from about 16 M entries, up to 8 tokens from about 64 M) and
+// X (M x K bf16, padded) fits in shared memory beside the reduction slots.
 //
 // Work items are (16-row tile, 256-wide K superblock) pairs in tile-major
 // order, and every warp of the grid takes one contiguous, equally sized range
@@ -46,6 +46,10 @@ constexpr int kXBlockBytes = 64 * 2 + 16;     // one 64-k block of one token, pa
 // free, so that a CTA of the LoRA-down kernel that precedes this one fits beside
 // a CTA of this one.
 constexpr int kResRegs = 112;
+// Most dynamic shared memory a CTA of this kernel uses (X copy, slots and
+// counters); larger plans go to the TMA-ring kernel. The kernel's limit is set
+// to this once, so that every plan up to it launches.
+constexpr int kResSmemCap = 200 * 1024;
 
 __device__ __forceinline__ void mma16816r(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                           uint32_t b0, uint32_t b1) {
@@ -309,78 +313,79 @@ k_decode_res(const __grid_constant__ ResParams p, const __grid_constant__ Nf4Cod
   uint32_t xrow[MT];
 #pragma unroll
   for (int m = 0; m < MT; ++m) xrow[m] = xbase + static_cast<uint32_t>(min(g + 8 * m, M - 1) * p.x_stride);
-
-  // item e of this warp's walk
-  auto item_at = [&](int e) -> int64_t { return reverse ? i1 - 1 - e : i0 + e; };
-  struct Fetch {
-    uint4 a0, a1, b0, b1;  // codes of rows g and g + 8 (32 bytes each)
-    int qa, qb;
-    float sa, sb;
-    bool va, vb;
-  };
-  auto fetch = [&](int64_t i, Fetch& f) {
-    const int64_t tile = i / nsb;
-    const int kb = static_cast<int>(i - tile * nsb) * 4 + t;
-    const int64_t na = tile * 16 + g, nb = na + 8;
-    f.va = kb < nkb_row && na < N;
-    f.vb = kb < nkb_row && nb < N;
-    const int64_t ba = na * nkb_row + kb, bb = nb * nkb_row + kb;
-    const uint8_t* pa = p.packed + ba * 32;
-    const uint8_t* pb = p.packed + bb * 32;
-    f.a0 = f.va ? ldg_stream(pa) : make_uint4(0u, 0u, 0u, 0u);
-    f.a1 = f.va ? ldg_stream(pa + 16) : make_uint4(0u, 0u, 0u, 0u);
-    f.b0 = f.vb ? ldg_stream(pb) : make_uint4(0u, 0u, 0u, 0u);
-    f.b1 = f.vb ? ldg_stream(pb + 16) : make_uint4(0u, 0u, 0u, 0u);
-    if (SINGLE) {
-      f.qa = f.qb = 0;
-      f.sa = f.va ? __ldg(p.absmax + ba) : 0.0f;
-      f.sb = f.vb ? __ldg(p.absmax + bb) : 0.0f;
-    } else {
-      f.qa = f.va ? static_cast<int>(__ldg(p.q + ba)) : 0;
-      f.sa = f.va ? __ldg(p.dqs + (ba >> 8)) : 0.0f;
-      f.qb = f.vb ? static_cast<int>(__ldg(p.q + bb)) : 0;
-      f.sb = f.vb ? __ldg(p.dqs + (bb >> 8)) : 0.0f;
-    }
-  };
-  // L2 prefetch of an item's codes: lane t == 0 of each row pair touches the
-  // 128-byte line that the row's four lanes read
-  auto prefetch_item = [&](int64_t i) {
-    const int64_t tile = i / nsb;
-    const int64_t sbk = i - tile * nsb;
-    if (t == 0) {
-      const int64_t na = tile * 16 + g, nb = na + 8;
-      if (na < N) prefetch_l2(p.packed + (na * nkb_row + sbk * 4) * 32);
-      if (nb < N) prefetch_l2(p.packed + (nb * nkb_row + sbk * 4) * 32);
-    }
-  };
+  const uint32_t row_bytes = static_cast<uint32_t>(K / 2);  // packed bytes per weight row
 
   bool entered = false;  // waited for the LoRA-down kernel (T, zeroed tickets)
   if (n_my > 0) {
-    Fetch cur, nxt;
-    fetch(item_at(0), cur);
-    if (n_my > 1) prefetch_item(item_at(1));
+    // walk position: tile and superblock of the current item, stepped by +-1
+    // item (no divisions in the loop)
+    const int64_t ifirst = reverse ? i1 - 1 : i0;
+    int64_t tile = ifirst / nsb;
+    int sb = static_cast<int>(ifirst - tile * nsb);
+    const int step = reverse ? -1 : 1;
+    // per-tile row state of this lane: rows g and g + 8 of the tile
+    const uint8_t* pa = nullptr;  // packed codes of row g, block t of superblock 0
+    const uint8_t* pb = nullptr;
+    uint32_t ba0 = 0, bb0 = 0;    // block index of (row, block t of superblock 0)
+    bool rowa = false, rowb = false;
+    auto set_tile = [&](int64_t tl) {
+      const int64_t na = tl * 16 + g, nb = na + 8;
+      rowa = na < N;
+      rowb = nb < N;
+      ba0 = static_cast<uint32_t>(na * nkb_row + t);
+      bb0 = static_cast<uint32_t>(nb * nkb_row + t);
+      pa = p.packed + static_cast<int64_t>(ba0) * 32;
+      pb = p.packed + static_cast<int64_t>(bb0) * 32;
+    };
+    set_tile(tile);
+    uint4 ca0, ca1, cb0, cb1;  // codes of the current item (rows g, g + 8; 32 bytes each)
+    float mA, mB;              // its block constants
+    auto fetch = [&](int sbk, uint4& a0, uint4& a1, uint4& b0, uint4& b1, float& ma, float& mb) {
+      const bool va = rowa && sbk * 4 + t < nkb_row, vb = rowb && sbk * 4 + t < nkb_row;
+      const uint32_t o = static_cast<uint32_t>(sbk) * 128u;  // 4 blocks x 32 bytes
+      const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+      a0 = va ? ldg_stream(pa + o) : z;
+      a1 = va ? ldg_stream(pa + o + 16) : z;
+      b0 = vb ? ldg_stream(pb + o) : z;
+      b1 = vb ? ldg_stream(pb + o + 16) : z;
+      const uint32_t ia = ba0 + static_cast<uint32_t>(sbk) * 4u, ib = bb0 + static_cast<uint32_t>(sbk) * 4u;
+      if (SINGLE) {
+        ma = va ? __ldg(p.absmax + ia) : 0.0f;
+        mb = vb ? __ldg(p.absmax + ib) : 0.0f;
+      } else {
+        ma = va ? __fmaf_rn(static_cast<float>(__ldg(p.q + ia)), __ldg(p.dqs + (ia >> 8)), mu) : 0.0f;
+        mb = vb ? __fmaf_rn(static_cast<float>(__ldg(p.q + ib)), __ldg(p.dqs + (ib >> 8)), mu) : 0.0f;
+      }
+    };
+    fetch(sb, ca0, ca1, cb0, cb1, mA, mB);
     float acc[2][MT][4];
 #pragma unroll
     for (int h = 0; h < 2; ++h)
 #pragma unroll
       for (int m = 0; m < MT; ++m) acc[h][m][0] = acc[h][m][1] = acc[h][m][2] = acc[h][m][3] = 0.0f;
-    int64_t tile = item_at(0) / nsb;
     // L2 prefetch of the tile's LoRA-up rows of B (read by whoever completes it)
     if (lane < 16 && tile * 16 + lane < N) prefetch_l2(p.Bl + (tile * 16 + lane) * p.r);
+#pragma unroll 1
     for (int e = 0; e < n_my; ++e) {
-      const int64_t i = item_at(e);
-      const int sb = static_cast<int>(i - tile * nsb);
-      if (e + 1 < n_my) fetch(item_at(e + 1), nxt);
-      if (e + 2 < n_my) prefetch_item(item_at(e + 2));
-      const float mA = cur.va ? (SINGLE ? cur.sa : __fmaf_rn(static_cast<float>(cur.qa), cur.sa, mu)) : 0.0f;
-      const float mB = cur.vb ? (SINGLE ? cur.sb : __fmaf_rn(static_cast<float>(cur.qb), cur.sb, mu)) : 0.0f;
+      // position of the next item
+      int sbn = sb + step;
+      const bool tile_ends = sbn < 0 || sbn >= nsb || e + 1 == n_my;
       const Nf4Lut la = make_nf4_lut(cb, mA);
       const Nf4Lut lb = make_nf4_lut(cb, mB);
+      const uint4 xa0 = ca0, xa1 = ca1, xb0 = cb0, xb1 = cb1;
+      if (!tile_ends) {  // next item in the same tile: load it now, prefetch the one after into L2
+        fetch(sbn, ca0, ca1, cb0, cb1, mA, mB);
+        const int sbp = sbn + step;
+        if (t == 0 && e + 2 < n_my && sbp >= 0 && sbp < nsb) {
+          if (rowa) prefetch_l2(pa + static_cast<uint32_t>(sbp) * 128u);
+          if (rowb) prefetch_l2(pb + static_cast<uint32_t>(sbp) * 128u);
+        }
+      }
       const uint32_t xblk = static_cast<uint32_t>((sb * 4 + t) * kXBlockBytes);
 #pragma unroll
       for (int c = 0; c < 2; ++c) {  // 16-byte half c of the lane's 32 code bytes: words 4c .. 4c + 3
-        const uint4 ca = c ? cur.a1 : cur.a0;
-        const uint4 cbw = c ? cur.b1 : cur.b0;
+        const uint4 ca = c ? xa1 : xa0;
+        const uint4 cbw = c ? xb1 : xb0;
 #pragma unroll
         for (int jj = 0; jj < 2; ++jj) {
           const int j = 2 * c + jj;  // group: k = 16 j .. 16 j + 15 of the block
@@ -406,9 +411,7 @@ k_decode_res(const __grid_constant__ ResParams p, const __grid_constant__ Nf4Cod
           }
         }
       }
-      if (e + 1 < n_my) cur = nxt;
-      const int64_t next_tile = e + 1 < n_my ? item_at(e + 1) / nsb : -1;
-      if (next_tile != tile) {  // end of this warp's piece of `tile`
+      if (tile_ends) {  // end of this warp's piece of `tile`
         if (!entered) {  // T and the zeroed tickets come from the preceding LoRA-down kernel
           pdl_enter();
           entered = true;
@@ -418,9 +421,15 @@ k_decode_res(const __grid_constant__ ResParams p, const __grid_constant__ Nf4Cod
         for (int h = 0; h < 2; ++h)
 #pragma unroll
           for (int m = 0; m < MT; ++m) acc[h][m][0] = acc[h][m][1] = acc[h][m][2] = acc[h][m][3] = 0.0f;
-        tile = next_tile;
-        if (tile >= 0 && lane < 16 && tile * 16 + lane < N) prefetch_l2(p.Bl + (tile * 16 + lane) * p.r);
+        if (e + 1 < n_my) {  // move to the neighbouring tile and load its first item
+          tile += step;
+          sbn = reverse ? nsb - 1 : 0;
+          set_tile(tile);
+          fetch(sbn, ca0, ca1, cb0, cb1, mA, mB);
+          if (lane < 16 && tile * 16 + lane < N) prefetch_l2(p.Bl + (tile * 16 + lane) * p.r);
+        }
       }
+      sb = sbn;
     }
   }
   // every path waits for the preceding grid before the next one may launch
@@ -431,10 +440,11 @@ k_decode_res(const __grid_constant__ ResParams p, const __grid_constant__ Nf4Cod
 
 // Work split and shared-memory plan of the X-resident kernel; ok == false when X
 // and the slots do not fit (the TMA-ring kernel then serves the call).
-ResPlan res_plan(int64_t M, int64_t N, int64_t K, int num_sms) {
+ResPlan res_plan(int64_t M, int64_t N, int64_t K, int num_sms, bool force) {
   ResPlan p{};
   p.ok = false;
   if (M < 1 || M > 16 || N < 1 || K < 64) return p;
+  if ((N + 16) * (K / 64) >= (int64_t(1) << 31)) return p;  // block indices are 32-bit in the kernel
   p.mt = M <= 8 ? 1 : 2;
   const int64_t nkb_row = K / 64;
   const int64_t nsb = (nkb_row + 3) / 4;
@@ -456,38 +466,36 @@ ResPlan res_plan(int64_t M, int64_t N, int64_t K, int num_sms) {
   int64_t xs = nsb * 4 * kXBlockBytes;
   xs = (xs + 63) / 128 * 128 + 64;
   p.x_stride = static_cast<int>(xs);
-  // reduction slots: the most tiles one warp's range touches
-  int64_t pmax = 1, ctiles = 1, maxcs = 1;
-  for (int64_t u = 0; u < p.n_units; ++u) {
-    const int64_t a = range_begin(u, p.n_items, p.n_units), b = range_begin(u + 1, p.n_items, p.n_units);
-    if (b > a) {
-      const int64_t tp = (b - 1) / nsb - a / nsb + 1;
-      if (tp > pmax) pmax = tp;
-    }
-  }
-  for (int64_t c = 0; c < p.grid; ++c) {
-    const int64_t u0 = c * kResWarps, u1 = (c + 1) * kResWarps < p.n_units ? (c + 1) * kResWarps : p.n_units;
-    if (u0 >= u1) continue;
-    const int64_t a = range_begin(u0, p.n_items, p.n_units);
-    const int64_t b = range_begin(u1, p.n_items, p.n_units);
-    if (b > a) {
-      const int64_t tc = (b - 1) / nsb - a / nsb + 1;
-      if (tc > ctiles) ctiles = tc;
-    }
-  }
-  for (int64_t tile = 0; tile < p.n_tiles; ++tile) {
-    const int64_t wf = owner_of(tile * nsb, p.n_items, p.n_units);
-    const int64_t wl = owner_of(tile * nsb + nsb - 1, p.n_items, p.n_units);
-    const int64_t cs = wl / kResWarps - wf / kResWarps + 1;
-    if (cs > maxcs) maxcs = cs;
-  }
+  // Reduction slots and counters, from bounds that need no loop over the
+  // ranges: a range of L consecutive items touches at most ceil((L - 1) / nsb)
+  // + 1 tiles, every warp range holds at most ceil(n_items / n_units) items
+  // and every CTA range at most kResWarps times that; a tile's nsb items are
+  // held by at most ceil((nsb - 1) / Lc) + 1 CTAs, Lc the fewest items of a
+  // CTA range (kResWarps * floor(n_items / n_units), or the last CTA's share).
+  const int64_t lw = (p.n_items + p.n_units - 1) / p.n_units;
+  const int64_t pmax = (lw - 1 + nsb - 1) / nsb + 1;
+  const int64_t lc_max = lw * kResWarps;
+  const int64_t ctiles = (lc_max - 1 + nsb - 1) / nsb + 1;
+  int64_t lc_min = (p.n_items / p.n_units) * kResWarps;
+  const int64_t last_units = p.n_units - static_cast<int64_t>(p.grid - 1) * kResWarps;  // warps of the last CTA
+  const int64_t last_min = (p.n_items / p.n_units) * last_units;
+  if (last_min < lc_min) lc_min = last_min;
+  if (lc_min < 1) lc_min = 1;
+  const int64_t maxcs = (nsb - 1 + lc_min - 1) / lc_min + 1;
   p.p_max = static_cast<int>(pmax);
   p.cta_tiles = static_cast<int>(ctiles);
   p.max_cta_seg = static_cast<int>(maxcs);
   const size_t xbytes = (static_cast<size_t>(M) * p.x_stride + 15) / 16 * 16;
   const size_t sbytes = static_cast<size_t>(kResWarps) * p.p_max * 32 * 4 * p.mt * sizeof(float);
   p.smem = xbytes + sbytes + static_cast<size_t>(p.cta_tiles) * 4;
-  p.ok = p.smem <= 200 * 1024;
+  // Measured crossover against the TMA-ring kernel (B200, L2-cold weights, CUDA
+  // graph replay): this kernel is faster for one token from about 16 M weights
+  // up (11008x4096: 19.7 against 22.9 us) and for 2..8 tokens from about 64 M
+  // weights up (8192x8192, M = 4: 27.8 against 31.5 us); the ring kernel keeps
+  // smaller weights and 9..16 tokens.
+  const int64_t nw = N * K;
+  const bool faster = (M == 1 && nw >= (int64_t(1) << 24)) || (M <= 8 && nw >= (int64_t(1) << 26));
+  p.ok = (faster || force) && p.smem <= static_cast<size_t>(kResSmemCap);
   return p;
 }
 
@@ -530,18 +538,18 @@ cudaError_t launch_decode_res_main(const Nf4View& w, const void* X, int64_t M, c
   cudaError_t e;
   if (rp.mt == 1) {
     if (single) {
-      if ((e = ensure_smem_limit<k_decode_res<1, true>>(smem)) != cudaSuccess) return e;
+      if ((e = ensure_smem_limit<k_decode_res<1, true>>(kResSmemCap)) != cudaSuccess) return e;
       e = launch_pdl(k_decode_res<1, true>, dim3(rp.grid), dim3(kResWarps * 32), smem, stream, p, cb);
     } else {
-      if ((e = ensure_smem_limit<k_decode_res<1, false>>(smem)) != cudaSuccess) return e;
+      if ((e = ensure_smem_limit<k_decode_res<1, false>>(kResSmemCap)) != cudaSuccess) return e;
       e = launch_pdl(k_decode_res<1, false>, dim3(rp.grid), dim3(kResWarps * 32), smem, stream, p, cb);
     }
   } else {
     if (single) {
-      if ((e = ensure_smem_limit<k_decode_res<2, true>>(smem)) != cudaSuccess) return e;
+      if ((e = ensure_smem_limit<k_decode_res<2, true>>(kResSmemCap)) != cudaSuccess) return e;
       e = launch_pdl(k_decode_res<2, true>, dim3(rp.grid), dim3(kResWarps * 32), smem, stream, p, cb);
     } else {
-      if ((e = ensure_smem_limit<k_decode_res<2, false>>(smem)) != cudaSuccess) return e;
+      if ((e = ensure_smem_limit<k_decode_res<2, false>>(kResSmemCap)) != cudaSuccess) return e;
       e = launch_pdl(k_decode_res<2, false>, dim3(rp.grid), dim3(kResWarps * 32), smem, stream, p, cb);
     }
   }

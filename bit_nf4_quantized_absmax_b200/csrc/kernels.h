@@ -108,7 +108,8 @@ struct ResPlan {
   int max_cta_seg;     // most CTAs holding pieces of one tile
   size_t smem;         // dynamic shared memory per CTA
 };
-ResPlan res_plan(int64_t M, int64_t N, int64_t K, int num_sms);
+// force: use it wherever it fits, not only where it measured faster.
+ResPlan res_plan(int64_t M, int64_t N, int64_t K, int num_sms, bool force = false);
 size_t res_partial_elems(const ResPlan& p);
 cudaError_t launch_decode_res_main(const Nf4View& w, const void* X, int64_t M, const void* B, int r, float s,
                                    void* Y, const float* T, float* partial, unsigned int* counters,
@@ -120,7 +121,10 @@ cudaError_t launch_decode_res_main(const Nf4View& w, const void* X, int64_t M, c
 cudaError_t launch_decode_fwd(const Nf4View& w, const void* X, int64_t M, const void* A, const void* B, int r,
                               float s, void* Y, float* T, float* partial, unsigned int* counters,
                               const DecodePlan& p, const ResPlan& rp, const float codebook[16], int32_t* err,
-                              cudaStream_t stream);
+                              cudaStream_t stream, const float* col_scale = nullptr);
+// col_scale (fp32 [r] or null): T's column j is multiplied by col_scale[j] as it
+// is formed (several adapters concatenated along r, each with its own scale);
+// the caller then passes s = 1.
 
 // ---- merge.cu: weighted LoRA adapters merged into the dequantized base ----
 constexpr int kMaxMergeAdapters = 8;
@@ -152,7 +156,13 @@ cudaError_t launch_gemm_lora_grad(const void* Q, int64_t R, const void* hi, cons
 cudaError_t launch_split_hilo(const float* T, int64_t M, int r, int rpad, void* hi, void* lo, int num_sms,
                               cudaStream_t stream);
 cudaError_t launch_lora_finish(const float* P, int splits, int64_t M, int r, int rpad, float s, float* f32,
-                               void* s_bf16, void* hi, void* lo, int num_sms, cudaStream_t stream);
+                               void* s_bf16, void* hi, void* lo, int num_sms, cudaStream_t stream,
+                               const float* col_scale = nullptr);
+// Several adapters concatenated along r: A_cat [sum r_a, K] (the A_a one after
+// another), B_cat [N, sum r_a] (the B_a side by side) and col_scale[j] = c_a of
+// the adapter of column j, from the adapters' A, B and c.
+cudaError_t launch_pack_adapters(const MergeAdapter* adapters, int n_adapters, int64_t N, int64_t K, void* A_cat,
+                                 void* B_cat, float* col_scale, int num_sms, cudaStream_t stream);
 cudaError_t launch_grad_reduce(const float* P, int splits, int64_t R, int rpad, int r, float s, bool transpose,
                                void* out, bool out_f32, int num_sms, cudaStream_t stream);
 cudaError_t launch_zero_bf16(void* p, int64_t n, int num_sms, cudaStream_t stream);

@@ -36,7 +36,8 @@ __global__ void k_split_hilo(const float* __restrict__ T, int64_t M, int r, int 
 // for j < rpad (zero columns stay zero). Two adjacent columns per thread.
 __global__ void k_lora_finish(const float* __restrict__ P, int splits, int64_t M, int r, int rpad, float s,
                               float* __restrict__ f32, __nv_bfloat16* __restrict__ s_bf16,
-                              __nv_bfloat16* __restrict__ hi, __nv_bfloat16* __restrict__ lo) {
+                              __nv_bfloat16* __restrict__ hi, __nv_bfloat16* __restrict__ lo,
+                              const float* __restrict__ col_scale) {
   pdl_enter();
   const int64_t n2 = M * rpad / 2;
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n2;
@@ -54,7 +55,11 @@ __global__ void k_lora_finish(const float* __restrict__ P, int splits, int64_t M
       if (j < r) f32[m * r + j] = v.x;
       if (j + 1 < r) f32[m * r + j + 1] = v.y;
     }
-    if (s_bf16) reinterpret_cast<uint32_t*>(s_bf16)[i] = pack_bf16x2(s * v.x, s * v.y);
+    if (s_bf16) {  // one scale, or one per rank column (several adapters; zero padding columns stay zero)
+      const float s0 = col_scale ? (j < r ? col_scale[j] : 0.0f) : s;
+      const float s1 = col_scale ? (j + 1 < r ? col_scale[j + 1] : 0.0f) : s;
+      reinterpret_cast<uint32_t*>(s_bf16)[i] = pack_bf16x2(s0 * v.x, s1 * v.y);
+    }
     if (hi) {
       const uint32_t h = pack_bf16x2(v.x, v.y);
       reinterpret_cast<uint32_t*>(hi)[i] = h;
@@ -161,6 +166,48 @@ __global__ void k_round_bf16(const float* __restrict__ src, __nv_bfloat16* __res
   for (int64_t i = done + t0; i < n; i += stride) dst[i] = __float2bfloat16_rn(src[i]);
 }
 
+// Several adapters side by side along r: A_cat rows are the A_a rows one
+// adapter after another, B_cat [N, rt] holds B_a in columns off_a .. off_a + r_a,
+// and col_scale[j] = c_a of column j. Plain copies (two bytes per element).
+struct PackArgs {
+  const __nv_bfloat16* A[kMaxMergeAdapters];
+  const __nv_bfloat16* B[kMaxMergeAdapters];
+  int r[kMaxMergeAdapters];
+  int off[kMaxMergeAdapters];
+  float c[kMaxMergeAdapters];
+  int n, rt;
+};
+
+__global__ void k_pack_adapters(const __grid_constant__ PackArgs a, int64_t N, int64_t K,
+                                __nv_bfloat16* __restrict__ A_cat, __nv_bfloat16* __restrict__ B_cat,
+                                float* __restrict__ col_scale) {
+  pdl_enter();
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  const int64_t t0 = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t na = static_cast<int64_t>(a.rt) * K;
+  const int64_t nb = N * a.rt;
+  for (int64_t i = t0; i < na + nb + a.rt; i += stride) {
+    if (i < na) {  // A_cat[j, k]: row j of the adapter that holds rank j
+      const int j = static_cast<int>(i / K);
+      int ad = 0;
+      while (ad + 1 < a.n && j >= a.off[ad + 1]) ++ad;
+      A_cat[i] = a.A[ad][static_cast<int64_t>(j - a.off[ad]) * K + (i - static_cast<int64_t>(j) * K)];
+    } else if (i < na + nb) {  // B_cat[n, j]
+      const int64_t e = i - na;
+      const int64_t n = e / a.rt;
+      const int j = static_cast<int>(e - n * a.rt);
+      int ad = 0;
+      while (ad + 1 < a.n && j >= a.off[ad + 1]) ++ad;
+      B_cat[e] = a.B[ad][n * a.r[ad] + (j - a.off[ad])];
+    } else {
+      const int j = static_cast<int>(i - na - nb);
+      int ad = 0;
+      while (ad + 1 < a.n && j >= a.off[ad + 1]) ++ad;
+      col_scale[j] = a.c[ad];
+    }
+  }
+}
+
 int grid_for(int64_t n, int num_sms) {
   int64_t g = (n + 255) / 256;
   const int64_t cap = static_cast<int64_t>(num_sms) * 8;
@@ -177,10 +224,30 @@ cudaError_t launch_split_hilo(const float* T, int64_t M, int r, int rpad, void* 
 }
 
 cudaError_t launch_lora_finish(const float* P, int splits, int64_t M, int r, int rpad, float s, float* f32,
-                               void* s_bf16, void* hi, void* lo, int num_sms, cudaStream_t stream) {
+                               void* s_bf16, void* hi, void* lo, int num_sms, cudaStream_t stream,
+                               const float* col_scale) {
   return launch_pdl(k_lora_finish, dim3(grid_for(M * rpad / 2, num_sms)), dim3(256), 0, stream, P, splits, M, r,
                     rpad, s, f32, static_cast<__nv_bfloat16*>(s_bf16), static_cast<__nv_bfloat16*>(hi),
-                    static_cast<__nv_bfloat16*>(lo));
+                    static_cast<__nv_bfloat16*>(lo), col_scale);
+}
+
+cudaError_t launch_pack_adapters(const MergeAdapter* adapters, int n_adapters, int64_t N, int64_t K, void* A_cat,
+                                 void* B_cat, float* col_scale, int num_sms, cudaStream_t stream) {
+  PackArgs a{};
+  int off = 0;
+  for (int i = 0; i < n_adapters; ++i) {
+    a.A[i] = static_cast<const __nv_bfloat16*>(adapters[i].A);
+    a.B[i] = static_cast<const __nv_bfloat16*>(adapters[i].B);
+    a.r[i] = adapters[i].r;
+    a.c[i] = adapters[i].c;
+    a.off[i] = off;
+    off += adapters[i].r;
+  }
+  a.n = n_adapters;
+  a.rt = off;
+  const int64_t work = static_cast<int64_t>(off) * (K + N) + off;
+  return launch_pdl(k_pack_adapters, dim3(grid_for(work, num_sms)), dim3(256), 0, stream, a, N, K,
+                    static_cast<__nv_bfloat16*>(A_cat), static_cast<__nv_bfloat16*>(B_cat), col_scale);
 }
 
 cudaError_t launch_grad_reduce(const float* P, int splits, int64_t R, int rpad, int r, float s, bool transpose,

@@ -393,6 +393,39 @@ typedef struct {
 qlora_status qlora_merge_lora(const qlora_nf4_weight* q, const qlora_lora_adapter* adapters,
                               int32_t n_adapters, void* W_out, qlora_stream_t stream);
 
+/* qlora_linear_fwd_multi -- several LoRA adapters applied at once to the same
+ * frozen weight without merging them ([C] 6: adapters trained on one quantized
+ * base are composed with weights):
+ *   Y = X W'^T + sum_a c_a (X A_a^T) B_a^T,   c_a = fp32(w_a * s_a),
+ * s_a = (float)alpha_a / (float)r_a and w_a the adapter's composition weight
+ * (the c_a of qlora_merge_lora, so that the result matches applying the merged
+ * weight up to the final bf16 rounding). The adapters are passed concatenated
+ * along the rank (qlora_pack_adapters builds the three arrays):
+ *   A_cat     : device bf16 [r_total, K], the A_a one after another.
+ *   B_cat     : device bf16 [N, r_total], the B_a side by side.
+ *   col_scale : device fp32 [r_total], c_a of the adapter of each rank column.
+ * 8 <= r_total <= 256, r_total % 8 == 0. Each rank column of T = X A_cat^T is
+ * multiplied by its scale as T is formed (fp32), then the LoRA term is added as
+ * in qlora_linear_fwd (which this equals for one adapter with c = s, up to where
+ * the scale is applied). X, M, Y, workspace and errors as in qlora_linear_fwd
+ * (no T is saved: this is the inference path). */
+qlora_status qlora_linear_fwd_multi(const qlora_nf4_weight* q, const void* X, int64_t M,
+                                    const void* A_cat, const void* B_cat, int32_t r_total,
+                                    const float* col_scale, void* Y, void* workspace,
+                                    size_t* workspace_bytes, qlora_stream_t stream);
+
+/* qlora_pack_adapters -- build the concatenated operands of
+ * qlora_linear_fwd_multi from n_adapters adapters (host array, read before the
+ * call returns; 1 <= n_adapters <= 8, each r_a in [8, 256] with r_a % 8 == 0,
+ * sum r_a <= 256) of a [rows, cols] weight: A_cat [sum r_a, cols] and B_cat
+ * [rows, sum r_a] (device bf16, 16-byte aligned, caller-owned) and col_scale
+ * [sum r_a] (device fp32) = fp32(weight_a * alpha_a / r_a) per column. One
+ * asynchronous copy kernel on `stream`; do it once per adapter set.
+ * Errors: INVALID_ARG, UNSUPPORTED, ALIGNMENT, CUDA, DEVICE. */
+qlora_status qlora_pack_adapters(const qlora_lora_adapter* adapters, int32_t n_adapters, int64_t rows,
+                                 int64_t cols, void* A_cat, void* B_cat, float* col_scale,
+                                 qlora_stream_t stream);
+
 /* qlora_paged_alloc -- allocate `bytes` of paged memory for optimizer state
  * ([C] 4: a unified pool that pages between GPU and CPU memory, so the state
  * need not be pre-allocated in device memory; [G] "Core Architecture &

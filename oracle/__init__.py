@@ -29,7 +29,7 @@ from .fp import bf16_bits_to_f32, f32_to_bf16_bits_rn, fma_f32
 from .nf4 import (BLOCK, DQ_BLOCK, nf4_codebook, fp4_codebook, quantize_nf4, dq_mean, double_quantize, quantize_nf4_dq,
                   dequantize_nf4_dq, pack_codes, unpack_codes, storage_bytes, QuantizedNF4, QuantizedNF4Single,
                   quantize_nf4_single, dequantize_nf4_single)
-from .linear import lora_scale, linear_fwd, linear_bwd
+from .linear import lora_scale, linear_fwd, linear_bwd, linear_fwd_multi
 from .merge import f64_to_bf16_bits_rn, merge_lora, merge_scale
 from .optim import adamw_step
 
@@ -38,6 +38,6 @@ __all__ = [
     "BLOCK", "DQ_BLOCK", "nf4_codebook", "fp4_codebook", "quantize_nf4", "dq_mean", "double_quantize", "quantize_nf4_dq",
     "dequantize_nf4_dq", "pack_codes", "unpack_codes", "storage_bytes", "QuantizedNF4", "QuantizedNF4Single",
     "quantize_nf4_single", "dequantize_nf4_single",
-    "lora_scale", "linear_fwd", "linear_bwd",
+    "lora_scale", "linear_fwd", "linear_bwd", "linear_fwd_multi",
     "f64_to_bf16_bits_rn", "merge_lora", "merge_scale", "adamw_step",
 ]

@@ -53,3 +53,24 @@ def linear_bwd(Wd: np.ndarray, X: np.ndarray, A: np.ndarray, B: np.ndarray, dY: 
     dA = s * (U.T @ X)
     dB = s * (dY.T @ (X @ A.T))
     return dX, dA, dB
+
+
+def linear_fwd_multi(Wd: np.ndarray, X: np.ndarray, adapters) -> np.ndarray:
+    """Several adapters applied at once without merging them ("QLoRA vs
+    ChatGPT", capability 6: adapters trained on one quantized base are composed
+    with weights): Y = X W'^T + sum_a c_a (X A_a^T) B_a^T in fp64, with
+    c_a = fp32(w_a * fp32(alpha_a / r_a)), the composition scale of the merge.
+
+    adapters: sequence of (A_a [r_a, K], B_a [N, r_a], alpha_a, w_a).
+    Reading: the pages name the composition, not its arithmetic; the scale of an
+    adapter is the one its merge into the weights uses. Returns Y [M, N].
+    """
+    Wd, X = np.asarray(Wd, dtype=np.float64), np.asarray(X, dtype=np.float64)
+    Y = X @ Wd.T
+    for A, B, alpha, w in adapters:
+        A, B = np.asarray(A, dtype=np.float64), np.asarray(B, dtype=np.float64)
+        s = np.float32(np.float32(alpha) / np.float32(A.shape[0]))
+        c = np.float64(np.float32(np.float32(w) * s))
+        Y = Y + c * ((X @ A.T) @ B.T)
+    return Y
+
