@@ -103,6 +103,14 @@ float lora_scale(float alpha, int32_t r) { return alpha / static_cast<float>(r);
 // environment selects the TMA-ring kernel for every shape, =1 the X-resident
 // kernel wherever it fits (for comparisons and tests); unset, the measured
 // crossover decides.
+// Training forward and dX with W' decoded inside the 2-CTA GEMMs
+// (QLORA_FWD_FUSED=1) instead of a dequant launch and a GEMM over the
+// dequantized copy; M >= 256.
+bool fused_forward(int64_t M) {
+  const char* e = std::getenv("QLORA_FWD_FUSED");
+  return M >= 256 && e && e[0] == '1';
+}
+
 int res_mode() {
   const char* e = std::getenv("QLORA_DECODE_RES");
   if (e && e[0] == '0') return 0;
@@ -221,7 +229,9 @@ qlora_status linear_bwd_impl(const qlora_nf4_weight* q, const void* X, int64_t M
   if (e == cudaSuccess) e = launch_grad_reduce(P, splits_b, N, rpad, r, s, false, dB, f32, di.num_sms, cs);
   // the LoRA gradients are complete: a cross-rank sum may start while dX runs
   if (e == cudaSuccess && grads_ready) e = cudaEventRecord(grads_ready, cs);
-  if (dX) {
+  if (dX && fused_forward(M)) {  // W' decoded inside the GEMM
+    if (e == cudaSuccess) e = launch_gemm_dx_nf4(dY, view(q), sU, A, M, r, rpad, dX, cb, di.num_sms, err, cs);
+  } else if (dX) {
     void* Wd = ws + off_wd;
     if (e == cudaSuccess)
       e = launch_dequantize(view(q), Wd, cb, di.num_sms, cs);
@@ -253,7 +263,7 @@ qlora_status quantize_dq_impl(const void* W_bf16, const qlora_nf4_weight* q, int
   if (W_bf16 && !aligned(W_bf16, 16)) return QLORA_ERR_ALIGNMENT;
   const int64_t numel = q->rows * q->cols;
   const int64_t nblk = numel / 64;
-  const size_t off_absmax = align_up(kQuantScratchBytes);
+  const size_t off_absmax = align_up(kQuantScratchAllBytes);
   const size_t need = off_absmax + align_up(static_cast<size_t>(nblk) * sizeof(float));
   bool launch = false;
   st = workspace_check(workspace, workspace_bytes, need, &launch);
@@ -329,6 +339,13 @@ qlora_status linear_fwd_impl(const qlora_nf4_weight* q, const void* X, int64_t M
   void* sT = ws + off_sT;
   float* P = reinterpret_cast<float*>(ws + off_part);
   const int splits_t = red_splits(M, rpad, K, kRefSms);
+  if (fused_forward(M)) {  // W' decoded inside the GEMM: no dequantized copy
+    cudaError_t e = launch_gemm_lora_t(X, A, M, K, r, rpad, P, splits_t, di.num_sms, err, cs);
+    if (e == cudaSuccess)
+      e = launch_lora_finish(P, splits_t, M, r, rpad, s, T_save, sT, nullptr, nullptr, di.num_sms, cs, col_scale);
+    if (e == cudaSuccess) e = launch_gemm_fwd_nf4(X, view(q), sT, B, M, r, rpad, Y, cb, di.num_sms, err, cs);
+    return cuda_status(e);
+  }
   cudaError_t e = launch_dequantize(view(q), Wd, cb, di.num_sms, cs);
   if (e == cudaSuccess) e = launch_gemm_lora_t(X, A, M, K, r, rpad, P, splits_t, di.num_sms, err, cs);
   if (e == cudaSuccess)

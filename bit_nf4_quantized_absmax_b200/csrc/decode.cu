@@ -380,14 +380,15 @@ k_decode(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUten
 
 // T[m, j] = sum_k X[m, k] A[j, k] for M <= 16 (fp32 on CUDA cores), one CTA per
 // adapter row j, 16-byte loads (8 k per thread and step). Block 0 also clears
-// the decode kernel's ticket counters. Small CTAs (128 threads, at most 64
-// registers each) so that one fits on an SM beside a CTA of either decode kernel.
-constexpr int kLoraDownThreads = 128;
-template <int MT>
-__global__ void __launch_bounds__(kLoraDownThreads, 8)
+// the decode kernel's ticket counters. NT threads: 256 before the TMA-ring
+// decode kernel; 128 with at most 64 registers before the X-resident one, so
+// that one CTA of it fits on an SM beside a CTA of that kernel.
+template <int MT, int NT>
+__global__ void __launch_bounds__(NT, NT == 128 ? 8 : 1)
 k_lora_t_small(const __nv_bfloat16* __restrict__ X, const __nv_bfloat16* __restrict__ A, int M, int64_t K, int r,
                float* __restrict__ T, unsigned int* __restrict__ counters, int64_t n_counters,
                const float* __restrict__ col_scale) {
+  constexpr int kLoraDownThreads = NT;
   __shared__ float red[kLoraDownThreads / 32][8 * MT];
   pdl_enter();  // after this, the decode kernel may start its main loop
   const int j = blockIdx.x;
@@ -489,7 +490,7 @@ cudaError_t launch_decode_fwd(const Nf4View& w, const void* X, int64_t M, const 
                               const DecodePlan& p, const ResPlan& rp, const float codebook[16], int32_t* err,
                               cudaStream_t stream, const float* col_scale) {
   if (rp.ok) {  // token values resident in shared memory (decode_res.cu)
-    cudaError_t e = launch_pdl(rp.mt == 1 ? k_lora_t_small<1> : k_lora_t_small<2>, dim3(r), dim3(kLoraDownThreads), 0, stream,
+    cudaError_t e = launch_pdl(rp.mt == 1 ? k_lora_t_small<1, 128> : k_lora_t_small<2, 128>, dim3(r), dim3(128), 0, stream,
                                reinterpret_cast<const __nv_bfloat16*>(X), reinterpret_cast<const __nv_bfloat16*>(A),
                                static_cast<int>(M), w.K, r, T, counters, rp.n_tiles, col_scale);
     if (e != cudaSuccess) return e;
@@ -506,7 +507,7 @@ cudaError_t launch_decode_fwd(const Nf4View& w, const void* X, int64_t M, const 
       !encode_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, static_cast<uint64_t>(w.K), static_cast<uint64_t>(M),
                  static_cast<uint64_t>(w.K) * 2, 64u, 8u * p.mt))
     return cudaErrorInvalidValue;
-  cudaError_t e = launch_pdl(p.mt == 1 ? k_lora_t_small<1> : k_lora_t_small<2>, dim3(r), dim3(kLoraDownThreads), 0, stream,
+  cudaError_t e = launch_pdl(p.mt == 1 ? k_lora_t_small<1, 256> : k_lora_t_small<2, 256>, dim3(r), dim3(256), 0, stream,
                              reinterpret_cast<const __nv_bfloat16*>(X), reinterpret_cast<const __nv_bfloat16*>(A),
                              static_cast<int>(M), w.K, r, T, counters, p.row_tiles, col_scale);
   if (e != cudaSuccess) return e;

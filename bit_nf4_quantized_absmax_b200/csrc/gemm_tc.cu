@@ -22,6 +22,7 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "nf4_lut.cuh"
 #include "tensor_map.h"
 
 namespace qlora {
@@ -116,6 +117,36 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, vo
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   while (!mbar_try_wait(bar, parity)) {
+    if (*abort_flag) return false;
+    if (clock64() - t0 > kWaitBoundCycles) {
+      report_error(err, code);
+      *abort_flag = 1;
+      return false;
+    }
+  }
+  return true;
+}
+
+// wait_or_abort with acquire at cluster scope: for a barrier that threads of
+// the peer CTA arrive on after writing their own shared memory, which the
+// pair's MMAs then read.
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+__device__ __forceinline__ bool wait_or_abort_cluster(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                                      int32_t* err, int32_t code) {
+  if (mbar_try_wait_cluster(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (!mbar_try_wait_cluster(bar, parity)) {
     if (*abort_flag) return false;
     if (clock64() - t0 > kWaitBoundCycles) {
       report_error(err, code);
@@ -651,6 +682,315 @@ k_tc_gemm2(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUt
 }
 
 // ---------------------------------------------------------------------------
+// Forward GEMM with the NF4 weight decoded into shared memory ("QLoRA vs
+// ChatGPT", capability 5: the frozen weight is dequantized on the fly, block by
+// block): C = X W'^T + [sT] B^T like k_tc_gemm2<false>, but the B stages of the
+// main k-blocks are written by eight decoder warps per CTA from the packed
+// codes and block constants (bit-identical W' to the standalone dequant), not
+// loaded by TMA from a dequantized copy of W' in memory. A k-block of 64 is one
+// 64-weight block of each weight row, so a lane pair decodes one row of a stage
+// (32 weights each) from 16 bytes of codes and one constant, and stores the
+// bf16 values in the 128-byte-swizzled K-major layout TMA would have written.
+// The leader CTA's full barrier of a stage counts the producer's arrival (with
+// the TMA bytes) and one arrival per decoder warp of both CTAs (the odd CTA's
+// remotely); decoder warps fence their generic stores for the async proxy
+// before arriving. The LoRA slab (sT against B) is TMA-loaded as before, and
+// the decoder warps arrive on its stages without writing.
+
+constexpr int kDecWarps = 8;     // decoder warps per group: one group fills one stage
+constexpr int kDecGroups = 2;    // groups take alternate k-blocks
+constexpr int kNf4Threads = kThreads + kDecGroups * kDecWarps * 32;
+
+struct Nf4Src {
+  const uint8_t* packed;
+  const int8_t* q;
+  const float* dqs;
+  const float* mean;
+  const float* absmax;   // single-level storage (q, dqs, mean unused) when not null
+  int64_t N, K;
+};
+
+// B_MN = false: the forward, B = W' [N, K] (K-major): the CTA's row rl of a
+// stage is weight row n0 + rl, block kb. B_MN = true: dX = dY W', B = W' with
+// the contraction along its rows (MN-major, two 64-column boxes per stage): row
+// rl of a stage is weight row 64 kb + (rl & 63), block column n0 / 64 + (rl >> 6).
+// Either way the row's 128 bytes sit at rl * 128 with the same swizzle.
+template <bool B_MN>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNf4Threads, 1)
+k_tc_gemm2_nf4(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmA2,
+               const __grid_constant__ CUtensorMap tmB2, const __grid_constant__ Nf4Src src, TileSched ts, int M,
+               int Nc, EpiParams ep, int32_t* err, const __grid_constant__ Nf4Codebook cb) {
+  using C = Cfg2<B_MN>;
+  constexpr int BN2 = 256;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
+  uint64_t* empty = full + C::STAGES;
+  uint64_t* accf = empty + C::STAGES;
+  uint64_t* acce = accf + 2;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(acce + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const int pair = blockIdx.x >> 1;
+  const int npairs = gridDim.x >> 1;
+  const int n_units = ts.tiles_m * ts.tiles_n * ts.splits;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(&full[s], 1 + 2 * kDecWarps);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&accf[a], 1);
+      mbar_init(&acce[a], 256);
+    }
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmA1);
+    prefetch_tmap(&tmA2);
+    prefetch_tmap(&tmB2);
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_holder)),
+                 "r"(C::TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();  // the peer's barriers are initialised before any remote use
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+  pdl_enter();  // inputs written by the preceding kernel are visible from here on
+
+  if (warp == 0) {
+    // ---------------- TMA producer (both CTAs): A always, B only for the slab ----------------
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int unit = pair; unit < n_units && ok; unit += npairs) {
+        int tm, tn, kb0, kb1;
+        decode_unit(ts, unit, tm, tn, kb0, kb1);
+        const int m0 = tm * 256 + static_cast<int>(rank) * 128;
+        const int n0 = tn * BN2 + static_cast<int>(rank) * 128;
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!wait_or_abort(&empty[stage], phase ^ 1u, abort_flag, err, DEV_TIMEOUT_SMEM_EMPTY)) {
+            ok = false;
+            break;
+          }
+          uint8_t* sa = smem + stage * C::STAGE_BYTES;
+          uint8_t* sb = sa + C::A_BYTES;
+          const bool slab = kb >= ts.nk1;
+          if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * (slab ? C::STAGE_BYTES : C::A_BYTES));
+          const uint32_t fbar = map_to_cta(smem_u32(&full[stage]), 0);
+          const int k0 = (slab ? kb - ts.nk1 : kb) * BK;
+          tma_load_2d_pair(sa, slab ? &tmA2 : &tmA1, fbar, k0, m0);
+          if (slab) {
+            if (B_MN) {
+              tma_load_2d_pair(sb, &tmB2, fbar, n0, k0);
+              tma_load_2d_pair(sb + 8192, &tmB2, fbar, n0 + 64, k0);
+            } else {
+              tma_load_2d_pair(sb, &tmB2, fbar, k0, n0);
+            }
+          }
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer (leader CTA only) ----------------
+    if (lane == 0 && rank == 0) {
+      constexpr uint32_t idesc = instr_desc(256, BN2, false, B_MN);
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int unit = pair; unit < n_units && ok; unit += npairs) {
+        int tm, tn, kb0, kb1;
+        decode_unit(ts, unit, tm, tn, kb0, kb1);
+        if (!wait_or_abort(&acce[acc], acc_phase ^ 1u, abort_flag, err, DEV_TIMEOUT_TMEM_EMPTY)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN2);
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!wait_or_abort_cluster(&full[stage], phase, abort_flag, err, DEV_TIMEOUT_TMA_FULL)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(smem + stage * C::STAGE_BYTES);
+          const uint32_t sb = sa + C::A_BYTES;
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k) {
+            const uint64_t da = smem_desc(sa + k * 32, 16, 1024);
+            const uint64_t db = B_MN ? smem_desc(sb + k * 2048, 8192, 1024) : smem_desc(sb + k * 32, 16, 1024);
+            mma_bf16_pair(d_tmem, da, db, idesc, (kb > kb0 || k > 0) ? 1u : 0u);
+          }
+          mma_commit_pair(&empty[stage]);
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        mma_commit_pair(&accf[acc]);
+        if (++acc == 2) {
+          acc = 0;
+          acc_phase ^= 1u;
+        }
+      }
+    }
+  } else if (warp < 6) {
+    // ---------------- epilogue (warps 2..5, both CTAs) ----------------
+    const int quarter = warp & 3;
+    const int row_in_tile = quarter * 32 + lane;
+    const uint32_t acce_leader0 = map_to_cta(smem_u32(&acce[0]), 0);
+    const uint32_t acce_leader1 = map_to_cta(smem_u32(&acce[1]), 0);
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int unit = pair; unit < n_units; unit += npairs) {
+      int tm, tn, kb0, kb1;
+      decode_unit(ts, unit, tm, tn, kb0, kb1);
+      if (!wait_or_abort(&accf[acc], acc_phase, abort_flag, err, DEV_TIMEOUT_ACCUM)) break;
+      tc_fence_after();
+      const int row = tm * 256 + static_cast<int>(rank) * 128 + row_in_tile;
+      const bool row_ok = row < M;
+#pragma unroll 1
+      for (int c = 0; c < BN2 / 32; ++c) {
+        float v[32];
+        tmem_ld32(tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
+                      static_cast<uint32_t>(acc * BN2 + c * 32),
+                  v);
+        const int col0 = tn * BN2 + c * 32;
+        if (!row_ok) continue;
+        __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(ep.C) + static_cast<int64_t>(row) * ep.ldc + col0;
+        if (col0 + 32 <= Nc && (ep.ldc % 8) == 0) {
+          uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            d4[q] = make_uint4(pack_bf16x2(v[8 * q + 0], v[8 * q + 1]), pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
+                               pack_bf16x2(v[8 * q + 4], v[8 * q + 5]), pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
+        } else {
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if (col0 + j < Nc) dst[j] = __float2bfloat16_rn(v[j]);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive_cluster(acc ? acce_leader1 : acce_leader0);
+      if (++acc == 2) {
+        acc = 0;
+        acc_phase ^= 1u;
+      }
+    }
+  } else {
+    // ---------------- decoder warps (6..13, both CTAs) ----------------
+    // lanes 2i and 2i + 1 of decoder warp d write row 16 d + i of the CTA's
+    // 128 B rows, weights 32 h .. 32 h + 31 (h = lane & 1) of the k-block
+    const int dw = (warp - 6) % kDecWarps;
+    const int group = (warp - 6) / kDecWarps;
+    const int rl = dw * 16 + (lane >> 1);
+    const int h = lane & 1;
+    const int64_t nkb = src.K / 64;
+    const bool single = src.absmax != nullptr;
+    const float mu = single ? 0.0f : __ldg(src.mean);
+    const uint32_t leader_full0 = map_to_cta(smem_u32(&full[0]), 0);
+    const uint32_t swz = static_cast<uint32_t>(rl & 7);
+    int stage = 0;
+    uint32_t phase = 0;
+    uint32_t it = 0;  // k-blocks so far (all units): group it % kDecGroups fills this one
+    bool ok = true;
+    for (int unit = pair; unit < n_units && ok; unit += npairs) {
+      int tm, tn, kb0, kb1;
+      decode_unit(ts, unit, tm, tn, kb0, kb1);
+      const int64_t n0 = static_cast<int64_t>(tn) * BN2 + static_cast<int64_t>(rank) * 128;
+      // codes and constant of the first main k-block of the tile, then one ahead
+      uint4 cur = make_uint4(0u, 0u, 0u, 0u);
+      float mcur = 0.0f;
+      auto fetch = [&](int kb, uint4& c, float& mval) {
+        const int64_t wrow = B_MN ? static_cast<int64_t>(kb) * 64 + (rl & 63) : n0 + rl;
+        const int64_t bcol = B_MN ? n0 / 64 + (rl >> 6) : kb;
+        if (kb >= ts.nk1 || wrow >= src.N || bcol >= nkb) {
+          c = make_uint4(0u, 0u, 0u, 0u);
+          mval = 0.0f;
+          return;
+        }
+        const int64_t b = wrow * nkb + bcol;
+        c = __ldg(reinterpret_cast<const uint4*>(src.packed + b * 32) + h);  // reused by every M tile: keep in L2
+        mval = single ? __ldg(src.absmax + b)
+                      : __fmaf_rn(static_cast<float>(__ldg(src.q + b)), __ldg(src.dqs + (b >> 8)), mu);
+      };
+      // this group's first k-block of the unit
+      int kbg = kb0 + static_cast<int>((static_cast<uint32_t>(group) - it) % kDecGroups);
+      fetch(kbg, cur, mcur);
+      for (int kb = kb0; kb < kb1; ++kb, ++it) {
+        if (static_cast<int>(it % kDecGroups) != group) {  // the other group's stage
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+          continue;
+        }
+        uint4 nxt;
+        float mnxt;
+        fetch(kb + kDecGroups < kb1 ? kb + kDecGroups : kb1, nxt, mnxt);
+        if (!wait_or_abort(&empty[stage], phase ^ 1u, abort_flag, err, DEV_TIMEOUT_SMEM_EMPTY)) {
+          ok = false;
+          break;
+        }
+        if (kb < ts.nk1) {
+          // decode 32 weights: bf16_rn(codebook[code] * m') for the codes of this row
+          const Nf4Lut t = make_nf4_lut(cb, mcur);
+          uint32_t o[16];
+          nf4_lookup8(t, cur.x, o + 0);
+          nf4_lookup8(t, cur.y, o + 4);
+          nf4_lookup8(t, cur.z, o + 8);
+          nf4_lookup8(t, cur.w, o + 12);
+          uint8_t* rowp = smem + stage * C::STAGE_BYTES + C::A_BYTES + rl * 128;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {  // 16-byte chunk 4 h + q of the row, 128-byte swizzle
+            const uint32_t chunk = (static_cast<uint32_t>(4 * h + q) ^ swz) * 16u;
+            *reinterpret_cast<uint4*>(rowp + chunk) = make_uint4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
+          }
+          // the tensor core reads the stage through the async proxy
+          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(leader_full0 + static_cast<uint32_t>(stage) * 8u);
+        cur = nxt;
+        mcur = mnxt;
+        if (++stage == C::STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();  // no CTA leaves while its peer may still signal it
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(C::TMEM_COLS)
+                 : "memory");
+  }
+}
+
+// ---------------------------------------------------------------------------
 // host side
 
 // 2-D bf16 tensor [outer, inner] with row stride ld (elements); box {64, box_outer}.
@@ -763,6 +1103,57 @@ cudaError_t launch_gemm_fwd(const void* X, const void* Wd, const void* sT, const
     return run_pair<false>(a1, b1, a2, b2, static_cast<int>(M), static_cast<int>(N), ep, num_sms, err, stream);
   return run<256, false, false, OUT_BF16>(a1, b1, &a2, &b2, static_cast<int>(M), static_cast<int>(N), 1, ep,
                                           num_sms, err, stream);
+}
+
+// GEMMs with W' decoded from NF4 inside the 2-CTA kernel (M >= 256):
+// forward Y[M,N] = X[M,K] dequant(w)^T + sT[M,rpad] Bl[N,r]^T (B_MN false), and
+// dX[M,K] = dY[M,N] dequant(w) + sU[M,rpad] Al[r,K] (B_MN true).
+template <bool B_MN>
+cudaError_t run_pair_nf4(const void* A1, int64_t K1, const Nf4View& w, const void* s_lora, const void* lora_w,
+                         int64_t M, int r, int rpad, void* out, const float codebook[16], int num_sms, int32_t* err,
+                         cudaStream_t stream) {
+  using C = Cfg2<B_MN>;
+  const int64_t N = w.N, K = w.K;
+  const int64_t Nc = B_MN ? K : N;  // output columns
+  Operand a1{A1, M, K1, K1, false};
+  Operand a2{s_lora, M, rpad, rpad, false};
+  Operand b2 = B_MN ? Operand{lora_w, K, r, K, true} : Operand{lora_w, N, r, r, false};
+  CUtensorMap ta1, ta2, tb2;
+  if (!map_operand(&ta1, a1, 128) || !map_operand(&ta2, a2, 128) || !map_operand(&tb2, b2, 128))
+    return cudaErrorInvalidValue;
+  TileSched ts;
+  ts.tiles_m = static_cast<int>((M + 255) / 256);
+  ts.tiles_n = static_cast<int>((Nc + 255) / 256);
+  ts.nk1 = static_cast<int>((K1 + BK - 1) / BK);
+  ts.nkb = ts.nk1 + static_cast<int>((rpad + BK - 1) / BK);
+  ts.splits = 1;
+  ts.kb_per_split = ts.nkb;
+  const int units = ts.tiles_m * ts.tiles_n;
+  int pairs = num_sms / 2;
+  if (pairs > units) pairs = units;
+  if (pairs < 1) pairs = 1;
+  Nf4Src src{w.packed, w.absmax_q, w.dq_scale, w.mean, w.absmax, N, K};
+  Nf4Codebook cb;
+  for (int i = 0; i < 16; ++i) cb.c[i] = codebook[i];
+  EpiParams ep{};
+  ep.C = out;
+  ep.ldc = Nc;
+  const cudaError_t e = ensure_smem_limit<k_tc_gemm2_nf4<B_MN>>(C::SMEM);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(k_tc_gemm2_nf4<B_MN>, dim3(2 * pairs), dim3(kNf4Threads), C::SMEM, stream, ta1, ta2, tb2, src,
+                    ts, static_cast<int>(M), static_cast<int>(Nc), ep, err, cb);
+}
+
+cudaError_t launch_gemm_fwd_nf4(const void* X, const Nf4View& w, const void* sT, const void* Bl, int64_t M, int r,
+                                int rpad, void* Y, const float codebook[16], int num_sms, int32_t* err,
+                                cudaStream_t stream) {
+  return run_pair_nf4<false>(X, w.K, w, sT, Bl, M, r, rpad, Y, codebook, num_sms, err, stream);
+}
+
+cudaError_t launch_gemm_dx_nf4(const void* dY, const Nf4View& w, const void* sU, const void* Al, int64_t M, int r,
+                               int rpad, void* dX, const float codebook[16], int num_sms, int32_t* err,
+                               cudaStream_t stream) {
+  return run_pair_nf4<true>(dY, w.N, w, sU, Al, M, r, rpad, dX, codebook, num_sms, err, stream);
 }
 
 // Backward dX: dX[M,K] = dY[M,N] W'[N,K] + sU[M,rpad] A[r,K]

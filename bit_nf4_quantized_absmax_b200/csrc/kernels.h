@@ -26,8 +26,10 @@ cudaError_t ensure_smem_limit(int bytes) {
 }
 
 // Quantize scratch besides the fp32 absmax: the 256 exponent-bin totals (u64)
-// of the exact sum of the constants.
+// of the exact sum of the constants (kQuantScratchBytes, the part a row shard's
+// caller exchanges), then a ticket counter and the mean (kQuantScratchAllBytes).
 constexpr size_t kQuantScratchBytes = 256 * sizeof(unsigned long long);
+constexpr size_t kQuantScratchAllBytes = kQuantScratchBytes + 16;
 
 // Number of non-empty pieces when `nkb` k-blocks are cut into pieces of
 // ceil(nkb / want) blocks. The split-reduction GEMMs and the kernels that sum
@@ -51,11 +53,14 @@ cudaError_t launch_quantize(const void* W, int64_t numel, uint8_t* packed, int8_
 // sum (zeroed and then added into); second, after the totals of all shards have
 // been summed, the mean over nblk_mean constants and the int8 codes and group
 // scales of this shard's nblk constants.
+// done / mean_out / mu_out (optional, together): the sums kernel also forms
+// the mean (a whole weight); mu_ready (optional): the coding kernel reads it.
 cudaError_t launch_quantize_first(const void* W, int64_t nblk, uint8_t* packed, float* absmax_scratch,
-                                  unsigned long long* totals, int num_sms, cudaStream_t stream, int dtype = 0);
+                                  unsigned long long* totals, int num_sms, cudaStream_t stream, int dtype = 0,
+                                  unsigned int* done = nullptr, float* mean_out = nullptr, float* mu_out = nullptr);
 cudaError_t launch_quantize_second(const float* absmax_scratch, int64_t nblk, const unsigned long long* totals,
                                    int64_t nblk_mean, int8_t* absmax_q, float* dq_scale, float* mean,
-                                   cudaStream_t stream);
+                                   cudaStream_t stream, const float* mu_ready = nullptr);
 
 // Single-level storage: the codes and the fp32 block constants m_b only (pass 1).
 cudaError_t launch_quantize_single(const void* W, int64_t numel, uint8_t* packed, float* absmax, int num_sms,
@@ -141,6 +146,15 @@ cudaError_t launch_merge(const Nf4View& w, const MergeAdapter* adapters, int n_a
 // ---- gemm_tc.cu: tcgen05 GEMMs ----
 cudaError_t launch_gemm_fwd(const void* X, const void* Wd, const void* sT, const void* Bl, int64_t M, int64_t N,
                             int64_t K, int r, int rpad, void* Y, int num_sms, int32_t* err, cudaStream_t stream);
+// The same forward with W' decoded from the NF4 storage inside the GEMM (no
+// dequantized copy of W' in memory); M >= 256.
+cudaError_t launch_gemm_fwd_nf4(const void* X, const Nf4View& w, const void* sT, const void* Bl, int64_t M, int r,
+                                int rpad, void* Y, const float codebook[16], int num_sms, int32_t* err,
+                                cudaStream_t stream);
+// dX with W' decoded inside the GEMM; M >= 256.
+cudaError_t launch_gemm_dx_nf4(const void* dY, const Nf4View& w, const void* sU, const void* Al, int64_t M, int r,
+                               int rpad, void* dX, const float codebook[16], int num_sms, int32_t* err,
+                               cudaStream_t stream);
 cudaError_t launch_gemm_dx(const void* dY, const void* Wd, const void* sU, const void* Al, int64_t M, int64_t N,
                            int64_t K, int r, int rpad, void* dX, int num_sms, int32_t* err, cudaStream_t stream);
 // Split-reduction partials P[splits][M][rpad] of X A^T (lora_t) and dY B (lora_u);

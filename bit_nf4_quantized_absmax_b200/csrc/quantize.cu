@@ -10,9 +10,10 @@
 //                  a 32-bin table + one compare), 4-bit packing.
 //   k_quant_sums   the exact sum of the absmax constants, as integer sums of
 //                  their 8-bit significands per exponent (order-independent).
-//   k_dq_quantize  forms the mean from those totals (every CTA, warp 0), then
-//                  one warp per 256 constants: centre on the mean, group
-//                  absmax, int8 codes with round-to-nearest-even.
+//                  The CTA that adds the last totals forms the mean from them.
+//   k_dq_quantize  one warp per 256 constants: centre on the mean, group
+//                  absmax, int8 codes with round-to-nearest-even (for a row
+//                  shard, every CTA first forms the mean from the summed totals).
 #include "common.cuh"
 #include "host_tables.h"
 #include "kernels.h"
@@ -128,13 +129,85 @@ __device__ __forceinline__ void encode16(const uint32_t (&d)[8], float ms, float
   }
 }
 
+// Fast path of encode16: the bin and the comparison from v' = RN(w * r) with
+// r = rcp.approx(m) (at most 1 ulp from 1/m), instead of the exact quotient
+// v = RN(w / m). For |w| <= m, |v' - w/m| <= 2^-23 + 2^-24 and |v - w/m| <=
+// 2^-24, so |v' - v| < 2^-22 and v' lies in [-1 - 2^-22, 1 + 2^-22]: the bin of
+// v' is a valid entry (|round(v' * 127)| <= 127), and the code from v' is the
+// nearest code of v whenever |v' - T| >= 2^-21 for the threshold T it is
+// compared with (v and v' are then on the same side of T; the rule counts the
+// thresholds at or below its input, and checks every fp32 input). Returns true
+// if some weight was within 2^-21 of its threshold; the caller then codes the
+// 16 weights again through the exact quotient.
+constexpr float kNearEps = 4.76837158203125e-07f;  // 2^-21
+
+__device__ __forceinline__ float rcp_approx(float x) {
+  float r;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
+}
+
+// The fast path reads the bin table as two arrays of 4-byte entries, the
+// thresholds T_j and the codes j + 1 (byte offset of bin b: 4 b, i.e. the low
+// byte of x's pattern shifted right by one), so each lookup of a warp touches
+// each bank once (the 8-byte entries of the exact path make bins b and b + 16
+// share banks).
+__device__ __forceinline__ bool encode16_fast(const uint32_t (&d)[8], float r, const unsigned char* tbin,
+                                              const unsigned char* cbin, uint32_t (&out)[2]) {
+  bool near = false;
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    uint32_t word = 0u;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const uint32_t bits = d[4 * k + (i >> 1)];
+      const float w = __uint_as_float((i & 1) ? (bits & 0xFFFF0000u) : (bits << 16));
+      const float v = __fmul_rn(w, r);
+      const float x = __fmaf_rn(v, kBinMul, kBinAdd);
+      const uint32_t off = (__float_as_uint(x) & 0xF8u) >> 1;
+      const float T = *reinterpret_cast<const float*>(tbin + off);
+      const uint32_t c1 = *reinterpret_cast<const uint32_t*>(cbin + off);
+      const float dv = __fsub_rn(v, T);
+      near = near || (fabsf(dv) < kNearEps);
+      const uint32_t c = c1 - __umulhi(__float_as_uint(dv), 2u);
+      word += c * (1u << (4 * i));
+    }
+    out[k] = word;
+  }
+  return near;
+}
+
+// The exact path for the rare group of 16 weights where the fast path came
+// within 2^-21 of a threshold; kept out of line so the common path keeps few
+// registers.
+__device__ __noinline__ uint2 encode16_exact(const uint4* __restrict__ src, bool v8, float m,
+                                             const unsigned char* bins) {
+  uint32_t d[8];
+  if (v8) {
+    ld_global_cs_v8(src, d);
+  } else {
+    const uint4 a = __ldcs(src), b = __ldcs(src + 1);
+    d[0] = a.x; d[1] = a.y; d[2] = a.z; d[3] = a.w; d[4] = b.x; d[5] = b.y; d[6] = b.z; d[7] = b.w;
+  }
+  uint32_t out[2];
+  encode16<false>(d, m, __frcp_rn(m), 1.0f, bins, out);
+  return make_uint2(out[0], out[1]);
+}
+
+__device__ __forceinline__ uint32_t absmax_bf16x2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
 // Four lanes per 64-weight block (16 weights each, one 32-byte load): a warp
 // reads 1 KB of contiguous weights per load instruction, and every lane of a
 // warp runs the same iterations (the block's four lanes share its absmax
 // through two shuffles).
 template <bool V8>
 __device__ __forceinline__ void pass1_loop(const uint4* __restrict__ W, int64_t nblk, uint32_t* __restrict__ packed,
-                                           float* __restrict__ absmax, const unsigned char* bins) {
+                                           float* __restrict__ absmax, const unsigned char* bins,
+                                           const unsigned char* tbin, const unsigned char* cbin) {
   const int lane = threadIdx.x & 31;
   const int qtr = lane & 3;
   const int64_t stride = static_cast<int64_t>(gridDim.x) * (kPass1Threads / 4);
@@ -154,10 +227,13 @@ __device__ __forceinline__ void pass1_loop(const uint4* __restrict__ W, int64_t 
 #pragma unroll
       for (int i = 0; i < 8; ++i) d[i] = 0u;
     }
-    // absmax on the bit patterns: for finite bf16, |w| orders as the unsigned 15-bit magnitude field
-    uint32_t mx = d[0] & 0x7FFF7FFFu;
+    // absmax: packed max of |w| (the sign bits of the result are dropped), then
+    // the two halves as unsigned 15-bit magnitude fields (for finite bf16, |w|
+    // orders as that field)
+    uint32_t mx = absmax_bf16x2(d[0], d[1]);
 #pragma unroll
-    for (int i = 1; i < 8; ++i) mx = max_u16x2(mx, d[i] & 0x7FFF7FFFu);
+    for (int i = 2; i < 8; ++i) mx = absmax_bf16x2(mx, d[i]);
+    mx &= 0x7FFF7FFFu;
     mx = max(mx & 0xFFFFu, mx >> 16);
     mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
     mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
@@ -173,7 +249,11 @@ __device__ __forceinline__ void pass1_loop(const uint4* __restrict__ W, int64_t 
         // to the zero code either way).
         const bool rare = m < 5.421010862e-20f || m > 1.8446744e19f;  // outside [2^-64, 2^64]
         if (!rare) {
-          encode16<false>(d, m, __frcp_rn(m), 1.0f, bins, out);
+          if (encode16_fast(d, rcp_approx(m), tbin, cbin, out)) {  // rare: reload and code exactly
+            const uint2 o = encode16_exact(W + blk * 8 + qtr * 2, V8, m, bins);
+            out[0] = o.x;
+            out[1] = o.y;
+          }
         } else {
           const float wsc = m < 5.421010862e-20f ? 1.8446744e19f : 5.421010862e-20f;
           const float ms = m * wsc;
@@ -189,20 +269,28 @@ __device__ __forceinline__ void pass1_loop(const uint4* __restrict__ W, int64_t 
 // k_quant_sums adds into, cleared here by CTA 0 before that kernel starts.
 __global__ void __launch_bounds__(kPass1Threads)
 k_quant_pass1(const uint4* __restrict__ W, bool v8, uint32_t* __restrict__ packed,
-              float* __restrict__ absmax, unsigned long long* __restrict__ zero_totals, int64_t nblk,
-              const __grid_constant__ QuantBinTable tab) {
+              float* __restrict__ absmax, unsigned long long* __restrict__ zero_totals,
+              unsigned int* __restrict__ zero_done, int64_t nblk, const __grid_constant__ QuantBinTable tab) {
   __shared__ uint2 s_bins[kBins];
+  __shared__ uint32_t s_tbin[kBins], s_cbin[kBins];
   const int tid = threadIdx.x;
-  if (tid < kBins) s_bins[tid] = make_uint2(__float_as_uint(tab.bins[tid].threshold), tab.bins[tid].j + 1u);
+  if (tid < kBins) {
+    s_bins[tid] = make_uint2(__float_as_uint(tab.bins[tid].threshold), tab.bins[tid].j + 1u);
+    s_tbin[tid] = __float_as_uint(tab.bins[tid].threshold);
+    s_cbin[tid] = tab.bins[tid].j + 1u;
+  }
   __syncthreads();
   pdl_enter();
   if (zero_totals && blockIdx.x == 0) zero_totals[tid] = 0ull;  // kPass1Threads == 256 bins
+  if (zero_done && blockIdx.x == 0 && tid == 0) *zero_done = 0u;
 
   const unsigned char* bins = reinterpret_cast<const unsigned char*>(s_bins);
+  const unsigned char* tbin = reinterpret_cast<const unsigned char*>(s_tbin);
+  const unsigned char* cbin = reinterpret_cast<const unsigned char*>(s_cbin);
   if (v8)
-    pass1_loop<true>(W, nblk, packed, absmax, bins);
+    pass1_loop<true>(W, nblk, packed, absmax, bins, tbin, cbin);
   else
-    pass1_loop<false>(W, nblk, packed, absmax, bins);
+    pass1_loop<false>(W, nblk, packed, absmax, bins, tbin, cbin);
 }
 
 // totals[e] += the 8-bit significands of the constants with exponent bin e (a
@@ -211,10 +299,19 @@ k_quant_pass1(const uint4* __restrict__ W, bool v8, uint32_t* __restrict__ packe
 // overflow; lanes that share a bin add first (match + reduce), then one shared
 // atomic; then one 64-bit global atomic per nonzero bin. Integer additions in
 // any order give the same totals.
+__device__ float mean_from_bins(const unsigned long long* __restrict__ totals, int64_t nblk, float* mean_out,
+                                bool store);
+
+// done (optional, zeroed by pass 1): the CTA that adds the last bin totals
+// (ticket) also forms the mean mu = fp32(RN_fp64(S) / nblk) from them, stores
+// it in mean_out (the weight's mean) and mu_out (for k_dq_quantize), so that
+// the coding kernel does not form it in every CTA.
 __global__ void __launch_bounds__(256)
 k_quant_sums(const float* __restrict__ absmax, int64_t nblk, int64_t per_cta,
-             unsigned long long* __restrict__ totals) {
+             unsigned long long* __restrict__ totals, unsigned int* __restrict__ done, float* __restrict__ mean_out,
+             float* __restrict__ mu_out) {
   __shared__ unsigned int s_hist[256];
+  __shared__ unsigned int s_last;
   s_hist[threadIdx.x] = 0u;
   __syncthreads();
   pdl_enter();
@@ -237,12 +334,24 @@ k_quant_sums(const float* __restrict__ absmax, int64_t nblk, int64_t per_cta,
   __syncthreads();
   const unsigned int v = s_hist[threadIdx.x];
   if (v) atomicAdd(&totals[threadIdx.x], static_cast<unsigned long long>(v));
+  if (!done) return;
+  __syncthreads();  // every bin of this CTA is added before its ticket
+  if (threadIdx.x == 0) {
+    unsigned int old;
+    asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], 1;" : "=r"(old) : "l"(done) : "memory");
+    s_last = old == gridDim.x - 1 ? 1u : 0u;
+  }
+  __syncthreads();
+  if (!s_last) return;
+  const float mu = mean_from_bins(totals, nblk, mean_out, true);
+  if (threadIdx.x == 0) *mu_out = mu;
 }
 
 // mu = fp32(RN_fp64(S) / nblk) from the exact bin totals (warp 0 of the CTA);
 // CTA 0 also stores it. nblk counts every constant the totals cover (the whole
 // tensor when this call only codes one shard of its constants).
-__device__ float mean_from_bins(const unsigned long long* __restrict__ totals, int64_t nblk, float* mean_out) {
+__device__ float mean_from_bins(const unsigned long long* __restrict__ totals, int64_t nblk, float* mean_out,
+                                bool store) {
   __shared__ unsigned long long s_tot[256];
   __shared__ unsigned int s_mask[8];
   __shared__ float s_mu;
@@ -250,7 +359,7 @@ __device__ float mean_from_bins(const unsigned long long* __restrict__ totals, i
     const int lane = threadIdx.x;
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
-      const unsigned long long x = totals[32 * k + lane];
+      const unsigned long long x = __ldcg(totals + 32 * k + lane);  // the atomics' results, from L2
       s_tot[32 * k + lane] = x;
       const unsigned int m = __ballot_sync(0xffffffffu, x != 0ull);
       if (lane == 0) s_mask[k] = m;
@@ -269,7 +378,7 @@ __device__ float mean_from_bins(const unsigned long long* __restrict__ totals, i
       const double S = limbs_to_double(L);
       const float mu = __double2float_rn(__ddiv_rn(S, static_cast<double>(nblk)));
       s_mu = mu;
-      if (blockIdx.x == 0) *mean_out = mu;
+      if (store) *mean_out = mu;
     }
   }
   __syncthreads();
@@ -279,9 +388,12 @@ __device__ float mean_from_bins(const unsigned long long* __restrict__ totals, i
 __global__ void __launch_bounds__(256)
 k_dq_quantize(const float* __restrict__ absmax, int64_t nblk, const unsigned long long* __restrict__ totals,
               int64_t nblk_mean, float* __restrict__ mean_out, int8_t* __restrict__ q, float* __restrict__ dq_scale,
-              int64_t ngrp) {
+              int64_t ngrp, const float* __restrict__ mu_ready) {
   pdl_enter();
-  const float mu = mean_from_bins(totals, nblk_mean, mean_out);
+  // the mean: formed by the sums kernel when it could (one weight on one GPU),
+  // else here from the bin totals (a row shard, after the totals of all shards
+  // were added), stored by CTA 0
+  const float mu = mu_ready ? __ldcg(mu_ready) : mean_from_bins(totals, nblk_mean, mean_out, blockIdx.x == 0);
   const int lane = threadIdx.x & 31;
   const int64_t g = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
   if (g >= ngrp) return;  // whole warp leaves together
@@ -350,21 +462,22 @@ int pass1_grid(int64_t nblk, int num_sms) {
 }
 
 cudaError_t launch_pass1(const void* W, int64_t nblk, uint8_t* packed, float* absmax, unsigned long long* zero_totals,
-                         int num_sms, cudaStream_t stream, int dtype) {
+                         unsigned int* zero_done, int num_sms, cudaStream_t stream, int dtype) {
   const QuantTables& tabs = quant_tables(dtype);
   QuantBinTable tab;
   for (int i = 0; i < kBins; ++i) tab.bins[i] = tabs.bins[i];
   const bool v8 = ((reinterpret_cast<uintptr_t>(W) | reinterpret_cast<uintptr_t>(packed)) & 31u) == 0;
   return launch_pdl(k_quant_pass1, dim3(pass1_grid(nblk, num_sms)), dim3(kPass1Threads), 0, stream,
                     reinterpret_cast<const uint4*>(W), v8, reinterpret_cast<uint32_t*>(packed), absmax, zero_totals,
-                    nblk, tab);
+                    zero_done, nblk, tab);
 }
 
 }  // namespace
 
 cudaError_t launch_quantize_first(const void* W, int64_t nblk, uint8_t* packed, float* absmax_scratch,
-                                  unsigned long long* totals, int num_sms, cudaStream_t stream, int dtype) {
-  cudaError_t e = launch_pass1(W, nblk, packed, absmax_scratch, totals, num_sms, stream, dtype);
+                                  unsigned long long* totals, int num_sms, cudaStream_t stream, int dtype,
+                                  unsigned int* done, float* mean_out, float* mu_out) {
+  cudaError_t e = launch_pass1(W, nblk, packed, absmax_scratch, totals, done, num_sms, stream, dtype);
   if (e != cudaSuccess) return e;
   // chunks of at least 512 constants and at most 8 CTAs per SM (the loop of a
   // CTA is latency bound, so many short chunks beat few long ones), at most
@@ -377,17 +490,17 @@ cudaError_t launch_quantize_first(const void* W, int64_t nblk, uint8_t* packed, 
   if (g > 0x7fffffff) return cudaErrorInvalidValue;
   const int64_t per_cta = (nblk + g - 1) / g;
   return launch_pdl(k_quant_sums, dim3(static_cast<unsigned>(g)), dim3(256), 0, stream,
-                    static_cast<const float*>(absmax_scratch), nblk, per_cta, totals);
+                    static_cast<const float*>(absmax_scratch), nblk, per_cta, totals, done, mean_out, mu_out);
 }
 
 cudaError_t launch_quantize_second(const float* absmax_scratch, int64_t nblk, const unsigned long long* totals,
                                    int64_t nblk_mean, int8_t* absmax_q, float* dq_scale, float* mean,
-                                   cudaStream_t stream) {
+                                   cudaStream_t stream, const float* mu_ready) {
   const int64_t ngrp = (nblk + 255) / 256;
   const int64_t dq_grid = (ngrp + 7) / 8;
   if (dq_grid > 0x7fffffff) return cudaErrorInvalidValue;
   return launch_pdl(k_dq_quantize, dim3(static_cast<unsigned>(dq_grid)), dim3(256), 0, stream, absmax_scratch,
-                    nblk, totals, nblk_mean, mean, absmax_q, dq_scale, ngrp);
+                    nblk, totals, nblk_mean, mean, absmax_q, dq_scale, ngrp, mu_ready);
 }
 
 cudaError_t launch_quantize(const void* W, int64_t numel, uint8_t* packed, int8_t* absmax_q, float* dq_scale,
@@ -395,6 +508,10 @@ cudaError_t launch_quantize(const void* W, int64_t numel, uint8_t* packed, int8_
                             cudaStream_t stream, int dtype) {
   const int64_t nblk = numel / 64;
   unsigned long long* totals = static_cast<unsigned long long*>(totals_scratch);
+  // (Forming the mean once, in the CTA of k_quant_sums that adds the last
+  // totals, measured slower than forming it in every CTA of k_dq_quantize:
+  // 43.6 against 41.9 us for 11008x4096, its ticket and the mean's store and
+  // load add round trips to the critical path.)
   cudaError_t e = launch_quantize_first(W, nblk, packed, absmax_scratch, totals, num_sms, stream, dtype);
   if (e != cudaSuccess) return e;
   return launch_quantize_second(absmax_scratch, nblk, totals, nblk, absmax_q, dq_scale, mean, stream);
@@ -402,7 +519,7 @@ cudaError_t launch_quantize(const void* W, int64_t numel, uint8_t* packed, int8_
 
 cudaError_t launch_quantize_single(const void* W, int64_t numel, uint8_t* packed, float* absmax, int num_sms,
                                    cudaStream_t stream, int dtype) {
-  return launch_pass1(W, numel / 64, packed, absmax, nullptr, num_sms, stream, dtype);
+  return launch_pass1(W, numel / 64, packed, absmax, nullptr, nullptr, num_sms, stream, dtype);
 }
 
 }  // namespace qlora

@@ -1,6 +1,6 @@
 // Exhaustive host check of the quantize kernel's binning rule, for the NF4 and
-// the FP4 tables: for every fp32 v in [-1, 1], the code the kernel forms from
-// its 32-bin table,
+// the FP4 tables: for every fp32 v in [-1 - 2^-19, 1 + 2^-19], the code the
+// kernel forms from its 32-bin table,
 //   x = fmaf(v, kBinMul, kBinAdd), entry = bins[(bits(x) & 0xF8) >> 3],
 //   code = (entry.j + 1) - [RN(v - entry.threshold) < 0],
 // must equal the number of decision thresholds T_i with v >= T_i (the nearest
@@ -42,7 +42,9 @@ static uint64_t check_range(uint32_t lo, uint32_t hi, int sign, int dtype) {
 }
 
 int main() {
-  const uint32_t end = 0x3F800001u;  // every bit pattern of [+0, 1]
+  // every bit pattern of [+0, 1 + 2^-19]: the quantize kernel's fast path feeds
+  // the rule RN(w * rcp.approx(m)), which can exceed 1 by less than 2^-22
+  const uint32_t end = 0x3F800011u;
   const unsigned nt = std::thread::hardware_concurrency() ? std::thread::hardware_concurrency() : 4;
   uint64_t total = 0;
   for (int dtype : {kDtypeNf4, kDtypeFp4}) {
