@@ -384,7 +384,7 @@ k_decode(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUten
 // decode kernel; 128 with at most 64 registers before the X-resident one, so
 // that one CTA of it fits on an SM beside a CTA of that kernel.
 template <int MT, int NT>
-__global__ void __launch_bounds__(NT, NT == 128 ? 8 : 1)
+__global__ void __launch_bounds__(NT, NT < 256 ? 16 * 64 / NT : 1)
 k_lora_t_small(const __nv_bfloat16* __restrict__ X, const __nv_bfloat16* __restrict__ A, int M, int64_t K, int r,
                float* __restrict__ T, unsigned int* __restrict__ counters, int64_t n_counters,
                const float* __restrict__ col_scale) {
