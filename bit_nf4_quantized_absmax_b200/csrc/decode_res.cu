@@ -28,11 +28,16 @@
 // (the reduction index is permuted, X alike), so each lane decodes whole
 // 64-weight blocks with one 16-entry bf16 table per block, bit-identical to the
 // standalone dequant. A lane loads its two blocks' codes (2 x 32 bytes) with
-// plain global loads one item ahead, and prefetches the item after that into
-// L2.
+// plain global loads one item ahead (also across tiles), and prefetches the
+// item after that into L2.
+//
+// The LoRA term of a tile, s (T B^T) for its 16 rows, is added to the piece of
+// the warp that decodes the tile's last superblock, right after that item, so
+// that the warp completing the tile only sums the pieces and stores Y.
 //
 // Every sum runs in an order fixed by the shapes (pieces in warp order within a
-// CTA, then CTAs in order), so repeated calls give identical bits.
+// CTA, then CTAs in order; the LoRA term in one fixed piece), so repeated calls
+// give identical bits.
 #include "common.cuh"
 #include "kernels.h"
 #include "nf4_lut.cuh"
@@ -134,59 +139,82 @@ __host__ __device__ inline size_t res_slot_off(const ResParams& p) {
   return (static_cast<size_t>(p.M) * p.x_stride + 15) / 16 * 16;
 }
 
+// LoRA term of one tile, added to the partial sums of the warp that decodes the
+// tile's last superblock: acc[m][i] = fmaf(s, l, acc[m][i]) with l = (T B^T)
+// for this lane's rows and tokens. Rows of B are the A operand, T^T (split into
+// bf16 hi + lo) the B operand. Ranks go in chunks of 64 with every load of a
+// chunk issued before its MMAs (one round trip to L2 per chunk). A step covers
+// ranks j0 .. j0 + 15; since r % 8 == 0 its upper half is either wholly inside
+// [0, r) or wholly outside (and then zero).
 template <int MT>
-__device__ __forceinline__ void lora_up_store(const float (&y)[MT][4], int64_t tile, int lane, const ResParams& p) {
+__device__ __forceinline__ void lora_accumulate(float (&acc)[MT][4], int64_t tile, int lane, const ResParams& p) {
   const int g = lane >> 2, t = lane & 3;
   const int64_t na = tile * 16 + g, nb = na + 8;
   const int r = p.r;
   float l[MT][4];
 #pragma unroll
   for (int m = 0; m < MT; ++m) l[m][0] = l[m][1] = l[m][2] = l[m][3] = 0.0f;
-  // LoRA up: rows of B are the A operand, T^T (split into bf16 hi + lo) the B
-  // operand. A step covers ranks j0 .. j0 + 15; since r % 8 == 0 its upper half
-  // is either wholly inside [0, r) or wholly outside (and then zero).
-  for (int j0 = 0; j0 < r; j0 += 16) {
-    const bool hi_in = j0 + 8 < r;
-    const __nv_bfloat16* Ba = p.Bl + na * r + j0 + 2 * t;
-    const __nv_bfloat16* Bb = p.Bl + nb * r + j0 + 2 * t;
-    const uint32_t b_a0 = na < p.N ? *reinterpret_cast<const uint32_t*>(Ba) : 0u;
-    const uint32_t b_a2 = na < p.N && hi_in ? *reinterpret_cast<const uint32_t*>(Ba + 8) : 0u;
-    const uint32_t b_a1 = nb < p.N ? *reinterpret_cast<const uint32_t*>(Bb) : 0u;
-    const uint32_t b_a3 = nb < p.N && hi_in ? *reinterpret_cast<const uint32_t*>(Bb + 8) : 0u;
+  for (int c0 = 0; c0 < r; c0 += 64) {
+    uint32_t bv[4][4];
+    float tv[4][MT][4];
 #pragma unroll
-    for (int m = 0; m < MT; ++m) {
-      const int tok = g + 8 * m;
-      float tv[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-      if (tok < p.M) {
+    for (int q = 0; q < 4; ++q) {
+      const int j0 = c0 + 16 * q;
+      const bool lo_in = j0 < r, hi_in = j0 + 8 < r;
+      const __nv_bfloat16* Ba = p.Bl + na * r + j0 + 2 * t;
+      const __nv_bfloat16* Bb = p.Bl + nb * r + j0 + 2 * t;
+      bv[q][0] = na < p.N && lo_in ? *reinterpret_cast<const uint32_t*>(Ba) : 0u;
+      bv[q][1] = nb < p.N && lo_in ? *reinterpret_cast<const uint32_t*>(Bb) : 0u;
+      bv[q][2] = na < p.N && hi_in ? *reinterpret_cast<const uint32_t*>(Ba + 8) : 0u;
+      bv[q][3] = nb < p.N && hi_in ? *reinterpret_cast<const uint32_t*>(Bb + 8) : 0u;
+#pragma unroll
+      for (int m = 0; m < MT; ++m) {
+        const int tok = g + 8 * m;
         const float* tp = p.T + static_cast<int64_t>(tok) * r + j0 + 2 * t;
-        tv[0] = __ldcg(tp);
-        tv[1] = __ldcg(tp + 1);
-        if (hi_in) {
-          tv[2] = __ldcg(tp + 8);
-          tv[3] = __ldcg(tp + 9);
-        }
+        const bool tin = tok < p.M;
+        tv[q][m][0] = tin && lo_in ? __ldcg(tp) : 0.0f;
+        tv[q][m][1] = tin && lo_in ? __ldcg(tp + 1) : 0.0f;
+        tv[q][m][2] = tin && hi_in ? __ldcg(tp + 8) : 0.0f;
+        tv[q][m][3] = tin && hi_in ? __ldcg(tp + 9) : 0.0f;
       }
-      uint32_t hi[2], lo[2];
+    }
 #pragma unroll
-      for (int q = 0; q < 2; ++q) {
-        const uint32_t h = pack_bf16x2(tv[2 * q], tv[2 * q + 1]);
-        hi[q] = h;
-        lo[q] = pack_bf16x2(tv[2 * q] - bf16lo_to_f32(h), tv[2 * q + 1] - bf16hi_to_f32(h));
+    for (int q = 0; q < 4; ++q) {
+#pragma unroll
+      for (int m = 0; m < MT; ++m) {
+        uint32_t hi[2], lo[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const uint32_t x = pack_bf16x2(tv[q][m][2 * h], tv[q][m][2 * h + 1]);
+          hi[h] = x;
+          lo[h] = pack_bf16x2(tv[q][m][2 * h] - bf16lo_to_f32(x), tv[q][m][2 * h + 1] - bf16hi_to_f32(x));
+        }
+        mma16816r(l[m], bv[q][0], bv[q][1], bv[q][2], bv[q][3], hi[0], hi[1]);
+        mma16816r(l[m], bv[q][0], bv[q][1], bv[q][2], bv[q][3], lo[0], lo[1]);
       }
-      mma16816r(l[m], b_a0, b_a1, b_a2, b_a3, hi[0], hi[1]);
-      mma16816r(l[m], b_a0, b_a1, b_a2, b_a3, lo[0], lo[1]);
     }
   }
+#pragma unroll
+  for (int m = 0; m < MT; ++m)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) acc[m][i] = __fmaf_rn(p.s, l[m][i], acc[m][i]);
+}
+
+// Y of this lane's rows and tokens (tokens >= M and rows >= N are not stored).
+template <int MT>
+__device__ __forceinline__ void store_y(const float (&y)[MT][4], int64_t tile, int lane, const ResParams& p) {
+  const int g = lane >> 2, t = lane & 3;
+  const int64_t na = tile * 16 + g, nb = na + 8;
 #pragma unroll
   for (int m = 0; m < MT; ++m) {
     const int tok0 = 8 * m + 2 * t, tok1 = tok0 + 1;
     if (na < p.N) {
-      if (tok0 < p.M) p.Y[static_cast<int64_t>(tok0) * p.N + na] = __float2bfloat16_rn(fmaf(p.s, l[m][0], y[m][0]));
-      if (tok1 < p.M) p.Y[static_cast<int64_t>(tok1) * p.N + na] = __float2bfloat16_rn(fmaf(p.s, l[m][1], y[m][1]));
+      if (tok0 < p.M) p.Y[static_cast<int64_t>(tok0) * p.N + na] = __float2bfloat16_rn(y[m][0]);
+      if (tok1 < p.M) p.Y[static_cast<int64_t>(tok1) * p.N + na] = __float2bfloat16_rn(y[m][1]);
     }
     if (nb < p.N) {
-      if (tok0 < p.M) p.Y[static_cast<int64_t>(tok0) * p.N + nb] = __float2bfloat16_rn(fmaf(p.s, l[m][2], y[m][2]));
-      if (tok1 < p.M) p.Y[static_cast<int64_t>(tok1) * p.N + nb] = __float2bfloat16_rn(fmaf(p.s, l[m][3], y[m][3]));
+      if (tok0 < p.M) p.Y[static_cast<int64_t>(tok0) * p.N + nb] = __float2bfloat16_rn(y[m][2]);
+      if (tok1 < p.M) p.Y[static_cast<int64_t>(tok1) * p.N + nb] = __float2bfloat16_rn(y[m][3]);
     }
   }
 }
@@ -195,22 +223,23 @@ __device__ __forceinline__ void lora_up_store(const float (&y)[MT][4], int64_t t
 // shared slot; the last of the CTA's warps holding pieces of the tile sums them
 // in warp order. A tile that other CTAs hold pieces of too goes on through a
 // global slot and ticket; the CTA that brings the last piece sums the CTAs'
-// pieces in CTA order. Whoever completes the tile adds the LoRA term and writes Y.
+// pieces in CTA order. Whoever completes the tile writes Y.
 template <int MT>
 __device__ __forceinline__ void publish(const float (&acc)[2][MT][4], int64_t tile, int lane, int warp,
-                                        float* slots, uint32_t cnt_base, const ResParams& p) {
+                                        float* slots, uint32_t cnt_base, const int64_t* s_wbeg,
+                                        const int64_t* s_wtile, const ResParams& p) {
   const int64_t nsb = (p.K / 64 + 3) / 4;
   const int64_t cta = blockIdx.x;
-  const int64_t gw = cta * kResWarps + warp;
-  const int64_t wf = owner_of(tile * nsb, p.n_items, p.n_units);
-  const int64_t wl = owner_of(tile * nsb + nsb - 1, p.n_items, p.n_units);
-  const int64_t lw0 = (wf > cta * kResWarps ? wf : cta * kResWarps);
-  const int64_t lw1 = (wl < cta * kResWarps + kResWarps - 1 ? wl : cta * kResWarps + kResWarps - 1);  // wl < n_units
-  const int n_local = static_cast<int>(lw1 - lw0 + 1);
+  const int64_t tb = tile * nsb, te = tb + nsb;  // the tile's items
+  // this CTA's warps holding pieces of the tile: warp w holds items
+  // [s_wbeg[w], s_wbeg[w + 1]), and the holders are consecutive around this warp
+  int lw0 = warp, lw1 = warp;
+  while (lw0 > 0 && s_wbeg[lw0] > tb) --lw0;
+  while (lw1 < kResWarps - 1 && s_wbeg[lw1 + 1] < te) ++lw1;
+  const int n_local = lw1 - lw0 + 1;
   constexpr int kSlot = 32 * 4 * MT;  // floats per warp slot
   // this warp's slot for the tile: index = tile - first tile of the warp's range
-  const int64_t my_first_tile = range_begin(gw, p.n_items, p.n_units) / nsb;
-  float* my_slot = slots + (static_cast<int64_t>(warp) * p.p_max + (tile - my_first_tile)) * kSlot;
+  float* my_slot = slots + (static_cast<int64_t>(warp) * p.p_max + (tile - s_wtile[warp])) * kSlot;
   float y[MT][4];
 #pragma unroll
   for (int m = 0; m < MT; ++m) {
@@ -224,18 +253,16 @@ __device__ __forceinline__ void publish(const float (&acc)[2][MT][4], int64_t ti
     for (int m = 0; m < MT; ++m)
       reinterpret_cast<float4*>(my_slot + lane * 4 * MT)[m] = make_float4(y[m][0], y[m][1], y[m][2], y[m][3]);
     __syncwarp();  // the lanes' slot stores are ordered before lane 0's release below
-    const int64_t cta_first_tile = range_begin(cta * kResWarps, p.n_items, p.n_units) / nsb;
     unsigned int old = 0;
     if (lane == 0)
-      old = atom_add_acq_rel_cta_shared(cnt_base + static_cast<uint32_t>(tile - cta_first_tile) * 4u, 1u);
+      old = atom_add_acq_rel_cta_shared(cnt_base + static_cast<uint32_t>(tile - s_wtile[0]) * 4u, 1u);
     old = __shfl_sync(0xffffffffu, old, 0);
     if (old != static_cast<unsigned int>(n_local - 1)) return;  // another warp of the CTA finishes the tile
     __syncwarp();  // lane 0's acquire is ordered before every lane's reads of the slots
 #pragma unroll
     for (int m = 0; m < MT; ++m) y[m][0] = y[m][1] = y[m][2] = y[m][3] = 0.0f;
-    for (int64_t w = lw0; w <= lw1; ++w) {  // warp order
-      const int64_t wt = range_begin(w, p.n_items, p.n_units) / nsb;
-      const float* sl = slots + (static_cast<int64_t>(w - cta * kResWarps) * p.p_max + (tile - wt)) * kSlot;
+    for (int w = lw0; w <= lw1; ++w) {  // warp order
+      const float* sl = slots + (static_cast<int64_t>(w) * p.p_max + (tile - s_wtile[w])) * kSlot;
 #pragma unroll
       for (int m = 0; m < MT; ++m) {
         const float4 v = reinterpret_cast<const float4*>(sl + lane * 4 * MT)[m];
@@ -243,8 +270,11 @@ __device__ __forceinline__ void publish(const float (&acc)[2][MT][4], int64_t ti
       }
     }
   }
-  const int64_t cf = wf / kResWarps, cl = wl / kResWarps;
-  if (cf != cl) {  // pieces in other CTAs too
+  if (tb < s_wbeg[0] || te > s_wbeg[kResWarps]) {  // pieces in other CTAs too
+    // CTAs holding the tile's first and last items (the divisions only on this
+    // path: at most two tiles per CTA)
+    const int64_t cf = owner_of(tb, p.n_items, p.n_units) / kResWarps;
+    const int64_t cl = owner_of(te - 1, p.n_items, p.n_units) / kResWarps;
     float* tp = p.gpart + static_cast<int64_t>(tile) * p.max_cta_seg * kSlot;
 #pragma unroll
     for (int m = 0; m < MT; ++m)
@@ -266,7 +296,7 @@ __device__ __forceinline__ void publish(const float (&acc)[2][MT][4], int64_t ti
       }
     }
   }
-  lora_up_store<MT>(y, tile, lane, p);
+  store_y<MT>(y, tile, lane, p);
 }
 
 // SINGLE: single-level storage (the block constant is absmax[b]); V8: the packed
@@ -286,6 +316,74 @@ k_decode_res(const __grid_constant__ ResParams p, const __grid_constant__ Nf4Cod
   unsigned int* cnt = reinterpret_cast<unsigned int*>(slots + static_cast<size_t>(kResWarps) * p.p_max * 32 * 4 * MT);
   const uint32_t cnt_base = smem_u32(cnt);
 
+  const int64_t gw = static_cast<int64_t>(blockIdx.x) * kResWarps + warp;
+  // this warp's items [i0, i1) (warps numbered n_units and above: none)
+  const int64_t i0 = range_begin(gw < p.n_units ? gw : p.n_units, p.n_items, p.n_units);
+  const int64_t i1 = range_begin(gw < p.n_units ? gw + 1 : p.n_units, p.n_items, p.n_units);
+  const int n_my = static_cast<int>(i1 - i0);
+  // the CTA's warp ranges and first tiles, for the tile epilogue
+  __shared__ int64_t s_wbeg[kResWarps + 1];
+  __shared__ int64_t s_wtile[kResWarps];
+  if (lane == 0) {
+    s_wbeg[warp] = i0;
+    s_wtile[warp] = i0 / nsb;
+  }
+  if (threadIdx.x == 0) {
+    const int64_t u = static_cast<int64_t>(blockIdx.x + 1) * kResWarps;
+    s_wbeg[kResWarps] = range_begin(u < p.n_units ? u : p.n_units, p.n_items, p.n_units);
+  }
+  const bool reverse = warp == kResWarps - 1;
+  const int step = reverse ? -1 : 1;
+  const int64_t ifirst = reverse ? i1 - 1 : i0;
+
+  // Fetch state, one item ahead of the compute: tile and superblock of the
+  // item being loaded and this lane's rows of that tile (rows g and g + 8).
+  int64_t ftile = n_my > 0 ? ifirst / nsb : 0;
+  int fsb = static_cast<int>(ifirst - ftile * nsb);
+  const uint8_t* pa = nullptr;  // packed codes of row g, block t of superblock 0
+  const uint8_t* pb = nullptr;
+  uint32_t ba0 = 0, bb0 = 0;    // block index of (row, block t of superblock 0)
+  bool rowa = false, rowb = false;
+  auto set_tile = [&](int64_t tl) {
+    const int64_t na = tl * 16 + g, nb = na + 8;
+    rowa = na < N;
+    rowb = nb < N;
+    ba0 = static_cast<uint32_t>(na * nkb_row + t);
+    bb0 = static_cast<uint32_t>(nb * nkb_row + t);
+    pa = p.packed + static_cast<int64_t>(ba0) * 32;
+    pb = p.packed + static_cast<int64_t>(bb0) * 32;
+  };
+  // Codes and raw block constants of the fetched item. The constants are
+  // combined only when the item is decoded, so that no instruction waits on
+  // these loads before then. Blocks outside the weight read zero codes and
+  // zero constants; their token values in shared memory are zero.
+  uint4 ca0, ca1, cb0, cb1;
+  int qa = 0, qb = 0;        // int8 codes of the block constants (double-quantized storage)
+  float da = 0.0f, db = 0.0f;  // their group scales, or the fp32 constants (single-level)
+  auto fetch = [&](int sbk) {
+    const bool va = rowa && sbk * 4 + t < nkb_row, vb = rowb && sbk * 4 + t < nkb_row;
+    const uint32_t o = static_cast<uint32_t>(sbk) * 128u;  // 4 blocks x 32 bytes
+    const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+    ca0 = va ? ldg_stream(pa + o) : z;
+    ca1 = va ? ldg_stream(pa + o + 16) : z;
+    cb0 = vb ? ldg_stream(pb + o) : z;
+    cb1 = vb ? ldg_stream(pb + o + 16) : z;
+    const uint32_t ia = ba0 + static_cast<uint32_t>(sbk) * 4u, ib = bb0 + static_cast<uint32_t>(sbk) * 4u;
+    if (SINGLE) {
+      da = va ? __ldg(p.absmax + ia) : 0.0f;
+      db = vb ? __ldg(p.absmax + ib) : 0.0f;
+    } else {
+      qa = va ? static_cast<int>(__ldg(p.q + ia)) : 0;
+      qb = vb ? static_cast<int>(__ldg(p.q + ib)) : 0;
+      da = va ? __ldg(p.dqs + (ia >> 8)) : 0.0f;
+      db = vb ? __ldg(p.dqs + (ib >> 8)) : 0.0f;
+    }
+  };
+  if (n_my > 0) {  // the first item's loads overlap the X copy below
+    set_tile(ftile);
+    fetch(fsb);
+  }
+
   // ---- prologue: counters, and X copied into shared memory (padded blocks,
   // zero beyond K). X is an input of the call, complete before the LoRA-down
   // kernel that precedes this one started.
@@ -303,11 +401,6 @@ k_decode_res(const __grid_constant__ ResParams p, const __grid_constant__ Nf4Cod
   }
   __syncthreads();
 
-  const int64_t gw = static_cast<int64_t>(blockIdx.x) * kResWarps + warp;
-  const int64_t i0 = gw < p.n_units ? range_begin(gw, p.n_items, p.n_units) : 0;
-  const int64_t i1 = gw < p.n_units ? range_begin(gw + 1, p.n_items, p.n_units) : 0;
-  const int n_my = static_cast<int>(i1 - i0);
-  const bool reverse = warp == kResWarps - 1;
   const float mu = SINGLE ? 0.0f : __ldg(p.mean);
   const uint32_t xbase = smem_u32(res_sm);
   // token rows of this lane's B fragments (tokens >= M read the last token:
@@ -315,69 +408,37 @@ k_decode_res(const __grid_constant__ ResParams p, const __grid_constant__ Nf4Cod
   uint32_t xrow[MT];
 #pragma unroll
   for (int m = 0; m < MT; ++m) xrow[m] = xbase + static_cast<uint32_t>(min(g + 8 * m, M - 1) * p.x_stride);
-  const uint32_t row_bytes = static_cast<uint32_t>(K / 2);  // packed bytes per weight row
 
   bool entered = false;  // waited for the LoRA-down kernel (T, zeroed tickets)
   if (n_my > 0) {
-    // walk position: tile and superblock of the current item, stepped by +-1
-    // item (no divisions in the loop)
-    const int64_t ifirst = reverse ? i1 - 1 : i0;
-    int64_t tile = ifirst / nsb;
-    int sb = static_cast<int>(ifirst - tile * nsb);
-    const int step = reverse ? -1 : 1;
-    // per-tile row state of this lane: rows g and g + 8 of the tile
-    const uint8_t* pa = nullptr;  // packed codes of row g, block t of superblock 0
-    const uint8_t* pb = nullptr;
-    uint32_t ba0 = 0, bb0 = 0;    // block index of (row, block t of superblock 0)
-    bool rowa = false, rowb = false;
-    auto set_tile = [&](int64_t tl) {
-      const int64_t na = tl * 16 + g, nb = na + 8;
-      rowa = na < N;
-      rowb = nb < N;
-      ba0 = static_cast<uint32_t>(na * nkb_row + t);
-      bb0 = static_cast<uint32_t>(nb * nkb_row + t);
-      pa = p.packed + static_cast<int64_t>(ba0) * 32;
-      pb = p.packed + static_cast<int64_t>(bb0) * 32;
-    };
-    set_tile(tile);
-    uint4 ca0, ca1, cb0, cb1;  // codes of the current item (rows g, g + 8; 32 bytes each)
-    float mA, mB;              // its block constants
-    auto fetch = [&](int sbk, uint4& a0, uint4& a1, uint4& b0, uint4& b1, float& ma, float& mb) {
-      const bool va = rowa && sbk * 4 + t < nkb_row, vb = rowb && sbk * 4 + t < nkb_row;
-      const uint32_t o = static_cast<uint32_t>(sbk) * 128u;  // 4 blocks x 32 bytes
-      const uint4 z = make_uint4(0u, 0u, 0u, 0u);
-      a0 = va ? ldg_stream(pa + o) : z;
-      a1 = va ? ldg_stream(pa + o + 16) : z;
-      b0 = vb ? ldg_stream(pb + o) : z;
-      b1 = vb ? ldg_stream(pb + o + 16) : z;
-      const uint32_t ia = ba0 + static_cast<uint32_t>(sbk) * 4u, ib = bb0 + static_cast<uint32_t>(sbk) * 4u;
-      if (SINGLE) {
-        ma = va ? __ldg(p.absmax + ia) : 0.0f;
-        mb = vb ? __ldg(p.absmax + ib) : 0.0f;
-      } else {
-        ma = va ? __fmaf_rn(static_cast<float>(__ldg(p.q + ia)), __ldg(p.dqs + (ia >> 8)), mu) : 0.0f;
-        mb = vb ? __fmaf_rn(static_cast<float>(__ldg(p.q + ib)), __ldg(p.dqs + (ib >> 8)), mu) : 0.0f;
-      }
-    };
-    fetch(sb, ca0, ca1, cb0, cb1, mA, mB);
+    // compute position: tile and superblock of the item being decoded, stepped
+    // by +-1 item (no divisions in the loop)
+    int64_t tile = ftile;
+    int sb = fsb;
     float acc[2][MT][4];
 #pragma unroll
     for (int h = 0; h < 2; ++h)
 #pragma unroll
       for (int m = 0; m < MT; ++m) acc[h][m][0] = acc[h][m][1] = acc[h][m][2] = acc[h][m][3] = 0.0f;
-    // L2 prefetch of the tile's LoRA-up rows of B (read by whoever completes it)
+    // L2 prefetch of the tile's LoRA-up rows of B (read by the warp that decodes its last superblock)
     if (lane < 16 && tile * 16 + lane < N) prefetch_l2(p.Bl + (tile * 16 + lane) * p.r);
 #pragma unroll 1
     for (int e = 0; e < n_my; ++e) {
-      // position of the next item
-      int sbn = sb + step;
-      const bool tile_ends = sbn < 0 || sbn >= nsb || e + 1 == n_my;
+      const float mA = SINGLE ? da : __fmaf_rn(static_cast<float>(qa), da, mu);
+      const float mB = SINGLE ? db : __fmaf_rn(static_cast<float>(qb), db, mu);
       const Nf4Lut la = make_nf4_lut(cb, mA);
       const Nf4Lut lb = make_nf4_lut(cb, mB);
       const uint4 xa0 = ca0, xa1 = ca1, xb0 = cb0, xb1 = cb1;
-      if (!tile_ends) {  // next item in the same tile: load it now, prefetch the one after into L2
-        fetch(sbn, ca0, ca1, cb0, cb1, mA, mB);
-        const int sbp = sbn + step;
+      if (e + 1 < n_my) {  // load the next item (in this tile or the neighbouring one)
+        fsb += step;
+        if (fsb < 0 || fsb >= nsb) {
+          ftile += step;
+          fsb = reverse ? nsb - 1 : 0;
+          set_tile(ftile);
+          if (lane < 16 && ftile * 16 + lane < N) prefetch_l2(p.Bl + (ftile * 16 + lane) * p.r);
+        }
+        fetch(fsb);
+        const int sbp = fsb + step;  // and the one after it into L2, when in the same tile
         if (t == 0 && e + 2 < n_my && sbp >= 0 && sbp < nsb) {
           if (rowa) prefetch_l2(pa + static_cast<uint32_t>(sbp) * 128u);
           if (rowb) prefetch_l2(pb + static_cast<uint32_t>(sbp) * 128u);
@@ -413,23 +474,26 @@ k_decode_res(const __grid_constant__ ResParams p, const __grid_constant__ Nf4Cod
           }
         }
       }
-      if (tile_ends) {  // end of this warp's piece of `tile`
+      if (sb == nsb - 1) {  // the tile's last superblock: its LoRA term goes into this piece
         if (!entered) {  // T and the zeroed tickets come from the preceding LoRA-down kernel
           pdl_enter();
           entered = true;
         }
-        publish<MT>(acc, tile, lane, warp, slots, cnt_base, p);
+        lora_accumulate<MT>(acc[0], tile, lane, p);
+      }
+      int sbn = sb + step;
+      if (sbn < 0 || sbn >= nsb || e + 1 == n_my) {  // end of this warp's piece of `tile`
+        if (!entered) {
+          pdl_enter();
+          entered = true;
+        }
+        publish<MT>(acc, tile, lane, warp, slots, cnt_base, s_wbeg, s_wtile, p);
 #pragma unroll
         for (int h = 0; h < 2; ++h)
 #pragma unroll
           for (int m = 0; m < MT; ++m) acc[h][m][0] = acc[h][m][1] = acc[h][m][2] = acc[h][m][3] = 0.0f;
-        if (e + 1 < n_my) {  // move to the neighbouring tile and load its first item
-          tile += step;
-          sbn = reverse ? nsb - 1 : 0;
-          set_tile(tile);
-          fetch(sbn, ca0, ca1, cb0, cb1, mA, mB);
-          if (lane < 16 && tile * 16 + lane < N) prefetch_l2(p.Bl + (tile * 16 + lane) * p.r);
-        }
+        tile += step;
+        sbn = reverse ? nsb - 1 : 0;
       }
       sb = sbn;
     }

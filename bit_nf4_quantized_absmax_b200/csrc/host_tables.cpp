@@ -81,14 +81,14 @@ void build(QuantTables& t, int dtype) {
     t.thresholds[i] = f;
   }
 
-  // Bin table. Bin b holds u = 128 + r in [8b, 8b + 7], r = round(v * 127) (ties
-  // to even), so it can only see v with v * 127 in [8b - 128.5, 8b - 120.5];
+  // Bin table. Bin b holds u = 64 + r in [4b, 4b + 3], r = round(v * 63.5) (ties
+  // to even), so it can only see v with v * 63.5 in [4b - 64.5, 4b - 60.5];
   // widen by 2^-20 for margin. Each widened bin must contain at most one
   // threshold (bins are ~0.063 wide, thresholds >= 0.08 apart); checked below.
   const double P = static_cast<double>(kBinMul);
   for (int b = 0; b < kBins; ++b) {
-    double lo = (8.0 * b - 128.5) / P - std::ldexp(1.0, -20);
-    double hi = (8.0 * b - 120.5) / P + std::ldexp(1.0, -20);
+    double lo = (4.0 * b - 64.5) / P - std::ldexp(1.0, -20);
+    double hi = (4.0 * b - 60.5) / P + std::ldexp(1.0, -20);
     int inside = -1, count = 0, below = 0;
     for (int i = 0; i < 15; ++i) {
       double T = t.thresholds[i];

@@ -8,13 +8,13 @@
 namespace qlora {
 
 // Bin mapping used by the quantize kernel: x = fmaf(v, kBinMul, kBinAdd) is
-// 1.5 * 2^23 + 128 + r with r = v * 127 rounded to the nearest integer (one
-// rounding; |r| <= 127 for v in [-1, 1]), so the low byte of x's bit pattern is
-// u = 128 + r in [1, 255], and bin = u >> 3 (the byte offset of the bin's
-// 8-byte table entry is u & 0xF8).
-constexpr float kBinMul = 127.0f;
-constexpr float kBinAdd = 12583040.0f;  // 1.5 * 2^23 + 128, exact in fp32
-constexpr int kBins = 32;
+// 1.5 * 2^23 + 64 + r with r = v * 63.5 rounded to the nearest integer (one
+// rounding, ties to even; |r| <= 64 for v in [-1 - 2^-19, 1 + 2^-19]), so the
+// low byte of x's bit pattern is u = 64 + r in [0, 128], and bin = u >> 2 (the
+// byte offset of the bin's entry in a table of 4-byte entries is u & 0xFC).
+constexpr float kBinMul = 63.5f;
+constexpr float kBinAdd = 12582976.0f;  // 1.5 * 2^23 + 64, exact in fp32
+constexpr int kBins = 33;
 
 struct BinEntry {
   float threshold;  // T_j

@@ -7,7 +7,7 @@
 //                  load each, 1 KB contiguous per warp instruction): the absmax
 //                  (packed 16-bit max of the magnitude bits), stored as fp32,
 //                  the exact quotient v = w / m, the nearest code (one lookup in
-//                  a 32-bin table + one compare), 4-bit packing.
+//                  a 33-bin table + one compare), 4-bit packing.
 //   k_quant_sums   the exact sum of the absmax constants, as integer sums of
 //                  their 8-bit significands per exponent (order-independent).
 //                  The CTA that adds the last totals forms the mean from them.
@@ -92,12 +92,6 @@ __device__ double limbs_to_double(const unsigned long long (&L)[5]) {
   return ldexp(static_cast<double>(mant), exp2);
 }
 
-__device__ __forceinline__ uint32_t max_u16x2(uint32_t a, uint32_t b) {
-  uint32_t r;
-  asm("max.u16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
-  return r;
-}
-
 // Codes of 16 weights of a block given m (possibly scaled by a power of two
 // together with the weights) and r = RN(1/m); out[k] packs weights 8k..8k+7.
 template <bool SCALED>
@@ -116,9 +110,9 @@ __device__ __forceinline__ void encode16(const uint32_t (&d)[8], float ms, float
       const float q0 = __fmul_rn(w, r);
       const float res = __fmaf_rn(q0, -ms, w);
       const float v = __fmaf_rn(res, r, q0);
-      // bin: low byte of RN(v * 127 + 1.5 * 2^23 + 128); entry = (T_j, j + 1)
+      // bin: low byte of RN(v * 63.5 + 1.5 * 2^23 + 64); entry = (T_j, j + 1)
       const float x = __fmaf_rn(v, kBinMul, kBinAdd);
-      const uint2 e = *reinterpret_cast<const uint2*>(bins + (__float_as_uint(x) & 0xF8u));
+      const uint2 e = *reinterpret_cast<const uint2*>(bins + ((__float_as_uint(x) & 0xFCu) << 1));
       // code = j + (v >= T_j) = (j + 1) - [v < T_j]; RN(v - T_j) has the sign of
       // v - T_j and is +0 when they are equal
       const float dv = __fsub_rn(v, __uint_as_float(e.x));
@@ -133,7 +127,7 @@ __device__ __forceinline__ void encode16(const uint32_t (&d)[8], float ms, float
 // r = rcp.approx(m) (at most 1 ulp from 1/m), instead of the exact quotient
 // v = RN(w / m). For |w| <= m, |v' - w/m| <= 2^-23 + 2^-24 and |v - w/m| <=
 // 2^-24, so |v' - v| < 2^-22 and v' lies in [-1 - 2^-22, 1 + 2^-22]: the bin of
-// v' is a valid entry (|round(v' * 127)| <= 127), and the code from v' is the
+// v' is a valid entry (|round(v' * 63.5)| <= 64), and the code from v' is the
 // nearest code of v whenever |v' - T| >= 2^-21 for the threshold T it is
 // compared with (v and v' are then on the same side of T; the rule counts the
 // thresholds at or below its input, and checks every fp32 input). Returns true
@@ -147,11 +141,28 @@ __device__ __forceinline__ float rcp_approx(float x) {
   return r;
 }
 
+// Paired fp32 arithmetic (one instruction for two IEEE single-precision
+// operations, each rounded to nearest even, no flush of subnormals).
+__device__ __forceinline__ void mul2_rn(float a0, float a1, float b0, float b1, float& r0, float& r1) {
+  asm("{.reg .b64 a, b, r; mov.b64 a, {%2, %3}; mov.b64 b, {%4, %5}; mul.rn.f32x2 r, a, b; mov.b64 {%0, %1}, r;}"
+      : "=f"(r0), "=f"(r1) : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+__device__ __forceinline__ void fma2_rn(float a0, float a1, float b0, float b1, float c0, float c1, float& r0,
+                                        float& r1) {
+  asm("{.reg .b64 a, b, c, r; mov.b64 a, {%2, %3}; mov.b64 b, {%4, %5}; mov.b64 c, {%6, %7};"
+      " fma.rn.f32x2 r, a, b, c; mov.b64 {%0, %1}, r;}"
+      : "=f"(r0), "=f"(r1) : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
+}
+__device__ __forceinline__ void sub2_rn(float a0, float a1, float b0, float b1, float& r0, float& r1) {
+  asm("{.reg .b64 a, b, r; mov.b64 a, {%2, %3}; mov.b64 b, {%4, %5}; sub.rn.f32x2 r, a, b; mov.b64 {%0, %1}, r;}"
+      : "=f"(r0), "=f"(r1) : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+
 // The fast path reads the bin table as two arrays of 4-byte entries, the
-// thresholds T_j and the codes j + 1 (byte offset of bin b: 4 b, i.e. the low
-// byte of x's pattern shifted right by one), so each lookup of a warp touches
-// each bank once (the 8-byte entries of the exact path make bins b and b + 16
-// share banks).
+// thresholds T_j and the codes j + 1 (byte offset of bin b: 4 b, the low byte
+// of x's pattern with its two low bits cleared), so each lookup of a warp
+// touches each bank once. The two weights of one bf16 pair go through the
+// quotient, the bin and the comparison together as one paired operation each.
 __device__ __forceinline__ bool encode16_fast(const uint32_t (&d)[8], float r, const unsigned char* tbin,
                                               const unsigned char* cbin, uint32_t (&out)[2]) {
   bool near = false;
@@ -159,18 +170,22 @@ __device__ __forceinline__ bool encode16_fast(const uint32_t (&d)[8], float r, c
   for (int k = 0; k < 2; ++k) {
     uint32_t word = 0u;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const uint32_t bits = d[4 * k + (i >> 1)];
-      const float w = __uint_as_float((i & 1) ? (bits & 0xFFFF0000u) : (bits << 16));
-      const float v = __fmul_rn(w, r);
-      const float x = __fmaf_rn(v, kBinMul, kBinAdd);
-      const uint32_t off = (__float_as_uint(x) & 0xF8u) >> 1;
-      const float T = *reinterpret_cast<const float*>(tbin + off);
-      const uint32_t c1 = *reinterpret_cast<const uint32_t*>(cbin + off);
-      const float dv = __fsub_rn(v, T);
-      near = near || (fabsf(dv) < kNearEps);
-      const uint32_t c = c1 - __umulhi(__float_as_uint(dv), 2u);
-      word += c * (1u << (4 * i));
+    for (int q = 0; q < 4; ++q) {  // weights 8k + 2q (low half of the pair) and 8k + 2q + 1
+      const uint32_t bits = d[4 * k + q];
+      float v0, v1, x0, x1, dv0, dv1;
+      mul2_rn(__uint_as_float(bits << 16), __uint_as_float(bits & 0xFFFF0000u), r, r, v0, v1);
+      fma2_rn(v0, v1, kBinMul, kBinMul, kBinAdd, kBinAdd, x0, x1);
+      const uint32_t o0 = __float_as_uint(x0) & 0xFCu, o1 = __float_as_uint(x1) & 0xFCu;
+      const float T0 = *reinterpret_cast<const float*>(tbin + o0);
+      const float T1 = *reinterpret_cast<const float*>(tbin + o1);
+      const uint32_t c0 = *reinterpret_cast<const uint32_t*>(cbin + o0);
+      const uint32_t c1 = *reinterpret_cast<const uint32_t*>(cbin + o1);
+      sub2_rn(v0, v1, T0, T1, dv0, dv1);
+      near = near || (fabsf(dv0) < kNearEps) || (fabsf(dv1) < kNearEps);
+      // code = j + (v >= T_j) = (j + 1) - [v < T_j]; RN(v - T_j) has the sign of
+      // v - T_j and is +0 when they are equal
+      word += (c0 - __umulhi(__float_as_uint(dv0), 2u)) * (1u << (8 * q));
+      word += (c1 - __umulhi(__float_as_uint(dv1), 2u)) * (1u << (8 * q + 4));
     }
     out[k] = word;
   }
@@ -267,7 +282,7 @@ __device__ __forceinline__ void pass1_loop(const uint4* __restrict__ W, int64_t 
 
 // zero_totals (double-quantized storage only): the 256 bin totals that
 // k_quant_sums adds into, cleared here by CTA 0 before that kernel starts.
-__global__ void __launch_bounds__(kPass1Threads)
+__global__ void __launch_bounds__(kPass1Threads, 8)
 k_quant_pass1(const uint4* __restrict__ W, bool v8, uint32_t* __restrict__ packed,
               float* __restrict__ absmax, unsigned long long* __restrict__ zero_totals,
               unsigned int* __restrict__ zero_done, int64_t nblk, const __grid_constant__ QuantBinTable tab) {

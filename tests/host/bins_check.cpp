@@ -1,7 +1,7 @@
 // Exhaustive host check of the quantize kernel's binning rule, for the NF4 and
 // the FP4 tables: for every fp32 v in [-1 - 2^-19, 1 + 2^-19], the code the
-// kernel forms from its 32-bin table,
-//   x = fmaf(v, kBinMul, kBinAdd), entry = bins[(bits(x) & 0xF8) >> 3],
+// kernel forms from its bin table,
+//   x = fmaf(v, kBinMul, kBinAdd), entry = bins[(bits(x) & 0xFC) >> 2],
 //   code = (entry.j + 1) - [RN(v - entry.threshold) < 0],
 // must equal the number of decision thresholds T_i with v >= T_i (the nearest
 // code, ties to the lower index). Exit status 0 iff no value disagrees.
@@ -28,7 +28,7 @@ static uint64_t check_range(uint32_t lo, uint32_t hi, int sign, int dtype) {
     const float x = std::fmaf(v, kBinMul, kBinAdd);
     uint32_t xb;
     std::memcpy(&xb, &x, 4);
-    const BinEntry& e = t.bins[(xb & 0xF8u) >> 3];
+    const BinEntry& e = t.bins[(xb & 0xFCu) >> 2];
     const float d = v - e.threshold;
     uint32_t db;
     std::memcpy(&db, &d, 4);
