@@ -18,13 +18,14 @@
 // A warp's range covers pieces ("segments") of one or more tiles. At the end of
 // a segment the warp stores its fp32 partial sums in a slot of the tile; the
 // warp that completes a tile (ticket counter, no waiting) sums the tile's slots
-// in slot order, adds the LoRA term s (T B^T) with a bf16 hi/lo split of T on
-// the tensor cores, and writes Y. The result depends only on the shapes, not on
-// timing.
+// in slot order and writes Y. The LoRA term s (T B^T), with a bf16 hi/lo split
+// of T on the tensor cores, goes into the piece of the warp that decodes the
+// tile's last superblock. The result depends only on the shapes, not on timing.
 #include <cuda.h>
 
 #include "common.cuh"
 #include "kernels.h"
+#include "lora_tile.cuh"
 #include "nf4_lut.cuh"
 #include "tensor_map.h"
 
@@ -32,15 +33,6 @@ namespace qlora {
 namespace {
 
 constexpr int kDecodeWarps = 8;
-
-__device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
-                                         uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-      "{%0,%1,%2,%3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
 
 // (Writing these shifts as high halves of products, to move them off the
 // integer ALU, measured 4% slower than plain shifts.)
@@ -81,96 +73,55 @@ __device__ __forceinline__ unsigned int atom_add_acq_rel_gpu(unsigned int* p, un
 }
 
 // End of a work unit's piece of 16-row tile `tile` (item row `item_row` of the
-// unit ranges): store the warp's fp32 partial sums in the tile's slot; the warp that brings the tile's last piece (ticket counter, no
-// waiting) sums the slots in slot order, adds s (T B^T) computed on the tensor
-// cores with T split into bf16 hi + lo, and writes Y.
+// unit ranges; this unit holds items [i_begin, i_end)): store the warp's fp32
+// partial sums in the tile's slot; the warp that brings the tile's last piece
+// (ticket counter, no waiting) sums the slots in slot order and writes Y. (The
+// tile's LoRA term is already in the piece of the unit that decoded the tile's
+// last superblock.)
 template <int MT>
 __device__ __forceinline__ void publish_segment(const float (&acc)[2][MT][4], int64_t item_row, int64_t tile,
-                                                int64_t unit, int lane, int64_t nsb, int64_t n_items,
-                                                int64_t n_units, int max_seg,
+                                                int64_t unit, int lane, int64_t nsb, int64_t i_begin, int64_t i_end,
+                                                int64_t n_items, int64_t n_units, int max_seg,
                                                 float* __restrict__ partial, unsigned int* __restrict__ counters,
-                                                const float* __restrict__ T, const __nv_bfloat16* __restrict__ Bl,
-                                                int r, float s, __nv_bfloat16* __restrict__ Y, int M, int64_t N) {
-  const int g = lane >> 2, t = lane & 3;
-  const int64_t w_first = item_owner(item_row * nsb, n_items, n_units);
-  const int64_t w_last = item_owner((item_row + 1) * nsb - 1, n_items, n_units);
+                                                __nv_bfloat16* __restrict__ Y, int M, int64_t N) {
+  // units holding the row's first and last items (a division only when the
+  // row reaches beyond this unit's range)
+  const int64_t gb = item_row * nsb, ge = gb + nsb;
+  const int64_t w_first = gb < i_begin ? floor_div_small((gb + 1) * n_units - 1, n_items) : unit;
+  const int64_t w_last = ge > i_end ? floor_div_small(ge * n_units - 1, n_items) : unit;
   const int nseg = static_cast<int>(w_last - w_first + 1);
   const int slot = static_cast<int>(unit - w_first);
   float* tile_part = partial + static_cast<int64_t>(tile) * max_seg * (32 * 4 * MT);
+  float y[MT][4];
 #pragma unroll
   for (int m = 0; m < MT; ++m) {
-    const float4 v = make_float4(acc[0][m][0] + acc[1][m][0], acc[0][m][1] + acc[1][m][1],
-                                 acc[0][m][2] + acc[1][m][2], acc[0][m][3] + acc[1][m][3]);
-    __stcg(reinterpret_cast<float4*>(tile_part + (slot * 32 + lane) * 4 * MT) + m, v);
+    y[m][0] = acc[0][m][0] + acc[1][m][0];
+    y[m][1] = acc[0][m][1] + acc[1][m][1];
+    y[m][2] = acc[0][m][2] + acc[1][m][2];
+    y[m][3] = acc[0][m][3] + acc[1][m][3];
   }
-  __syncwarp();  // the lanes' partial stores are ordered before lane 0's release below
   if (nseg > 1) {
+#pragma unroll
+    for (int m = 0; m < MT; ++m)
+      __stcg(reinterpret_cast<float4*>(tile_part + (slot * 32 + lane) * 4 * MT) + m,
+             make_float4(y[m][0], y[m][1], y[m][2], y[m][3]));
+    __syncwarp();  // the lanes' partial stores are ordered before lane 0's release below
     unsigned int ticket = 0;
     if (lane == 0) ticket = atom_add_acq_rel_gpu(&counters[tile], 1u);
     ticket = __shfl_sync(0xffffffffu, ticket, 0);
     if (ticket != static_cast<unsigned int>(nseg - 1)) return;  // another warp completes the tile
     __syncwarp();  // lane 0's acquire is ordered before every lane's reads of the slots
-  }
-
-  float y[MT][4];
 #pragma unroll
-  for (int m = 0; m < MT; ++m) y[m][0] = y[m][1] = y[m][2] = y[m][3] = 0.0f;
-  for (int sl = 0; sl < nseg; ++sl) {
+    for (int m = 0; m < MT; ++m) y[m][0] = y[m][1] = y[m][2] = y[m][3] = 0.0f;
+    for (int sl = 0; sl < nseg; ++sl) {
 #pragma unroll
-    for (int m = 0; m < MT; ++m) {
-      const float4 v = __ldcg(reinterpret_cast<const float4*>(tile_part + (sl * 32 + lane) * 4 * MT) + m);
-      y[m][0] += v.x; y[m][1] += v.y; y[m][2] += v.z; y[m][3] += v.w;
-    }
-  }
-  // LoRA up: rows of B are the A operand, T^T (split into bf16 hi + lo) the B
-  // operand. A step covers ranks j0 .. j0 + 15; since r % 8 == 0 its upper half
-  // is either wholly inside [0, r) or wholly outside (and then zero).
-  const int64_t na = tile * 16 + g, nb = na + 8;
-  float l[MT][4];
-#pragma unroll
-  for (int m = 0; m < MT; ++m) l[m][0] = l[m][1] = l[m][2] = l[m][3] = 0.0f;
-  for (int j0 = 0; j0 < r; j0 += 16) {
-    const bool hi_in = j0 + 8 < r;
-    const uint32_t b_a0 = na < N ? *reinterpret_cast<const uint32_t*>(Bl + na * r + j0 + 2 * t) : 0u;
-    const uint32_t b_a2 = na < N && hi_in ? *reinterpret_cast<const uint32_t*>(Bl + na * r + j0 + 2 * t + 8) : 0u;
-    const uint32_t b_a1 = nb < N ? *reinterpret_cast<const uint32_t*>(Bl + nb * r + j0 + 2 * t) : 0u;
-    const uint32_t b_a3 = nb < N && hi_in ? *reinterpret_cast<const uint32_t*>(Bl + nb * r + j0 + 2 * t + 8) : 0u;
-#pragma unroll
-    for (int m = 0; m < MT; ++m) {
-      const int tok = g + 8 * m;
-      float tv[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-      if (tok < M) {
-        const float* tp = T + static_cast<int64_t>(tok) * r + j0 + 2 * t;
-        tv[0] = __ldcg(tp);
-        tv[1] = __ldcg(tp + 1);
-        if (hi_in) {
-          tv[2] = __ldcg(tp + 8);
-          tv[3] = __ldcg(tp + 9);
-        }
+      for (int m = 0; m < MT; ++m) {
+        const float4 v = __ldcg(reinterpret_cast<const float4*>(tile_part + (sl * 32 + lane) * 4 * MT) + m);
+        y[m][0] += v.x; y[m][1] += v.y; y[m][2] += v.z; y[m][3] += v.w;
       }
-      uint32_t hi[2], lo[2];
-#pragma unroll
-      for (int p = 0; p < 2; ++p) {
-        const uint32_t h = pack_bf16x2(tv[2 * p], tv[2 * p + 1]);
-        hi[p] = h;
-        lo[p] = pack_bf16x2(tv[2 * p] - bf16lo_to_f32(h), tv[2 * p + 1] - bf16hi_to_f32(h));
-      }
-      mma16816(l[m], b_a0, b_a1, b_a2, b_a3, hi[0], hi[1]);
-      mma16816(l[m], b_a0, b_a1, b_a2, b_a3, lo[0], lo[1]);
     }
   }
-#pragma unroll
-  for (int m = 0; m < MT; ++m) {
-    const int tok0 = 8 * m + 2 * t, tok1 = tok0 + 1;
-    if (na < N) {
-      if (tok0 < M) Y[static_cast<int64_t>(tok0) * N + na] = __float2bfloat16_rn(fmaf(s, l[m][0], y[m][0]));
-      if (tok1 < M) Y[static_cast<int64_t>(tok1) * N + na] = __float2bfloat16_rn(fmaf(s, l[m][1], y[m][1]));
-    }
-    if (nb < N) {
-      if (tok0 < M) Y[static_cast<int64_t>(tok0) * N + nb] = __float2bfloat16_rn(fmaf(s, l[m][2], y[m][2]));
-      if (tok1 < M) Y[static_cast<int64_t>(tok1) * N + nb] = __float2bfloat16_rn(fmaf(s, l[m][3], y[m][3]));
-    }
-  }
+  store_tile_y<MT>(y, tile, lane, Y, M, N);
 }
 
 // CTA items are (128-row group, 256-wide K superblock) pairs in group-major
@@ -350,7 +301,7 @@ k_decode(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUten
               lookup4_sel(lb, half ? hi16(sbw) : sbw, half ? hi16(tb) : tb, a1, a3);  // row g + 8
 #pragma unroll
               for (int m = 0; m < MT; ++m)
-                mma16816(acc[half][m], a0, a1, a2, a3, half ? xv[m].z : xv[m].x, half ? xv[m].w : xv[m].y);
+                mma_bf16_16816(acc[half][m], a0, a1, a2, a3, half ? xv[m].z : xv[m].x, half ? xv[m].w : xv[m].y);
             }
           }
         }
@@ -362,14 +313,21 @@ k_decode(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUten
         stage = 0;
         phase ^= 1u;
       }
+      if (sb == nsb - 1) {  // the row's last superblock: the tile's LoRA term goes into this piece
+        if (!entered) {  // T and the zeroed counters come from the preceding LoRA-down kernel
+          pdl_enter();
+          entered = true;
+        }
+        lora_tile_accumulate<MT>(acc[0], rg * kDecodeWarps + warp, lane, T, Bl, r, s, M, N);
+      }
     }
     if (!ok) break;
     if (!entered) {  // T and the zeroed counters come from the preceding LoRA-down kernel
       pdl_enter();
       entered = true;
     }
-    publish_segment<MT>(acc, rg, rg * kDecodeWarps + warp, cta, lane, nsb, n_items, n_ctas, max_seg, partial,
-                        counters, T, Bl, r, s, Y, M, N);
+    publish_segment<MT>(acc, rg, rg * kDecodeWarps + warp, cta, lane, nsb, i_begin, i_end, n_items, n_ctas, max_seg,
+                        partial, counters, Y, M, N);
     ++rg;
     sb = 0;
   }

@@ -40,6 +40,7 @@
 // give identical bits.
 #include "common.cuh"
 #include "kernels.h"
+#include "lora_tile.cuh"
 #include "nf4_lut.cuh"
 
 namespace qlora {
@@ -57,15 +58,6 @@ constexpr int kResRegs = 112;
 // counters); larger plans go to the TMA-ring kernel. The kernel's limit is set
 // to this once, so that every plan up to it launches.
 constexpr int kResSmemCap = 200 * 1024;
-
-__device__ __forceinline__ void mma16816r(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
-                                          uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-      "{%0,%1,%2,%3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
 
 __device__ __forceinline__ void lookup4(const Nf4Lut& L, uint32_t s, uint32_t sel, uint32_t& o01, uint32_t& o23) {
   const uint32_t lo = prmt(prmt(L.lo[0], L.lo[1], s), prmt(L.lo[2], L.lo[3], s), sel);
@@ -137,86 +129,6 @@ struct ResParams {
 // Shared memory: X [M][x_stride] | slots [kResWarps][p_max][32][4 MT] fp32 | counters [cta_tiles] u32
 __host__ __device__ inline size_t res_slot_off(const ResParams& p) {
   return (static_cast<size_t>(p.M) * p.x_stride + 15) / 16 * 16;
-}
-
-// LoRA term of one tile, added to the partial sums of the warp that decodes the
-// tile's last superblock: acc[m][i] = fmaf(s, l, acc[m][i]) with l = (T B^T)
-// for this lane's rows and tokens. Rows of B are the A operand, T^T (split into
-// bf16 hi + lo) the B operand. Ranks go in chunks of 64 with every load of a
-// chunk issued before its MMAs (one round trip to L2 per chunk). A step covers
-// ranks j0 .. j0 + 15; since r % 8 == 0 its upper half is either wholly inside
-// [0, r) or wholly outside (and then zero).
-template <int MT>
-__device__ __forceinline__ void lora_accumulate(float (&acc)[MT][4], int64_t tile, int lane, const ResParams& p) {
-  const int g = lane >> 2, t = lane & 3;
-  const int64_t na = tile * 16 + g, nb = na + 8;
-  const int r = p.r;
-  float l[MT][4];
-#pragma unroll
-  for (int m = 0; m < MT; ++m) l[m][0] = l[m][1] = l[m][2] = l[m][3] = 0.0f;
-  for (int c0 = 0; c0 < r; c0 += 64) {
-    uint32_t bv[4][4];
-    float tv[4][MT][4];
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int j0 = c0 + 16 * q;
-      const bool lo_in = j0 < r, hi_in = j0 + 8 < r;
-      const __nv_bfloat16* Ba = p.Bl + na * r + j0 + 2 * t;
-      const __nv_bfloat16* Bb = p.Bl + nb * r + j0 + 2 * t;
-      bv[q][0] = na < p.N && lo_in ? *reinterpret_cast<const uint32_t*>(Ba) : 0u;
-      bv[q][1] = nb < p.N && lo_in ? *reinterpret_cast<const uint32_t*>(Bb) : 0u;
-      bv[q][2] = na < p.N && hi_in ? *reinterpret_cast<const uint32_t*>(Ba + 8) : 0u;
-      bv[q][3] = nb < p.N && hi_in ? *reinterpret_cast<const uint32_t*>(Bb + 8) : 0u;
-#pragma unroll
-      for (int m = 0; m < MT; ++m) {
-        const int tok = g + 8 * m;
-        const float* tp = p.T + static_cast<int64_t>(tok) * r + j0 + 2 * t;
-        const bool tin = tok < p.M;
-        tv[q][m][0] = tin && lo_in ? __ldcg(tp) : 0.0f;
-        tv[q][m][1] = tin && lo_in ? __ldcg(tp + 1) : 0.0f;
-        tv[q][m][2] = tin && hi_in ? __ldcg(tp + 8) : 0.0f;
-        tv[q][m][3] = tin && hi_in ? __ldcg(tp + 9) : 0.0f;
-      }
-    }
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-#pragma unroll
-      for (int m = 0; m < MT; ++m) {
-        uint32_t hi[2], lo[2];
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const uint32_t x = pack_bf16x2(tv[q][m][2 * h], tv[q][m][2 * h + 1]);
-          hi[h] = x;
-          lo[h] = pack_bf16x2(tv[q][m][2 * h] - bf16lo_to_f32(x), tv[q][m][2 * h + 1] - bf16hi_to_f32(x));
-        }
-        mma16816r(l[m], bv[q][0], bv[q][1], bv[q][2], bv[q][3], hi[0], hi[1]);
-        mma16816r(l[m], bv[q][0], bv[q][1], bv[q][2], bv[q][3], lo[0], lo[1]);
-      }
-    }
-  }
-#pragma unroll
-  for (int m = 0; m < MT; ++m)
-#pragma unroll
-    for (int i = 0; i < 4; ++i) acc[m][i] = __fmaf_rn(p.s, l[m][i], acc[m][i]);
-}
-
-// Y of this lane's rows and tokens (tokens >= M and rows >= N are not stored).
-template <int MT>
-__device__ __forceinline__ void store_y(const float (&y)[MT][4], int64_t tile, int lane, const ResParams& p) {
-  const int g = lane >> 2, t = lane & 3;
-  const int64_t na = tile * 16 + g, nb = na + 8;
-#pragma unroll
-  for (int m = 0; m < MT; ++m) {
-    const int tok0 = 8 * m + 2 * t, tok1 = tok0 + 1;
-    if (na < p.N) {
-      if (tok0 < p.M) p.Y[static_cast<int64_t>(tok0) * p.N + na] = __float2bfloat16_rn(y[m][0]);
-      if (tok1 < p.M) p.Y[static_cast<int64_t>(tok1) * p.N + na] = __float2bfloat16_rn(y[m][1]);
-    }
-    if (nb < p.N) {
-      if (tok0 < p.M) p.Y[static_cast<int64_t>(tok0) * p.N + nb] = __float2bfloat16_rn(y[m][2]);
-      if (tok1 < p.M) p.Y[static_cast<int64_t>(tok1) * p.N + nb] = __float2bfloat16_rn(y[m][3]);
-    }
-  }
 }
 
 // A warp has finished its piece of tile `tile`. Store the piece in the warp's
@@ -296,7 +208,7 @@ __device__ __forceinline__ void publish(const float (&acc)[2][MT][4], int64_t ti
       }
     }
   }
-  store_y<MT>(y, tile, lane, p);
+  store_tile_y<MT>(y, tile, lane, p.Y, p.M, p.N);
 }
 
 // SINGLE: single-level storage (the block constant is absmax[b]); V8: the packed
@@ -469,7 +381,7 @@ k_decode_res(const __grid_constant__ ResParams p, const __grid_constant__ Nf4Cod
               lookup4(lb, half ? (sbw >> 16) : sbw, half ? (tb >> 16) : tb, a1, a3);   // row g + 8
 #pragma unroll
               for (int m = 0; m < MT; ++m)
-                mma16816r(acc[half][m], a0, a1, a2, a3, half ? xv[m].z : xv[m].x, half ? xv[m].w : xv[m].y);
+                mma_bf16_16816(acc[half][m], a0, a1, a2, a3, half ? xv[m].z : xv[m].x, half ? xv[m].w : xv[m].y);
             }
           }
         }
@@ -479,7 +391,7 @@ k_decode_res(const __grid_constant__ ResParams p, const __grid_constant__ Nf4Cod
           pdl_enter();
           entered = true;
         }
-        lora_accumulate<MT>(acc[0], tile, lane, p);
+        lora_tile_accumulate<MT>(acc[0], tile, lane, p.T, p.Bl, p.r, p.s, p.M, p.N);
       }
       int sbn = sb + step;
       if (sbn < 0 || sbn >= nsb || e + 1 == n_my) {  // end of this warp's piece of `tile`
