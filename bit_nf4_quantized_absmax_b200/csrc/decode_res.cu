@@ -6,9 +6,10 @@
 // Y[M, N] = X W'^T + s T B^T, T = X A^T from the LoRA-down kernel that runs
 // first (k_lora_t_small in decode.cu).
 //
-// Used where it measured faster than the TMA-ring kernel of decode.cu (one
-// token on weights from about 16 M entries, up to 8 tokens from about 64 M) and
-// X (M x K bf16, padded) fits in shared memory beside the reduction slots.
+// Used where it measured faster than the TMA-ring kernel of decode.cu (up to 4
+// tokens on most weights from 4 M entries, up to 8 on tall ones; the rule is in
+// res_plan) and X (M x K bf16, padded) fits in shared memory beside the
+// reduction slots.
 //
 // Work items are (16-row tile, 256-wide K superblock) pairs in tile-major
 // order, and every warp of the grid takes one contiguous, equally sized range
@@ -467,12 +468,17 @@ ResPlan res_plan(int64_t M, int64_t N, int64_t K, int num_sms, bool force) {
   const size_t sbytes = static_cast<size_t>(kResWarps) * p.p_max * 32 * 4 * p.mt * sizeof(float);
   p.smem = xbytes + sbytes + static_cast<size_t>(p.cta_tiles) * 4;
   // Measured crossover against the TMA-ring kernel (B200, L2-cold weights, CUDA
-  // graph replay): this kernel is faster for one token from about 16 M weights
-  // up (11008x4096: 19.7 against 22.9 us) and for 2..8 tokens from about 64 M
-  // weights up (8192x8192, M = 4: 27.8 against 31.5 us); the ring kernel keeps
-  // smaller weights and 9..16 tokens.
+  // graph replay of the whole call, M = 1 / 2 / 4 / 8 tokens): this kernel is
+  // faster on square and wide-K-short weights up to 4 tokens (4096x4096: 11.5 /
+  // 12.5 / 12.5 against 13.1 / 13.3 / 13.7 us; 2048x2048 from 7.6 against 8.1;
+  // 8192x22016 at 1 and 2 tokens: 49.6 / 51.5 against 61.4 / 63.0) and on tall
+  // weights (N > K) up to 8 tokens (11008x4096: 17.7 / 18.0 / 18.6 / 19.5
+  // against 21.3 / 21.6 / 21.8 / 22.2); it is slower on K > N below 2^26
+  // entries (4096x11008: 24.1 / 26.6 / 29.6 against 22.9 / 23.5 / 23.9) and
+  // at 8 tokens on square weights (4096x4096: 17.1 against 14.4).
   const int64_t nw = N * K;
-  const bool faster = (M == 1 && nw >= (int64_t(1) << 24)) || (M <= 8 && nw >= (int64_t(1) << 26));
+  const bool faster = (M <= 4 && nw >= (int64_t(1) << 22) && !(K > N && nw < (int64_t(1) << 26))) ||
+                      (M <= 8 && K < N && nw >= (int64_t(1) << 24));
   p.ok = (faster || force) && p.smem <= static_cast<size_t>(kResSmemCap);
   return p;
 }

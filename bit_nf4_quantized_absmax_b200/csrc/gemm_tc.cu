@@ -47,6 +47,7 @@ struct TileSched {
   int nkb;        // total k-blocks (main + slab)
   int nk1;        // k-blocks of the main pair
   int kb_per_split;
+  int group_m;    // 0: tiles M-fastest; else (one split) bands of group_m M tiles, M-fastest inside a band
 };
 
 // DUAL: every k-block multiplies one A tile by two B tiles (B1 then B2) into
@@ -157,11 +158,27 @@ __device__ __forceinline__ bool wait_or_abort_cluster(uint64_t* bar, uint32_t pa
   return true;
 }
 
+// Tile (tm, tn) and k-block range of work unit `unit`. Consecutive units run
+// at the same time on consecutive CTAs (pairs), so the order decides which A
+// and B slabs are read from DRAM together: with bands of group_m M tiles the
+// ~74 tiles in flight on 148 SMs cover about 8 x 9 tiles, so each wave reads
+// about 17 slabs instead of the 16 + 5 of an M-fastest order.
 __device__ __forceinline__ void decode_unit(const TileSched& ts, int unit, int& tm, int& tn, int& kb0, int& kb1) {
-  tm = unit % ts.tiles_m;
-  const int rest = unit / ts.tiles_m;
-  tn = rest % ts.tiles_n;
-  const int split = rest / ts.tiles_n;
+  int split = 0;
+  if (ts.group_m > 0) {
+    const int band = ts.group_m * ts.tiles_n;
+    const int b = unit / band;
+    const int first_m = b * ts.group_m;
+    const int gm = min(ts.tiles_m - first_m, ts.group_m);
+    const int r = unit - b * band;
+    tm = first_m + r % gm;
+    tn = r / gm;
+  } else {
+    tm = unit % ts.tiles_m;
+    const int rest = unit / ts.tiles_m;
+    tn = rest % ts.tiles_n;
+    split = rest / ts.tiles_n;
+  }
   kb0 = split * ts.kb_per_split;
   kb1 = min(ts.nkb, kb0 + ts.kb_per_split);
 }
@@ -1033,7 +1050,7 @@ cudaError_t run(const Operand& a1, const Operand& b1, const Operand* a2, const O
     ta2 = ta1;
     tb2 = tb1;
   }
-  TileSched ts;
+  TileSched ts{};  // group_m = 0: M-fastest
   ts.tiles_m = static_cast<int>((M + BM - 1) / BM);
   ts.tiles_n = static_cast<int>((Nc + BN - 1) / BN);
   ts.nk1 = static_cast<int>((a1.k + BK - 1) / BK);
@@ -1062,7 +1079,11 @@ cudaError_t run_pair(const Operand& a1, const Operand& b1, const Operand& a2, co
   // each CTA loads 128 rows of A and 128 of B's output dimension per box
   if (!map_operand(&ta1, a1, 128) || !map_operand(&tb1, b1, 128)) return cudaErrorInvalidValue;
   if (!map_operand(&ta2, a2, 128) || !map_operand(&tb2, b2, 128)) return cudaErrorInvalidValue;
-  TileSched ts;
+  TileSched ts{};
+  // dX (MN-major B): bands of 8 M tiles cut its DRAM reads (465 -> 416 MB on
+  // 11008x4096, M = 4096); the forward keeps the M-fastest order, which reads
+  // W' once (141 MB against 220 MB banded)
+  ts.group_m = B_MN ? 8 : 0;
   ts.tiles_m = static_cast<int>((M + 255) / 256);
   ts.tiles_n = static_cast<int>((Nc + 255) / 256);
   ts.nk1 = static_cast<int>((a1.k + BK - 1) / BK);
@@ -1121,7 +1142,11 @@ cudaError_t run_pair_nf4(const void* A1, int64_t K1, const Nf4View& w, const voi
   CUtensorMap ta1, ta2, tb2;
   if (!map_operand(&ta1, a1, 128) || !map_operand(&ta2, a2, 128) || !map_operand(&tb2, b2, 128))
     return cudaErrorInvalidValue;
-  TileSched ts;
+  TileSched ts{};
+  // dX (MN-major B): bands of 8 M tiles cut its DRAM reads (465 -> 416 MB on
+  // 11008x4096, M = 4096); the forward keeps the M-fastest order, which reads
+  // W' once (141 MB against 220 MB banded)
+  ts.group_m = B_MN ? 8 : 0;
   ts.tiles_m = static_cast<int>((M + 255) / 256);
   ts.tiles_n = static_cast<int>((Nc + 255) / 256);
   ts.nk1 = static_cast<int>((K1 + BK - 1) / BK);
