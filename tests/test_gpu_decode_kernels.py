@@ -49,3 +49,31 @@ def test_decode_kernel_cases(mode, monkeypatch):
         ok, err = gemm_close(bf16_to_f32_np(Y), Yr)
         assert ok, (mode, N, K, M, r, err)
         assert np.allclose(T.cpu().numpy(), Tr, rtol=1e-4, atol=1e-4 * np.abs(Tr).max())
+
+
+DEFAULT_CASES = [  # (N, K, M, r): shapes the library's own choice sends to the X-resident kernel
+    (8192, 2048, 8, 64),  # K < N, 2^24 entries: up to 8 tokens
+    (2048, 2048, 4, 64),  # square, 2^22 entries: up to 4 tokens
+    (2048, 2048, 2, 64),
+]
+
+
+def test_decode_default_choice_cases(monkeypatch):
+    """The library's own kernel choice (no QLORA_DECODE_RES) on shapes past the
+    crossover, against the fp64 oracle, with identical bits on a repeat."""
+    monkeypatch.delenv("QLORA_DECODE_RES", raising=False)
+    dev = require_gpu()
+    for i, (N, K, M, r) in enumerate(DEFAULT_CASES):
+        inp = syn.make_linear(N, K, M, r=r, alpha=16.0, seed=60 + i, workload="test", dy_std=1.0)
+        W, A, B, X = (t.to(dev).contiguous() for t in (inp.W, inp.A, inp.B, inp.X))
+        q = b.qlora_quantize_nf4_dq(W)
+        Y, _ = b.qlora_linear_fwd(q, X, A, B, inp.alpha)
+        Y2, _ = b.qlora_linear_fwd(q, X, A, B, inp.alpha)
+        torch.cuda.synchronize()
+        assert b.qlora_device_error() == 0
+        assert torch.equal(Y, Y2), (N, K, M)
+        Xn, An, Bn = (bf16_to_f32_np(t).astype(np.float64) for t in (inp.X, inp.A, inp.B))
+        Yr, _ = oracle.linear_fwd(_wd(inp.W, False).astype(np.float64), Xn, An, Bn,
+                                  oracle.lora_scale(inp.alpha, inp.r))
+        ok, err = gemm_close(bf16_to_f32_np(Y), Yr)
+        assert ok, (N, K, M, r, err)
