@@ -263,7 +263,7 @@ qlora_status quantize_dq_impl(const void* W_bf16, const qlora_nf4_weight* q, int
   if (W_bf16 && !aligned(W_bf16, 16)) return QLORA_ERR_ALIGNMENT;
   const int64_t numel = q->rows * q->cols;
   const int64_t nblk = numel / 64;
-  const size_t off_absmax = align_up(kQuantScratchAllBytes);
+  const size_t off_absmax = align_up(kQuantScratchBytes);
   const size_t need = off_absmax + align_up(static_cast<size_t>(nblk) * sizeof(float));
   bool launch = false;
   st = workspace_check(workspace, workspace_bytes, need, &launch);

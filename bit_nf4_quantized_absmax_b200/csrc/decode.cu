@@ -452,7 +452,7 @@ cudaError_t launch_decode_fwd(const Nf4View& w, const void* X, int64_t M, const 
                                reinterpret_cast<const __nv_bfloat16*>(X), reinterpret_cast<const __nv_bfloat16*>(A),
                                static_cast<int>(M), w.K, r, T, counters, rp.n_tiles, col_scale);
     if (e != cudaSuccess) return e;
-    return launch_decode_res_main(w, X, M, B, r, s, Y, T, partial, counters, rp, codebook, err, stream);
+    return launch_decode_res_main(w, X, M, B, r, s, Y, T, partial, counters, rp, codebook, stream);
   }
   if (w.N >= (int64_t(1) << 31) || w.K >= (int64_t(1) << 31)) return cudaErrorInvalidValue;  // TMA coordinates
   Nf4Codebook cb;

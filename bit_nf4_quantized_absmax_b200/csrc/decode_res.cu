@@ -124,7 +124,6 @@ struct ResParams {
   int p_max;               // reduction slots per warp
   int cta_tiles;           // CTA-local tile counters per CTA
   int max_cta_seg;         // most CTAs holding pieces of one tile
-  int32_t* err;
 };
 
 // Shared memory: X [M][x_stride] | slots [kResWarps][p_max][32][4 MT] fp32 | counters [cta_tiles] u32
@@ -489,8 +488,7 @@ size_t res_partial_elems(const ResPlan& p) {
 
 cudaError_t launch_decode_res_main(const Nf4View& w, const void* X, int64_t M, const void* B, int r, float s,
                                    void* Y, const float* T, float* partial, unsigned int* counters,
-                                   const ResPlan& rp, const float codebook[16], int32_t* err,
-                                   cudaStream_t stream) {
+                                   const ResPlan& rp, const float codebook[16], cudaStream_t stream) {
   Nf4Codebook cb;
   for (int i = 0; i < 16; ++i) cb.c[i] = codebook[i];
   ResParams p;
@@ -516,7 +514,6 @@ cudaError_t launch_decode_res_main(const Nf4View& w, const void* X, int64_t M, c
   p.p_max = rp.p_max;
   p.cta_tiles = rp.cta_tiles;
   p.max_cta_seg = rp.max_cta_seg;
-  p.err = err;
   const bool single = w.absmax != nullptr;
   const int smem = static_cast<int>(rp.smem);
   cudaError_t e;

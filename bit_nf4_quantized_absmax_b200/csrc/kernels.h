@@ -26,10 +26,8 @@ cudaError_t ensure_smem_limit(int bytes) {
 }
 
 // Quantize scratch besides the fp32 absmax: the 256 exponent-bin totals (u64)
-// of the exact sum of the constants (kQuantScratchBytes, the part a row shard's
-// caller exchanges), then a ticket counter and the mean (kQuantScratchAllBytes).
+// of the exact sum of the constants (the part a row shard's caller exchanges).
 constexpr size_t kQuantScratchBytes = 256 * sizeof(unsigned long long);
-constexpr size_t kQuantScratchAllBytes = kQuantScratchBytes + 16;
 
 // Number of non-empty pieces when `nkb` k-blocks are cut into pieces of
 // ceil(nkb / want) blocks. The split-reduction GEMMs and the kernels that sum
@@ -53,14 +51,11 @@ cudaError_t launch_quantize(const void* W, int64_t numel, uint8_t* packed, int8_
 // sum (zeroed and then added into); second, after the totals of all shards have
 // been summed, the mean over nblk_mean constants and the int8 codes and group
 // scales of this shard's nblk constants.
-// done / mean_out / mu_out (optional, together): the sums kernel also forms
-// the mean (a whole weight); mu_ready (optional): the coding kernel reads it.
 cudaError_t launch_quantize_first(const void* W, int64_t nblk, uint8_t* packed, float* absmax_scratch,
-                                  unsigned long long* totals, int num_sms, cudaStream_t stream, int dtype = 0,
-                                  unsigned int* done = nullptr, float* mean_out = nullptr, float* mu_out = nullptr);
+                                  unsigned long long* totals, int num_sms, cudaStream_t stream, int dtype = 0);
 cudaError_t launch_quantize_second(const float* absmax_scratch, int64_t nblk, const unsigned long long* totals,
                                    int64_t nblk_mean, int8_t* absmax_q, float* dq_scale, float* mean,
-                                   cudaStream_t stream, const float* mu_ready = nullptr);
+                                   cudaStream_t stream);
 
 // Single-level storage: the codes and the fp32 block constants m_b only (pass 1).
 cudaError_t launch_quantize_single(const void* W, int64_t numel, uint8_t* packed, float* absmax, int num_sms,
@@ -118,7 +113,7 @@ ResPlan res_plan(int64_t M, int64_t N, int64_t K, int num_sms, bool force = fals
 size_t res_partial_elems(const ResPlan& p);
 cudaError_t launch_decode_res_main(const Nf4View& w, const void* X, int64_t M, const void* B, int r, float s,
                                    void* Y, const float* T, float* partial, unsigned int* counters,
-                                   const ResPlan& rp, const float codebook[16], int32_t* err, cudaStream_t stream);
+                                   const ResPlan& rp, const float codebook[16], cudaStream_t stream);
 
 // T [M, r] fp32 receives X A^T; partial [decode_partial_elems] fp32 and
 // counters [decode_counter_words] are scratch. With rp.ok the X-resident kernel

@@ -284,8 +284,8 @@ __device__ __forceinline__ void pass1_loop(const uint4* __restrict__ W, int64_t 
 // k_quant_sums adds into, cleared here by CTA 0 before that kernel starts.
 __global__ void __launch_bounds__(kPass1Threads, 8)
 k_quant_pass1(const uint4* __restrict__ W, bool v8, uint32_t* __restrict__ packed,
-              float* __restrict__ absmax, unsigned long long* __restrict__ zero_totals,
-              unsigned int* __restrict__ zero_done, int64_t nblk, const __grid_constant__ QuantBinTable tab) {
+              float* __restrict__ absmax, unsigned long long* __restrict__ zero_totals, int64_t nblk,
+              const __grid_constant__ QuantBinTable tab) {
   __shared__ uint2 s_bins[kBins];
   __shared__ uint32_t s_tbin[kBins], s_cbin[kBins];
   const int tid = threadIdx.x;
@@ -297,7 +297,6 @@ k_quant_pass1(const uint4* __restrict__ W, bool v8, uint32_t* __restrict__ packe
   __syncthreads();
   pdl_enter();
   if (zero_totals && blockIdx.x == 0) zero_totals[tid] = 0ull;  // kPass1Threads == 256 bins
-  if (zero_done && blockIdx.x == 0 && tid == 0) *zero_done = 0u;
 
   const unsigned char* bins = reinterpret_cast<const unsigned char*>(s_bins);
   const unsigned char* tbin = reinterpret_cast<const unsigned char*>(s_tbin);
@@ -314,19 +313,10 @@ k_quant_pass1(const uint4* __restrict__ W, bool v8, uint32_t* __restrict__ packe
 // overflow; lanes that share a bin add first (match + reduce), then one shared
 // atomic; then one 64-bit global atomic per nonzero bin. Integer additions in
 // any order give the same totals.
-__device__ float mean_from_bins(const unsigned long long* __restrict__ totals, int64_t nblk, float* mean_out,
-                                bool store);
-
-// done (optional, zeroed by pass 1): the CTA that adds the last bin totals
-// (ticket) also forms the mean mu = fp32(RN_fp64(S) / nblk) from them, stores
-// it in mean_out (the weight's mean) and mu_out (for k_dq_quantize), so that
-// the coding kernel does not form it in every CTA.
 __global__ void __launch_bounds__(256)
 k_quant_sums(const float* __restrict__ absmax, int64_t nblk, int64_t per_cta,
-             unsigned long long* __restrict__ totals, unsigned int* __restrict__ done, float* __restrict__ mean_out,
-             float* __restrict__ mu_out) {
+             unsigned long long* __restrict__ totals) {
   __shared__ unsigned int s_hist[256];
-  __shared__ unsigned int s_last;
   s_hist[threadIdx.x] = 0u;
   __syncthreads();
   pdl_enter();
@@ -349,17 +339,6 @@ k_quant_sums(const float* __restrict__ absmax, int64_t nblk, int64_t per_cta,
   __syncthreads();
   const unsigned int v = s_hist[threadIdx.x];
   if (v) atomicAdd(&totals[threadIdx.x], static_cast<unsigned long long>(v));
-  if (!done) return;
-  __syncthreads();  // every bin of this CTA is added before its ticket
-  if (threadIdx.x == 0) {
-    unsigned int old;
-    asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], 1;" : "=r"(old) : "l"(done) : "memory");
-    s_last = old == gridDim.x - 1 ? 1u : 0u;
-  }
-  __syncthreads();
-  if (!s_last) return;
-  const float mu = mean_from_bins(totals, nblk, mean_out, true);
-  if (threadIdx.x == 0) *mu_out = mu;
 }
 
 // mu = fp32(RN_fp64(S) / nblk) from the exact bin totals (warp 0 of the CTA);
@@ -403,12 +382,12 @@ __device__ float mean_from_bins(const unsigned long long* __restrict__ totals, i
 __global__ void __launch_bounds__(256)
 k_dq_quantize(const float* __restrict__ absmax, int64_t nblk, const unsigned long long* __restrict__ totals,
               int64_t nblk_mean, float* __restrict__ mean_out, int8_t* __restrict__ q, float* __restrict__ dq_scale,
-              int64_t ngrp, const float* __restrict__ mu_ready) {
+              int64_t ngrp) {
   pdl_enter();
   // the mean: formed by the sums kernel when it could (one weight on one GPU),
   // else here from the bin totals (a row shard, after the totals of all shards
   // were added), stored by CTA 0
-  const float mu = mu_ready ? __ldcg(mu_ready) : mean_from_bins(totals, nblk_mean, mean_out, blockIdx.x == 0);
+  const float mu = mean_from_bins(totals, nblk_mean, mean_out, blockIdx.x == 0);
   const int lane = threadIdx.x & 31;
   const int64_t g = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
   if (g >= ngrp) return;  // whole warp leaves together
@@ -477,22 +456,21 @@ int pass1_grid(int64_t nblk, int num_sms) {
 }
 
 cudaError_t launch_pass1(const void* W, int64_t nblk, uint8_t* packed, float* absmax, unsigned long long* zero_totals,
-                         unsigned int* zero_done, int num_sms, cudaStream_t stream, int dtype) {
+                         int num_sms, cudaStream_t stream, int dtype) {
   const QuantTables& tabs = quant_tables(dtype);
   QuantBinTable tab;
   for (int i = 0; i < kBins; ++i) tab.bins[i] = tabs.bins[i];
   const bool v8 = ((reinterpret_cast<uintptr_t>(W) | reinterpret_cast<uintptr_t>(packed)) & 31u) == 0;
   return launch_pdl(k_quant_pass1, dim3(pass1_grid(nblk, num_sms)), dim3(kPass1Threads), 0, stream,
                     reinterpret_cast<const uint4*>(W), v8, reinterpret_cast<uint32_t*>(packed), absmax, zero_totals,
-                    zero_done, nblk, tab);
+                    nblk, tab);
 }
 
 }  // namespace
 
 cudaError_t launch_quantize_first(const void* W, int64_t nblk, uint8_t* packed, float* absmax_scratch,
-                                  unsigned long long* totals, int num_sms, cudaStream_t stream, int dtype,
-                                  unsigned int* done, float* mean_out, float* mu_out) {
-  cudaError_t e = launch_pass1(W, nblk, packed, absmax_scratch, totals, done, num_sms, stream, dtype);
+                                  unsigned long long* totals, int num_sms, cudaStream_t stream, int dtype) {
+  cudaError_t e = launch_pass1(W, nblk, packed, absmax_scratch, totals, num_sms, stream, dtype);
   if (e != cudaSuccess) return e;
   // chunks of at least 512 constants and at most 8 CTAs per SM (the loop of a
   // CTA is latency bound, so many short chunks beat few long ones), at most
@@ -505,17 +483,17 @@ cudaError_t launch_quantize_first(const void* W, int64_t nblk, uint8_t* packed, 
   if (g > 0x7fffffff) return cudaErrorInvalidValue;
   const int64_t per_cta = (nblk + g - 1) / g;
   return launch_pdl(k_quant_sums, dim3(static_cast<unsigned>(g)), dim3(256), 0, stream,
-                    static_cast<const float*>(absmax_scratch), nblk, per_cta, totals, done, mean_out, mu_out);
+                    static_cast<const float*>(absmax_scratch), nblk, per_cta, totals);
 }
 
 cudaError_t launch_quantize_second(const float* absmax_scratch, int64_t nblk, const unsigned long long* totals,
                                    int64_t nblk_mean, int8_t* absmax_q, float* dq_scale, float* mean,
-                                   cudaStream_t stream, const float* mu_ready) {
+                                   cudaStream_t stream) {
   const int64_t ngrp = (nblk + 255) / 256;
   const int64_t dq_grid = (ngrp + 7) / 8;
   if (dq_grid > 0x7fffffff) return cudaErrorInvalidValue;
   return launch_pdl(k_dq_quantize, dim3(static_cast<unsigned>(dq_grid)), dim3(256), 0, stream, absmax_scratch,
-                    nblk, totals, nblk_mean, mean, absmax_q, dq_scale, ngrp, mu_ready);
+                    nblk, totals, nblk_mean, mean, absmax_q, dq_scale, ngrp);
 }
 
 cudaError_t launch_quantize(const void* W, int64_t numel, uint8_t* packed, int8_t* absmax_q, float* dq_scale,
@@ -534,7 +512,7 @@ cudaError_t launch_quantize(const void* W, int64_t numel, uint8_t* packed, int8_
 
 cudaError_t launch_quantize_single(const void* W, int64_t numel, uint8_t* packed, float* absmax, int num_sms,
                                    cudaStream_t stream, int dtype) {
-  return launch_pass1(W, numel / 64, packed, absmax, nullptr, nullptr, num_sms, stream, dtype);
+  return launch_pass1(W, numel / 64, packed, absmax, nullptr, num_sms, stream, dtype);
 }
 
 }  // namespace qlora

@@ -24,7 +24,7 @@ namespace {
 // Llama-65B linear weight): 2.25 KiB of bin totals, ticket and mean + 16 MiB of
 // absmax per device.
 constexpr int64_t kNoAllocMaxBlocks = int64_t(1) << 22;
-constexpr size_t kBinsBytes = (qlora::kQuantScratchAllBytes + 255) / 256 * 256;
+constexpr size_t kBinsBytes = (qlora::kQuantScratchBytes + 255) / 256 * 256;
 constexpr size_t kScratchBytes = kBinsBytes + static_cast<size_t>(kNoAllocMaxBlocks) * sizeof(float);
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
