@@ -178,6 +178,7 @@ qlora_status linear_bwd_impl(const qlora_nf4_weight* q, const void* X, int64_t M
   const size_t off_wd = L.add(dX ? static_cast<size_t>(N) * K * 2 : 0);
   const size_t off_thi = L.add(mp), off_tlo = L.add(mp);
   const size_t off_su = L.add(mp), off_uhi = L.add(mp), off_ulo = L.add(mp);
+  const size_t off_tail = L.add(dX ? kPairTailBytes : 0);
   const int splits_t = red_splits(M, rpad, K, di.num_sms);
   const int splits_u = red_splits(M, rpad, N, di.num_sms);
   size_t pmax = static_cast<size_t>(splits_a) * K * rpad;
@@ -230,12 +231,14 @@ qlora_status linear_bwd_impl(const qlora_nf4_weight* q, const void* X, int64_t M
   // the LoRA gradients are complete: a cross-rank sum may start while dX runs
   if (e == cudaSuccess && grads_ready) e = cudaEventRecord(grads_ready, cs);
   if (dX && fused_forward(M)) {  // W' decoded inside the GEMM
-    if (e == cudaSuccess) e = launch_gemm_dx_nf4(dY, view(q), sU, A, M, r, rpad, dX, cb, di.num_sms, err, cs);
+    if (e == cudaSuccess)
+      e = launch_gemm_dx_nf4(dY, view(q), sU, A, M, r, rpad, dX, ws + off_tail, cb, di.num_sms, err, cs);
   } else if (dX) {
     void* Wd = ws + off_wd;
     if (e == cudaSuccess)
       e = launch_dequantize(view(q), Wd, cb, di.num_sms, cs);
-    if (e == cudaSuccess) e = launch_gemm_dx(dY, Wd, sU, A, M, N, K, r, rpad, dX, di.num_sms, err, cs);
+    if (e == cudaSuccess)
+      e = launch_gemm_dx(dY, Wd, sU, A, M, N, K, r, rpad, dX, ws + off_tail, di.num_sms, err, cs);
   }
   return cuda_status(e);
 }
@@ -305,7 +308,7 @@ qlora_status linear_fwd_impl(const qlora_nf4_weight* q, const void* X, int64_t M
   const bool decode = M <= 16;
   // workspace layout
   Layout L;
-  size_t off_T = 0, off_part = 0, off_cnt = 0, off_wd = 0, off_sT = 0;
+  size_t off_T = 0, off_part = 0, off_cnt = 0, off_wd = 0, off_sT = 0, off_tail = 0;
   DecodePlan dplan{};
   ResPlan rplan{};
   if (decode) {
@@ -320,6 +323,7 @@ qlora_status linear_fwd_impl(const qlora_nf4_weight* q, const void* X, int64_t M
     off_wd = L.add(static_cast<size_t>(N) * K * 2);
     off_sT = L.add(static_cast<size_t>(M) * rpad * 2);
     off_part = L.add(static_cast<size_t>(red_splits(M, rpad, K, di.num_sms)) * M * rpad * sizeof(float));
+    off_tail = L.add(kPairTailBytes);
   }
   bool launch = false;
   st = workspace_check(workspace, workspace_bytes, L.total(), &launch);
@@ -343,14 +347,15 @@ qlora_status linear_fwd_impl(const qlora_nf4_weight* q, const void* X, int64_t M
     cudaError_t e = launch_gemm_lora_t(X, A, M, K, r, rpad, P, splits_t, di.num_sms, err, cs);
     if (e == cudaSuccess)
       e = launch_lora_finish(P, splits_t, M, r, rpad, s, T_save, sT, nullptr, nullptr, di.num_sms, cs, col_scale);
-    if (e == cudaSuccess) e = launch_gemm_fwd_nf4(X, view(q), sT, B, M, r, rpad, Y, cb, di.num_sms, err, cs);
+    if (e == cudaSuccess)
+      e = launch_gemm_fwd_nf4(X, view(q), sT, B, M, r, rpad, Y, ws + off_tail, cb, di.num_sms, err, cs);
     return cuda_status(e);
   }
   cudaError_t e = launch_dequantize(view(q), Wd, cb, di.num_sms, cs);
   if (e == cudaSuccess) e = launch_gemm_lora_t(X, A, M, K, r, rpad, P, splits_t, di.num_sms, err, cs);
   if (e == cudaSuccess)
     e = launch_lora_finish(P, splits_t, M, r, rpad, s, T_save, sT, nullptr, nullptr, di.num_sms, cs, col_scale);
-  if (e == cudaSuccess) e = launch_gemm_fwd(X, Wd, sT, B, M, N, K, r, rpad, Y, di.num_sms, err, cs);
+  if (e == cudaSuccess) e = launch_gemm_fwd(X, Wd, sT, B, M, N, K, r, rpad, Y, ws + off_tail, di.num_sms, err, cs);
   return cuda_status(e);
 }
 

@@ -18,7 +18,9 @@
 // CTA leave its loops.
 #include <cuda.h>
 
+#include <atomic>
 #include <cstdlib>
+#include <random>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -48,6 +50,9 @@ struct TileSched {
   int nk1;        // k-blocks of the main pair
   int kb_per_split;
   int group_m;    // 0: tiles M-fastest; else (one split) bands of group_m M tiles, M-fastest inside a band
+  // 2-CTA kernels: units [0, full_units) are whole tiles; the remaining tail_tiles
+  // tiles are two units each, k-blocks [0, kb_half) and [kb_half, nkb)
+  int full_units, tail_tiles, kb_half;
 };
 
 // DUAL: every k-block multiplies one A tile by two B tiles (B1 then B2) into
@@ -181,6 +186,24 @@ __device__ __forceinline__ void decode_unit(const TileSched& ts, int unit, int& 
   }
   kb0 = split * ts.kb_per_split;
   kb1 = min(ts.nkb, kb0 + ts.kb_per_split);
+}
+
+// Work unit of the 2-CTA kernels: tile (tm, tn), k-blocks [kb0, kb1), and for
+// half a split tile its half (0, 1; -1 for a whole tile) and tail index.
+__device__ __forceinline__ void decode_unit_pair(const TileSched& ts, int unit, int& tm, int& tn, int& kb0, int& kb1,
+                                                 int& half, int& tail) {
+  int t = unit;
+  half = -1;
+  tail = 0;
+  if (unit >= ts.full_units) {
+    const int v = unit - ts.full_units;
+    tail = v >> 1;
+    half = v & 1;
+    t = ts.full_units + tail;
+  }
+  decode_unit(ts, t, tm, tn, kb0, kb1);
+  if (half == 0) kb1 = ts.kb_half;
+  if (half == 1) kb0 = ts.kb_half;
 }
 
 template <int BN, bool A_MN, bool B_MN, int OUT, bool DUAL = false>
@@ -504,11 +527,114 @@ struct Cfg2 {
   static constexpr int SMEM = STAGES * STAGE_BYTES + 1024 + 256;
 };
 
+// The tail of a pair GEMM's persistent schedule: when the last wave would leave
+// at least half of the pairs idle, each of its tiles is split in two halves
+// along K that run side by side. For each warp's 32 rows, each half writes its
+// fp32 partial, then swaps the launch's tag into the rows' flag (acquire-
+// release, GPU scope); the half that finds the tag already there adds the other
+// partial to its own accumulator and writes C, then puts the flag back to
+// another value, so that a replay of the same launch (a CUDA graph) starts
+// clean. No half waits for the other, and own + other is the same sum in either
+// order.
+struct TailParams {
+  float* part;               // fp32 [2 halves][kPairMaxTail][2 ranks][128 rows][256 cols]
+  unsigned long long* flag;  // [kPairMaxTail][2 ranks][4 warps]
+  unsigned long long tag;    // unique to the launch
+};
+
+__device__ __forceinline__ unsigned long long atom_exch_acq_rel_gpu(unsigned long long* p, unsigned long long v) {
+  unsigned long long old;
+  asm volatile("atom.exch.acq_rel.gpu.global.b64 %0, [%1], %2;" : "=l"(old) : "l"(p), "l"(v) : "memory");
+  return old;
+}
+
+// Epilogue of one unit by one of warps 2..5 of a CTA of the pair (32 of the
+// CTA's 128 rows of the 256 x 256 tile in accumulator `acc`): bf16 C, or for
+// half a split tile the partial and, by the second half to arrive, the sum.
+// AHEAD: load the other partial's next chunk while a chunk is summed (32 more
+// registers; the NF4-decoding kernel, at 704 threads, has none to spare).
+template <bool AHEAD>
+__device__ __forceinline__ void pair_epilogue_unit(uint32_t tmem_base, int acc, int quarter, int lane, uint32_t rank,
+                                                   int tm, int tn, int half, int tail, int M, int Nc,
+                                                   const EpiParams& ep, const TailParams& tp) {
+  constexpr int BN2 = 256;
+  constexpr size_t kPart = 128 * 256;  // floats of one (half, tail, rank) partial
+  const int row_in_tile = quarter * 32 + lane;
+  const int row = tm * 256 + static_cast<int>(rank) * 128 + row_in_tile;
+  const bool row_ok = row < M;
+  const uint32_t tacc = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(acc * BN2);
+  const float* other = nullptr;
+  unsigned long long* flag = tp.flag + (static_cast<size_t>(tail) * 2 + rank) * 4 + quarter;
+  if (half >= 0) {
+    float* mine = tp.part + ((static_cast<size_t>(half) * kPairMaxTail + tail) * 2 + rank) * kPart +
+                  static_cast<size_t>(row_in_tile) * BN2;
+#pragma unroll 1
+    for (int c = 0; c < BN2 / 32; ++c) {
+      float v[32];
+      tmem_ld32(tacc + static_cast<uint32_t>(c * 32), v);
+      if (row_ok) {
+        float4* d = reinterpret_cast<float4*>(mine + c * 32);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) __stcg(d + q, make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]));
+      }
+    }
+    __syncwarp();  // the lanes' partial stores are ordered before lane 0's release below
+    unsigned long long prev = 0;
+    if (lane == 0) prev = atom_exch_acq_rel_gpu(flag, tp.tag);
+    if (!__shfl_sync(0xffffffffu, prev == tp.tag ? 1 : 0, 0)) return;  // the other half finishes these rows
+    __syncwarp();  // lane 0's acquire is ordered before every lane's reads of the other partial
+    other = tp.part + ((static_cast<size_t>(1 - half) * kPairMaxTail + tail) * 2 + rank) * kPart +
+            static_cast<size_t>(row_in_tile) * BN2;
+  }
+  float4 nxt[8];
+  if (AHEAD && other && row_ok) {
+#pragma unroll
+    for (int q = 0; q < 8; ++q) nxt[q] = __ldcg(reinterpret_cast<const float4*>(other) + q);
+  }
+#pragma unroll 1
+  for (int c = 0; c < BN2 / 32; ++c) {
+    float v[32];
+    tmem_ld32(tacc + static_cast<uint32_t>(c * 32), v);
+    const int col0 = tn * BN2 + c * 32;
+    if (!row_ok) continue;
+    if (other) {
+      float4 cur[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+        cur[q] = AHEAD ? nxt[q] : __ldcg(reinterpret_cast<const float4*>(other + c * 32) + q);
+      if (AHEAD && c + 1 < BN2 / 32) {
+#pragma unroll
+        for (int q = 0; q < 8; ++q) nxt[q] = __ldcg(reinterpret_cast<const float4*>(other + (c + 1) * 32) + q);
+      }
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        v[4 * q] += cur[q].x;
+        v[4 * q + 1] += cur[q].y;
+        v[4 * q + 2] += cur[q].z;
+        v[4 * q + 3] += cur[q].w;
+      }
+    }
+    __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(ep.C) + static_cast<int64_t>(row) * ep.ldc + col0;
+    if (col0 + 32 <= Nc && (ep.ldc % 8) == 0) {
+      uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        d4[q] = make_uint4(pack_bf16x2(v[8 * q + 0], v[8 * q + 1]), pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
+                           pack_bf16x2(v[8 * q + 4], v[8 * q + 5]), pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; ++j)
+        if (col0 + j < Nc) dst[j] = __float2bfloat16_rn(v[j]);
+    }
+  }
+  if (half >= 0 && lane == 0) *flag = ~tp.tag;
+}
+
 template <bool B_MN>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 k_tc_gemm2(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmB1,
            const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2, TileSched ts, int M,
-           int Nc, EpiParams ep, int32_t* err) {
+           int Nc, EpiParams ep, int32_t* err, TailParams tp) {
   using C = Cfg2<B_MN>;
   constexpr int BN2 = 256;
   extern __shared__ uint8_t smem_raw[];
@@ -525,7 +651,7 @@ k_tc_gemm2(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUt
   const uint32_t rank = cluster_ctarank();
   const int pair = blockIdx.x >> 1;
   const int npairs = gridDim.x >> 1;
-  const int n_units = ts.tiles_m * ts.tiles_n * ts.splits;
+  const int n_units = ts.full_units + 2 * ts.tail_tiles;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
@@ -565,8 +691,8 @@ k_tc_gemm2(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUt
       uint32_t phase = 0;
       bool ok = true;
       for (int unit = pair; unit < n_units && ok; unit += npairs) {
-        int tm, tn, kb0, kb1;
-        decode_unit(ts, unit, tm, tn, kb0, kb1);
+        int tm, tn, kb0, kb1, half, tail;
+        decode_unit_pair(ts, unit, tm, tn, kb0, kb1, half, tail);
         const int m0 = tm * 256 + static_cast<int>(rank) * 128;
         const int n0 = tn * BN2 + static_cast<int>(rank) * 128;
         for (int kb = kb0; kb < kb1; ++kb) {
@@ -606,8 +732,8 @@ k_tc_gemm2(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUt
       uint32_t acc_phase = 0;
       bool ok = true;
       for (int unit = pair; unit < n_units && ok; unit += npairs) {
-        int tm, tn, kb0, kb1;
-        decode_unit(ts, unit, tm, tn, kb0, kb1);
+        int tm, tn, kb0, kb1, half, tail;
+        decode_unit_pair(ts, unit, tm, tn, kb0, kb1, half, tail);
         if (!wait_or_abort(&acce[acc], acc_phase ^ 1u, abort_flag, err, DEV_TIMEOUT_TMEM_EMPTY)) {
           ok = false;
           break;
@@ -645,39 +771,16 @@ k_tc_gemm2(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUt
   } else {
     // ---------------- epilogue (warps 2..5, both CTAs) ----------------
     const int quarter = warp & 3;
-    const int row_in_tile = quarter * 32 + lane;
     const uint32_t acce_leader0 = map_to_cta(smem_u32(&acce[0]), 0);
     const uint32_t acce_leader1 = map_to_cta(smem_u32(&acce[1]), 0);
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int unit = pair; unit < n_units; unit += npairs) {
-      int tm, tn, kb0, kb1;
-      decode_unit(ts, unit, tm, tn, kb0, kb1);
+      int tm, tn, kb0, kb1, half, tail;
+      decode_unit_pair(ts, unit, tm, tn, kb0, kb1, half, tail);
       if (!wait_or_abort(&accf[acc], acc_phase, abort_flag, err, DEV_TIMEOUT_ACCUM)) break;
       tc_fence_after();
-      const int row = tm * 256 + static_cast<int>(rank) * 128 + row_in_tile;
-      const bool row_ok = row < M;
-#pragma unroll 1
-      for (int c = 0; c < BN2 / 32; ++c) {
-        float v[32];
-        tmem_ld32(tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
-                      static_cast<uint32_t>(acc * BN2 + c * 32),
-                  v);
-        const int col0 = tn * BN2 + c * 32;
-        if (!row_ok) continue;
-        __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(ep.C) + static_cast<int64_t>(row) * ep.ldc + col0;
-        if (col0 + 32 <= Nc && (ep.ldc % 8) == 0) {
-          uint4* d4 = reinterpret_cast<uint4*>(dst);
-#pragma unroll
-          for (int q = 0; q < 4; ++q)
-            d4[q] = make_uint4(pack_bf16x2(v[8 * q + 0], v[8 * q + 1]), pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
-                               pack_bf16x2(v[8 * q + 4], v[8 * q + 5]), pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
-        } else {
-#pragma unroll
-          for (int j = 0; j < 32; ++j)
-            if (col0 + j < Nc) dst[j] = __float2bfloat16_rn(v[j]);
-        }
-      }
+      pair_epilogue_unit<true>(tmem_base, acc, quarter, lane, rank, tm, tn, half, tail, M, Nc, ep, tp);
       tc_fence_before();
       mbar_arrive_cluster(acc ? acce_leader1 : acce_leader0);
       if (++acc == 2) {
@@ -736,7 +839,7 @@ template <bool B_MN>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kNf4Threads, 1)
 k_tc_gemm2_nf4(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmA2,
                const __grid_constant__ CUtensorMap tmB2, const __grid_constant__ Nf4Src src, TileSched ts, int M,
-               int Nc, EpiParams ep, int32_t* err, const __grid_constant__ Nf4Codebook cb) {
+               int Nc, EpiParams ep, int32_t* err, const __grid_constant__ Nf4Codebook cb, TailParams tp) {
   using C = Cfg2<B_MN>;
   constexpr int BN2 = 256;
   extern __shared__ uint8_t smem_raw[];
@@ -753,7 +856,7 @@ k_tc_gemm2_nf4(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__
   const uint32_t rank = cluster_ctarank();
   const int pair = blockIdx.x >> 1;
   const int npairs = gridDim.x >> 1;
-  const int n_units = ts.tiles_m * ts.tiles_n * ts.splits;
+  const int n_units = ts.full_units + 2 * ts.tail_tiles;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
@@ -792,8 +895,8 @@ k_tc_gemm2_nf4(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__
       uint32_t phase = 0;
       bool ok = true;
       for (int unit = pair; unit < n_units && ok; unit += npairs) {
-        int tm, tn, kb0, kb1;
-        decode_unit(ts, unit, tm, tn, kb0, kb1);
+        int tm, tn, kb0, kb1, half, tail;
+        decode_unit_pair(ts, unit, tm, tn, kb0, kb1, half, tail);
         const int m0 = tm * 256 + static_cast<int>(rank) * 128;
         const int n0 = tn * BN2 + static_cast<int>(rank) * 128;
         for (int kb = kb0; kb < kb1; ++kb) {
@@ -833,8 +936,8 @@ k_tc_gemm2_nf4(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__
       uint32_t acc_phase = 0;
       bool ok = true;
       for (int unit = pair; unit < n_units && ok; unit += npairs) {
-        int tm, tn, kb0, kb1;
-        decode_unit(ts, unit, tm, tn, kb0, kb1);
+        int tm, tn, kb0, kb1, half, tail;
+        decode_unit_pair(ts, unit, tm, tn, kb0, kb1, half, tail);
         if (!wait_or_abort(&acce[acc], acc_phase ^ 1u, abort_flag, err, DEV_TIMEOUT_TMEM_EMPTY)) {
           ok = false;
           break;
@@ -872,39 +975,16 @@ k_tc_gemm2_nf4(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__
   } else if (warp < 6) {
     // ---------------- epilogue (warps 2..5, both CTAs) ----------------
     const int quarter = warp & 3;
-    const int row_in_tile = quarter * 32 + lane;
     const uint32_t acce_leader0 = map_to_cta(smem_u32(&acce[0]), 0);
     const uint32_t acce_leader1 = map_to_cta(smem_u32(&acce[1]), 0);
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int unit = pair; unit < n_units; unit += npairs) {
-      int tm, tn, kb0, kb1;
-      decode_unit(ts, unit, tm, tn, kb0, kb1);
+      int tm, tn, kb0, kb1, half, tail;
+      decode_unit_pair(ts, unit, tm, tn, kb0, kb1, half, tail);
       if (!wait_or_abort(&accf[acc], acc_phase, abort_flag, err, DEV_TIMEOUT_ACCUM)) break;
       tc_fence_after();
-      const int row = tm * 256 + static_cast<int>(rank) * 128 + row_in_tile;
-      const bool row_ok = row < M;
-#pragma unroll 1
-      for (int c = 0; c < BN2 / 32; ++c) {
-        float v[32];
-        tmem_ld32(tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
-                      static_cast<uint32_t>(acc * BN2 + c * 32),
-                  v);
-        const int col0 = tn * BN2 + c * 32;
-        if (!row_ok) continue;
-        __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(ep.C) + static_cast<int64_t>(row) * ep.ldc + col0;
-        if (col0 + 32 <= Nc && (ep.ldc % 8) == 0) {
-          uint4* d4 = reinterpret_cast<uint4*>(dst);
-#pragma unroll
-          for (int q = 0; q < 4; ++q)
-            d4[q] = make_uint4(pack_bf16x2(v[8 * q + 0], v[8 * q + 1]), pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
-                               pack_bf16x2(v[8 * q + 4], v[8 * q + 5]), pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
-        } else {
-#pragma unroll
-          for (int j = 0; j < 32; ++j)
-            if (col0 + j < Nc) dst[j] = __float2bfloat16_rn(v[j]);
-        }
-      }
+      pair_epilogue_unit<false>(tmem_base, acc, quarter, lane, rank, tm, tn, half, tail, M, Nc, ep, tp);
       tc_fence_before();
       mbar_arrive_cluster(acc ? acce_leader1 : acce_leader0);
       if (++acc == 2) {
@@ -930,8 +1010,8 @@ k_tc_gemm2_nf4(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__
     uint32_t it = 0;  // k-blocks so far (all units): group it % kDecGroups fills this one
     bool ok = true;
     for (int unit = pair; unit < n_units && ok; unit += npairs) {
-      int tm, tn, kb0, kb1;
-      decode_unit(ts, unit, tm, tn, kb0, kb1);
+      int tm, tn, kb0, kb1, half, tail;
+      decode_unit_pair(ts, unit, tm, tn, kb0, kb1, half, tail);
       const int64_t n0 = static_cast<int64_t>(tn) * BN2 + static_cast<int64_t>(rank) * 128;
       // codes and constant of the first main k-block of the tile, then one ahead
       uint4 cur = make_uint4(0u, 0u, 0u, 0u);
@@ -1071,9 +1151,53 @@ cudaError_t run(const Operand& a1, const Operand& b1, const Operand* a2, const O
   return launch_pdl(kern, dim3(grid), dim3(kThreads), C::SMEM, stream, ta1, tb1, ta2, tb2, ts, M, Nc, ep, err);
 }
 
+// Units and pairs of a 2-CTA GEMM (ts.tiles_m, tiles_n, nkb set): whole tiles,
+// and when the last wave would leave at least half of the pairs idle and the
+// reduction is long, its tiles split in two along K (both halves then run in
+// that wave).
+int plan_pair_units(TileSched& ts, int num_sms, bool can_split) {
+  const int tiles = ts.tiles_m * ts.tiles_n;
+  int pairs = num_sms / 2;
+  if (pairs < 1) pairs = 1;
+  const int rem = tiles % pairs;
+  ts.full_units = tiles;
+  ts.tail_tiles = 0;
+  ts.kb_half = ts.nkb;
+  // (halves of fewer than ~48 k-blocks measured slower: the split tile's
+  // epilogue outweighs half a short tile; 4096x4096 at M = 4096: 118 -> 126 us)
+  if (can_split && rem > 0 && 2 * rem <= pairs && rem <= kPairMaxTail && ts.nkb >= 96) {
+    ts.full_units = tiles - rem;
+    ts.tail_tiles = rem;
+    ts.kb_half = (ts.nkb + 1) / 2;
+  }
+  const int units = ts.full_units + 2 * ts.tail_tiles;
+  return pairs < units ? pairs : units;
+}
+
+// A tag unique to each launch of a 2-CTA GEMM (the tail's flags compare
+// against it): a 64-bit counter from a random start.
+unsigned long long next_pair_tag() {
+  static std::atomic<unsigned long long> counter{[] {
+    std::random_device rd;
+    return (static_cast<unsigned long long>(rd()) << 32) ^ static_cast<unsigned long long>(rd());
+  }()};
+  return counter.fetch_add(1, std::memory_order_relaxed);
+}
+
+TailParams tail_params(void* tail_ws) {
+  TailParams tp{};
+  if (tail_ws) {
+    tp.part = static_cast<float*>(tail_ws);
+    tp.flag = reinterpret_cast<unsigned long long*>(static_cast<char*>(tail_ws) +
+                                                   static_cast<size_t>(kPairMaxTail) * 2 * 2 * 128 * 256 * sizeof(float));
+    tp.tag = next_pair_tag();
+  }
+  return tp;
+}
+
 template <bool B_MN>
 cudaError_t run_pair(const Operand& a1, const Operand& b1, const Operand& a2, const Operand& b2, int M, int Nc,
-                     const EpiParams& ep, int num_sms, int32_t* err, cudaStream_t stream) {
+                     const EpiParams& ep, void* tail_ws, int num_sms, int32_t* err, cudaStream_t stream) {
   using C = Cfg2<B_MN>;
   CUtensorMap ta1, tb1, ta2, tb2;
   // each CTA loads 128 rows of A and 128 of B's output dimension per box
@@ -1090,14 +1214,12 @@ cudaError_t run_pair(const Operand& a1, const Operand& b1, const Operand& a2, co
   ts.nkb = ts.nk1 + static_cast<int>((a2.k + BK - 1) / BK);
   ts.splits = 1;
   ts.kb_per_split = ts.nkb;
-  const int units = ts.tiles_m * ts.tiles_n;
-  int pairs = num_sms / 2;
-  if (pairs > units) pairs = units;
-  if (pairs < 1) pairs = 1;
+  const int pairs = plan_pair_units(ts, num_sms, tail_ws != nullptr);
   auto kern = k_tc_gemm2<B_MN>;
   const cudaError_t e = ensure_smem_limit<k_tc_gemm2<B_MN>>(C::SMEM);
   if (e != cudaSuccess) return e;
-  return launch_pdl(kern, dim3(2 * pairs), dim3(kThreads), C::SMEM, stream, ta1, tb1, ta2, tb2, ts, M, Nc, ep, err);
+  return launch_pdl(kern, dim3(2 * pairs), dim3(kThreads), C::SMEM, stream, ta1, tb1, ta2, tb2, ts, M, Nc, ep, err,
+                    tail_params(tail_ws));
 }
 
 }  // namespace
@@ -1114,14 +1236,16 @@ bool use_pair_kernel(int64_t M) {
 
 // Forward main GEMM: Y[M,N] = X[M,K] W'[N,K]^T + sT[M,rpad] Bl[N,r]^T
 cudaError_t launch_gemm_fwd(const void* X, const void* Wd, const void* sT, const void* Bl, int64_t M, int64_t N,
-                            int64_t K, int r, int rpad, void* Y, int num_sms, int32_t* err, cudaStream_t stream) {
+                            int64_t K, int r, int rpad, void* Y, void* tail_ws, int num_sms, int32_t* err,
+                            cudaStream_t stream) {
   Operand a1{X, M, K, K, false}, b1{Wd, N, K, K, false};
   Operand a2{sT, M, rpad, rpad, false}, b2{Bl, N, r, r, false};
   EpiParams ep{};
   ep.C = Y;
   ep.ldc = N;
   if (use_pair_kernel(M))
-    return run_pair<false>(a1, b1, a2, b2, static_cast<int>(M), static_cast<int>(N), ep, num_sms, err, stream);
+    return run_pair<false>(a1, b1, a2, b2, static_cast<int>(M), static_cast<int>(N), ep, tail_ws, num_sms, err,
+                           stream);
   return run<256, false, false, OUT_BF16>(a1, b1, &a2, &b2, static_cast<int>(M), static_cast<int>(N), 1, ep,
                                           num_sms, err, stream);
 }
@@ -1131,8 +1255,8 @@ cudaError_t launch_gemm_fwd(const void* X, const void* Wd, const void* sT, const
 // dX[M,K] = dY[M,N] dequant(w) + sU[M,rpad] Al[r,K] (B_MN true).
 template <bool B_MN>
 cudaError_t run_pair_nf4(const void* A1, int64_t K1, const Nf4View& w, const void* s_lora, const void* lora_w,
-                         int64_t M, int r, int rpad, void* out, const float codebook[16], int num_sms, int32_t* err,
-                         cudaStream_t stream) {
+                         int64_t M, int r, int rpad, void* out, void* tail_ws, const float codebook[16], int num_sms,
+                         int32_t* err, cudaStream_t stream) {
   using C = Cfg2<B_MN>;
   const int64_t N = w.N, K = w.K;
   const int64_t Nc = B_MN ? K : N;  // output columns
@@ -1153,10 +1277,7 @@ cudaError_t run_pair_nf4(const void* A1, int64_t K1, const Nf4View& w, const voi
   ts.nkb = ts.nk1 + static_cast<int>((rpad + BK - 1) / BK);
   ts.splits = 1;
   ts.kb_per_split = ts.nkb;
-  const int units = ts.tiles_m * ts.tiles_n;
-  int pairs = num_sms / 2;
-  if (pairs > units) pairs = units;
-  if (pairs < 1) pairs = 1;
+  const int pairs = plan_pair_units(ts, num_sms, tail_ws != nullptr);
   Nf4Src src{w.packed, w.absmax_q, w.dq_scale, w.mean, w.absmax, N, K};
   Nf4Codebook cb;
   for (int i = 0; i < 16; ++i) cb.c[i] = codebook[i];
@@ -1166,31 +1287,33 @@ cudaError_t run_pair_nf4(const void* A1, int64_t K1, const Nf4View& w, const voi
   const cudaError_t e = ensure_smem_limit<k_tc_gemm2_nf4<B_MN>>(C::SMEM);
   if (e != cudaSuccess) return e;
   return launch_pdl(k_tc_gemm2_nf4<B_MN>, dim3(2 * pairs), dim3(kNf4Threads), C::SMEM, stream, ta1, ta2, tb2, src,
-                    ts, static_cast<int>(M), static_cast<int>(Nc), ep, err, cb);
+                    ts, static_cast<int>(M), static_cast<int>(Nc), ep, err, cb, tail_params(tail_ws));
 }
 
 cudaError_t launch_gemm_fwd_nf4(const void* X, const Nf4View& w, const void* sT, const void* Bl, int64_t M, int r,
-                                int rpad, void* Y, const float codebook[16], int num_sms, int32_t* err,
+                                int rpad, void* Y, void* tail_ws, const float codebook[16], int num_sms, int32_t* err,
                                 cudaStream_t stream) {
-  return run_pair_nf4<false>(X, w.K, w, sT, Bl, M, r, rpad, Y, codebook, num_sms, err, stream);
+  return run_pair_nf4<false>(X, w.K, w, sT, Bl, M, r, rpad, Y, tail_ws, codebook, num_sms, err, stream);
 }
 
 cudaError_t launch_gemm_dx_nf4(const void* dY, const Nf4View& w, const void* sU, const void* Al, int64_t M, int r,
-                               int rpad, void* dX, const float codebook[16], int num_sms, int32_t* err,
+                               int rpad, void* dX, void* tail_ws, const float codebook[16], int num_sms, int32_t* err,
                                cudaStream_t stream) {
-  return run_pair_nf4<true>(dY, w.N, w, sU, Al, M, r, rpad, dX, codebook, num_sms, err, stream);
+  return run_pair_nf4<true>(dY, w.N, w, sU, Al, M, r, rpad, dX, tail_ws, codebook, num_sms, err, stream);
 }
 
 // Backward dX: dX[M,K] = dY[M,N] W'[N,K] + sU[M,rpad] A[r,K]
 cudaError_t launch_gemm_dx(const void* dY, const void* Wd, const void* sU, const void* Al, int64_t M, int64_t N,
-                           int64_t K, int r, int rpad, void* dX, int num_sms, int32_t* err, cudaStream_t stream) {
+                           int64_t K, int r, int rpad, void* dX, void* tail_ws, int num_sms, int32_t* err,
+                           cudaStream_t stream) {
   Operand a1{dY, M, N, N, false}, b1{Wd, K, N, K, true};
   Operand a2{sU, M, rpad, rpad, false}, b2{Al, K, r, K, true};
   EpiParams ep{};
   ep.C = dX;
   ep.ldc = K;
   if (use_pair_kernel(M))
-    return run_pair<true>(a1, b1, a2, b2, static_cast<int>(M), static_cast<int>(K), ep, num_sms, err, stream);
+    return run_pair<true>(a1, b1, a2, b2, static_cast<int>(M), static_cast<int>(K), ep, tail_ws, num_sms, err,
+                          stream);
   return run<256, false, true, OUT_BF16>(a1, b1, &a2, &b2, static_cast<int>(M), static_cast<int>(K), 1, ep,
                                          num_sms, err, stream);
 }

@@ -139,19 +139,28 @@ cudaError_t launch_merge(const Nf4View& w, const MergeAdapter* adapters, int n_a
                          const float codebook[16], int num_sms, cudaStream_t stream);
 
 // ---- gemm_tc.cu: tcgen05 GEMMs ----
+// Scratch of the 2-CTA GEMMs for the tiles of a last wave split in two along K:
+// at most kPairMaxTail such tiles, each with two fp32 halves of 256 x 256 and
+// eight 64-bit flags. `tail_ws` (kPairTailBytes, 256-byte aligned) may be null:
+// the tail is then not split.
+constexpr int kPairMaxTail = 37;
+constexpr size_t kPairTailBytes =
+    static_cast<size_t>(kPairMaxTail) * (2 * 2 * 128 * 256 * sizeof(float) + 8 * sizeof(unsigned long long));
 cudaError_t launch_gemm_fwd(const void* X, const void* Wd, const void* sT, const void* Bl, int64_t M, int64_t N,
-                            int64_t K, int r, int rpad, void* Y, int num_sms, int32_t* err, cudaStream_t stream);
+                            int64_t K, int r, int rpad, void* Y, void* tail_ws, int num_sms, int32_t* err,
+                            cudaStream_t stream);
 // The same forward with W' decoded from the NF4 storage inside the GEMM (no
 // dequantized copy of W' in memory); M >= 256.
 cudaError_t launch_gemm_fwd_nf4(const void* X, const Nf4View& w, const void* sT, const void* Bl, int64_t M, int r,
-                                int rpad, void* Y, const float codebook[16], int num_sms, int32_t* err,
+                                int rpad, void* Y, void* tail_ws, const float codebook[16], int num_sms, int32_t* err,
                                 cudaStream_t stream);
 // dX with W' decoded inside the GEMM; M >= 256.
 cudaError_t launch_gemm_dx_nf4(const void* dY, const Nf4View& w, const void* sU, const void* Al, int64_t M, int r,
-                               int rpad, void* dX, const float codebook[16], int num_sms, int32_t* err,
+                               int rpad, void* dX, void* tail_ws, const float codebook[16], int num_sms, int32_t* err,
                                cudaStream_t stream);
 cudaError_t launch_gemm_dx(const void* dY, const void* Wd, const void* sU, const void* Al, int64_t M, int64_t N,
-                           int64_t K, int r, int rpad, void* dX, int num_sms, int32_t* err, cudaStream_t stream);
+                           int64_t K, int r, int rpad, void* dX, void* tail_ws, int num_sms, int32_t* err,
+                           cudaStream_t stream);
 // Split-reduction partials P[splits][M][rpad] of X A^T (lora_t) and dY B (lora_u);
 // launch_lora_finish sums them and writes the fp32 / scaled / hi+lo operands.
 cudaError_t launch_gemm_lora_t(const void* X, const void* Al, int64_t M, int64_t K, int r, int rpad, float* P,

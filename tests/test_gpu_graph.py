@@ -64,3 +64,58 @@ def test_graph_replay_matches_eager():
     got = dict(outs, T=T, p=p32, m=m, v=v, packed=q.packed, absmax=qs.absmax)
     for k, ref in eager.items():
         assert torch.equal(got[k], ref), k
+
+
+def test_graph_replays_split_tail_tiles():
+    """A forward whose large GEMM splits its tiles in two along K (a reduction
+    of 8192 over two tiles; the backward's dX GEMM, a reduction of 512, keeps
+    whole tiles): the halves meet through flags that carry a tag of the launch,
+    so repeated replays of one captured launch must give the eager bits every
+    time, and the results must match the oracle."""
+    import numpy as np
+
+    import oracle
+    from tests.helpers import bf16_to_f32_np, gemm_close
+
+    dev = require_gpu()
+    N, K, M = 512, 8192, 256  # one M tile, two N tiles: every tile is split
+    inp = syn.make_linear(N, K, M, r=16, alpha=16.0, seed=23, workload="test", dy_std=0.5)
+    W, A, B, X, dY = (t.to(dev).contiguous() for t in (inp.W, inp.A, inp.B, inp.X, inp.dY))
+    q = b.qlora_quantize_nf4_dq(W)
+    Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+    dX = torch.empty(M, K, dtype=torch.bfloat16, device=dev)
+    dA = torch.empty(16, K, dtype=torch.bfloat16, device=dev)
+    dB = torch.empty(N, 16, dtype=torch.bfloat16, device=dev)
+    T = torch.empty(M, 16, dtype=torch.float32, device=dev)
+    ws_f = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    ws_b = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def step():
+        b.qlora_linear_fwd(q, X, A, B, inp.alpha, Y=Y, T_save=T, workspace=ws_f)
+        b.qlora_linear_bwd(q, X, A, B, inp.alpha, dY, T_saved=T, dX=dX, dA=dA, dB=dB, workspace=ws_b)
+
+    step()
+    torch.cuda.synchronize()
+    eager_y, eager_dx = Y.clone(), dX.clone()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=side):
+        step()
+    for _ in range(3):
+        Y.zero_()
+        dX.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        assert b.qlora_device_error() == 0
+        assert torch.equal(Y, eager_y)
+        assert torch.equal(dX, eager_dx)
+    Wd = oracle.bf16_bits_to_f32(oracle.dequantize_nf4_dq(oracle.quantize_nf4_dq(bf16_to_f32_np(inp.W))))
+    Xn, An, Bn, dYn = (bf16_to_f32_np(t).astype(np.float64) for t in (inp.X, inp.A, inp.B, inp.dY))
+    s = oracle.lora_scale(inp.alpha, inp.r)
+    Yr, _ = oracle.linear_fwd(Wd.astype(np.float64), Xn, An, Bn, s)
+    ok, err = gemm_close(bf16_to_f32_np(eager_y), Yr)
+    assert ok, err
+    dXr = oracle.linear_bwd(Wd.astype(np.float64), Xn, An, Bn, dYn, s)[0]
+    ok, err = gemm_close(bf16_to_f32_np(eager_dx), dXr)
+    assert ok, err
