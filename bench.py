@@ -45,7 +45,7 @@ SHAPES = syn.LLAMA7B_SHAPES
 # `bench.py --profile-case` (dram__bytes_read.sum + dram__bytes_write.sum per
 # launch, one pass). Valid only for the kernel sources it was taken on.
 ROOFLINE_SHAPE = (11008, 4096)
-TRAFFIC_RECORD = {"fingerprint": "ab40865e325867c5", "bytes": 305.1e6}
+TRAFFIC_RECORD = {"fingerprint": "6808c8a4a1587ff7", "bytes": 303.8e6}
 TRAFFIC_SOURCES = ("common.cuh", "nf4_lut.cuh", "dequant.cu", "gemm_tc.cu", "lora_misc.cu", "api.cu")
 
 
@@ -825,7 +825,8 @@ def run_ours(args, rank, world, dev):
     # dominant call: the training forward (M = 4096) on the 11008x4096 linear, i.e.
     # one dequant, the LoRA-down GEMM + finish and the 2-CTA tcgen05 GEMM with the
     # LoRA slab; algorithmic flops over its measured duration (events on the stream).
-    fwd_us = 1e3 * statistics.mean(a.elapsed_time(b) for a, b in ev[roof_part])
+    # median over the K calls: a call that met a power-capped clock dip does not move it
+    fwd_us = 1e3 * statistics.median(a.elapsed_time(b) for a, b in ev[roof_part])
     achieved = train_flops(*ROOFLINE_SHAPE)[0] / fwd_us / 1e6
     traffic = TRAFFIC_RECORD["bytes"] if TRAFFIC_RECORD["fingerprint"] == source_fingerprint() else None
     # the call is timed alone (its own event pair, a few hundred microseconds), so

@@ -46,8 +46,11 @@ __global__ void k_lora_finish(const float* __restrict__ P, int splits, int64_t M
     const int64_t m = e / rpad;
     const int j = static_cast<int>(e % rpad);
     float2 v = make_float2(0.0f, 0.0f);
+    // unrolled so that the loads of several splits are in flight together; the
+    // additions still run in split order
+#pragma unroll 8
     for (int p = 0; p < splits; ++p) {
-      const float2 pv = reinterpret_cast<const float2*>(P + (static_cast<int64_t>(p) * M) * rpad)[i];
+      const float2 pv = __ldcg(reinterpret_cast<const float2*>(P + (static_cast<int64_t>(p) * M) * rpad) + i);
       v.x += pv.x;
       v.y += pv.y;
     }
