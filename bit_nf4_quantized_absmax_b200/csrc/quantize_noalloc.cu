@@ -21,7 +21,7 @@
 namespace {
 
 // At most 2^22 blocks of 64 weights (268,435,456 weights, e.g. any single
-// Llama-65B linear weight): 2.25 KiB of bin totals, ticket and mean + 16 MiB of
+// Llama-65B linear weight): 2 KiB of bin totals + 16 MiB of
 // absmax per device.
 constexpr int64_t kNoAllocMaxBlocks = int64_t(1) << 22;
 constexpr size_t kBinsBytes = (qlora::kQuantScratchBytes + 255) / 256 * 256;
