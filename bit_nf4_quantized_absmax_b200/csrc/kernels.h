@@ -55,7 +55,7 @@ cudaError_t launch_quantize_first(const void* W, int64_t nblk, uint8_t* packed, 
                                   unsigned long long* totals, int num_sms, cudaStream_t stream, int dtype = 0);
 cudaError_t launch_quantize_second(const float* absmax_scratch, int64_t nblk, const unsigned long long* totals,
                                    int64_t nblk_mean, int8_t* absmax_q, float* dq_scale, float* mean,
-                                   cudaStream_t stream);
+                                   int num_sms, cudaStream_t stream);
 
 // Single-level storage: the codes and the fp32 block constants m_b only (pass 1).
 cudaError_t launch_quantize_single(const void* W, int64_t numel, uint8_t* packed, float* absmax, int num_sms,

@@ -9,11 +9,13 @@
 //                  the exact quotient v = w / m, the nearest code (one lookup in
 //                  a 33-bin table + one compare), 4-bit packing.
 //   k_quant_sums   the exact sum of the absmax constants, as integer sums of
-//                  their 8-bit significands per exponent (order-independent).
-//                  The CTA that adds the last totals forms the mean from them.
-//   k_dq_quantize  one warp per 256 constants: centre on the mean, group
-//                  absmax, int8 codes with round-to-nearest-even (for a row
-//                  shard, every CTA first forms the mean from the summed totals).
+//                  their 8-bit significands per exponent (order-independent),
+//                  eight loads in flight per thread and two running bins in
+//                  registers per thread.
+//   k_dq_quantize  every CTA forms the mean from the 256 bin totals (the
+//                  320-bit sum added across one warp), then one warp per 256
+//                  constants at a time: centre on the mean, group absmax, int8
+//                  codes with round-to-nearest-even. One wave of CTAs.
 #include "common.cuh"
 #include "host_tables.h"
 #include "kernels.h"
@@ -310,9 +312,15 @@ k_quant_pass1(const uint4* __restrict__ W, bool v8, uint32_t* __restrict__ packe
 // totals[e] += the 8-bit significands of the constants with exponent bin e (a
 // constant m = sig * 2^(E - 134), E = max(exponent field, 1)). Each CTA takes a
 // contiguous chunk of at most 2^24 constants, so its 32-bit shared bins cannot
-// overflow; lanes that share a bin add first (match + reduce), then one shared
-// atomic; then one 64-bit global atomic per nonzero bin. Integer additions in
-// any order give the same totals.
+// overflow. A thread loads eight constants at a time (all eight loads issued
+// before any is used) and adds each significand into one of two running bins
+// held in registers; the constants of one weight span few binades, so the
+// shared bins see an atomic only for a third exponent in a thread's share and
+// once per running bin at the end; then one 64-bit global atomic per nonzero
+// bin. Integer additions in any order give the same totals.
+constexpr int kSumsUnroll = 8;
+constexpr int kSumsChunk = kSumsUnroll * 256;  // constants per CTA per loop trip
+
 __global__ void __launch_bounds__(256)
 k_quant_sums(const float* __restrict__ absmax, int64_t nblk, int64_t per_cta,
              unsigned long long* __restrict__ totals) {
@@ -320,55 +328,77 @@ k_quant_sums(const float* __restrict__ absmax, int64_t nblk, int64_t per_cta,
   s_hist[threadIdx.x] = 0u;
   __syncthreads();
   pdl_enter();
-  const int lane = threadIdx.x & 31;
   const int64_t b0 = static_cast<int64_t>(blockIdx.x) * per_cta;
   const int64_t b1 = b0 + per_cta < nblk ? b0 + per_cta : nblk;
-  for (int64_t i = b0 + threadIdx.x; i - lane < b1; i += blockDim.x) {  // warp-uniform trip count
-    uint32_t hE = 1u, hsig = 0u;
-    if (i < b1) {
-      const uint32_t u = __float_as_uint(__ldg(absmax + i));
-      const uint32_t e = u >> 23;
-      const uint32_t mant7 = (u >> 16) & 0x7Fu;
-      hE = e ? e : 1u;
-      hsig = e ? (mant7 | 0x80u) : mant7;
+  uint32_t ea = 0u, eb = 0u, sa = 0u, sb = 0u;  // running bins (bin 0 = none: E >= 1)
+  for (int64_t base = b0; base < b1; base += kSumsChunk) {
+    float v[kSumsUnroll];
+#pragma unroll
+    for (int k = 0; k < kSumsUnroll; ++k) {
+      const int64_t i = base + threadIdx.x + k * 256;
+      v[k] = i < b1 ? __ldg(absmax + i) : 0.0f;
     }
-    const unsigned int same = __match_any_sync(0xffffffffu, hE);
-    const unsigned int tot = __reduce_add_sync(same, hsig);
-    if (lane == __ffs(same) - 1 && tot) atomicAdd(&s_hist[hE], tot);
+#pragma unroll
+    for (int k = 0; k < kSumsUnroll; ++k) {
+      const uint32_t u = __float_as_uint(v[k]);
+      const uint32_t e = u >> 23;
+      const uint32_t E = e ? e : 1u;
+      const uint32_t sig = ((u >> 16) & 0x7Fu) | (e ? 0x80u : 0u);
+      if (sig == 0u) continue;  // a zero constant adds nothing
+      if (E == ea) {
+        sa += sig;
+      } else if (E == eb) {
+        sb += sig;
+      } else if (ea == 0u) {
+        ea = E;
+        sa = sig;
+      } else if (eb == 0u) {
+        eb = E;
+        sb = sig;
+      } else {
+        atomicAdd(&s_hist[E], sig);
+      }
+    }
   }
+  if (sa) atomicAdd(&s_hist[ea], sa);
+  if (sb) atomicAdd(&s_hist[eb], sb);
   __syncthreads();
   const unsigned int v = s_hist[threadIdx.x];
   if (v) atomicAdd(&totals[threadIdx.x], static_cast<unsigned long long>(v));
 }
 
-// mu = fp32(RN_fp64(S) / nblk) from the exact bin totals (warp 0 of the CTA);
-// CTA 0 also stores it. nblk counts every constant the totals cover (the whole
-// tensor when this call only codes one shard of its constants).
+// mu = fp32(RN_fp64(S) / nblk) from the exact bin totals, formed by warp 0 of
+// the CTA: lane l adds bins l, l + 32, ..., l + 224 into a 320-bit partial sum,
+// the partial sums are added across the warp (integer additions with carries,
+// so any order gives the same bits), and lane 0 rounds the total once. CTA 0
+// also stores it. nblk counts every constant the totals cover (the whole tensor
+// when this call only codes one shard of its constants).
 __device__ float mean_from_bins(const unsigned long long* __restrict__ totals, int64_t nblk, float* mean_out,
                                 bool store) {
-  __shared__ unsigned long long s_tot[256];
-  __shared__ unsigned int s_mask[8];
   __shared__ float s_mu;
   if (threadIdx.x < 32) {
     const int lane = threadIdx.x;
+    unsigned long long L[5] = {0, 0, 0, 0, 0};
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
       const unsigned long long x = __ldcg(totals + 32 * k + lane);  // the atomics' results, from L2
-      s_tot[32 * k + lane] = x;
-      const unsigned int m = __ballot_sync(0xffffffffu, x != 0ull);
-      if (lane == 0) s_mask[k] = m;
+      if (x) acc_bin(L, x, 32 * k + lane);  // bin 0 is always empty
     }
-    __syncwarp();
-    if (lane == 0) {
-      unsigned long long L[5] = {0, 0, 0, 0, 0};
-      for (int k = 0; k < 8; ++k) {
-        unsigned int m = s_mask[k];
-        while (m) {
-          const int b = __ffs(m) - 1;
-          m &= m - 1u;
-          acc_bin(L, s_tot[32 * k + b], 32 * k + b);
-        }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      unsigned long long carry = 0ull;
+#pragma unroll
+      for (int j = 0; j < 5; ++j) {
+        const unsigned long long y = __shfl_down_sync(0xffffffffu, L[j], o);
+        const unsigned long long s1 = L[j] + y;
+        const unsigned long long c1 = s1 < y ? 1ull : 0ull;
+        const unsigned long long s2 = s1 + carry;
+        const unsigned long long c2 = s2 < s1 ? 1ull : 0ull;
+        L[j] = s2;
+        carry = c1 + c2;
       }
+    }
+    if (lane == 0) {
       const double S = limbs_to_double(L);
       const float mu = __double2float_rn(__ddiv_rn(S, static_cast<double>(nblk)));
       s_mu = mu;
@@ -384,58 +414,58 @@ k_dq_quantize(const float* __restrict__ absmax, int64_t nblk, const unsigned lon
               int64_t nblk_mean, float* __restrict__ mean_out, int8_t* __restrict__ q, float* __restrict__ dq_scale,
               int64_t ngrp) {
   pdl_enter();
-  // the mean: formed by the sums kernel when it could (one weight on one GPU),
-  // else here from the bin totals (a row shard, after the totals of all shards
-  // were added), stored by CTA 0
+  // the mean, formed in every CTA from the bin totals (for a row shard, after
+  // the totals of all shards were added), stored by CTA 0
   const float mu = mean_from_bins(totals, nblk_mean, mean_out, blockIdx.x == 0);
   const int lane = threadIdx.x & 31;
-  const int64_t g = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
-  if (g >= ngrp) return;  // whole warp leaves together
-  const int64_t i0 = g * 256 + lane * 8;
-  float c[8];
-  bool ok[8];
-  if (i0 + 8 <= nblk) {
-    const float4 a = *reinterpret_cast<const float4*>(absmax + i0);
-    const float4 b = *reinterpret_cast<const float4*>(absmax + i0 + 4);
-    const float mm[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+  const int64_t gstride = static_cast<int64_t>(gridDim.x) * 8;
+  for (int64_t g = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5); g < ngrp; g += gstride) {
+    const int64_t i0 = g * 256 + lane * 8;
+    float c[8];
+    bool ok[8];
+    if (i0 + 8 <= nblk) {
+      const float4 a = *reinterpret_cast<const float4*>(absmax + i0);
+      const float4 b = *reinterpret_cast<const float4*>(absmax + i0 + 4);
+      const float mm[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
 #pragma unroll
-    for (int j = 0; j < 8; ++j) { c[j] = __fsub_rn(mm[j], mu); ok[j] = true; }
-  } else {
+      for (int j = 0; j < 8; ++j) { c[j] = __fsub_rn(mm[j], mu); ok[j] = true; }
+    } else {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        ok[j] = (i0 + j) < nblk;
+        c[j] = ok[j] ? __fsub_rn(absmax[i0 + j], mu) : 0.0f;
+      }
+    }
+    float s = 0.0f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) s = fmaxf(s, fabsf(c[j]));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s = fmaxf(s, __shfl_xor_sync(0xffffffffu, s, o));
+    const float sc = __fdiv_rn(s, 127.0f);
+    int8_t qq[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-      ok[j] = (i0 + j) < nblk;
-      c[j] = ok[j] ? __fsub_rn(absmax[i0 + j], mu) : 0.0f;
+      int v = 0;
+      if (s > 0.0f) {
+        v = __float2int_rn(__fdiv_rn(c[j], sc));
+        v = max(-127, min(127, v));
+      }
+      qq[j] = static_cast<int8_t>(v);
     }
-  }
-  float s = 0.0f;
+    if (i0 + 8 <= nblk) {
+      uint2 pk;
+      pk.x = (uint32_t)(uint8_t)qq[0] | ((uint32_t)(uint8_t)qq[1] << 8) | ((uint32_t)(uint8_t)qq[2] << 16) |
+             ((uint32_t)(uint8_t)qq[3] << 24);
+      pk.y = (uint32_t)(uint8_t)qq[4] | ((uint32_t)(uint8_t)qq[5] << 8) | ((uint32_t)(uint8_t)qq[6] << 16) |
+             ((uint32_t)(uint8_t)qq[7] << 24);
+      *reinterpret_cast<uint2*>(q + i0) = pk;
+    } else {
 #pragma unroll
-  for (int j = 0; j < 8; ++j) s = fmaxf(s, fabsf(c[j]));
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) s = fmaxf(s, __shfl_xor_sync(0xffffffffu, s, o));
-  const float sc = __fdiv_rn(s, 127.0f);
-  int8_t qq[8];
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    int v = 0;
-    if (s > 0.0f) {
-      v = __float2int_rn(__fdiv_rn(c[j], sc));
-      v = max(-127, min(127, v));
+      for (int j = 0; j < 8; ++j)
+        if (ok[j]) q[i0 + j] = qq[j];
     }
-    qq[j] = static_cast<int8_t>(v);
+    if (lane == 0) dq_scale[g] = sc;
   }
-  if (i0 + 8 <= nblk) {
-    uint2 pk;
-    pk.x = (uint32_t)(uint8_t)qq[0] | ((uint32_t)(uint8_t)qq[1] << 8) | ((uint32_t)(uint8_t)qq[2] << 16) |
-           ((uint32_t)(uint8_t)qq[3] << 24);
-    pk.y = (uint32_t)(uint8_t)qq[4] | ((uint32_t)(uint8_t)qq[5] << 8) | ((uint32_t)(uint8_t)qq[6] << 16) |
-           ((uint32_t)(uint8_t)qq[7] << 24);
-    *reinterpret_cast<uint2*>(q + i0) = pk;
-  } else {
-#pragma unroll
-    for (int j = 0; j < 8; ++j)
-      if (ok[j]) q[i0 + j] = qq[j];
-  }
-  if (lane == 0) dq_scale[g] = sc;
 }
 
 // Persistent grid of pass 1: exactly the CTAs that are resident at once (four
@@ -472,11 +502,10 @@ cudaError_t launch_quantize_first(const void* W, int64_t nblk, uint8_t* packed, 
                                   unsigned long long* totals, int num_sms, cudaStream_t stream, int dtype) {
   cudaError_t e = launch_pass1(W, nblk, packed, absmax_scratch, totals, num_sms, stream, dtype);
   if (e != cudaSuccess) return e;
-  // chunks of at least 512 constants and at most 8 CTAs per SM (the loop of a
-  // CTA is latency bound, so many short chunks beat few long ones), at most
-  // 2^24 constants each
-  int64_t g = (nblk + 511) / 512;
-  if (g > 8 * num_sms) g = 8 * num_sms;
+  // chunks of at least one loop trip of a CTA and at most 4 CTAs per SM, at
+  // most 2^24 constants each
+  int64_t g = (nblk + kSumsChunk - 1) / kSumsChunk;
+  if (g > 4 * num_sms) g = 4 * num_sms;
   const int64_t min_g = (nblk + (int64_t(1) << 24) - 1) >> 24;
   if (g < min_g) g = min_g;
   if (g < 1) g = 1;
@@ -488,9 +517,12 @@ cudaError_t launch_quantize_first(const void* W, int64_t nblk, uint8_t* packed, 
 
 cudaError_t launch_quantize_second(const float* absmax_scratch, int64_t nblk, const unsigned long long* totals,
                                    int64_t nblk_mean, int8_t* absmax_q, float* dq_scale, float* mean,
-                                   cudaStream_t stream) {
+                                   int num_sms, cudaStream_t stream) {
   const int64_t ngrp = (nblk + 255) / 256;
-  const int64_t dq_grid = (ngrp + 7) / 8;
+  // one wave (8 CTAs of 256 threads fill an SM), so that the mean is formed
+  // once per resident CTA; the warps loop over the groups
+  int64_t dq_grid = (ngrp + 7) / 8;
+  if (dq_grid > 8 * static_cast<int64_t>(num_sms)) dq_grid = 8 * static_cast<int64_t>(num_sms);
   if (dq_grid > 0x7fffffff) return cudaErrorInvalidValue;
   return launch_pdl(k_dq_quantize, dim3(static_cast<unsigned>(dq_grid)), dim3(256), 0, stream, absmax_scratch,
                     nblk, totals, nblk_mean, mean, absmax_q, dq_scale, ngrp);
@@ -507,7 +539,7 @@ cudaError_t launch_quantize(const void* W, int64_t numel, uint8_t* packed, int8_
   // load add round trips to the critical path.)
   cudaError_t e = launch_quantize_first(W, nblk, packed, absmax_scratch, totals, num_sms, stream, dtype);
   if (e != cudaSuccess) return e;
-  return launch_quantize_second(absmax_scratch, nblk, totals, nblk, absmax_q, dq_scale, mean, stream);
+  return launch_quantize_second(absmax_scratch, nblk, totals, nblk, absmax_q, dq_scale, mean, num_sms, stream);
 }
 
 cudaError_t launch_quantize_single(const void* W, int64_t numel, uint8_t* packed, float* absmax, int num_sms,

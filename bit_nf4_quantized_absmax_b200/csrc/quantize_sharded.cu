@@ -103,7 +103,7 @@ qlora_status qlora_quantize_nf4_dq_shard_end(const qlora_nf4_weight* q, int64_t 
   if ((st = sm_count(&sms)) != QLORA_OK) return st;
   const cudaError_t e = qlora::launch_quantize_second(
       static_cast<const float*>(workspace), nblk, reinterpret_cast<const unsigned long long*>(bin_totals), nblk_all,
-      q->absmax_q, q->dq_scale, q->mean, reinterpret_cast<cudaStream_t>(stream));
+      q->absmax_q, q->dq_scale, q->mean, sms, reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
 }
 
