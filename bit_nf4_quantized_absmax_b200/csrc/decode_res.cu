@@ -474,7 +474,12 @@ ResPlan res_plan(int64_t M, int64_t N, int64_t K, int num_sms, bool force) {
   // weights (N > K) up to 8 tokens (11008x4096: 17.7 / 18.0 / 18.6 / 19.5
   // against 21.3 / 21.6 / 21.8 / 22.2); it is slower on K > N below 2^26
   // entries (4096x11008: 24.1 / 26.6 / 29.6 against 22.9 / 23.5 / 23.9) and
-  // at 8 tokens on square weights (4096x4096: 17.1 against 14.4).
+  // at 8 tokens on square weights (4096x4096: 17.1 against 14.4; 8192x8192 is
+  // the exception, 26.6 against 28.5, left to the ring kernel). With two token
+  // tiles (9 to 16 tokens) it is slower on every measured shape but the
+  // smallest (at 12 / 16 tokens, 11008x4096: 33.6 / 38.2 against 26.0 / 26.8;
+  // 4096x4096: 26.6 / 30.5 against 18.4 / 19.1; 2048x2048: 10.9 / 12.2 against
+  // 12.3 / 13.1), so it serves at most 8.
   const int64_t nw = N * K;
   const bool faster = (M <= 4 && nw >= (int64_t(1) << 22) && !(K > N && nw < (int64_t(1) << 26))) ||
                       (M <= 8 && K < N && nw >= (int64_t(1) << 24));

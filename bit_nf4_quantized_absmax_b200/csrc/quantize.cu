@@ -15,7 +15,8 @@
 //   k_dq_quantize  every CTA forms the mean from the 256 bin totals (the
 //                  320-bit sum added across one warp), then one warp per 256
 //                  constants at a time: centre on the mean, group absmax, int8
-//                  codes with round-to-nearest-even. One wave of CTAs.
+//                  codes with round-to-nearest-even. One wave of the CTAs
+//                  resident at once.
 #include "common.cuh"
 #include "host_tables.h"
 #include "kernels.h"
@@ -519,10 +520,18 @@ cudaError_t launch_quantize_second(const float* absmax_scratch, int64_t nblk, co
                                    int64_t nblk_mean, int8_t* absmax_q, float* dq_scale, float* mean,
                                    int num_sms, cudaStream_t stream) {
   const int64_t ngrp = (nblk + 255) / 256;
-  // one wave (8 CTAs of 256 threads fill an SM), so that the mean is formed
-  // once per resident CTA; the warps loop over the groups
+  // one wave of the CTAs resident at once, so that the mean is formed once per
+  // resident CTA; the warps loop over the groups
+  static std::atomic<int> per_sm_cache{0};  // the same on every B200; racing writers store equal values
+  int per_sm = per_sm_cache.load(std::memory_order_relaxed);
+  if (per_sm == 0) {
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_dq_quantize, 256, 0) != cudaSuccess || per_sm < 1)
+      per_sm = 4;
+    per_sm_cache.store(per_sm, std::memory_order_relaxed);
+  }
   int64_t dq_grid = (ngrp + 7) / 8;
-  if (dq_grid > 8 * static_cast<int64_t>(num_sms)) dq_grid = 8 * static_cast<int64_t>(num_sms);
+  const int64_t cap = static_cast<int64_t>(per_sm) * num_sms;
+  if (dq_grid > cap) dq_grid = cap;
   if (dq_grid > 0x7fffffff) return cudaErrorInvalidValue;
   return launch_pdl(k_dq_quantize, dim3(static_cast<unsigned>(dq_grid)), dim3(256), 0, stream, absmax_scratch,
                     nblk, totals, nblk_mean, mean, absmax_q, dq_scale, ngrp);
